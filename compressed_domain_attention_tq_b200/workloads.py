@@ -1,0 +1,153 @@
+"""Seeded synthetic workloads for int4 KV-cache decode.
+
+This module only draws random inputs; it holds none of the method's
+arithmetic (no rotation, quantization or attention).  Both the CUDA path and
+the CPU oracle are fed from it.
+
+The shapes stand in for the model runs on the pages (Open-TQ-Metal abstract:
+Llama 3.1 70B at 128K context and Gemma 4 with attn_scale = 1.0; AdapTQ post,
+performance section: 4 heads x d=128 x 4096 cached tokens).  No model weights
+or datasets are used: K, V and Q are i.i.d. normal draws with the structure
+each workload names (fixed outlier K channels, heavy-tailed token rows,
+ragged context lengths).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    context: int                  # cached tokens before the per-step append
+    capacity: int                 # cache rows per (sequence, kv head)
+    in_dtype: torch.dtype         # dtype of K, V, Q inputs
+    rotation: bool
+    attn_scales: tuple
+    outlier_channels: int = 0     # K channels per kv head multiplied by outlier_scale
+    outlier_scale: float = 1.0
+    heavy_row_frac: float = 0.0   # fraction of token rows (K and V) multiplied by heavy_scale
+    heavy_scale: float = 1.0
+    ragged: tuple | None = None   # (lo, hi): per-sequence context ~ U{lo..hi}
+    append_per_step: int = 1      # tokens quantize-appended per decode step
+    notes: str = field(default="", compare=False)
+
+    @property
+    def group(self) -> int:
+        return 32
+
+
+WORKLOADS = {
+    "tiny_mha_4k": Workload(
+        "tiny_mha_4k", batch=1, num_q_heads=4, num_kv_heads=4, head_dim=128, context=4096,
+        capacity=4097, in_dtype=torch.float32, rotation=False,
+        attn_scales=(1 / math.sqrt(128),),
+        notes="MHA, fp32 N(0,1); run with rotation off and on"),
+    "llama70b_gqa_32k": Workload(
+        "llama70b_gqa_32k", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=32768, capacity=32769, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0,
+        notes="64/8 GQA, bf16, 4 fixed K channels per head x10"),
+    "llama70b_gqa_128k": Workload(
+        "llama70b_gqa_128k", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0,
+        notes="64/8 GQA at 128K, bf16, outlier K channels; plus bulk prefill quantize"),
+    "ragged_b16": Workload(
+        "ragged_b16", batch=16, num_q_heads=64, num_kv_heads=8, head_dim=128, context=65536,
+        capacity=65537, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), heavy_row_frac=0.02, heavy_scale=8.0,
+        ragged=(8192, 65536),
+        notes="batch 16, per-sequence length U{8192..65536}, 2% token rows x8"),
+    "wide_d256": Workload(
+        "wide_d256", batch=4, num_q_heads=32, num_kv_heads=16, head_dim=256, context=65536,
+        capacity=65537, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1.0, 1 / 16.0),
+        notes="32/16 GQA, d=256; attn_scale 1.0 and 1/sqrt(256)"),
+}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def make_signs(head_dim: int, seed: int) -> torch.Tensor:
+    """Random +-1 int8 signs for the rotation (CPU tensor, from the seed)."""
+    g = _gen(1_000_003 + seed, "cpu")
+    return (torch.randint(0, 2, (head_dim,), generator=g, dtype=torch.int8) * 2 - 1).to(torch.int8)
+
+
+def make_context_lengths(w: Workload, seed: int) -> torch.Tensor:
+    """Per-sequence cached context (int32, CPU)."""
+    if w.ragged is None:
+        return torch.full((w.batch,), w.context, dtype=torch.int32)
+    lo, hi = w.ragged
+    g = _gen(2_000_003 + seed, "cpu")
+    return torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int32)
+
+
+def make_outlier_channels(w: Workload, seed: int) -> torch.Tensor:
+    """[Hkv][outlier_channels] fixed channel indices per kv head (CPU int64)."""
+    g = _gen(3_000_003 + seed, "cpu")
+    if w.outlier_channels == 0:
+        return torch.zeros((w.num_kv_heads, 0), dtype=torch.int64)
+    return torch.stack([torch.randperm(w.head_dim, generator=g)[:w.outlier_channels]
+                        for _ in range(w.num_kv_heads)])
+
+
+def make_kv(w: Workload, seed: int, device="cpu", tokens: int | None = None,
+            token_offset: int = 0) -> tuple[torch.Tensor, torch.Tensor]:
+    """K, V of shape [B][Hkv][tokens][d] in w.in_dtype.
+
+    Rows are drawn N(0,1); the workload's structure (outlier K channels, heavy
+    token rows) is applied as plain input scaling.  `token_offset` shifts the
+    seed stream so a per-step append token differs from the cached ones.
+    """
+    n = w.capacity if tokens is None else tokens
+    g = _gen(seed * 7919 + token_offset + 17, device)
+    shape = (w.batch, w.num_kv_heads, n, w.head_dim)
+    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if w.outlier_channels:
+        ch = make_outlier_channels(w, seed).to(device)
+        for h in range(w.num_kv_heads):
+            k[:, h, :, ch[h]] *= w.outlier_scale
+    if w.heavy_row_frac > 0:
+        m = torch.rand((w.batch, 1, n, 1), generator=g, device=device) < w.heavy_row_frac
+        k = torch.where(m, k * w.heavy_scale, k)
+        v = torch.where(m, v * w.heavy_scale, v)
+    return k.to(w.in_dtype), v.to(w.in_dtype)
+
+
+def make_query(w: Workload, seed: int, device="cpu", step: int = 0) -> torch.Tensor:
+    """Q of shape [B][Hq][d] (one decode token) in w.in_dtype."""
+    g = _gen(seed * 104729 + 31 + step, device)
+    q = torch.randn((w.batch, w.num_q_heads, w.head_dim), generator=g, device=device,
+                    dtype=torch.float32)
+    return q.to(w.in_dtype)
+
+
+def shrink(w: Workload, context: int, batch: int | None = None,
+           num_kv_heads: int | None = None) -> Workload:
+    """Same structure at a smaller size (parity tests the oracle finishes in seconds)."""
+    nk = w.num_kv_heads if num_kv_heads is None else num_kv_heads
+    G = w.num_q_heads // w.num_kv_heads
+    rag = None
+    if w.ragged is not None:
+        rag = (max(1, context // 8), context)
+    return Workload(w.name + f"_small{context}", batch=w.batch if batch is None else batch,
+                    num_q_heads=G * nk, num_kv_heads=nk, head_dim=w.head_dim, context=context,
+                    capacity=context + w.append_per_step, in_dtype=w.in_dtype,
+                    rotation=w.rotation, attn_scales=w.attn_scales,
+                    outlier_channels=w.outlier_channels, outlier_scale=w.outlier_scale,
+                    heavy_row_frac=w.heavy_row_frac, heavy_scale=w.heavy_scale, ragged=rag,
+                    append_per_step=w.append_per_step)

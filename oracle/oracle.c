@@ -1,0 +1,342 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for int4 KV-cache quantization and
+ * decode attention over the packed int4 cache.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library.  It shares
+ * no code, header, table or constant with the CUDA path and includes nothing
+ * from it.
+ *
+ * Sources (web pages on the method; cited by title and section):
+ *  [OTM]    "Open-TQ-Metal: Fused Compressed-Domain Attention for Long-Context
+ *           LLM Inference on Apple Silicon" (arXiv 2604.16957v1), abstract:
+ *           the KV cache is quantized to int4 as it is produced and attention
+ *           is computed directly on the compressed representation, with no
+ *           intermediate dequantized matrix; attn_scale is 1/sqrt(d) (Llama)
+ *           or 1.0 (Gemma 4).
+ *  [OTM-F]  zingnex forum summary of Open-TQ-Metal, sections "on-the-fly
+ *           quantization", "compressed-domain attention", "eliminating
+ *           intermediate matrices", "numerical stability".
+ *  [AdapTQ] zingnex post on AdapTQ, section "Fast Hadamard Rotation (HAR)":
+ *           an in-place O(d log d) Hadamard rotation before quantization
+ *           spreads outliers.
+ *  [SRFT]   agents-report.net post "SRFT + int4 KV-cache on Apple Silicon",
+ *           section on the core method: sign-randomized rotation (the
+ *           sign-randomized Hadamard is reported equivalent in quality), then
+ *           per-group abs-max, symmetric int4, nibble packing.
+ *
+ * Readings where the pages are silent (all listed in the design notes):
+ *  - rotation R = (1/sqrt d) * H_d * diag(sigma), H_d Sylvester-ordered,
+ *    H[i][j] = (-1)^popcount(i & j); sigma in {+1,-1}^d; inverse is R^T.
+ *  - rotated vector computed in fp64 with the explicit d x d matrix and
+ *    rounded once to fp32.
+ *  - groups of 32 consecutive rotated coordinates; scale s = fl32(amax / 7)
+ *    (fp32 IEEE division); codes c = clamp(rne(fl32(y / s)), -7, 7) with
+ *    round-half-to-even of the fp32 quotient; an all-zero group has s = 0 and
+ *    codes 0.
+ *  - attention output = exact softmax attention over the dequantized values
+ *    s*c in the rotated basis, mapped back with R^T, all in fp64.
+ *
+ * Build: gcc -O2 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_GROUP 32
+
+/* ------------------------------------------------------------------ */
+/* inputs                                                               */
+/* ------------------------------------------------------------------ */
+
+/* bf16 -> fp32 is exact: the 16 bits are the high half of the fp32 word. */
+static float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* element `idx` of an fp32 (dtype 0) or bf16 (dtype 1) array, as fp32 */
+static float load_input(const void* base, int dtype, int64_t idx) {
+  if (dtype == 0) return ((const float*)base)[idx];
+  return bf16_bits_to_float(((const uint16_t*)base)[idx]);
+}
+
+/* ------------------------------------------------------------------ */
+/* rotation ([AdapTQ] HAR; [SRFT] sign-randomized rotation)             */
+/* ------------------------------------------------------------------ */
+
+static int popcount_u32(uint32_t x) {
+  int n = 0;
+  while (x) { n += (int)(x & 1u); x >>= 1; }
+  return n;
+}
+
+/* Sylvester-ordered Walsh-Hadamard entry H_d[i][j] = (-1)^popcount(i&j). */
+int oracle_hadamard_entry(int i, int j) {
+  return (popcount_u32((uint32_t)(i & j)) & 1) ? -1 : 1;
+}
+
+/* R[i*d + j] = H[i][j] * sigma[j] / sqrt(d); identity when signs == NULL. */
+int oracle_rotation_matrix(int d, const int8_t* signs, double* R) {
+  if (d <= 0 || (d & (d - 1)) != 0 || !R) return -1;
+  double inv = 1.0 / sqrt((double)d);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) {
+      if (!signs) R[(int64_t)i * d + j] = (i == j) ? 1.0 : 0.0;
+      else R[(int64_t)i * d + j] = inv * (double)oracle_hadamard_entry(i, j) * (double)signs[j];
+    }
+  return 0;
+}
+
+/* y = fl32(R x): fp64 matrix-vector product, rounded once to fp32. */
+void oracle_rotate_vector(int d, const double* R, const float* x, float* y) {
+  for (int i = 0; i < d; ++i) {
+    double acc = 0.0;
+    for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * (double)x[j];
+    y[i] = (float)acc;
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* quantization ([SRFT] per-group abs-max, symmetric int4)              */
+/* ------------------------------------------------------------------ */
+
+/* codes[d] in [-7,7], scales[d/32]; y already rotated (or not). */
+void oracle_quantize_vector(int d, const float* y, int8_t* codes, float* scales) {
+  int ng = d / ORACLE_GROUP;
+  for (int g = 0; g < ng; ++g) {
+    const float* yg = y + g * ORACLE_GROUP;
+    float amax = 0.0f;
+    for (int i = 0; i < ORACLE_GROUP; ++i) {
+      float a = fabsf(yg[i]);
+      if (a > amax) amax = a;
+    }
+    volatile float seven = 7.0f;          /* keep the division in fp32 IEEE */
+    float s = amax / seven;
+    scales[g] = s;
+    for (int i = 0; i < ORACLE_GROUP; ++i) {
+      int c = 0;
+      if (amax > 0.0f) {
+        volatile float quot = yg[i] / s;  /* fp32 quotient, rounded once */
+        float r = nearbyintf(quot);       /* round half to even (default mode) */
+        if (r > 7.0f) r = 7.0f;
+        if (r < -7.0f) r = -7.0f;
+        c = (int)r;
+      }
+      codes[g * ORACLE_GROUP + i] = (int8_t)c;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* nibble packing ([SRFT] "nibble pack"; byte order is this library's)  */
+/* ------------------------------------------------------------------ */
+/*
+ * Packed row of one vector: d/2 bytes.  Coordinate i (rotated basis) with
+ * group g = i / 32 and in-group index j = i % 32 lives in
+ *     byte  = (j / 4) * (2 * ng) + 2 * g + (j % 4) / 2,      ng = d / 32
+ *     nibble = j % 2          (0 = bits 0..3, 1 = bits 4..7)
+ * as a 4-bit two's-complement code.  I.e. the row is 8 sub-blocks; sub-block
+ * r holds in-group coordinates 4r..4r+3 of every group, two bytes per group.
+ */
+int64_t oracle_packed_byte_index(int d, int i) {
+  int ng = d / ORACLE_GROUP;
+  int g = i / ORACLE_GROUP, j = i % ORACLE_GROUP;
+  return (int64_t)(j / 4) * (2 * ng) + 2 * g + (j % 4) / 2;
+}
+
+void oracle_pack_vector(int d, const int8_t* codes, uint8_t* packed) {
+  memset(packed, 0, (size_t)d / 2);
+  for (int i = 0; i < d; ++i) {
+    int64_t b = oracle_packed_byte_index(d, i);
+    uint8_t nib = (uint8_t)(codes[i] & 0x0F);
+    int shift = ((i % ORACLE_GROUP) % 2) ? 4 : 0;
+    packed[b] = (uint8_t)(packed[b] | (nib << shift));
+  }
+}
+
+void oracle_unpack_vector(int d, const uint8_t* packed, int8_t* codes) {
+  for (int i = 0; i < d; ++i) {
+    int64_t b = oracle_packed_byte_index(d, i);
+    int shift = ((i % ORACLE_GROUP) % 2) ? 4 : 0;
+    int nib = (packed[b] >> shift) & 0x0F;
+    codes[i] = (int8_t)(nib >= 8 ? nib - 16 : nib);
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* quantize-append ([OTM-F] on-the-fly quantization)                    */
+/* ------------------------------------------------------------------ */
+/*
+ * k, v: [B][Hkv][n_new][d] fp32 (dtype 0) or bf16 (dtype 1).
+ * Token n of (b, h) goes to cache row pos[b] + n of that (b, h) slot.
+ * caches: packed [B][Hkv][capacity][d/2], scales [B][Hkv][capacity][d/32].
+ */
+int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                           int n_new, int d, const int32_t* pos, const int8_t* signs,
+                           uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                           float* v_scales, int64_t capacity, int nthreads) {
+  if (d % ORACLE_GROUP != 0 || (d & (d - 1)) != 0) return -1;
+  for (int b = 0; b < B; ++b)
+    if (pos[b] < 0 || (int64_t)pos[b] + n_new > capacity) return -1;
+  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
+  if (!R) return -2;
+  oracle_rotation_matrix(d, signs, R);
+  int ng = d / ORACLE_GROUP;
+  int64_t nvec = (int64_t)B * Hkv * n_new;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#endif
+  for (int64_t idx = 0; idx < nvec; ++idx) {
+    float x[512], y[512];
+    int8_t codes[512];
+    int64_t b = idx / ((int64_t)Hkv * n_new);
+    int64_t h = (idx / n_new) % Hkv;
+    int64_t n = idx % n_new;
+    int64_t row = ((int64_t)b * Hkv + h) * capacity + pos[b] + n;
+    for (int kv = 0; kv < 2; ++kv) {
+      const void* src = kv ? v : k;
+      for (int i = 0; i < d; ++i) x[i] = load_input(src, in_dtype, idx * d + i);
+      if (signs) oracle_rotate_vector(d, R, x, y);
+      else memcpy(y, x, sizeof(float) * (size_t)d);
+      float* sc = (kv ? v_scales : k_scales) + row * ng;
+      uint8_t* pk = (kv ? v_packed : k_packed) + row * (d / 2);
+      oracle_quantize_vector(d, y, codes, sc);
+      oracle_pack_vector(d, codes, pk);
+    }
+  }
+  free(R);
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* decode attention over the packed cache ([OTM] sdpa_int4)             */
+/* ------------------------------------------------------------------ */
+/*
+ * q: [B][Hq][d] fp32/bf16, one query token per sequence.  Query head hq uses
+ * KV head hq / (Hq/Hkv).  Sequence b attends cache rows 0..ctx_lens[b]-1.
+ * out: [B][Hq][d] fp64, in the unrotated basis.
+ *   q_r = R q;  S_t = attn_scale * sum_i q_r[i] * s_k[t][g(i)] * c_k[t][i]
+ *   p = softmax(S);  o_r[i] = sum_t p_t * s_v[t][g(i)] * c_v[t][i];  o = R^T o_r
+ */
+int oracle_sdpa_int4_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int d,
+                            const uint8_t* k_packed, const float* k_scales,
+                            const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                            const int32_t* ctx_lens, const int8_t* signs, double attn_scale,
+                            double* out, int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d % ORACLE_GROUP != 0 || (d & (d - 1)) != 0) return -1;
+  for (int b = 0; b < B; ++b)
+    if (ctx_lens[b] < 1 || ctx_lens[b] > capacity) return -1;
+  int G = Hq / Hkv, ng = d / ORACLE_GROUP;
+  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
+  if (!R) return -2;
+  oracle_rotation_matrix(d, signs, R);
+  int64_t nrows = (int64_t)B * Hq;
+  int fail = 0;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+#endif
+  for (int64_t bh = 0; bh < nrows; ++bh) {
+    int64_t b = bh / Hq, hq = bh % Hq, hk = hq / G;
+    int64_t T = ctx_lens[b];
+    double qv[512], qr[512], orot[512];
+    int8_t codes[512];
+    double* S = (double*)malloc(sizeof(double) * (size_t)T);
+    if (!S) { fail = 1; continue; }
+    for (int i = 0; i < d; ++i) qv[i] = (double)load_input(q, q_dtype, bh * d + i);
+    for (int i = 0; i < d; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * qv[j];
+      qr[i] = acc;
+    }
+    int64_t base = ((int64_t)b * Hkv + hk) * capacity;
+    double smax = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      oracle_unpack_vector(d, k_packed + (base + t) * (d / 2), codes);
+      const float* sk = k_scales + (base + t) * ng;
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i) dot += qr[i] * ((double)sk[i / ORACLE_GROUP] * (double)codes[i]);
+      S[t] = attn_scale * dot;
+      if (S[t] > smax) smax = S[t];
+    }
+    double Z = 0.0;
+    for (int64_t t = 0; t < T; ++t) { S[t] = exp(S[t] - smax); Z += S[t]; }
+    for (int i = 0; i < d; ++i) orot[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+      oracle_unpack_vector(d, v_packed + (base + t) * (d / 2), codes);
+      const float* sv = v_scales + (base + t) * ng;
+      double p = S[t] / Z;
+      for (int i = 0; i < d; ++i) orot[i] += p * ((double)sv[i / ORACLE_GROUP] * (double)codes[i]);
+    }
+    for (int j = 0; j < d; ++j) {   /* o = R^T o_r */
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += R[(int64_t)i * d + j] * orot[i];
+      out[bh * d + j] = acc;
+    }
+    free(S);
+  }
+  free(R);
+  return fail ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* unquantized attention, for the fidelity report only                  */
+/* ------------------------------------------------------------------ */
+/*
+ * k, v: [B][Hkv][capacity][d] fp32/bf16 (the original vectors, unrotated).
+ * out: [B][Hq][d] fp64 = softmax(attn_scale q k^T) v, in fp64.
+ */
+int oracle_exact_attention(const void* q, int q_dtype, const void* k, const void* v,
+                           int kv_dtype, int B, int Hq, int Hkv, int d, int64_t capacity,
+                           const int32_t* ctx_lens, double attn_scale, double* out,
+                           int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+  int G = Hq / Hkv;
+  int64_t nrows = (int64_t)B * Hq;
+  int fail = 0;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+#endif
+  for (int64_t bh = 0; bh < nrows; ++bh) {
+    int64_t b = bh / Hq, hq = bh % Hq, hk = hq / G;
+    int64_t T = ctx_lens[b];
+    double* S = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!S) { fail = 1; continue; }
+    int64_t base = ((int64_t)b * Hkv + hk) * capacity;
+    double smax = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i)
+        dot += (double)load_input(q, q_dtype, bh * d + i) *
+               (double)load_input(k, kv_dtype, (base + t) * d + i);
+      S[t] = attn_scale * dot;
+      if (S[t] > smax) smax = S[t];
+    }
+    double Z = 0.0;
+    for (int64_t t = 0; t < T; ++t) { S[t] = exp(S[t] - smax); Z += S[t]; }
+    for (int i = 0; i < d; ++i) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < T; ++t) acc += S[t] * (double)load_input(v, kv_dtype, (base + t) * d + i);
+      out[bh * d + i] = acc / Z;
+    }
+    free(S);
+  }
+  return fail ? -2 : 0;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

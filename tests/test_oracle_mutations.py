@@ -1,0 +1,45 @@
+"""Shows the oracle pins are sharp: each plausible mistake, planted in a
+temporary copy of the oracle (CPU only), makes tests/test_oracle_pins.py fail.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "scale_divisor_8": ("float s = amax / seven;", "float s = amax / 8.0f;"),
+    "round_half_away": ("float r = nearbyintf(quot);", "float r = roundf(quot);"),
+    "nibble_order_swapped": ("    int shift = ((i % ORACLE_GROUP) % 2) ? 4 : 0;\n    packed[b]",
+                             "    int shift = ((i % ORACLE_GROUP) % 2) ? 0 : 4;\n    packed[b]"),
+    "query_rotated_by_transpose": ("acc += R[(int64_t)i * d + j] * qv[j];",
+                                   "acc += R[(int64_t)j * d + i] * qv[j];"),
+    "output_not_inverse_rotated": ("acc += R[(int64_t)i * d + j] * orot[i];",
+                                   "acc += R[(int64_t)j * d + i] * orot[i];"),
+    "signs_applied_after_hadamard": ("* (double)signs[j];", "* (double)signs[i];"),
+    "value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP]", "(double)sv[0]"),
+    "gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512]",
+                       "hk = hq % Hkv;\n    int64_t T = ctx_lens[b];\n    double qv[512]"),
+    "missing_softmax_normalizer": ("double p = S[t] / Z;", "double p = S[t];"),
+    "byte_index_group_stride": ("+ 2 * g + (j % 4) / 2;", "+ g + (j % 4) / 2;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    (tmp_path / "oracle").mkdir()
+    (tmp_path / "oracle" / "oracle.c").write_text(src.replace(old, new))
+    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), tmp_path / "oracle" / "__init__.py")
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), tmp_path / "tests" / "golden")
+    for f in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), tmp_path / "tests" / f)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_oracle_pins.py"], cwd=tmp_path, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 1 and "failed" in r.stdout, r.stdout[-2000:]

@@ -1,0 +1,395 @@
+"""Pins for the CPU oracle: checks against facts the pages and mathematics fix.
+
+Nothing here re-types the oracle's own formulas.  Each check comes from an
+independent source: the Sylvester recursion for Hadamard matrices,
+orthogonality, the quantizer's half-step error bound, exact recovery of values
+already on the int4 grid, hand-derived round-half-even ties and byte layouts
+(tests/golden), closed-form attention cases, the page's 40 GB -> 12.5 GB
+footprint, and a brute-force numpy softmax on tiny inputs.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from conftest import GOLDEN
+
+
+def sylvester(d):
+    H = np.array([[1.0]])
+    while H.shape[0] < d:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def rand_signs(rng, d):
+    return (rng.integers(0, 2, d) * 2 - 1).astype(np.int8)
+
+
+# ---------------------------------------------------------------- rotation
+
+@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_matches_sylvester_recursion(d):
+    R = oracle.rotation_matrix(d, np.ones(d, np.int8))
+    np.testing.assert_array_equal(np.rint(R * np.sqrt(d)), sylvester(d))
+
+
+@pytest.mark.parametrize("d", [4, 32, 128, 256])
+def test_hadamard_integer_identity(d):
+    H = np.array([[oracle.hadamard_entry(i, j) for j in range(d)] for i in range(d)], np.int64)
+    np.testing.assert_array_equal(H @ H, d * np.eye(d, dtype=np.int64))
+
+
+def test_rotation_hand_values():
+    with open(os.path.join(GOLDEN, "rotation_d2_d4.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    i, cases = 0, 0
+    while i < len(lines):
+        head = dict(kv.split("=") for kv in lines[i].split())
+        d = int(head["d"])
+        signs = np.array([int(s) for s in head["signs"].split(",")], np.int8)
+        want = np.array([[float(x) for x in lines[i + 1 + r].split()] for r in range(d)])
+        R = oracle.rotation_matrix(d, signs)
+        np.testing.assert_allclose(R * np.sqrt(d), want, rtol=0, atol=1e-15)
+        i += 1 + d
+        cases += 1
+    assert cases == 3
+
+
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
+def test_rotation_orthogonal(d):
+    rng = np.random.default_rng(d)
+    R = oracle.rotation_matrix(d, rand_signs(rng, d))
+    assert np.max(np.abs(R.T @ R - np.eye(d))) <= 1e-15
+
+
+def test_rotation_off_is_identity():
+    np.testing.assert_array_equal(oracle.rotation_matrix(64, None), np.eye(64))
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_rotation_preserves_norm_and_dot(d):
+    rng = np.random.default_rng(7)
+    s = rand_signs(rng, d)
+    R = oracle.rotation_matrix(d, s)
+    x = rng.standard_normal((16, d))
+    y = x @ R.T
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    assert abs((R @ q) @ (R @ k) - q @ k) <= 1e-12 * np.linalg.norm(q) * np.linalg.norm(k)
+
+
+def test_rotate_rounds_once_to_fp32():
+    rng = np.random.default_rng(3)
+    d = 128
+    s = rand_signs(rng, d)
+    x = rng.standard_normal((8, d)).astype(np.float32)
+    y = oracle.rotate(x, s)
+    exact = x.astype(np.float64) @ oracle.rotation_matrix(d, s).T
+    # one rounding of the fp64 product: within half an fp32 ulp (plus fp64 noise)
+    ulp = np.spacing(np.abs(exact).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(y.astype(np.float64) - exact) <= 0.5 * ulp + 1e-15)
+
+
+def test_wht_inverse_is_transpose():
+    rng = np.random.default_rng(11)
+    d = 128
+    R = oracle.rotation_matrix(d, rand_signs(rng, d))
+    x = rng.standard_normal(d)
+    np.testing.assert_allclose(R.T @ (R @ x), x, atol=1e-13)
+
+
+# ------------------------------------------------------------ quantization
+
+def _read_ties():
+    with open(os.path.join(GOLDEN, "quant_ties.txt")) as f:
+        lines = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    groups = []
+    for i in range(0, len(lines), 3):
+        assert lines[i][0] == "scale" and lines[i + 1][0] == "values" and lines[i + 2][0] == "codes"
+        groups.append((float(lines[i][1]), np.array(lines[i + 1][1:], np.float32),
+                       np.array(lines[i + 2][1:], np.int64)))
+    return groups
+
+
+def test_quantizer_hand_ties_round_half_even():
+    groups = _read_ties()
+    assert len(groups) == 4
+    y = np.concatenate([g[1] for g in groups])[None, :]    # d = 128, four groups
+    codes, scales = oracle.quantize_vectors(y)
+    np.testing.assert_array_equal(scales[0], np.array([g[0] for g in groups], np.float32))
+    np.testing.assert_array_equal(codes[0].astype(np.int64), np.concatenate([g[2] for g in groups]))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_quantizer_half_step_bound_and_absmax_code(d):
+    rng = np.random.default_rng(d + 1)
+    y = (rng.standard_normal((64, d)) * rng.uniform(0.01, 100, (64, 1))).astype(np.float32)
+    y[0, :32] = 0.0                                   # an all-zero group
+    codes, scales = oracle.quantize_vectors(y)
+    assert codes.min() >= -7 and codes.max() <= 7
+    s = np.repeat(scales.astype(np.float64), 32, axis=1)
+    err = np.abs(y.astype(np.float64) - s * codes)
+    assert np.all(err <= s / 2 * (1 + 2.0 ** -20))
+    grp = np.abs(codes.reshape(64, d // 32, 32)).max(axis=2)
+    nonzero = np.abs(y.reshape(64, d // 32, 32)).max(axis=2) > 0
+    assert np.all(grp[nonzero] == 7)
+    assert np.all(scales[~nonzero] == 0) and np.all(grp[~nonzero] == 0)
+
+
+@pytest.mark.parametrize("d", [32, 128, 256])
+def test_quantizer_exact_recovery_on_grid(d):
+    rng = np.random.default_rng(d + 2)
+    n = 32
+    c = rng.integers(-7, 8, (n, d)).astype(np.int8)
+    c.reshape(n, d // 32, 32)[:, :, 5] = rng.choice([-7, 7], (n, d // 32))
+    e = rng.integers(-20, 20, (n, d // 32)).astype(np.float64)
+    s0 = np.exp2(e)
+    y = (np.repeat(s0, 32, axis=1) * c).astype(np.float32)
+    codes, scales = oracle.quantize_vectors(y)
+    np.testing.assert_array_equal(codes, c)
+    np.testing.assert_array_equal(scales, s0.astype(np.float32))
+
+
+def test_quantizer_scale_is_fp32_division_by_seven():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((40, 32)).astype(np.float32)
+    _, scales = oracle.quantize_vectors(y)
+    amax = np.abs(y).max(axis=1)
+    np.testing.assert_array_equal(scales[:, 0], (amax / np.float32(7)).astype(np.float32))
+
+
+# ----------------------------------------------------------------- packing
+
+def test_pack_hand_layout():
+    with open(os.path.join(GOLDEN, "pack_layout.txt")) as f:
+        lines = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    for i in range(0, len(lines), 3):
+        d = int(lines[i][0].split("=")[1])
+        codes = np.zeros((1, d), np.int8)
+        for tok in lines[i + 1][1:]:
+            k, c = tok.split(":")
+            codes[0, int(k)] = int(c)
+        want = np.zeros(d // 2, np.uint8)
+        for tok in lines[i + 2][1:]:
+            k, b = tok.split(":")
+            want[int(k)] = int(b, 16)
+        packed = oracle.pack(codes)
+        np.testing.assert_array_equal(packed[0], want)
+        np.testing.assert_array_equal(oracle.unpack(packed, d), codes)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
+def test_pack_is_a_bijection(d):
+    idx = sorted(oracle.packed_byte_index(d, i) * 2 + (i % 32) % 2 for i in range(d))
+    assert idx == list(range(d))                     # every nibble used exactly once
+    rng = np.random.default_rng(d)
+    c = rng.integers(-8, 8, (50, d)).astype(np.int8)
+    np.testing.assert_array_equal(oracle.unpack(oracle.pack(c), d), c)
+
+
+def test_compression_closed_form():
+    with open(os.path.join(GOLDEN, "compression.txt")) as f:
+        vals = dict(ln.split() for ln in f if ln.strip() and not ln.startswith("#"))
+    d = int(vals["head_dim"])
+    cache = oracle.empty_cache(1, 1, 1, d)
+    int4_bytes = cache[0].nbytes + cache[1].nbytes
+    assert int4_bytes == int(vals["int4_bytes_per_vector"])
+    assert 2 * d == int(vals["bf16_bytes_per_vector"])
+    assert (2 * d) / int4_bytes == float(vals["ratio"])
+    n = 80 * 8 * 2 * 131072
+    assert n * 2 * d == int(vals["llama70b_128k_bf16_bytes"]) == 40 * 2 ** 30
+    assert n * int4_bytes == int(vals["llama70b_128k_int4_bytes"]) == int(12.5 * 2 ** 30)
+
+
+# ---------------------------------------------------------- quantize-append
+
+def test_quantize_append_positions_and_untouched_rows():
+    rng = np.random.default_rng(9)
+    B, H, n, d, cap = 2, 3, 5, 64, 16
+    k = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    v = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    cache = oracle.empty_cache(B, H, cap, d)
+    for a in cache:
+        a[...] = 0xAB if a.dtype == np.uint8 else -1.0
+    pos = np.array([0, 9], np.int32)
+    oracle.quantize_append(k, v, pos, None, cache)
+    kp, ks, vp, vs = cache
+    for b in range(B):
+        rows = np.arange(pos[b], pos[b] + n)
+        codes, scales = oracle.quantize_vectors(k[b].reshape(-1, d))
+        np.testing.assert_array_equal(kp[b][:, rows].reshape(-1, d // 2), oracle.pack(codes))
+        np.testing.assert_array_equal(ks[b][:, rows].reshape(-1, d // 32), scales)
+        codes, scales = oracle.quantize_vectors(v[b].reshape(-1, d))
+        np.testing.assert_array_equal(vp[b][:, rows].reshape(-1, d // 2), oracle.pack(codes))
+        other = np.setdiff1d(np.arange(cap), rows)
+        assert np.all(kp[b][:, other] == 0xAB) and np.all(vs[b][:, other] == -1.0)
+
+
+def test_quantize_append_bf16_input_is_exact_conversion():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((1, 1, 4, 128)).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)      # truncate to bf16
+    xb = (bits.astype(np.uint32) << 16).view(np.float32)
+    c1 = oracle.empty_cache(1, 1, 4, 128)
+    c2 = oracle.empty_cache(1, 1, 4, 128)
+    s = rand_signs(rng, 128)
+    oracle.quantize_append(bits, bits, [0], s, c1)
+    oracle.quantize_append(xb, xb, [0], s, c2)
+    for a, b in zip(c1, c2):
+        np.testing.assert_array_equal(a, b)
+
+
+# ----------------------------------------------------------------- decode
+
+def _random_cache(rng, B, H, T, d):
+    codes_k = rng.integers(-7, 8, (B, H, T, d)).astype(np.int8)
+    codes_v = rng.integers(-7, 8, (B, H, T, d)).astype(np.int8)
+    sk = rng.uniform(0.05, 0.5, (B, H, T, d // 32)).astype(np.float32)
+    sv = rng.uniform(0.05, 0.5, (B, H, T, d // 32)).astype(np.float32)
+    kp = oracle.pack(codes_k.reshape(-1, d)).reshape(B, H, T, d // 2)
+    vp = oracle.pack(codes_v.reshape(-1, d)).reshape(B, H, T, d // 2)
+    khat = np.repeat(sk.astype(np.float64), 32, axis=-1) * codes_k
+    vhat = np.repeat(sv.astype(np.float64), 32, axis=-1) * codes_v
+    return (kp, sk, vp, sv), khat, vhat
+
+
+def _numpy_attention(q, k, v, scale):
+    """Independent brute force: softmax(scale * q k^T) v with a plain exp/sum."""
+    s = scale * (k @ q)
+    w = np.exp(s - s.max())
+    return (w / w.sum()) @ v
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 7, 40])
+@pytest.mark.parametrize("d", [32, 64])
+def test_decode_brute_force_rotation_off(T, d):
+    rng = np.random.default_rng(T * 100 + d)
+    B, Hkv, G = 2, 2, 3
+    cache, khat, vhat = _random_cache(rng, B, Hkv, T, d)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    scale = 1 / np.sqrt(d)
+    out = oracle.sdpa_int4_decode(q, cache, [T] * B, None, scale, Hkv)
+    for b in range(B):
+        for h in range(Hkv * G):
+            want = _numpy_attention(q[b, h].astype(np.float64), khat[b, h // G], vhat[b, h // G], scale)
+            np.testing.assert_allclose(out[b, h], want, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("T", [1, 5, 33])
+def test_decode_rotation_on_is_attention_in_unrotated_basis(T):
+    """With rotation, the cache holds R k; attention must equal plain attention
+    over the dequantized vectors mapped back by R^T (catches a missing or
+    transposed rotation of q or of the output)."""
+    rng = np.random.default_rng(T)
+    d, Hkv, G = 64, 1, 2
+    s = rand_signs(rng, d)
+    R = oracle.rotation_matrix(d, s)
+    cache, khat_r, vhat_r = _random_cache(rng, 1, Hkv, T, d)
+    q = rng.standard_normal((1, G, d)).astype(np.float32)
+    out = oracle.sdpa_int4_decode(q, cache, [T], s, 0.3, Hkv)
+    k_unrot = khat_r[0, 0] @ R          # rows: R^T k_r
+    v_unrot = vhat_r[0, 0] @ R
+    for h in range(G):
+        want = _numpy_attention(q[0, h].astype(np.float64), k_unrot, v_unrot, 0.3)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-11, atol=1e-12)
+
+
+def test_decode_single_token_returns_value():
+    rng = np.random.default_rng(1)
+    d = 128
+    cache, _, vhat = _random_cache(rng, 1, 1, 1, d)
+    q = rng.standard_normal((1, 4, d)).astype(np.float32)
+    out = oracle.sdpa_int4_decode(q, cache, [1], None, 1.0, 1)
+    for h in range(4):
+        np.testing.assert_array_equal(out[0, h], vhat[0, 0, 0])
+
+
+def test_decode_constant_scores_give_mean():
+    rng = np.random.default_rng(2)
+    d, T = 128, 37
+    cache, _, vhat = _random_cache(rng, 1, 1, T, d)
+    q = np.zeros((1, 2, d), np.float32)
+    s = rand_signs(rng, d)
+    out = oracle.sdpa_int4_decode(q, cache, [T], s, 1.0, 1)
+    R = oracle.rotation_matrix(d, s)
+    np.testing.assert_allclose(out[0, 0], vhat[0, 0].mean(axis=0) @ R, rtol=0, atol=1e-13)
+
+
+def test_decode_gqa_head_mapping_and_ctx_lens():
+    rng = np.random.default_rng(4)
+    B, Hkv, G, d, cap = 2, 4, 2, 32, 9
+    cache, khat, vhat = _random_cache(rng, B, Hkv, cap, d)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    ctx = [9, 4]
+    out = oracle.sdpa_int4_decode(q, cache, ctx, None, 0.5, Hkv)
+    for b in range(B):
+        for h in range(Hkv * G):
+            T = ctx[b]
+            want = _numpy_attention(q[b, h].astype(np.float64), khat[b, h // G, :T], vhat[b, h // G, :T], 0.5)
+            np.testing.assert_allclose(out[b, h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_decode_large_scores_are_stable():
+    rng = np.random.default_rng(6)
+    d, T = 128, 64
+    cache, khat, vhat = _random_cache(rng, 1, 1, T, d)
+    q = (rng.standard_normal((1, 1, d)) * 300).astype(np.float32)
+    out = oracle.sdpa_int4_decode(q, cache, [T], None, 1.0, 1)
+    assert np.all(np.isfinite(out))
+    want = _numpy_attention(q[0, 0].astype(np.float64), khat[0, 0], vhat[0, 0], 1.0)
+    np.testing.assert_allclose(out[0, 0], want, rtol=1e-10, atol=1e-12)
+
+
+def test_decode_bf16_query_equals_fp32_of_same_values():
+    rng = np.random.default_rng(8)
+    d, T = 128, 10
+    cache, _, _ = _random_cache(rng, 1, 1, T, d)
+    x = rng.standard_normal((1, 2, d)).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    xb = (bits.astype(np.uint32) << 16).view(np.float32)
+    s = rand_signs(rng, d)
+    a = oracle.sdpa_int4_decode(bits, cache, [T], s, 0.1, 1)
+    b = oracle.sdpa_int4_decode(xb, cache, [T], s, 0.1, 1)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_end_to_end_on_grid_rotation_off_is_exact_attention():
+    """Quantize-append then decode on inputs already on the int4 grid gives the
+    unquantized attention (up to fp64 rounding)."""
+    rng = np.random.default_rng(10)
+    B, Hkv, G, T, d = 1, 2, 4, 12, 64
+    c = rng.integers(-7, 8, (2, B, Hkv, T, d))
+    c[..., 3] = 7          # every group needs a full-scale code
+    c[..., 35] = -7
+    k = (c[0] * 0.25).astype(np.float32)
+    v = (c[1] * 0.125).astype(np.float32)
+    cache = oracle.empty_cache(B, Hkv, T, d)
+    oracle.quantize_append(k, v, [0], None, cache)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    got = oracle.sdpa_int4_decode(q, cache, [T], None, 0.2, Hkv)
+    want = oracle.exact_attention(q, k, v, [T], 0.2)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+def test_exact_attention_brute_force():
+    rng = np.random.default_rng(13)
+    B, Hkv, G, T, d = 1, 2, 2, 9, 32
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    out = oracle.exact_attention(q, k, v, [T], 0.7)
+    for h in range(Hkv * G):
+        want = _numpy_attention(q[0, h].astype(np.float64), k[0, h // G].astype(np.float64),
+                                v[0, h // G].astype(np.float64), 0.7)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-12, atol=1e-14)
+
+
+def test_oracle_rejects_bad_shapes():
+    q = np.zeros((1, 3, 64), np.float32)
+    cache = oracle.empty_cache(1, 2, 4, 64)
+    with pytest.raises(ValueError):
+        oracle.sdpa_int4_decode(q, cache, [4], None, 1.0, 2)      # 3 % 2 != 0
+    with pytest.raises(ValueError):
+        oracle.sdpa_int4_decode(np.zeros((1, 2, 64), np.float32), cache, [5], None, 1.0, 2)
