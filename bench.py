@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark: one decode step of the int4 KV-cache path on B200.
+
+A step = quantize-append of one new token (K and V of every kv head) into the
+packed int4 cache + sdpa_int4 decode of one query token over the whole
+context, on the 64/8-head, d=128, 128K-context Llama-3.1-70B-shaped layer
+(synthetic seeded inputs, bf16).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (weak scaling, N replicas)
+
+Timing: CUDA events on the launching stream around each step, L2 flushed by
+a 256 MiB write before every timed step (outside the events), barrier +
+synchronize around the K timed steps, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sdpa_int4 decode µs/step + effective KV GB/s (% of 8 TB/s) at 128K ctx"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default="llama70b_gqa_128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kv_bytes(w, ctx_tokens):
+    """Packed codes + fp32 scales of K and V read by one decode (all sequences)."""
+    per_vec = w.head_dim // 2 + 4 * (w.head_dim // 32)
+    return 2 * per_vec * w.num_kv_heads * int(sum(ctx_tokens))
+
+
+def lib_source_hash():
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "compressed_domain_attention_tq_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        with open(os.path.join(cs, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != lib_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.proc = None
+        self.path = f"/tmp/tq_clocks_{os.getpid()}.csv"
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def run_tq(args):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_domain_attention_tq_b200 as tq
+    from compressed_domain_attention_tq_b200 import workloads as wl
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.WORKLOADS[args.workload]
+    seed = args.seed + 1000 * rank
+    B, Hq, Hkv, d, T = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.context
+    stream = torch.cuda.current_stream()
+
+    signs = wl.make_signs(d, seed) if w.rotation else None
+    ctx = wl.make_context_lengths(w, seed)                    # cached tokens per sequence
+    cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
+    k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
+    pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # bulk prefill: all cached tokens quantized in one call
+    prefill = None
+    if not args.no_prefill:
+        times = []
+        for i in range(4):
+            flush.fill_(i)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            cache.append(k_all, v_all, pos0)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i:
+                times.append(e0.elapsed_time(e1) / 1e3)
+        t = min(times)
+        nvec = 2 * B * Hkv * k_all.shape[2]
+        moved = k_all.numel() * k_all.element_size() * 2 + nvec * (d // 2 + 4 * (d // 32))
+        prefill = {"tokens": int(k_all.shape[2]), "us": round(t * 1e6, 2),
+                   "tokens_per_s": round(B * k_all.shape[2] / t, 1),
+                   "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),
+                   "bytes_moved": int(moved)}
+    else:
+        cache.append(k_all, v_all, pos0)
+    del k_all, v_all
+
+    # per-step inputs: one new token appended after the cached context
+    k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
+    q = wl.make_query(w, seed, device=dev)
+    pos = ctx.to(dev)
+    ctx_dev = (ctx + 1).to(dev)
+    max_ctx = int((ctx + 1).max())
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    scale = w.attn_scales[0]
+    ws = cache.workspace(Hq, max_ctx)
+
+    def step():
+        cache.append(k_new, v_new, pos)
+        cache.decode(q, ctx_dev, max_ctx, scale, out)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_((i + 7) & 0xFF)
+        ev[i][0].record(stream)
+        cache.append(k_new, v_new, pos)
+        ev[i][1].record(stream)
+        cache.decode(q, ctx_dev, max_ctx, scale, out)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    t_q = [e[0].elapsed_time(e[1]) / 1e3 for e in ev]
+    t_d = [e[1].elapsed_time(e[2]) / 1e3 for e in ev]
+    t_s = [e[0].elapsed_time(e[2]) / 1e3 for e in ev]
+    step_s = sum(t_s) / len(t_s)
+    dec_s = sum(t_d) / len(t_d)
+    q_s = sum(t_q) / len(t_q)
+    if world > 1:
+        tt = torch.tensor([step_s, dec_s, q_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        step_s, dec_s, q_s = tt.tolist()
+
+    # end to end through the public API with pinned host buffers
+    h_q = q.cpu().pin_memory()
+    h_k, h_v = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+    e2e_t = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        cache.append(d_k, d_v, pos)
+        cache.decode(d_q, ctx_dev, max_ctx, scale, out)
+        h_out.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_t.append(a.elapsed_time(b) / 1e3)
+    e2e_s = sum(e2e_t) / len(e2e_t)
+    if world > 1:
+        tt = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_s = tt.item()
+
+    kvb = kv_bytes(w, (ctx + 1).tolist())
+    qo_bytes = q.numel() * q.element_size() + out.numel() * out.element_size()
+    algo = kvb + qo_bytes
+    peak, peak_kind = measured_peaks()
+    dec_gbs = algo / dec_s / 1e9
+    value = world * kvb / step_s / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
+        "us_per_step": round(step_s * 1e6, 2), "decode_us": round(dec_s * 1e6, 2),
+        "quantize_append_us": round(q_s * 1e6, 2),
+        "pct_of_8TBps": round(100 * kvb / step_s / 1e9 / NOMINAL_HBM_GBS, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 codes, fp32 accumulation", "data": "synthetic (seeded N(0,1), bf16)",
+        "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
+                   "context": max_ctx, "rotation": w.rotation, "attn_scale": scale,
+                   "kv_bytes_per_step": kvb, "l2": "flushed before each timed step (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "sdpa_int4 decode (split-K + merge)",
+                     "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(dec_gbs / peak, 4), "peak_kind": peak_kind,
+                     "algorithmic_bytes": algo, "traffic": ncu_traffic("decode")},
+        "e2e": {"value": round(world * kvb / e2e_s / 1e9, 1), "unit": "GB/s",
+                "us_per_step": round(e2e_s * 1e6, 2),
+                "h2d_bytes_per_step": int(h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()),
+                "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "bulk_prefill": prefill,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, seed)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def oracle_sample(w, seed, kv_head=0):
+    """Inputs of one kv head (its G query heads) at the full context, from the
+    seeded CPU generator, quantized by the oracle."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from compressed_domain_attention_tq_b200 import workloads as wl
+
+    k, v = wl.make_kv(w, seed, device="cpu", tokens=w.capacity)
+    k = k[:1, kv_head:kv_head + 1].contiguous()
+    v = v[:1, kv_head:kv_head + 1].contiguous()
+    G = w.num_q_heads // w.num_kv_heads
+    q = wl.make_query(w, seed)[:1, kv_head * G:(kv_head + 1) * G].contiguous()
+
+    def bits(t):
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    signs = wl.make_signs(w.head_dim, seed).numpy() if w.rotation else None
+    cache = oracle.empty_cache(1, 1, w.capacity, w.head_dim)
+    thr = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.quantize_append(bits(k[:, :, :-1]), bits(v[:, :, :-1]), [0], signs, cache, threads=thr)
+    t_q = time.perf_counter() - t0
+    return dict(k_new=bits(k[:, :, -1:]), v_new=bits(v[:, :, -1:]), q=bits(q), signs=signs,
+                cache=cache, threads=thr, prefill_s=t_q, G=G, T=w.capacity - 1)
+
+
+def oracle_step(s, w):
+    import oracle
+    oracle.quantize_append(s["k_new"], s["v_new"], [s["T"]], s["signs"], s["cache"], threads=s["threads"])
+    return oracle.sdpa_int4_decode(s["q"], s["cache"], [s["T"] + 1], s["signs"], w.attn_scales[0], 1,
+                                   threads=s["threads"])
+
+
+def cpu_baseline(w, seed):
+    s = oracle_sample(w, seed)
+    ts = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        oracle_step(s, w)
+        ts.append(time.perf_counter() - t0)
+    t = min(ts)
+    kvb = 2 * (s["T"] + 1) * (w.head_dim // 2 + 4 * (w.head_dim // 32))
+    return {"value": round(kvb / t / 1e9, 4), "unit": "GB/s", "cores": s["threads"], "kind": "oracle",
+            "us_per_step_sample": round(t * 1e6, 1),
+            "sample": (f"kv head 0 of {w.num_kv_heads} ({s['G']} query heads) at {s['T'] + 1}-token "
+                       f"context: quantize-append 1 token + decode, best of 3; oracle prefill of the "
+                       f"sample took {s['prefill_s']:.1f} s")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from compressed_domain_attention_tq_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    s = oracle_sample(w, args.seed)
+    for _ in range(args.warmup):
+        oracle_step(s, w)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(s, w)
+        ts.append(time.perf_counter() - t0)
+    t = sum(ts) / len(ts)
+    kvb = 2 * (s["T"] + 1) * (w.head_dim // 2 + 4 * (w.head_dim // 32))
+    val = kvb / t / 1e9
+    sample = (f"kv head 0 of {w.num_kv_heads} ({s['G']} query heads) at {s['T'] + 1}-token context; "
+              f"each step = oracle quantize-append of 1 token + fp64 decode")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), bf16)",
+        "config": {"workload": w.name, "batch": 1, "q_heads": s["G"], "kv_heads": 1,
+                   "head_dim": w.head_dim, "context": s["T"] + 1},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": s["threads"], "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_tq(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,115 @@
+"""ctypes binding of libtq (include/tq.h).  Argument marshalling only: every
+step of quantization and attention runs in the CUDA kernels of libtq.so.
+
+There is no fallback: if libtq.so is missing or no CUDA device is present the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtq.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA = 0, -1, -2, -3, -4
+TQ_F32, TQ_BF16 = 0, 1
+
+SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
+           "tq_sdpa_int4_decode", "tq_status_string")
+
+_lib = None
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Load libtq.so (built in-tree by compressed_domain_attention_tq_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: run `python -m compressed_domain_attention_tq_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    lib.tq_quantize_append.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, i64, P]
+    lib.tq_quantize_append.restype = i32
+    lib.tq_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.tq_decode_workspace_bytes.restype = sz
+    lib.tq_decode_chunk_tokens.argtypes = [i32, i32, i32, i32, i32]
+    lib.tq_decode_chunk_tokens.restype = i32
+    lib.tq_sdpa_int4_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64, P, i32,
+                                        P, f32, P, P, sz, P]
+    lib.tq_sdpa_int4_decode.restype = i32
+    lib.tq_status_string.argtypes = [i32]
+    lib.tq_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().tq_status_string(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype == torch.bfloat16:
+        return TQ_BF16
+    raise TypeError(f"expected float32 or bfloat16, got {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+def quantize_append(k, v, pos, signs, k_packed, k_scales, v_packed, v_scales, stream=None):
+    """Quantize k, v [B][Hkv][n_new][d] into cache rows pos[b] .. pos[b]+n_new-1."""
+    _need_cuda(k, v, pos, signs, k_packed, k_scales, v_packed, v_scales)
+    B, H, n, d = k.shape
+    rc = load().tq_quantize_append(_ptr(k), _ptr(v), _dtype_code(k), B, H, n, d, 32, _ptr(pos),
+                                   _ptr(signs), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+                                   _ptr(v_scales), k_packed.shape[2], _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_quantize_append")
+
+
+def decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx) -> int:
+    return int(load().tq_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx))
+
+
+def decode_chunk_tokens(batch, num_q_heads, num_kv_heads, head_dim, max_ctx) -> int:
+    return int(load().tq_decode_chunk_tokens(batch, num_q_heads, num_kv_heads, head_dim, max_ctx))
+
+
+def sdpa_int4_decode(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs,
+                     attn_scale, out, workspace, stream=None):
+    """out[B][Hq][d] (fp32) = attention of q over the packed cache (see include/tq.h)."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out, workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode(_ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, _ptr(k_packed),
+                                    _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+                                    k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs),
+                                    float(attn_scale), _ptr(out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode")

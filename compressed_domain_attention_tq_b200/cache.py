@@ -1,0 +1,58 @@
+"""Int4KVCache: the packed int4 KV cache of one attention layer on one GPU.
+
+The call shape follows the AdapTQ engine (AdapTQ post, section "native Python
+API": an engine of fixed dim, heads and capacity with append(k, v) and
+compute(q)).  Torch only provides the device buffers and the stream; both
+operations run in libtq's kernels.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+
+class Int4KVCache:
+    def __init__(self, batch: int, num_kv_heads: int, head_dim: int, capacity: int,
+                 device="cuda", signs: torch.Tensor | None = None):
+        if head_dim % 32:
+            raise ValueError("head_dim must be a multiple of 32")
+        self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
+        dev = torch.device(device)
+        shape = (batch, num_kv_heads, capacity)
+        self.k_packed = torch.zeros(*shape, head_dim // 2, dtype=torch.uint8, device=dev)
+        self.v_packed = torch.zeros(*shape, head_dim // 2, dtype=torch.uint8, device=dev)
+        self.k_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
+        self.v_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
+        self.signs = None if signs is None else signs.to(device=dev, dtype=torch.int8).contiguous()
+        self._ws = None
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.k_packed, self.v_packed, self.k_scales, self.v_scales))
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor, stream=None) -> None:
+        """Quantize k, v [B][Hkv][n][d] into rows pos[b] .. pos[b]+n-1."""
+        _lib.quantize_append(k, v, pos, self.signs, self.k_packed, self.k_scales, self.v_packed,
+                             self.v_scales, stream)
+
+    def workspace(self, num_q_heads: int, max_ctx: int) -> torch.Tensor:
+        need = _lib.decode_workspace_bytes(self.batch, num_q_heads, self.num_kv_heads, self.head_dim, max_ctx)
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
+        return self._ws
+
+    def decode(self, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
+               attn_scale: float | None = None, out: torch.Tensor | None = None, stream=None):
+        """Attention of q [B][Hq][d] over rows 0..ctx_lens[b]-1; returns fp32 [B][Hq][d]."""
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_int4_decode(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
+                              ctx_lens, max_ctx, self.signs, attn_scale, out, ws, stream)
+        return out

@@ -1,0 +1,150 @@
+// tq_api.cu -- the C ABI of libtq (declared in include/tq.h): host-side
+// validation, the split-K plan, and kernel dispatch.  Nothing here allocates;
+// every buffer belongs to the caller (as in the AdapTQ post, section "zero
+// heap allocation": no allocation on the hot path).
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+namespace tq {
+
+static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Chunk the context so that (B * Hkv * n_chunks) is a few CTAs per SM: each
+// chunk is a multiple of 64 tokens, between 64 and 8192.
+bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan) {
+  if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
+  if (d != 128 && d != 256) return false;
+  const int64_t units = (int64_t)B * Hkv;
+  const int64_t target = 4LL * kSmCount;
+  const int64_t want_chunks = units >= target ? 1 : ceil_div(target, units);
+  int64_t chunk = ceil_div(max_ctx, want_chunks);
+  chunk = ceil_div(chunk, 64) * 64;
+  if (chunk < 64) chunk = 64;
+  if (chunk > 8192) chunk = 8192;
+  plan->chunk = (int)chunk;
+  plan->n_chunks = (int)ceil_div(max_ctx, chunk);
+  plan->part_stride = d + 4;
+  plan->header_bytes = (size_t)ceil_div(4LL * B, 256) * 256;
+  plan->ws_bytes = plan->header_bytes +
+                   sizeof(float) * (size_t)B * Hq * plan->n_chunks * plan->part_stride;
+  return true;
+}
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_status_string(tq_status status) {
+  switch (status) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument (pointer, size, shape or alignment)";
+    case TQ_ERR_UNSUPPORTED: return "unsupported configuration (head_dim, group or GQA ratio)";
+    case TQ_ERR_WORKSPACE: return "workspace missing or smaller than tq_decode_workspace_bytes()";
+    case TQ_ERR_CUDA: return "CUDA launch or runtime error";
+  }
+  return "unknown status";
+}
+
+tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                             int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                             int32_t group, const int32_t* pos, const int8_t* signs,
+                             uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                             float* v_scales, int64_t capacity, void* cuda_stream) {
+  if (!k || !v || !pos || !k_packed || !k_scales || !v_packed || !v_scales) return TQ_ERR_INVALID_ARG;
+  if (in_dtype != TQ_F32 && in_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (batch < 1 || num_kv_heads < 1 || n_new < 1 || capacity < n_new) return TQ_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_packed) || !aligned16(v_packed) ||
+      !aligned16(k_scales) || !aligned16(v_scales))
+    return TQ_ERR_INVALID_ARG;
+  QuantizeArgs a;
+  a.k = k;
+  a.v = v;
+  a.bf16 = in_dtype == TQ_BF16;
+  a.B = batch;
+  a.Hkv = num_kv_heads;
+  a.n_new = n_new;
+  a.d = head_dim;
+  a.pos = pos;
+  a.signs = signs;
+  a.k_packed = k_packed;
+  a.k_scales = k_scales;
+  a.v_packed = v_packed;
+  a.v_scales = v_scales;
+  a.capacity = capacity;
+  return launch_quantize(a, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? TQ_OK
+                                                                                     : TQ_ERR_CUDA;
+}
+
+size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t max_ctx) {
+  DecodePlan p;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p)) return 0;
+  return p.ws_bytes;
+}
+
+int32_t tq_decode_chunk_tokens(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t max_ctx) {
+  DecodePlan p;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p)) return 0;
+  return p.chunk;
+}
+
+tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t group, const uint8_t* k_packed, const float* k_scales,
+                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                              float attn_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* cuda_stream) {
+  if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
+    return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (batch < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads != 0)
+    return TQ_ERR_INVALID_ARG;
+  if (max_ctx < 1 || capacity < max_ctx) return TQ_ERR_INVALID_ARG;
+  if (!(attn_scale > 0.0f) || !isfinite(attn_scale)) return TQ_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (num_q_heads / num_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(v_packed) ||
+      !aligned16(k_scales) || !aligned16(v_scales))
+    return TQ_ERR_INVALID_ARG;
+  DecodeArgs a;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan))
+    return TQ_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < a.plan.ws_bytes) return TQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
+  a.q = q;
+  a.q_bf16 = q_dtype == TQ_BF16;
+  a.B = batch;
+  a.Hq = num_q_heads;
+  a.Hkv = num_kv_heads;
+  a.d = head_dim;
+  a.k_packed = k_packed;
+  a.k_scales = k_scales;
+  a.v_packed = v_packed;
+  a.v_scales = v_scales;
+  a.capacity = capacity;
+  a.ctx_lens = ctx_lens;
+  a.max_ctx = max_ctx;
+  a.signs = signs;
+  a.attn_scale = attn_scale;
+  a.out = out;
+  a.workspace = workspace;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (launch_decode_simt(a, s) != cudaSuccess) return TQ_ERR_CUDA;
+  if (launch_merge(a, s) != cudaSuccess) return TQ_ERR_CUDA;
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// tq_internal.h -- declarations shared by the libtq translation units.
+// Not part of the public ABI (include/tq.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tq {
+
+constexpr int kGroup = 32;  // quantization group (rotated coordinates)
+constexpr int kSmCount = 148;  // B200; sizes the split-K plan (a host-only, device-free choice)
+
+// Split-K work decomposition of one decode call (host side, deterministic).
+struct DecodePlan {
+  int chunk;        // context tokens per chunk (multiple of 64)
+  int n_chunks;     // ceil(max_ctx / chunk)
+  int part_stride;  // floats per (b, q head, chunk) partial: d + 4 (16-byte rows)
+  size_t header_bytes;  // int32 flags[B], rounded up to 256 bytes
+  size_t ws_bytes;  // header + partials
+};
+
+bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan);
+
+struct QuantizeArgs {
+  const void* k;
+  const void* v;
+  int bf16;
+  int B, Hkv, n_new, d;
+  const int32_t* pos;
+  const int8_t* signs;
+  uint8_t* k_packed;
+  float* k_scales;
+  uint8_t* v_packed;
+  float* v_scales;
+  int64_t capacity;
+};
+
+struct DecodeArgs {
+  const void* q;
+  int q_bf16;
+  int B, Hq, Hkv, d;
+  const uint8_t* k_packed;
+  const float* k_scales;
+  const uint8_t* v_packed;
+  const float* v_scales;
+  int64_t capacity;
+  const int32_t* ctx_lens;
+  int max_ctx;
+  const int8_t* signs;
+  float attn_scale;
+  float* out;
+  void* workspace;
+  DecodePlan plan;
+};
+
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace tq

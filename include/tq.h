@@ -1,0 +1,164 @@
+/*
+ * tq.h -- C ABI of libtq: on-the-fly int4 KV-cache quantization and decode
+ * attention computed directly on the packed int4 cache (B200, sm_100a).
+ *
+ * The two operations follow the statement of the problem in
+ * "Open-TQ-Metal: Fused Compressed-Domain Attention for Long-Context LLM
+ * Inference on Apple Silicon" (arXiv 2604.16957v1), abstract: the KV cache is
+ * quantized to int4 as it is generated, and attention (the fused "sdpa_int4"
+ * kernel) runs on the compressed representation with no intermediate
+ * dequantized K/V matrix.  The rotation is the Hadamard rotation of the AdapTQ
+ * post (section "Fast Hadamard Rotation (HAR)") with random signs, which the
+ * "SRFT + int4 KV-cache on Apple Silicon" post (core-method section) reports
+ * as equivalent to its sign-randomized FFT; quantization is that post's
+ * per-group abs-max symmetric int4 with nibble packing.  The call shape
+ * mirrors AdapTQ's engine (section "native Python API": fixed capacity,
+ * append(k, v), compute(q)), and, like that engine (section "zero heap
+ * allocation"), no call allocates: the caller passes every buffer.
+ *
+ * Conventions for every call:
+ *  - All pointers except `signs == NULL` markers are DEVICE pointers on the
+ *    current CUDA device, owned by the caller; the library never allocates,
+ *    frees or retains them.
+ *  - Calls only enqueue work on `cuda_stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and return without synchronizing.
+ *  - Arguments are validated on the host before any launch; an invalid call
+ *    returns an error and enqueues nothing.  A failed launch returns
+ *    TQ_ERR_CUDA.
+ *  - Results are deterministic: the same inputs give bit-identical outputs.
+ *
+ * Data layout (row-major, dense):
+ *  - head_dim d in {128, 256}; group size g = 32; ng = d / 32 groups.
+ *  - packed cache: uint8 [B][Hkv][capacity][d/2], one row per token.  Rotated
+ *    coordinate i (group gi = i/32, in-group j = i%32) is stored as a 4-bit
+ *    two's-complement code in byte (j/4)*(2*ng) + 2*gi + (j%4)/2 of its row,
+ *    low nibble when j is even, high nibble when j is odd.  Codes are in
+ *    [-7, 7].
+ *  - scales: float [B][Hkv][capacity][ng]; scale = fl32(amax / 7) of the
+ *    group's rotated values (0 for an all-zero group).
+ *  - dequantized value of coordinate i = scale[i/32] * code[i], in the
+ *    rotated basis R x, R = H_d diag(signs) / sqrt(d) (Sylvester H_d).
+ *  - Alignment: packed rows, scale rows, q and out must be 16-byte aligned;
+ *    with the layout above this holds when the base pointers are.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = -1,   /* bad pointer, size, shape or alignment */
+  TQ_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. head_dim 64) */
+  TQ_ERR_WORKSPACE = -3,     /* workspace NULL or smaller than required */
+  TQ_ERR_CUDA = -4           /* a CUDA launch or runtime call failed */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/*
+ * tq_quantize_append -- quantize n_new tokens of K and V per (sequence, kv
+ * head) and write them into cache rows pos[b] .. pos[b]+n_new-1 of sequence
+ * b.  ("On-the-fly quantization": Open-TQ-Metal abstract; rotation: AdapTQ
+ * post, section "Fast Hadamard Rotation (HAR)"; abs-max int4 + nibble pack:
+ * SRFT post, core-method section.)
+ *
+ *  k, v        [B][Hkv][n_new][d] inputs, dtype in_dtype (fp32 or bf16).
+ *  group       must be 32.
+ *  pos         device int32 [B]: first cache row to write for each sequence.
+ *              Rows with pos[b]+n >= capacity (or pos[b] < 0) are skipped on
+ *              the device (no write); the host cannot check device memory.
+ *  signs       device int8 [d] of +1/-1, or NULL for no rotation.  Each
+ *              vector x is rotated to y = H_d (signs * x) / sqrt(d) before
+ *              quantization.
+ *  k_packed, v_packed  uint8 [B][Hkv][capacity][d/2] (written rows only).
+ *  k_scales, v_scales  float [B][Hkv][capacity][d/32] (written rows only).
+ *
+ * With signs == NULL the codes and scales are bit-identical to the plain
+ * definition (fp32 IEEE division, round half to even).  With rotation the
+ * rotated vector is computed in fp32, so a code may differ by 1 from one
+ * computed with an exactly rounded rotation.
+ * Returns TQ_ERR_INVALID_ARG for NULL pointers (other than signs), B, Hkv or
+ * n_new < 1, capacity < n_new, misaligned pointers; TQ_ERR_UNSUPPORTED for
+ * head_dim not in {128, 256} or group != 32.
+ */
+TQ_API tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                             int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                             int32_t group, const int32_t* pos, const int8_t* signs,
+                             uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                             float* v_scales, int64_t capacity, void* cuda_stream);
+
+/*
+ * tq_decode_workspace_bytes -- bytes of device workspace tq_sdpa_int4_decode
+ * needs for these sizes (split-K partials and per-sequence flags).  Host only.
+ * Returns 0 for invalid sizes.
+ */
+TQ_API size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t max_ctx);
+
+/*
+ * tq_decode_chunk_tokens -- context tokens per split-K chunk that
+ * tq_sdpa_int4_decode uses for these sizes (host only; a deterministic
+ * function of its arguments).  Returns 0 for invalid sizes.
+ */
+TQ_API int32_t tq_decode_chunk_tokens(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t max_ctx);
+
+/*
+ * tq_sdpa_int4_decode -- GQA decode attention of one query token per
+ * sequence over the packed int4 cache ("fused sdpa_int4": Open-TQ-Metal
+ * abstract; no dequantized K/V matrix is formed: forum summary, section
+ * "eliminating intermediate matrices"; fp32 accumulation with a running
+ * maximum: section "numerical stability").
+ *
+ *  q           [B][Hq][d], dtype q_dtype, in the unrotated basis.
+ *  Hq % Hkv == 0; query head h attends kv head h / (Hq / Hkv).
+ *  ctx_lens    device int32 [B]: sequence b attends cache rows
+ *              0 .. ctx_lens[b]-1.  Must satisfy 1 <= ctx_lens[b] <= max_ctx.
+ *              Values outside that range are clamped on the device; every
+ *              call writes int32 flag[b] at the start of the workspace: 1 if
+ *              ctx_lens[b] was out of range, else 0.
+ *  max_ctx     host bound on ctx_lens (grid sizing); max_ctx <= capacity.
+ *  signs       the same signs the cache was written with, or NULL.
+ *              The query is rotated by them; the output is rotated back.
+ *  attn_scale  softmax temperature: scores = attn_scale * q.k (1/sqrt(d)
+ *              for Llama-style models, 1.0 for Gemma 4: Open-TQ-Metal
+ *              abstract).  Any finite value > 0.
+ *  out         float [B][Hq][d], in the unrotated basis.
+ *  workspace   device scratch of at least
+ *              tq_decode_workspace_bytes(B, Hq, Hkv, d, max_ctx) bytes,
+ *              16-byte aligned; contents need no initialization.
+ *
+ * Returns TQ_ERR_INVALID_ARG for NULL pointers (other than signs), shapes
+ * that do not divide, max_ctx < 1 or > capacity, non-finite or non-positive
+ * attn_scale, misaligned pointers; TQ_ERR_UNSUPPORTED for head_dim not in
+ * {128, 256}, group != 32 or Hq/Hkv > 16; TQ_ERR_WORKSPACE when the
+ * workspace is NULL or too small.
+ */
+TQ_API tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t group, const uint8_t* k_packed, const float* k_scales,
+                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                              float attn_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* cuda_stream);
+
+/* tq_status_string -- static English text for a status code. */
+TQ_API const char* tq_status_string(tq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

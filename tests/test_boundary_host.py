@@ -1,0 +1,157 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol include/tq.h declares, and rejects invalid calls on the host before
+any launch (these calls never reach the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_domain_attention_tq_b200 import _lib
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "tq.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(tq_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from compressed_domain_attention_tq_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert set(_lib.SYMBOLS) <= set(syms) or set(syms) <= set(_lib.SYMBOLS) or syms
+    assert len(syms) >= 5
+    for s in syms:
+        assert hasattr(lib, s), f"libtq.so does not export {s}"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln and ln.split()[-1].startswith("tq_")})
+    assert exported == declared_symbols()
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4):
+        assert _lib.status_string(code)
+    assert "unknown" in _lib.status_string(7)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,T", [(1, 4, 4, 128, 4096), (1, 64, 8, 128, 32769),
+                                          (1, 64, 8, 128, 131073), (16, 64, 8, 128, 65536),
+                                          (4, 32, 16, 256, 65536), (3, 8, 1, 256, 1)])
+def test_decode_plan_properties(lib, B, Hq, Hkv, d, T):
+    chunk = _lib.decode_chunk_tokens(B, Hq, Hkv, d, T)
+    ws = _lib.decode_workspace_bytes(B, Hq, Hkv, d, T)
+    assert chunk % 64 == 0 and 64 <= chunk <= 8192
+    n_chunks = -(-T // chunk)
+    assert (n_chunks - 1) * chunk < T <= n_chunks * chunk
+    header = -(-4 * B // 256) * 256
+    assert ws == header + 4 * B * Hq * n_chunks * (d + 4)
+    assert _lib.decode_workspace_bytes(B, Hq, Hkv, d, T) == ws          # deterministic
+
+
+@pytest.mark.parametrize("args", [(0, 8, 8, 128, 10), (1, 6, 4, 128, 10), (1, 8, 8, 96, 10),
+                                  (1, 8, 8, 128, 0)])
+def test_decode_plan_rejects_invalid_sizes(lib, args):
+    assert _lib.decode_workspace_bytes(*args) == 0
+    assert _lib.decode_chunk_tokens(*args) == 0
+
+
+class FakeBuffers:
+    """Aligned host memory standing in for device pointers; the calls below
+    fail validation before anything dereferences them."""
+
+    def __init__(self):
+        self.buf = ctypes.create_string_buffer(1 << 16)
+        base = ctypes.addressof(self.buf)
+        self.base = (base + 255) // 256 * 256
+
+    def p(self, off=0):
+        return ctypes.c_void_p(self.base + off)
+
+
+def quantize(lib, fb, **kw):
+    a = dict(k=fb.p(0), v=fb.p(256), dtype=1, B=1, H=8, n=1, d=128, group=32, pos=fb.p(512),
+             signs=None, kp=fb.p(1024), ks=fb.p(2048), vp=fb.p(3072), vs=fb.p(4096), cap=16,
+             stream=None)
+    a.update(kw)
+    return lib.tq_quantize_append(a["k"], a["v"], a["dtype"], a["B"], a["H"], a["n"], a["d"],
+                                  a["group"], a["pos"], a["signs"], a["kp"], a["ks"], a["vp"],
+                                  a["vs"], a["cap"], a["stream"])
+
+
+def decode(lib, fb, **kw):
+    a = dict(q=fb.p(0), dtype=1, B=1, Hq=8, Hkv=2, d=128, group=32, kp=fb.p(1024), ks=fb.p(2048),
+             vp=fb.p(3072), vs=fb.p(4096), cap=64, ctx=fb.p(512), max_ctx=64, signs=None,
+             scale=0.125, out=fb.p(8192), ws=fb.p(16384), ws_bytes=1 << 15, stream=None)
+    a.update(kw)
+    return lib.tq_sdpa_int4_decode(a["q"], a["dtype"], a["B"], a["Hq"], a["Hkv"], a["d"],
+                                   a["group"], a["kp"], a["ks"], a["vp"], a["vs"], a["cap"],
+                                   a["ctx"], a["max_ctx"], a["signs"], a["scale"], a["out"],
+                                   a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), _lib.TQ_ERR_INVALID_ARG), (dict(pos=None), _lib.TQ_ERR_INVALID_ARG),
+    (dict(vs=None), _lib.TQ_ERR_INVALID_ARG), (dict(dtype=7), _lib.TQ_ERR_INVALID_ARG),
+    (dict(B=0), _lib.TQ_ERR_INVALID_ARG), (dict(n=0), _lib.TQ_ERR_INVALID_ARG),
+    (dict(cap=0), _lib.TQ_ERR_INVALID_ARG), (dict(n=20, cap=16), _lib.TQ_ERR_INVALID_ARG),
+    (dict(d=64), _lib.TQ_ERR_UNSUPPORTED), (dict(d=96), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(group=64), _lib.TQ_ERR_UNSUPPORTED), ("misaligned_k", _lib.TQ_ERR_INVALID_ARG),
+    ("misaligned_scales", _lib.TQ_ERR_INVALID_ARG)])
+def test_quantize_rejects_on_host(lib, kw, code):
+    fb = FakeBuffers()
+    if kw == "misaligned_k":
+        kw = dict(k=fb.p(2))
+    elif kw == "misaligned_scales":
+        kw = dict(ks=fb.p(2052))
+    assert quantize(lib, fb, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), _lib.TQ_ERR_INVALID_ARG), (dict(ctx=None), _lib.TQ_ERR_INVALID_ARG),
+    (dict(out=None), _lib.TQ_ERR_INVALID_ARG), (dict(dtype=2), _lib.TQ_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.TQ_ERR_INVALID_ARG), (dict(Hq=1, Hkv=2), _lib.TQ_ERR_INVALID_ARG),
+    (dict(max_ctx=0), _lib.TQ_ERR_INVALID_ARG), (dict(max_ctx=65), _lib.TQ_ERR_INVALID_ARG),
+    (dict(scale=0.0), _lib.TQ_ERR_INVALID_ARG), (dict(scale=-1.0), _lib.TQ_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.TQ_ERR_INVALID_ARG), (dict(scale=float("nan")), _lib.TQ_ERR_INVALID_ARG),
+    (dict(d=64), _lib.TQ_ERR_UNSUPPORTED), (dict(group=16), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(Hq=34, Hkv=2), _lib.TQ_ERR_UNSUPPORTED), (dict(ws=None), _lib.TQ_ERR_WORKSPACE),
+    (dict(ws_bytes=100), _lib.TQ_ERR_WORKSPACE), ("misaligned_q", _lib.TQ_ERR_INVALID_ARG),
+    ("misaligned_ws", _lib.TQ_ERR_INVALID_ARG)])
+def test_decode_rejects_on_host(lib, kw, code):
+    fb = FakeBuffers()
+    if kw == "misaligned_q":
+        kw = dict(q=fb.p(4))
+    elif kw == "misaligned_ws":
+        kw = dict(ws=fb.p(16392))
+    assert decode(lib, fb, **kw) == code
+
+
+def test_workspace_size_is_exact_threshold(lib):
+    fb = FakeBuffers()
+    need = _lib.decode_workspace_bytes(1, 8, 2, 128, 64)
+    assert decode(lib, fb, ws_bytes=need - 1) == _lib.TQ_ERR_WORKSPACE
+
+
+def test_product_path_has_no_oracle_import():
+    """The product package never imports the oracle (test infrastructure)."""
+    pkg = os.path.join(ROOT, "compressed_domain_attention_tq_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".h", ".cuh", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "oracle.c" not in txt and "liboracle" not in txt, f

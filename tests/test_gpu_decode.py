@@ -1,0 +1,138 @@
+"""GPU decode attention vs the oracle on the same (oracle-quantized) cache.
+
+The oracle quantizes the seeded inputs; that cache is uploaded and both the
+CUDA path and the oracle attend over it.  Gates: per (sequence, query head)
+relative L2 <= 1e-4 and max abs <= 1e-3 * max|v_hat|.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressed_domain_attention_tq_b200 import _lib
+from conftest import require_cuda
+from helpers import THREADS, check_attention, oracle_cache, to_oracle, upload_cache
+
+pytestmark = pytest.mark.gpu
+
+
+def make_case(B, Hkv, G, d, T_cap, dtype, seed, heavy=False, outliers=False):
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(B, Hkv, T_cap, d, generator=g)
+    v = torch.randn(B, Hkv, T_cap, d, generator=g)
+    if outliers:
+        k[..., [3, 17, 64, 100 % d]] *= 10
+    if heavy:
+        m = torch.rand(B, 1, T_cap, 1, generator=g) < 0.02
+        k = torch.where(m, k * 8, k)
+        v = torch.where(m, v * 8, v)
+    q = torch.randn(B, Hkv * G, d, generator=g)
+    return k.to(dtype), v.to(dtype), q.to(dtype)
+
+
+def run_decode(cache_dev, q, ctx, max_ctx, signs, scale, Hkv):
+    B, Hq, d = q.shape
+    dev = "cuda"
+    ws = torch.empty(_lib.decode_workspace_bytes(B, Hq, Hkv, d, max_ctx), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    kp, ks, vp, vs = cache_dev
+    _lib.sdpa_int4_decode(q.to(dev), kp, ks, vp, vs, torch.tensor(ctx, dtype=torch.int32, device=dev),
+                          max_ctx, None if signs is None else signs.to(dev), scale, out, ws)
+    torch.cuda.synchronize()
+    flags = ws[: 4 * B].view(torch.int32).cpu().numpy()
+    return out.cpu().numpy(), flags
+
+
+def signs_for(d, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+
+
+def parity(B, Hkv, G, d, ctx, dtype=torch.bfloat16, rot=True, scale=None, seed=0, heavy=False,
+           outliers=False, max_ctx=None):
+    max_ctx = max(ctx) if max_ctx is None else max_ctx
+    T_cap = max(max(ctx), max_ctx)
+    k, v, q = make_case(B, Hkv, G, d, T_cap, dtype, seed, heavy, outliers)
+    signs = signs_for(d, seed + 1) if rot else None
+    cache = oracle_cache(k, v, signs)
+    scale = 1 / math.sqrt(d) if scale is None else scale
+    got, flags = run_decode(upload_cache(cache), q, ctx, max_ctx, signs, scale, Hkv)
+    want = oracle.sdpa_int4_decode(to_oracle(q), cache, ctx, None if signs is None else signs.numpy(),
+                                   scale, Hkv, threads=THREADS)
+    assert np.all(flags == 0)
+    return check_attention(got, want, cache, ctx, G, f"B={B} Hkv={Hkv} G={G} d={d} ctx={ctx}")
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("G", [1, 2, 8, 16])
+@pytest.mark.parametrize("T", [1, 31, 64, 65, 1000])
+def test_decode_small_shapes(d, G, T):
+    require_cuda()
+    parity(1, 2, G, d, [T], seed=d + G + T)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_decode_chunk_boundaries(d):
+    require_cuda()
+    B, Hkv, G = 1, 1, 8
+    for T in (2500, 8000):
+        chunk = _lib.decode_chunk_tokens(B, Hkv * G, Hkv, d, T)
+        for t in sorted({chunk - 1, chunk, chunk + 1, 2 * chunk + 5, T}):
+            if 1 <= t <= T:
+                parity(B, Hkv, G, d, [t], seed=t, max_ctx=T)
+
+
+@pytest.mark.parametrize("rot", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_tiny_mha_full_size(rot, dtype):
+    """Tiny MHA decode at its full size: B=1, 4 heads, d=128, 4096 tokens."""
+    require_cuda()
+    parity(1, 4, 1, 128, [4096], dtype=dtype, rot=rot, seed=11)
+
+
+def test_decode_ragged_batch_heavy_rows():
+    require_cuda()
+    ctx = [1, 700, 2049, 3000, 64, 4096]
+    parity(len(ctx), 2, 8, 128, ctx, seed=21, heavy=True)
+
+
+def test_decode_outlier_channels():
+    require_cuda()
+    parity(1, 8, 8, 128, [3333], seed=31, outliers=True)
+
+
+@pytest.mark.parametrize("scale", [1.0, 1 / 16.0])
+def test_decode_wide_head_attn_scales(scale):
+    """d=256, G=2, at attn_scale 1.0 (peaked softmax) and 1/sqrt(256)."""
+    require_cuda()
+    parity(2, 2, 2, 256, [3000, 1777], scale=scale, seed=41)
+
+
+def test_decode_attn_scale_one_d128_peaked():
+    require_cuda()
+    parity(1, 2, 8, 128, [2000], scale=1.0, seed=51)
+
+
+def test_decode_flags_and_clamping():
+    require_cuda()
+    B, Hkv, G, d, T = 3, 1, 4, 128, 200
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 61)
+    signs = signs_for(d, 62)
+    cache = oracle_cache(k, v, signs)
+    got, flags = run_decode(upload_cache(cache), q, [0, 150, 999], 128, signs, 0.1, Hkv)
+    assert list(flags) == [1, 0, 1]
+    want = oracle.sdpa_int4_decode(to_oracle(q), cache, [1, 150, 128], signs.numpy(), 0.1, Hkv)
+    check_attention(got, want, cache, [1, 150, 128], G, "clamped")
+
+
+def test_decode_is_deterministic():
+    require_cuda()
+    B, Hkv, G, d, T = 1, 2, 8, 128, 5000
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 71)
+    signs = signs_for(d, 72)
+    cache = upload_cache(oracle_cache(k, v, signs))
+    a, _ = run_decode(cache, q, [T], T, signs, 0.08, Hkv)
+    b, _ = run_decode(cache, q, [T], T, signs, 0.08, Hkv)
+    np.testing.assert_array_equal(a, b)
