@@ -121,10 +121,11 @@ def test_decode_flags_and_clamping():
     k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 61)
     signs = signs_for(d, 62)
     cache = oracle_cache(k, v, signs)
-    got, flags = run_decode(upload_cache(cache), q, [0, 150, 999], 128, signs, 0.1, Hkv)
+    # max_ctx = 160: 0 is below 1 and 999 above 160, both flagged and clamped
+    got, flags = run_decode(upload_cache(cache), q, [0, 150, 999], 160, signs, 0.1, Hkv)
     assert list(flags) == [1, 0, 1]
-    want = oracle.sdpa_int4_decode(to_oracle(q), cache, [1, 150, 128], signs.numpy(), 0.1, Hkv)
-    check_attention(got, want, cache, [1, 150, 128], G, "clamped")
+    want = oracle.sdpa_int4_decode(to_oracle(q), cache, [1, 150, 160], signs.numpy(), 0.1, Hkv)
+    check_attention(got, want, cache, [1, 150, 160], G, "clamped")
 
 
 def test_decode_is_deterministic():
