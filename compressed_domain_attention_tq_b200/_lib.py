@@ -15,10 +15,12 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA = 0, -1, -2, -3, -4
+TQ_ERR_SCRATCH_LIMIT = -5
+STATIC_SCRATCH_BYTES = 8 << 20   # TQ_STATIC_SCRATCH_BYTES in include/tq.h
 TQ_F32, TQ_BF16 = 0, 1
 
 SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
-           "tq_sdpa_int4_decode", "tq_status_string")
+           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_static_scratch", "tq_status_string")
 
 _lib = None
 
@@ -47,6 +49,9 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64, P, i32,
                                         P, f32, P, P, sz, P]
     lib.tq_sdpa_int4_decode.restype = i32
+    lib.tq_sdpa_int4_decode_static_scratch.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P,
+                                                       i64, P, i32, P, f32, P, P]
+    lib.tq_sdpa_int4_decode_static_scratch.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -113,3 +118,18 @@ def sdpa_int4_decode(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ct
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode")
+
+
+def sdpa_int4_decode_static_scratch(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx,
+                                    signs, attn_scale, out, stream=None):
+    """sdpa_int4_decode using libtq's built-in device scratch instead of a
+    caller workspace (for callers that cannot allocate; see include/tq.h)."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_static_scratch(
+        _ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, _ptr(k_packed), _ptr(k_scales),
+        _ptr(v_packed), _ptr(v_scales), k_packed.shape[2], _ptr(ctx_lens), int(max_ctx),
+        _ptr(signs), float(attn_scale), _ptr(out), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_static_scratch")

@@ -48,6 +48,8 @@ const char* tq_status_string(tq_status status) {
     case TQ_ERR_UNSUPPORTED: return "unsupported configuration (head_dim, group or GQA ratio)";
     case TQ_ERR_WORKSPACE: return "workspace missing or smaller than tq_decode_workspace_bytes()";
     case TQ_ERR_CUDA: return "CUDA launch or runtime error";
+    case TQ_ERR_SCRATCH_LIMIT:
+      return "sizes need more decode scratch than the built-in TQ_STATIC_SCRATCH_BYTES";
   }
   return "unknown status";
 }

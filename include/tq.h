@@ -62,8 +62,12 @@ typedef enum {
   TQ_ERR_INVALID_ARG = -1,   /* bad pointer, size, shape or alignment */
   TQ_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. head_dim 64) */
   TQ_ERR_WORKSPACE = -3,     /* workspace NULL or smaller than required */
-  TQ_ERR_CUDA = -4           /* a CUDA launch or runtime call failed */
+  TQ_ERR_CUDA = -4,          /* a CUDA launch or runtime call failed */
+  TQ_ERR_SCRATCH_LIMIT = -5  /* sizes need more scratch than TQ_STATIC_SCRATCH_BYTES */
 } tq_status;
+
+/* Bytes of the built-in device scratch of tq_sdpa_int4_decode_static_scratch. */
+#define TQ_STATIC_SCRATCH_BYTES (8u << 20)
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 
@@ -153,6 +157,37 @@ TQ_API tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t ba
                               const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
                               float attn_scale, float* out, void* workspace,
                               size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * tq_sdpa_int4_decode_static_scratch -- tq_sdpa_int4_decode without a
+ * caller-provided workspace.  The method's pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory: a plug-in
+ * running inside a host framework that owns all device memory and hands out
+ * no scratch, or a latency-critical caller that cannot accept cudaMalloc's
+ * device-wide synchronization.
+ *
+ * Arguments, validation and results are those of tq_sdpa_int4_decode; the
+ * workspace is a file-scope device array of TQ_STATIC_SCRATCH_BYTES (8 MiB)
+ * inside libtq, which every GPU that loads the library holds until the
+ * process exits.  The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.
+ *  - Sizes whose workspace (tq_decode_workspace_bytes) exceeds
+ *    TQ_STATIC_SCRATCH_BYTES are rejected with TQ_ERR_SCRATCH_LIMIT before
+ *    any launch.
+ *  - The first call on a device looks up the array's device address on that
+ *    device (the current one); make that first call before any stream
+ *    capture.  A failed lookup returns TQ_ERR_CUDA.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents.  The decode writes every scratch byte it reads, so nothing
+ *    needs clearing between calls, but calls whose kernels overlap on the GPU
+ *    (different streams without ordering between them) race on the array and
+ *    give wrong results: order them on one stream or with events.
+ */
+TQ_API tq_status tq_sdpa_int4_decode_static_scratch(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, const uint8_t* k_packed, const float* k_scales,
+    const uint8_t* v_packed, const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out, void* cuda_stream);
 
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);
