@@ -4,6 +4,8 @@
 // heap allocation": no allocation on the hot path).
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include "../../include/tq.h"
 #include "tq_internal.h"
@@ -12,25 +14,41 @@ namespace tq {
 
 static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Chunk the context so that (B * Hkv * n_chunks) is a few CTAs per SM: each
-// chunk is a multiple of 64 tokens, between 64 and 8192.
+// Split the context into chunks (multiples of 128 tokens, the decode's
+// pipeline stage) for persistent CTAs, one per SM: pick the chunk count per
+// sequence that minimises (waves of items over the SMs) x (chunk + a fixed
+// per-item cost), where an item is one (sequence, kv head, chunk).
 bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
   if (d != 128 && d != 256) return false;
   const int64_t units = (int64_t)B * Hkv;
-  const int64_t target = 4LL * kSmCount;
-  const int64_t want_chunks = units >= target ? 1 : ceil_div(target, units);
-  int64_t chunk = ceil_div(max_ctx, want_chunks);
-  chunk = ceil_div(chunk, 64) * 64;
-  if (chunk < 64) chunk = 64;
-  if (chunk > 8192) chunk = 8192;
-  plan->chunk = (int)chunk;
-  plan->n_chunks = (int)ceil_div(max_ctx, chunk);
+  const int64_t step = 128, per_item_cost = 384;
+  const int64_t max_n = ceil_div(max_ctx, step);
+  int64_t best_chunk = ceil_div(max_ctx, step) * step, best_cost = -1;
+  for (int64_t n = 1; n <= max_n && n <= 4096; ++n) {
+    const int64_t chunk = ceil_div(ceil_div(max_ctx, n), step) * step;
+    const int64_t items = units * ceil_div(max_ctx, chunk);
+    const int64_t cost = ceil_div(items, kSmCount) * (chunk + per_item_cost);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_chunk = chunk;
+    }
+  }
+  plan->chunk = (int)best_chunk;
+  plan->n_chunks = (int)ceil_div(max_ctx, best_chunk);
   plan->part_stride = d + 4;
   plan->header_bytes = (size_t)ceil_div(4LL * B, 256) * 256;
   plan->ws_bytes = plan->header_bytes +
                    sizeof(float) * (size_t)B * Hq * plan->n_chunks * plan->part_stride;
   return true;
+}
+
+// A failed CUDA call becomes TQ_ERR_CUDA; with the environment variable
+// TQ_DEBUG set, its CUDA error string is also printed on stderr.
+static tq_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return TQ_OK;
+  if (getenv("TQ_DEBUG")) fprintf(stderr, "libtq: %s: %s\n", where, cudaGetErrorString(e));
+  return TQ_ERR_CUDA;
 }
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -82,8 +100,8 @@ tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, in
   a.v_packed = v_packed;
   a.v_scales = v_scales;
   a.capacity = capacity;
-  return launch_quantize(a, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess ? TQ_OK
-                                                                                     : TQ_ERR_CUDA;
+  return cuda_status(launch_quantize(a, static_cast<cudaStream_t>(cuda_stream)),
+                     "tq_quantize_append");
 }
 
 size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
@@ -144,9 +162,11 @@ tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
   a.out = out;
   a.workspace = workspace;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  if (launch_decode_simt(a, s) != cudaSuccess) return TQ_ERR_CUDA;
-  if (launch_merge(a, s) != cudaSuccess) return TQ_ERR_CUDA;
-  return TQ_OK;
+  const cudaError_t e = decode_mma_supported(head_dim, num_q_heads / num_kv_heads)
+                            ? launch_decode_mma(a, s)
+                            : launch_decode_simt(a, s);
+  if (e != cudaSuccess) return cuda_status(e, "tq_sdpa_int4_decode (split-K kernel)");
+  return cuda_status(launch_merge(a, s), "tq_sdpa_int4_decode (merge kernel)");
 }
 
 }  // extern "C"

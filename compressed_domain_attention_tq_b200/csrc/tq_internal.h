@@ -12,7 +12,7 @@ constexpr int kSmCount = 148;  // B200; sizes the split-K plan (a host-only, dev
 
 // Split-K work decomposition of one decode call (host side, deterministic).
 struct DecodePlan {
-  int chunk;        // context tokens per chunk (multiple of 64)
+  int chunk;        // context tokens per chunk (multiple of 128)
   int n_chunks;     // ceil(max_ctx / chunk)
   int part_stride;  // floats per (b, q head, chunk) partial: d + 4 (16-byte rows)
   size_t header_bytes;  // int32 flags[B], rounded up to 256 bytes
@@ -55,6 +55,8 @@ struct DecodeArgs {
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
+bool decode_mma_supported(int d, int G);
+cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace tq

@@ -54,8 +54,12 @@ def test_status_strings(lib):
 def test_decode_plan_properties(lib, B, Hq, Hkv, d, T):
     chunk = _lib.decode_chunk_tokens(B, Hq, Hkv, d, T)
     ws = _lib.decode_workspace_bytes(B, Hq, Hkv, d, T)
-    assert chunk % 64 == 0 and 64 <= chunk <= 8192
+    assert chunk % 128 == 0 and chunk >= 128      # whole 128-token pipeline stages
     n_chunks = -(-T // chunk)
+    # (sequence, kv head, chunk) items fill their waves over the 148 SMs well
+    if T >= 128 * 148:
+        items = B * Hkv * n_chunks
+        assert items / (-(-items // 148) * 148) >= 0.85
     assert (n_chunks - 1) * chunk < T <= n_chunks * chunk
     header = -(-4 * B // 256) * 256
     assert ws == header + 4 * B * Hq * n_chunks * (d + 4)
