@@ -10,13 +10,15 @@
 // high-precision accumulators, without an approximate softmax).
 //
 // Work: persistent CTAs, one per SM, walk a list of items (sequence b, kv
-// head, context chunk).  A producer warp streams each item's rows (packed K,
-// packed V, K scales, V scales) into a ring of shared-memory stages with 1-D
-// bulk async copies completing on mbarriers; 8 consumer warps each take 16
-// tokens of every stage.  Each warp keeps its own running (max, sum, acc) and
-// the 8 are merged per item in shared memory into one split-K partial
-// (max in log2 units, sum, unnormalized acc[d]) per query head; merge_kernel
-// combines the chunks and rotates the output back.
+// head, context chunk).  Each item's rows (packed K, packed V, K scales, V
+// scales) stream through a ring of shared-memory stages filled by 1-D bulk
+// async copies that complete on mbarriers.  There is no producer warp: every
+// consumer warp takes 16 tokens of each stage, and the last warp to finish a
+// stage (counted with a shared-memory atomic) refills it with the next stage,
+// so all warps of the CTA compute.  Each warp keeps its own running (max, sum,
+// acc); the warps are merged per item in shared memory into one split-K
+// partial (max in log2 units, sum, unnormalized acc[d]) per query head, and
+// merge.cu combines the chunks and rotates the output back.
 //
 // Exactness on the tensor cores.  Codes (-7..7) are exact in f16.  The fp32
 // operand of each contraction is split into hi + lo f16 parts (about 22 bits):
@@ -25,10 +27,11 @@
 //    the product.  Each head's rotated, scaled query is first multiplied by a
 //    power of two so its largest element lies in [2^13, 2^14) (f16 range).
 //    Per group of 32 dims the product is scaled by the token's fp32 K scale.
-//  - P.V: the operand is P' = p * s_v[token, group] * 2^-F_g, split into
-//    hi + lo.  F_g (per warp and group) keeps P' below 2^15: it is set from
-//    the first tile's V scales and raised, with an exact power-of-two rescale
-//    of that group's accumulators, whenever a later tile would overflow.
+//  - P.V: the operand is P' = 2^(S - m - F) * s_v[token, group], split into
+//    hi + lo.  F (per warp) keeps P' below 2^15: it is set from the first
+//    tile's V scales and raised, with an exact power-of-two rescale of the
+//    accumulators and the running sum, whenever a later tile would overflow.
+//    The partial then reports max m + F.
 // Two arrangements (template PATH):
 //  - PATH 0 (heads on rows, 5..8 query heads per kv head, d = 128): scores
 //    C = [q hi; q lo] x K^T; P.V C = [P' hi; P' lo] x V, where the score
@@ -49,11 +52,8 @@
 namespace tq {
 namespace {
 
-constexpr int kWarps = 8;                       // consumer warps per CTA
-constexpr int kMmaThreads = (kWarps + 1) * 32;  // + one producer warp
-constexpr int kStageTokens = 16 * kWarps;       // tokens per pipeline stage
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr long long kWaitCycles = 4000000000LL; // ~2 s at 2 GHz: a wait never lasts this long
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz: a wait never lasts this long
 constexpr uint32_t kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------- PTX helpers
@@ -64,10 +64,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -90,8 +86,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` of `bar`, giving up after kWaitCycles or as soon as
 // another thread of the CTA has set *abort.  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -103,6 +98,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// Bounded wait that ignores *abort (drains copies still in flight).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return;
+}
+
 // 1-D bulk async copy global -> shared (16-byte aligned, size % 16 == 0),
 // completing `bytes` of transaction count on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
@@ -112,10 +114,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           "r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void named_barrier_consumers() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -183,32 +181,65 @@ __device__ __forceinline__ int slot_row(int k) {
   return (k & 8) | (a ^ (3 * (k & 1)));
 }
 
+// 2^x with the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, which no softmax weight here needs)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// 2^e as a float for |e| <= 126
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
 // ------------------------------------------------------------ configuration
 
 template <int D, int PATH>
 struct Cfg {
-  static constexpr int NG = D / 32;        // quantization groups per vector
-  static constexpr int RB = D / 2;         // packed bytes per row
-  static constexpr int SB = 2 * NG;        // bytes of one of a row's 8 sub-blocks
+  static constexpr int NW = 8;                  // warps per CTA (all consumers)
+  static constexpr int TPW = D == 128 ? 2 : 1;  // 16-token tiles per warp per stage
+  static constexpr int THREADS = 32 * NW;
+  static constexpr int ST = 16 * TPW * NW;      // tokens per pipeline stage
+  static constexpr int NG = D / 32;             // quantization groups per vector
+  static constexpr int RB = D / 2;              // packed bytes per row
+  static constexpr int SB = 2 * NG;             // bytes of one of a row's 8 sub-blocks
   static constexpr int NH = PATH == 0 ? 8 : 4;  // query heads per kv head (max)
   static constexpr int NACC = PATH == 0 ? 4 * NG : 2 * NG;  // accumulator fragments
   static constexpr int NS = D == 128 ? 4 : 3;                // pipeline stages
   static constexpr int KC = 0;                               // stage: packed K rows
-  static constexpr int VC = kStageTokens * RB;               //        packed V rows
-  static constexpr int KS = 2 * kStageTokens * RB;           //        K scales
-  static constexpr int VS = KS + kStageTokens * NG * 4;      //        V scales
-  static constexpr int STAGE = VS + kStageTokens * NG * 4;
-  static constexpr int BAR = NS * STAGE;                     // full[NS], empty[NS]
-  static constexpr int QS = BAR + 16 * NS;                   // float [NH][D] query
-  static constexpr int QEXP = QS + 4 * NH * D;               // float [NH]
-  static constexpr int MACC = QEXP + 4 * 8;                  // float [kWarps][NH][D]
-  static constexpr int MM = MACC + 4 * kWarps * NH * D;      // float [kWarps][NH] max
-  static constexpr int ML = MM + 4 * kWarps * NH;            // float [kWarps][NH] sum
-  static constexpr int MW = ML + 4 * kWarps * NH;            // float [kWarps][NH] weight
-  static constexpr int MTOT = MW + 4 * kWarps * NH;          // float [NH] max, [NH] sum
-  static constexpr int ABORT = MTOT + 4 * 2 * NH;            // int
+  static constexpr int VC = ST * RB;                         //        packed V rows
+  static constexpr int KS = 2 * ST * RB;                     //        K scales
+  static constexpr int VS = KS + ST * NG * 4;                //        V scales
+  static constexpr int STAGE = VS + ST * NG * 4;
+  static constexpr int al(int x) { return (x + 127) / 128 * 128; }  // 128-byte regions
+  static constexpr int BAR = NS * STAGE;                     // uint64 full[NS]
+  static constexpr int CNT = al(BAR + 8 * NS);               // int finished-warp count[NS]
+  static constexpr int CUR = al(CNT + 4 * NS);               // int refill cursor[8]
+  static constexpr int QA = al(CUR + 32);                    // f16 [NG][2][16][16] score A
+  static constexpr int QS = al(QA + NG * 2 * 16 * 16 * 2);   // float [NH][D] query
+  static constexpr int QEXP = al(QS + 4 * NH * D);           // float [NH]
+  static constexpr int MACC = al(QEXP + 4 * 8);              // float [NW][NH][D]
+  static constexpr int MM = al(MACC + 4 * NW * NH * D);      // float [NW][NH] max
+  static constexpr int ML = al(MM + 4 * NW * NH);            // float [NW][NH] sum
+  static constexpr int MW = al(ML + 4 * NW * NH);            // float [NW][NH] weight
+  static constexpr int MTOT = al(MW + 4 * NW * NH);          // float [NH] max, [NH] sum
+  static constexpr int ABORT = al(MTOT + 4 * 2 * NH);        // int
   static constexpr int BYTES = ABORT + 16;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
+  static_assert(STAGE % 16 == 0 && VC % 16 == 0 && KS % 16 == 0 && VS % 16 == 0, "alignment");
 };
+
+template <int THREADS>
+__device__ __forceinline__ void barrier_all() {
+  asm volatile("bar.sync 1, %0;" ::"n"(THREADS) : "memory");
+}
 
 __device__ __forceinline__ int clamp_ctx_mma(int T, int max_ctx) {
   return T < 1 ? 1 : (T > max_ctx ? max_ctx : T);
@@ -229,21 +260,61 @@ __device__ __forceinline__ bool item_range(const DecodeArgs& a, int it, int& b, 
   return t0 < t1;
 }
 
-// Per-thread state of one consumer warp for one item.
+// Refill cursor (shared memory, used by one thread at a time): cur[0] item,
+// cur[1] next token, cur[2] end token, cur[3] sequence, cur[4] kv head,
+// cur[5] stages issued.  Issues the next stage of this CTA's stage sequence
+// into `slot`; returns false when the sequence is exhausted.
+template <int D, int PATH>
+__device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* smem, int* cur,
+                                           uint64_t* full, int n_items, int slot) {
+  using C = Cfg<D, PATH>;
+  int it = cur[0], t = cur[1], t1 = cur[2];
+  int b = cur[3], kvh = cur[4];
+  while (t >= t1) {
+    it += gridDim.x;
+    if (it >= n_items) {
+      cur[0] = it;
+      return false;
+    }
+    int c, t0;
+    item_range(a, it, b, kvh, c, t0, t1);
+    t = t0;
+  }
+  const int n = min(C::ST, t1 - t);
+  const uint32_t cb = n * C::RB, sb = n * C::NG * 4;
+  unsigned char* stg = smem + slot * C::STAGE;
+  const int64_t row = ((int64_t)b * a.Hkv + kvh) * a.capacity + t;
+  uint64_t* bar = full + slot;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // earlier reads of the slot
+  mbar_arrive_expect_tx(bar, 2 * cb + 2 * sb);
+  bulk_g2s(stg + C::KC, a.k_packed + row * C::RB, cb, bar);
+  bulk_g2s(stg + C::VC, a.v_packed + row * C::RB, cb, bar);
+  bulk_g2s(stg + C::KS, a.k_scales + row * C::NG, sb, bar);
+  bulk_g2s(stg + C::VS, a.v_scales + row * C::NG, sb, bar);
+  cur[0] = it;
+  cur[1] = t + C::ST;
+  cur[2] = t1;
+  cur[3] = b;
+  cur[4] = kvh;
+  cur[5] += 1;
+  return true;
+}
+
+// Per-thread state of one warp for one item.
 template <int D, int PATH>
 struct WarpState {
-  float acc[Cfg<D, PATH>::NACC][4];     // P.V accumulators (fragments)
-  uint32_t qa[D / 32][2][4];            // score A fragments: [group][k-step][reg]
-  float vsc[D / 32];                    // 2^-F_g: V-scale normalisation per group
-  float m;                              // running max of this thread's head (log2 units)
-  float l;                              // this thread's share of the running sum
-  float qexp;                           // 2^E of this thread's head (query normalisation)
-  bool vset;                            // vsc initialised for this item
+  float acc[Cfg<D, PATH>::NACC][4];  // P.V accumulators (fragments), scaled by 2^-F
+  uint32_t qa_addr;                  // this lane's ldmatrix row address of the score A tiles
+  float m;                           // running max of this thread's head (log2 units)
+  float l;                           // this thread's share of the running sum, scaled by 2^-F
+  float qexp;                        // 2^E of this thread's head (query normalisation)
+  int F;                             // V-scale normalisation exponent
+  bool fset;                         // F chosen for this item
 };
 
 // Rotated, scaled query of the item's G heads -> smem (normalised by a power
-// of two per head), then every consumer thread builds its score A fragments.
-// Warp w < NH prepares head w; the FWHT runs in registers and shuffles.
+// of two per head), then every thread builds its score A fragments.  Warp
+// w < NH prepares head w; the FWHT runs in registers and shuffles.
 template <int D, int PATH>
 __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, unsigned char* smem,
                                            WarpState<D, PATH>& st) {
@@ -293,59 +364,63 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
       int ex = 0;
-      frexpf(amax, &ex);                       // amax = m * 2^ex, m in [0.5, 1)
-      int sh = amax > 0.0f ? 14 - ex : 0;      // amax * 2^sh in [2^13, 2^14)
+      frexpf(amax, &ex);                   // amax = m * 2^ex, m in [0.5, 1)
+      int sh = amax > 0.0f ? 14 - ex : 0;  // amax * 2^sh in [2^13, 2^14)
       sh = max(-120, min(120, sh));
-      const float scale = ldexpf(1.0f, sh);
 #pragma unroll
-      for (int e = 0; e < E; ++e) qs[h * D + lane * E + e] = x[e] * scale;
-      if (lane == 0) qexp[h] = ldexpf(1.0f, -sh);
+      for (int e = 0; e < E; ++e) qs[h * D + lane * E + e] = x[e] * pow2i(sh);
+      if (lane == 0) qexp[h] = pow2i(-sh);
     } else {
 #pragma unroll
       for (int e = 0; e < E; ++e) qs[h * D + lane * E + e] = 0.0f;
       if (lane == 0) qexp[h] = 1.0f;
     }
   }
-  named_barrier_consumers();
-  const int gid = lane >> 2, tig = lane & 3;
+  barrier_all<C::THREADS>();
+  // Score A tiles in shared memory, f16 [group][k-step][row][k]: row r < 8 is
+  // the hi part of head h(r), row 8 + r its lo part; MMA index k of k-step ks
+  // is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in which
+  // the K-code words are unpacked.  The two 16-byte halves of a row swap when
+  // row bit 2 is set, so ldmatrix phases hit distinct banks.
+  __half* qa = reinterpret_cast<__half*>(smem + C::QA);
+  for (int idx = threadIdx.x; idx < (D / 32) * 2 * 256; idx += C::THREADS) {
+    const int k = idx & 15, row = (idx >> 4) & 15, gks = idx >> 8;
+    const int g = gks >> 1, ks = gks & 1;
+    const int hr = PATH == 0 ? (row & 7) : ((row & 7) >> 1);
+    const int dim = 32 * g + 8 * ((k & 7) >> 1) + 2 * ks + (k >> 3) + 4 * (k & 1);
+    const float v = qs[hr * D + dim];
+    const __half hi = __float2half_rn(v);
+    const __half val = row < 8 ? hi : __float2half_rn(v - __half2float(hi));
+    const int half16 = (k >> 3) ^ ((row >> 2) & 1);
+    qa[(gks * 16 + row) * 16 + half16 * 8 + (k & 7)] = val;
+  }
+  barrier_all<C::THREADS>();
+  const int gid = lane >> 2;
   const int hrow = PATH == 0 ? gid : gid >> 1;
-  const float* qr = qs + hrow * D;
-#pragma unroll
-  for (int g = 0; g < D / 32; ++g)
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      const int e0 = 32 * g + 8 * tig + 2 * ks;
-      const float v0 = qr[e0], v1 = qr[e0 + 4], v2 = qr[e0 + 1], v3 = qr[e0 + 5];
-      const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
-      const __half h2 = __float2half_rn(v2), h3 = __float2half_rn(v3);
-      st.qa[g][ks][0] = f16x2(__half2float(h0), __half2float(h1));
-      st.qa[g][ks][1] = f16x2(v0 - __half2float(h0), v1 - __half2float(h1));
-      st.qa[g][ks][2] = f16x2(__half2float(h2), __half2float(h3));
-      st.qa[g][ks][3] = f16x2(v2 - __half2float(h2), v3 - __half2float(h3));
-    }
+  {
+    const int mi = lane >> 3, row = (lane & 7) + 8 * (mi & 1), kb = mi >> 1;
+    st.qa_addr = smem_u32(smem + C::QA) + row * 32 + ((kb ^ ((row >> 2) & 1)) * 16);
+  }
   st.qexp = qexp[hrow];
 }
 
-// Multiply the accumulator fragments of group g by f.
 template <int D, int PATH>
-__device__ __forceinline__ void scale_group(WarpState<D, PATH>& st, int g, float f) {
-  constexpr int PER = PATH == 0 ? 4 : 2;
+__device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
 #pragma unroll
   for (int j = 0; j < Cfg<D, PATH>::NACC; ++j)
-    if (j / PER == g) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) st.acc[j][r] *= f;
-    }
+    for (int r = 0; r < 4; ++r) st.acc[j][r] *= f;
 }
 
-// One 16-token tile of one warp: rows r0 .. r0+15 of the stage, the first
-// `valid` of them real tokens.  rho[i]: tile rows of this thread's MMA slots
-// 2tig, 2tig+1, 8+2tig, 9+2tig; krow[nt]: tile row of score n-tile nt's
-// column gid.
-template <int D, int PATH>
-__device__ __forceinline__ void process_tile(const unsigned char* stg, int r0, int valid, int gid,
-                                             int tig, const int (&rho)[4], const int (&krow)[2],
-                                             WarpState<D, PATH>& st) {
+// TPW consecutive 16-token tiles of one warp: tile u covers rows r0 + 16u ..
+// r0 + 16u + 15 of the stage, and the first `nvalid` rows from r0 on are real
+// tokens (all of them when FULL).  rho[i]: tile rows of this thread's MMA
+// slots 2tig, 2tig+1, 8+2tig, 9+2tig; krow[nt]: tile row of score n-tile nt's
+// column gid.  The tiles share one softmax update.
+template <int D, int PATH, int TPW, bool FULL>
+__device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, int nvalid,
+                                              int gid, int tig, const int (&rho)[4],
+                                              const int (&krow)[2], WarpState<D, PATH>& st) {
   using C = Cfg<D, PATH>;
   constexpr int NG = C::NG, RB = C::RB, SB = C::SB;
   const unsigned char* kc = stg + C::KC + r0 * RB;
@@ -353,179 +428,209 @@ __device__ __forceinline__ void process_tile(const unsigned char* stg, int r0, i
   const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
   const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
 
-  // ---- scores S = qexp * sum_g s_k[t, g] * (q_hi + q_lo) . c_k[t, group g]
-  float S[4];
+  // ---- scores (before the qexp factor) S = sum_g s_k[t, g] * (q_hi + q_lo) . c_k[t, group g]
+  uint32_t kw[TPW][2][NG];  // per tile and n-tile: sub-blocks 2tig, 2tig+1 of token krow[nt]
+  float sk[TPW][4][NG];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    uint32_t kw[NG];  // sub-blocks 2tig and 2tig+1 of the n-tile's token gid
-    const uint4* kp = reinterpret_cast<const uint4*>(kc + krow[nt] * RB + 2 * SB * tig);
+  for (int u = 0; u < TPW; ++u) {
 #pragma unroll
-    for (int q = 0; q < NG / 4; ++q) {
-      const uint4 v = kp[q];
-      kw[4 * q] = v.x;
-      kw[4 * q + 1] = v.y;
-      kw[4 * q + 2] = v.z;
-      kw[4 * q + 3] = v.w;
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint4* kp = reinterpret_cast<const uint4*>(kc + (16 * u + krow[nt]) * RB + 2 * SB * tig);
+#pragma unroll
+      for (int q = 0; q < NG / 4; ++q) {
+        const uint4 v = kp[q];
+        kw[u][nt][4 * q] = v.x;
+        kw[u][nt][4 * q + 1] = v.y;
+        kw[u][nt][4 * q + 2] = v.z;
+        kw[u][nt][4 * q + 3] = v.w;
+      }
     }
-    float sk0[NG], sk1[NG];
 #pragma unroll
-    for (int q = 0; q < NG / 4; ++q) {
-      const float4 a0 = reinterpret_cast<const float4*>(ks + rho[2 * nt] * NG)[q];
-      const float4 a1 = reinterpret_cast<const float4*>(ks + rho[2 * nt + 1] * NG)[q];
-      sk0[4 * q] = a0.x; sk0[4 * q + 1] = a0.y; sk0[4 * q + 2] = a0.z; sk0[4 * q + 3] = a0.w;
-      sk1[4 * q] = a1.x; sk1[4 * q + 1] = a1.y; sk1[4 * q + 2] = a1.z; sk1[4 * q + 3] = a1.w;
-    }
-    float s0 = 0.0f, s1 = 0.0f;
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      // in-group coordinates 8tig .. 8tig+7 of group g, nibble j <-> 8tig + j
-      const uint32_t X = prmt(kw[g / 2], kw[NG / 2 + g / 2], (g & 1) ? 0x7632u : 0x5410u);
-      const uint32_t Y = X >> 8;
-      float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      mma16816(c, st.qa[g][0][0], st.qa[g][0][1], st.qa[g][0][2], st.qa[g][0][3], codes_lo(X),
-               codes_hi(X));
-      mma16816(c, st.qa[g][1][0], st.qa[g][1][1], st.qa[g][1][2], st.qa[g][1][3], codes_lo(Y),
-               codes_hi(Y));
-      s0 = fmaf(sk0[g], c[0] + c[2], s0);
-      s1 = fmaf(sk1[g], c[1] + c[3], s1);
-    }
-    S[2 * nt] = s0 * st.qexp;
-    S[2 * nt + 1] = s1 * st.qexp;
+      for (int q = 0; q < NG / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(ks + (16 * u + rho[i]) * NG)[q];
+        sk[u][i][4 * q] = v.x;
+        sk[u][i][4 * q + 1] = v.y;
+        sk[u][i][4 * q + 2] = v.z;
+        sk[u][i][4 * q + 3] = v.w;
+      }
   }
+  float S[TPW][4];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) S[u][i] = 0.0f;
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    uint32_t a[2][4];
+    ldsm_x4(st.qa_addr + (2 * g) * 512, a[0][0], a[0][1], a[0][2], a[0][3]);
+    ldsm_x4(st.qa_addr + (2 * g + 1) * 512, a[1][0], a[1][1], a[1][2], a[1][3]);
+#pragma unroll
+    for (int u = 0; u < TPW; ++u)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        // in-group coordinates 8tig .. 8tig+7 of group g, nibble j <-> 8tig + j
+        const uint32_t X =
+            prmt(kw[u][nt][g / 2], kw[u][nt][NG / 2 + g / 2], (g & 1) ? 0x7632u : 0x5410u);
+        const uint32_t Y = X >> 8;
+        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], codes_lo(X), codes_hi(X));
+        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], codes_lo(Y), codes_hi(Y));
+        S[u][2 * nt] = fmaf(sk[u][2 * nt][g], c[0] + c[2], S[u][2 * nt]);
+        S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], c[1] + c[3], S[u][2 * nt + 1]);
+      }
+  }
+  bool vld[TPW][4];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      vld[u][i] = FULL || 16 * u + rho[i] < nvalid;
+      if (!vld[u][i]) S[u][i] = -INFINITY;
+    }
 
   // ---- online softmax (log2 units) for this thread's head
-  bool vld[4];
+  float mx = S[0][0];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    vld[i] = rho[i] < valid;
-    if (!vld[i]) S[i] = -INFINITY;
-  }
-  float mx = fmaxf(fmaxf(S[0], S[1]), fmaxf(S[2], S[3]));
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, S[u][i]);
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-  const float m_new = fmaxf(st.m, mx);
+  const float m_new = fmaxf(st.m, mx * st.qexp);
   if (__any_sync(kFull, m_new > st.m)) {
-    const float alpha = exp2f(st.m - m_new);  // 0 on the first tile, 1 if unchanged
+    const float alpha = ex2(st.m - m_new);  // 0 on the first tile, 1 if unchanged
     // PATH 1 accumulates head tig; its softmax state lives on lane 8 * tig
-    const float al = PATH == 0 ? alpha : __shfl_sync(kFull, alpha, 8 * tig);
-#pragma unroll
-    for (int j = 0; j < C::NACC; ++j)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) st.acc[j][r] *= al;
+    scale_acc(st, PATH == 0 ? alpha : __shfl_sync(kFull, alpha, 8 * tig));
     st.l *= alpha;
     st.m = m_new;
   }
-  float p[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = exp2f(S[i] - st.m);
-  st.l += (p[0] + p[1]) + (p[2] + p[3]);
 
-  // ---- P' = p * s_v * 2^-F_g, with F_g kept so that P' < 2^15
-  float sv[4][NG];
+  // ---- V scales and p' = 2^(S - m - F), keeping p' * s_v below 2^15
+  float sv[TPW][4][NG];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int u = 0; u < TPW; ++u)
 #pragma unroll
-    for (int q = 0; q < NG / 4; ++q) {
-      const float4 a = reinterpret_cast<const float4*>(vs + rho[i] * NG)[q];
-      sv[i][4 * q] = vld[i] ? a.x : 0.0f;
-      sv[i][4 * q + 1] = vld[i] ? a.y : 0.0f;
-      sv[i][4 * q + 2] = vld[i] ? a.z : 0.0f;
-      sv[i][4 * q + 3] = vld[i] ? a.w : 0.0f;
-    }
-  float pv[4][NG];
-  float pmax = 0.0f;
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      pv[i][g] = p[i] * (sv[i][g] * st.vsc[g]);
-      pmax = fmaxf(pmax, pv[i][g]);
-    }
-  if (__any_sync(kFull, !st.vset || pmax > 16384.0f)) {
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      float vm = fmaxf(fmaxf(sv[0][g], sv[1][g]), fmaxf(sv[2][g], sv[3][g]));
-      vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 1));
-      vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 2));
-      if (!st.vset || vm * st.vsc[g] > 16384.0f) {
-        int ex = 0;
-        frexpf(vm, &ex);
-        int sh = vm > 0.0f ? 7 - ex : 0;  // vm * 2^sh in [64, 128)
-        sh = max(-120, min(120, sh));
-        const float nv = ldexpf(1.0f, sh);
-        if (st.vset) scale_group(st, g, nv / st.vsc[g]);  // exact: powers of two
-        st.vsc[g] = nv;
+      for (int q = 0; q < NG / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(vs + (16 * u + rho[i]) * NG)[q];
+        sv[u][i][4 * q] = vld[u][i] ? v.x : 0.0f;
+        sv[u][i][4 * q + 1] = vld[u][i] ? v.y : 0.0f;
+        sv[u][i][4 * q + 2] = vld[u][i] ? v.z : 0.0f;
+        sv[u][i][4 * q + 3] = vld[u][i] ? v.w : 0.0f;
       }
+  float smax[TPW][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i][g] = p[i] * (sv[i][g] * st.vsc[g]);
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      smax[u][i] = sv[u][i][0];
+#pragma unroll
+      for (int g = 1; g < NG; ++g) smax[u][i] = fmaxf(smax[u][i], sv[u][i][g]);
     }
-    st.vset = true;
+  float p[TPW][4];
+  float mF = st.m + (float)st.F;
+  float pm = 0.0f;
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
+      pm = fmaxf(pm, p[u][i] * smax[u][i]);
+    }
+  if (__any_sync(kFull, !st.fset || pm > 16384.0f)) {
+    float vm = 0.0f;
+#pragma unroll
+    for (int u = 0; u < TPW; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) vm = fmaxf(vm, smax[u][i]);
+    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 1));
+    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 2));
+    int ex = 0;
+    frexpf(vm, &ex);
+    int Fn = vm > 0.0f ? ex - 7 : 0;  // vm * 2^-Fn in [64, 128)
+    Fn = max(-60, min(60, Fn));
+    if (!st.fset) {
+      st.F = Fn;
+      st.fset = true;
+    } else if (Fn > st.F) {
+      const float f = pow2i(st.F - Fn);  // exact
+      scale_acc(st, f);
+      st.l *= f;
+      st.F = Fn;
+    }
+    mF = st.m + (float)st.F;
+#pragma unroll
+    for (int u = 0; u < TPW; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
   }
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) st.l += (p[u][0] + p[u][1]) + (p[u][2] + p[u][3]);
 
   // ---- P.V on the packed values
-  uint32_t vw[4][NG / 2];  // sub-block gid of rows rho[0..3]
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const unsigned char* vp = vc + rho[i] * RB + SB * gid;
-    if (NG == 4) {
-      const uint2 v = *reinterpret_cast<const uint2*>(vp);
-      vw[i][0] = v.x;
-      vw[i][1] = v.y;
-    } else {
+  for (int u = 0; u < TPW; ++u) {
+    uint32_t vw[4][NG / 2];  // sub-block gid of rows rho[0..3] of tile u
 #pragma unroll
-      for (int q = 0; q < NG / 8; ++q) {
-        const uint4 v = reinterpret_cast<const uint4*>(vp)[q];
-        vw[i][4 * q] = v.x;
-        vw[i][4 * q + 1] = v.y;
-        vw[i][4 * q + 2] = v.z;
-        vw[i][4 * q + 3] = v.w;
+    for (int i = 0; i < 4; ++i) {
+      const unsigned char* vp = vc + (16 * u + rho[i]) * RB + SB * gid;
+      if (NG == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(vp);
+        vw[i][0] = v.x;
+        vw[i][1] = v.y;
+      } else {
+#pragma unroll
+        for (int q = 0; q < NG / 8; ++q) {
+          const uint4 v = reinterpret_cast<const uint4*>(vp)[q];
+          vw[i][4 * q] = v.x;
+          vw[i][4 * q + 1] = v.y;
+          vw[i][4 * q + 2] = v.z;
+          vw[i][4 * q + 3] = v.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
+      // codes c = 0..3 of dims 32g + 4gid + c: low halves rows rho0 / rho2,
+      // high halves rows rho1 / rho3
+      const uint32_t X = prmt(vw[0][g / 2], vw[1][g / 2], sel);
+      const uint32_t Y = prmt(vw[2][g / 2], vw[3][g / 2], sel);
+      const float x0 = p[u][0] * sv[u][0][g], x1 = p[u][1] * sv[u][1][g];
+      const float x2 = p[u][2] * sv[u][2][g], x3 = p[u][3] * sv[u][3][g];
+      const float h0 = split_hi(x0), h1 = split_hi(x1), h2 = split_hi(x2), h3 = split_hi(x3);
+      if (PATH == 0) {
+        const uint32_t a0 = f16x2(h0, h1), a1 = f16x2(x0 - h0, x1 - h1);
+        const uint32_t a2 = f16x2(h2, h3), a3 = f16x2(x2 - h2, x3 - h3);
+        mma16816(st.acc[4 * g + 0], a0, a1, a2, a3, codes_lo(X), codes_lo(Y));
+        mma16816(st.acc[4 * g + 1], a0, a1, a2, a3, codes_hi(X), codes_hi(Y));
+        mma16816(st.acc[4 * g + 2], a0, a1, a2, a3, codes_lo(X >> 8), codes_lo(Y >> 8));
+        mma16816(st.acc[4 * g + 3], a0, a1, a2, a3, codes_hi(X >> 8), codes_hi(Y >> 8));
+      } else {
+        const bool lo = gid & 1;  // column gid = (head gid / 2, part gid % 2)
+        const uint32_t b0 = f16x2(lo ? x0 - h0 : h0, lo ? x1 - h1 : h1);
+        const uint32_t b1 = f16x2(lo ? x2 - h2 : h2, lo ? x3 - h3 : h3);
+        mma16816(st.acc[2 * g + 0], codes_lo(X), codes_hi(X), codes_lo(Y), codes_hi(Y), b0, b1);
+        mma16816(st.acc[2 * g + 1], codes_lo(X >> 8), codes_hi(X >> 8), codes_lo(Y >> 8),
+                 codes_hi(Y >> 8), b0, b1);
       }
     }
   }
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
-    // codes c = 0..3 of dims 32g + 4gid + c: low halves rows rho0 / rho2,
-    // high halves rows rho1 / rho3
-    const uint32_t X = prmt(vw[0][g / 2], vw[1][g / 2], sel);
-    const uint32_t Y = prmt(vw[2][g / 2], vw[3][g / 2], sel);
-    const float h0 = split_hi(pv[0][g]), h1 = split_hi(pv[1][g]);
-    const float h2 = split_hi(pv[2][g]), h3 = split_hi(pv[3][g]);
-    if (PATH == 0) {
-      const uint32_t a0 = f16x2(h0, h1), a1 = f16x2(pv[0][g] - h0, pv[1][g] - h1);
-      const uint32_t a2 = f16x2(h2, h3), a3 = f16x2(pv[2][g] - h2, pv[3][g] - h3);
-      mma16816(st.acc[4 * g + 0], a0, a1, a2, a3, codes_lo(X), codes_lo(Y));
-      mma16816(st.acc[4 * g + 1], a0, a1, a2, a3, codes_hi(X), codes_hi(Y));
-      mma16816(st.acc[4 * g + 2], a0, a1, a2, a3, codes_lo(X >> 8), codes_lo(Y >> 8));
-      mma16816(st.acc[4 * g + 3], a0, a1, a2, a3, codes_hi(X >> 8), codes_hi(Y >> 8));
-    } else {
-      const bool lo = gid & 1;  // column gid = (head gid / 2, part gid % 2)
-      const uint32_t b0 = f16x2(lo ? pv[0][g] - h0 : h0, lo ? pv[1][g] - h1 : h1);
-      const uint32_t b1 = f16x2(lo ? pv[2][g] - h2 : h2, lo ? pv[3][g] - h3 : h3);
-      mma16816(st.acc[2 * g + 0], codes_lo(X), codes_hi(X), codes_lo(Y), codes_hi(Y), b0, b1);
-      mma16816(st.acc[2 * g + 1], codes_lo(X >> 8), codes_hi(X >> 8), codes_lo(Y >> 8),
-               codes_hi(Y >> 8), b0, b1);
-    }
-  }
 }
 
-// Wait for phase `parity` of `bar` for at most kWaitCycles (used only to drain
-// copies still in flight after the pipeline gave up).
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return;
-}
-
-// End of an item: the 8 warps' (max, sum, acc) per head are merged in shared
-// memory and written as the item's split-K partial.  If the pipeline gave up,
-// the partial's max is NaN, so the decode's output for these heads is NaN.
+// End of an item: the warps' (max, sum, acc) per head are merged in shared
+// memory and written as the item's split-K partial (max reported as m + F,
+// with sum and acc scaled by 2^-F).  If the pipeline gave up, the partial's
+// max is NaN, so the decode's output for these heads is NaN.
 template <int D, int PATH>
 __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* smem,
                                             const WarpState<D, PATH>& st, int b, int kvh, int c,
                                             bool aborted) {
   using C = Cfg<D, PATH>;
-  constexpr int NH = C::NH, NG = C::NG;
+  constexpr int NH = C::NH, NG = C::NG, NW = C::NW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int G = a.Hq / a.Hkv;
@@ -538,7 +643,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
   float l = st.l;
   l += __shfl_xor_sync(kFull, l, 1);
   l += __shfl_xor_sync(kFull, l, 2);
-  const float m = aborted ? __int_as_float(0x7fc00000) : st.m;
+  const float m = aborted ? __int_as_float(0x7fc00000) : st.m + (float)st.F;
   if (PATH == 0) {
     if (tig == 0) {
       mm[warp * NH + gid] = m;
@@ -546,14 +651,12 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
     }
     float* dst = macc + (warp * NH + gid) * D;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      const float inv = 1.0f / st.vsc[g];  // exact: a power of two
+    for (int g = 0; g < NG; ++g)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        dst[32 * g + 8 * tig + cc] = (st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2]) * inv;
-        dst[32 * g + 8 * tig + 4 + cc] = (st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3]) * inv;
+        dst[32 * g + 8 * tig + cc] = st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2];
+        dst[32 * g + 8 * tig + 4 + cc] = st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3];
       }
-    }
   } else {
     if (tig == 0 && (gid & 1) == 0) {
       mm[warp * NH + (gid >> 1)] = m;
@@ -561,25 +664,23 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
     }
     float* dst = macc + (warp * NH + tig) * D;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      const float inv = 1.0f / st.vsc[g];
+    for (int g = 0; g < NG; ++g)
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {
         const int dim = 32 * g + 4 * gid + 2 * pp;
-        dst[dim] = (st.acc[2 * g + pp][0] + st.acc[2 * g + pp][1]) * inv;
-        dst[dim + 1] = (st.acc[2 * g + pp][2] + st.acc[2 * g + pp][3]) * inv;
+        dst[dim] = st.acc[2 * g + pp][0] + st.acc[2 * g + pp][1];
+        dst[dim + 1] = st.acc[2 * g + pp][2] + st.acc[2 * g + pp][3];
       }
-    }
   }
-  named_barrier_consumers();
+  barrier_all<C::THREADS>();
   const int tid = threadIdx.x;
   if (tid < G) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * NH + tid]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mm[w * NH + tid]);
     float L = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const float wt = exp2f(mm[w * NH + tid] - M);  // NaN if that warp gave up
       mw[w * NH + tid] = wt;
       L = fmaf(wt, ml[w * NH + tid], L);
@@ -587,15 +688,15 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
     mtot[tid] = M;
     mtot[NH + tid] = L;
   }
-  named_barrier_consumers();
+  barrier_all<C::THREADS>();
   const int stride = a.plan.part_stride;
   float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) +
                                          a.plan.header_bytes);
-  for (int idx = tid; idx < G * D; idx += kWarps * 32) {
+  for (int idx = tid; idx < G * D; idx += C::THREADS) {
     const int h = idx / D, i = idx % D;
     float s = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) s = fmaf(mw[w * NH + h], macc[(w * NH + h) * D + i], s);
+    for (int w = 0; w < NW; ++w) s = fmaf(mw[w * NH + h], macc[(w * NH + h) * D + i], s);
     float* dst = part + (((int64_t)b * a.Hq + (int64_t)kvh * G + h) * a.plan.n_chunks + c) * stride;
     dst[i] = s;
     if (i == 0) {
@@ -605,62 +706,32 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
   }
 }
 
-// Producer: one thread streams every stage of this CTA's items.
 template <int D, int PATH>
-__device__ __forceinline__ void produce(const DecodeArgs& a, unsigned char* smem, uint64_t* full,
-                                        uint64_t* empty, volatile int* abort, int n_items) {
-  using C = Cfg<D, PATH>;
-  uint32_t sc = 0;  // stages issued so far
-  bool ok = true;
-  for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-    int b, kvh, c, t0, t1;
-    if (!item_range(a, it, b, kvh, c, t0, t1)) continue;
-    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.capacity;
-    for (int t = t0; t < t1; t += kStageTokens, ++sc) {
-      const int slot = sc % C::NS;
-      const uint32_t round = sc / C::NS;
-      if (!mbar_wait(empty + slot, (round & 1) ^ 1, abort)) {
-        ok = false;
-        break;
-      }
-      const int n = min(kStageTokens, t1 - t);
-      const uint32_t cb = n * C::RB, sb = n * C::NG * 4;
-      unsigned char* stg = smem + slot * C::STAGE;
-      const int64_t row = row0 + t;
-      mbar_arrive_expect_tx(full + slot, 2 * cb + 2 * sb);
-      bulk_g2s(stg + C::KC, a.k_packed + row * C::RB, cb, full + slot);
-      bulk_g2s(stg + C::VC, a.v_packed + row * C::RB, cb, full + slot);
-      bulk_g2s(stg + C::KS, a.k_scales + row * C::NG, sb, full + slot);
-      bulk_g2s(stg + C::VS, a.v_scales + row * C::NG, sb, full + slot);
-    }
-  }
-  if (!ok)  // copies still in flight must land before the CTA exits
-    for (uint32_t s = sc > (uint32_t)C::NS ? sc - C::NS : 0; s < sc; ++s)
-      mbar_drain(full + s % C::NS, (s / C::NS) & 1);
-}
-
-template <int D, int PATH>
-__global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(DecodeArgs a) {
   using C = Cfg<D, PATH>;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR);
-  uint64_t* empty = full + C::NS;
+  int* cnt = reinterpret_cast<int*>(smem + C::CNT);
+  int* cur = reinterpret_cast<int*>(smem + C::CUR);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::ABORT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, kWarps);
+      cnt[s] = 0;
     }
     *abort = 0;
+    cur[0] = (int)blockIdx.x - (int)gridDim.x;  // before this CTA's first item
+    cur[1] = cur[2] = cur[3] = cur[4] = cur[5] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int s = 0; s < C::NS; ++s)
+      if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
   }
+  // the merge kernel may be scheduled now; it waits for this grid's writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
-  const int n_items = a.B * a.Hkv * a.plan.n_chunks;
-  if (warp == kWarps) {
-    if (lane == 0) produce<D, PATH>(a, smem, full, empty, abort, n_items);
-    return;
-  }
+
   const int gid = lane >> 2, tig = lane & 3;
   const int rho[4] = {slot_row(2 * tig), slot_row(2 * tig + 1), 8 + slot_row(2 * tig),
                       8 + slot_row(2 * tig + 1)};
@@ -679,37 +750,52 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(DecodeArgs a
     for (int j = 0; j < C::NACC; ++j)
 #pragma unroll
       for (int r = 0; r < 4; ++r) st.acc[j][r] = 0.0f;
-#pragma unroll
-    for (int g = 0; g < C::NG; ++g) st.vsc[g] = 1.0f;
     st.m = -INFINITY;
     st.l = 0.0f;
-    st.vset = false;
-    for (int t = t0; t < t1; t += kStageTokens, ++sc) {
+    st.F = 0;
+    st.fset = false;
+    for (int t = t0; t < t1; t += C::ST, ++sc) {
       const int slot = sc % C::NS;
-      const uint32_t round = sc / C::NS;
-      const bool ok = mbar_wait(full + slot, round & 1, abort);
-      const int valid = min(16, min(kStageTokens, t1 - t) - 16 * warp);
-      if (ok && valid > 0)
-        process_tile<D, PATH>(smem + slot * C::STAGE, 16 * warp, valid, gid, tig, rho, krow, st);
+      const bool ok = mbar_wait(full + slot, (sc / C::NS) & 1, abort);
+      const int nvalid = min(16 * C::TPW, min(C::ST, t1 - t) - 16 * C::TPW * warp);
+      const unsigned char* stg = smem + slot * C::STAGE;
+      if (ok && nvalid == 16 * C::TPW)
+        process_tiles<D, PATH, C::TPW, true>(stg, 16 * C::TPW * warp, nvalid, gid, tig, rho, krow,
+                                             st);
+      else if (ok && nvalid > 0)
+        process_tiles<D, PATH, C::TPW, false>(stg, 16 * C::TPW * warp, nvalid, gid, tig, rho,
+                                              krow, st);
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty + slot);
+      if (lane == 0) {  // the last warp out of the stage refills it
+        __threadfence_block();
+        if (atomicAdd(cnt + slot, 1) == C::NW - 1) {
+          cnt[slot] = 0;
+          __threadfence_block();
+          if (!*abort) issue_next<D, PATH>(a, smem, cur, full, n_items, slot);
+        }
+      }
     }
     finish_item<D, PATH>(a, smem, st, b, kvh, c, *abort != 0);
+  }
+  if (threadIdx.x == 0 && *abort) {  // copies still in flight must land before exit
+    const uint32_t issued = (uint32_t)cur[5];
+    for (uint32_t s = issued > (uint32_t)C::NS ? issued - C::NS : 0; s < issued; ++s)
+      mbar_drain(full + s % C::NS, (s / C::NS) & 1);
   }
 }
 
 template <int D, int PATH>
 cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
   using C = Cfg<D, PATH>;
-  cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D, PATH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES);
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(decode_mma_kernel<D, PATH>, C::BYTES, smem_set);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kSmCount;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   const int grid = n_items < sms ? n_items : sms;
-  decode_mma_kernel<D, PATH><<<grid, kMmaThreads, C::BYTES, stream>>>(a);
+  decode_mma_kernel<D, PATH><<<grid, C::THREADS, C::BYTES, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -717,6 +803,11 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
 
 bool decode_mma_supported(int d, int G) {
   return (d == 128 && G >= 1 && G <= 8) || (d == 256 && G >= 1 && G <= 4);
+}
+
+int decode_stage_tokens(int d, int G) {
+  if (!decode_mma_supported(d, G)) return 128;
+  return d == 128 ? Cfg<128, 0>::ST : Cfg<256, 1>::ST;
 }
 
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {

@@ -1,5 +1,5 @@
 // decode_simt.cu -- split-K decode attention on the packed int4 cache using
-// CUDA cores, and the log-sum-exp merge that finishes every decode call.
+// CUDA cores (the path for GQA shapes the tensor-core decode does not cover).
 //
 // Attention runs directly on the packed codes ("fused sdpa_int4",
 // Open-TQ-Metal abstract): codes are unpacked in registers and scaled by
@@ -11,8 +11,8 @@
 // CTA (chunk, kv head, sequence): loads the G = Hq/Hkv query rows, rotates
 // them with the cache's signs, then streams the chunk's K/V tiles through
 // shared memory.  Each chunk leaves (running max m in log2 units, sum l,
-// unnormalized acc[d]) per query head in the workspace; the merge kernel
-// combines the chunks and rotates the result back (R^T = diag(signs) H / sqrt d).
+// unnormalized acc[d]) per query head in the workspace; merge.cu combines the
+// chunks and rotates the result back.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -62,6 +62,7 @@ template <int D>
 __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   constexpr int NG = D / 32, ROWB = D / 2, ROWP = ROWB + 16;
   constexpr int SLICES = D / 8;                 // 8-coordinate slices per head
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
   const int raw_T = a.ctx_lens[b];
@@ -213,35 +214,6 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   }
 }
 
-// merge: one CTA of D threads per (sequence, query head)
-template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
-  __shared__ float o[D];
-  const int b = blockIdx.x / a.Hq;
-  const int hq = blockIdx.x % a.Hq;
-  const int T = clamp_ctx(a.ctx_lens[b], a.max_ctx);
-  const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
-  const float* part = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
-                                                     a.plan.header_bytes) +
-                      ((int64_t)b * a.Hq + hq) * a.plan.n_chunks * a.plan.part_stride;
-  const int stride = a.plan.part_stride;
-  float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, part[c * stride + D]);
-  float L = 0.0f, acc = 0.0f;
-  const int i = threadIdx.x;
-  for (int c = 0; c < nc; ++c) {
-    const float w = exp2f(part[c * stride + D] - M);
-    L = fmaf(w, part[c * stride + D + 1], L);
-    acc = fmaf(w, part[c * stride + i], acc);
-  }
-  o[i] = acc / L;
-  if (a.signs) {
-    fwht_rows<D>(o, 1);
-    o[i] = o[i] * (float)a.signs[i] * rsqrtf((float)D);
-  }
-  a.out[((int64_t)b * a.Hq + hq) * D + i] = o[i];
-}
-
 template <int D>
 size_t simt_smem_bytes(int G) {
   constexpr int NG = D / 32, ROWP = D / 2 + 16;
@@ -256,20 +228,21 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
   dim3 grid(a.plan.n_chunks, a.Hkv, a.B);
   if (a.d == 128) {
     const size_t sm = simt_smem_bytes<128>(G);
-    cudaFuncSetAttribute(decode_simt_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    static std::atomic<uint64_t> smem_set{0};
+    // the limit covers every group size the host accepts (up to 16 query heads)
+    const cudaError_t e =
+        ensure_smem_limit(decode_simt_kernel<128>, (int)simt_smem_bytes<128>(16), smem_set);
+    if (e != cudaSuccess) return e;
     decode_simt_kernel<128><<<grid, 128, sm, stream>>>(a);
   } else {
     const size_t sm = simt_smem_bytes<256>(G);
-    cudaFuncSetAttribute(decode_simt_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    static std::atomic<uint64_t> smem_set{0};
+    // the limit covers every group size the host accepts (up to 16 query heads)
+    const cudaError_t e =
+        ensure_smem_limit(decode_simt_kernel<256>, (int)simt_smem_bytes<256>(16), smem_set);
+    if (e != cudaSuccess) return e;
     decode_simt_kernel<256><<<grid, 128, sm, stream>>>(a);
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
-  const int blocks = a.B * a.Hq;
-  if (a.d == 128) merge_kernel<128><<<blocks, 128, 0, stream>>>(a);
-  else merge_kernel<256><<<blocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

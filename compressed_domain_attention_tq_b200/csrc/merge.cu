@@ -1,0 +1,141 @@
+// merge.cu -- the second kernel of every decode call: combines the split-K
+// partials of each (sequence, query head) by log-sum-exp and rotates the
+// result back to the unrotated basis.
+//
+// Partial c of a head holds (acc[0..d), m, l): the chunk's unnormalized sum
+// of p v in the rotated basis, its running max m (log2 units) and sum l.
+//   M = max_c m_c,  w_c = 2^(m_c - M),  o_rot = sum_c w_c acc_c / sum_c w_c l_c
+//   o = R^T o_rot = diag(signs) H o_rot / sqrt(d)   (R = H diag(signs) / sqrt(d))
+// (Open-TQ-Metal abstract: the attention output is that of the compressed
+// cache; the query was rotated by the cache's signs, so V's output is rotated
+// back.)
+//
+// One CTA of d threads per (sequence, query head).  The kernel is launched
+// with programmatic stream serialization: it may start while the split-K
+// kernel drains and waits at griddepcontrol.wait before reading partials.
+#include <math.h>
+
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r += red[w];
+  __syncthreads();
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
+  extern __shared__ float ml_s[];  // [n_chunks] chunk max, then weight; [n_chunks] chunk sum
+  __shared__ float o[D];
+  __shared__ float red[8];
+  const int b = blockIdx.x / a.Hq;
+  const int hq = blockIdx.x % a.Hq;
+  const int i = threadIdx.x;
+  // inputs the split-K kernel does not write are read before waiting for it
+  const int raw = a.ctx_lens[b];
+  const float sgn = a.signs ? (float)a.signs[i] : 1.0f;
+  const int T = raw < 1 ? 1 : (raw > a.max_ctx ? a.max_ctx : raw);
+  const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
+  const int stride = a.plan.part_stride;
+  float* w_s = ml_s;
+  float* l_s = ml_s + a.plan.n_chunks;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float* part = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
+                                                     a.plan.header_bytes) +
+                      ((int64_t)b * a.Hq + hq) * a.plan.n_chunks * stride;
+
+  float mloc = -INFINITY;
+  for (int c = i; c < nc; c += D) {  // (m, l) of chunk c
+    const float2 ml = *reinterpret_cast<const float2*>(part + (int64_t)c * stride + D);
+    w_s[c] = ml.x;
+    l_s[c] = ml.y;
+    mloc = fmaxf(mloc, ml.x);
+  }
+  const float M = block_max(mloc, red);  // its barriers also publish w_s, l_s
+  float lloc = 0.0f;
+  for (int c = i; c < nc; c += D) {
+    const float w = exp2f(w_s[c] - M);  // NaN if a partial is NaN
+    lloc = fmaf(w, l_s[c], lloc);
+    w_s[c] = w;
+  }
+  const float L = block_sum(lloc, red);  // ends with __syncthreads: weights visible
+
+  constexpr int U = 16;  // chunk loads in flight per thread
+  float acc[U];
+#pragma unroll
+  for (int k = 0; k < U; ++k) acc[k] = 0.0f;
+  for (int c0 = 0; c0 < nc; c0 += U) {
+    float v[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) v[k] = c0 + k < nc ? part[(int64_t)(c0 + k) * stride + i] : 0.0f;
+#pragma unroll
+    for (int k = 0; k < U; ++k)
+      if (c0 + k < nc) acc[k] = fmaf(w_s[c0 + k], v[k], acc[k]);
+  }
+#pragma unroll
+  for (int k = U / 2; k > 0; k >>= 1)
+#pragma unroll
+    for (int j = 0; j < k; ++j) acc[j] += acc[j + k];
+  o[i] = acc[0] / L;
+
+  if (a.signs) {  // o = diag(signs) H o / sqrt(d), H in Sylvester order
+    __syncthreads();
+    for (int bit = 1; bit < D; bit <<= 1) {  // each pair is owned by one thread per stage
+      if (i < D / 2) {
+        const int lo = ((i & ~(bit - 1)) << 1) | (i & (bit - 1));
+        const float u = o[lo], w = o[lo | bit];
+        o[lo] = u + w;
+        o[lo | bit] = u - w;
+      }
+      __syncthreads();
+    }
+    o[i] = o[i] * sgn * rsqrtf((float)D);
+  }
+  a.out[((int64_t)b * a.Hq + hq) * D + i] = o[i];
+}
+
+template <int D>
+cudaError_t launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.Hq);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 2 * sizeof(float) * (size_t)a.plan.n_chunks;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cfg.dynamicSmemBytes > 48 * 1024) {
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e = ensure_smem_limit(merge_kernel<D>, 64 * 1024, smem_set);
+    if (e != cudaSuccess) return e;
+    if (cfg.dynamicSmemBytes > 64 * 1024) return cudaErrorInvalidValue;
+  }
+  return cudaLaunchKernelEx(&cfg, merge_kernel<D>, a);
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
+  return a.d == 128 ? launch_merge_d<128>(a, stream) : launch_merge_d<256>(a, stream);
+}
+
+}  // namespace tq

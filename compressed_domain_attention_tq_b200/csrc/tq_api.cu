@@ -14,15 +14,15 @@ namespace tq {
 
 static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Split the context into chunks (multiples of 128 tokens, the decode's
-// pipeline stage) for persistent CTAs, one per SM: pick the chunk count per
+// Split the context into chunks (multiples of the decode's pipeline stage,
+// 192 or 128 tokens) for persistent CTAs, one per SM: pick the chunk count per
 // sequence that minimises (waves of items over the SMs) x (chunk + a fixed
 // per-item cost), where an item is one (sequence, kv head, chunk).
 bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
   if (d != 128 && d != 256) return false;
   const int64_t units = (int64_t)B * Hkv;
-  const int64_t step = 128, per_item_cost = 384;
+  const int64_t step = decode_stage_tokens(d, Hq / Hkv), per_item_cost = 384;
   const int64_t max_n = ceil_div(max_ctx, step);
   int64_t best_chunk = ceil_div(max_ctx, step) * step, best_cost = -1;
   for (int64_t n = 1; n <= max_n && n <= 4096; ++n) {

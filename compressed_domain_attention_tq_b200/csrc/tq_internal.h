@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace tq {
 
 constexpr int kGroup = 32;  // quantization group (rotated coordinates)
@@ -12,7 +14,7 @@ constexpr int kSmCount = 148;  // B200; sizes the split-K plan (a host-only, dev
 
 // Split-K work decomposition of one decode call (host side, deterministic).
 struct DecodePlan {
-  int chunk;        // context tokens per chunk (multiple of 128)
+  int chunk;        // context tokens per chunk (multiple of the decode's stage)
   int n_chunks;     // ceil(max_ctx / chunk)
   int part_stride;  // floats per (b, q head, chunk) partial: d + 4 (16-byte rows)
   size_t header_bytes;  // int32 flags[B], rounded up to 256 bytes
@@ -53,9 +55,25 @@ struct DecodeArgs {
   DecodePlan plan;
 };
 
+// Raise a kernel's dynamic shared memory limit once per device (the first
+// launch on each device), so later launches, including those made while a
+// stream is being captured into a CUDA graph, only enqueue work.
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 bool decode_mma_supported(int d, int G);
+int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
