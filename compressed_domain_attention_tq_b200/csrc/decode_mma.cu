@@ -5,15 +5,15 @@
 // Open-TQ-Metal abstract): no dequantized K/V matrix exists anywhere (forum
 // summary, section "eliminating intermediate matrices"); codes are widened to
 // f16 in registers, and the fp32 group scales are applied around the
-// contractions.  Softmax runs online with a running maximum, fp32 sums and
-// exact exp2 (section "numerical stability": the scaling trick and
-// high-precision accumulators, without an approximate softmax).
+// contractions.  Softmax runs online with a running maximum and fp32 sums
+// (section "numerical stability": the scaling trick and high-precision
+// accumulators); exp2 is the hardware approximation, relative error ~2^-22.
 //
 // Work: persistent CTAs, one per SM, walk a list of items (sequence b, kv
 // head, context chunk).  Each item's rows (packed K, packed V, K scales, V
 // scales) stream through a ring of shared-memory stages filled by 1-D bulk
 // async copies that complete on mbarriers.  There is no producer warp: every
-// consumer warp takes 16 tokens of each stage, and the last warp to finish a
+// warp takes TPW 16-token tiles of each stage, and the last warp to finish a
 // stage (counted with a shared-memory atomic) refills it with the next stage,
 // so all warps of the CTA compute.  Each warp keeps its own running (max, sum,
 // acc); the warps are merged per item in shared memory into one split-K
