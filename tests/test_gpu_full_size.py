@@ -1,0 +1,104 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times.
+
+Each workload is generated on the GPU from its seed, quantized by the CUDA path
+(one bulk tq_quantize_append call, then one single-token append as in a decode
+step) and decoded over the whole context.  The oracle checks sampled outputs it
+can compute one by one:
+  - codes and scales of sampled token rows, from those rows' exact inputs;
+  - the decode of sampled kv heads (all their query heads), over that head's
+    GPU-written packed cache.
+Gates as in the other GPU tests: rotation on -> at most 0.01% of codes differ,
+each by 1, scales within 4 ulp; attention rel-L2 <= 1e-4 and max-abs <=
+1e-3 * max|v_hat| per (sequence, query head).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressed_domain_attention_tq_b200 import Int4KVCache
+from compressed_domain_attention_tq_b200 import workloads as wl
+from conftest import require_cuda
+from helpers import THREADS, check_attention, to_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_workload(name, attn_scale=None, seed=0, sample_rows=64, sample_heads=2):
+    require_cuda()
+    dev = torch.device("cuda", 0)
+    w = wl.WORKLOADS[name]
+    B, Hq, Hkv, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
+    G = Hq // Hkv
+    signs = wl.make_signs(d, seed) if w.rotation else None
+    ctx = wl.make_context_lengths(w, seed)
+    cache = Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
+    k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
+    cache.append(k_all, v_all, torch.zeros(B, dtype=torch.int32, device=dev))
+    k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
+    cache.append(k_new, v_new, ctx.to(dev))
+    q = wl.make_query(w, seed, device=dev)
+    scale = w.attn_scales[0] if attn_scale is None else attn_scale
+    T = ctx + 1
+    out = cache.decode(q, T.to(dev), int(T.max()), scale)
+    torch.cuda.synchronize()
+    gen = np.random.default_rng(seed + 7)
+    sg = None if signs is None else signs.numpy()
+
+    # ---- quantizer: sampled rows of the bulk call
+    n_diff = n_tot = 0
+    for _ in range(sample_rows):
+        b, h = int(gen.integers(B)), int(gen.integers(Hkv))
+        t = int(gen.integers(int(ctx[b])))
+        for src, packed, scales in ((k_all, cache.k_packed, cache.k_scales),
+                                    (v_all, cache.v_packed, cache.v_scales)):
+            x = src[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
+            ref = oracle.empty_cache(1, 1, 1, d)
+            oracle.quantize_append(to_oracle(x), to_oracle(x), np.zeros(1, np.int32), sg, ref)
+            got_codes = oracle.unpack(packed[b, h, t:t + 1].cpu().numpy(), d).astype(np.int64)
+            want_codes = oracle.unpack(ref[0][0, 0], d).astype(np.int64)
+            diff = np.abs(got_codes - want_codes)
+            assert diff.max() <= (1 if sg is not None else 0), f"{name} b={b} h={h} t={t}"
+            n_diff += int((diff > 0).sum())
+            n_tot += diff.size
+            got_s = scales[b, h, t].cpu().numpy().view(np.int32).astype(np.int64)
+            want_s = ref[1][0, 0, 0].view(np.int32).astype(np.int64)
+            assert np.abs(got_s - want_s).max() <= (4 if sg is not None else 0)
+    assert n_diff <= max(1e-4 * n_tot, 1), f"{name}: {n_diff}/{n_tot} codes differ"
+
+    # ---- decode: sampled (sequence, kv head) pairs over the GPU-written cache
+    got = out.cpu().numpy()
+    q_host = to_oracle(q.cpu())
+    for _ in range(sample_heads):
+        b, h = int(gen.integers(B)), int(gen.integers(Hkv))
+        Tb = int(T[b])
+        sub = [np.ascontiguousarray(a[b:b + 1, h:h + 1, :Tb].cpu().numpy())
+               for a in (cache.k_packed, cache.k_scales, cache.v_packed, cache.v_scales)]
+        qs = np.ascontiguousarray(q_host[b:b + 1, h * G:(h + 1) * G])
+        want = oracle.sdpa_int4_decode(qs, sub, [Tb], sg, scale, 1, threads=THREADS)
+        check_attention(got[b:b + 1, h * G:(h + 1) * G], want, sub, [Tb], G,
+                        f"{name} b={b} kv head {h}")
+    return n_diff, n_tot
+
+
+def test_full_size_tiny_mha_4k():
+    _run_workload("tiny_mha_4k", sample_rows=128, sample_heads=4)
+
+
+def test_full_size_llama70b_gqa_32k():
+    _run_workload("llama70b_gqa_32k")
+
+
+def test_full_size_llama70b_gqa_128k():
+    _run_workload("llama70b_gqa_128k")
+
+
+def test_full_size_ragged_b16():
+    _run_workload("ragged_b16", sample_heads=3)
+
+
+@pytest.mark.parametrize("scale", [1.0, 1 / 16.0])
+def test_full_size_wide_d256(scale):
+    _run_workload("wide_d256", attn_scale=scale)
