@@ -317,26 +317,55 @@ struct WarpState {
 // w < NH prepares head w; the FWHT runs in registers and shuffles.
 template <int D, int PATH>
 __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, unsigned char* smem,
-                                           WarpState<D, PATH>& st) {
+                                           WarpState<D, PATH>& st, bool start_stream,
+                                           int* cur, uint64_t* full, int n_items) {
   using C = Cfg<D, PATH>;
   constexpr int E = D / 32;  // elements per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv;
   float* qs = reinterpret_cast<float*>(smem + C::QS);
   float* qexp = reinterpret_cast<float*>(smem + C::QEXP);
-  if (warp < C::NH) {
-    const int h = warp;
+  // Heads are prepared by warps 0 .. NW/2 - 1 (two heads each when NH == 8), so
+  // the last warp is free to issue the first copies meanwhile.
+  constexpr int HPW = C::NH / (C::NW / 2) > 0 ? C::NH / (C::NW / 2) : 1;  // heads per warp
+  for (int hh = 0; hh < HPW; ++hh) {
+    const int h = warp * HPW + hh;
+    if (warp >= C::NW / 2 || h >= C::NH) break;
     float x[E];
     if (h < G) {
       const int64_t base = ((int64_t)b * a.Hq + (int64_t)kvh * G + h) * D + lane * E;
+      if (a.q_bf16) {  // E consecutive bf16 values: one 8- or 16-byte load
+        uint32_t u[E / 2];
+        if (E == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + base);
+          u[0] = v.x;
+          u[1] = v.y;
+        } else {
+          const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + base);
+          u[0] = v.x;
+          u[1] = v.y;
+          u[E > 4 ? 2 : 0] = v.z;
+          u[E > 4 ? 3 : 1] = v.w;
+        }
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        float v = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[base + e])
-                           : static_cast<const float*>(a.q)[base + e];
-        if (a.signs) v *= (float)a.signs[lane * E + e];
-        x[e] = v;
+        for (int e = 0; e < E; ++e)
+          x[e] = __uint_as_float(e & 1 ? (u[e / 2] & 0xFFFF0000u) : (u[e / 2] << 16));
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + base + e);
+          x[e] = v.x;
+          x[e + 1] = v.y;
+          x[e + 2] = v.z;
+          x[e + 3] = v.w;
+        }
       }
       if (a.signs) {
+        int8_t sg[E];  // byte loads: the signs pointer has no alignment requirement
+#pragma unroll
+        for (int e = 0; e < E; ++e) sg[e] = a.signs[lane * E + e];
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] *= (float)sg[e];
 #pragma unroll
         for (int bit = 1; bit < E; bit <<= 1)
 #pragma unroll
@@ -377,6 +406,11 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     }
   }
   barrier_all<C::THREADS>();
+  // The first item's query loads have landed; only now does the last warp
+  // start the stream, so those few loads do not queue behind it.
+  if (start_stream && threadIdx.x == C::THREADS - 32)
+    for (int s = 0; s < C::NS; ++s)
+      if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
   // Score A tiles in shared memory, f16 [group][k-step][row][k]: row r < 8 is
   // the hi part of head h(r), row 8 + r its lo part; MMA index k of k-step ks
   // is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in which
@@ -412,23 +446,24 @@ __device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
     for (int r = 0; r < 4; ++r) st.acc[j][r] *= f;
 }
 
-// TPW consecutive 16-token tiles of one warp: tile u covers rows r0 + 16u ..
-// r0 + 16u + 15 of the stage, and the first `nvalid` rows from r0 on are real
-// tokens (all of them when FULL).  rho[i]: tile rows of this thread's MMA
-// slots 2tig, 2tig+1, 8+2tig, 9+2tig; krow[nt]: tile row of score n-tile nt's
-// column gid.  The tiles share one softmax update.
+// The per-stage work of one warp is split so that the P.V of one stage and
+// the scores of the next run as one straight-line block the compiler can
+// interleave; the branchy softmax update follows it.  A warp owns TPW
+// consecutive 16-token tiles of each stage: tile u covers rows r0 + 16u ..
+// r0 + 16u + 15, of which the first `nvalid` rows from r0 on are real tokens.
+// rho[i]: tile rows of this thread's MMA slots 2tig, 2tig+1, 8+2tig, 9+2tig;
+// krow[nt]: tile row of score n-tile nt's column gid.
+
+// Scores before the qexp factor, S = sum_g s_k[t, g] (q_hi + q_lo) . c_k[t, g];
+// unless FULL, rows past nvalid get -inf.  Branch-free.
 template <int D, int PATH, int TPW, bool FULL>
-__device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, int nvalid,
-                                              int gid, int tig, const int (&rho)[4],
-                                              const int (&krow)[2], WarpState<D, PATH>& st) {
+__device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, int nvalid, int tig,
+                                            const int (&rho)[4], const int (&krow)[2],
+                                            const WarpState<D, PATH>& st, float (&S)[TPW][4]) {
   using C = Cfg<D, PATH>;
   constexpr int NG = C::NG, RB = C::RB, SB = C::SB;
   const unsigned char* kc = stg + C::KC + r0 * RB;
-  const unsigned char* vc = stg + C::VC + r0 * RB;
   const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
-  const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
-
-  // ---- scores (before the qexp factor) S = sum_g s_k[t, g] * (q_hi + q_lo) . c_k[t, group g]
   uint32_t kw[TPW][2][NG];  // per tile and n-tile: sub-blocks 2tig, 2tig+1 of token krow[nt]
   float sk[TPW][4][NG];
 #pragma unroll
@@ -456,7 +491,6 @@ __device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, 
         sk[u][i][4 * q + 3] = v.w;
       }
   }
-  float S[TPW][4];
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
@@ -481,16 +515,17 @@ __device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, 
         S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], c[1] + c[3], S[u][2 * nt + 1]);
       }
   }
-  bool vld[TPW][4];
+  if (!FULL)
 #pragma unroll
-  for (int u = 0; u < TPW; ++u)
+    for (int u = 0; u < TPW; ++u)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      vld[u][i] = FULL || 16 * u + rho[i] < nvalid;
-      if (!vld[u][i]) S[u][i] = -INFINITY;
-    }
+      for (int i = 0; i < 4; ++i) S[u][i] = 16 * u + rho[i] < nvalid ? S[u][i] : -INFINITY;
+}
 
-  // ---- online softmax (log2 units) for this thread's head
+// Running max of this thread's head (log2 units) over the tiles' scores; when
+// it grows, the accumulators and the running sum are rescaled.
+template <int D, int PATH, int TPW>
+__device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], WarpState<D, PATH>& st) {
   float mx = S[0][0];
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
@@ -506,46 +541,44 @@ __device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, 
     st.l *= alpha;
     st.m = m_new;
   }
+}
 
-  // ---- V scales and p' = 2^(S - m - F), keeping p' * s_v below 2^15
-  float sv[TPW][4][NG];
+// V scales (unless FULL, zero past nvalid) and the weights p' = 2^(S - m - F),
+// keeping p' * s_v below 2^14 (raising F with an exact rescale when needed).
+template <int D, int PATH, int TPW, bool FULL>
+__device__ __forceinline__ void tile_weights(const unsigned char* stg, int r0, int nvalid,
+                                             const int (&rho)[4], const float (&S)[TPW][4],
+                                             WarpState<D, PATH>& st, float (&p)[TPW][4],
+                                             float (&sv)[TPW][4][D / 32]) {
+  using C = Cfg<D, PATH>;
+  constexpr int NG = C::NG;
+  const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool ok = FULL || 16 * u + rho[i] < nvalid;
+#pragma unroll
+      for (int q = 0; q < NG / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(vs + (16 * u + rho[i]) * NG)[q];
+        sv[u][i][4 * q] = ok ? v.x : 0.0f;
+        sv[u][i][4 * q + 1] = ok ? v.y : 0.0f;
+        sv[u][i][4 * q + 2] = ok ? v.z : 0.0f;
+        sv[u][i][4 * q + 3] = ok ? v.w : 0.0f;
+      }
+    }
+  // p' <= 2^-F, so P' stays below 2^14 while every V scale is at most
+  // 2^(14+F); positive floats order like their bit patterns.
+  int vbits = 0;
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int q = 0; q < NG / 4; ++q) {
-        const float4 v = reinterpret_cast<const float4*>(vs + (16 * u + rho[i]) * NG)[q];
-        sv[u][i][4 * q] = vld[u][i] ? v.x : 0.0f;
-        sv[u][i][4 * q + 1] = vld[u][i] ? v.y : 0.0f;
-        sv[u][i][4 * q + 2] = vld[u][i] ? v.z : 0.0f;
-        sv[u][i][4 * q + 3] = vld[u][i] ? v.w : 0.0f;
-      }
-  float smax[TPW][4];
-#pragma unroll
-  for (int u = 0; u < TPW; ++u)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      smax[u][i] = sv[u][i][0];
-#pragma unroll
-      for (int g = 1; g < NG; ++g) smax[u][i] = fmaxf(smax[u][i], sv[u][i][g]);
-    }
-  float p[TPW][4];
-  float mF = st.m + (float)st.F;
-  float pm = 0.0f;
-#pragma unroll
-  for (int u = 0; u < TPW; ++u)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
-      pm = fmaxf(pm, p[u][i] * smax[u][i]);
-    }
-  if (__any_sync(kFull, !st.fset || pm > 16384.0f)) {
-    float vm = 0.0f;
-#pragma unroll
-    for (int u = 0; u < TPW; ++u)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) vm = fmaxf(vm, smax[u][i]);
+      for (int g = 0; g + 1 < NG; g += 2)
+        vbits = __vimax3_s32(vbits, __float_as_int(sv[u][i][g]), __float_as_int(sv[u][i][g + 1]));
+  if (__any_sync(kFull, !st.fset || vbits > __float_as_int(pow2i(14 + st.F)))) {
+    float vm = __int_as_float(vbits);
     vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 1));
     vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 2));
     int ex = 0;
@@ -553,24 +586,36 @@ __device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, 
     int Fn = vm > 0.0f ? ex - 7 : 0;  // vm * 2^-Fn in [64, 128)
     Fn = max(-60, min(60, Fn));
     if (!st.fset) {
-      st.F = Fn;
-      st.fset = true;
+      if (vm > 0.0f) {
+        st.F = Fn;
+        st.fset = true;
+      }
     } else if (Fn > st.F) {
       const float f = pow2i(st.F - Fn);  // exact
       scale_acc(st, f);
       st.l *= f;
       st.F = Fn;
     }
-    mF = st.m + (float)st.F;
-#pragma unroll
-    for (int u = 0; u < TPW; ++u)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
   }
+  // m = -inf only while every score so far is -inf (no real token yet)
+  const float mF = st.m == -INFINITY ? 0.0f : st.m + (float)st.F;
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
 #pragma unroll
   for (int u = 0; u < TPW; ++u) st.l += (p[u][0] + p[u][1]) + (p[u][2] + p[u][3]);
+}
 
-  // ---- P.V on the packed values
+// P.V on the packed values with P' = p' * s_v split into hi + lo.  Branch-free.
+template <int D, int PATH, int TPW>
+__device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gid,
+                                        const int (&rho)[4], const float (&p)[TPW][4],
+                                        const float (&sv)[TPW][4][D / 32],
+                                        WarpState<D, PATH>& st) {
+  using C = Cfg<D, PATH>;
+  constexpr int NG = C::NG, RB = C::RB, SB = C::SB;
+  const unsigned char* vc = stg + C::VC + r0 * RB;
 #pragma unroll
   for (int u = 0; u < TPW; ++u) {
     uint32_t vw[4][NG / 2];  // sub-block gid of rows rho[0..3] of tile u
@@ -619,6 +664,19 @@ __device__ __forceinline__ void process_tiles(const unsigned char* stg, int r0, 
       }
     }
   }
+}
+
+// One warp's share of a stage: scores, softmax update and P.V of its TPW tiles
+// (rows r0 .. r0 + 16 TPW - 1, of which the first nvalid are real tokens).
+template <int D, int PATH, int TPW, bool FULL>
+__device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, int nvalid, int gid,
+                                            int tig, const int (&rho)[4], const int (&krow)[2],
+                                            WarpState<D, PATH>& st) {
+  float S[TPW][4], p[TPW][4], sv[TPW][4][D / 32];
+  tile_scores<D, PATH, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
+  tile_max<D, PATH, TPW>(tig, S, st);
+  tile_weights<D, PATH, TPW, FULL>(stg, r0, nvalid, rho, S, st, p, sv);
+  tile_pv<D, PATH, TPW>(stg, r0, gid, rho, p, sv, st);
 }
 
 // End of an item: the warps' (max, sum, acc) per head are merged in shared
@@ -725,8 +783,6 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
     cur[0] = (int)blockIdx.x - (int)gridDim.x;  // before this CTA's first item
     cur[1] = cur[2] = cur[3] = cur[4] = cur[5] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int s = 0; s < C::NS; ++s)
-      if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
   }
   // the merge kernel may be scheduled now; it waits for this grid's writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -745,7 +801,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
       const int raw = a.ctx_lens[b];
       static_cast<int32_t*>(a.workspace)[b] = (raw < 1 || raw > a.max_ctx) ? 1 : 0;
     }
-    prep_query<D, PATH>(a, b, kvh, smem, st);
+    prep_query<D, PATH>(a, b, kvh, smem, st, sc == 0, cur, full, n_items);
 #pragma unroll
     for (int j = 0; j < C::NACC; ++j)
 #pragma unroll
@@ -754,17 +810,17 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
     st.l = 0.0f;
     st.F = 0;
     st.fset = false;
-    for (int t = t0; t < t1; t += C::ST, ++sc) {
+    const int nst = (t1 - t0 + C::ST - 1) / C::ST;
+    const int r0 = 16 * C::TPW * warp;
+    for (int k = 0; k < nst; ++k, ++sc) {
       const int slot = sc % C::NS;
-      const bool ok = mbar_wait(full + slot, (sc / C::NS) & 1, abort);
-      const int nvalid = min(16 * C::TPW, min(C::ST, t1 - t) - 16 * C::TPW * warp);
       const unsigned char* stg = smem + slot * C::STAGE;
-      if (ok && nvalid == 16 * C::TPW)
-        process_tiles<D, PATH, C::TPW, true>(stg, 16 * C::TPW * warp, nvalid, gid, tig, rho, krow,
-                                             st);
-      else if (ok && nvalid > 0)
-        process_tiles<D, PATH, C::TPW, false>(stg, 16 * C::TPW * warp, nvalid, gid, tig, rho,
-                                              krow, st);
+      mbar_wait(full + slot, (sc / C::NS) & 1, abort);
+      const int nv = min(C::ST, t1 - t0 - k * C::ST) - r0;  // real rows from r0 on
+      if (nv >= 16 * C::TPW)
+        stage_tiles<D, PATH, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st);
+      else if (nv > 0)
+        stage_tiles<D, PATH, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st);
       __syncwarp();
       if (lane == 0) {  // the last warp out of the stage refills it
         __threadfence_block();
