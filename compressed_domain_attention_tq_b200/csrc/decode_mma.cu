@@ -306,7 +306,8 @@ struct WarpState {
   float acc[Cfg<D, PATH>::NACC][4];  // P.V accumulators (fragments), scaled by 2^-F
   uint32_t qa_addr;                  // this lane's ldmatrix row address of the score A tiles
   float m;                           // running max of this thread's head (log2 units)
-  float l;                           // this thread's share of the running sum, scaled by 2^-F
+  float2 l;                          // this thread's share of the running sum (two partial
+                                     // sums, added at the end), scaled by 2^-F
   float qexp;                        // 2^E of this thread's head (query normalisation)
   int F;                             // V-scale normalisation exponent
   bool fset;                         // F chosen for this item
@@ -440,10 +441,15 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
 
 template <int D, int PATH>
 __device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
+  const float2 ff = make_float2(f, f);
 #pragma unroll
   for (int j = 0; j < Cfg<D, PATH>::NACC; ++j)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) st.acc[j][r] *= f;
+    for (int r = 0; r < 4; r += 2) {
+      const float2 v = __fmul2_rn(make_float2(st.acc[j][r], st.acc[j][r + 1]), ff);
+      st.acc[j][r] = v.x;
+      st.acc[j][r + 1] = v.y;
+    }
 }
 
 // The per-stage work of one warp is split so that the P.V of one stage and
@@ -511,8 +517,9 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
         float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], codes_lo(X), codes_hi(X));
         mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], codes_lo(Y), codes_hi(Y));
-        S[u][2 * nt] = fmaf(sk[u][2 * nt][g], c[0] + c[2], S[u][2 * nt]);
-        S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], c[1] + c[3], S[u][2 * nt + 1]);
+        const float2 x = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
+        S[u][2 * nt] = fmaf(sk[u][2 * nt][g], x.x, S[u][2 * nt]);
+        S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], x.y, S[u][2 * nt + 1]);
       }
   }
   if (!FULL)
@@ -538,7 +545,7 @@ __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], Warp
     const float alpha = ex2(st.m - m_new);  // 0 on the first tile, 1 if unchanged
     // PATH 1 accumulates head tig; its softmax state lives on lane 8 * tig
     scale_acc(st, PATH == 0 ? alpha : __shfl_sync(kFull, alpha, 8 * tig));
-    st.l *= alpha;
+    st.l = __fmul2_rn(st.l, make_float2(alpha, alpha));
     st.m = m_new;
   }
 }
@@ -593,18 +600,22 @@ __device__ __forceinline__ void tile_weights(const unsigned char* stg, int r0, i
     } else if (Fn > st.F) {
       const float f = pow2i(st.F - Fn);  // exact
       scale_acc(st, f);
-      st.l *= f;
+      st.l = __fmul2_rn(st.l, make_float2(f, f));
       st.F = Fn;
     }
   }
   // m = -inf only while every score so far is -inf (no real token yet)
   const float mF = st.m == -INFINITY ? 0.0f : st.m + (float)st.F;
+  const float2 qe = make_float2(st.qexp, st.qexp), nm = make_float2(-mF, -mF);
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) p[u][i] = ex2(fmaf(S[u][i], st.qexp, -mF));
-#pragma unroll
-  for (int u = 0; u < TPW; ++u) st.l += (p[u][0] + p[u][1]) + (p[u][2] + p[u][3]);
+    for (int i = 0; i < 4; i += 2) {
+      const float2 arg = __ffma2_rn(make_float2(S[u][i], S[u][i + 1]), qe, nm);
+      p[u][i] = ex2(arg.x);
+      p[u][i + 1] = ex2(arg.y);
+      st.l = __fadd2_rn(st.l, make_float2(p[u][i], p[u][i + 1]));
+    }
 }
 
 // P.V on the packed values with P' = p' * s_v split into hi + lo.  Branch-free.
@@ -638,29 +649,44 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
       }
     }
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
-      // codes c = 0..3 of dims 32g + 4gid + c: low halves rows rho0 / rho2,
-      // high halves rows rho1 / rho3
-      const uint32_t X = prmt(vw[0][g / 2], vw[1][g / 2], sel);
-      const uint32_t Y = prmt(vw[2][g / 2], vw[3][g / 2], sel);
-      const float x0 = p[u][0] * sv[u][0][g], x1 = p[u][1] * sv[u][1][g];
-      const float x2 = p[u][2] * sv[u][2][g], x3 = p[u][3] * sv[u][3][g];
-      const float h0 = split_hi(x0), h1 = split_hi(x1), h2 = split_hi(x2), h3 = split_hi(x3);
-      if (PATH == 0) {
-        const uint32_t a0 = f16x2(h0, h1), a1 = f16x2(x0 - h0, x1 - h1);
-        const uint32_t a2 = f16x2(h2, h3), a3 = f16x2(x2 - h2, x3 - h3);
-        mma16816(st.acc[4 * g + 0], a0, a1, a2, a3, codes_lo(X), codes_lo(Y));
-        mma16816(st.acc[4 * g + 1], a0, a1, a2, a3, codes_hi(X), codes_hi(Y));
-        mma16816(st.acc[4 * g + 2], a0, a1, a2, a3, codes_lo(X >> 8), codes_lo(Y >> 8));
-        mma16816(st.acc[4 * g + 3], a0, a1, a2, a3, codes_hi(X >> 8), codes_hi(Y >> 8));
-      } else {
-        const bool lo = gid & 1;  // column gid = (head gid / 2, part gid % 2)
-        const uint32_t b0 = f16x2(lo ? x0 - h0 : h0, lo ? x1 - h1 : h1);
-        const uint32_t b1 = f16x2(lo ? x2 - h2 : h2, lo ? x3 - h3 : h3);
-        mma16816(st.acc[2 * g + 0], codes_lo(X), codes_hi(X), codes_lo(Y), codes_hi(Y), b0, b1);
-        mma16816(st.acc[2 * g + 1], codes_lo(X >> 8), codes_hi(X >> 8), codes_lo(Y >> 8),
-                 codes_hi(Y >> 8), b0, b1);
+    for (int gp = 0; gp < NG; gp += 2) {
+      // P' = p' * s_v of rows rho[0..3] for groups gp, gp + 1, split exactly
+      // into f16-representable hi + lo (two groups per packed multiply)
+      float wh[4][2], wl[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __fmul2_rn(make_float2(p[u][i], p[u][i]),
+                                    make_float2(sv[u][i][gp], sv[u][i][gp + 1]));
+        const float2 h = make_float2(split_hi(x.x), split_hi(x.y));
+        const float2 l = __ffma2_rn(h, make_float2(-1.0f, -1.0f), x);  // exact
+        wh[i][0] = h.x;
+        wh[i][1] = h.y;
+        wl[i][0] = l.x;
+        wl[i][1] = l.y;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int g = gp + e;
+        const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
+        // codes c = 0..3 of dims 32g + 4gid + c: low halves rows rho0 / rho2,
+        // high halves rows rho1 / rho3
+        const uint32_t X = prmt(vw[0][g / 2], vw[1][g / 2], sel);
+        const uint32_t Y = prmt(vw[2][g / 2], vw[3][g / 2], sel);
+        if (PATH == 0) {
+          const uint32_t a0 = f16x2(wh[0][e], wh[1][e]), a1 = f16x2(wl[0][e], wl[1][e]);
+          const uint32_t a2 = f16x2(wh[2][e], wh[3][e]), a3 = f16x2(wl[2][e], wl[3][e]);
+          mma16816(st.acc[4 * g + 0], a0, a1, a2, a3, codes_lo(X), codes_lo(Y));
+          mma16816(st.acc[4 * g + 1], a0, a1, a2, a3, codes_hi(X), codes_hi(Y));
+          mma16816(st.acc[4 * g + 2], a0, a1, a2, a3, codes_lo(X >> 8), codes_lo(Y >> 8));
+          mma16816(st.acc[4 * g + 3], a0, a1, a2, a3, codes_hi(X >> 8), codes_hi(Y >> 8));
+        } else {
+          const bool lo = gid & 1;  // column gid = (head gid / 2, part gid % 2)
+          const uint32_t b0 = f16x2(lo ? wl[0][e] : wh[0][e], lo ? wl[1][e] : wh[1][e]);
+          const uint32_t b1 = f16x2(lo ? wl[2][e] : wh[2][e], lo ? wl[3][e] : wh[3][e]);
+          mma16816(st.acc[2 * g + 0], codes_lo(X), codes_hi(X), codes_lo(Y), codes_hi(Y), b0, b1);
+          mma16816(st.acc[2 * g + 1], codes_lo(X >> 8), codes_hi(X >> 8), codes_lo(Y >> 8),
+                   codes_hi(Y >> 8), b0, b1);
+        }
       }
     }
   }
@@ -698,7 +724,7 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
   float* mw = reinterpret_cast<float*>(smem + C::MW);
   float* mtot = reinterpret_cast<float*>(smem + C::MTOT);
 
-  float l = st.l;
+  float l = st.l.x + st.l.y;
   l += __shfl_xor_sync(kFull, l, 1);
   l += __shfl_xor_sync(kFull, l, 2);
   const float m = aborted ? __int_as_float(0x7fc00000) : st.m + (float)st.F;
@@ -807,7 +833,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
 #pragma unroll
       for (int r = 0; r < 4; ++r) st.acc[j][r] = 0.0f;
     st.m = -INFINITY;
-    st.l = 0.0f;
+    st.l = make_float2(0.0f, 0.0f);
     st.F = 0;
     st.fset = false;
     const int nst = (t1 - t0 + C::ST - 1) / C::ST;
