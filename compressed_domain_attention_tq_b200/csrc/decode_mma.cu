@@ -196,6 +196,13 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "r"(addr));
 }
 
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^e as a float for |e| <= 126
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -533,11 +540,12 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
 // it grows, the accumulators and the running sum are rescaled.
 template <int D, int PATH, int TPW>
 __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], WarpState<D, PATH>& st) {
-  float mx = S[0][0];
-#pragma unroll
-  for (int u = 0; u < TPW; ++u)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, S[u][i]);
+  float mx;
+  if (TPW == 2)
+    mx = fmax3(fmax3(S[0][0], S[0][1], S[0][2]), fmax3(S[0][3], S[TPW - 1][0], S[TPW - 1][1]),
+               fmaxf(S[TPW - 1][2], S[TPW - 1][3]));
+  else
+    mx = fmaxf(fmax3(S[0][0], S[0][1], S[0][2]), S[0][3]);
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
   const float m_new = fmaxf(st.m, mx * st.qexp);
@@ -550,13 +558,10 @@ __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], Warp
   }
 }
 
-// V scales (unless FULL, zero past nvalid) and the weights p' = 2^(S - m - F),
-// keeping p' * s_v below 2^14 (raising F with an exact rescale when needed).
+// V scales of the warp's rows (unless FULL, zero past nvalid).
 template <int D, int PATH, int TPW, bool FULL>
-__device__ __forceinline__ void tile_weights(const unsigned char* stg, int r0, int nvalid,
-                                             const int (&rho)[4], const float (&S)[TPW][4],
-                                             WarpState<D, PATH>& st, float (&p)[TPW][4],
-                                             float (&sv)[TPW][4][D / 32]) {
+__device__ __forceinline__ void load_vscales(const unsigned char* stg, int r0, int nvalid,
+                                             const int (&rho)[4], float (&sv)[TPW][4][D / 32]) {
   using C = Cfg<D, PATH>;
   constexpr int NG = C::NG;
   const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
@@ -574,36 +579,17 @@ __device__ __forceinline__ void tile_weights(const unsigned char* stg, int r0, i
         sv[u][i][4 * q + 3] = ok ? v.w : 0.0f;
       }
     }
-  // p' <= 2^-F, so P' stays below 2^14 while every V scale is at most
-  // 2^(14+F); positive floats order like their bit patterns.
-  int vbits = 0;
-#pragma unroll
-  for (int u = 0; u < TPW; ++u)
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int g = 0; g + 1 < NG; g += 2)
-        vbits = __vimax3_s32(vbits, __float_as_int(sv[u][i][g]), __float_as_int(sv[u][i][g + 1]));
-  if (__any_sync(kFull, !st.fset || vbits > __float_as_int(pow2i(14 + st.F)))) {
-    float vm = __int_as_float(vbits);
-    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 1));
-    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 2));
-    int ex = 0;
-    frexpf(vm, &ex);
-    int Fn = vm > 0.0f ? ex - 7 : 0;  // vm * 2^-Fn in [64, 128)
-    Fn = max(-60, min(60, Fn));
-    if (!st.fset) {
-      if (vm > 0.0f) {
-        st.F = Fn;
-        st.fset = true;
-      }
-    } else if (Fn > st.F) {
-      const float f = pow2i(st.F - Fn);  // exact
-      scale_acc(st, f);
-      st.l = __fmul2_rn(st.l, make_float2(f, f));
-      st.F = Fn;
-    }
-  }
+}
+
+// The weights p' = 2^(S - m - F), keeping p' * s_v below 2^14: the exponent F
+// follows the largest V scale seen (raised with an exact power-of-two rescale
+// of acc, l and these weights, which is rare, so the weights are computed
+// first with the current F and the check runs beside them).
+template <int D, int PATH, int TPW>
+__device__ __forceinline__ void tile_weights(const float (&S)[TPW][4],
+                                             const float (&sv)[TPW][4][D / 32],
+                                             WarpState<D, PATH>& st, float (&p)[TPW][4]) {
+  constexpr int NG = D / 32, NV = 4 * TPW * NG;
   // m = -inf only while every score so far is -inf (no real token yet)
   const float mF = st.m == -INFINITY ? 0.0f : st.m + (float)st.F;
   const float2 qe = make_float2(st.qexp, st.qexp), nm = make_float2(-mF, -mF);
@@ -614,8 +600,45 @@ __device__ __forceinline__ void tile_weights(const unsigned char* stg, int r0, i
       const float2 arg = __ffma2_rn(make_float2(S[u][i], S[u][i + 1]), qe, nm);
       p[u][i] = ex2(arg.x);
       p[u][i + 1] = ex2(arg.y);
-      st.l = __fadd2_rn(st.l, make_float2(p[u][i], p[u][i + 1]));
     }
+  // p' <= 2^-F, so P' stays below 2^14 while every V scale is at most
+  // 2^(14+F); non-negative floats order like their bit patterns
+  int w[NV];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int g = 0; g < NG; ++g) w[(u * 4 + i) * NG + g] = __float_as_int(sv[u][i][g]);
+  int vbits = 0;
+#pragma unroll
+  for (int j = 0; j + 1 < NV; j += 2) vbits = __vimax3_s32(vbits, w[j], w[j + 1]);
+  if (__any_sync(kFull, !st.fset || vbits > __float_as_int(pow2i(14 + st.F)))) {
+    float vm = __int_as_float(vbits);
+    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 1));
+    vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, 2));
+    int ex = 0;
+    frexpf(vm, &ex);
+    int Fn = vm > 0.0f ? ex - 7 : 0;  // vm * 2^-Fn in [64, 128)
+    Fn = max(-60, min(60, Fn));
+    // F stays 0 until the first non-zero V scale, then only rises
+    const int Fnew = st.fset ? max(st.F, Fn) : (vm > 0.0f ? Fn : st.F);
+    if (Fnew != st.F) {
+      const float f = pow2i(st.F - Fnew);  // exact
+      scale_acc(st, f);
+      st.l = __fmul2_rn(st.l, make_float2(f, f));
+#pragma unroll
+      for (int u = 0; u < TPW; ++u)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[u][i] *= f;
+      st.F = Fnew;
+    }
+    if (vm > 0.0f) st.fset = true;
+  }
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) st.l = __fadd2_rn(st.l, make_float2(p[u][i], p[u][i + 1]));
 }
 
 // P.V on the packed values with P' = p' * s_v split into hi + lo.  Branch-free.
@@ -701,7 +724,8 @@ __device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, in
   float S[TPW][4], p[TPW][4], sv[TPW][4][D / 32];
   tile_scores<D, PATH, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
   tile_max<D, PATH, TPW>(tig, S, st);
-  tile_weights<D, PATH, TPW, FULL>(stg, r0, nvalid, rho, S, st, p, sv);
+  load_vscales<D, PATH, TPW, FULL>(stg, r0, nvalid, rho, sv);
+  tile_weights<D, PATH, TPW>(S, sv, st, p);
   tile_pv<D, PATH, TPW>(stg, r0, gid, rho, p, sv, st);
 }
 

@@ -137,3 +137,27 @@ def test_decode_is_deterministic():
     a, _ = run_decode(cache, q, [T], T, signs, 0.08, Hkv)
     b, _ = run_decode(cache, q, [T], T, signs, 0.08, Hkv)
     np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("d,G", [(128, 8), (128, 2), (256, 2)])
+def test_decode_zero_v_prefix(d, G):
+    """V exactly zero on the first tokens (zero V scales), then random: the
+    V-scale exponent is first chosen after real tokens already count in the
+    softmax sum, which must then be rescaled with the accumulators.  An
+    all-zero V must give an exact zero output."""
+    require_cuda()
+    B, Hkv, T = 1, 2, 3000
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 81)
+    signs = signs_for(d, 82)
+    for zero_to in (700, T):
+        vz = v.clone()
+        vz[:, :, :zero_to] = 0
+        cache = oracle_cache(k, vz, signs)
+        got, flags = run_decode(upload_cache(cache), q, [T], T, signs, 1 / math.sqrt(d), Hkv)
+        assert np.all(flags == 0)
+        if zero_to == T:
+            assert np.all(got == 0.0)
+            continue
+        want = oracle.sdpa_int4_decode(to_oracle(q), cache, [T], signs.numpy(), 1 / math.sqrt(d),
+                                       Hkv, threads=THREADS)
+        check_attention(got, want, cache, [T], G, f"zero V prefix d={d} G={G}")
