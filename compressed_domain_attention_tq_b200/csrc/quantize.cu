@@ -6,10 +6,14 @@
 // nibble packing and 128-bit stores (SRFT post, core method: rotation, scale,
 // group abs-max and int4 packing fused into a single kernel).
 //
-// Work decomposition: each thread owns 128 consecutive coordinates of one
-// vector (d = 128: one thread per vector; d = 256: two neighbouring lanes per
-// vector, joined by one shuffle butterfly stage).  Seven butterfly stages run
-// in registers, so the rotation costs no shuffles at d = 128.
+// Work decomposition (bulk appends): each thread owns 128 consecutive
+// coordinates of one vector (d = 128: one thread per vector; d = 256: two
+// neighbouring lanes per vector, joined by one shuffle butterfly stage).
+// Seven butterfly stages run in registers, so the rotation costs no shuffles
+// at d = 128.  The inputs reach registers through shared memory: each warp
+// copies its next batch of 32 slices with coalesced 16-byte cp.async while it
+// computes the current one, and reads its slice at a padded pitch (no bank
+// conflicts).  Small appends (a decode step) use one warp per vector instead.
 //
 // Codes are c = rne(fl32(y / s)) with s = fl32(amax / 7) (fp32 IEEE
 // division, round half to even).  Instead of one IEEE division per element,
@@ -40,190 +44,324 @@ __device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t nib_src, int po
   return r;
 }
 
-// 128 consecutive inputs -> fp32, sign flips applied (bf16 flips the sign bit
-// before widening; fp32 flips it after).
+// Async 16-byte global -> shared copy; src_bytes = 0 zero-fills without reading.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bulk path layout.  A warp quantizes batches of 32 slices (a slice = 128
+// consecutive coordinates of one vector: d = 128 -> 32 vectors, d = 256 -> 16
+// vectors, two lanes each).  A batch is VPB consecutive input vectors, i.e.
+// one contiguous span of the K (then V) input, copied with coalesced 16-byte
+// cp.async into shared memory at a pitch of slice + 16 bytes, so that lane t
+// then reads its own slice t without bank conflicts.  Two buffers per warp:
+// the next batch is in flight while the current one is computed.
+template <bool BF16>
+struct QCfg {
+  static constexpr int EB = BF16 ? 2 : 4;       // input bytes per element
+  static constexpr int SLICE = 128 * EB;        // bytes of a 128-coordinate slice
+  static constexpr int PITCH = SLICE + 16;      // shared-memory slice pitch
+  static constexpr int BUF = 32 * PITCH;        // one batch buffer
+  static constexpr int WARPS = BF16 ? 8 : 4;    // warps per CTA (one CTA per SM)
+  static constexpr int THREADS = 32 * WARPS;
+  static constexpr int MASKS = 2 * 192 * 4;     // sign masks of the two 128-slices
+  static constexpr int BYTES = MASKS + WARPS * 2 * BUF;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
+};
+
+// This lane's slice of a staged batch -> fp32, sign flips applied (bf16 flips
+// the sign bit before widening; fp32 flips it after).
 template <bool BF16, bool ROT>
-__device__ __forceinline__ void load_slice(const void* base, int64_t elem_off, bool valid,
-                                           const uint32_t* __restrict__ smask,
+__device__ __forceinline__ void read_slice(const unsigned char* slice, const uint32_t* smask,
                                            float (&x)[128]) {
   if (BF16) {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem_off);
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      uint4 w = valid ? __ldcs(p + c) : make_uint4(0, 0, 0, 0);
-      uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      const uint4 w = reinterpret_cast<const uint4*>(slice)[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         uint32_t u = ws[k];
-        if (ROT) u ^= smask[c * 4 + k];   // bit 15 / bit 31 = sign of element 2k / 2k+1
+        if (ROT) u ^= smask[c * 4 + k];  // bit 15 / bit 31 = sign of element 2k / 2k+1
         x[c * 8 + 2 * k] = __uint_as_float(u << 16);
         x[c * 8 + 2 * k + 1] = __uint_as_float(u & 0xFFFF0000u);
       }
     }
   } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_off);
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-      float4 f = valid ? __ldcs(p + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      float fs[4] = {f.x, f.y, f.z, f.w};
+      const uint4 w = reinterpret_cast<const uint4*>(slice)[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        uint32_t u = __float_as_uint(fs[k]);
-        if (ROT) u ^= smask[64 + c * 4 + k];   // per-element masks (bit 31)
+        uint32_t u = ws[k];
+        if (ROT) u ^= smask[64 + c * 4 + k];  // per-element masks (bit 31)
         x[c * 4 + k] = __uint_as_float(u);
       }
     }
   }
 }
 
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// a - b for two lanes at once (fma with -1 rounds like the subtraction)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// Rotation (unless !ROT), group-32 abs-max scales and int4 codes of one
+// 128-coordinate slice, packed into the row layout: words[16] are the slice's
+// packed row words (d = 128: the whole row; d = 256: after the lane-pair
+// exchange, this lane's half of the row), scales[4] its groups' scales.
+// Butterfly stages run in the order bits 1, 2, 4, ... with u + w / u - w in
+// fp32 (two lanes at once from bit 2 on), the same operations as the
+// small-append kernel, so both give bit-identical codes.
+template <int D, bool ROT>
+__device__ __forceinline__ void quantize_slice(float (&x)[128], int sub, uint32_t (&words)[16],
+                                               float (&scales)[4]) {
+  constexpr int L = D / 128;
+  if (ROT) {
+#pragma unroll
+    for (int i = 0; i < 128; i += 2) {
+      const float u = x[i], w = x[i + 1];
+      x[i] = u + w;
+      x[i + 1] = u - w;
+    }
+#pragma unroll
+    for (int bit = 2; bit < 128; bit <<= 1)
+#pragma unroll
+      for (int i = 0; i < 128; i += 2)
+        if ((i & bit) == 0) {
+          const float2 u = make_float2(x[i], x[i + 1]), w = make_float2(x[i | bit], x[(i | bit) + 1]);
+          const float2 s = __fadd2_rn(u, w), d = sub2(u, w);
+          x[i] = s.x;
+          x[i + 1] = s.y;
+          x[i | bit] = d.x;
+          x[(i | bit) + 1] = d.y;
+        }
+    if (L == 2) {  // butterfly on coordinate bit 7 across the lane pair
+      const float sgn = sub ? -1.0f : 1.0f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
+        x[i] = fmaf(sgn, x[i], other);
+      }
+    }
+    const float2 norm = (D == 128) ? make_float2(kInvSqrt128, kInvSqrt128) : make_float2(0.0625f, 0.0625f);
+#pragma unroll
+    for (int i = 0; i < 128; i += 2) {
+      const float2 v = __fmul2_rn(make_float2(x[i], x[i + 1]), norm);
+      x[i] = v.x;
+      x[i + 1] = v.y;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float* xg = x + 32 * g;
+    float m[11];
+#pragma unroll
+    for (int j = 0; j < 10; ++j) m[j] = fmax3(fabsf(xg[3 * j]), fabsf(xg[3 * j + 1]), fabsf(xg[3 * j + 2]));
+    m[10] = fmaxf(fabsf(xg[30]), fabsf(xg[31]));
+    const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]),
+                             fmax3(fmax3(m[6], m[7], m[8]), m[9], m[10]));
+    const float s = __fdiv_rn(amax, 7.0f);
+    scales[g] = s;
+    const float r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+    const bool big = !(r <= 3.0e38f);  // subnormal scale: use the division throughout
+    const float2 rlo = make_float2(r * kBracketLo, r * kBracketLo);
+    const float2 rhi = make_float2(r * kBracketHi, r * kBracketHi);
+    const float2 magic = make_float2(kRneMagic, kRneMagic);
+    float code[32];
+    uint32_t diff = big ? 1u : 0u;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float2 v = make_float2(xg[j], xg[j + 1]);
+      const float2 flo = __ffma2_rn(v, rlo, magic), fhi = __ffma2_rn(v, rhi, magic);
+      diff |= (__float_as_uint(flo.x) ^ __float_as_uint(fhi.x)) |
+              (__float_as_uint(flo.y) ^ __float_as_uint(fhi.y));
+      code[j] = flo.x;
+      code[j + 1] = flo.y;
+    }
+    if (diff) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float c = rintf(__fdiv_rn(xg[j], s));
+        c = fminf(fmaxf(c, -7.0f), 7.0f);
+        code[j] = kRneMagic + c;  // exact: |c| <= 7
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xg[j] = code[j];
+  }
+
+  // Pack: group g (of this slice's 4), in-group j -> local word 2*(j/4) + g/2,
+  // bit 16*(g%2) + 4*(j%4).  For d = 128 local words are the row's 16 words;
+  // for d = 256 local word (2r + g/2) is row word 4r + 2*sub + g/2.  Each code
+  // is held as the float M + c (bits 0x4B400000 + c), so the bits minus
+  // (0x4B400000 - 8) are c + 8 in 1..15: a word is sum_k (c_k + 8) 16^k, built
+  // by shift-adds on the raw bits (wrapping; the constant is removed once),
+  // and flipping bit 3 of each nibble gives the two's-complement nibbles.
+  constexpr uint32_t kBias = (0x4B400000u - 8u) * 0x11111111u;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {
+      uint32_t w = 0u;
+#pragma unroll
+      for (int k = 7; k >= 0; --k) {
+        const int g = 2 * gp + k / 4, j = 4 * r + k % 4;
+        w = (w << 4) + __float_as_uint(x[32 * g + j]);
+      }
+      words[2 * r + gp] = (w - kBias) ^ 0x88888888u;
+    }
+
+  if (L == 2) {
+    // Lane 0 keeps sub-blocks 0..3, lane 1 keeps 4..7; each needs the
+    // partner's two words of those sub-blocks.
+    uint32_t recv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      // lane 1 sends sub-block k / 2, lane 0 sub-block 4 + k / 2 (static indices)
+      const uint32_t send = sub ? words[2 * (k / 2) + (k % 2)] : words[2 * (4 + k / 2) + (k % 2)];
+      recv[k] = __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+    uint32_t out[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      // r = sub ? 4 + q4 : q4; row words 4r..4r+3 =
+      // [lane0 w(2r), lane0 w(2r+1), lane1 w(2r), lane1 w(2r+1)]
+      const uint32_t own0 = sub ? words[2 * (4 + q4)] : words[2 * q4];
+      const uint32_t own1 = sub ? words[2 * (4 + q4) + 1] : words[2 * q4 + 1];
+      const uint32_t oth0 = recv[2 * q4], oth1 = recv[2 * q4 + 1];
+      out[4 * q4 + 0] = sub ? oth0 : own0;
+      out[4 * q4 + 1] = sub ? oth1 : own1;
+      out[4 * q4 + 2] = sub ? own0 : oth0;
+      out[4 * q4 + 3] = sub ? own1 : oth1;
+    }
+#pragma unroll
+    for (int w = 0; w < 16; ++w) words[w] = out[w];
+  }
+}
+
 template <int D, bool BF16, bool ROT>
-__global__ void __launch_bounds__(128) quantize_kernel(QuantizeArgs a) {
-  constexpr int L = D / 128;  // threads per vector
-  // Sign masks per 128-coordinate slice: [0, 64) XOR masks for bf16 pairs
-  // (bit 15 / bit 31), [64, 192) XOR masks for single fp32 elements (bit 31).
-  __shared__ uint32_t smask[192];
-  __shared__ uint32_t smask_hi[192];
+__global__ void __launch_bounds__(QCfg<BF16>::THREADS, 1) quantize_staged_kernel(QuantizeArgs a) {
+  using Q = QCfg<BF16>;
+  constexpr int L = D / 128;         // lanes per vector
+  constexpr int VPB = 32 / L;        // vectors per batch
+  constexpr int VB = D * Q::EB;      // input bytes per vector
+  constexpr int CPL = Q::SLICE / 16; // 16-byte copies per lane per batch
+  extern __shared__ __align__(16) unsigned char smem[];
+  // Sign masks per 128-coordinate slice (second slice at +192): [0, 64) XOR
+  // masks for bf16 pairs (bit 15 / bit 31), [64, 192) for fp32 (bit 31).
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (ROT) {
     for (int i = threadIdx.x; i < 128 * L; i += blockDim.x) {
       const int e = i % 128;
-      uint32_t* m = (i / 128) ? smask_hi : smask;
+      uint32_t* m = smask + (i / 128) * 192;
       m[64 + e] = (a.signs[i] < 0) ? 0x80000000u : 0u;
       if ((e & 1) == 0)
         m[e / 2] = ((a.signs[i] < 0) ? 0x00008000u : 0u) | ((a.signs[i + 1] < 0) ? 0x80000000u : 0u);
     }
-    __syncthreads();
   }
+  __syncthreads();
+  unsigned char* buf = smem + Q::MASKS + warp * 2 * Q::BUF;
   const int64_t per_kv = (int64_t)a.B * a.Hkv * a.n_new;
   const int64_t nvec = 2 * per_kv;
-  const int sub = (L == 2) ? (int)(threadIdx.x & 1) : 0;
-  const int64_t vec_stride = ((int64_t)gridDim.x * blockDim.x) / L;
-  const uint32_t* mymask = sub ? smask_hi : smask;
+  const int64_t nbatch = (nvec + VPB - 1) / VPB;
+  const int64_t nw = (int64_t)gridDim.x * Q::WARPS;
+  const unsigned char* kin = static_cast<const unsigned char*>(a.k);
+  const unsigned char* vin = static_cast<const unsigned char*>(a.v);
+  const bool narrow = per_kv <= 0x7fffffffLL;  // 32-bit index arithmetic suffices
 
-  for (int64_t vec = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;; vec += vec_stride) {
-    bool valid = vec < nvec;
-    if (L == 1) {
-      if (!valid) break;
-    } else if (__all_sync(0xffffffffu, !valid)) {
-      break;
+  // batch bi (VPB consecutive vectors: one contiguous span of K, then of V)
+  // -> padded slices of buffer dst; vectors past the end are zero-filled
+  auto issue = [&](int64_t bi, unsigned char* dst) {
+    const int64_t v0 = bi * VPB;
+    if (v0 + VPB <= per_kv || (v0 >= per_kv && v0 + VPB <= nvec)) {
+      // the whole batch is one contiguous span of K or of V: lane offsets once,
+      // then constant steps (the byte offset of copy c is 512 c + 16 lane)
+      const unsigned char* src = (v0 < per_kv ? kin + v0 * VB : vin + (v0 - per_kv) * VB) + 16 * lane;
+      const int o = 16 * lane;
+      unsigned char* d0 = dst + ((o / VB) * L + (o % VB) / Q::SLICE) * Q::PITCH + (o % VB) % Q::SLICE;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        // 512 c is a whole number of slices (512 = 2 slices at bf16, 1 at fp32)
+        cp_async16(d0 + (512 * c / Q::SLICE) * Q::PITCH, src + 512 * c, 16u);
+      }
+      cp_async_commit();
+      return;
     }
-    const int kv = valid ? (int)(vec / per_kv) : 0;
-    const int64_t rem = valid ? vec % per_kv : 0;
-    const int64_t bh = rem / a.n_new;
-    const int64_t n = rem % a.n_new;
-    const int b = (int)(bh / a.Hkv);
-    const int64_t p = valid ? (int64_t)a.pos[b] + n : -1;
-    const bool store = valid && p >= 0 && p < a.capacity;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int o = (c * 32 + lane) * 16;  // byte offset within the batch
+      const int vi = o / VB, ov = o % VB;
+      const int64_t v = v0 + vi;
+      const bool ok = v < nvec;
+      const unsigned char* src = ok ? (v < per_kv ? kin + v * VB : vin + (v - per_kv) * VB) + ov : kin;
+      cp_async16(dst + (vi * L + ov / Q::SLICE) * Q::PITCH + ov % Q::SLICE, src, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
 
+  int64_t bi = (int64_t)blockIdx.x * Q::WARPS + warp;
+  if (bi < nbatch) issue(bi, buf);
+  for (int k = 0; bi < nbatch; ++k, bi += nw) {
+    const unsigned char* cur = buf + (k & 1) * Q::BUF;
+    if (bi + nw < nbatch) {
+      issue(bi + nw, buf + ((k + 1) & 1) * Q::BUF);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const int sub = (L == 2) ? (lane & 1) : 0;
     float x[128];
-    load_slice<BF16, ROT>(kv ? a.v : a.k, rem * D + sub * 128, valid, mymask, x);
+    read_slice<BF16, ROT>(cur + lane * Q::PITCH, smask + sub * 192, x);
+    __syncwarp();  // the next iteration refills the other buffer, and this one after it
 
-    if (ROT) {
-#pragma unroll
-      for (int bit = 1; bit < 128; bit <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          if ((i & bit) == 0) {
-            const float u = x[i], w = x[i | bit];
-            x[i] = u + w;
-            x[i | bit] = u - w;
-          }
-        }
-      }
-      if (L == 2) {  // butterfly on coordinate bit 7 across the lane pair
-        const float sgn = sub ? -1.0f : 1.0f;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
-          x[i] = fmaf(sgn, x[i], other);
-        }
-      }
-      const float norm = (D == 128) ? kInvSqrt128 : 0.0625f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) x[i] *= norm;
-    }
-
-    float scales[4];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      float* xg = x + 32 * g;
-      float amax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xg[j]));
-      const float s = __fdiv_rn(amax, 7.0f);
-      scales[g] = s;
-      const float r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
-      const bool big = !(r <= 3.0e38f);   // subnormal scale: use the division throughout
-      const float rlo = r * kBracketLo, rhi = r * kBracketHi;
-      float code[32];
-      bool ambiguous = big;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float flo = fmaf(xg[j], rlo, kRneMagic);
-        const float fhi = fmaf(xg[j], rhi, kRneMagic);
-        ambiguous |= (flo != fhi);
-        code[j] = flo;
-      }
-      if (ambiguous) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float c = rintf(__fdiv_rn(xg[j], s));
-          c = fminf(fmaxf(c, -7.0f), 7.0f);
-          code[j] = kRneMagic + c;   // exact: |c| <= 7
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 32; ++j) xg[j] = code[j];
-    }
-
-    // Pack: group g (of this thread's 4), in-group j -> local word 2*(j/4) + g/2,
-    // bit 16*(g%2) + 4*(j%4).  For d = 128 local words are the row's 16 words;
-    // for d = 256 local word (2r + g/2) is row word 4r + 2*sub + g/2.
     uint32_t words[16];
-#pragma unroll
-    for (int w = 0; w < 16; ++w) words[w] = 0u;
-#pragma unroll
-    for (int g = 0; g < 4; ++g)
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        words[2 * (j / 4) + g / 2] =
-            bfi4(words[2 * (j / 4) + g / 2], __float_as_uint(x[32 * g + j]), 16 * (g % 2) + 4 * (j % 4));
+    float scales[4];
+    quantize_slice<D, ROT>(x, sub, words, scales);
 
-    if (L == 2) {
-      // Lane 0 keeps sub-blocks 0..3, lane 1 keeps 4..7; each needs the
-      // partner's two words of those sub-blocks.
-      uint32_t recv[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int r_send = sub ? (k / 2) : (4 + k / 2);
-        const uint32_t send = words[2 * r_send + (k % 2)];
-        recv[k] = __shfl_xor_sync(0xffffffffu, send, 1);
+    const int64_t v = bi * VPB + lane / L;
+    if (v < nvec) {
+      const bool kv = v >= per_kv;
+      const int64_t rem = kv ? v - per_kv : v;
+      int64_t bh, n;
+      if (narrow) {
+        const uint32_t r32 = (uint32_t)rem, bh32 = r32 / (uint32_t)a.n_new;
+        bh = bh32;
+        n = r32 - bh32 * (uint32_t)a.n_new;
+      } else {
+        bh = rem / a.n_new;
+        n = rem - bh * a.n_new;
       }
-      uint32_t out[16];
+      const int b = (int)((uint32_t)bh / (uint32_t)a.Hkv);
+      const int64_t p = (int64_t)a.pos[b] + n;
+      if (p >= 0 && p < a.capacity) {
+        const int64_t row = bh * a.capacity + p;
+        uint8_t* packed = kv ? a.v_packed : a.k_packed;
+        float* scl = kv ? a.v_scales : a.k_scales;
+        uint4* dst = reinterpret_cast<uint4*>(packed + row * (D / 2) + sub * 64);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int r = sub ? 4 + q4 : q4;
-        // row words 4r..4r+3 = [lane0 w(2r), lane0 w(2r+1), lane1 w(2r), lane1 w(2r+1)]
-        const uint32_t own0 = words[2 * r], own1 = words[2 * r + 1];
-        const uint32_t oth0 = recv[2 * q4], oth1 = recv[2 * q4 + 1];
-        out[4 * q4 + 0] = sub ? oth0 : own0;
-        out[4 * q4 + 1] = sub ? oth1 : own1;
-        out[4 * q4 + 2] = sub ? own0 : oth0;
-        out[4 * q4 + 3] = sub ? own1 : oth1;
+        for (int c = 0; c < 4; ++c)
+          dst[c] = make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+        *reinterpret_cast<float4*>(scl + row * (D / 32) + sub * 4) =
+            make_float4(scales[0], scales[1], scales[2], scales[3]);
       }
-#pragma unroll
-      for (int w = 0; w < 16; ++w) words[w] = out[w];
-    }
-
-    if (store) {
-      const int64_t row = bh * a.capacity + p;
-      uint8_t* packed = kv ? a.v_packed : a.k_packed;
-      float* scl = kv ? a.v_scales : a.k_scales;
-      uint4* dst = reinterpret_cast<uint4*>(packed + row * (D / 2) + sub * 64);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        dst[c] = make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
-      *reinterpret_cast<float4*>(scl + row * (D / 32) + sub * 4) =
-          make_float4(scales[0], scales[1], scales[2], scales[3]);
     }
   }
 }
@@ -314,16 +452,17 @@ __global__ void __launch_bounds__(128) quantize_warp_kernel(QuantizeArgs a) {
 
 template <int D, bool BF16, bool ROT>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
-  constexpr int L = D / 128;
-  const int64_t threads = 2LL * a.B * a.Hkv * a.n_new * L;
-  int64_t blocks = (threads + 127) / 128;
-  int dev = 0, sms = 148;
+  using Q = QCfg<BF16>;
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(quantize_staged_kernel<D, BF16, ROT>, Q::BYTES, smem_set);
+  if (e != cudaSuccess) return e;
+  const int64_t nbatch = (2LL * a.B * a.Hkv * a.n_new + 32 / (D / 128) - 1) / (32 / (D / 128));
+  int dev = 0, sms = kSmCount;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t cap = (int64_t)sms * 8;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  quantize_kernel<D, BF16, ROT><<<(unsigned)blocks, 128, 0, stream>>>(a);
+  int64_t blocks = (nbatch + Q::WARPS - 1) / Q::WARPS;
+  if (blocks > sms) blocks = sms;
+  quantize_staged_kernel<D, BF16, ROT><<<(unsigned)blocks, Q::THREADS, Q::BYTES, stream>>>(a);
   return cudaGetLastError();
 }
 
