@@ -191,6 +191,11 @@ def run_tq(args):
                    "bytes_moved": int(moved)}
     else:
         cache.append(k_all, v_all, pos0)
+    # host copy of sequence 0's first kv heads for the fidelity report
+    n_fid = min(2, Hkv)
+    ctx0 = int(ctx[0])
+    fid_k = k_all[0, :n_fid, :ctx0].float().cpu() if rank == 0 else None
+    fid_v = v_all[0, :n_fid, :ctx0].float().cpu() if rank == 0 else None
     del k_all, v_all
 
     # per-step inputs: one new token appended after the cached context
@@ -291,6 +296,29 @@ def run_tq(args):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_s = tt.item()
 
+    # comparisons on the same GPU (rank 0): bf16 dequantize-then-attend, and
+    # fidelity of this path's output to unquantized fp64 attention
+    baseline = fid = None
+    if rank == 0:
+        import numpy as np
+        cache.decode(q, ctx_dev, max_ctx, scale, out)
+        bl = dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, cache.signs,
+                                     min(args.steps, 50), 3, stream)
+        o_ours, o_bl = out.double().flatten(1), bl.pop("out").double().flatten(1)
+        bl["cosine_vs_int4_path_min"] = round(float(torch.nn.functional.cosine_similarity(
+            o_ours, o_bl, dim=1).min()), 5)
+        bl["int4_decode_speedup"] = round(bl["dequantize_then_attend_us"] / (dec_s * 1e6), 2)
+        baseline = bl
+        khat, _ = cache.dequantize(ctx0 + 1, torch.float32)
+        G = Hq // Hkv
+        fid_k = np.concatenate([fid_k.numpy(), k_new[0, :n_fid].float().cpu().numpy()], 1)
+        fid_v = np.concatenate([fid_v.numpy(), v_new[0, :n_fid].float().cpu().numpy()], 1)
+        fid = fidelity(fid_k, fid_v, q[0, :n_fid * G].float().cpu().numpy(),
+                       out[0, :n_fid * G].cpu().numpy(), khat[0, :n_fid].cpu().numpy(),
+                       None if cache.signs is None else cache.signs.cpu(), scale, G)
+        fid["sample"] = f"sequence 0, kv heads 0..{n_fid - 1} ({n_fid * G} query heads), {ctx0 + 1} tokens"
+        del khat
+
     kvb = kv_bytes(w, (ctx + 1).tolist())
     qo_bytes = q.numel() * q.element_size() + out.numel() * out.element_size()
     algo = kvb + qo_bytes
@@ -327,6 +355,8 @@ def run_tq(args):
                   "with pinned host copies, per step",
         "clocks": clocks,
         "bulk_prefill": prefill,
+        "bf16_dequantize_then_attend": baseline,
+        "fidelity_vs_unquantized_fp64": fid,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, seed)
@@ -335,6 +365,98 @@ def run_tq(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def rotation_matrix(d, signs, device):
+    """R = H_d diag(signs) / sqrt(d) (Sylvester H_d) as fp64 on `device`; identity without signs."""
+    import torch
+    if signs is None:
+        return torch.eye(d, dtype=torch.float64, device=device)
+    H = torch.ones(1, 1, dtype=torch.float64)
+    while H.shape[0] < d:
+        H = torch.cat([torch.cat([H, H], 1), torch.cat([H, -H], 1)], 0)
+    return (H * signs.double().cpu()[None, :] / math.sqrt(d)).to(device)
+
+
+def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, signs, steps, warmup, stream):
+    """In-house bf16 dequantize-then-attend on the same GPU: every step
+    materializes bf16 K and V from the packed cache (tq_dequantize, one pass)
+    and runs torch's bf16 scaled_dot_product_attention over them (query rotated
+    into the cache basis, output rotated back).  Also times the attention alone
+    on the materialized bf16 cache (what a bf16 KV cache would cost)."""
+    import torch
+    import torch.nn.functional as F
+
+    from compressed_domain_attention_tq_b200 import _lib
+    B, Hq, d = q.shape
+    Hkv = cache.k_packed.shape[1]
+    dev = q.device
+    R = rotation_matrix(d, signs, dev).float()
+    Kb = torch.empty(B, Hkv, max_ctx, d, dtype=torch.bfloat16, device=dev)
+    Vb = torch.empty_like(Kb)
+    lens = ctx_dev.long()
+    mask = None
+    if int(lens.min()) < max_ctx:  # ragged batch: mask each sequence's tail
+        mask = (torch.arange(max_ctx, device=dev)[None, :] < lens[:, None])[:, None, None, :]
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+
+    def attend():
+        qr = (q.float() @ R.T).to(torch.bfloat16)[:, :, None, :]
+        o = F.scaled_dot_product_attention(qr, Kb, Vb, attn_mask=mask, scale=scale, enable_gqa=True)
+        out.copy_(o[:, :, 0].float() @ R)
+
+    def full():
+        _lib.dequantize(cache.k_packed, cache.k_scales, max_ctx, Kb)
+        _lib.dequantize(cache.v_packed, cache.v_scales, max_ctx, Vb)
+        attend()
+
+    for _ in range(warmup):
+        full()
+    torch.cuda.synchronize()
+    res = {}
+    for name, fn in (("dequantize_then_attend", full), ("attend_only_bf16_cache", attend)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(steps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        res[name + "_us"] = round(a.elapsed_time(b) * 1e3 / steps, 2)
+        del g
+    res["bf16_cache_bytes"] = 2 * Kb.numel() * Kb.element_size()
+    res["out"] = out
+    return res
+
+
+def fidelity(k_h, v_h, q_h, out_h, khat_h, signs, scale, G):
+    """Fidelity of the int4 path to unquantized fp64 attention (report only).
+
+    k_h, v_h [n][T][d] unquantized (unrotated) inputs of n kv heads; q_h [n*G][d];
+    out_h [n*G][d] the CUDA path's output; khat_h [n][T][d] dequantized keys
+    (rotated basis).  Cosine similarity of each query head's output with exact
+    softmax attention, and agreement of argmax_t q.k between the unquantized
+    and the dequantized keys."""
+    import numpy as np
+    d = k_h.shape[-1]
+    R = rotation_matrix(d, signs, "cpu").numpy()
+    cos, agree = [], []
+    for h in range(k_h.shape[0]):
+        K, V = k_h[h].astype(np.float64), v_h[h].astype(np.float64)
+        Q = q_h[h * G:(h + 1) * G].astype(np.float64)
+        S = K @ Q.T * scale
+        P = np.exp(S - S.max(0, keepdims=True))
+        O = (P.T @ V) / P.sum(0)[:, None]
+        Og = out_h[h * G:(h + 1) * G].astype(np.float64)
+        cos += list((O * Og).sum(1) / (np.linalg.norm(O, axis=1) * np.linalg.norm(Og, axis=1)))
+        Sq = khat_h[h].astype(np.float64) @ (Q @ R.T).T
+        agree += list(S.argmax(0) == Sq.argmax(0))
+    return {"cosine_min": round(float(min(cos)), 7), "cosine_mean": round(float(np.mean(cos)), 7),
+            "top1_qk_argmax_agreement": round(float(np.mean(agree)), 4), "query_heads": len(cos)}
 
 
 def oracle_sample(w, seed, kv_head=0):

@@ -20,7 +20,8 @@ STATIC_SCRATCH_BYTES = 8 << 20   # TQ_STATIC_SCRATCH_BYTES in include/tq.h
 TQ_F32, TQ_BF16 = 0, 1
 
 SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
-           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_static_scratch", "tq_status_string")
+           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_static_scratch", "tq_dequantize",
+           "tq_status_string")
 
 _lib = None
 
@@ -52,6 +53,8 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode_static_scratch.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P,
                                                        i64, P, i32, P, f32, P, P]
     lib.tq_sdpa_int4_decode_static_scratch.restype = i32
+    lib.tq_dequantize.argtypes = [P, P, i32, i32, i64, i32, i32, P, i32, P]
+    lib.tq_dequantize.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -133,3 +136,14 @@ def sdpa_int4_decode_static_scratch(q, k_packed, k_scales, v_packed, v_scales, c
         _ptr(signs), float(attn_scale), _ptr(out), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode_static_scratch")
+
+
+def dequantize(packed, scales, rows, out, stream=None):
+    """out[B][Hkv][rows][d] (fp32 or bf16) = scale * code of rows 0 .. rows-1 of
+    each sequence of a packed cache [B][Hkv][capacity][d/2] (rotated basis)."""
+    _need_cuda(packed, scales, out)
+    B, H, cap, half = packed.shape
+    rc = load().tq_dequantize(_ptr(packed), _ptr(scales), B * H, int(rows), cap, 2 * half, 32,
+                              _ptr(out), _dtype_code(out), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_dequantize")

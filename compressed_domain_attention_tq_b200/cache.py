@@ -56,3 +56,13 @@ class Int4KVCache:
         _lib.sdpa_int4_decode(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
                               ctx_lens, max_ctx, self.signs, attn_scale, out, ws, stream)
         return out
+
+    def dequantize(self, rows: int, dtype=torch.bfloat16, stream=None):
+        """Dequantized K and V of rows 0 .. rows-1 of every sequence, [B][Hkv][rows][d]
+        in the rotated basis (scale * code; not used by decode)."""
+        k = torch.empty(self.batch, self.num_kv_heads, rows, self.head_dim, dtype=dtype,
+                        device=self.k_packed.device)
+        v = torch.empty_like(k)
+        _lib.dequantize(self.k_packed, self.k_scales, rows, k, stream)
+        _lib.dequantize(self.v_packed, self.v_scales, rows, v, stream)
+        return k, v

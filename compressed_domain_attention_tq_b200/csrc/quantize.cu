@@ -38,12 +38,6 @@ constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21 (exact)
 constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21 (exact)
 constexpr int64_t kSmallAppendVectors = 8192;  // up to this many: one warp per vector
 
-__device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t nib_src, int pos) {
-  uint32_t r;
-  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(r) : "r"(nib_src), "r"(word), "r"(pos));
-  return r;
-}
-
 // Async 16-byte global -> shared copy; src_bytes = 0 zero-fills without reading.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));

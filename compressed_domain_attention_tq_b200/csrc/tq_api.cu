@@ -104,6 +104,27 @@ tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, in
                      "tq_quantize_append");
 }
 
+tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_seq, int32_t rows,
+                        int64_t row_stride, int32_t head_dim, int32_t group, void* out,
+                        tq_dtype out_dtype, void* cuda_stream) {
+  if (!packed || !scales || !out) return TQ_ERR_INVALID_ARG;
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (n_seq < 1 || rows < 1 || row_stride < rows) return TQ_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
+  DequantizeArgs a;
+  a.packed = packed;
+  a.scales = scales;
+  a.n_seq = n_seq;
+  a.rows = rows;
+  a.row_stride = row_stride;
+  a.d = head_dim;
+  a.out = out;
+  a.bf16 = out_dtype == TQ_BF16;
+  return cuda_status(launch_dequantize(a, static_cast<cudaStream_t>(cuda_stream)), "tq_dequantize");
+}
+
 size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                  int32_t head_dim, int32_t max_ctx) {
   DecodePlan p;

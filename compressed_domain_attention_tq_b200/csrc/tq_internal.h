@@ -37,6 +37,15 @@ struct QuantizeArgs {
   int64_t capacity;
 };
 
+struct DequantizeArgs {
+  const uint8_t* packed;
+  const float* scales;
+  int n_seq, rows, d;
+  int64_t row_stride;
+  void* out;
+  int bf16;
+};
+
 struct DecodeArgs {
   const void* q;
   int q_bf16;
@@ -71,6 +80,7 @@ cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& d
 }
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 bool decode_mma_supported(int d, int G);
 int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path

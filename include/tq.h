@@ -189,6 +189,28 @@ TQ_API tq_status tq_sdpa_int4_decode_static_scratch(
     const uint8_t* v_packed, const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
     int32_t max_ctx, const int8_t* signs, float attn_scale, float* out, void* cuda_stream);
 
+/*
+ * tq_dequantize -- materialize dequantized rows of a packed cache: value of
+ * coordinate i = scale[i/32] * code[i], in the rotated basis the cache holds
+ * (the layout above).  Not part of the decode path, which never forms these
+ * values (Open-TQ-Metal abstract: attention on the compressed representation
+ * with no intermediate dequantized K/V matrix); it serves callers that need
+ * the plain values, and a dequantize-then-attend comparison.
+ *
+ *  packed      uint8 rows of d/2 bytes, scales float rows of d/32: n_seq
+ *              sequences of `rows` rows each, sequence s starting at row
+ *              s * row_stride (e.g. n_seq = B * Hkv, row_stride = capacity).
+ *  out         [n_seq][rows][d] of out_dtype (fp32: exact products; bf16:
+ *              the fp32 product rounded to nearest even).
+ *
+ * Returns TQ_ERR_INVALID_ARG for NULL pointers, n_seq or rows < 1,
+ * row_stride < rows, misaligned pointers (16 bytes); TQ_ERR_UNSUPPORTED for
+ * head_dim not in {128, 256} or group != 32.
+ */
+TQ_API tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_seq,
+                               int32_t rows, int64_t row_stride, int32_t head_dim, int32_t group,
+                               void* out, tq_dtype out_dtype, void* cuda_stream);
+
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);
 

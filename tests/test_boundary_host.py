@@ -144,6 +144,23 @@ def test_decode_rejects_on_host(lib, kw, code):
     assert decode(lib, fb, **kw) == code
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(packed=None), _lib.TQ_ERR_INVALID_ARG), (dict(scales=None), _lib.TQ_ERR_INVALID_ARG),
+    (dict(out=None), _lib.TQ_ERR_INVALID_ARG), (dict(dtype=3), _lib.TQ_ERR_INVALID_ARG),
+    (dict(n_seq=0), _lib.TQ_ERR_INVALID_ARG), (dict(rows=0), _lib.TQ_ERR_INVALID_ARG),
+    (dict(rows=65, stride=64), _lib.TQ_ERR_INVALID_ARG), (dict(d=64), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(group=16), _lib.TQ_ERR_UNSUPPORTED), (dict(out=8), _lib.TQ_ERR_INVALID_ARG)])
+def test_dequantize_rejects_on_host(lib, kw, code):
+    fb = FakeBuffers()
+    a = dict(packed=fb.p(1024), scales=fb.p(2048), n_seq=2, rows=64, stride=64, d=128, group=32,
+             out=fb.p(4096), dtype=1, stream=None)
+    if kw.get("out") == 8:
+        kw = dict(out=fb.p(4104))
+    a.update(kw)
+    assert lib.tq_dequantize(a["packed"], a["scales"], a["n_seq"], a["rows"], a["stride"], a["d"],
+                             a["group"], a["out"], a["dtype"], a["stream"]) == code
+
+
 def test_workspace_size_is_exact_threshold(lib):
     fb = FakeBuffers()
     need = _lib.decode_workspace_bytes(1, 8, 2, 128, 64)
