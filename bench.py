@@ -4,7 +4,9 @@
 A step = quantize-append of one new token (K and V of every kv head) into the
 packed int4 cache + sdpa_int4 decode of one query token over the whole
 context, on the 64/8-head, d=128, 128K-context Llama-3.1-70B-shaped layer
-(synthetic seeded inputs, bf16).  Prints one JSON line (rank 0).
+(synthetic seeded inputs, bf16), made with one tq_sdpa_int4_decode_append call
+(the two-call step, append then decode, is timed beside it).  Prints one JSON
+line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...   (weak scaling, N replicas)
@@ -208,9 +210,8 @@ def run_tq(args):
     scale = w.attn_scales[0]
     ws = cache.workspace(Hq, max_ctx)
 
-    def step():
-        cache.append(k_new, v_new, pos)
-        cache.decode(q, ctx_dev, max_ctx, scale, out)
+    def step():  # one decode step in one call: append the new token, then attend
+        cache.decode_append(q, k_new, v_new, ctx_dev, max_ctx, scale, out)
 
     for i in range(args.warmup):
         flush.fill_(i & 0xFF)
@@ -224,7 +225,13 @@ def run_tq(args):
     kvb_step = kv_bytes(w, (ctx + 1).tolist())
     use_flush = kvb_step <= l2_bytes  # else every step's reads already exceed the L2
     g_step, g_dec, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_two = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
+        for i in range(args.steps):
+            if use_flush:
+                flush.fill_(i & 0xFF)
+            step()
+    with torch.cuda.graph(g_two):  # the same step as two calls (append, then decode)
         for i in range(args.steps):
             if use_flush:
                 flush.fill_(i & 0xFF)
@@ -241,6 +248,7 @@ def run_tq(args):
     for i in range(max(1, args.warmup // args.steps + 1)):
         g_step.replay()
         g_dec.replay()
+        g_two.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -248,7 +256,7 @@ def run_tq(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     ev[0].record(stream)
     g_step.replay()
     ev[1].record(stream)
@@ -257,6 +265,8 @@ def run_tq(args):
     if use_flush:
         g_flush.replay()
     ev[3].record(stream)
+    g_two.replay()
+    ev[4].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -264,11 +274,13 @@ def run_tq(args):
     flush_s = ev[2].elapsed_time(ev[3]) / 1e3 / args.steps if use_flush else 0.0
     step_s = ev[0].elapsed_time(ev[1]) / 1e3 / args.steps - flush_s
     dec_s = ev[1].elapsed_time(ev[2]) / 1e3 / args.steps - flush_s
+    two_s = ev[3].elapsed_time(ev[4]) / 1e3 / args.steps - flush_s
     q_s = max(step_s - dec_s, 0.0)
     if world > 1:
-        tt = torch.tensor([step_s, dec_s, q_s], dtype=torch.float64, device=dev)
+        tt = torch.tensor([step_s, dec_s, q_s, two_s], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        step_s, dec_s, q_s = tt.tolist()
+        step_s, dec_s, q_s, two_s = tt.tolist()
+    del g_step, g_dec, g_flush, g_two
 
     # end to end through the public API with pinned host buffers
     h_q = q.cpu().pin_memory()
@@ -283,8 +295,7 @@ def run_tq(args):
         d_q.copy_(h_q, non_blocking=True)
         d_k.copy_(h_k, non_blocking=True)
         d_v.copy_(h_v, non_blocking=True)
-        cache.append(d_k, d_v, pos)
-        cache.decode(d_q, ctx_dev, max_ctx, scale, out)
+        cache.decode_append(d_q, d_k, d_v, ctx_dev, max_ctx, scale, out)
         h_out.copy_(out, non_blocking=True)
         b.record(stream)
         b.synchronize()
@@ -329,7 +340,8 @@ def run_tq(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
         "us_per_step": round(step_s * 1e6, 2), "decode_us": round(dec_s * 1e6, 2),
-        "quantize_append_us": round(q_s * 1e6, 2),
+        "append_in_step_us": round(q_s * 1e6, 2),
+        "two_call_step_us": round(two_s * 1e6, 2),
         "pct_of_8TBps": round(100 * kvb / step_s / 1e9 / NOMINAL_HBM_GBS, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 codes, fp32 accumulation", "data": "synthetic (seeded N(0,1), bf16)",
@@ -349,10 +361,12 @@ def run_tq(args):
                 "us_per_step": round(e2e_s * 1e6, 2),
                 "h2d_bytes_per_step": int(h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()),
                 "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
+        "step": ("tq_sdpa_int4_decode_append: the decode kernel quantizes the new token of each "
+                 "kv head into the cache, then attends (split-K kernel + merge, 2 launches)"),
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
-                  "launching stream (decode split from a K-decode graph); e2e: public API calls "
-                  "with pinned host copies, per step",
+                  "launching stream (decode split from a K-decode graph; the two-call step "
+                  "from a third graph); e2e: public API calls with pinned host copies, per step",
         "clocks": clocks,
         "bulk_prefill": prefill,
         "bf16_dequantize_then_attend": baseline,

@@ -20,7 +20,8 @@ STATIC_SCRATCH_BYTES = 8 << 20   # TQ_STATIC_SCRATCH_BYTES in include/tq.h
 TQ_F32, TQ_BF16 = 0, 1
 
 SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
-           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_static_scratch", "tq_dequantize",
+           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_append", "tq_sdpa_int4_decode_static_scratch",
+           "tq_dequantize",
            "tq_status_string")
 
 _lib = None
@@ -50,6 +51,9 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64, P, i32,
                                         P, f32, P, P, sz, P]
     lib.tq_sdpa_int4_decode.restype = i32
+    lib.tq_sdpa_int4_decode_append.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P,
+                                               i64, P, i32, P, f32, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_append.restype = i32
     lib.tq_sdpa_int4_decode_static_scratch.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P,
                                                        i64, P, i32, P, f32, P, P]
     lib.tq_sdpa_int4_decode_static_scratch.restype = i32
@@ -121,6 +125,24 @@ def sdpa_int4_decode(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ct
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode")
+
+
+def sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                            max_ctx, signs, attn_scale, out, workspace, stream=None):
+    """One decode step: quantize k_new, v_new [B][Hkv][1][d] into row ctx_lens[b]-1
+    of the cache, then out[B][Hq][d] = attention of q over rows 0..ctx_lens[b]-1."""
+    _need_cuda(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out, workspace)
+    if k_new.dtype != v_new.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_append(
+        _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq, Hkv, d, 32,
+        _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), k_packed.shape[2],
+        _ptr(ctx_lens), int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_append")
 
 
 def sdpa_int4_decode_static_scratch(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx,

@@ -57,6 +57,21 @@ class Int4KVCache:
                               ctx_lens, max_ctx, self.signs, attn_scale, out, ws, stream)
         return out
 
+    def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float | None = None,
+                      out: torch.Tensor | None = None, stream=None):
+        """One decode step: append k_new, v_new [B][Hkv][1][d] at row ctx_lens[b]-1, then
+        attend q [B][Hq][d] over rows 0..ctx_lens[b]-1 (lengths include the new token)."""
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_int4_decode_append(q, k_new, v_new, self.k_packed, self.k_scales, self.v_packed,
+                                     self.v_scales, ctx_lens, max_ctx, self.signs, attn_scale, out,
+                                     ws, stream)
+        return out
+
     def dequantize(self, rows: int, dtype=torch.bfloat16, stream=None):
         """Dequantized K and V of rows 0 .. rows-1 of every sequence, [B][Hkv][rows][d]
         in the rotated basis (scale * code; not used by decode)."""

@@ -47,6 +47,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "quantize_vector.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -837,6 +838,29 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   // the merge kernel may be scheduled now; it waits for this grid's writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
+
+  // Fused append: for every (sequence, kv head) whose last chunk is one of this
+  // CTA's items, warps 4 and 5 quantize that kv head's new K and V token into
+  // row T - 1 (T the clamped context length) while the other warps prepare the
+  // first query.  Only that chunk reads the row, and this CTA issues no copy
+  // before the barrier that follows (in the first item's query preparation);
+  // the proxy fence orders these generic writes before the bulk copies.
+  if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
+    const bool isv = warp == 5;
+    const int eb = a.kv_bf16 ? 2 : 4;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      int b, kvh, c, t0, t1;
+      if (!item_range(a, it, b, kvh, c, t0, t1)) continue;
+      if (t1 != clamp_ctx_mma(a.ctx_lens[b], a.max_ctx)) continue;  // not the last chunk
+      const int64_t bh = (int64_t)b * a.Hkv + kvh;
+      const int64_t row = bh * a.capacity + (t1 - 1);
+      quantize_vector_warp<D>(static_cast<const unsigned char*>(isv ? a.v_new : a.k_new) + bh * D * eb,
+                              a.kv_bf16, a.signs,
+                              const_cast<uint8_t*>(isv ? a.v_packed : a.k_packed) + row * (D / 2),
+                              const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
 
   const int gid = lane >> 2, tig = lane & 3;
   const int rho[4] = {slot_row(2 * tig), slot_row(2 * tig + 1), 8 + slot_row(2 * tig),

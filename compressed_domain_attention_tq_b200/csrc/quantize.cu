@@ -27,6 +27,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "quantize_vector.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -361,15 +362,10 @@ __global__ void __launch_bounds__(QCfg<BF16>::THREADS, 1) quantize_staged_kernel
 }
 
 // Small appends (a decode step quantizes 2 * B * Hkv vectors): one warp per
-// vector, lane l holding coordinates E*l .. E*l+E-1 (E = D/32), so a step's
-// few vectors finish in a few hundred cycles instead of one long serial
-// thread each.  The butterfly stages run in the same order and with the same
-// operations as quantize_kernel's (bits 1, 2, 4, ...), so the rotated values
-// are bit-identical; codes use the IEEE division directly.
+// vector (quantize_vector_warp), so a step's few vectors finish in a few
+// hundred cycles instead of one long serial thread each.
 template <int D>
 __global__ void __launch_bounds__(128) quantize_warp_kernel(QuantizeArgs a) {
-  constexpr int E = D / 32;        // coordinates per lane
-  constexpr int GL = 32 / E;       // lanes per quantization group
   const int lane = threadIdx.x & 31;
   const int64_t per_kv = (int64_t)a.B * a.Hkv * a.n_new;
   const int64_t vec = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -378,70 +374,14 @@ __global__ void __launch_bounds__(128) quantize_warp_kernel(QuantizeArgs a) {
   const int64_t rem = vec % per_kv;
   const int64_t bh = rem / a.n_new, n = rem % a.n_new;
   const int b = (int)(bh / a.Hkv);
-  const int64_t p = (int64_t)a.pos[b] + n;
+  int64_t p = (int64_t)a.pos[b] + n;
+  if (a.pos_is_ctx) p = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
   if (p < 0 || p >= a.capacity) return;  // whole warp
-  float x[E];
-  const int64_t off = rem * D + lane * E;
-  const void* src = kv ? a.v : a.k;
-  if (a.bf16) {
-    const uint16_t* s16 = static_cast<const uint16_t*>(src) + off;
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] = __uint_as_float((uint32_t)s16[e] << 16);
-  } else {
-    const float* s32 = static_cast<const float*>(src) + off;
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] = s32[e];
-  }
-  if (a.signs) {
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-      if (a.signs[lane * E + e] < 0) x[e] = __uint_as_float(__float_as_uint(x[e]) ^ 0x80000000u);
-#pragma unroll
-    for (int bit = 1; bit < E; bit <<= 1)
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if ((e & bit) == 0) {
-          const float u = x[e], w = x[e | bit];
-          x[e] = u + w;
-          x[e | bit] = u - w;
-        }
-#pragma unroll
-    for (int lb = 1; lb < 32; lb <<= 1)
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float v = __shfl_xor_sync(0xffffffffu, x[e], lb);
-        x[e] = (lane & lb) ? v - x[e] : x[e] + v;
-      }
-    const float norm = (D == 128) ? kInvSqrt128 : 0.0625f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) x[e] *= norm;
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
-#pragma unroll
-  for (int o = 1; o < GL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = __fdiv_rn(amax, 7.0f);
-  uint32_t half[E / 4];  // 4 codes per 16-bit half-word
-#pragma unroll
-  for (int h = 0; h < E / 4; ++h) half[h] = 0u;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float c = 0.0f;
-    if (s > 0.0f) c = fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -7.0f), 7.0f);
-    half[e / 4] |= ((uint32_t)(int)c & 0xFu) << (4 * (e % 4));
-  }
-  // coordinate i = E*lane + e: group g = lane / GL, in-group j = E*(lane % GL) + e,
-  // sub-block j / 4, so half-word h sits at byte (j0/4 + h) * 2*NG + 2*g
-  constexpr int NG = D / 32;
-  const int g = lane / GL;
-  const int j0 = E * (lane % GL);
   const int64_t row = bh * a.capacity + p;
-  uint8_t* packed = (kv ? a.v_packed : a.k_packed) + row * (D / 2);
-#pragma unroll
-  for (int h = 0; h < E / 4; ++h)
-    *reinterpret_cast<uint16_t*>(packed + (j0 / 4 + h) * 2 * NG + 2 * g) = (uint16_t)half[h];
-  if (lane % GL == 0) (kv ? a.v_scales : a.k_scales)[row * NG + g] = s;
+  const int eb = a.bf16 ? 2 : 4;
+  quantize_vector_warp<D>(static_cast<const unsigned char*>(kv ? a.v : a.k) + rem * D * eb, a.bf16,
+                          a.signs, (kv ? a.v_packed : a.k_packed) + row * (D / 2),
+                          (kv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
 }
 
 template <int D, bool BF16, bool ROT>
@@ -464,7 +404,7 @@ cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const int64_t nvec = 2LL * a.B * a.Hkv * a.n_new;
-  if (nvec <= kSmallAppendVectors) {
+  if (nvec <= kSmallAppendVectors || a.pos_is_ctx) {
     const unsigned blocks = (unsigned)((nvec + 3) / 4);
     if (a.d == 128) quantize_warp_kernel<128><<<blocks, 128, 0, stream>>>(a);
     else quantize_warp_kernel<256><<<blocks, 128, 0, stream>>>(a);

@@ -139,16 +139,25 @@ int32_t tq_decode_chunk_tokens(int32_t batch, int32_t num_q_heads, int32_t num_k
   return p.chunk;
 }
 
-tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
-                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                              int32_t group, const uint8_t* k_packed, const float* k_scales,
-                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
-                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
-                              float attn_scale, float* out, void* workspace,
-                              size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+// Shared by tq_sdpa_int4_decode and tq_sdpa_int4_decode_append (k_new, v_new
+// non-NULL: append the new token of every (sequence, kv head) first).
+static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new,
+                             tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t group,
+                             const uint8_t* k_packed, const float* k_scales,
+                             const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                             const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                             float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+                             void* cuda_stream, const char* where) {
   if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
     return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  const bool append = k_new != nullptr || v_new != nullptr;
+  if (append && (!k_new || !v_new || (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16) ||
+                 !aligned16(k_new) || !aligned16(v_new)))
+    return TQ_ERR_INVALID_ARG;
   if (batch < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
       num_q_heads % num_kv_heads != 0)
     return TQ_ERR_INVALID_ARG;
@@ -182,12 +191,68 @@ tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
   a.attn_scale = attn_scale;
   a.out = out;
   a.workspace = workspace;
+  a.k_new = nullptr;
+  a.v_new = nullptr;
+  a.kv_bf16 = kv_dtype == TQ_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const cudaError_t e = decode_mma_supported(head_dim, num_q_heads / num_kv_heads)
-                            ? launch_decode_mma(a, s)
-                            : launch_decode_simt(a, s);
-  if (e != cudaSuccess) return cuda_status(e, "tq_sdpa_int4_decode (split-K kernel)");
-  return cuda_status(launch_merge(a, s), "tq_sdpa_int4_decode (merge kernel)");
+  const bool mma = decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
+  if (append && mma) {  // the decode kernel quantizes the new tokens itself
+    a.k_new = k_new;
+    a.v_new = v_new;
+  } else if (append) {  // the CUDA-core decode: one small-append launch first
+    QuantizeArgs qa;
+    qa.k = k_new;
+    qa.v = v_new;
+    qa.bf16 = kv_dtype == TQ_BF16;
+    qa.B = batch;
+    qa.Hkv = num_kv_heads;
+    qa.n_new = 1;
+    qa.d = head_dim;
+    qa.pos = ctx_lens;
+    qa.pos_is_ctx = 1;
+    qa.max_ctx = max_ctx;
+    qa.signs = signs;
+    qa.k_packed = const_cast<uint8_t*>(k_packed);
+    qa.k_scales = const_cast<float*>(k_scales);
+    qa.v_packed = const_cast<uint8_t*>(v_packed);
+    qa.v_scales = const_cast<float*>(v_scales);
+    qa.capacity = capacity;
+    const cudaError_t e = launch_quantize(qa, s);
+    if (e != cudaSuccess) return cuda_status(e, where);
+  }
+  const cudaError_t e = mma ? launch_decode_mma(a, s) : launch_decode_simt(a, s);
+  if (e != cudaSuccess) return cuda_status(e, where);
+  return cuda_status(launch_merge(a, s), where);
+}
+
+extern "C" {
+
+tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t group, const uint8_t* k_packed, const float* k_scales,
+                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                              float attn_scale, float* out, void* workspace,
+                              size_t workspace_bytes, void* cuda_stream) {
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode");
+}
+
+tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
+                                     const void* v_new, tq_dtype kv_dtype, int32_t batch,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t group, uint8_t* k_packed, float* k_scales,
+                                     uint8_t* v_packed, float* v_scales, int64_t capacity,
+                                     const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                                     float attn_scale, float* out, void* workspace,
+                                     size_t workspace_bytes, void* cuda_stream) {
+  if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
+  return decode_impl(q, q_dtype, k_new, v_new, kv_dtype, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode_append");
 }
 
 }  // extern "C"

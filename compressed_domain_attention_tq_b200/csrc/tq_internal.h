@@ -35,6 +35,8 @@ struct QuantizeArgs {
   uint8_t* v_packed;
   float* v_scales;
   int64_t capacity;
+  int pos_is_ctx = 0;  // 1: token n of sequence b goes to row clamp(pos[b], 1, max_ctx) - 1 + n
+  int max_ctx = 0;
 };
 
 struct DequantizeArgs {
@@ -62,6 +64,9 @@ struct DecodeArgs {
   float* out;
   void* workspace;
   DecodePlan plan;
+  const void* k_new;  // fused append (decode_mma only): [B][Hkv][1][d] new K and V, or NULL
+  const void* v_new;
+  int kv_bf16;
 };
 
 // Raise a kernel's dynamic shared memory limit once per device (the first

@@ -159,6 +159,36 @@ TQ_API tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t ba
                               size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * tq_sdpa_int4_decode_append -- one decode step in one call: the new token's K
+ * and V of every (sequence, kv head) are quantized into the cache (as
+ * tq_quantize_append does, bit-identically) and the query then attends over
+ * the cache including that token ("quantize the KV cache as it is generated,
+ * then attend on the compressed cache": Open-TQ-Metal abstract; forum summary,
+ * section "on-the-fly quantization").
+ *
+ *  k_new, v_new  [B][Hkv][1][d] of kv_dtype (fp32 or bf16), unrotated.
+ *  ctx_lens      lengths INCLUDING the new token: with T_b = ctx_lens[b]
+ *                clamped to [1, max_ctx] (flagged as in tq_sdpa_int4_decode),
+ *                the new token is written to row T_b - 1 and rows 0 .. T_b - 1
+ *                are attended.
+ *  Every other argument is as in tq_sdpa_int4_decode; the cache buffers are
+ *  written (row T_b - 1 of each sequence and kv head) as well as read.
+ *
+ * On the tensor-core decode (head_dim 128 with Hq/Hkv <= 8, head_dim 256 with
+ * Hq/Hkv <= 4) the decode kernel quantizes the new tokens itself: the CTA that
+ * attends a sequence's last chunk writes its row before copying it, so the
+ * step is the decode's launches only.  Otherwise a small append launch runs
+ * first.  Returns the errors of tq_sdpa_int4_decode, and TQ_ERR_INVALID_ARG
+ * for NULL or misaligned k_new / v_new or an invalid kv_dtype.
+ */
+TQ_API tq_status tq_sdpa_int4_decode_append(
+    const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
+    uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales, int64_t capacity,
+    const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, float attn_scale, float* out,
+    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * tq_sdpa_int4_decode_static_scratch -- tq_sdpa_int4_decode without a
  * caller-provided workspace.  The method's pages have no counterpart to this
  * call; it exists for callers that cannot allocate device memory: a plug-in

@@ -161,6 +161,26 @@ def test_dequantize_rejects_on_host(lib, kw, code):
                              a["group"], a["out"], a["dtype"], a["stream"]) == code
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(k_new=None), _lib.TQ_ERR_INVALID_ARG), (dict(v_new=None), _lib.TQ_ERR_INVALID_ARG),
+    (dict(kv_dtype=5), _lib.TQ_ERR_INVALID_ARG), (dict(k_new=20), _lib.TQ_ERR_INVALID_ARG),
+    (dict(q=None), _lib.TQ_ERR_INVALID_ARG), (dict(d=64), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(max_ctx=65), _lib.TQ_ERR_INVALID_ARG), (dict(ws_bytes=100), _lib.TQ_ERR_WORKSPACE)])
+def test_decode_append_rejects_on_host(lib, kw, code):
+    fb = FakeBuffers()
+    a = dict(q=fb.p(0), dtype=1, k_new=fb.p(32768), v_new=fb.p(36864), kv_dtype=1, B=1, Hq=8, Hkv=2,
+             d=128, group=32, kp=fb.p(1024), ks=fb.p(2048), vp=fb.p(3072), vs=fb.p(4096), cap=64,
+             ctx=fb.p(512), max_ctx=64, signs=None, scale=0.125, out=fb.p(8192), ws=fb.p(16384),
+             ws_bytes=1 << 15, stream=None)
+    if kw.get("k_new") == 20:
+        kw = dict(k_new=fb.p(32788))
+    a.update(kw)
+    assert lib.tq_sdpa_int4_decode_append(
+        a["q"], a["dtype"], a["k_new"], a["v_new"], a["kv_dtype"], a["B"], a["Hq"], a["Hkv"], a["d"],
+        a["group"], a["kp"], a["ks"], a["vp"], a["vs"], a["cap"], a["ctx"], a["max_ctx"], a["signs"],
+        a["scale"], a["out"], a["ws"], a["ws_bytes"], a["stream"]) == code
+
+
 def test_workspace_size_is_exact_threshold(lib):
     fb = FakeBuffers()
     need = _lib.decode_workspace_bytes(1, 8, 2, 128, 64)

@@ -1,0 +1,81 @@
+"""tq_sdpa_int4_decode_append (one decode step in one call) against the two-call
+step it replaces: tq_quantize_append of the new token at row T_b - 1, then
+tq_sdpa_int4_decode.  The whole cache and the output must be bit-identical
+(same quantizer arithmetic, same decode kernels and plan), and the two-call
+step itself is checked against the oracle by the other GPU tests.  Covers the
+tensor-core decodes (the kernel quantizes the new tokens itself), the CUDA-core
+decode (small append launch first), clamped lengths and a one-token context."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressed_domain_attention_tq_b200 import _lib
+from conftest import require_cuda
+from helpers import THREADS, check_attention, oracle_cache, to_oracle, upload_cache
+
+pytestmark = pytest.mark.gpu
+
+
+def step_pair(B, Hkv, G, d, ctx, max_ctx, dtype=torch.bfloat16, seed=0, rot=True):
+    cap = max_ctx + 3
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(B, Hkv, cap, d, generator=g).to(dtype)
+    v = torch.randn(B, Hkv, cap, d, generator=g).to(dtype)
+    q = torch.randn(B, Hkv * G, d, generator=g).to(dtype)
+    k_new = torch.randn(B, Hkv, 1, d, generator=g).to(dtype)
+    v_new = torch.randn(B, Hkv, 1, d, generator=g).to(dtype)
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8) if rot else None
+    base = upload_cache(oracle_cache(k, v, signs))  # every row filled; row T_b - 1 gets replaced
+    dev = "cuda"
+    ctx_d = torch.tensor(ctx, dtype=torch.int32, device=dev)
+    sg = None if signs is None else signs.to(dev)
+    scale = 1 / math.sqrt(d)
+    ws = torch.empty(_lib.decode_workspace_bytes(B, Hkv * G, Hkv, d, max_ctx), dtype=torch.uint8, device=dev)
+    # two calls
+    c2 = [t.clone() for t in base]
+    pos = (torch.clamp(ctx_d, 1, max_ctx) - 1).to(torch.int32)
+    _lib.quantize_append(k_new.to(dev), v_new.to(dev), pos, sg, *c2)
+    out2 = torch.empty(B, Hkv * G, d, device=dev)
+    _lib.sdpa_int4_decode(q.to(dev), *c2, ctx_d, max_ctx, sg, scale, out2, ws)
+    torch.cuda.synchronize()
+    flags2 = ws[: 4 * B].view(torch.int32).cpu().numpy().copy()
+    # one call
+    c1 = [t.clone() for t in base]
+    out1 = torch.empty(B, Hkv * G, d, device=dev)
+    _lib.sdpa_int4_decode_append(q.to(dev), k_new.to(dev), v_new.to(dev), *c1, ctx_d, max_ctx, sg,
+                                 scale, out1, ws)
+    torch.cuda.synchronize()
+    flags1 = ws[: 4 * B].view(torch.int32).cpu().numpy().copy()
+    for a, b in zip(c1, c2):
+        assert torch.equal(a, b)
+    assert not torch.equal(c1[0], base[0])  # the new rows were written
+    np.testing.assert_array_equal(out1.cpu().numpy(), out2.cpu().numpy())
+    np.testing.assert_array_equal(flags1, flags2)
+    return c1, q, signs, out1, scale, flags1
+
+
+@pytest.mark.parametrize("d,G", [(128, 8), (128, 5), (128, 2), (256, 2), (256, 4), (128, 16), (256, 8)])
+def test_fused_step_matches_two_calls(d, G):
+    require_cuda()
+    step_pair(2, 2, G, d, [700, 1537], 1600, seed=d + G)
+
+
+def test_fused_step_one_token_and_clamped():
+    require_cuda()
+    c, q, signs, out, scale, flags = step_pair(3, 2, 8, 128, [1, 40, 999], 64, seed=5)
+    assert list(flags) == [0, 0, 1]
+
+
+def test_fused_step_vs_oracle_fp32_inputs():
+    """End to end against the oracle: fused step on fp32 inputs, rotation off
+    (codes bit-exact), then the oracle decodes the written cache."""
+    require_cuda()
+    B, Hkv, G, d = 1, 2, 8, 128
+    c, q, signs, out, scale, _ = step_pair(B, Hkv, G, d, [2049], 2100, dtype=torch.float32, seed=9,
+                                           rot=False)
+    cache = [t.cpu().numpy() for t in c]
+    want = oracle.sdpa_int4_decode(to_oracle(q), cache, [2049], None, scale, Hkv, threads=THREADS)
+    check_attention(out.cpu().numpy(), want, cache, [2049], G, "fused step")
