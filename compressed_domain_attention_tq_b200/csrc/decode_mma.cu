@@ -334,9 +334,16 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   const int G = a.Hq / a.Hkv;
   float* qs = reinterpret_cast<float*>(smem + C::QS);
   float* qexp = reinterpret_cast<float*>(smem + C::QEXP);
-  // Heads are prepared by warps 0 .. NW/2 - 1 (two heads each when NH == 8), so
-  // the last warp is free to issue the first copies meanwhile.
+  // Heads are prepared by warps 0 .. NW/2 - 1 (two heads each when NH == 8)
+  // while the last warp issues the first copies; with a fused append it first
+  // waits (named barrier 2, warps 4, 5 and NW - 1) for the new tokens' rows.
   constexpr int HPW = C::NH / (C::NW / 2) > 0 ? C::NH / (C::NW / 2) : 1;  // heads per warp
+  if (start_stream && threadIdx.x >= C::THREADS - 32) {
+    if (a.k_new != nullptr) asm volatile("bar.sync 2, 96;" ::: "memory");
+    if (threadIdx.x == C::THREADS - 32)
+      for (int s = 0; s < C::NS; ++s)
+        if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
+  }
   for (int hh = 0; hh < HPW; ++hh) {
     const int h = warp * HPW + hh;
     if (warp >= C::NW / 2 || h >= C::NH) break;
@@ -415,11 +422,6 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     }
   }
   barrier_all<C::THREADS>();
-  // The first item's query loads have landed; only now does the last warp
-  // start the stream, so those few loads do not queue behind it.
-  if (start_stream && threadIdx.x == C::THREADS - 32)
-    for (int s = 0; s < C::NS; ++s)
-      if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
   // Score A tiles in shared memory, f16 [group][k-step][row][k]: row r < 8 is
   // the hi part of head h(r), row 8 + r its lo part; MMA index k of k-step ks
   // is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in which
@@ -841,10 +843,11 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
 
   // Fused append: for every (sequence, kv head) whose last chunk is one of this
   // CTA's items, warps 4 and 5 quantize that kv head's new K and V token into
-  // row T - 1 (T the clamped context length) while the other warps prepare the
-  // first query.  Only that chunk reads the row, and this CTA issues no copy
-  // before the barrier that follows (in the first item's query preparation);
-  // the proxy fence orders these generic writes before the bulk copies.
+  // row T - 1 (T the clamped context length) while warps 0 .. 3 prepare the
+  // first query.  Only that chunk reads the row; the proxy fence orders these
+  // generic writes before the bulk copies, which the last warp issues only
+  // after named barrier 2 (both warps arrive here exactly once).
+  static_assert(C::NW == 8, "the fused append uses warps 4, 5 and 7");
   if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
     const bool isv = warp == 5;
     const int eb = a.kv_bf16 ? 2 : 4;
@@ -860,6 +863,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
                               const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
+    asm volatile("bar.arrive 2, 96;" ::: "memory");
   }
 
   const int gid = lane >> 2, tig = lane & 3;
