@@ -384,6 +384,226 @@ __global__ void __launch_bounds__(128) quantize_warp_kernel(QuantizeArgs a) {
                           (kv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
 }
 
+// d = 128 with bf16 inputs: two lanes per vector, 64 coordinates each (lane
+// 2v + sub holds coordinates 64 sub .. 64 sub + 63, groups 2 sub, 2 sub + 1).
+// Six butterfly stages run in registers and the seventh (coordinate bit 6)
+// across the lane pair, in the same order and with the same operations as the
+// other quantize kernels; half the registers per thread let 16 warps share an
+// SM.  A warp batch is 16 vectors (32 slices of 128 bytes at a 144-byte pitch).
+struct QHalf {
+  static constexpr int SLICE = 128;         // 64 bf16
+  static constexpr int PITCH = SLICE + 16;  // shared-memory slice pitch
+  static constexpr int BUF = 32 * PITCH;
+  static constexpr int WARPS = 16;
+  static constexpr int THREADS = 32 * WARPS;
+  static constexpr int MASKS = 2 * 32 * 4;  // bf16 pair masks of the two 64-slices
+  static constexpr int BYTES = MASKS + WARPS * 2 * BUF;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
+};
+
+template <bool ROT>
+__global__ void __launch_bounds__(QHalf::THREADS, 1) quantize_half_kernel(QuantizeArgs a) {
+  using Q = QHalf;
+  constexpr int D = 128, VPB = 16, VB = 256, CPL = 8;  // vectors / bytes per vector / copies per lane
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem);  // [2][32]: bit 15 / 31 = sign of 2k / 2k+1
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (ROT)
+    for (int i = threadIdx.x; i < 64; i += blockDim.x)
+      smask[i] = ((a.signs[2 * i] < 0) ? 0x00008000u : 0u) | ((a.signs[2 * i + 1] < 0) ? 0x80000000u : 0u);
+  __syncthreads();
+  unsigned char* buf = smem + Q::MASKS + warp * 2 * Q::BUF;
+  const int64_t per_kv = (int64_t)a.B * a.Hkv * a.n_new;
+  const int64_t nvec = 2 * per_kv;
+  const int64_t nbatch = (nvec + VPB - 1) / VPB;
+  const int64_t nw = (int64_t)gridDim.x * Q::WARPS;
+  const unsigned char* kin = static_cast<const unsigned char*>(a.k);
+  const unsigned char* vin = static_cast<const unsigned char*>(a.v);
+  const bool narrow = per_kv <= 0x7fffffffLL;
+
+  // batch bi -> padded slices of buffer dst; the byte offset of copy c is
+  // 512 c + 16 lane: vector 2c + lane / 16, slice 2 (that) + (lane % 16) / 8
+  auto issue = [&](int64_t bi, unsigned char* dst) {
+    const int64_t v0 = bi * VPB;
+    const int ov = 16 * (lane & 15);
+    unsigned char* d0 = dst + (2 * (lane >> 4) + ov / Q::SLICE) * Q::PITCH + ov % Q::SLICE;
+    if (v0 + VPB <= per_kv || (v0 >= per_kv && v0 + VPB <= nvec)) {
+      const unsigned char* src = (v0 < per_kv ? kin + v0 * VB : vin + (v0 - per_kv) * VB) + 16 * lane;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) cp_async16(d0 + 4 * c * Q::PITCH, src + 512 * c, 16u);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const int64_t v = v0 + 2 * c + (lane >> 4);
+        const bool ok = v < nvec;
+        const unsigned char* src = ok ? (v < per_kv ? kin + v * VB : vin + (v - per_kv) * VB) + ov : kin;
+        cp_async16(d0 + 4 * c * Q::PITCH, src, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  int64_t bi = (int64_t)blockIdx.x * Q::WARPS + warp;
+  if (bi < nbatch) issue(bi, buf);
+  const int sub = lane & 1;
+  for (int k = 0; bi < nbatch; ++k, bi += nw) {
+    const unsigned char* cur = buf + (k & 1) * Q::BUF;
+    if (bi + nw < nbatch) {
+      issue(bi + nw, buf + ((k + 1) & 1) * Q::BUF);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 w = reinterpret_cast<const uint4*>(cur + lane * Q::PITCH)[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t u = ws[kk];
+        if (ROT) u ^= smask[sub * 32 + c * 4 + kk];
+        x[c * 8 + 2 * kk] = __uint_as_float(u << 16);
+        x[c * 8 + 2 * kk + 1] = __uint_as_float(u & 0xFFFF0000u);
+      }
+    }
+    __syncwarp();  // the next iteration refills the other buffer, and this one after it
+
+    if (ROT) {
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float u = x[i], w = x[i + 1];
+        x[i] = u + w;
+        x[i + 1] = u - w;
+      }
+#pragma unroll
+      for (int bit = 2; bit < 64; bit <<= 1)
+#pragma unroll
+        for (int i = 0; i < 64; i += 2)
+          if ((i & bit) == 0) {
+            const float2 u = make_float2(x[i], x[i + 1]), w = make_float2(x[i | bit], x[(i | bit) + 1]);
+            const float2 s = __fadd2_rn(u, w), d = sub2(u, w);
+            x[i] = s.x;
+            x[i + 1] = s.y;
+            x[i | bit] = d.x;
+            x[(i | bit) + 1] = d.y;
+          }
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {  // coordinate bit 6, across the lane pair
+        const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
+        x[i] = sub ? other - x[i] : x[i] + other;
+      }
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float2 v = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(kInvSqrt128, kInvSqrt128));
+        x[i] = v.x;
+        x[i + 1] = v.y;
+      }
+    }
+    float scales[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      float* xg = x + 32 * g;
+      float m[11];
+#pragma unroll
+      for (int j = 0; j < 10; ++j) m[j] = fmax3(fabsf(xg[3 * j]), fabsf(xg[3 * j + 1]), fabsf(xg[3 * j + 2]));
+      m[10] = fmaxf(fabsf(xg[30]), fabsf(xg[31]));
+      const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]),
+                               fmax3(fmax3(m[6], m[7], m[8]), m[9], m[10]));
+      const float s = __fdiv_rn(amax, 7.0f);
+      scales[g] = s;
+      const float r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+      const bool big = !(r <= 3.0e38f);
+      const float2 rlo = make_float2(r * kBracketLo, r * kBracketLo);
+      const float2 rhi = make_float2(r * kBracketHi, r * kBracketHi);
+      const float2 magic = make_float2(kRneMagic, kRneMagic);
+      float code[32];
+      uint32_t diff = big ? 1u : 0u;
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 v = make_float2(xg[j], xg[j + 1]);
+        const float2 flo = __ffma2_rn(v, rlo, magic), fhi = __ffma2_rn(v, rhi, magic);
+        diff |= (__float_as_uint(flo.x) ^ __float_as_uint(fhi.x)) |
+                (__float_as_uint(flo.y) ^ __float_as_uint(fhi.y));
+        code[j] = flo.x;
+        code[j + 1] = flo.y;
+      }
+      if (diff) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float c = rintf(__fdiv_rn(xg[j], s));
+          c = fminf(fmaxf(c, -7.0f), 7.0f);
+          code[j] = kRneMagic + c;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) xg[j] = code[j];
+    }
+    // local word r: this lane's groups, in-group 4r .. 4r + 3 (group 0 in bits
+    // 0..15, group 1 in 16..31) = row word 2r + sub; nibbles by shift-adds on
+    // the magic-float bits (see quantize_slice)
+    constexpr uint32_t kBias = (0x4B400000u - 8u) * 0x11111111u;
+    uint32_t w[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      uint32_t acc = 0u;
+#pragma unroll
+      for (int kk = 7; kk >= 0; --kk) acc = (acc << 4) + __float_as_uint(x[32 * (kk / 4) + 4 * r + kk % 4]);
+      w[r] = (acc - kBias) ^ 0x88888888u;
+    }
+    // 16-byte chunk c = row words 4c .. 4c + 3 = [w0(2c), w1(2c), w0(2c+1), w1(2c+1)]
+    // (wS = lane S's local words); lane 0 writes chunks 0, 1 and lane 1 chunks 2, 3
+    uint32_t recv[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) recv[kk] = __shfl_xor_sync(0xffffffffu, sub ? w[kk] : w[4 + kk], 1);
+    const int64_t v = bi * VPB + (lane >> 1);
+    if (v < nvec) {
+      const bool kv = v >= per_kv;
+      const int64_t rem = kv ? v - per_kv : v;
+      int64_t bh, n;
+      if (narrow) {
+        const uint32_t r32 = (uint32_t)rem, bh32 = r32 / (uint32_t)a.n_new;
+        bh = bh32;
+        n = r32 - bh32 * (uint32_t)a.n_new;
+      } else {
+        bh = rem / a.n_new;
+        n = rem - bh * a.n_new;
+      }
+      const int b = (int)((uint32_t)bh / (uint32_t)a.Hkv);
+      const int64_t p = (int64_t)a.pos[b] + n;
+      if (p >= 0 && p < a.capacity) {
+        const int64_t row = bh * a.capacity + p;
+        uint4* dst = reinterpret_cast<uint4*>((kv ? a.v_packed : a.k_packed) + row * (D / 2) + 32 * sub);
+        if (sub == 0) {
+          dst[0] = make_uint4(w[0], recv[0], w[1], recv[1]);
+          dst[1] = make_uint4(w[2], recv[2], w[3], recv[3]);
+        } else {
+          dst[0] = make_uint4(recv[0], w[4], recv[1], w[5]);
+          dst[1] = make_uint4(recv[2], w[6], recv[3], w[7]);
+        }
+        *reinterpret_cast<float2*>((kv ? a.v_scales : a.k_scales) + row * 4 + 2 * sub) =
+            make_float2(scales[0], scales[1]);
+      }
+    }
+  }
+}
+
+template <bool ROT>
+cudaError_t launch_half(const QuantizeArgs& a, cudaStream_t stream) {
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(quantize_half_kernel<ROT>, QHalf::BYTES, smem_set);
+  if (e != cudaSuccess) return e;
+  const int64_t nbatch = (2LL * a.B * a.Hkv * a.n_new + 15) / 16;
+  int dev = 0, sms = kSmCount;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t blocks = (nbatch + QHalf::WARPS - 1) / QHalf::WARPS;
+  if (blocks > sms) blocks = sms;
+  quantize_half_kernel<ROT><<<(unsigned)blocks, QHalf::THREADS, QHalf::BYTES, stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D, bool BF16, bool ROT>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
   using Q = QCfg<BF16>;
@@ -412,7 +632,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   }
   const bool rot = a.signs != nullptr;
   if (a.d == 128) {
-    if (a.bf16) return rot ? launch_q<128, true, true>(a, stream) : launch_q<128, true, false>(a, stream);
+    if (a.bf16) return rot ? launch_half<true>(a, stream) : launch_half<false>(a, stream);
     return rot ? launch_q<128, false, true>(a, stream) : launch_q<128, false, false>(a, stream);
   }
   if (a.bf16) return rot ? launch_q<256, true, true>(a, stream) : launch_q<256, true, false>(a, stream);

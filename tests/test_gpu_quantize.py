@@ -68,7 +68,7 @@ def compare(gpu, ref, d, rot, label):
 @pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("rot", [False, True])
-@pytest.mark.parametrize("B,H,n", [(1, 1, 1), (2, 3, 33), (1, 8, 257), (3, 2, 1000)])
+@pytest.mark.parametrize("B,H,n", [(1, 1, 1), (2, 3, 33), (1, 8, 257), (3, 2, 1000), (1, 3, 2999)])
 def test_quantize_matches_oracle(d, dtype, rot, B, H, n):
     require_cuda()
     seed = d + n + B * 7 + (1 if rot else 0)
