@@ -489,10 +489,11 @@ __global__ void __launch_bounds__(QHalf::THREADS, 1) quantize_half_kernel(Quanti
             x[i | bit] = d.x;
             x[(i | bit) + 1] = d.y;
           }
+      const float sgn = sub ? -1.0f : 1.0f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {  // coordinate bit 6, across the lane pair
         const float other = __shfl_xor_sync(0xffffffffu, x[i], 1);
-        x[i] = sub ? other - x[i] : x[i] + other;
+        x[i] = fmaf(sgn, x[i], other);  // lane 0: u + w, lane 1: u - w (exact sign flip)
       }
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
