@@ -20,8 +20,8 @@ STATIC_SCRATCH_BYTES = 8 << 20   # TQ_STATIC_SCRATCH_BYTES in include/tq.h
 TQ_F32, TQ_BF16 = 0, 1
 
 SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
-           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_append", "tq_sdpa_int4_decode_static_scratch",
-           "tq_dequantize",
+           "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_append", "tq_sdpa_int4_decode_lse",
+           "tq_merge_lse", "tq_sdpa_int4_decode_static_scratch", "tq_dequantize",
            "tq_status_string")
 
 _lib = None
@@ -54,6 +54,11 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode_append.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P,
                                                i64, P, i32, P, f32, P, P, sz, P]
     lib.tq_sdpa_int4_decode_append.restype = i32
+    lib.tq_sdpa_int4_decode_lse.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64, P, i32,
+                                            P, f32, P, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_lse.restype = i32
+    lib.tq_merge_lse.argtypes = [P, P, i32, i32, i32, i32, P, P]
+    lib.tq_merge_lse.restype = i32
     lib.tq_sdpa_int4_decode_static_scratch.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P,
                                                        i64, P, i32, P, f32, P, P]
     lib.tq_sdpa_int4_decode_static_scratch.restype = i32
@@ -125,6 +130,30 @@ def sdpa_int4_decode(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ct
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode")
+
+
+def sdpa_int4_decode_lse(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs,
+                         attn_scale, out, lse, workspace, stream=None):
+    """sdpa_int4_decode that also writes lse[B][Hq][2] = (max in log2 units, sum) per head."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out, lse, workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_lse(_ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, _ptr(k_packed),
+                                        _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+                                        k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs),
+                                        float(attn_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_lse")
+
+
+def merge_lse(outs, lses, out, stream=None):
+    """out[B][Hq][d] from outs[R][B][Hq][d] and lses[R][B][Hq][2] over R disjoint context parts."""
+    _need_cuda(outs, lses, out)
+    R, B, Hq, d = outs.shape
+    rc = load().tq_merge_lse(_ptr(outs), _ptr(lses), R, B, Hq, d, _ptr(out), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_merge_lse")
 
 
 def sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,

@@ -109,6 +109,31 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
     o[i] = o[i] * sgn * rsqrtf((float)D);
   }
   a.out[((int64_t)b * a.Hq + hq) * D + i] = o[i];
+  if (a.lse != nullptr && i == 0)  // the head's softmax state, for merging across contexts
+    *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + hq) * 2) = make_float2(M, L);
+}
+
+// Outputs of several context parts of the same heads (each normalized, with
+// its (max, sum) in log2 units) -> the output over their union:
+//   M = max_r m_r,  w_r = 2^(m_r - M) l_r,  o = sum_r w_r o_r / sum_r w_r.
+__global__ void __launch_bounds__(256) merge_lse_kernel(const float* __restrict__ outs,
+                                                        const float* __restrict__ lses, int n_parts,
+                                                        int64_t n_heads, int d, float* __restrict__ out) {
+  const int64_t total = n_heads * d;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t h = idx / d;
+    float M = -INFINITY;
+    for (int r = 0; r < n_parts; ++r) M = fmaxf(M, lses[((int64_t)r * n_heads + h) * 2]);
+    float num = 0.0f, den = 0.0f;
+    for (int r = 0; r < n_parts; ++r) {
+      const float2 ml = *reinterpret_cast<const float2*>(lses + ((int64_t)r * n_heads + h) * 2);
+      const float w = exp2f(ml.x - M) * ml.y;  // NaN if a part is NaN
+      num = fmaf(w, outs[(int64_t)r * total + idx], num);
+      den += w;
+    }
+    out[idx] = num / den;
+  }
 }
 
 template <int D>
@@ -133,6 +158,15 @@ cudaError_t launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_merge_lse(const float* outs, const float* lses, int n_parts, int64_t n_heads,
+                             int d, float* out, cudaStream_t stream) {
+  const int64_t total = n_heads * d;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  merge_lse_kernel<<<(unsigned)blocks, 256, 0, stream>>>(outs, lses, n_parts, n_heads, d, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
   return a.d == 128 ? launch_merge_d<128>(a, stream) : launch_merge_d<256>(a, stream);

@@ -150,7 +150,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
                              float attn_scale, float* out, void* workspace, size_t workspace_bytes,
-                             void* cuda_stream, const char* where) {
+                             void* cuda_stream, const char* where, float* lse = nullptr) {
   if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
     return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
@@ -167,7 +167,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (num_q_heads / num_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(v_packed) ||
-      !aligned16(k_scales) || !aligned16(v_scales))
+      !aligned16(k_scales) || !aligned16(v_scales) || (lse && (reinterpret_cast<uintptr_t>(lse) & 7u)))
     return TQ_ERR_INVALID_ARG;
   DecodeArgs a;
   if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan))
@@ -194,6 +194,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   a.k_new = nullptr;
   a.v_new = nullptr;
   a.kv_bf16 = kv_dtype == TQ_BF16;
+  a.lse = lse;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const bool mma = decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
   if (append && mma) {  // the decode kernel quantizes the new tokens itself
@@ -238,6 +239,32 @@ tq_status tq_sdpa_int4_decode(const void* q, tq_dtype q_dtype, int32_t batch,
                      head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
                      max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
                      "tq_sdpa_int4_decode");
+}
+
+tq_status tq_sdpa_int4_decode_lse(const void* q, tq_dtype q_dtype, int32_t batch,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t group, const uint8_t* k_packed, const float* k_scales,
+                                  const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                                  const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                                  float attn_scale, float* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* cuda_stream) {
+  if (!lse) return TQ_ERR_INVALID_ARG;
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode_lse", lse);
+}
+
+tq_status tq_merge_lse(const float* outs, const float* lses, int32_t n_parts, int32_t batch,
+                       int32_t num_q_heads, int32_t head_dim, float* out, void* cuda_stream) {
+  if (!outs || !lses || !out) return TQ_ERR_INVALID_ARG;
+  if (n_parts < 1 || batch < 1 || num_q_heads < 1 || head_dim < 1) return TQ_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(lses) & 7u) || !aligned16(outs) || !aligned16(out))
+    return TQ_ERR_INVALID_ARG;
+  return cuda_status(launch_merge_lse(outs, lses, n_parts, (int64_t)batch * num_q_heads, head_dim,
+                                      out, static_cast<cudaStream_t>(cuda_stream)),
+                     "tq_merge_lse");
 }
 
 tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,

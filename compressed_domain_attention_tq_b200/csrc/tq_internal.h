@@ -67,6 +67,7 @@ struct DecodeArgs {
   const void* k_new;  // fused append (decode_mma only): [B][Hkv][1][d] new K and V, or NULL
   const void* v_new;
   int kv_bf16;
+  float* lse;  // NULL, or [B][Hq][2]: each head's (max in log2 units, sum) for merging contexts
 };
 
 // Raise a kernel's dynamic shared memory limit once per device (the first
@@ -91,5 +92,7 @@ bool decode_mma_supported(int d, int G);
 int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_merge_lse(const float* outs, const float* lses, int n_parts, int64_t n_heads,
+                             int d, float* out, cudaStream_t stream);
 
 }  // namespace tq

@@ -189,6 +189,41 @@ TQ_API tq_status tq_sdpa_int4_decode_append(
     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * tq_sdpa_int4_decode_lse -- tq_sdpa_int4_decode that also returns each head's
+ * softmax state, so that outputs over disjoint parts of a context (for
+ * instance the token shards of several GPUs) can be combined exactly with
+ * tq_merge_lse.  The pages do not describe this step: it is split-K
+ * flash-decoding's log-sum-exp merge taken across calls.
+ *
+ *  lse   float [B][Hq][2], 8-byte aligned: (M, L) per head, M the maximum of
+ *        attn_scale * q.k over the attended tokens in log2 units and
+ *        L = sum_t 2^(attn_scale * q.k_t * log2(e) - M), so that the head's
+ *        output is sum_t 2^(... - M) v_t / L.
+ * Every other argument and error is that of tq_sdpa_int4_decode;
+ * TQ_ERR_INVALID_ARG also for a NULL or misaligned lse.
+ */
+TQ_API tq_status tq_sdpa_int4_decode_lse(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, const uint8_t* k_packed, const float* k_scales,
+    const uint8_t* v_packed, const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out, float* lse,
+    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * tq_merge_lse -- combine n_parts outputs of tq_sdpa_int4_decode_lse over
+ * disjoint parts of the same sequences' contexts into the output over their
+ * union: M = max_r M_r, w_r = 2^(M_r - M) L_r, out = sum_r w_r out_r / sum_r w_r.
+ *
+ *  outs  float [n_parts][B][Hq][d] (16-byte aligned), lses float
+ *        [n_parts][B][Hq][2] (8-byte aligned), out float [B][Hq][d]
+ *        (16-byte aligned; may not alias outs).
+ * Returns TQ_ERR_INVALID_ARG for NULL or misaligned pointers or sizes < 1,
+ * TQ_ERR_UNSUPPORTED for head_dim not in {128, 256}.
+ */
+TQ_API tq_status tq_merge_lse(const float* outs, const float* lses, int32_t n_parts, int32_t batch,
+                              int32_t num_q_heads, int32_t head_dim, float* out, void* cuda_stream);
+
+/*
  * tq_sdpa_int4_decode_static_scratch -- tq_sdpa_int4_decode without a
  * caller-provided workspace.  The method's pages have no counterpart to this
  * call; it exists for callers that cannot allocate device memory: a plug-in

@@ -181,6 +181,20 @@ def test_decode_append_rejects_on_host(lib, kw, code):
         a["scale"], a["out"], a["ws"], a["ws_bytes"], a["stream"]) == code
 
 
+def test_lse_calls_reject_on_host(lib):
+    fb = FakeBuffers()
+    # merge: NULL, sizes, head_dim, misaligned
+    assert lib.tq_merge_lse(None, fb.p(0), 2, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_merge_lse(fb.p(0), fb.p(2048), 0, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_merge_lse(fb.p(0), fb.p(2048), 2, 1, 8, 64, fb.p(4096), None) == _lib.TQ_ERR_UNSUPPORTED
+    assert lib.tq_merge_lse(fb.p(0), fb.p(2052), 2, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
+    # decode_lse: NULL lse, misaligned lse
+    for lse in (None, fb.p(20484)):
+        assert lib.tq_sdpa_int4_decode_lse(fb.p(0), 1, 1, 8, 2, 128, 32, fb.p(1024), fb.p(2048),
+                                           fb.p(3072), fb.p(4096), 64, fb.p(512), 64, None, 0.125,
+                                           fb.p(8192), lse, fb.p(16384), 1 << 15, None) == _lib.TQ_ERR_INVALID_ARG
+
+
 def test_workspace_size_is_exact_threshold(lib):
     fb = FakeBuffers()
     need = _lib.decode_workspace_bytes(1, 8, 2, 128, 64)
