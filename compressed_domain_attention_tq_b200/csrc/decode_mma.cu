@@ -209,6 +209,10 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) 
 
 // ------------------------------------------------------------ configuration
 
+// Batches up to this size use the list of non-empty items (its prefix sums
+// live in shared memory); larger ones walk every (sequence, kv head, chunk).
+constexpr int kMaxListB = 1024;
+
 template <int D, int PATH>
 struct Cfg {
   static constexpr int NW = 8;                  // warps per CTA (all consumers)
@@ -239,7 +243,8 @@ struct Cfg {
   static constexpr int MW = al(ML + 4 * NW * NH);            // float [NW][NH] weight
   static constexpr int MTOT = al(MW + 4 * NW * NH);          // float [NH] max, [NH] sum
   static constexpr int ABORT = al(MTOT + 4 * 2 * NH);        // int
-  static constexpr int BYTES = ABORT + 16;
+  static constexpr int PFX = al(ABORT + 16);                 // int [kMaxListB + 1] item prefix
+  static constexpr int BYTES = PFX + 4 * (kMaxListB + 1);
   static_assert(BYTES <= 227 * 1024, "shared memory");
   static_assert(STAGE % 16 == 0 && VC % 16 == 0 && KS % 16 == 0 && VS % 16 == 0, "alignment");
 };
@@ -254,9 +259,30 @@ __device__ __forceinline__ int clamp_ctx_mma(int T, int max_ctx) {
 }
 
 // Item it -> (sequence b, kv head, chunk c) and its token range [t0, t1).
-// Returns false for an item past the end of its sequence.
-__device__ __forceinline__ bool item_range(const DecodeArgs& a, int it, int& b, int& kvh, int& c,
-                                           int& t0, int& t1) {
+// With the item list (pfx != nullptr) the items are only the chunks that hold
+// tokens, sequence by sequence (pfx[b] = items of the sequences before b), so
+// that CTAs taking every gridDim.x-th item get equal shares even when the
+// sequences' lengths differ; otherwise every chunk of the max_ctx plan is an
+// item and those past a sequence's end return false.
+__device__ __forceinline__ bool item_range(const DecodeArgs& a, const int* pfx, int it, int& b,
+                                           int& kvh, int& c, int& t0, int& t1) {
+  if (pfx != nullptr) {
+    int lo = 0, hi = a.B;  // pfx[0] = 0 <= it < pfx[B]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pfx[mid] <= it) lo = mid;
+      else hi = mid;
+    }
+    b = lo;
+    const int T = clamp_ctx_mma(a.ctx_lens[b], a.max_ctx);
+    const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
+    const int r = it - pfx[b];
+    kvh = r / nc;
+    c = r % nc;
+    t0 = c * a.plan.chunk;
+    t1 = min(T, t0 + a.plan.chunk);
+    return true;
+  }
   const int nc = a.plan.n_chunks;
   c = it % nc;
   const int bh = it / nc;
@@ -270,12 +296,16 @@ __device__ __forceinline__ bool item_range(const DecodeArgs& a, int it, int& b, 
 
 // Refill cursor (shared memory, used by one thread at a time): cur[0] item,
 // cur[1] next token, cur[2] end token, cur[3] sequence, cur[4] kv head,
-// cur[5] stages issued.  Issues the next stage of this CTA's stage sequence
+// cur[5] stages issued; cur[6] items in the call, cur[7] 1 if the item list
+// in smem + PFX is used (both set once at kernel start and only read after).
+// Issues the next stage of this CTA's stage sequence
 // into `slot`; returns false when the sequence is exhausted.
 template <int D, int PATH>
 __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* smem, int* cur,
-                                           uint64_t* full, int n_items, int slot) {
+                                           uint64_t* full, int slot) {
   using C = Cfg<D, PATH>;
+  const int n_items = cur[6];
+  const int* pfx = cur[7] ? reinterpret_cast<const int*>(smem + C::PFX) : nullptr;
   int it = cur[0], t = cur[1], t1 = cur[2];
   int b = cur[3], kvh = cur[4];
   while (t >= t1) {
@@ -285,7 +315,7 @@ __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* s
       return false;
     }
     int c, t0;
-    item_range(a, it, b, kvh, c, t0, t1);
+    item_range(a, pfx, it, b, kvh, c, t0, t1);
     t = t0;
   }
   const int n = min(C::ST, t1 - t);
@@ -327,7 +357,7 @@ struct WarpState {
 template <int D, int PATH>
 __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, unsigned char* smem,
                                            WarpState<D, PATH>& st, bool start_stream,
-                                           int* cur, uint64_t* full, int n_items) {
+                                           int* cur, uint64_t* full) {
   using C = Cfg<D, PATH>;
   constexpr int E = D / 32;  // elements per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -342,7 +372,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     if (a.k_new != nullptr) asm volatile("bar.sync 2, 96;" ::: "memory");
     if (threadIdx.x == C::THREADS - 32)
       for (int s = 0; s < C::NS; ++s)
-        if (!issue_next<D, PATH>(a, smem, cur, full, n_items, s)) break;
+        if (!issue_next<D, PATH>(a, smem, cur, full, s)) break;
   }
   for (int hh = 0; hh < HPW; ++hh) {
     const int h = warp * HPW + hh;
@@ -826,7 +856,6 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   int* cur = reinterpret_cast<int*>(smem + C::CUR);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::ABORT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(full + s, 1);
@@ -839,6 +868,43 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   }
   // the merge kernel may be scheduled now; it waits for this grid's writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // The item list: pfx[b + 1] = Hkv * (chunks of sequence b), then an
+  // inclusive scan by warp 0.
+  // (Built only when some sequence has fewer chunks than the plan; otherwise
+  // the list is the plain enumeration and no scan is needed.)
+  int* pfx = reinterpret_cast<int*>(smem + C::PFX);
+  bool shorter = false;
+  if (a.B <= kMaxListB) {
+    for (int b = threadIdx.x; b < a.B; b += C::THREADS) {
+      const int T = clamp_ctx_mma(a.ctx_lens[b], a.max_ctx);
+      const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
+      pfx[b + 1] = a.Hkv * nc;
+      shorter |= nc < a.plan.n_chunks;
+    }
+    if (threadIdx.x == 0) pfx[0] = 0;
+  }
+  if (!__syncthreads_or(shorter)) pfx = nullptr;
+  if (pfx != nullptr) {
+    if (warp == 0) {
+      int carry = 0;
+      for (int base = 1; base <= a.B; base += 32) {
+        const int i = base + lane;
+        int v = i <= a.B ? pfx[i] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, v, o);
+          if (lane >= o) v += y;
+        }
+        if (i <= a.B) pfx[i] = v + carry;
+        carry += __shfl_sync(kFull, v, 31);
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    cur[6] = pfx != nullptr ? pfx[a.B] : a.B * a.Hkv * a.plan.n_chunks;
+    cur[7] = pfx != nullptr;
+  }
   __syncthreads();
 
   // Fused append: for every (sequence, kv head) whose last chunk is one of this
@@ -851,9 +917,9 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
     const bool isv = warp == 5;
     const int eb = a.kv_bf16 ? 2 : 4;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    for (int it = blockIdx.x; it < cur[6]; it += gridDim.x) {
       int b, kvh, c, t0, t1;
-      if (!item_range(a, it, b, kvh, c, t0, t1)) continue;
+      if (!item_range(a, pfx, it, b, kvh, c, t0, t1)) continue;
       if (t1 != clamp_ctx_mma(a.ctx_lens[b], a.max_ctx)) continue;  // not the last chunk
       const int64_t bh = (int64_t)b * a.Hkv + kvh;
       const int64_t row = bh * a.capacity + (t1 - 1);
@@ -872,14 +938,16 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   const int krow[2] = {slot_row(gid), 8 + slot_row(gid)};
   WarpState<D, PATH> st;
   uint32_t sc = 0;  // stages consumed so far
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+  for (int it = blockIdx.x; it < cur[6]; it += gridDim.x) {
     int b, kvh, c, t0, t1;
-    if (!item_range(a, it, b, kvh, c, t0, t1)) continue;
+    if (!item_range(a, cur[7] ? reinterpret_cast<const int*>(smem + C::PFX) : nullptr, it, b, kvh,
+                    c, t0, t1))
+      continue;
     if (threadIdx.x == 0 && kvh == 0 && c == 0) {
       const int raw = a.ctx_lens[b];
       static_cast<int32_t*>(a.workspace)[b] = (raw < 1 || raw > a.max_ctx) ? 1 : 0;
     }
-    prep_query<D, PATH>(a, b, kvh, smem, st, sc == 0, cur, full, n_items);
+    prep_query<D, PATH>(a, b, kvh, smem, st, sc == 0, cur, full);
 #pragma unroll
     for (int j = 0; j < C::NACC; ++j)
 #pragma unroll
@@ -905,7 +973,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
         if (atomicAdd(cnt + slot, 1) == C::NW - 1) {
           cnt[slot] = 0;
           __threadfence_block();
-          if (!*abort) issue_next<D, PATH>(a, smem, cur, full, n_items, slot);
+          if (!*abort) issue_next<D, PATH>(a, smem, cur, full, slot);
         }
       }
     }
