@@ -10,9 +10,10 @@
 // cache; the query was rotated by the cache's signs, so V's output is rotated
 // back.)
 //
-// One CTA of d threads per (sequence, query head).  The kernel is launched
-// with programmatic stream serialization: it may start while the split-K
-// kernel drains and waits at griddepcontrol.wait before reading partials.
+// One CTA of d threads (thread i: output coordinate i) per (sequence, query
+// head), launched with programmatic stream serialization: it may start while
+// the split-K kernel drains and waits at griddepcontrol.wait before reading
+// partials.
 #include <math.h>
 
 #include "tq_internal.h"
@@ -20,95 +21,76 @@
 namespace tq {
 namespace {
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = red[0];
-  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
-  __syncthreads();
-  return r;
-}
-
-__device__ __forceinline__ float block_sum(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = red[0];
-  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r += red[w];
-  __syncthreads();
-  return r;
-}
-
 template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
-  extern __shared__ float ml_s[];  // [n_chunks] chunk max, then weight; [n_chunks] chunk sum
-  __shared__ float o[D];
-  __shared__ float red[8];
+__global__ void __launch_bounds__(D) merge_kernel(DecodeArgs a) {
+  __shared__ float o[D];  // cross-warp butterfly stages
   const int b = blockIdx.x / a.Hq;
   const int hq = blockIdx.x % a.Hq;
-  const int i = threadIdx.x;
+  const int i = threadIdx.x, lane = i & 31;
   // inputs the split-K kernel does not write are read before waiting for it
   const int raw = a.ctx_lens[b];
   const float sgn = a.signs ? (float)a.signs[i] : 1.0f;
   const int T = raw < 1 ? 1 : (raw > a.max_ctx ? a.max_ctx : raw);
   const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
   const int stride = a.plan.part_stride;
-  float* w_s = ml_s;
-  float* l_s = ml_s + a.plan.n_chunks;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* part = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
                                                      a.plan.header_bytes) +
                       ((int64_t)b * a.Hq + hq) * a.plan.n_chunks * stride;
 
-  float mloc = -INFINITY;
-  for (int c = i; c < nc; c += D) {  // (m, l) of chunk c
-    const float2 ml = *reinterpret_cast<const float2*>(part + (int64_t)c * stride + D);
-    w_s[c] = ml.x;
-    l_s[c] = ml.y;
-    mloc = fmaxf(mloc, ml.x);
-  }
-  const float M = block_max(mloc, red);  // its barriers also publish w_s, l_s
-  float lloc = 0.0f;
-  for (int c = i; c < nc; c += D) {
-    const float w = exp2f(w_s[c] - M);  // NaN if a partial is NaN
-    lloc = fmaf(w, l_s[c], lloc);
-    w_s[c] = w;
-  }
-  const float L = block_sum(lloc, red);  // ends with __syncthreads: weights visible
-
-  constexpr int U = 16;  // chunk loads in flight per thread
-  float acc[U];
+  // Every thread reads the chunks' (m, l) itself (the same addresses across the
+  // block: broadcast loads), so no block-wide reductions are needed.
+  float M = -INFINITY;
+  for (int c = 0; c < nc; ++c) M = fmaxf(M, part[(int64_t)c * stride + D]);
+  constexpr int U = 8;  // chunks in flight per thread
+  float acc[U], lsum[U];
 #pragma unroll
-  for (int k = 0; k < U; ++k) acc[k] = 0.0f;
+  for (int k = 0; k < U; ++k) acc[k] = lsum[k] = 0.0f;
   for (int c0 = 0; c0 < nc; c0 += U) {
+    float2 ml[U];
     float v[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k) v[k] = c0 + k < nc ? part[(int64_t)(c0 + k) * stride + i] : 0.0f;
+    for (int k = 0; k < U; ++k) {
+      const bool ok = c0 + k < nc;
+      const float* pc = part + (int64_t)(c0 + k) * stride;
+      ml[k] = ok ? *reinterpret_cast<const float2*>(pc + D) : make_float2(-INFINITY, 0.0f);
+      v[k] = ok ? pc[i] : 0.0f;
+    }
 #pragma unroll
     for (int k = 0; k < U; ++k)
-      if (c0 + k < nc) acc[k] = fmaf(w_s[c0 + k], v[k], acc[k]);
+      if (c0 + k < nc) {
+        const float w = exp2f(ml[k].x - M);  // NaN if a partial is NaN
+        lsum[k] = fmaf(w, ml[k].y, lsum[k]);
+        acc[k] = fmaf(w, v[k], acc[k]);
+      }
   }
 #pragma unroll
   for (int k = U / 2; k > 0; k >>= 1)
 #pragma unroll
-    for (int j = 0; j < k; ++j) acc[j] += acc[j + k];
-  o[i] = acc[0] / L;
-
-  if (a.signs) {  // o = diag(signs) H o / sqrt(d), H in Sylvester order
-    __syncthreads();
-    for (int bit = 1; bit < D; bit <<= 1) {  // each pair is owned by one thread per stage
-      if (i < D / 2) {
-        const int lo = ((i & ~(bit - 1)) << 1) | (i & (bit - 1));
-        const float u = o[lo], w = o[lo | bit];
-        o[lo] = u + w;
-        o[lo | bit] = u - w;
-      }
-      __syncthreads();
+    for (int j = 0; j < k; ++j) {
+      acc[j] += acc[j + k];
+      lsum[j] += lsum[j + k];
     }
-    o[i] = o[i] * sgn * rsqrtf((float)D);
+  const float L = lsum[0];
+  float x = acc[0] / L;
+
+  if (a.signs) {  // o = diag(signs) H o / sqrt(d), H in Sylvester order, bits 1, 2, 4, ...
+#pragma unroll
+    for (int bit = 1; bit < 32; bit <<= 1) {  // coordinate bits within the warp
+      const float other = __shfl_xor_sync(0xffffffffu, x, bit);
+      x = (lane & bit) ? other - x : x + other;
+    }
+#pragma unroll
+    for (int bit = 32; bit < D; bit <<= 1) {  // across warps
+      o[i] = x;
+      __syncthreads();
+      const float other = o[i ^ bit];
+      __syncthreads();
+      x = (i & bit) ? other - x : x + other;
+    }
+    x = x * sgn * rsqrtf((float)D);
   }
-  a.out[((int64_t)b * a.Hq + hq) * D + i] = o[i];
+  a.out[((int64_t)b * a.Hq + hq) * D + i] = x;
   if (a.lse != nullptr && i == 0)  // the head's softmax state, for merging across contexts
     *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + hq) * 2) = make_float2(M, L);
 }
@@ -141,19 +123,13 @@ cudaError_t launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * a.Hq);
   cfg.blockDim = dim3(D);
-  cfg.dynamicSmemBytes = 2 * sizeof(float) * (size_t)a.plan.n_chunks;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cfg.dynamicSmemBytes > 48 * 1024) {
-    static std::atomic<uint64_t> smem_set{0};
-    const cudaError_t e = ensure_smem_limit(merge_kernel<D>, 64 * 1024, smem_set);
-    if (e != cudaSuccess) return e;
-    if (cfg.dynamicSmemBytes > 64 * 1024) return cudaErrorInvalidValue;
-  }
   return cudaLaunchKernelEx(&cfg, merge_kernel<D>, a);
 }
 
