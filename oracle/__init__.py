@@ -15,7 +15,8 @@ Every function here is pinned by ``tests/test_oracle_pins.py`` against facts
 the pages or mathematics fix (Sylvester recursion, orthogonality, the
 quantizer's half-step bound, exact recovery on the int4 grid, round-half-even
 ties, hand-derived byte layouts, closed-form attention cases and brute-force
-softmax on tiny inputs).
+softmax on tiny inputs; the SRFT variant against numpy's FFT, the Hartley
+transform's involution and attention over a cache built exactly on the grid).
 """
 from __future__ import annotations
 
@@ -75,6 +76,16 @@ def _load():
     lib.oracle_exact_attention.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i64, P, f64,
                                            P, i32]
     lib.oracle_exact_attention.restype = i32
+    lib.oracle_dht_entry.argtypes = [i32, i32, i32]
+    lib.oracle_dht_entry.restype = f64
+    lib.oracle_srft_matrix.argtypes = [i32, P, P, P]
+    lib.oracle_srft_matrix.restype = i32
+    lib.oracle_quantize_append_srft.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P,
+                                                P, P, i64, i32]
+    lib.oracle_quantize_append_srft.restype = i32
+    lib.oracle_sdpa_int4_decode_srft.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, i64, P,
+                                                 P, P, P, f64, P, i32]
+    lib.oracle_sdpa_int4_decode_srft.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     _lib = lib
@@ -130,6 +141,41 @@ def rotate(x: np.ndarray, signs=None) -> np.ndarray:
     lib = _load()
     for r in range(n):
         lib.oracle_rotate_vector(d, _ptr(R), _ptr(x[r]), _ptr(y[r]))
+    return y
+
+
+def _lambda_array(lam, d):
+    if lam is None:
+        return None
+    a = np.ascontiguousarray(lam, dtype=np.float32)
+    if a.shape != (d,) or not np.all(np.isfinite(a)) or not np.all(a > 0):
+        raise ValueError("lambda must be d positive finite float32 values")
+    return a
+
+
+def dht_entry(d: int, k: int, j: int) -> float:
+    """Orthonormal discrete Hartley transform entry cas(2 pi k j / d) / sqrt(d)."""
+    return float(_load().oracle_dht_entry(d, k, j))
+
+
+def srft_matrix(d: int, signs=None, lam=None) -> np.ndarray:
+    """Store map of the SRFT variant: A = diag(lam) F_d diag(signs), fp64 (d, d)."""
+    A = np.empty((d, d), dtype=np.float64)
+    if _load().oracle_srft_matrix(d, _ptr(_signs_array(signs)), _ptr(_lambda_array(lam, d)),
+                                  _ptr(A)) != 0:
+        raise ValueError("d must be positive")
+    return A
+
+
+def srft_rotate(x: np.ndarray, signs=None, lam=None) -> np.ndarray:
+    """fl32(A x) for each row of x (float32, (n, d)), A the SRFT store map."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, d = x.shape
+    A = srft_matrix(d, signs, lam)
+    y = np.empty_like(x)
+    lib = _load()
+    for r in range(n):
+        lib.oracle_rotate_vector(d, _ptr(A), _ptr(x[r]), _ptr(y[r]))
     return y
 
 
@@ -196,6 +242,46 @@ def quantize_append(k, v, pos, signs, cache, threads: int = 1) -> None:
                                         threads)
     if rc != 0:
         raise ValueError(f"oracle_quantize_append failed ({rc})")
+
+
+def quantize_append_srft(k, v, pos, signs, lambda_k, lambda_v, cache, threads: int = 1) -> None:
+    """SRFT variant of quantize_append: stored rows are fl32(lambda (.) F (signs (.) x))."""
+    k, dt = _input_array(k)
+    v, dt2 = _input_array(v)
+    if dt != dt2 or k.shape != v.shape:
+        raise ValueError("k and v must share dtype and shape")
+    B, Hkv, n_new, d = k.shape
+    kp, ks, vp, vs = cache
+    cap = kp.shape[2]
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    s = _signs_array(signs)
+    lk, lv = _lambda_array(lambda_k, d), _lambda_array(lambda_v, d)
+    rc = _load().oracle_quantize_append_srft(_ptr(k), _ptr(v), dt, B, Hkv, n_new, d, _ptr(pos),
+                                             _ptr(s), _ptr(lk), _ptr(lv), _ptr(kp), _ptr(ks),
+                                             _ptr(vp), _ptr(vs), cap, threads)
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_append_srft failed ({rc})")
+
+
+def sdpa_int4_decode_srft(q, cache, ctx_lens, signs, lambda_k, lambda_v, attn_scale: float,
+                          num_kv_heads: int, threads: int = 1) -> np.ndarray:
+    """SRFT variant of sdpa_int4_decode: q_r = F (signs (.) q) / lambda_k,
+    o = signs (.) F (o_r / lambda_v); returns (B, Hq, d) fp64."""
+    q, qdt = _input_array(q)
+    B, Hq, d = q.shape
+    kp, ks, vp, vs = [np.ascontiguousarray(a) for a in cache]
+    cap = kp.shape[2]
+    ctx = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+    s = _signs_array(signs)
+    lk, lv = _lambda_array(lambda_k, d), _lambda_array(lambda_v, d)
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    rc = _load().oracle_sdpa_int4_decode_srft(_ptr(q), qdt, B, Hq, num_kv_heads, d, _ptr(kp),
+                                              _ptr(ks), _ptr(vp), _ptr(vs), cap, _ptr(ctx),
+                                              _ptr(s), _ptr(lk), _ptr(lv), float(attn_scale),
+                                              _ptr(out), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_sdpa_int4_decode_srft failed ({rc})")
+    return out
 
 
 def sdpa_int4_decode(q, cache, ctx_lens, signs, attn_scale: float, num_kv_heads: int,

@@ -36,6 +36,14 @@
  *    codes 0.
  *  - attention output = exact softmax attention over the dequantized values
  *    s*c in the rotated basis, mapped back with R^T, all in fp64.
+ *  - SRFT variant ([SRFT], core method: a sign-randomized Fourier transform
+ *    instead of the Hadamard one, usable at widths that are not powers of
+ *    two, followed by a per-coordinate scale lambda): the transform is the
+ *    orthonormal discrete Hartley transform F[k][j] = cas(2 pi k j / d) /
+ *    sqrt(d), cas = cos + sin (real, symmetric, F F = I).  The stored vector
+ *    is y = fl32(lambda (.) F (sigma (.) x)); K and V have their own lambda.
+ *    Scores use q_r = F (sigma (.) q) / lambda_K, so q_r . y_k = q . k; the
+ *    output is sigma (.) F (o_r / lambda_V).
  *
  * Build: gcc -O2 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC.
  */
@@ -101,6 +109,47 @@ void oracle_rotate_vector(int d, const double* R, const float* x, float* y) {
     for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * (double)x[j];
     y[i] = (float)acc;
   }
+}
+
+/* ------------------------------------------------------------------ */
+/* SRFT rotation ([SRFT] core method: sign-randomized Fourier transform, */
+/* any width, then a per-coordinate scale lambda)                        */
+/* ------------------------------------------------------------------ */
+
+/* Orthonormal discrete Hartley transform entry F_d[k][j] = cas(2 pi k j / d) / sqrt(d);
+   the product k j is reduced mod d first so the angle is computed exactly. */
+double oracle_dht_entry(int d, int k, int j) {
+  int64_t t = ((int64_t)k * (int64_t)j) % d;
+  double th = 2.0 * acos(-1.0) * (double)t / (double)d;
+  return (cos(th) + sin(th)) / sqrt((double)d);
+}
+
+/* Store map A[k*d + j] = lambda[k] * F_d[k][j] * sigma[j] (y = A x); lambda NULL = ones,
+   signs NULL = ones.  Any d >= 1. */
+int oracle_srft_matrix(int d, const int8_t* signs, const float* lambda, double* A) {
+  if (d <= 0 || !A) return -1;
+  for (int k = 0; k < d; ++k)
+    for (int j = 0; j < d; ++j) {
+      double v = oracle_dht_entry(d, k, j);
+      if (signs) v *= (double)signs[j];
+      if (lambda) v *= (double)lambda[k];
+      A[(int64_t)k * d + j] = v;
+    }
+  return 0;
+}
+
+/* Query map Q[k*d + j] = F_d[k][j] * sigma[j] / lambda_k[k] (q_r = Q q) and output map
+   O[j*d + k] = sigma[j] * F_d[j][k] / lambda_v[k] (o = O o_r). */
+static void srft_query_output_maps(int d, const int8_t* signs, const float* lambda_k,
+                                   const float* lambda_v, double* Q, double* O) {
+  for (int k = 0; k < d; ++k)
+    for (int j = 0; j < d; ++j) {
+      double f = oracle_dht_entry(d, k, j);
+      double sj = signs ? (double)signs[j] : 1.0;
+      Q[(int64_t)k * d + j] = f * sj / (lambda_k ? (double)lambda_k[k] : 1.0);
+      /* F is symmetric: F[j][k] = F[k][j] */
+      O[(int64_t)j * d + k] = sj * f / (lambda_v ? (double)lambda_v[k] : 1.0);
+    }
 }
 
 /* ------------------------------------------------------------------ */
@@ -178,16 +227,12 @@ void oracle_unpack_vector(int d, const uint8_t* packed, int8_t* codes) {
  * Token n of (b, h) goes to cache row pos[b] + n of that (b, h) slot.
  * caches: packed [B][Hkv][capacity][d/2], scales [B][Hkv][capacity][d/32].
  */
-int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, int Hkv,
-                           int n_new, int d, const int32_t* pos, const int8_t* signs,
-                           uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
-                           float* v_scales, int64_t capacity, int nthreads) {
-  if (d % ORACLE_GROUP != 0 || (d & (d - 1)) != 0) return -1;
-  for (int b = 0; b < B; ++b)
-    if (pos[b] < 0 || (int64_t)pos[b] + n_new > capacity) return -1;
-  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
-  if (!R) return -2;
-  oracle_rotation_matrix(d, signs, R);
+/* The store maps Ak, Av (d x d, y = fl32(A x)) or NULL for y = x. */
+static int quantize_append_maps(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                                int n_new, int d, const int32_t* pos, const double* Ak,
+                                const double* Av, uint8_t* k_packed, float* k_scales,
+                                uint8_t* v_packed, float* v_scales, int64_t capacity,
+                                int nthreads) {
   int ng = d / ORACLE_GROUP;
   int64_t nvec = (int64_t)B * Hkv * n_new;
 #ifdef _OPENMP
@@ -203,8 +248,9 @@ int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, in
     int64_t row = ((int64_t)b * Hkv + h) * capacity + pos[b] + n;
     for (int kv = 0; kv < 2; ++kv) {
       const void* src = kv ? v : k;
+      const double* A = kv ? Av : Ak;
       for (int i = 0; i < d; ++i) x[i] = load_input(src, in_dtype, idx * d + i);
-      if (signs) oracle_rotate_vector(d, R, x, y);
+      if (A) oracle_rotate_vector(d, A, x, y);
       else memcpy(y, x, sizeof(float) * (size_t)d);
       float* sc = (kv ? v_scales : k_scales) + row * ng;
       uint8_t* pk = (kv ? v_packed : k_packed) + row * (d / 2);
@@ -212,8 +258,53 @@ int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, in
       oracle_pack_vector(d, codes, pk);
     }
   }
-  free(R);
   return 0;
+}
+
+static int check_append(int B, int n_new, int d, const int32_t* pos, int64_t capacity) {
+  if (d % ORACLE_GROUP != 0 || d > 512) return -1;
+  for (int b = 0; b < B; ++b)
+    if (pos[b] < 0 || (int64_t)pos[b] + n_new > capacity) return -1;
+  return 0;
+}
+
+/* Hadamard rotation (signs) or none (signs == NULL). */
+int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                           int n_new, int d, const int32_t* pos, const int8_t* signs,
+                           uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                           float* v_scales, int64_t capacity, int nthreads) {
+  if ((d & (d - 1)) != 0 || check_append(B, n_new, d, pos, capacity) != 0) return -1;
+  double* R = NULL;
+  if (signs) {
+    R = (double*)malloc(sizeof(double) * (size_t)d * d);
+    if (!R) return -2;
+    oracle_rotation_matrix(d, signs, R);
+  }
+  int rc = quantize_append_maps(k, v, in_dtype, B, Hkv, n_new, d, pos, R, R, k_packed, k_scales,
+                                v_packed, v_scales, capacity, nthreads);
+  free(R);
+  return rc;
+}
+
+/* SRFT rotation: y = fl32(lambda (.) F (sigma (.) x)), lambda_k for K, lambda_v for V. */
+int oracle_quantize_append_srft(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                                int n_new, int d, const int32_t* pos, const int8_t* signs,
+                                const float* lambda_k, const float* lambda_v, uint8_t* k_packed,
+                                float* k_scales, uint8_t* v_packed, float* v_scales,
+                                int64_t capacity, int nthreads) {
+  if (check_append(B, n_new, d, pos, capacity) != 0) return -1;
+  double* Ak = (double*)malloc(sizeof(double) * (size_t)d * d);
+  double* Av = (double*)malloc(sizeof(double) * (size_t)d * d);
+  int rc = -2;
+  if (Ak && Av) {
+    oracle_srft_matrix(d, signs, lambda_k, Ak);
+    oracle_srft_matrix(d, signs, lambda_v, Av);
+    rc = quantize_append_maps(k, v, in_dtype, B, Hkv, n_new, d, pos, Ak, Av, k_packed, k_scales,
+                              v_packed, v_scales, capacity, nthreads);
+  }
+  free(Ak);
+  free(Av);
+  return rc;
 }
 
 /* ------------------------------------------------------------------ */
@@ -226,18 +317,13 @@ int oracle_quantize_append(const void* k, const void* v, int in_dtype, int B, in
  *   q_r = R q;  S_t = attn_scale * sum_i q_r[i] * s_k[t][g(i)] * c_k[t][i]
  *   p = softmax(S);  o_r[i] = sum_t p_t * s_v[t][g(i)] * c_v[t][i];  o = R^T o_r
  */
-int oracle_sdpa_int4_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int d,
-                            const uint8_t* k_packed, const float* k_scales,
-                            const uint8_t* v_packed, const float* v_scales, int64_t capacity,
-                            const int32_t* ctx_lens, const int8_t* signs, double attn_scale,
-                            double* out, int nthreads) {
-  if (Hkv <= 0 || Hq % Hkv != 0 || d % ORACLE_GROUP != 0 || (d & (d - 1)) != 0) return -1;
-  for (int b = 0; b < B; ++b)
-    if (ctx_lens[b] < 1 || ctx_lens[b] > capacity) return -1;
+/* Q: query map (q_r = Q q), O: output map (o = O o_r), both d x d. */
+static int sdpa_int4_decode_maps(const void* q, int q_dtype, int B, int Hq, int Hkv, int d,
+                                 const uint8_t* k_packed, const float* k_scales,
+                                 const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                                 const int32_t* ctx_lens, const double* Q, const double* O,
+                                 double attn_scale, double* out, int nthreads) {
   int G = Hq / Hkv, ng = d / ORACLE_GROUP;
-  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
-  if (!R) return -2;
-  oracle_rotation_matrix(d, signs, R);
   int64_t nrows = (int64_t)B * Hq;
   int fail = 0;
 #ifdef _OPENMP
@@ -254,7 +340,7 @@ int oracle_sdpa_int4_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, 
     for (int i = 0; i < d; ++i) qv[i] = (double)load_input(q, q_dtype, bh * d + i);
     for (int i = 0; i < d; ++i) {
       double acc = 0.0;
-      for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * qv[j];
+      for (int j = 0; j < d; ++j) acc += Q[(int64_t)i * d + j] * qv[j];
       qr[i] = acc;
     }
     int64_t base = ((int64_t)b * Hkv + hk) * capacity;
@@ -276,15 +362,64 @@ int oracle_sdpa_int4_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, 
       double p = S[t] / Z;
       for (int i = 0; i < d; ++i) orot[i] += p * ((double)sv[i / ORACLE_GROUP] * (double)codes[i]);
     }
-    for (int j = 0; j < d; ++j) {   /* o = R^T o_r */
+    for (int j = 0; j < d; ++j) {   /* o = O o_r */
       double acc = 0.0;
-      for (int i = 0; i < d; ++i) acc += R[(int64_t)i * d + j] * orot[i];
+      for (int i = 0; i < d; ++i) acc += O[(int64_t)j * d + i] * orot[i];
       out[bh * d + j] = acc;
     }
     free(S);
   }
-  free(R);
   return fail ? -2 : 0;
+}
+
+static int check_decode(int B, int Hq, int Hkv, int d, const int32_t* ctx_lens, int64_t capacity) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || d % ORACLE_GROUP != 0 || d > 512) return -1;
+  for (int b = 0; b < B; ++b)
+    if (ctx_lens[b] < 1 || ctx_lens[b] > capacity) return -1;
+  return 0;
+}
+
+/* Hadamard rotation (signs; q_r = R q, o = R^T o_r) or none (signs == NULL). */
+int oracle_sdpa_int4_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int d,
+                            const uint8_t* k_packed, const float* k_scales,
+                            const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                            const int32_t* ctx_lens, const int8_t* signs, double attn_scale,
+                            double* out, int nthreads) {
+  if ((d & (d - 1)) != 0 || check_decode(B, Hq, Hkv, d, ctx_lens, capacity) != 0) return -1;
+  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
+  double* RT = (double*)malloc(sizeof(double) * (size_t)d * d);
+  int rc = -2;
+  if (R && RT) {
+    oracle_rotation_matrix(d, signs, R);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) RT[(int64_t)j * d + i] = R[(int64_t)i * d + j];
+    rc = sdpa_int4_decode_maps(q, q_dtype, B, Hq, Hkv, d, k_packed, k_scales, v_packed, v_scales,
+                               capacity, ctx_lens, R, RT, attn_scale, out, nthreads);
+  }
+  free(R);
+  free(RT);
+  return rc;
+}
+
+/* SRFT rotation: q_r = F (sigma (.) q) / lambda_k, o = sigma (.) F (o_r / lambda_v). */
+int oracle_sdpa_int4_decode_srft(const void* q, int q_dtype, int B, int Hq, int Hkv, int d,
+                                 const uint8_t* k_packed, const float* k_scales,
+                                 const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                                 const int32_t* ctx_lens, const int8_t* signs,
+                                 const float* lambda_k, const float* lambda_v, double attn_scale,
+                                 double* out, int nthreads) {
+  if (check_decode(B, Hq, Hkv, d, ctx_lens, capacity) != 0) return -1;
+  double* Q = (double*)malloc(sizeof(double) * (size_t)d * d);
+  double* O = (double*)malloc(sizeof(double) * (size_t)d * d);
+  int rc = -2;
+  if (Q && O) {
+    srft_query_output_maps(d, signs, lambda_k, lambda_v, Q, O);
+    rc = sdpa_int4_decode_maps(q, q_dtype, B, Hq, Hkv, d, k_packed, k_scales, v_packed, v_scales,
+                               capacity, ctx_lens, Q, O, attn_scale, out, nthreads);
+  }
+  free(Q);
+  free(O);
+  return rc;
 }
 
 /* ------------------------------------------------------------------ */

@@ -15,16 +15,28 @@ MUTATIONS = {
     "round_half_away": ("float r = nearbyintf(quot);", "float r = roundf(quot);"),
     "nibble_order_swapped": ("    int shift = ((i % ORACLE_GROUP) % 2) ? 4 : 0;\n    packed[b]",
                              "    int shift = ((i % ORACLE_GROUP) % 2) ? 0 : 4;\n    packed[b]"),
-    "query_rotated_by_transpose": ("acc += R[(int64_t)i * d + j] * qv[j];",
-                                   "acc += R[(int64_t)j * d + i] * qv[j];"),
-    "output_not_inverse_rotated": ("acc += R[(int64_t)i * d + j] * orot[i];",
-                                   "acc += R[(int64_t)j * d + i] * orot[i];"),
+    "query_rotated_by_transpose": ("acc += Q[(int64_t)i * d + j] * qv[j];",
+                                   "acc += Q[(int64_t)j * d + i] * qv[j];"),
+    "output_not_inverse_rotated": ("acc += O[(int64_t)j * d + i] * orot[i];",
+                                   "acc += O[(int64_t)i * d + j] * orot[i];"),
     "signs_applied_after_hadamard": ("* (double)signs[j];", "* (double)signs[i];"),
     "value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP]", "(double)sv[0]"),
     "gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512]",
                        "hk = hq % Hkv;\n    int64_t T = ctx_lens[b];\n    double qv[512]"),
     "missing_softmax_normalizer": ("double p = S[t] / Z;", "double p = S[t];"),
     "byte_index_group_stride": ("+ 2 * g + (j % 4) / 2;", "+ g + (j % 4) / 2;"),
+    "hartley_cos_minus_sin": ("return (cos(th) + sin(th)) / sqrt((double)d);",
+                              "return (cos(th) - sin(th)) / sqrt((double)d);"),
+    "hartley_unnormalized": ("return (cos(th) + sin(th)) / sqrt((double)d);",
+                             "return (cos(th) + sin(th)) / (double)d;"),
+    "srft_sign_on_output_index": ("if (signs) v *= (double)signs[j];",
+                                  "if (signs) v *= (double)signs[k];"),
+    "srft_lambda_on_input_index": ("if (lambda) v *= (double)lambda[k];",
+                                   "if (lambda) v *= (double)lambda[j];"),
+    "srft_query_times_lambda": ("f * sj / (lambda_k ? (double)lambda_k[k] : 1.0);",
+                                "f * sj * (lambda_k ? (double)lambda_k[k] : 1.0);"),
+    "srft_output_without_lambda": ("sj * f / (lambda_v ? (double)lambda_v[k] : 1.0);", "sj * f;"),
+    "srft_output_sign_index": ("O[(int64_t)j * d + k] = sj", "O[(int64_t)j * d + k] = (signs ? (double)signs[k] : 1.0)"),
 }
 
 

@@ -393,3 +393,110 @@ def test_oracle_rejects_bad_shapes():
         oracle.sdpa_int4_decode(q, cache, [4], None, 1.0, 2)      # 3 % 2 != 0
     with pytest.raises(ValueError):
         oracle.sdpa_int4_decode(np.zeros((1, 2, 64), np.float32), cache, [5], None, 1.0, 2)
+
+
+# ------------------------------------------------------- SRFT variant
+# The SRFT post (core method) replaces the Hadamard rotation by a
+# sign-randomized Fourier transform that works at widths that are not powers of
+# two, followed by a per-coordinate scale lambda.  The oracle's transform is the
+# orthonormal discrete Hartley transform; these pins check it against numpy's
+# FFT (H = Re X - Im X for X = fft(x)), against the transform's algebra, and
+# the whole variant against attention over a cache built exactly on the grid.
+
+def _hartley_from_fft(d):
+    X = np.fft.fft(np.eye(d), axis=0)          # column j = DFT of e_j
+    return (X.real - X.imag) / np.sqrt(d)
+
+
+def _rand_lambda(rng, d):
+    return np.exp2(rng.uniform(-1.0, 1.0, d)).astype(np.float32)
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 5, 12, 32, 96, 160, 256])
+def test_dht_matches_numpy_fft(d):
+    F = oracle.srft_matrix(d)
+    np.testing.assert_allclose(F, _hartley_from_fft(d), rtol=0, atol=1e-14)
+
+
+def test_dht_hand_values_d4():
+    # cas(pi k j / 2) for k, j in 0..3: cos + sin of multiples of 90 degrees
+    want = np.array([[1, 1, 1, 1], [1, 1, -1, -1], [1, -1, 1, -1], [1, -1, -1, 1]]) / 2.0
+    np.testing.assert_allclose(oracle.srft_matrix(4), want, rtol=0, atol=1e-15)
+    assert oracle.dht_entry(4, 1, 1) == pytest.approx(1.0 / 2.0, abs=1e-15)
+
+
+@pytest.mark.parametrize("d", [32, 96, 160, 224])
+def test_dht_is_symmetric_orthogonal_involution(d):
+    F = oracle.srft_matrix(d)
+    np.testing.assert_array_equal(F, F.T)
+    assert np.max(np.abs(F @ F - np.eye(d))) <= 1e-13
+
+
+@pytest.mark.parametrize("d", [32, 96, 192])
+def test_srft_store_map_is_lambda_hartley_signs(d):
+    rng = np.random.default_rng(d + 7)
+    s, lam = rand_signs(rng, d), _rand_lambda(rng, d)
+    A = oracle.srft_matrix(d, s, lam)
+    want = lam.astype(np.float64)[:, None] * _hartley_from_fft(d) * s.astype(np.float64)[None, :]
+    np.testing.assert_allclose(A, want, rtol=0, atol=1e-13)
+    x = rng.standard_normal((5, d)).astype(np.float32)
+    y = oracle.srft_rotate(x, s, lam)
+    np.testing.assert_allclose(y, (x.astype(np.float64) @ want.T).astype(np.float32), rtol=2e-7,
+                               atol=1e-7)
+
+
+def test_srft_group_uniform_power_of_two_lambda_scales_exactly():
+    """lambda = 2^e constant on each group multiplies that group's scale by 2^e
+    exactly and leaves its codes unchanged (the quantizer is scale-equivariant)."""
+    rng = np.random.default_rng(3)
+    d = 96
+    s = rand_signs(rng, d)
+    e = np.repeat(np.array([-2, 0, 3]), 32)
+    lam = np.exp2(e).astype(np.float32)
+    x = rng.standard_normal((1, 1, 4, d)).astype(np.float32)
+    c1, c2 = oracle.empty_cache(1, 1, 4, d), oracle.empty_cache(1, 1, 4, d)
+    oracle.quantize_append_srft(x, x, [0], s, None, None, c1)
+    oracle.quantize_append_srft(x, x, [0], s, lam, None, c2)
+    np.testing.assert_array_equal(c1[0], c2[0])
+    np.testing.assert_array_equal(c1[1] * np.exp2([-2, 0, 3]).astype(np.float32), c2[1])
+    np.testing.assert_array_equal(c1[2], c2[2])       # V uses its own (unit) lambda
+    np.testing.assert_array_equal(c1[3], c2[3])
+
+
+@pytest.mark.parametrize("d", [32, 96, 160])
+def test_srft_end_to_end_on_grid_is_exact_attention(d):
+    """K and V are built so that their SRFT images (with random signs and
+    random lambdas) lie on the int4 grid: quantize-append then decode must give
+    the unquantized attention over the original vectors.  Catches a query map
+    that multiplies by lambda instead of dividing, an output map without the
+    inverse transform or without 1/lambda_V, and a transposed sign."""
+    rng = np.random.default_rng(d)
+    B, Hkv, G, T = 1, 2, 3, 9
+    s = rand_signs(rng, d)
+    lk, lv = _rand_lambda(rng, d), _rand_lambda(rng, d)
+    Fh = _hartley_from_fft(d)
+    inv_store = lambda lam: (s.astype(np.float64)[:, None] * Fh) / lam.astype(np.float64)[None, :]
+    c = rng.integers(-7, 8, (2, B, Hkv, T, d))
+    c[..., ::32] = 7                      # a full-scale code in every group
+    yk, yv = c[0] * 0.25, c[1] * 0.125
+    k = (yk @ inv_store(lk).T).astype(np.float32)
+    v = (yv @ inv_store(lv).T).astype(np.float32)
+    cache = oracle.empty_cache(B, Hkv, T, d)
+    oracle.quantize_append_srft(k, v, [0], s, lk, lv, cache)
+    codes = oracle.unpack(cache[0].reshape(-1, d // 2), d).reshape(c[0].shape)
+    np.testing.assert_array_equal(codes, c[0])
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    got = oracle.sdpa_int4_decode_srft(q, cache, [T], s, lk, lv, 0.3, Hkv)
+    want = oracle.exact_attention(q, k, v, [T], 0.3)
+    np.testing.assert_allclose(got, want, rtol=2e-6, atol=2e-6 * np.abs(want).max())
+
+
+def test_srft_reduces_to_hartley_when_unit_signs_and_lambda():
+    rng = np.random.default_rng(5)
+    d = 96
+    x = rng.standard_normal((3, d)).astype(np.float32)
+    ones = np.ones(d, np.int8)
+    np.testing.assert_array_equal(oracle.srft_rotate(x, ones, np.ones(d, np.float32)),
+                                  oracle.srft_rotate(x))
+    np.testing.assert_allclose(oracle.srft_rotate(x), x.astype(np.float64) @ _hartley_from_fft(d).T,
+                               rtol=2e-7, atol=1e-7)
