@@ -22,7 +22,8 @@ TQ_F32, TQ_BF16 = 0, 1
 SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_tokens",
            "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_append", "tq_sdpa_int4_decode_lse",
            "tq_merge_lse", "tq_sdpa_int4_decode_static_scratch", "tq_dequantize",
-           "tq_status_string")
+           "tq_decode_srft_workspace_bytes", "tq_quantize_append_srft", "tq_sdpa_int4_decode_srft",
+           "tq_sdpa_int4_decode_append_srft", "tq_status_string")
 
 _lib = None
 
@@ -64,6 +65,17 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode_static_scratch.restype = i32
     lib.tq_dequantize.argtypes = [P, P, i32, i32, i64, i32, i32, P, i32, P]
     lib.tq_dequantize.restype = i32
+    lib.tq_decode_srft_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.tq_decode_srft_workspace_bytes.restype = sz
+    lib.tq_quantize_append_srft.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                            P, i64, P]
+    lib.tq_quantize_append_srft.restype = i32
+    lib.tq_sdpa_int4_decode_srft.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64, P, i32,
+                                             P, P, P, f32, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_srft.restype = i32
+    lib.tq_sdpa_int4_decode_append_srft.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P, P,
+                                                    P, P, i64, P, i32, P, P, P, f32, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_append_srft.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -198,3 +210,62 @@ def dequantize(packed, scales, rows, out, stream=None):
                               _ptr(out), _dtype_code(out), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_dequantize")
+
+
+# ------------------------------------------------------------------ SRFT variant
+# The rotation of "SRFT + int4 KV-cache on Apple Silicon" (core method): the
+# orthonormal discrete Hartley transform with random signs, then per-coordinate
+# scales lambda_k / lambda_v (float32 [d] CUDA tensors, or None for ones).
+
+def decode_srft_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx) -> int:
+    return int(load().tq_decode_srft_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
+                                                     max_ctx))
+
+
+def quantize_append_srft(k, v, pos, signs, lambda_k, lambda_v, k_packed, k_scales, v_packed,
+                         v_scales, stream=None):
+    """Quantize k, v [B][Hkv][n_new][d] with the SRFT rotation into rows pos[b] .. pos[b]+n_new-1."""
+    _need_cuda(k, v, pos, signs, lambda_k, lambda_v, k_packed, k_scales, v_packed, v_scales)
+    B, H, n, d = k.shape
+    rc = load().tq_quantize_append_srft(_ptr(k), _ptr(v), _dtype_code(k), B, H, n, d, 32, _ptr(pos),
+                                        _ptr(signs), _ptr(lambda_k), _ptr(lambda_v),
+                                        _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+                                        _ptr(v_scales), k_packed.shape[2], _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_quantize_append_srft")
+
+
+def sdpa_int4_decode_srft(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs,
+                          lambda_k, lambda_v, attn_scale, out, workspace, stream=None):
+    """out[B][Hq][d] (fp32, unrotated) = attention of q over an SRFT cache."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, lambda_k, lambda_v, out,
+               workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_srft(
+        _ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+        _ptr(v_scales), k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs),
+        _ptr(lambda_k), _ptr(lambda_v), float(attn_scale), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_srft")
+
+
+def sdpa_int4_decode_append_srft(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                                 max_ctx, signs, lambda_k, lambda_v, attn_scale, out, workspace,
+                                 stream=None):
+    """One decode step over an SRFT cache (append of k_new, v_new at row ctx_lens[b]-1, then attend)."""
+    _need_cuda(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, lambda_k,
+               lambda_v, out, workspace)
+    if k_new.dtype != v_new.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_append_srft(
+        _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq, Hkv, d, 32,
+        _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), k_packed.shape[2],
+        _ptr(ctx_lens), int(max_ctx), _ptr(signs), _ptr(lambda_k), _ptr(lambda_v),
+        float(attn_scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_append_srft")

@@ -4,6 +4,12 @@ The call shape follows the AdapTQ engine (AdapTQ post, section "native Python
 API": an engine of fixed dim, heads and capacity with append(k, v) and
 compute(q)).  Torch only provides the device buffers and the stream; both
 operations run in libtq's kernels.
+
+rotation="hadamard" (default): signs + Walsh-Hadamard rotation (or none when
+signs is None), head_dim 128 or 256.  rotation="srft": the SRFT post's variant
+(core method): signs + orthonormal discrete Hartley transform, then the
+per-coordinate scales lambda_k / lambda_v (float32 [d], None = ones); head_dim
+any multiple of 32 up to 256.
 """
 from __future__ import annotations
 
@@ -16,9 +22,15 @@ from . import _lib
 
 class Int4KVCache:
     def __init__(self, batch: int, num_kv_heads: int, head_dim: int, capacity: int,
-                 device="cuda", signs: torch.Tensor | None = None):
+                 device="cuda", signs: torch.Tensor | None = None, rotation: str = "hadamard",
+                 lambda_k: torch.Tensor | None = None, lambda_v: torch.Tensor | None = None):
         if head_dim % 32:
             raise ValueError("head_dim must be a multiple of 32")
+        if rotation not in ("hadamard", "srft"):
+            raise ValueError("rotation must be 'hadamard' or 'srft'")
+        if rotation == "hadamard" and (lambda_k is not None or lambda_v is not None):
+            raise ValueError("lambda_k / lambda_v belong to the srft rotation")
+        self.srft = rotation == "srft"
         self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
         dev = torch.device(device)
         shape = (batch, num_kv_heads, capacity)
@@ -27,6 +39,8 @@ class Int4KVCache:
         self.k_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
         self.v_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
         self.signs = None if signs is None else signs.to(device=dev, dtype=torch.int8).contiguous()
+        self.lambda_k = None if lambda_k is None else lambda_k.to(device=dev, dtype=torch.float32).contiguous()
+        self.lambda_v = None if lambda_v is None else lambda_v.to(device=dev, dtype=torch.float32).contiguous()
         self._ws = None
 
     def nbytes(self) -> int:
@@ -34,11 +48,17 @@ class Int4KVCache:
 
     def append(self, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor, stream=None) -> None:
         """Quantize k, v [B][Hkv][n][d] into rows pos[b] .. pos[b]+n-1."""
+        if self.srft:
+            _lib.quantize_append_srft(k, v, pos, self.signs, self.lambda_k, self.lambda_v,
+                                      self.k_packed, self.k_scales, self.v_packed, self.v_scales,
+                                      stream)
+            return
         _lib.quantize_append(k, v, pos, self.signs, self.k_packed, self.k_scales, self.v_packed,
                              self.v_scales, stream)
 
     def workspace(self, num_q_heads: int, max_ctx: int) -> torch.Tensor:
-        need = _lib.decode_workspace_bytes(self.batch, num_q_heads, self.num_kv_heads, self.head_dim, max_ctx)
+        sizer = _lib.decode_srft_workspace_bytes if self.srft else _lib.decode_workspace_bytes
+        need = sizer(self.batch, num_q_heads, self.num_kv_heads, self.head_dim, max_ctx)
         if need == 0:
             raise ValueError("invalid decode sizes")
         if self._ws is None or self._ws.numel() < need:
@@ -53,6 +73,11 @@ class Int4KVCache:
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         ws = self.workspace(q.shape[1], max_ctx)
+        if self.srft:
+            _lib.sdpa_int4_decode_srft(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
+                                       ctx_lens, max_ctx, self.signs, self.lambda_k, self.lambda_v,
+                                       attn_scale, out, ws, stream)
+            return out
         _lib.sdpa_int4_decode(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
                               ctx_lens, max_ctx, self.signs, attn_scale, out, ws, stream)
         return out
@@ -67,6 +92,12 @@ class Int4KVCache:
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         ws = self.workspace(q.shape[1], max_ctx)
+        if self.srft:
+            _lib.sdpa_int4_decode_append_srft(q, k_new, v_new, self.k_packed, self.k_scales,
+                                              self.v_packed, self.v_scales, ctx_lens, max_ctx,
+                                              self.signs, self.lambda_k, self.lambda_v, attn_scale,
+                                              out, ws, stream)
+            return out
         _lib.sdpa_int4_decode_append(q, k_new, v_new, self.k_packed, self.k_scales, self.v_packed,
                                      self.v_scales, ctx_lens, max_ctx, self.signs, attn_scale, out,
                                      ws, stream)

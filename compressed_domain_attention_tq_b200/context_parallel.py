@@ -47,6 +47,8 @@ def decode(cache, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
     max_ctx    host bound on this rank's ctx_lens.
     Every rank calls this with the same q, attn_scale and group; every rank
     returns the full output (fp32 [B][Hq][d], unrotated basis)."""
+    if cache.srft:
+        raise NotImplementedError("context-parallel decode runs on Hadamard-rotated caches")
     if attn_scale is None:
         attn_scale = 1.0 / math.sqrt(cache.head_dim)
     B, Hq, d = q.shape

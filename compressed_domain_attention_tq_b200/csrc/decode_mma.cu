@@ -380,7 +380,16 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     float x[E];
     if (h < G) {
       const int64_t base = ((int64_t)b * a.Hq + (int64_t)kvh * G + h) * D + lane * E;
-      if (a.q_bf16) {  // E consecutive bf16 values: one 8- or 16-byte load
+      if (a.q_rot != nullptr) {  // SRFT variant: the query is already rotated (fp32)
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(a.q_rot + base + e);
+          x[e] = v.x;
+          x[e + 1] = v.y;
+          x[e + 2] = v.z;
+          x[e + 3] = v.w;
+        }
+      } else if (a.q_bf16) {  // E consecutive bf16 values: one 8- or 16-byte load
         uint32_t u[E / 2];
         if (E == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + base);
@@ -406,7 +415,8 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
           x[e + 3] = v.w;
         }
       }
-      if (a.signs) {
+      const bool wht = a.signs != nullptr && a.q_rot == nullptr;
+      if (wht) {
         int8_t sg[E];  // byte loads: the signs pointer has no alignment requirement
 #pragma unroll
         for (int e = 0; e < E; ++e) sg[e] = a.signs[lane * E + e];
@@ -429,7 +439,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
             x[e] = (lane & bit) ? v - x[e] : x[e] + v;
           }
       }
-      const float mul = a.attn_scale * kLog2e * (a.signs ? rsqrtf((float)D) : 1.0f);
+      const float mul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
       float amax = 0.0f;
 #pragma unroll
       for (int e = 0; e < E; ++e) {

@@ -84,15 +84,23 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   uint8_t* ktile = reinterpret_cast<uint8_t*>(alpha + 16);     // [kTile][ROWP]
   uint8_t* vtile = ktile + kTile * ROWP;
 
-  // q' = attn_scale * log2(e) * R q
+  // q' = attn_scale * log2(e) * R q (the SRFT variant's R q comes rotated in q_rot)
   const int64_t qbase = ((int64_t)b * a.Hq + (int64_t)kvh * G) * D;
+  const bool wht = a.signs != nullptr && a.q_rot == nullptr;
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    float x = load_q(a.q, a.q_bf16, qbase + i);
-    if (a.signs) x *= (float)a.signs[i % D];
+    float x;
+    if (a.q_rot != nullptr) {
+      x = a.q_rot[qbase + i];
+    } else {
+      x = load_q(a.q, a.q_bf16, qbase + i);
+      if (a.signs) x *= (float)a.signs[i % D];
+    }
     qs[i] = x;
   }
-  if (a.signs) fwht_rows<D>(qs, G);
-  const float qmul = a.attn_scale * kLog2e * (a.signs ? rsqrtf((float)D) : 1.0f);
+  if constexpr ((D & (D - 1)) == 0) {
+    if (wht) fwht_rows<D>(qs, G);
+  }
+  const float qmul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
   __syncthreads();
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) qs[i] *= qmul;
   if (threadIdx.x < 16) {
@@ -221,29 +229,36 @@ size_t simt_smem_bytes(int G) {
          2 * (size_t)kTile * ROWP;
 }
 
-}  // namespace
 
-cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
+template <int D>
+cudaError_t launch_simt_d(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   dim3 grid(a.plan.n_chunks, a.Hkv, a.B);
-  if (a.d == 128) {
-    const size_t sm = simt_smem_bytes<128>(G);
-    static std::atomic<uint64_t> smem_set{0};
-    // the limit covers every group size the host accepts (up to 16 query heads)
-    const cudaError_t e =
-        ensure_smem_limit(decode_simt_kernel<128>, (int)simt_smem_bytes<128>(16), smem_set);
-    if (e != cudaSuccess) return e;
-    decode_simt_kernel<128><<<grid, 128, sm, stream>>>(a);
-  } else {
-    const size_t sm = simt_smem_bytes<256>(G);
-    static std::atomic<uint64_t> smem_set{0};
-    // the limit covers every group size the host accepts (up to 16 query heads)
-    const cudaError_t e =
-        ensure_smem_limit(decode_simt_kernel<256>, (int)simt_smem_bytes<256>(16), smem_set);
-    if (e != cudaSuccess) return e;
-    decode_simt_kernel<256><<<grid, 128, sm, stream>>>(a);
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  // the limit covers every group size the host accepts (up to 16 query heads)
+  const cudaError_t e =
+      ensure_smem_limit(decode_simt_kernel<D>, (int)simt_smem_bytes<D>(16), smem_set);
+  if (e != cudaSuccess) return e;
+  decode_simt_kernel<D><<<grid, 128, simt_smem_bytes<D>(G), stream>>>(a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// head_dim 128 or 256; with the SRFT variant (rotated queries given) any
+// multiple of 32 up to 256
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 32: return launch_simt_d<32>(a, stream);
+    case 64: return launch_simt_d<64>(a, stream);
+    case 96: return launch_simt_d<96>(a, stream);
+    case 128: return launch_simt_d<128>(a, stream);
+    case 160: return launch_simt_d<160>(a, stream);
+    case 192: return launch_simt_d<192>(a, stream);
+    case 224: return launch_simt_d<224>(a, stream);
+    case 256: return launch_simt_d<256>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tq

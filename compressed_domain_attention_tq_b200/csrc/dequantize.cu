@@ -3,10 +3,10 @@
 // never forms these values): one thread per packed 32-bit word.
 //
 // Row layout (see tq.h): coordinate i = 32 g + j of a row sits in byte
-// (j/4)*(2*ng) + 2g + (j%4)/2, low nibble for even j.  A 32-bit word w of a row
-// therefore holds sub-block s = 4w / (2 ng) of two groups g0 = (4w mod 2 ng)/2
-// and g0 + 1: its 16-bit half k carries coordinates 32 (g0 + k) + 4 s + n in
-// nibble n (n = 0..3).
+// (j/4)*(2*ng) + 2g + (j%4)/2, low nibble for even j.  The 16-bit half-word h
+// of a row (bytes 2h, 2h + 1) therefore belongs to sub-block s = h / ng and
+// group g = h mod ng, and carries coordinates 32 g + 4 s + n in nibble n
+// (n = 0..3); a 32-bit word w holds half-words 2w and 2w + 1.
 #include <cuda_bf16.h>
 
 #include "tq_internal.h"
@@ -25,10 +25,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantizeArgs a) {
     const int64_t seq = rr / a.rows, r = rr % a.rows;
     const int64_t src_row = seq * a.row_stride + r;
     const uint32_t word = reinterpret_cast<const uint32_t*>(a.packed + src_row * (D / 2))[wi];
-    const int s = (4 * wi) / (2 * NG), g0 = ((4 * wi) % (2 * NG)) / 2;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int g = g0 + k;
+      const int hw = 2 * wi + k, s = hw / NG, g = hw % NG;
       const float sc = a.scales[src_row * NG + g];
       float v[4];
 #pragma unroll
@@ -64,11 +63,27 @@ cudaError_t launch_dq(const DequantizeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+
+template <int D>
+cudaError_t launch_dq_d(const DequantizeArgs& a, cudaStream_t stream) {
+  return a.bf16 ? launch_dq<D, true>(a, stream) : launch_dq<D, false>(a, stream);
+}
+
 }  // namespace
 
+// head_dim: any multiple of 32 up to 256
 cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t stream) {
-  if (a.d == 128) return a.bf16 ? launch_dq<128, true>(a, stream) : launch_dq<128, false>(a, stream);
-  return a.bf16 ? launch_dq<256, true>(a, stream) : launch_dq<256, false>(a, stream);
+  switch (a.d) {
+    case 32: return launch_dq_d<32>(a, stream);
+    case 64: return launch_dq_d<64>(a, stream);
+    case 96: return launch_dq_d<96>(a, stream);
+    case 128: return launch_dq_d<128>(a, stream);
+    case 160: return launch_dq_d<160>(a, stream);
+    case 192: return launch_dq_d<192>(a, stream);
+    case 224: return launch_dq_d<224>(a, stream);
+    case 256: return launch_dq_d<256>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tq

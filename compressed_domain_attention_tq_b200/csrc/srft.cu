@@ -1,0 +1,297 @@
+// srft.cu -- the SRFT variant of the rotation (SRFT post, core method): a
+// sign-randomized Fourier transform in place of the Hadamard one, usable at
+// any width d = 32 M (M = 1 .. 8, so also d = 96, 160, 192, 224), followed by
+// a per-coordinate scale lambda before the group abs-max quantization.
+//
+// The transform is the orthonormal discrete Hartley transform F (real,
+// symmetric, F F = I), computed two vectors at a time by srft.cuh.  With
+// signs sigma and scales lambda_K, lambda_V:
+//   stored K row  y_k = lambda_K (.) F (sigma (.) k)   (V likewise with lambda_V)
+//   query         q_r = F (sigma (.) q) / lambda_K     so q_r . y_k = q . k
+//   output        o   = sigma (.) F (o_r / lambda_V)
+// Kernels:
+//   srft_quantize_kernel  one warp per (sequence, kv head, token): K and V of
+//                         the token form one complex transform; then group
+//                         abs-max, int4 codes and the packed row layout of the
+//                         Hadamard path.
+//   srft_query_kernel     one warp per pair of query heads -> q_r (fp32) in the
+//                         decode workspace; the decode kernels read it instead
+//                         of rotating q themselves.
+//   srft_merge_kernel     one CTA per pair of query heads: the split-K log-sum-
+//                         exp merge of each head, 1 / lambda_V, then one warp
+//                         maps both heads back.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "srft.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int kQWarps = 8;  // warps per quantize CTA
+
+template <int M>
+__global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArgs a) {
+  constexpr int D = 32 * M;
+  __shared__ float ybuf[kQWarps][2][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  HartleyTwiddles<M> tw;
+  hartley_twiddles<M>(tw, lane);
+  const float norm = 0.5f / sqrtf((float)D);
+  float sg[M], mk[M], mv[M];
+#pragma unroll
+  for (int j2 = 0; j2 < M; ++j2) sg[j2] = a.signs ? (float)a.signs[lane + 32 * j2] : 1.0f;
+#pragma unroll
+  for (int k2 = 0; k2 < M; ++k2) {
+    const int k = k2 + M * brev5(lane);
+    mk[k2] = a.lambda_k ? norm * a.lambda_k[k] : norm;
+    mv[k2] = a.lambda_v ? norm * a.lambda_v[k] : norm;
+  }
+  float* yk = ybuf[warp][0];
+  float* yv = ybuf[warp][1];
+  const int64_t pairs = (int64_t)a.B * a.Hkv * a.n_new;
+  for (int64_t p = (int64_t)blockIdx.x * kQWarps + warp; p < pairs;
+       p += (int64_t)gridDim.x * kQWarps) {
+    const int64_t bh = p / a.n_new, n = p % a.n_new;
+    const int b = (int)(bh / a.Hkv);
+    int64_t pos = (int64_t)a.pos[b] + n;
+    if (a.pos_is_ctx) pos = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
+    if (pos < 0 || pos >= a.capacity) continue;  // the whole warp
+    const int64_t row = bh * a.capacity + pos;
+    float re[M], im[M];
+#pragma unroll
+    for (int j2 = 0; j2 < M; ++j2) {
+      const int64_t idx = p * D + lane + 32 * j2;
+      float xk, xv;
+      if (a.bf16) {
+        xk = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.k)[idx] << 16);
+        xv = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.v)[idx] << 16);
+      } else {
+        xk = static_cast<const float*>(a.k)[idx];
+        xv = static_cast<const float*>(a.v)[idx];
+      }
+      re[j2] = sg[j2] * xk;
+      im[j2] = sg[j2] * xv;
+    }
+    float hx[M], hy[M];
+    hartley_pair_warp<M>(re, im, tw, hx, hy);
+#pragma unroll
+    for (int k2 = 0; k2 < M; ++k2) {
+      const int k = k2 + M * brev5(lane);
+      yk[k] = hx[k2] * mk[k2];
+      yv[k] = hy[k2] * mv[k2];
+    }
+    __syncwarp();
+    // lane holds in-group coordinate j = lane of every group g (coordinate 32 g + lane)
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const float* y = kv ? yv : yk;
+      uint8_t* prow = (kv ? a.v_packed : a.k_packed) + row * (D / 2);
+      float* srow = (kv ? a.v_scales : a.k_scales) + row * M;
+#pragma unroll
+      for (int g = 0; g < M; ++g) {
+        const float x = y[32 * g + lane];
+        float amax = fabsf(x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = __fdiv_rn(amax, 7.0f);
+        float c = 0.0f;
+        if (s > 0.0f) c = fminf(fmaxf(rintf(__fdiv_rn(x, s)), -7.0f), 7.0f);
+        // byte (j / 4) * 2M + 2 g + (j % 4) / 2, nibble j % 2: four lanes make one half-word
+        uint32_t nib = ((uint32_t)(int)c & 0xFu) << (4 * (lane & 3));
+        nib |= __shfl_xor_sync(0xffffffffu, nib, 1);
+        nib |= __shfl_xor_sync(0xffffffffu, nib, 2);
+        if ((lane & 3) == 0)
+          *reinterpret_cast<uint16_t*>(prow + (lane >> 2) * 2 * M + 2 * g) = (uint16_t)nib;
+        if (lane == g) srow[g] = s;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <int M>
+__global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
+  constexpr int D = 32 * M;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pairs_per_b = (a.Hq + 1) / 2;
+  const int64_t p = (int64_t)blockIdx.x * 4 + warp;
+  if (p >= (int64_t)a.B * pairs_per_b) return;  // the whole warp
+  const int b = (int)(p / pairs_per_b), h0 = 2 * (int)(p % pairs_per_b);
+  const bool two = h0 + 1 < a.Hq;
+  HartleyTwiddles<M> tw;
+  hartley_twiddles<M>(tw, lane);
+  float re[M], im[M];
+  const int64_t base0 = ((int64_t)b * a.Hq + h0) * D;
+#pragma unroll
+  for (int j2 = 0; j2 < M; ++j2) {
+    const int j = lane + 32 * j2;
+    const float sg = a.signs ? (float)a.signs[j] : 1.0f;
+    float x0, x1 = 0.0f;
+    if (a.q_bf16) {
+      const uint16_t* q = static_cast<const uint16_t*>(a.q);
+      x0 = __uint_as_float((uint32_t)q[base0 + j] << 16);
+      if (two) x1 = __uint_as_float((uint32_t)q[base0 + D + j] << 16);
+    } else {
+      const float* q = static_cast<const float*>(a.q);
+      x0 = q[base0 + j];
+      if (two) x1 = q[base0 + D + j];
+    }
+    re[j2] = sg * x0;
+    im[j2] = sg * x1;
+  }
+  float hx[M], hy[M];
+  hartley_pair_warp<M>(re, im, tw, hx, hy);
+  const float norm = 0.5f / sqrtf((float)D);
+  float* q_rot = const_cast<float*>(a.q_rot);
+#pragma unroll
+  for (int k2 = 0; k2 < M; ++k2) {
+    const int k = k2 + M * brev5(lane);
+    const float mul = a.lambda_k ? __fdiv_rn(norm, a.lambda_k[k]) : norm;
+    q_rot[base0 + k] = hx[k2] * mul;
+    if (two) q_rot[base0 + D + k] = hy[k2] * mul;
+  }
+}
+
+// Log-sum-exp merge of one head's chunk partials (acc[i], m, l) for
+// coordinate i; returns acc / l and sets the head's (M, L).
+__device__ __forceinline__ float combine_chunks(const float* part, int nc, int stride, int d, int i,
+                                                float& Mx, float& L) {
+  Mx = -INFINITY;
+  for (int c = 0; c < nc; ++c) Mx = fmaxf(Mx, part[(int64_t)c * stride + d]);
+  constexpr int U = 4;
+  float acc[U], ls[U];
+#pragma unroll
+  for (int k = 0; k < U; ++k) acc[k] = ls[k] = 0.0f;
+  for (int c0 = 0; c0 < nc; c0 += U) {
+#pragma unroll
+    for (int k = 0; k < U; ++k)
+      if (c0 + k < nc) {
+        const float* pc = part + (int64_t)(c0 + k) * stride;
+        const float w = exp2f(pc[d] - Mx);
+        ls[k] = fmaf(w, pc[d + 1], ls[k]);
+        acc[k] = fmaf(w, pc[i], acc[k]);
+      }
+  }
+  L = (ls[0] + ls[2]) + (ls[1] + ls[3]);
+  return ((acc[0] + acc[2]) + (acc[1] + acc[3])) / L;
+}
+
+template <int M>
+__global__ void __launch_bounds__(32 * M) srft_merge_kernel(DecodeArgs a) {
+  constexpr int D = 32 * M;
+  __shared__ float z[2][D];
+  const int pairs_per_b = (a.Hq + 1) / 2;
+  const int b = blockIdx.x / pairs_per_b, h0 = 2 * (blockIdx.x % pairs_per_b);
+  const int i = threadIdx.x, lane = i & 31;
+  const int raw = a.ctx_lens[b];
+  const int T = raw < 1 ? 1 : (raw > a.max_ctx ? a.max_ctx : raw);
+  const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
+  const int stride = a.plan.part_stride;
+  const float lv = a.lambda_v ? a.lambda_v[i] : 1.0f;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float* parts = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
+                                                      a.plan.header_bytes);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = h0 + hh;
+    float x = 0.0f;
+    if (h < a.Hq) {
+      float Mx, L;
+      const float* part = parts + ((int64_t)b * a.Hq + h) * a.plan.n_chunks * stride;
+      x = combine_chunks(part, nc, stride, D, i, Mx, L) / lv;
+      if (a.lse != nullptr && i == 0)
+        *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + h) * 2) = make_float2(Mx, L);
+    }
+    z[hh][i] = x;
+  }
+  __syncthreads();
+  if (i >= 32) return;
+  HartleyTwiddles<M> tw;
+  hartley_twiddles<M>(tw, lane);
+  float re[M], im[M];
+#pragma unroll
+  for (int j2 = 0; j2 < M; ++j2) {
+    re[j2] = z[0][lane + 32 * j2];
+    im[j2] = z[1][lane + 32 * j2];
+  }
+  float hx[M], hy[M];
+  hartley_pair_warp<M>(re, im, tw, hx, hy);
+  const float norm = 0.5f / sqrtf((float)D);
+  const int64_t base0 = ((int64_t)b * a.Hq + h0) * D;
+#pragma unroll
+  for (int k2 = 0; k2 < M; ++k2) {
+    const int k = k2 + M * brev5(lane);
+    const float sg = a.signs ? (float)a.signs[k] * norm : norm;
+    a.out[base0 + k] = hx[k2] * sg;
+    if (h0 + 1 < a.Hq) a.out[base0 + D + k] = hy[k2] * sg;
+  }
+}
+
+template <int M>
+cudaError_t launch_quantize_srft_m(const QuantizeArgs& a, cudaStream_t stream) {
+  const int64_t pairs = (int64_t)a.B * a.Hkv * a.n_new;
+  int64_t blocks = (pairs + kQWarps - 1) / kQWarps;
+  const int64_t cap = (int64_t)kSmCount * (M <= 4 ? 8 : 4);
+  if (blocks > cap) blocks = cap;
+  srft_quantize_kernel<M><<<(unsigned)blocks, 32 * kQWarps, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int M>
+cudaError_t launch_srft_query_m(const DecodeArgs& a, cudaStream_t stream) {
+  const int64_t warps = (int64_t)a.B * ((a.Hq + 1) / 2);
+  srft_query_kernel<M><<<(unsigned)((warps + 3) / 4), 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int M>
+cudaError_t launch_srft_merge_m(const DecodeArgs& a, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * ((a.Hq + 1) / 2));
+  cfg.blockDim = dim3(32 * M);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, srft_merge_kernel<M>, a);
+}
+
+#define TQ_SRFT_DISPATCH(FN, ARG)            \
+  switch (d / 32) {                          \
+    case 1: return FN<1>(ARG, stream);       \
+    case 2: return FN<2>(ARG, stream);       \
+    case 3: return FN<3>(ARG, stream);       \
+    case 4: return FN<4>(ARG, stream);       \
+    case 5: return FN<5>(ARG, stream);       \
+    case 6: return FN<6>(ARG, stream);       \
+    case 7: return FN<7>(ARG, stream);       \
+    case 8: return FN<8>(ARG, stream);       \
+    default: return cudaErrorInvalidValue;   \
+  }
+
+}  // namespace
+
+bool srft_head_dim_supported(int d) { return d >= 32 && d <= 256 && d % 32 == 0; }
+
+cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream) {
+  const int d = a.d;
+  TQ_SRFT_DISPATCH(launch_quantize_srft_m, a)
+}
+
+cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream) {
+  const int d = a.d;
+  TQ_SRFT_DISPATCH(launch_srft_query_m, a)
+}
+
+cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream) {
+  const int d = a.d;
+  TQ_SRFT_DISPATCH(launch_srft_merge_m, a)
+}
+
+}  // namespace tq

@@ -18,9 +18,9 @@ static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // 192 or 128 tokens) for persistent CTAs, one per SM: pick the chunk count per
 // sequence that minimises (waves of items over the SMs) x (chunk + a fixed
 // per-item cost), where an item is one (sequence, kv head, chunk).
-bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan) {
+bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan, bool srft) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
-  if (d != 128 && d != 256) return false;
+  if (srft ? !srft_head_dim_supported(d) : (d != 128 && d != 256)) return false;
   const int64_t units = (int64_t)B * Hkv;
   const int64_t step = decode_stage_tokens(d, Hq / Hkv), per_item_cost = 384;
   const int64_t max_n = ceil_div(max_ctx, step);
@@ -40,6 +40,11 @@ bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* pl
   plan->header_bytes = (size_t)ceil_div(4LL * B, 256) * 256;
   plan->ws_bytes = plan->header_bytes +
                    sizeof(float) * (size_t)B * Hq * plan->n_chunks * plan->part_stride;
+  plan->qrot_offset = 0;
+  if (srft) {  // the rotated queries follow the partials
+    plan->qrot_offset = (size_t)ceil_div((int64_t)plan->ws_bytes, 256) * 256;
+    plan->ws_bytes = plan->qrot_offset + sizeof(float) * (size_t)B * Hq * d;
+  }
   return true;
 }
 
@@ -52,6 +57,19 @@ static tq_status cuda_status(cudaError_t e, const char* where) {
 }
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// The rotation of a call: the Hadamard rotation (signs) or none, or the SRFT
+// variant (srft: signs, optional per-coordinate scales of K and V).
+struct Rotation {
+  bool srft = false;
+  const float* lambda_k = nullptr;
+  const float* lambda_v = nullptr;
+};
+
+static bool head_dim_ok(int d, const Rotation& rot) {
+  return rot.srft ? srft_head_dim_supported(d) : (d == 128 || d == 256);
+}
 
 }  // namespace tq
 
@@ -72,18 +90,22 @@ const char* tq_status_string(tq_status status) {
   return "unknown status";
 }
 
-tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
-                             int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
-                             int32_t group, const int32_t* pos, const int8_t* signs,
-                             uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
-                             float* v_scales, int64_t capacity, void* cuda_stream) {
+}  // extern "C"
+
+static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                               int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                               int32_t group, const int32_t* pos, const int8_t* signs,
+                               const Rotation& rot, uint8_t* k_packed, float* k_scales,
+                               uint8_t* v_packed, float* v_scales, int64_t capacity,
+                               void* cuda_stream, const char* where) {
   if (!k || !v || !pos || !k_packed || !k_scales || !v_packed || !v_scales) return TQ_ERR_INVALID_ARG;
   if (in_dtype != TQ_F32 && in_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
   if (batch < 1 || num_kv_heads < 1 || n_new < 1 || capacity < n_new) return TQ_ERR_INVALID_ARG;
-  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_packed) || !aligned16(v_packed) ||
-      !aligned16(k_scales) || !aligned16(v_scales))
+      !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(rot.lambda_k) ||
+      !aligned4(rot.lambda_v))
     return TQ_ERR_INVALID_ARG;
   QuantizeArgs a;
   a.k = k;
@@ -100,8 +122,33 @@ tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, in
   a.v_packed = v_packed;
   a.v_scales = v_scales;
   a.capacity = capacity;
-  return cuda_status(launch_quantize(a, static_cast<cudaStream_t>(cuda_stream)),
-                     "tq_quantize_append");
+  a.lambda_k = rot.lambda_k;
+  a.lambda_v = rot.lambda_v;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  return cuda_status(rot.srft ? launch_quantize_srft(a, s) : launch_quantize(a, s), where);
+}
+
+extern "C" {
+
+tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                             int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                             int32_t group, const int32_t* pos, const int8_t* signs,
+                             uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                             float* v_scales, int64_t capacity, void* cuda_stream) {
+  return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs,
+                       Rotation{}, k_packed, k_scales, v_packed, v_scales, capacity, cuda_stream,
+                       "tq_quantize_append");
+}
+
+tq_status tq_quantize_append_srft(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                                  int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                                  int32_t group, const int32_t* pos, const int8_t* signs,
+                                  const float* lambda_k, const float* lambda_v,
+                                  uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                                  float* v_scales, int64_t capacity, void* cuda_stream) {
+  return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs,
+                       Rotation{true, lambda_k, lambda_v}, k_packed, k_scales, v_packed,
+                       v_scales, capacity, cuda_stream, "tq_quantize_append_srft");
 }
 
 tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_seq, int32_t rows,
@@ -110,7 +157,7 @@ tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_se
   if (!packed || !scales || !out) return TQ_ERR_INVALID_ARG;
   if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
   if (n_seq < 1 || rows < 1 || row_stride < rows) return TQ_ERR_INVALID_ARG;
-  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (!srft_head_dim_supported(head_dim)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(out)) return TQ_ERR_INVALID_ARG;
   DequantizeArgs a;
@@ -132,6 +179,13 @@ size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
   return p.ws_bytes;
 }
 
+size_t tq_decode_srft_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t max_ctx) {
+  DecodePlan p;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p, true)) return 0;
+  return p.ws_bytes;
+}
+
 int32_t tq_decode_chunk_tokens(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                int32_t head_dim, int32_t max_ctx) {
   DecodePlan p;
@@ -150,7 +204,8 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
                              const uint8_t* v_packed, const float* v_scales, int64_t capacity,
                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
                              float attn_scale, float* out, void* workspace, size_t workspace_bytes,
-                             void* cuda_stream, const char* where, float* lse = nullptr) {
+                             void* cuda_stream, const char* where, float* lse = nullptr,
+                             const Rotation& rot = Rotation{}) {
   if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
     return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
@@ -163,14 +218,15 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     return TQ_ERR_INVALID_ARG;
   if (max_ctx < 1 || capacity < max_ctx) return TQ_ERR_INVALID_ARG;
   if (!(attn_scale > 0.0f) || !isfinite(attn_scale)) return TQ_ERR_INVALID_ARG;
-  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (num_q_heads / num_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(v_packed) ||
-      !aligned16(k_scales) || !aligned16(v_scales) || (lse && (reinterpret_cast<uintptr_t>(lse) & 7u)))
+      !aligned16(k_scales) || !aligned16(v_scales) || (lse && (reinterpret_cast<uintptr_t>(lse) & 7u)) ||
+      !aligned4(rot.lambda_k) || !aligned4(rot.lambda_v))
     return TQ_ERR_INVALID_ARG;
   DecodeArgs a;
-  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan))
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan, rot.srft))
     return TQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < a.plan.ws_bytes) return TQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
@@ -195,9 +251,14 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   a.v_new = nullptr;
   a.kv_bf16 = kv_dtype == TQ_BF16;
   a.lse = lse;
+  a.lambda_k = rot.lambda_k;
+  a.lambda_v = rot.lambda_v;
+  a.q_rot = rot.srft ? reinterpret_cast<const float*>(static_cast<unsigned char*>(workspace) +
+                                                      a.plan.qrot_offset)
+                     : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const bool mma = decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
-  if (append && mma) {  // the decode kernel quantizes the new tokens itself
+  if (append && mma && !rot.srft) {  // the decode kernel quantizes the new tokens itself
     a.k_new = k_new;
     a.v_new = v_new;
   } else if (append) {  // the CUDA-core decode: one small-append launch first
@@ -218,12 +279,18 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     qa.v_packed = const_cast<uint8_t*>(v_packed);
     qa.v_scales = const_cast<float*>(v_scales);
     qa.capacity = capacity;
-    const cudaError_t e = launch_quantize(qa, s);
+    qa.lambda_k = rot.lambda_k;
+    qa.lambda_v = rot.lambda_v;
+    const cudaError_t e = rot.srft ? launch_quantize_srft(qa, s) : launch_quantize(qa, s);
+    if (e != cudaSuccess) return cuda_status(e, where);
+  }
+  if (rot.srft) {  // rotated queries into the workspace, read by the decode kernel
+    const cudaError_t e = launch_srft_query(a, s);
     if (e != cudaSuccess) return cuda_status(e, where);
   }
   const cudaError_t e = mma ? launch_decode_mma(a, s) : launch_decode_simt(a, s);
   if (e != cudaSuccess) return cuda_status(e, where);
-  return cuda_status(launch_merge(a, s), where);
+  return cuda_status(rot.srft ? launch_merge_srft(a, s) : launch_merge(a, s), where);
 }
 
 extern "C" {
@@ -259,12 +326,40 @@ tq_status tq_merge_lse(const float* outs, const float* lses, int32_t n_parts, in
                        int32_t num_q_heads, int32_t head_dim, float* out, void* cuda_stream) {
   if (!outs || !lses || !out) return TQ_ERR_INVALID_ARG;
   if (n_parts < 1 || batch < 1 || num_q_heads < 1 || head_dim < 1) return TQ_ERR_INVALID_ARG;
-  if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+  if (!srft_head_dim_supported(head_dim)) return TQ_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(lses) & 7u) || !aligned16(outs) || !aligned16(out))
     return TQ_ERR_INVALID_ARG;
   return cuda_status(launch_merge_lse(outs, lses, n_parts, (int64_t)batch * num_q_heads, head_dim,
                                       out, static_cast<cudaStream_t>(cuda_stream)),
                      "tq_merge_lse");
+}
+
+tq_status tq_sdpa_int4_decode_srft(const void* q, tq_dtype q_dtype, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t group, const uint8_t* k_packed, const float* k_scales,
+                                   const uint8_t* v_packed, const float* v_scales,
+                                   int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx,
+                                   const int8_t* signs, const float* lambda_k,
+                                   const float* lambda_v, float attn_scale, float* out,
+                                   void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode_srft", nullptr, Rotation{true, lambda_k, lambda_v});
+}
+
+tq_status tq_sdpa_int4_decode_append_srft(
+    const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
+    uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales, int64_t capacity,
+    const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, const float* lambda_k,
+    const float* lambda_v, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+    void* cuda_stream) {
+  if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
+  return decode_impl(q, q_dtype, k_new, v_new, kv_dtype, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode_append_srft", nullptr, Rotation{true, lambda_k, lambda_v});
 }
 
 tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,

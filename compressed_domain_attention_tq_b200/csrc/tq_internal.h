@@ -18,10 +18,14 @@ struct DecodePlan {
   int n_chunks;     // ceil(max_ctx / chunk)
   int part_stride;  // floats per (b, q head, chunk) partial: d + 4 (16-byte rows)
   size_t header_bytes;  // int32 flags[B], rounded up to 256 bytes
-  size_t ws_bytes;  // header + partials
+  size_t qrot_offset;   // SRFT variant: rotated queries float[B][Hq][d] at this offset (else 0)
+  size_t ws_bytes;  // header + partials (+ rotated queries)
 };
 
-bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan);
+// srft: the SRFT variant's plan (any head_dim accepted by srft_head_dim_supported,
+// plus room for the rotated queries); otherwise head_dim 128 or 256.
+bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan,
+                      bool srft = false);
 
 struct QuantizeArgs {
   const void* k;
@@ -37,6 +41,8 @@ struct QuantizeArgs {
   int64_t capacity;
   int pos_is_ctx = 0;  // 1: token n of sequence b goes to row clamp(pos[b], 1, max_ctx) - 1 + n
   int max_ctx = 0;
+  const float* lambda_k = nullptr;  // SRFT variant: per-coordinate scales (NULL = ones)
+  const float* lambda_v = nullptr;
 };
 
 struct DequantizeArgs {
@@ -68,6 +74,10 @@ struct DecodeArgs {
   const void* v_new;
   int kv_bf16;
   float* lse;  // NULL, or [B][Hq][2]: each head's (max in log2 units, sum) for merging contexts
+  const float* q_rot = nullptr;     // SRFT variant: [B][Hq][d] rotated queries F(sigma q)/lambda_K;
+                                    // the decode kernels read these instead of rotating q
+  const float* lambda_k = nullptr;  // SRFT variant: per-coordinate scales (NULL = ones)
+  const float* lambda_v = nullptr;
 };
 
 // Raise a kernel's dynamic shared memory limit once per device (the first
@@ -92,6 +102,10 @@ bool decode_mma_supported(int d, int G);
 int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+bool srft_head_dim_supported(int d);
+cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream);
+cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_lse(const float* outs, const float* lses, int n_parts, int64_t n_heads,
                              int d, float* out, cudaStream_t stream);
 

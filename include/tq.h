@@ -28,7 +28,8 @@
  *  - Results are deterministic: the same inputs give bit-identical outputs.
  *
  * Data layout (row-major, dense):
- *  - head_dim d in {128, 256}; group size g = 32; ng = d / 32 groups.
+ *  - head_dim d in {128, 256} (the SRFT calls below: any multiple of 32 up to
+ *    256); group size g = 32; ng = d / 32 groups.
  *  - packed cache: uint8 [B][Hkv][capacity][d/2], one row per token.  Rotated
  *    coordinate i (group gi = i/32, in-group j = i%32) is stored as a 4-bit
  *    two's-complement code in byte (j/4)*(2*ng) + 2*gi + (j%4)/2 of its row,
@@ -218,7 +219,7 @@ TQ_API tq_status tq_sdpa_int4_decode_lse(
  *        [n_parts][B][Hq][2] (8-byte aligned), out float [B][Hq][d]
  *        (16-byte aligned; may not alias outs).
  * Returns TQ_ERR_INVALID_ARG for NULL or misaligned pointers or sizes < 1,
- * TQ_ERR_UNSUPPORTED for head_dim not in {128, 256}.
+ * TQ_ERR_UNSUPPORTED for head_dim not a multiple of 32 in [32, 256].
  */
 TQ_API tq_status tq_merge_lse(const float* outs, const float* lses, int32_t n_parts, int32_t batch,
                               int32_t num_q_heads, int32_t head_dim, float* out, void* cuda_stream);
@@ -270,11 +271,70 @@ TQ_API tq_status tq_sdpa_int4_decode_static_scratch(
  *
  * Returns TQ_ERR_INVALID_ARG for NULL pointers, n_seq or rows < 1,
  * row_stride < rows, misaligned pointers (16 bytes); TQ_ERR_UNSUPPORTED for
- * head_dim not in {128, 256} or group != 32.
+ * head_dim not a multiple of 32 in [32, 256] or group != 32.
  */
 TQ_API tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_seq,
                                int32_t rows, int64_t row_stride, int32_t head_dim, int32_t group,
                                void* out, tq_dtype out_dtype, void* cuda_stream);
+
+/*
+ * SRFT variant of the rotation ("SRFT + int4 KV-cache on Apple Silicon",
+ * core method: a sign-randomized Fourier transform in place of the Hadamard
+ * one, suited to widths that are not powers of two, then a per-coordinate
+ * scale lambda before the group abs-max quantization).  The transform is the
+ * orthonormal discrete Hartley transform
+ *     F[k][j] = (cos(2 pi k j / d) + sin(2 pi k j / d)) / sqrt(d),
+ * the real member of the Fourier family (F = F^T, F F = I).  A cache written
+ * by tq_quantize_append_srft holds, for every token,
+ *     K row: y = lambda_k (.) F (signs (.) k),   V row: lambda_v (.) F (signs (.) v)
+ * in the packed layout above, and the SRFT decode calls use
+ *     q_r = F (signs (.) q) / lambda_k,   out = signs (.) F (o_r / lambda_v),
+ * so q_r . y = q . k and the output is in the unrotated basis.
+ *
+ *  head_dim      any multiple of 32 from 32 to 256 (e.g. 96, 160, 192).
+ *  signs         int8 [d] of +1/-1 (device), or NULL for all +1.
+ *  lambda_k/_v   float [d] (device, 4-byte aligned) of positive finite values,
+ *                or NULL for all 1.  Values are not checked on the device.
+ * The cache, q, k/v and out layouts, alignment, ownership and errors are those
+ * of the Hadamard calls; head_dim outside the set above gives
+ * TQ_ERR_UNSUPPORTED, a misaligned lambda TQ_ERR_INVALID_ARG.  A cache must be
+ * read with the rotation (signs, lambdas) it was written with.
+ */
+
+/* Workspace bytes for tq_sdpa_int4_decode_srft(_append): the split-K partials
+ * plus the rotated queries (4 * B * Hq * d bytes); 0 for invalid sizes. */
+TQ_API size_t tq_decode_srft_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t head_dim,
+                                             int32_t max_ctx);
+
+/* tq_quantize_append with the SRFT rotation (one complex FFT per token turns
+ * its K and V rows together). */
+TQ_API tq_status tq_quantize_append_srft(
+    const void* k, const void* v, tq_dtype in_dtype, int32_t batch, int32_t num_kv_heads,
+    int32_t n_new, int32_t head_dim, int32_t group, const int32_t* pos, const int8_t* signs,
+    const float* lambda_k, const float* lambda_v, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, void* cuda_stream);
+
+/* tq_sdpa_int4_decode over an SRFT cache.  Launches: one query-rotation
+ * kernel, the split-K decode (tensor cores for head_dim 128 with Hq/Hkv <= 8
+ * and head_dim 256 with Hq/Hkv <= 4, CUDA cores otherwise) and the merge with
+ * the inverse transform.  workspace_bytes >= tq_decode_srft_workspace_bytes(). */
+TQ_API tq_status tq_sdpa_int4_decode_srft(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, const uint8_t* k_packed, const float* k_scales,
+    const uint8_t* v_packed, const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, const float* lambda_k, const float* lambda_v,
+    float attn_scale, float* out, void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* tq_sdpa_int4_decode_append over an SRFT cache: the new tokens are quantized
+ * by a tq_quantize_append_srft launch, then the query attends. */
+TQ_API tq_status tq_sdpa_int4_decode_append_srft(
+    const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
+    uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales, int64_t capacity,
+    const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, const float* lambda_k,
+    const float* lambda_v, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+    void* cuda_stream);
 
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);

@@ -148,8 +148,9 @@ def test_decode_rejects_on_host(lib, kw, code):
     (dict(packed=None), _lib.TQ_ERR_INVALID_ARG), (dict(scales=None), _lib.TQ_ERR_INVALID_ARG),
     (dict(out=None), _lib.TQ_ERR_INVALID_ARG), (dict(dtype=3), _lib.TQ_ERR_INVALID_ARG),
     (dict(n_seq=0), _lib.TQ_ERR_INVALID_ARG), (dict(rows=0), _lib.TQ_ERR_INVALID_ARG),
-    (dict(rows=65, stride=64), _lib.TQ_ERR_INVALID_ARG), (dict(d=64), _lib.TQ_ERR_UNSUPPORTED),
-    (dict(group=16), _lib.TQ_ERR_UNSUPPORTED), (dict(out=8), _lib.TQ_ERR_INVALID_ARG)])
+    (dict(rows=65, stride=64), _lib.TQ_ERR_INVALID_ARG), (dict(d=80), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(d=288), _lib.TQ_ERR_UNSUPPORTED), (dict(group=16), _lib.TQ_ERR_UNSUPPORTED),
+    (dict(out=8), _lib.TQ_ERR_INVALID_ARG)])
 def test_dequantize_rejects_on_host(lib, kw, code):
     fb = FakeBuffers()
     a = dict(packed=fb.p(1024), scales=fb.p(2048), n_seq=2, rows=64, stride=64, d=128, group=32,
@@ -186,7 +187,7 @@ def test_lse_calls_reject_on_host(lib):
     # merge: NULL, sizes, head_dim, misaligned
     assert lib.tq_merge_lse(None, fb.p(0), 2, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
     assert lib.tq_merge_lse(fb.p(0), fb.p(2048), 0, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
-    assert lib.tq_merge_lse(fb.p(0), fb.p(2048), 2, 1, 8, 64, fb.p(4096), None) == _lib.TQ_ERR_UNSUPPORTED
+    assert lib.tq_merge_lse(fb.p(0), fb.p(2048), 2, 1, 8, 80, fb.p(4096), None) == _lib.TQ_ERR_UNSUPPORTED
     assert lib.tq_merge_lse(fb.p(0), fb.p(2052), 2, 1, 8, 128, fb.p(4096), None) == _lib.TQ_ERR_INVALID_ARG
     # decode_lse: NULL lse, misaligned lse
     for lse in (None, fb.p(20484)):

@@ -41,7 +41,7 @@ def run_gpu(k, v, pos, signs, cap):
     return [t.cpu().numpy() for t in (kp, ks, vp, vs)]
 
 
-def compare(gpu, ref, d, rot, label):
+def compare(gpu, ref, d, rot, label, max_scale_ulp=4):
     kp, ks, vp, vs = gpu
     rkp, rks, rvp, rvs = ref
     if not rot:
@@ -61,7 +61,7 @@ def compare(gpu, ref, d, rot, label):
     assert n_diff <= 1e-4 * n_tot, f"{label}: {n_diff}/{n_tot} codes differ"
     for a, b in ((ks, rks), (vs, rvs)):
         ulp = np.abs(a.view(np.int32).astype(np.int64) - b.view(np.int32).astype(np.int64))
-        assert ulp.max() <= 4, f"{label}: scale ulp {ulp.max()}"
+        assert ulp.max() <= max_scale_ulp, f"{label}: scale ulp {ulp.max()}"
     return n_diff, n_tot
 
 
