@@ -75,16 +75,16 @@ def lib_source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
+def ncu_traffic(kernel_key, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current kernel sources and this workload (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_hash") != lib_source_hash():
+    if not e or e.get("source_hash") != lib_source_hash() or e.get("workload_name") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -165,8 +165,11 @@ def run_tq(args):
     stream = torch.cuda.current_stream()
 
     signs = wl.make_signs(d, seed) if w.rotation else None
+    srft = w.rotation and w.rotation_kind == "srft"
+    lk, lv = wl.make_lambdas(w, seed)
     ctx = wl.make_context_lengths(w, seed)                    # cached tokens per sequence
-    cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
+    cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs,
+                           rotation="srft" if srft else "hadamard", lambda_k=lk, lambda_v=lv)
     k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
     pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -313,7 +316,8 @@ def run_tq(args):
     if rank == 0:
         import numpy as np
         cache.decode(q, ctx_dev, max_ctx, scale, out)
-        bl = dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, cache.signs,
+        Qm, Om = basis_maps(d, signs, lk, lv, srft, dev)
+        bl = dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, Qm, Om,
                                      min(args.steps, 50), 3, stream)
         o_ours, o_bl = out.double().flatten(1), bl.pop("out").double().flatten(1)
         bl["cosine_vs_int4_path_min"] = round(float(torch.nn.functional.cosine_similarity(
@@ -326,11 +330,24 @@ def run_tq(args):
         fid_v = np.concatenate([fid_v.numpy(), v_new[0, :n_fid].float().cpu().numpy()], 1)
         fid = fidelity(fid_k, fid_v, q[0, :n_fid * G].float().cpu().numpy(),
                        out[0, :n_fid * G].cpu().numpy(), khat[0, :n_fid].cpu().numpy(),
-                       None if cache.signs is None else cache.signs.cpu(), scale, G)
+                       Qm.cpu().numpy(), scale, G)
         fid["sample"] = f"sequence 0, kv heads 0..{n_fid - 1} ({n_fid * G} query heads), {ctx0 + 1} tokens"
         del khat
 
     kvb = kv_bytes(w, (ctx + 1).tolist())
+    mma = (d == 128 and Hq // Hkv <= 8) or (d == 256 and Hq // Hkv <= 4)
+    if srft:
+        launches_per_step = 4
+        step_desc = ("tq_sdpa_int4_decode_append_srft: SRFT quantize-append of the new token, query "
+                     "rotation, split-K decode, merge with the inverse transform (4 launches)")
+    elif mma:
+        launches_per_step = 2
+        step_desc = ("tq_sdpa_int4_decode_append: the decode kernel quantizes the new token of each "
+                     "kv head into the cache, then attends (split-K kernel + merge, 2 launches)")
+    else:
+        launches_per_step = 3
+        step_desc = ("tq_sdpa_int4_decode_append: quantize-append of the new token, split-K "
+                     "decode, merge (3 launches)")
     qo_bytes = q.numel() * q.element_size() + out.numel() * out.element_size()
     algo = kvb + qo_bytes
     peak, peak_kind = measured_peaks()
@@ -346,7 +363,9 @@ def run_tq(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 codes, fp32 accumulation", "data": "synthetic (seeded N(0,1), bf16)",
         "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
-                   "context": max_ctx, "rotation": w.rotation, "attn_scale": scale,
+                   "context": max_ctx,
+                   "rotation": (w.rotation_kind if w.rotation else False),
+                   "attn_scale": scale,
                    "kv_bytes_per_step": kvb,
                    "l2": (f"flushed by a {flush.numel()} B write before each step inside the "
                           f"graph; its separately timed cost is subtracted") if use_flush else
@@ -356,14 +375,13 @@ def run_tq(args):
         "roofline": {"bound": "hbm", "kernel": "sdpa_int4 decode (split-K + merge)",
                      "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4), "peak_kind": peak_kind,
-                     "algorithmic_bytes": algo, "traffic": ncu_traffic("decode")},
+                     "algorithmic_bytes": algo, "traffic": ncu_traffic("decode", w.name)},
         "e2e": {"value": round(world * kvb / e2e_s / 1e9, 1), "unit": "GB/s",
                 "us_per_step": round(e2e_s * 1e6, 2),
                 "h2d_bytes_per_step": int(h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()),
                 "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())},
-        "gpu_launches": 2 * args.steps,
-        "step": ("tq_sdpa_int4_decode_append: the decode kernel quantizes the new token of each "
-                 "kv head into the cache, then attends (split-K kernel + merge, 2 launches)"),
+        "gpu_launches": launches_per_step * args.steps,
+        "step": step_desc,
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
                   "launching stream (decode split from a K-decode graph; the two-call step "
                   "from a third graph); e2e: public API calls with pinned host copies, per step",
@@ -392,12 +410,30 @@ def rotation_matrix(d, signs, device):
     return (H * signs.double().cpu()[None, :] / math.sqrt(d)).to(device)
 
 
-def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, signs, steps, warmup, stream):
+def basis_maps(d, signs, lk, lv, srft, device):
+    """(Qm, Om), fp64 on `device`: q_r = Qm q takes a query into the cache's basis and
+    o = Om o_r takes an output back.  Hadamard: R and R^T.  SRFT: diag(1/lambda_k) F
+    diag(signs) and diag(signs) F diag(1/lambda_v), F the orthonormal Hartley matrix
+    (Re - Im of the unitary DFT matrix)."""
+    import torch
+    if not srft:
+        R = rotation_matrix(d, signs, device)
+        return R, R.T.contiguous()
+    X = torch.fft.fft(torch.eye(d, dtype=torch.float64), dim=0)
+    F = (X.real - X.imag) / math.sqrt(d)
+    one = torch.ones(d, dtype=torch.float64)
+    s = one if signs is None else signs.double().cpu()
+    ik = one if lk is None else 1.0 / lk.double().cpu()
+    iv = one if lv is None else 1.0 / lv.double().cpu()
+    return ((ik[:, None] * F * s[None, :]).to(device), (s[:, None] * F * iv[None, :]).to(device))
+
+
+def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, Qm, Om, steps, warmup, stream):
     """In-house bf16 dequantize-then-attend on the same GPU: every step
     materializes bf16 K and V from the packed cache (tq_dequantize, one pass)
     and runs torch's bf16 scaled_dot_product_attention over them (query rotated
-    into the cache basis, output rotated back).  Also times the attention alone
-    on the materialized bf16 cache (what a bf16 KV cache would cost)."""
+    into the cache basis by Qm, output back by Om).  Also times the attention
+    alone on the materialized bf16 cache (what a bf16 KV cache would cost)."""
     import torch
     import torch.nn.functional as F
 
@@ -405,7 +441,7 @@ def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, signs, steps, war
     B, Hq, d = q.shape
     Hkv = cache.k_packed.shape[1]
     dev = q.device
-    R = rotation_matrix(d, signs, dev).float()
+    Qf, Of = Qm.float(), Om.float()
     Kb = torch.empty(B, Hkv, max_ctx, d, dtype=torch.bfloat16, device=dev)
     Vb = torch.empty_like(Kb)
     lens = ctx_dev.long()
@@ -415,9 +451,9 @@ def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, signs, steps, war
     out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
 
     def attend():
-        qr = (q.float() @ R.T).to(torch.bfloat16)[:, :, None, :]
+        qr = (q.float() @ Qf.T).to(torch.bfloat16)[:, :, None, :]
         o = F.scaled_dot_product_attention(qr, Kb, Vb, attn_mask=mask, scale=scale, enable_gqa=True)
-        out.copy_(o[:, :, 0].float() @ R)
+        out.copy_(o[:, :, 0].float() @ Of.T)
 
     def full():
         _lib.dequantize(cache.k_packed, cache.k_scales, max_ctx, Kb)
@@ -447,17 +483,15 @@ def dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, signs, steps, war
     return res
 
 
-def fidelity(k_h, v_h, q_h, out_h, khat_h, signs, scale, G):
+def fidelity(k_h, v_h, q_h, out_h, khat_h, Qm, scale, G):
     """Fidelity of the int4 path to unquantized fp64 attention (report only).
 
     k_h, v_h [n][T][d] unquantized (unrotated) inputs of n kv heads; q_h [n*G][d];
     out_h [n*G][d] the CUDA path's output; khat_h [n][T][d] dequantized keys
-    (rotated basis).  Cosine similarity of each query head's output with exact
+    (cache basis); Qm the query's map into that basis.  Cosine similarity of each query head's output with exact
     softmax attention, and agreement of argmax_t q.k between the unquantized
     and the dequantized keys."""
     import numpy as np
-    d = k_h.shape[-1]
-    R = rotation_matrix(d, signs, "cpu").numpy()
     cos, agree = [], []
     for h in range(k_h.shape[0]):
         K, V = k_h[h].astype(np.float64), v_h[h].astype(np.float64)
@@ -467,7 +501,7 @@ def fidelity(k_h, v_h, q_h, out_h, khat_h, signs, scale, G):
         O = (P.T @ V) / P.sum(0)[:, None]
         Og = out_h[h * G:(h + 1) * G].astype(np.float64)
         cos += list((O * Og).sum(1) / (np.linalg.norm(O, axis=1) * np.linalg.norm(Og, axis=1)))
-        Sq = khat_h[h].astype(np.float64) @ (Q @ R.T).T
+        Sq = khat_h[h].astype(np.float64) @ (Q @ Qm.T).T
         agree += list(S.argmax(0) == Sq.argmax(0))
     return {"cosine_min": round(float(min(cos)), 7), "cosine_mean": round(float(np.mean(cos)), 7),
             "top1_qk_argmax_agreement": round(float(np.mean(agree)), 4), "query_heads": len(cos)}
@@ -492,20 +526,35 @@ def oracle_sample(w, seed, kv_head=0):
         return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
 
     signs = wl.make_signs(w.head_dim, seed).numpy() if w.rotation else None
+    lk, lv = wl.make_lambdas(w, seed)
+    lam = None if lk is None else (lk.numpy(), lv.numpy())
     cache = oracle.empty_cache(1, 1, w.capacity, w.head_dim)
     thr = oracle.max_threads()
+    s = dict(k_new=bits(k[:, :, -1:]), v_new=bits(v[:, :, -1:]), q=bits(q), signs=signs, lam=lam,
+             cache=cache, threads=thr, G=G, T=w.capacity - 1)
     t0 = time.perf_counter()
-    oracle.quantize_append(bits(k[:, :, :-1]), bits(v[:, :, :-1]), [0], signs, cache, threads=thr)
-    t_q = time.perf_counter() - t0
-    return dict(k_new=bits(k[:, :, -1:]), v_new=bits(v[:, :, -1:]), q=bits(q), signs=signs,
-                cache=cache, threads=thr, prefill_s=t_q, G=G, T=w.capacity - 1)
+    oracle_append(s, bits(k[:, :, :-1]), bits(v[:, :, :-1]), 0)
+    s["prefill_s"] = time.perf_counter() - t0
+    return s
+
+
+def oracle_append(s, k, v, pos):
+    import oracle
+    if s["lam"] is None:
+        oracle.quantize_append(k, v, [pos], s["signs"], s["cache"], threads=s["threads"])
+    else:
+        oracle.quantize_append_srft(k, v, [pos], s["signs"], s["lam"][0], s["lam"][1], s["cache"],
+                                    threads=s["threads"])
 
 
 def oracle_step(s, w):
     import oracle
-    oracle.quantize_append(s["k_new"], s["v_new"], [s["T"]], s["signs"], s["cache"], threads=s["threads"])
-    return oracle.sdpa_int4_decode(s["q"], s["cache"], [s["T"] + 1], s["signs"], w.attn_scales[0], 1,
-                                   threads=s["threads"])
+    oracle_append(s, s["k_new"], s["v_new"], s["T"])
+    if s["lam"] is None:
+        return oracle.sdpa_int4_decode(s["q"], s["cache"], [s["T"] + 1], s["signs"],
+                                       w.attn_scales[0], 1, threads=s["threads"])
+    return oracle.sdpa_int4_decode_srft(s["q"], s["cache"], [s["T"] + 1], s["signs"], s["lam"][0],
+                                        s["lam"][1], w.attn_scales[0], 1, threads=s["threads"])
 
 
 def cpu_baseline(w, seed):

@@ -381,6 +381,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     if (h < G) {
       const int64_t base = ((int64_t)b * a.Hq + (int64_t)kvh * G + h) * D + lane * E;
       if (a.q_rot != nullptr) {  // SRFT variant: the query is already rotated (fp32)
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // by the preceding grid
 #pragma unroll
         for (int e = 0; e < E; e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(a.q_rot + base + e);
@@ -1007,6 +1008,19 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   const int grid = n_items < sms ? n_items : sms;
+  if (a.q_rot != nullptr) {  // overlap the query-rotation grid (see prep_query)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<D, PATH>, a);
+  }
   decode_mma_kernel<D, PATH><<<grid, C::THREADS, C::BYTES, stream>>>(a);
   return cudaGetLastError();
 }

@@ -22,13 +22,29 @@ namespace tq {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kTile = 64;
+constexpr int kTile = 64;      // tokens per shared-memory tile
+constexpr int kThreads = 128;
 
-// code of in-group coordinate j of group g in a packed row (d = 32*ng)
-__device__ __forceinline__ int nibble_at(const uint8_t* row, int ng, int g, int j) {
-  const int byte = (j / 4) * (2 * ng) + 2 * g + (j % 4) / 2;
-  const int v = (row[byte] >> (4 * (j % 2))) & 0xF;
-  return v >= 8 ? v - 16 : v;
+// Token parts of the P.V work: the (head, 8-dim slice) items are split over
+// TP interleaved token subsets while that keeps at most 2 items per thread,
+// so small G (MHA) still occupies every thread; the parts are summed once per
+// chunk.  Shared by the host (shared-memory size) and the kernel.
+__host__ __device__ constexpr int simt_token_parts(int G, int slices) {
+  int tp = 1;
+  while (tp < 16 && G * slices * tp * 2 <= 2 * kThreads) tp *= 2;
+  return tp;
+}
+
+// Row pitch of a staged packed row in 32-bit words: odd, so lanes reading the
+// same offset of consecutive rows hit distinct banks.
+template <int D>
+__host__ __device__ constexpr int simt_pitch_words() { return D / 8 + 1; }
+
+// the 4 codes of a 16-bit half-word (in-group coordinates 4r .. 4r+3 of one group)
+__device__ __forceinline__ float code_of(uint32_t hw, int m) {
+  // u = nibble; (u ^ 8) | 2^23 as a float is 2^23 + 8 + c for the two's-complement code c
+  const uint32_t u = (hw >> (4 * m)) & 0xFu;
+  return __int_as_float((int)(u ^ 0x4B000008u)) - 8388616.0f;
 }
 
 // In-place Walsh-Hadamard transform of `n` rows of length D in shared memory
@@ -54,17 +70,24 @@ __device__ __forceinline__ float load_q(const void* q, int bf16, int64_t idx) {
   return static_cast<const float*>(q)[idx];
 }
 
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+
 __device__ __forceinline__ int clamp_ctx(int T, int max_ctx) {
   return T < 1 ? 1 : (T > max_ctx ? max_ctx : T);
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
-  constexpr int NG = D / 32, ROWB = D / 2, ROWP = ROWB + 16;
+__global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
+  constexpr int NG = D / 32;
+  constexpr int PW = simt_pitch_words<D>();     // staged row pitch (words)
   constexpr int SLICES = D / 8;                 // 8-coordinate slices per head
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int G = a.Hq / a.Hkv;
+  const int TP = simt_token_parts(G, SLICES);
   const int raw_T = a.ctx_lens[b];
   const int T = clamp_ctx(raw_T, a.max_ctx);
   if (chunk == 0 && kvh == 0 && threadIdx.x == 0)
@@ -76,18 +99,18 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   float* qs = reinterpret_cast<float*>(smem);                  // [G][D]
   float* sp = qs + G * D;                                      // [G][kTile] scores / probs
-  float* kscale = sp + G * kTile;                              // [kTile][NG]
-  float* vscale = kscale + kTile * NG;                         // [kTile][NG]
-  float* mstate = vscale + kTile * NG;                         // [G] running max (log2)
+  float* scl = sp + G * kTile;                                 // [2 buffers][K, V][kTile][NG]
+  float* mstate = scl + 4 * kTile * NG;                        // [G] running max (log2)
   float* lstate = mstate + 16;                                 // [G] running sum
   float* alpha = lstate + 16;                                  // [G] rescale of this tile
-  uint8_t* ktile = reinterpret_cast<uint8_t*>(alpha + 16);     // [kTile][ROWP]
-  uint8_t* vtile = ktile + kTile * ROWP;
+  float* red = alpha + 16;                                     // [TP][G][D] (TP > 1)
+  // [2 buffers][K, V][kTile][PW] staged packed rows
+  uint32_t* tiles = reinterpret_cast<uint32_t*>(red + (TP > 1 ? TP * G * D : 0));
 
   // q' = attn_scale * log2(e) * R q (the SRFT variant's R q comes rotated in q_rot)
   const int64_t qbase = ((int64_t)b * a.Hq + (int64_t)kvh * G) * D;
   const bool wht = a.signs != nullptr && a.q_rot == nullptr;
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+  for (int i = threadIdx.x; i < G * D; i += kThreads) {
     float x;
     if (a.q_rot != nullptr) {
       x = a.q_rot[qbase + i];
@@ -102,57 +125,83 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
   }
   const float qmul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
   __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) qs[i] *= qmul;
+  for (int i = threadIdx.x; i < G * D; i += kThreads) qs[i] *= qmul;
   if (threadIdx.x < 16) {
     mstate[threadIdx.x] = -INFINITY;
     lstate[threadIdx.x] = 0.0f;
   }
 
-  // PV work items: (head, 8-coordinate slice); at most 4 per thread.
-  const int items = G * SLICES;
+  // P.V work items (head h, token part tp, slice sl), sl fastest; at most 4 per thread
+  const int items = G * SLICES * TP;
   float acc[4][8];
 #pragma unroll
   for (int it = 0; it < 4; ++it)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[it][e] = 0.0f;
+  // score parts: two threads per token when there is a single head
+  const int SP = G == 1 ? 2 : 1;
 
   const int64_t rowbase = ((int64_t)b * a.Hkv + kvh) * a.capacity;
-  for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
+  // Tiles are staged by 4-byte cp.async into two buffers: tile i + 1 is in
+  // flight while tile i is computed.
+  auto stage = [&](int t0, int buf) {
     const int nt = min(kTile, t_end - t0);
-    __syncthreads();
-    // stage the tile's packed rows and scales
-    for (int idx = threadIdx.x; idx < nt * (ROWB / 16); idx += blockDim.x) {
-      const int r = idx / (ROWB / 16), c = idx % (ROWB / 16);
-      const int64_t src = (rowbase + t0 + r) * ROWB + c * 16;
-      *reinterpret_cast<uint4*>(ktile + r * ROWP + c * 16) =
-          *reinterpret_cast<const uint4*>(a.k_packed + src);
-      *reinterpret_cast<uint4*>(vtile + r * ROWP + c * 16) =
-          *reinterpret_cast<const uint4*>(a.v_packed + src);
+    uint32_t* kt = tiles + buf * 2 * kTile * PW;
+    uint32_t* vt = kt + kTile * PW;
+    const uint32_t* kg = reinterpret_cast<const uint32_t*>(a.k_packed + (rowbase + t0) * (D / 2));
+    const uint32_t* vg = reinterpret_cast<const uint32_t*>(a.v_packed + (rowbase + t0) * (D / 2));
+    for (int idx = threadIdx.x; idx < nt * (D / 8); idx += kThreads) {
+      const int r = idx / (D / 8), w = idx % (D / 8);
+      cp_async4(kt + r * PW + w, kg + idx);
+      cp_async4(vt + r * PW + w, vg + idx);
     }
-    for (int idx = threadIdx.x; idx < nt * NG; idx += blockDim.x) {
-      kscale[idx] = a.k_scales[(rowbase + t0) * NG + idx];
-      vscale[idx] = a.v_scales[(rowbase + t0) * NG + idx];
+    float* ks = scl + buf * 2 * kTile * NG;
+    for (int idx = threadIdx.x; idx < nt * NG; idx += kThreads) {
+      cp_async4(ks + idx, a.k_scales + (rowbase + t0) * NG + idx);
+      cp_async4(ks + kTile * NG + idx, a.v_scales + (rowbase + t0) * NG + idx);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  stage(t_begin, 0);
+  int buf = 0;
+  for (int t0 = t_begin; t0 < t_end; t0 += kTile, buf ^= 1) {
+    const int nt = min(kTile, t_end - t0);
+    if (t0 + kTile < t_end) {  // the other buffer was released by the barrier ending the last tile
+      stage(t0 + kTile, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
+    const uint32_t* ktile = tiles + buf * 2 * kTile * PW;
+    const uint32_t* vtile = ktile + kTile * PW;
+    const float* kscale = scl + buf * 2 * kTile * NG;
+    const float* vscale = kscale + kTile * NG;
 
-    // scores: thread -> (token tt, heads hh, hh+2, ...)
-    {
-      const int tt = threadIdx.x % kTile, hh = threadIdx.x / kTile;
-      for (int h = hh; h < G; h += 2) {
-        float s = -INFINITY;
-        if (tt < nt) {
-          const uint8_t* row = ktile + tt * ROWP;
-          s = 0.0f;
-          for (int g = 0; g < NG; ++g) {
-            float dot = 0.0f;
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j)
-              dot = fmaf(qs[h * D + 32 * g + j], (float)nibble_at(row, NG, g, j), dot);
-            s = fmaf(kscale[tt * NG + g], dot, s);
+    // scores S[h][t] = sum_g s_k[t][g] sum_{j in g} c[t][j] q'[h][32 g + j]
+    for (int idx = threadIdx.x; idx < kTile * G * SP; idx += kThreads) {
+      const int part = SP == 2 ? (idx & 1) : 0;
+      const int tt = SP == 2 ? (idx >> 1) : idx % kTile;
+      const int h = SP == 2 ? 0 : idx / kTile;
+      float s = 0.0f;
+      if (tt < nt) {
+        const uint16_t* row = reinterpret_cast<const uint16_t*>(ktile + tt * PW);
+        const int r_lo = SP == 2 ? 4 * part : 0, r_hi = SP == 2 ? r_lo + 4 : 8;
+        for (int g = 0; g < NG; ++g) {
+          float dot = 0.0f;
+          for (int r = r_lo; r < r_hi; ++r) {
+            const uint32_t hw = row[r * NG + g];   // half-word at byte r * 2NG + 2g
+            const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + 32 * g + 4 * r);
+            dot = fmaf(qv.x, code_of(hw, 0), dot);
+            dot = fmaf(qv.y, code_of(hw, 1), dot);
+            dot = fmaf(qv.z, code_of(hw, 2), dot);
+            dot = fmaf(qv.w, code_of(hw, 3), dot);
           }
+          s = fmaf(kscale[tt * NG + g], dot, s);
         }
-        sp[h * kTile + tt] = s;
       }
+      if (SP == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);  // idx, idx ^ 1: the same token
+      if (part == 0) sp[h * kTile + tt] = tt < nt ? s : -INFINITY;
     }
     __syncthreads();
     // online softmax update: warp w handles heads w, w+4, ...
@@ -178,39 +227,65 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
       }
     }
     __syncthreads();
-    // P.V on the packed values
+    // P.V on the packed values: item (h, tp, sl) adds tokens tp, tp + TP, ... of the tile
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
-      const int item = threadIdx.x + it * 128;
+      const int item = threadIdx.x + it * kThreads;
       if (item < items) {
-        const int h = item / SLICES, sl = item % SLICES;
-        const int g = sl / 4, j0 = (sl % 4) * 8;
+        const int sl = item % SLICES, rest = item / SLICES;
+        const int tp = rest % TP, h = rest / TP;
+        const int g = sl / 4, r0 = (sl % 4) * 2;
         const float al = alpha[h];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[it][e] *= al;
-        for (int tt = 0; tt < nt; ++tt) {
+        for (int tt = tp; tt < nt; tt += TP) {
           const float pw = sp[h * kTile + tt] * vscale[tt * NG + g];
-          const uint8_t* row = vtile + tt * ROWP;
+          const uint16_t* row = reinterpret_cast<const uint16_t*>(vtile + tt * PW);
+          const uint32_t hw0 = row[r0 * NG + g], hw1 = row[(r0 + 1) * NG + g];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            acc[it][e] = fmaf(pw, (float)nibble_at(row, NG, g, j0 + e), acc[it][e]);
+          for (int m = 0; m < 4; ++m) {
+            acc[it][m] = fmaf(pw, code_of(hw0, m), acc[it][m]);
+            acc[it][4 + m] = fmaf(pw, code_of(hw1, m), acc[it][4 + m]);
+          }
         }
       }
     }
+    __syncthreads();  // the tile's buffers and scores are free for the next stage
   }
 
   // partials: ws[b][hq][chunk][0..D) = acc, [D] = m, [D+1] = l
   float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) + a.plan.header_bytes);
   const int stride = a.plan.part_stride;
+  if (TP == 1) {
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int item = threadIdx.x + it * 128;
-    if (item < items) {
-      const int h = item / SLICES, sl = item % SLICES;
+    for (int it = 0; it < 4; ++it) {
+      const int item = threadIdx.x + it * kThreads;
+      if (item < items) {
+        const int sl = item % SLICES, h = item / SLICES;
+        const int64_t hq = (int64_t)kvh * G + h;
+        float* dst = part + (((int64_t)b * a.Hq + hq) * a.plan.n_chunks + chunk) * stride;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[sl * 8 + e] = acc[it][e];
+      }
+    }
+  } else {  // sum the token parts in shared memory (fixed order: deterministic)
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int item = threadIdx.x + it * kThreads;
+      if (item < items) {
+        const int sl = item % SLICES, rest = item / SLICES;
+        const int tp = rest % TP, h = rest / TP;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[(tp * G + h) * D + sl * 8 + e] = acc[it][e];
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+      float v = 0.0f;
+      for (int tp = 0; tp < TP; ++tp) v += red[tp * G * D + i];
+      const int h = i / D, c = i % D;
       const int64_t hq = (int64_t)kvh * G + h;
-      float* dst = part + (((int64_t)b * a.Hq + hq) * a.plan.n_chunks + chunk) * stride;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[sl * 8 + e] = acc[it][e];
+      part[(((int64_t)b * a.Hq + hq) * a.plan.n_chunks + chunk) * stride + c] = v;
     }
   }
   __syncthreads();
@@ -224,22 +299,28 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeArgs a) {
 
 template <int D>
 size_t simt_smem_bytes(int G) {
-  constexpr int NG = D / 32, ROWP = D / 2 + 16;
-  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 2 * kTile * NG + 48) +
-         2 * (size_t)kTile * ROWP;
+  constexpr int NG = D / 32;
+  const int TP = simt_token_parts(G, D / 8);
+  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 48 +
+                          (TP > 1 ? (size_t)TP * G * D : 0)) +
+         4 * sizeof(uint32_t) * (size_t)kTile * simt_pitch_words<D>();
 }
 
+template <int D>
+size_t simt_smem_max() {  // over every group size the host accepts (up to 16 query heads)
+  size_t m = 0;
+  for (int G = 1; G <= 16; ++G) m = simt_smem_bytes<D>(G) > m ? simt_smem_bytes<D>(G) : m;
+  return m;
+}
 
 template <int D>
 cudaError_t launch_simt_d(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   dim3 grid(a.plan.n_chunks, a.Hkv, a.B);
   static std::atomic<uint64_t> smem_set{0};
-  // the limit covers every group size the host accepts (up to 16 query heads)
-  const cudaError_t e =
-      ensure_smem_limit(decode_simt_kernel<D>, (int)simt_smem_bytes<D>(16), smem_set);
+  const cudaError_t e = ensure_smem_limit(decode_simt_kernel<D>, (int)simt_smem_max<D>(), smem_set);
   if (e != cudaSuccess) return e;
-  decode_simt_kernel<D><<<grid, 128, simt_smem_bytes<D>(G), stream>>>(a);
+  decode_simt_kernel<D><<<grid, kThreads, simt_smem_bytes<D>(G), stream>>>(a);
   return cudaGetLastError();
 }
 

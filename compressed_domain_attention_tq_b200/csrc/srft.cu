@@ -115,6 +115,9 @@ __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArg
 template <int M>
 __global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
   constexpr int D = 32 * M;
+  // the decode kernel may start streaming the cache now; it waits for this
+  // grid (griddepcontrol.wait) before it reads the rotated queries
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pairs_per_b = (a.Hq + 1) / 2;
   const int64_t p = (int64_t)blockIdx.x * 4 + warp;
@@ -155,62 +158,59 @@ __global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
   }
 }
 
-// Log-sum-exp merge of one head's chunk partials (acc[i], m, l) for
-// coordinate i; returns acc / l and sets the head's (M, L).
-__device__ __forceinline__ float combine_chunks(const float* part, int nc, int stride, int d, int i,
-                                                float& Mx, float& L) {
-  Mx = -INFINITY;
-  for (int c = 0; c < nc; ++c) Mx = fmaxf(Mx, part[(int64_t)c * stride + d]);
-  constexpr int U = 4;
-  float acc[U], ls[U];
-#pragma unroll
-  for (int k = 0; k < U; ++k) acc[k] = ls[k] = 0.0f;
-  for (int c0 = 0; c0 < nc; c0 += U) {
-#pragma unroll
-    for (int k = 0; k < U; ++k)
-      if (c0 + k < nc) {
-        const float* pc = part + (int64_t)(c0 + k) * stride;
-        const float w = exp2f(pc[d] - Mx);
-        ls[k] = fmaf(w, pc[d + 1], ls[k]);
-        acc[k] = fmaf(w, pc[i], acc[k]);
-      }
-  }
-  L = (ls[0] + ls[2]) + (ls[1] + ls[3]);
-  return ((acc[0] + acc[2]) + (acc[1] + acc[3])) / L;
-}
-
 template <int M>
 __global__ void __launch_bounds__(32 * M) srft_merge_kernel(DecodeArgs a) {
   constexpr int D = 32 * M;
   __shared__ float z[2][D];
   const int pairs_per_b = (a.Hq + 1) / 2;
   const int b = blockIdx.x / pairs_per_b, h0 = 2 * (blockIdx.x % pairs_per_b);
+  const bool two = h0 + 1 < a.Hq;
   const int i = threadIdx.x, lane = i & 31;
+  // everything that does not depend on the split-K partials runs before the wait
+  HartleyTwiddles<M> tw;
+  if (i < 32) hartley_twiddles<M>(tw, lane);
   const int raw = a.ctx_lens[b];
   const int T = raw < 1 ? 1 : (raw > a.max_ctx ? a.max_ctx : raw);
   const int nc = (T + a.plan.chunk - 1) / a.plan.chunk;
   const int stride = a.plan.part_stride;
   const float lv = a.lambda_v ? a.lambda_v[i] : 1.0f;
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float* parts = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
-                                                      a.plan.header_bytes);
+  const float* p0 = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.workspace) +
+                                                   a.plan.header_bytes) +
+                    ((int64_t)b * a.Hq + h0) * a.plan.n_chunks * stride;
+  const float* p1 = two ? p0 + (int64_t)a.plan.n_chunks * stride : p0;
+  // log-sum-exp merge of both heads' chunks: M = max m_c, o = sum 2^(m_c - M) acc_c / sum 2^(m_c - M) l_c
+  float M0 = -INFINITY, M1 = -INFINITY;
+  for (int c = 0; c < nc; ++c) {
+    M0 = fmaxf(M0, p0[(int64_t)c * stride + D]);
+    M1 = fmaxf(M1, p1[(int64_t)c * stride + D]);
+  }
+  constexpr int U = 4;
+  float a0[U], l0[U], a1[U], l1[U];
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = h0 + hh;
-    float x = 0.0f;
-    if (h < a.Hq) {
-      float Mx, L;
-      const float* part = parts + ((int64_t)b * a.Hq + h) * a.plan.n_chunks * stride;
-      x = combine_chunks(part, nc, stride, D, i, Mx, L) / lv;
-      if (a.lse != nullptr && i == 0)
-        *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + h) * 2) = make_float2(Mx, L);
-    }
-    z[hh][i] = x;
+  for (int k = 0; k < U; ++k) a0[k] = l0[k] = a1[k] = l1[k] = 0.0f;
+  for (int c0 = 0; c0 < nc; c0 += U) {
+#pragma unroll
+    for (int k = 0; k < U; ++k)
+      if (c0 + k < nc) {
+        const float* q0 = p0 + (int64_t)(c0 + k) * stride;
+        const float* q1 = p1 + (int64_t)(c0 + k) * stride;
+        const float w0 = exp2f(q0[D] - M0), w1 = exp2f(q1[D] - M1);
+        l0[k] = fmaf(w0, q0[D + 1], l0[k]);
+        a0[k] = fmaf(w0, q0[i], a0[k]);
+        l1[k] = fmaf(w1, q1[D + 1], l1[k]);
+        a1[k] = fmaf(w1, q1[i], a1[k]);
+      }
+  }
+  const float L0 = (l0[0] + l0[2]) + (l0[1] + l0[3]), L1 = (l1[0] + l1[2]) + (l1[1] + l1[3]);
+  z[0][i] = ((a0[0] + a0[2]) + (a0[1] + a0[3])) / L0 / lv;
+  z[1][i] = two ? ((a1[0] + a1[2]) + (a1[1] + a1[3])) / L1 / lv : 0.0f;
+  if (a.lse != nullptr && i == 0) {
+    *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + h0) * 2) = make_float2(M0, L0);
+    if (two) *reinterpret_cast<float2*>(a.lse + ((int64_t)b * a.Hq + h0 + 1) * 2) = make_float2(M1, L1);
   }
   __syncthreads();
   if (i >= 32) return;
-  HartleyTwiddles<M> tw;
-  hartley_twiddles<M>(tw, lane);
   float re[M], im[M];
 #pragma unroll
   for (int j2 = 0; j2 < M; ++j2) {
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(32 * M) srft_merge_kernel(DecodeArgs a) {
     const int k = k2 + M * brev5(lane);
     const float sg = a.signs ? (float)a.signs[k] * norm : norm;
     a.out[base0 + k] = hx[k2] * sg;
-    if (h0 + 1 < a.Hq) a.out[base0 + D + k] = hy[k2] * sg;
+    if (two) a.out[base0 + D + k] = hy[k2] * sg;
   }
 }
 

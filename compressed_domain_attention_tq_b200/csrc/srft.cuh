@@ -17,8 +17,9 @@
 //   H_y[k] = (Im Z[k] + Im Z[d-k] + Re Z[k] - Re Z[d-k]) / 2
 // (H = Re X - Im X for the e^{-i} DFT), where Z[d-k] sits in lane lane ^ 31,
 // slot M - k2 (k2 > 0), or in lane brev5((32 - k1) mod 32), slot 0 (k2 = 0).
-// Twiddles are computed once per warp in double (sincospi of the exact
-// fraction) and rounded to fp32; the transform's arithmetic is fp32.
+// Twiddles are computed once per warp in double (three sincospi calls per
+// lane, the rest as exact powers and squares) and rounded to fp32; the
+// transform's arithmetic is fp32.
 // Each input is first scaled by a power of two that brings its largest
 // magnitude into [0.5, 1), and its transform scaled back (both exact): the
 // rounding error a transform of z leaves in X and Y is relative to |z|, so
@@ -42,26 +43,45 @@ struct HartleyTwiddles {
   int src0;      // lane holding Z[d - k] for this lane's slot 0
 };
 
-// exp(-2 pi i num / den), each part rounded once to fp32
-__device__ __forceinline__ float2 cis_neg(int num, int den) {
+// exp(-2 pi i num / den) in double
+__device__ __forceinline__ double2 cis_neg(int num, int den) {
   double s, c;
   sincospi(2.0 * (double)num / (double)den, &s, &c);
-  return make_float2((float)c, (float)-s);
+  return make_double2(c, -s);
 }
+
+__device__ __forceinline__ double2 cmul_d(double2 a, double2 b) {
+  return make_double2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+
+__device__ __forceinline__ float2 to_f2(double2 a) { return make_float2((float)a.x, (float)a.y); }
 
 template <int M>
 __device__ __forceinline__ void hartley_twiddles(HartleyTwiddles<M>& tw, int lane) {
   constexpr int D = 32 * M;
+  // powers of exp(-2 pi i / M) and of exp(-2 pi i lane / d)
+  const double2 bm = cis_neg(1, M), bb = cis_neg(lane, D);
+  double2 pm = make_double2(1.0, 0.0), pb = make_double2(1.0, 0.0);
 #pragma unroll
-  for (int t = 0; t < M; ++t) tw.wm[t] = cis_neg(t, M);
-#pragma unroll
-  for (int k2 = 0; k2 < M; ++k2) tw.wb[k2] = cis_neg(lane * k2, D);
+  for (int t = 0; t < M; ++t) {
+    tw.wm[t] = to_f2(pm);
+    tw.wb[t] = to_f2(pb);
+    pm = cmul_d(pm, bm);
+    pb = cmul_d(pb, bb);
+  }
+  // radix-2 stages: a_s = exp(-2 pi i u_s / 32) with u_s = (lane mod h) 2^s, h = 16 >> s;
+  // u_{s+1} = 2 u_s - 16 b (b: bit 3 - s of lane), so a_{s+1} = a_s^2 (-1)^b
+  double2 a = cis_neg(lane & 15, 32);
 #pragma unroll
   for (int s = 0; s < 5; ++s) {
     const int h = 16 >> s;
     const bool upper = (lane & h) != 0;
-    tw.wc[s] = upper ? cis_neg(lane & (h - 1), 2 * h) : make_float2(1.0f, 0.0f);
+    tw.wc[s] = upper ? to_f2(a) : make_float2(1.0f, 0.0f);
     tw.sg[s] = upper ? -1.0f : 1.0f;
+    if (s < 4) {
+      a = cmul_d(a, a);
+      if ((lane >> (3 - s)) & 1) a = make_double2(-a.x, -a.y);
+    }
   }
   tw.src0 = brev5((32 - brev5(lane)) & 31);
 }

@@ -15,20 +15,24 @@ namespace tq {
 static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Split the context into chunks (multiples of the decode's pipeline stage,
-// 192 or 128 tokens) for persistent CTAs, one per SM: pick the chunk count per
-// sequence that minimises (waves of items over the SMs) x (chunk + a fixed
-// per-item cost), where an item is one (sequence, kv head, chunk).
+// 192 or 128 tokens): pick the chunk count per sequence that minimises
+// (waves of items over the CTA slots) x (chunk + a fixed per-item cost), where
+// an item is one (sequence, kv head, chunk).  The tensor-core decode runs
+// persistent CTAs, one per SM; the CUDA-core decode runs one 128-thread CTA
+// per item, several resident per SM.
 bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan, bool srft) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
   if (srft ? !srft_head_dim_supported(d) : (d != 128 && d != 256)) return false;
   const int64_t units = (int64_t)B * Hkv;
-  const int64_t step = decode_stage_tokens(d, Hq / Hkv), per_item_cost = 384;
+  const bool mma = decode_mma_supported(d, Hq / Hkv);
+  const int64_t step = decode_stage_tokens(d, Hq / Hkv), per_item_cost = mma ? 384 : 256;
+  const int64_t slots = mma ? kSmCount : 4 * kSmCount;
   const int64_t max_n = ceil_div(max_ctx, step);
   int64_t best_chunk = ceil_div(max_ctx, step) * step, best_cost = -1;
   for (int64_t n = 1; n <= max_n && n <= 4096; ++n) {
     const int64_t chunk = ceil_div(ceil_div(max_ctx, n), step) * step;
     const int64_t items = units * ceil_div(max_ctx, chunk);
-    const int64_t cost = ceil_div(items, kSmCount) * (chunk + per_item_cost);
+    const int64_t cost = ceil_div(items, slots) * (chunk + per_item_cost);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best_chunk = chunk;

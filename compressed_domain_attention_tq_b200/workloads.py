@@ -6,10 +6,12 @@ the CPU oracle are fed from it.
 
 The shapes stand in for the model runs on the pages (Open-TQ-Metal abstract:
 Llama 3.1 70B at 128K context and Gemma 4 with attn_scale = 1.0; AdapTQ post,
-performance section: 4 heads x d=128 x 4096 cached tokens).  No model weights
-or datasets are used: K, V and Q are i.i.d. normal draws with the structure
-each workload names (fixed outlier K channels, heavy-tailed token rows,
-ragged context lengths).
+performance section: 4 heads x d=128 x 4096 cached tokens; SRFT post: head
+widths that are not powers of two).  No model weights or datasets are used:
+K, V and Q are i.i.d. normal draws with the structure each workload names
+(fixed outlier K channels, heavy-tailed token rows, ragged context lengths).
+The SRFT variant's per-coordinate scales lambda come from calibration on the
+pages; here they are drawn from the seed (2^U(-s, s) per coordinate).
 """
 from __future__ import annotations
 
@@ -37,6 +39,8 @@ class Workload:
     heavy_scale: float = 1.0
     ragged: tuple | None = None   # (lo, hi): per-sequence context ~ U{lo..hi}
     append_per_step: int = 1      # tokens quantize-appended per decode step
+    rotation_kind: str = "hadamard"   # "hadamard" or "srft" (when rotation is on)
+    lambda_spread: float = 1.0        # srft: lambda = 2^U(-spread, spread) per coordinate
     notes: str = field(default="", compare=False)
 
     @property
@@ -71,6 +75,18 @@ WORKLOADS = {
         capacity=65537, in_dtype=torch.bfloat16, rotation=True,
         attn_scales=(1.0, 1 / 16.0),
         notes="32/16 GQA, d=256; attn_scale 1.0 and 1/sqrt(256)"),
+    "llama70b_gqa_128k_srft": Workload(
+        "llama70b_gqa_128k_srft", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0,
+        rotation_kind="srft",
+        notes="the 128K GQA layer with the SRFT rotation and per-coordinate lambdas"),
+    "mha32_d96_32k": Workload(
+        "mha32_d96_32k", batch=1, num_q_heads=32, num_kv_heads=32, head_dim=96, context=32768,
+        capacity=32769, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(96),), outlier_channels=4, outlier_scale=10.0,
+        rotation_kind="srft",
+        notes="32-head MHA at head_dim 96 (not a power of two), SRFT rotation, 32K context"),
 }
 
 
@@ -84,6 +100,17 @@ def make_signs(head_dim: int, seed: int) -> torch.Tensor:
     """Random +-1 int8 signs for the rotation (CPU tensor, from the seed)."""
     g = _gen(1_000_003 + seed, "cpu")
     return (torch.randint(0, 2, (head_dim,), generator=g, dtype=torch.int8) * 2 - 1).to(torch.int8)
+
+
+def make_lambdas(w: Workload, seed: int):
+    """SRFT workloads: (lambda_k, lambda_v), float32 [d] CPU tensors of
+    2^U(-spread, spread); (None, None) otherwise."""
+    if not (w.rotation and w.rotation_kind == "srft"):
+        return None, None
+    g = _gen(4_000_003 + seed, "cpu")
+    e = torch.empty(2, w.head_dim).uniform_(-w.lambda_spread, w.lambda_spread, generator=g)
+    lam = torch.exp2(e).to(torch.float32)
+    return lam[0].contiguous(), lam[1].contiguous()
 
 
 def make_context_lengths(w: Workload, seed: int) -> torch.Tensor:
@@ -150,4 +177,5 @@ def shrink(w: Workload, context: int, batch: int | None = None,
                     rotation=w.rotation, attn_scales=w.attn_scales,
                     outlier_channels=w.outlier_channels, outlier_scale=w.outlier_scale,
                     heavy_row_frac=w.heavy_row_frac, heavy_scale=w.heavy_scale, ragged=rag,
-                    append_per_step=w.append_per_step)
+                    append_per_step=w.append_per_step, rotation_kind=w.rotation_kind,
+                    lambda_spread=w.lambda_spread)

@@ -8,7 +8,8 @@ can compute one by one:
   - the decode of sampled kv heads (all their query heads), over that head's
     GPU-written packed cache.
 Gates as in the other GPU tests: rotation on -> at most 0.01% of codes differ,
-each by 1, scales within 4 ulp; attention rel-L2 <= 1e-4 and max-abs <=
+each by 1, scales within 4 ulp (32 ulp with the SRFT rotation, whose fp32 FFT
+error is relative to the whole row); attention rel-L2 <= 1e-4 and max-abs <=
 1e-3 * max|v_hat| per (sequence, query head).
 """
 import math
@@ -33,8 +34,11 @@ def _run_workload(name, attn_scale=None, seed=0, sample_rows=64, sample_heads=2)
     B, Hq, Hkv, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
     G = Hq // Hkv
     signs = wl.make_signs(d, seed) if w.rotation else None
+    srft = w.rotation and w.rotation_kind == "srft"
+    lk, lv = wl.make_lambdas(w, seed)
     ctx = wl.make_context_lengths(w, seed)
-    cache = Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
+    cache = Int4KVCache(B, Hkv, d, w.capacity, dev, signs,
+                        rotation="srft" if srft else "hadamard", lambda_k=lk, lambda_v=lv)
     k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
     cache.append(k_all, v_all, torch.zeros(B, dtype=torch.int32, device=dev))
     k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
@@ -46,26 +50,33 @@ def _run_workload(name, attn_scale=None, seed=0, sample_rows=64, sample_heads=2)
     torch.cuda.synchronize()
     gen = np.random.default_rng(seed + 7)
     sg = None if signs is None else signs.numpy()
+    lk_h, lv_h = (None, None) if lk is None else (lk.numpy(), lv.numpy())
+    scale_ulp = 32 if srft else (4 if sg is not None else 0)
 
     # ---- quantizer: sampled rows of the bulk call
     n_diff = n_tot = 0
     for _ in range(sample_rows):
         b, h = int(gen.integers(B)), int(gen.integers(Hkv))
         t = int(gen.integers(int(ctx[b])))
-        for src, packed, scales in ((k_all, cache.k_packed, cache.k_scales),
-                                    (v_all, cache.v_packed, cache.v_scales)):
-            x = src[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
-            ref = oracle.empty_cache(1, 1, 1, d)
-            oracle.quantize_append(to_oracle(x), to_oracle(x), np.zeros(1, np.int32), sg, ref)
+        xk = k_all[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
+        xv = v_all[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
+        ref = oracle.empty_cache(1, 1, 1, d)
+        if srft:
+            oracle.quantize_append_srft(to_oracle(xk), to_oracle(xv), np.zeros(1, np.int32), sg,
+                                        lk_h, lv_h, ref)
+        else:
+            oracle.quantize_append(to_oracle(xk), to_oracle(xv), np.zeros(1, np.int32), sg, ref)
+        for packed, scales, rp, rs in ((cache.k_packed, cache.k_scales, ref[0], ref[1]),
+                                       (cache.v_packed, cache.v_scales, ref[2], ref[3])):
             got_codes = oracle.unpack(packed[b, h, t:t + 1].cpu().numpy(), d).astype(np.int64)
-            want_codes = oracle.unpack(ref[0][0, 0], d).astype(np.int64)
+            want_codes = oracle.unpack(rp[0, 0], d).astype(np.int64)
             diff = np.abs(got_codes - want_codes)
             assert diff.max() <= (1 if sg is not None else 0), f"{name} b={b} h={h} t={t}"
             n_diff += int((diff > 0).sum())
             n_tot += diff.size
             got_s = scales[b, h, t].cpu().numpy().view(np.int32).astype(np.int64)
-            want_s = ref[1][0, 0, 0].view(np.int32).astype(np.int64)
-            assert np.abs(got_s - want_s).max() <= (4 if sg is not None else 0)
+            want_s = rs[0, 0, 0].view(np.int32).astype(np.int64)
+            assert np.abs(got_s - want_s).max() <= scale_ulp
     assert n_diff <= max(1e-4 * n_tot, 1), f"{name}: {n_diff}/{n_tot} codes differ"
 
     # ---- decode: sampled (sequence, kv head) pairs over the GPU-written cache
@@ -77,7 +88,11 @@ def _run_workload(name, attn_scale=None, seed=0, sample_rows=64, sample_heads=2)
         sub = [np.ascontiguousarray(a[b:b + 1, h:h + 1, :Tb].cpu().numpy())
                for a in (cache.k_packed, cache.k_scales, cache.v_packed, cache.v_scales)]
         qs = np.ascontiguousarray(q_host[b:b + 1, h * G:(h + 1) * G])
-        want = oracle.sdpa_int4_decode(qs, sub, [Tb], sg, scale, 1, threads=THREADS)
+        if srft:
+            want = oracle.sdpa_int4_decode_srft(qs, sub, [Tb], sg, lk_h, lv_h, scale, 1,
+                                                threads=THREADS)
+        else:
+            want = oracle.sdpa_int4_decode(qs, sub, [Tb], sg, scale, 1, threads=THREADS)
         check_attention(got[b:b + 1, h * G:(h + 1) * G], want, sub, [Tb], G,
                         f"{name} b={b} kv head {h}")
     return n_diff, n_tot
@@ -102,3 +117,11 @@ def test_full_size_ragged_b16():
 @pytest.mark.parametrize("scale", [1.0, 1 / 16.0])
 def test_full_size_wide_d256(scale):
     _run_workload("wide_d256", attn_scale=scale)
+
+
+def test_full_size_llama70b_gqa_128k_srft():
+    _run_workload("llama70b_gqa_128k_srft")
+
+
+def test_full_size_mha32_d96_32k():
+    _run_workload("mha32_d96_32k", sample_heads=3)
