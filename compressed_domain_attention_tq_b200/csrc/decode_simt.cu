@@ -26,13 +26,22 @@ constexpr int kTile = 64;      // tokens per shared-memory tile
 constexpr int kThreads = 128;
 
 // Token parts of the P.V work: the (head, 8-dim slice) items are split over
-// TP interleaved token subsets while that keeps at most 2 items per thread,
-// so small G (MHA) still occupies every thread; the parts are summed once per
-// chunk.  Shared by the host (shared-memory size) and the kernel.
+// TP interleaved token subsets, TP chosen (up to 32, at most 4 items per
+// thread) to fill the block's threads best, so small G (MHA) still occupies
+// every thread; the parts are summed once per chunk.  Shared by the host
+// (shared-memory size) and the kernel.
 __host__ __device__ constexpr int simt_token_parts(int G, int slices) {
-  int tp = 1;
-  while (tp < 16 && G * slices * tp * 2 <= 2 * kThreads) tp *= 2;
-  return tp;
+  int best = 1, best_num = 0, best_den = 1;
+  for (int tp = 1; tp <= 32 && G * slices * tp <= 4 * kThreads; tp *= 2) {
+    const int items = G * slices * tp;
+    const int den = ((items + kThreads - 1) / kThreads) * kThreads;  // thread slots used
+    if (items * best_den > best_num * den) {  // strictly better fill
+      best = tp;
+      best_num = items;
+      best_den = den;
+    }
+  }
+  return best;
 }
 
 // Row pitch of a staged packed row in 32-bit words: odd, so lanes reading the
@@ -40,11 +49,15 @@ __host__ __device__ constexpr int simt_token_parts(int G, int slices) {
 template <int D>
 __host__ __device__ constexpr int simt_pitch_words() { return D / 8 + 1; }
 
-// the 4 codes of a 16-bit half-word (in-group coordinates 4r .. 4r+3 of one group)
-__device__ __forceinline__ float code_of(uint32_t hw, int m) {
-  // u = nibble; (u ^ 8) | 2^23 as a float is 2^23 + 8 + c for the two's-complement code c
-  const uint32_t u = (hw >> (4 * m)) & 0xFu;
-  return __int_as_float((int)(u ^ 0x4B000008u)) - 8388616.0f;
+// Code m of a 16-bit half-word (in-group coordinates 4r .. 4r+3 of one group)
+// as the exact float 16^m c.  t = hw ^ 0x8888 holds the biased nibbles c + 8;
+// masking nibble m in place and setting the exponent bits of 2^23 gives the
+// float 2^23 + 16^m (c + 8), from which one subtraction leaves 16^m c.  The
+// factor 16^m is folded into the query (scores) or removed from the sums at
+// the end (P.V), both exactly.
+__device__ __forceinline__ float code16m(uint32_t t, int m) {
+  return __int_as_float((int)((t & (0xFu << (4 * m))) | 0x4B000000u)) -
+         (8388608.0f + 8.0f * (float)(1 << (4 * m)));
 }
 
 // In-place Walsh-Hadamard transform of `n` rows of length D in shared memory
@@ -103,9 +116,10 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   float* mstate = scl + 4 * kTile * NG;                        // [G] running max (log2)
   float* lstate = mstate + 16;                                 // [G] running sum
   float* alpha = lstate + 16;                                  // [G] rescale of this tile
-  float* red = alpha + 16;                                     // [TP][G][D] (TP > 1)
-  // [2 buffers][K, V][kTile][PW] staged packed rows
-  uint32_t* tiles = reinterpret_cast<uint32_t*>(red + (TP > 1 ? TP * G * D : 0));
+  // [2 buffers][K, V][kTile][PW] staged packed rows; after the last tile the same
+  // space holds the token parts' sums [TP][G][D] (TP > 1)
+  uint32_t* tiles = reinterpret_cast<uint32_t*>(alpha + 16);
+  float* red = reinterpret_cast<float*>(tiles);
 
   // q' = attn_scale * log2(e) * R q (the SRFT variant's R q comes rotated in q_rot)
   const int64_t qbase = ((int64_t)b * a.Hq + (int64_t)kvh * G) * D;
@@ -125,7 +139,9 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   }
   const float qmul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
   __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += kThreads) qs[i] *= qmul;
+  // 16^-(i mod 4): the codes of the score loop come scaled by 16^(i mod 4)
+  for (int i = threadIdx.x; i < G * D; i += kThreads)
+    qs[i] *= qmul * __int_as_float((127 - 4 * (i & 3)) << 23);
   if (threadIdx.x < 16) {
     mstate[threadIdx.x] = -INFINITY;
     lstate[threadIdx.x] = 0.0f;
@@ -188,16 +204,16 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
         const uint16_t* row = reinterpret_cast<const uint16_t*>(ktile + tt * PW);
         const int r_lo = SP == 2 ? 4 * part : 0, r_hi = SP == 2 ? r_lo + 4 : 8;
         for (int g = 0; g < NG; ++g) {
-          float dot = 0.0f;
+          float d0 = 0.0f, d1 = 0.0f, d2 = 0.0f, d3 = 0.0f;  // four independent chains
           for (int r = r_lo; r < r_hi; ++r) {
-            const uint32_t hw = row[r * NG + g];   // half-word at byte r * 2NG + 2g
+            const uint32_t t = row[r * NG + g] ^ 0x8888u;   // half-word at byte r * 2NG + 2g
             const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + 32 * g + 4 * r);
-            dot = fmaf(qv.x, code_of(hw, 0), dot);
-            dot = fmaf(qv.y, code_of(hw, 1), dot);
-            dot = fmaf(qv.z, code_of(hw, 2), dot);
-            dot = fmaf(qv.w, code_of(hw, 3), dot);
+            d0 = fmaf(qv.x, code16m(t, 0), d0);
+            d1 = fmaf(qv.y, code16m(t, 1), d1);
+            d2 = fmaf(qv.z, code16m(t, 2), d2);
+            d3 = fmaf(qv.w, code16m(t, 3), d3);
           }
-          s = fmaf(kscale[tt * NG + g], dot, s);
+          s = fmaf(kscale[tt * NG + g], (d0 + d1) + (d2 + d3), s);
         }
       }
       if (SP == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);  // idx, idx ^ 1: the same token
@@ -236,22 +252,30 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
         const int tp = rest % TP, h = rest / TP;
         const int g = sl / 4, r0 = (sl % 4) * 2;
         const float al = alpha[h];
+        if (al != 1.0f) {  // the running max moved
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[it][e] *= al;
+          for (int e = 0; e < 8; ++e) acc[it][e] *= al;
+        }
         for (int tt = tp; tt < nt; tt += TP) {
           const float pw = sp[h * kTile + tt] * vscale[tt * NG + g];
           const uint16_t* row = reinterpret_cast<const uint16_t*>(vtile + tt * PW);
-          const uint32_t hw0 = row[r0 * NG + g], hw1 = row[(r0 + 1) * NG + g];
+          const uint32_t t0 = row[r0 * NG + g] ^ 0x8888u, t1 = row[(r0 + 1) * NG + g] ^ 0x8888u;
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            acc[it][m] = fmaf(pw, code_of(hw0, m), acc[it][m]);
-            acc[it][4 + m] = fmaf(pw, code_of(hw1, m), acc[it][4 + m]);
+            acc[it][m] = fmaf(pw, code16m(t0, m), acc[it][m]);
+            acc[it][4 + m] = fmaf(pw, code16m(t1, m), acc[it][4 + m]);
           }
         }
       }
     }
     __syncthreads();  // the tile's buffers and scores are free for the next stage
   }
+
+  // slot e of a P.V item holds 16^(e mod 4) times its sum
+#pragma unroll
+  for (int it = 0; it < 4; ++it)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[it][e] *= __int_as_float((127 - 4 * (e & 3)) << 23);
 
   // partials: ws[b][hq][chunk][0..D) = acc, [D] = m, [D+1] = l
   float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) + a.plan.header_bytes);
@@ -301,9 +325,10 @@ template <int D>
 size_t simt_smem_bytes(int G) {
   constexpr int NG = D / 32;
   const int TP = simt_token_parts(G, D / 8);
-  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 48 +
-                          (TP > 1 ? (size_t)TP * G * D : 0)) +
-         4 * sizeof(uint32_t) * (size_t)kTile * simt_pitch_words<D>();
+  const size_t tile_words = 4 * (size_t)kTile * simt_pitch_words<D>();
+  const size_t red_words = TP > 1 ? (size_t)TP * G * D : 0;
+  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 48) +
+         sizeof(uint32_t) * (tile_words > red_words ? tile_words : red_words);
 }
 
 template <int D>

@@ -31,6 +31,21 @@ namespace tq {
 namespace {
 
 constexpr int kQWarps = 8;  // warps per quantize CTA
+constexpr float kRneMagic = 12582912.0f;                   // 1.5 * 2^23: x + M rounds x to an integer
+constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21 (exact)
+constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21 (exact)
+
+// c = clamp(rne(fl32(x / s)), -7, 7) without a division per element: x is
+// rounded with reciprocals bracketing 1/s from below and above (2^-21 apart,
+// far more than their rounding error); rounding is monotone, so when both
+// give the same integer it is rne(fl32(x / s)), else (x / s within ~1e-5 of a
+// half-integer, or a subnormal s) the IEEE division decides.
+__device__ __forceinline__ float int4_code(float x, float s, float r, bool big) {
+  const float lo = fmaf(x, r * kBracketLo, kRneMagic), hi = fmaf(x, r * kBracketHi, kRneMagic);
+  float c = lo - kRneMagic;
+  if (big || lo != hi) c = rintf(__fdiv_rn(x, s));
+  return fminf(fmaxf(c, -7.0f), 7.0f);
+}
 
 template <int M>
 __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArgs a) {
@@ -51,19 +66,18 @@ __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArg
   }
   float* yk = ybuf[warp][0];
   float* yv = ybuf[warp][1];
-  const int64_t pairs = (int64_t)a.B * a.Hkv * a.n_new;
-  for (int64_t p = (int64_t)blockIdx.x * kQWarps + warp; p < pairs;
-       p += (int64_t)gridDim.x * kQWarps) {
-    const int64_t bh = p / a.n_new, n = p % a.n_new;
-    const int b = (int)(bh / a.Hkv);
+  const int pairs = a.B * a.Hkv * a.n_new;  // < 2^31 (checked on the host)
+  for (int p = blockIdx.x * kQWarps + warp; p < pairs; p += gridDim.x * kQWarps) {
+    const int bh = p / a.n_new, n = p % a.n_new;
+    const int b = bh / a.Hkv;
     int64_t pos = (int64_t)a.pos[b] + n;
     if (a.pos_is_ctx) pos = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
     if (pos < 0 || pos >= a.capacity) continue;  // the whole warp
-    const int64_t row = bh * a.capacity + pos;
+    const int64_t row = (int64_t)bh * a.capacity + pos;
     float re[M], im[M];
 #pragma unroll
     for (int j2 = 0; j2 < M; ++j2) {
-      const int64_t idx = p * D + lane + 32 * j2;
+      const int64_t idx = (int64_t)p * D + lane + 32 * j2;
       float xk, xv;
       if (a.bf16) {
         xk = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.k)[idx] << 16);
@@ -97,10 +111,11 @@ __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArg
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float s = __fdiv_rn(amax, 7.0f);
-        float c = 0.0f;
-        if (s > 0.0f) c = fminf(fmaxf(rintf(__fdiv_rn(x, s)), -7.0f), 7.0f);
+        const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+        const float c = s > 0.0f ? int4_code(x, s, r, !(r <= 3.0e38f)) : 0.0f;
         // byte (j / 4) * 2M + 2 g + (j % 4) / 2, nibble j % 2: four lanes make one half-word
-        uint32_t nib = ((uint32_t)(int)c & 0xFu) << (4 * (lane & 3));
+        // c + 1.5 * 2^23 has the bits 0x4B400000 + c: its low nibble is c's two's complement
+        uint32_t nib = (__float_as_uint(c + kRneMagic) & 0xFu) << (4 * (lane & 3));
         nib |= __shfl_xor_sync(0xffffffffu, nib, 1);
         nib |= __shfl_xor_sync(0xffffffffu, nib, 2);
         if ((lane & 3) == 0)

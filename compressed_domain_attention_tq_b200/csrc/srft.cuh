@@ -108,11 +108,16 @@ __device__ __forceinline__ void hartley_pair_warp(const float (&re_in)[M], const
   int ex = 0, ey = 0;
   if (mx > 0.0f) frexpf(mx, &ex);
   if (my > 0.0f) frexpf(my, &ey);
+  // multiplying by 2^-e and 2^e is what ldexpf computes (both are correctly
+  // rounded); the float powers are exact while e stays in [-126, 126]
+  const bool fast = ex >= -126 && ex <= 126 && ey >= -126 && ey <= 126;  // warp-uniform
+  const float sxi = __int_as_float((127 - (fast ? ex : 0)) << 23);
+  const float syi = __int_as_float((127 - (fast ? ey : 0)) << 23);
   float re[M], im[M];
 #pragma unroll
   for (int j2 = 0; j2 < M; ++j2) {
-    re[j2] = ldexpf(re_in[j2], -ex);
-    im[j2] = ldexpf(im_in[j2], -ey);
+    re[j2] = fast ? re_in[j2] * sxi : ldexpf(re_in[j2], -ex);
+    im[j2] = fast ? im_in[j2] * syi : ldexpf(im_in[j2], -ey);
   }
   float ar[M], ai[M];
   // A: M-point DFT within the lane
@@ -163,8 +168,14 @@ __device__ __forceinline__ void hartley_pair_warp(const float (&re_in)[M], const
       qi = __shfl_xor_sync(0xffffffffu, ai[M - k2], 31);
     }
     // an all-zero input's transform is exactly zero (not its partner's rounding residue)
-    hx[k2] = mx > 0.0f ? ldexpf((ar[k2] + qr) + (qi - ai[k2]), ex) : 0.0f;
-    hy[k2] = my > 0.0f ? ldexpf((ai[k2] + qi) + (ar[k2] - qr), ey) : 0.0f;
+    const float vx = (ar[k2] + qr) + (qi - ai[k2]), vy = (ai[k2] + qi) + (ar[k2] - qr);
+    if (fast) {
+      hx[k2] = mx > 0.0f ? vx * __int_as_float((127 + ex) << 23) : 0.0f;
+      hy[k2] = my > 0.0f ? vy * __int_as_float((127 + ey) << 23) : 0.0f;
+    } else {
+      hx[k2] = mx > 0.0f ? ldexpf(vx, ex) : 0.0f;
+      hy[k2] = my > 0.0f ? ldexpf(vy, ey) : 0.0f;
+    }
   }
 }
 

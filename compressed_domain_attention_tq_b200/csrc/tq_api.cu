@@ -105,6 +105,7 @@ static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, 
   if (!k || !v || !pos || !k_packed || !k_scales || !v_packed || !v_scales) return TQ_ERR_INVALID_ARG;
   if (in_dtype != TQ_F32 && in_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
   if (batch < 1 || num_kv_heads < 1 || n_new < 1 || capacity < n_new) return TQ_ERR_INVALID_ARG;
+  if ((int64_t)batch * num_kv_heads * n_new > INT32_MAX) return TQ_ERR_INVALID_ARG;
   if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_packed) || !aligned16(v_packed) ||

@@ -95,7 +95,8 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
  * rotated vector is computed in fp32, so a code may differ by 1 from one
  * computed with an exactly rounded rotation.
  * Returns TQ_ERR_INVALID_ARG for NULL pointers (other than signs), B, Hkv or
- * n_new < 1, capacity < n_new, misaligned pointers; TQ_ERR_UNSUPPORTED for
+ * n_new < 1, capacity < n_new, batch * num_kv_heads * n_new > 2^31 - 1,
+ * misaligned pointers; TQ_ERR_UNSUPPORTED for
  * head_dim not in {128, 256} or group != 32.
  */
 TQ_API tq_status tq_quantize_append(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
