@@ -11,7 +11,9 @@ widths that are not powers of two).  No model weights or datasets are used:
 K, V and Q are i.i.d. normal draws with the structure each workload names
 (fixed outlier K channels, heavy-tailed token rows, ragged context lengths).
 The SRFT variant's per-coordinate scales lambda come from calibration on the
-pages; here they are drawn from the seed (2^U(-s, s) per coordinate).
+pages; here they are drawn from the seed (2^U(-s, s) per coordinate, s = 1/4:
+close to one, as a variance-equalizing calibration over these i.i.d. inputs
+would give; the parity tests use a wider spread).
 """
 from __future__ import annotations
 
@@ -40,7 +42,7 @@ class Workload:
     ragged: tuple | None = None   # (lo, hi): per-sequence context ~ U{lo..hi}
     append_per_step: int = 1      # tokens quantize-appended per decode step
     rotation_kind: str = "hadamard"   # "hadamard" or "srft" (when rotation is on)
-    lambda_spread: float = 1.0        # srft: lambda = 2^U(-spread, spread) per coordinate
+    lambda_spread: float = 0.25       # srft: lambda = 2^U(-spread, spread) per coordinate
     notes: str = field(default="", compare=False)
 
     @property
