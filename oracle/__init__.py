@@ -86,6 +86,20 @@ def _load():
     lib.oracle_sdpa_int4_decode_srft.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, i64, P,
                                                  P, P, P, f64, P, i32]
     lib.oracle_sdpa_int4_decode_srft.restype = i32
+    lib.oracle_lloyd_max_gaussian.argtypes = [i32, P]
+    lib.oracle_lloyd_max_gaussian.restype = i32
+    lib.oracle_cb_quantize_vector.argtypes = [i32, P, i32, P, P, P]
+    lib.oracle_cb_quantize_vector.restype = None
+    lib.oracle_cb_pack_vector.argtypes = [i32, i32, P, P]
+    lib.oracle_cb_pack_vector.restype = None
+    lib.oracle_cb_unpack_vector.argtypes = [i32, i32, P, P]
+    lib.oracle_cb_unpack_vector.restype = None
+    lib.oracle_quantize_append_cb.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, P, P, P,
+                                              P, P, i64, i32]
+    lib.oracle_quantize_append_cb.restype = i32
+    lib.oracle_sdpa_cb_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P,
+                                          f64, P, i32]
+    lib.oracle_sdpa_cb_decode.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     _lib = lib
@@ -320,4 +334,107 @@ def exact_attention(q, k, v, ctx_lens, attn_scale: float, threads: int = 1) -> n
                                         _ptr(ctx), float(attn_scale), _ptr(out), threads)
     if rc != 0:
         raise ValueError(f"oracle_exact_attention failed ({rc})")
+    return out
+
+
+# ------------------------------------------------------------ codebook variant
+# AdapTQ's Max-Lloyd codebook indices at 2, 3 or 4 bits per coordinate (see the
+# header of oracle.c for the quantizer and the packed layout).
+
+def lloyd_max_gaussian(bits: int) -> np.ndarray:
+    """Gaussian Max-Lloyd codebook of 2**bits increasing levels (fp64)."""
+    out = np.empty(1 << bits, dtype=np.float64)
+    if _load().oracle_lloyd_max_gaussian(bits, _ptr(out)) != 0:
+        raise ValueError("bits must be in 1..8")
+    return out
+
+
+def _levels_array(levels, bits):
+    c = np.ascontiguousarray(levels, dtype=np.float32)
+    if c.shape != (1 << bits,) or not np.all(np.diff(c) > 0):
+        raise ValueError("levels must be 2**bits strictly increasing float32 values")
+    return c
+
+
+def cb_row_bytes(d: int, bits: int) -> int:
+    return d * bits // 8
+
+
+def cb_quantize_vectors(y: np.ndarray, bits: int, levels):
+    """Codebook indices (uint8 (n, d)) and sigma scales (float32 (n, d/32)) of rotated rows y."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    n, d = y.shape
+    c = _levels_array(levels, bits)
+    idx = np.empty((n, d), dtype=np.uint8)
+    scales = np.empty((n, d // _GROUP), dtype=np.float32)
+    lib = _load()
+    for r in range(n):
+        lib.oracle_cb_quantize_vector(d, _ptr(y[r]), bits, _ptr(c), _ptr(idx[r]), _ptr(scales[r]))
+    return idx, scales
+
+
+def cb_pack(idx: np.ndarray, bits: int) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.uint8)
+    n, d = idx.shape
+    out = np.empty((n, cb_row_bytes(d, bits)), dtype=np.uint8)
+    lib = _load()
+    for r in range(n):
+        lib.oracle_cb_pack_vector(d, bits, _ptr(idx[r]), _ptr(out[r]))
+    return out
+
+
+def cb_unpack(packed: np.ndarray, d: int, bits: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    n = packed.shape[0]
+    out = np.empty((n, d), dtype=np.uint8)
+    lib = _load()
+    for r in range(n):
+        lib.oracle_cb_unpack_vector(d, bits, _ptr(packed[r]), _ptr(out[r]))
+    return out
+
+
+def empty_cb_cache(B: int, Hkv: int, capacity: int, d: int, bits: int):
+    """Zeroed (k_packed, k_scales, v_packed, v_scales) of a codebook cache."""
+    rb = cb_row_bytes(d, bits)
+    return (np.zeros((B, Hkv, capacity, rb), np.uint8),
+            np.zeros((B, Hkv, capacity, d // _GROUP), np.float32),
+            np.zeros((B, Hkv, capacity, rb), np.uint8),
+            np.zeros((B, Hkv, capacity, d // _GROUP), np.float32))
+
+
+def quantize_append_cb(k, v, pos, signs, bits: int, levels, cache, threads: int = 1) -> None:
+    """Codebook variant of quantize_append (Hadamard rotation with signs, or none)."""
+    k, dt = _input_array(k)
+    v, dt2 = _input_array(v)
+    if dt != dt2 or k.shape != v.shape:
+        raise ValueError("k and v must share dtype and shape")
+    B, Hkv, n_new, d = k.shape
+    kp, ks, vp, vs = cache
+    cap = kp.shape[2]
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    s = _signs_array(signs)
+    c = _levels_array(levels, bits)
+    rc = _load().oracle_quantize_append_cb(_ptr(k), _ptr(v), dt, B, Hkv, n_new, d, _ptr(pos), _ptr(s),
+                                           bits, _ptr(c), _ptr(kp), _ptr(ks), _ptr(vp), _ptr(vs), cap,
+                                           threads)
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_append_cb failed ({rc})")
+
+
+def sdpa_cb_decode(q, cache, ctx_lens, signs, bits: int, levels, attn_scale: float,
+                   num_kv_heads: int, threads: int = 1) -> np.ndarray:
+    """fp64 attention of q over a codebook cache; returns (B, Hq, d) fp64."""
+    q, qdt = _input_array(q)
+    B, Hq, d = q.shape
+    kp, ks, vp, vs = [np.ascontiguousarray(a) for a in cache]
+    cap = kp.shape[2]
+    ctx = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+    s = _signs_array(signs)
+    c = _levels_array(levels, bits)
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    rc = _load().oracle_sdpa_cb_decode(_ptr(q), qdt, B, Hq, num_kv_heads, d, bits, _ptr(c), _ptr(kp),
+                                       _ptr(ks), _ptr(vp), _ptr(vs), cap, _ptr(ctx), _ptr(s),
+                                       float(attn_scale), _ptr(out), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_sdpa_cb_decode failed ({rc})")
     return out

@@ -36,6 +36,18 @@
  *    codes 0.
  *  - attention output = exact softmax attention over the dequantized values
  *    s*c in the rotated basis, mapped back with R^T, all in fp64.
+ *  - codebook variant ([AdapTQ], sections "unified SIMD pipeline",
+ *    "precomputed lookup tables", "performance and quality": 2-, 3- and 4-bit
+ *    indices into a Max-Lloyd codebook with +-3 sigma clipping; int2 is the
+ *    future work of [OTM-F]): per group of 32 rotated coordinates a scale
+ *    sigma = fl32(sqrt(S / 32)), S = sum of y^2 in fp64; u = fl32(y / sigma)
+ *    clipped to [-3, 3]; index = number of thresholds t_i < u, where
+ *    t_i = fl32(fl32(C_i + C_{i+1}) * 0.5) for the fp32 levels C_0 < ... <
+ *    C_{L-1}, L = 2^bits; the value is sigma * C[index].  Indices are packed
+ *    little-endian: index j of group g occupies bits bits*j .. bits*j+bits-1
+ *    of the group's 4*bits bytes, groups in order.  The Gaussian Max-Lloyd
+ *    codebook is the fixed point of "thresholds at midpoints, levels at the
+ *    cell means of N(0,1)".
  *  - SRFT variant ([SRFT], core method: a sign-randomized Fourier transform
  *    instead of the Hadamard one, usable at widths that are not powers of
  *    two, followed by a per-coordinate scale lambda): the transform is the
@@ -420,6 +432,201 @@ int oracle_sdpa_int4_decode_srft(const void* q, int q_dtype, int B, int Hq, int 
   free(Q);
   free(O);
   return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* codebook variant ([AdapTQ] Max-Lloyd codebook, 2/3/4-bit indices)   */
+/* ------------------------------------------------------------------ */
+
+static double std_normal_pdf(double x) { return exp(-0.5 * x * x) / sqrt(2.0 * acos(-1.0)); }
+static double std_normal_cdf(double x) { return 0.5 * erfc(-x / sqrt(2.0)); }
+
+/* Gaussian Max-Lloyd codebook of 2^bits levels (fp64, increasing): iterate
+   thresholds = midpoints of adjacent levels, levels = means of N(0,1) over
+   their cells, E[X | a < X < b] = (pdf(a) - pdf(b)) / (cdf(b) - cdf(a)). */
+int oracle_lloyd_max_gaussian(int bits, double* levels) {
+  if (bits < 1 || bits > 8 || !levels) return -1;
+  int L = 1 << bits;
+  for (int i = 0; i < L; ++i) levels[i] = -3.0 + 6.0 * (i + 0.5) / L;  /* start: uniform on [-3, 3] */
+  for (int it = 0; it < 100000; ++it) {
+    double change = 0.0;
+    for (int i = 0; i < L; ++i) {
+      double a = (i == 0) ? -INFINITY : 0.5 * (levels[i - 1] + levels[i]);
+      double b = (i == L - 1) ? INFINITY : 0.5 * (levels[i] + levels[i + 1]);
+      double pa = isinf(a) ? 0.0 : std_normal_pdf(a), pb = isinf(b) ? 0.0 : std_normal_pdf(b);
+      double ca = isinf(a) ? 0.0 : std_normal_cdf(a), cb = isinf(b) ? 1.0 : std_normal_cdf(b);
+      double m = (pa - pb) / (cb - ca);
+      change = fmax(change, fabs(m - levels[i]));
+      levels[i] = m;
+    }
+    if (change < 1e-15) break;
+  }
+  return 0;
+}
+
+/* thresholds t_i = fl32(fl32(C_i + C_{i+1}) * 0.5), i < L - 1 */
+static void cb_thresholds(int L, const float* C, float* t) {
+  for (int i = 0; i + 1 < L; ++i) {
+    volatile float sum = C[i] + C[i + 1];
+    t[i] = sum * 0.5f;
+  }
+}
+
+/* indices[d], scales[d/32] of an already-rotated vector y */
+void oracle_cb_quantize_vector(int d, const float* y, int bits, const float* C, uint8_t* idx,
+                               float* scales) {
+  int L = 1 << bits, ng = d / ORACLE_GROUP;
+  float t[255];
+  cb_thresholds(L, C, t);
+  for (int g = 0; g < ng; ++g) {
+    const float* yg = y + g * ORACLE_GROUP;
+    double S = 0.0;
+    for (int j = 0; j < ORACLE_GROUP; ++j) S += (double)yg[j] * (double)yg[j];
+    float sigma = (float)sqrt(S / (double)ORACLE_GROUP);
+    scales[g] = sigma;
+    for (int j = 0; j < ORACLE_GROUP; ++j) {
+      float u = 0.0f;
+      if (sigma > 0.0f) {
+        volatile float quot = yg[j] / sigma;  /* fp32 quotient, rounded once */
+        u = quot;
+      }
+      if (u > 3.0f) u = 3.0f;
+      if (u < -3.0f) u = -3.0f;
+      int k = 0;
+      for (int i = 0; i + 1 < L; ++i)
+        if (u > t[i]) ++k;
+      idx[g * ORACLE_GROUP + j] = (uint8_t)k;
+    }
+  }
+}
+
+/* row bytes d * bits / 8: index j of group g at bits bits*j.. of the group's bytes */
+void oracle_cb_pack_vector(int d, int bits, const uint8_t* idx, uint8_t* packed) {
+  int gbytes = 4 * bits;
+  memset(packed, 0, (size_t)d * bits / 8);
+  for (int i = 0; i < d; ++i) {
+    int g = i / ORACLE_GROUP, j = i % ORACLE_GROUP;
+    for (int k = 0; k < bits; ++k) {
+      int bit = bits * j + k;
+      if ((idx[i] >> k) & 1) packed[g * gbytes + bit / 8] |= (uint8_t)(1u << (bit % 8));
+    }
+  }
+}
+
+void oracle_cb_unpack_vector(int d, int bits, const uint8_t* packed, uint8_t* idx) {
+  int gbytes = 4 * bits;
+  for (int i = 0; i < d; ++i) {
+    int g = i / ORACLE_GROUP, j = i % ORACLE_GROUP, v = 0;
+    for (int k = 0; k < bits; ++k) {
+      int bit = bits * j + k;
+      v |= ((packed[g * gbytes + bit / 8] >> (bit % 8)) & 1) << k;
+    }
+    idx[i] = (uint8_t)v;
+  }
+}
+
+/* Hadamard rotation (signs) or none, then the codebook quantizer; cache rows of
+   d * bits / 8 bytes and d / 32 scales. */
+int oracle_quantize_append_cb(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                              int n_new, int d, const int32_t* pos, const int8_t* signs, int bits,
+                              const float* C, uint8_t* k_packed, float* k_scales,
+                              uint8_t* v_packed, float* v_scales, int64_t capacity, int nthreads) {
+  if ((d & (d - 1)) != 0 || check_append(B, n_new, d, pos, capacity) != 0) return -1;
+  if (bits < 2 || bits > 4) return -1;
+  for (int i = 0; i + 1 < (1 << bits); ++i)
+    if (!(C[i] < C[i + 1])) return -1;
+  double* R = NULL;
+  if (signs) {
+    R = (double*)malloc(sizeof(double) * (size_t)d * d);
+    if (!R) return -2;
+    oracle_rotation_matrix(d, signs, R);
+  }
+  int ng = d / ORACLE_GROUP, rowb = d * bits / 8;
+  int64_t nvec = (int64_t)B * Hkv * n_new;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#endif
+  for (int64_t idx = 0; idx < nvec; ++idx) {
+    float x[512], y[512];
+    uint8_t ci[512];
+    int64_t b = idx / ((int64_t)Hkv * n_new);
+    int64_t h = (idx / n_new) % Hkv;
+    int64_t n = idx % n_new;
+    int64_t row = ((int64_t)b * Hkv + h) * capacity + pos[b] + n;
+    for (int kv = 0; kv < 2; ++kv) {
+      const void* src = kv ? v : k;
+      for (int i = 0; i < d; ++i) x[i] = load_input(src, in_dtype, idx * d + i);
+      if (R) oracle_rotate_vector(d, R, x, y);
+      else memcpy(y, x, sizeof(float) * (size_t)d);
+      oracle_cb_quantize_vector(d, y, bits, C, ci, (kv ? v_scales : k_scales) + row * ng);
+      oracle_cb_pack_vector(d, bits, ci, (kv ? v_packed : k_packed) + row * rowb);
+    }
+  }
+  free(R);
+  return 0;
+}
+
+/* attention over a codebook cache: k_hat = sigma_k * C[index], v_hat likewise,
+   q_r = R q, o = R^T o_r (R = identity without signs); fp64 */
+int oracle_sdpa_cb_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int d, int bits,
+                          const float* C, const uint8_t* k_packed, const float* k_scales,
+                          const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                          const int32_t* ctx_lens, const int8_t* signs, double attn_scale,
+                          double* out, int nthreads) {
+  if ((d & (d - 1)) != 0 || check_decode(B, Hq, Hkv, d, ctx_lens, capacity) != 0) return -1;
+  if (bits < 2 || bits > 4) return -1;
+  double* R = (double*)malloc(sizeof(double) * (size_t)d * d);
+  if (!R) return -2;
+  oracle_rotation_matrix(d, signs, R);
+  int G = Hq / Hkv, ng = d / ORACLE_GROUP, rowb = d * bits / 8;
+  int64_t nrows = (int64_t)B * Hq;
+  int fail = 0;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+#endif
+  for (int64_t bh = 0; bh < nrows; ++bh) {
+    int64_t b = bh / Hq, hq = bh % Hq, hk = hq / G;
+    int64_t T = ctx_lens[b];
+    double qv[512], qr[512], orot[512];
+    uint8_t ci[512];
+    double* S = (double*)malloc(sizeof(double) * (size_t)T);
+    if (!S) { fail = 1; continue; }
+    for (int i = 0; i < d; ++i) qv[i] = (double)load_input(q, q_dtype, bh * d + i);
+    for (int i = 0; i < d; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * qv[j];
+      qr[i] = acc;
+    }
+    int64_t base = ((int64_t)b * Hkv + hk) * capacity;
+    double smax = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      oracle_cb_unpack_vector(d, bits, k_packed + (base + t) * rowb, ci);
+      const float* sk = k_scales + (base + t) * ng;
+      double dot = 0.0;
+      for (int i = 0; i < d; ++i) dot += qr[i] * ((double)sk[i / ORACLE_GROUP] * (double)C[ci[i]]);
+      S[t] = attn_scale * dot;
+      if (S[t] > smax) smax = S[t];
+    }
+    double Z = 0.0;
+    for (int64_t t = 0; t < T; ++t) { S[t] = exp(S[t] - smax); Z += S[t]; }
+    for (int i = 0; i < d; ++i) orot[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+      oracle_cb_unpack_vector(d, bits, v_packed + (base + t) * rowb, ci);
+      const float* sv = v_scales + (base + t) * ng;
+      double p = S[t] / Z;
+      for (int i = 0; i < d; ++i) orot[i] += p * ((double)sv[i / ORACLE_GROUP] * (double)C[ci[i]]);
+    }
+    for (int j = 0; j < d; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += R[(int64_t)i * d + j] * orot[i];
+      out[bh * d + j] = acc;
+    }
+    free(S);
+  }
+  free(R);
+  return fail ? -2 : 0;
 }
 
 /* ------------------------------------------------------------------ */

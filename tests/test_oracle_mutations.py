@@ -20,10 +20,14 @@ MUTATIONS = {
     "output_not_inverse_rotated": ("acc += O[(int64_t)j * d + i] * orot[i];",
                                    "acc += O[(int64_t)i * d + j] * orot[i];"),
     "signs_applied_after_hadamard": ("* (double)signs[j];", "* (double)signs[i];"),
-    "value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP]", "(double)sv[0]"),
-    "gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512]",
-                       "hk = hq % Hkv;\n    int64_t T = ctx_lens[b];\n    double qv[512]"),
-    "missing_softmax_normalizer": ("double p = S[t] / Z;", "double p = S[t];"),
+    "value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP] * (double)codes[i]",
+                                "(double)sv[0] * (double)codes[i]"),
+    "gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512], qr[512], orot[512];\n    int8_t codes",
+                       "hk = hq % Hkv;\n    int64_t T = ctx_lens[b];\n    double qv[512], qr[512], orot[512];\n    int8_t codes"),
+    "cb_gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512], qr[512], orot[512];\n    uint8_t ci",
+                          "hk = hq % Hkv;\n    int64_t T = ctx_lens[b];\n    double qv[512], qr[512], orot[512];\n    uint8_t ci"),
+    "missing_softmax_normalizer": ("double p = S[t] / Z;\n      for (int i = 0; i < d; ++i) orot[i] += p * ((double)sv[i / ORACLE_GROUP] * (double)codes[i]);",
+                                   "double p = S[t];\n      for (int i = 0; i < d; ++i) orot[i] += p * ((double)sv[i / ORACLE_GROUP] * (double)codes[i]);"),
     "byte_index_group_stride": ("+ 2 * g + (j % 4) / 2;", "+ g + (j % 4) / 2;"),
     "hartley_cos_minus_sin": ("return (cos(th) + sin(th)) / sqrt((double)d);",
                               "return (cos(th) - sin(th)) / sqrt((double)d);"),
@@ -37,6 +41,14 @@ MUTATIONS = {
                                 "f * sj * (lambda_k ? (double)lambda_k[k] : 1.0);"),
     "srft_output_without_lambda": ("sj * f / (lambda_v ? (double)lambda_v[k] : 1.0);", "sj * f;"),
     "srft_output_sign_index": ("O[(int64_t)j * d + k] = sj", "O[(int64_t)j * d + k] = (signs ? (double)signs[k] : 1.0)"),
+    "cb_tie_goes_up": ("if (u > t[i]) ++k;", "if (u >= t[i]) ++k;"),
+    "cb_sample_std": ("float sigma = (float)sqrt(S / (double)ORACLE_GROUP);",
+                      "float sigma = (float)sqrt(S / (double)(ORACLE_GROUP - 1));"),
+    "cb_clip_at_two": ("if (u > 3.0f) u = 3.0f;", "if (u > 2.0f) u = 2.0f;"),
+    "cb_bit_order_reversed": ("|= (uint8_t)(1u << (bit % 8));", "|= (uint8_t)(1u << (7 - bit % 8));"),
+    "lloyd_cell_mean_sign": ("double m = (pa - pb) / (cb - ca);", "double m = (pb - pa) / (cb - ca);"),
+    "cb_value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP] * (double)C[ci[i]]",
+                                   "(double)sv[0] * (double)C[ci[i]]"),
 }
 
 

@@ -500,3 +500,177 @@ def test_srft_reduces_to_hartley_when_unit_signs_and_lambda():
                                   oracle.srft_rotate(x))
     np.testing.assert_allclose(oracle.srft_rotate(x), x.astype(np.float64) @ _hartley_from_fft(d).T,
                                rtol=2e-7, atol=1e-7)
+
+
+# --------------------------------------------------- codebook variant
+# AdapTQ (unified SIMD pipeline; precomputed lookup tables; performance and
+# quality): 2/3/4-bit indices into a Max-Lloyd codebook with +-3 sigma
+# clipping.  The pins check the Gaussian Max-Lloyd codebook against its closed
+# form at 1 bit, its defining conditions by independent numerical integration
+# and Max's published distortions; the quantizer against nearest-level
+# assignment with an RMS scale computed here; the layout by hand-derived bytes.
+
+from math import erf as _erf, exp as _exp, pi as _pi, sqrt as _sqrt
+
+
+def _phi(x):
+    return _exp(-0.5 * x * x) / _sqrt(2 * _pi)
+
+
+def _integrate(f, a, b, n=20001):
+    """Simpson's rule on [a, b] (a, b finite)."""
+    x = np.linspace(a, b, n)
+    y = np.array([f(t) for t in x])
+    h = (b - a) / (n - 1)
+    return h / 3 * (y[0] + y[-1] + 4 * y[1:-1:2].sum() + 2 * y[2:-1:2].sum())
+
+
+def test_lloyd_max_one_bit_closed_form():
+    c = oracle.lloyd_max_gaussian(1)
+    np.testing.assert_allclose(c, [-_sqrt(2 / _pi), _sqrt(2 / _pi)], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("bits,dist", [(1, 0.3634), (2, 0.1175), (3, 0.03454), (4, 0.009497)])
+def test_lloyd_max_distortion_matches_published_table(bits, dist):
+    """Mean squared error of the Gaussian Max-Lloyd quantizer (Max, 1960), by
+    numerical integration over [-10, 10]."""
+    c = oracle.lloyd_max_gaussian(bits)
+    t = np.concatenate([[-10.0], 0.5 * (c[1:] + c[:-1]), [10.0]])
+    mse = sum(_integrate(lambda x, ci=ci: (x - ci) ** 2 * _phi(x), t[i], t[i + 1])
+              for i, ci in enumerate(c))
+    assert mse == pytest.approx(dist, rel=2e-3)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_lloyd_max_levels_are_cell_means(bits):
+    c = oracle.lloyd_max_gaussian(bits)
+    np.testing.assert_allclose(c, -c[::-1], atol=1e-12)          # symmetric
+    t = np.concatenate([[-12.0], 0.5 * (c[1:] + c[:-1]), [12.0]])
+    for i in range(len(c)):
+        num = _integrate(lambda x: x * _phi(x), t[i], t[i + 1])
+        den = _integrate(_phi, t[i], t[i + 1])
+        assert num / den == pytest.approx(c[i], abs=1e-7)
+
+
+def _rms_sigma(y):
+    return np.float32(np.sqrt(np.sum(y.astype(np.float64) ** 2) / 32))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_cb_quantizer_is_nearest_level_with_rms_scale(bits):
+    rng = np.random.default_rng(bits)
+    c = oracle.lloyd_max_gaussian(bits).astype(np.float32)
+    y = (rng.standard_normal((200, 64)) * np.exp(rng.uniform(-5, 5, (200, 1)))).astype(np.float32)
+    y[:, 7] *= 9                                               # outliers beyond 3 sigma
+    idx, sc = oracle.cb_quantize_vectors(y, bits, c)
+    for r in range(200):
+        for g in range(2):
+            yg = y[r, 32 * g:32 * g + 32]
+            s = _rms_sigma(yg)
+            assert sc[r, g] == s
+            u = np.clip((yg / s).astype(np.float32), -3, 3)
+            want = np.argmin(np.abs(u[:, None].astype(np.float64) - c[None, :]), axis=1)
+            np.testing.assert_array_equal(idx[r, 32 * g:32 * g + 32], want)
+
+
+def test_cb_quantizer_tie_and_zero_group_take_the_lower_level():
+    c = oracle.lloyd_max_gaussian(2).astype(np.float32)        # middle threshold is exactly 0
+    y = np.zeros((2, 32), np.float32)
+    y[1, 1:] = 1.0                                             # sigma = sqrt(31/32); y[1,0] = 0 sits on it
+    idx, sc = oracle.cb_quantize_vectors(y, 2, c)
+    assert sc[0, 0] == 0 and np.all(idx[0] == 1)
+    assert idx[1, 0] == 1 and np.all(idx[1, 1:] == 3)
+
+
+def test_cb_quantizer_scale_equivariance():
+    rng = np.random.default_rng(8)
+    c = oracle.lloyd_max_gaussian(3).astype(np.float32)
+    y = rng.standard_normal((20, 64)).astype(np.float32)
+    i1, s1 = oracle.cb_quantize_vectors(y, 3, c)
+    i2, s2 = oracle.cb_quantize_vectors(y * np.float32(2.0 ** 7), 3, c)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_array_equal(s1 * np.float32(2.0 ** 7), s2)
+
+
+def test_cb_pack_hand_layout():
+    idx = np.zeros((1, 64), np.uint8)
+    idx[0, :4] = [1, 2, 3, 0]
+    p2 = oracle.cb_pack(idx, 2)
+    assert p2.shape == (1, 16) and p2[0, 0] == 0x39 and not p2[0, 1:].any()
+    idx = np.zeros((1, 64), np.uint8)
+    idx[0, 0], idx[0, 1] = 5, 3                                # bits 0-2 = 101, bits 3-5 = 011
+    idx[0, 10] = 7                                             # bits 30, 31 | 32: straddles bytes 3, 4
+    idx[0, 32] = 6                                             # group 1 starts at byte 12
+    p3 = oracle.cb_pack(idx, 3)
+    assert p3.shape == (1, 24)
+    assert p3[0, 0] == 0x1D and p3[0, 3] == 0xC0 and p3[0, 4] == 0x01 and p3[0, 12] == 0x06
+    assert p3[0, [1, 2, 5, 6, 7, 8, 9, 10, 11]].sum() == 0
+    idx = np.zeros((1, 32), np.uint8)
+    idx[0, 0], idx[0, 1], idx[0, 31] = 0xA, 0x3, 0xF
+    p4 = oracle.cb_pack(idx, 4)
+    assert p4[0, 0] == 0x3A and p4[0, 15] == 0xF0
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_cb_pack_is_a_bijection(bits):
+    rng = np.random.default_rng(bits + 20)
+    idx = rng.integers(0, 1 << bits, (50, 128)).astype(np.uint8)
+    np.testing.assert_array_equal(oracle.cb_unpack(oracle.cb_pack(idx, bits), 128, bits), idx)
+
+
+def _random_cb_cache(rng, B, H, T, d, bits, c):
+    ik = rng.integers(0, 1 << bits, (B, H, T, d)).astype(np.uint8)
+    iv = rng.integers(0, 1 << bits, (B, H, T, d)).astype(np.uint8)
+    sk = rng.uniform(0.05, 0.5, (B, H, T, d // 32)).astype(np.float32)
+    sv = rng.uniform(0.05, 0.5, (B, H, T, d // 32)).astype(np.float32)
+    kp = oracle.cb_pack(ik.reshape(-1, d), bits).reshape(B, H, T, -1)
+    vp = oracle.cb_pack(iv.reshape(-1, d), bits).reshape(B, H, T, -1)
+    c64 = c.astype(np.float64)
+    khat = np.repeat(sk.astype(np.float64), 32, axis=-1) * c64[ik]
+    vhat = np.repeat(sv.astype(np.float64), 32, axis=-1) * c64[iv]
+    return (kp, sk, vp, sv), khat, vhat
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_cb_decode_brute_force_rotation_off(bits):
+    rng = np.random.default_rng(bits + 30)
+    B, Hkv, G, T, d = 2, 2, 3, 17, 64
+    c = oracle.lloyd_max_gaussian(bits).astype(np.float32)
+    cache, khat, vhat = _random_cb_cache(rng, B, Hkv, T, d, bits, c)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    out = oracle.sdpa_cb_decode(q, cache, [T, T - 5], None, bits, c, 0.2, Hkv)
+    for b, Tb in ((0, T), (1, T - 5)):
+        for h in range(Hkv * G):
+            want = _numpy_attention(q[b, h].astype(np.float64), khat[b, h // G, :Tb],
+                                    vhat[b, h // G, :Tb], 0.2)
+            np.testing.assert_allclose(out[b, h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_cb_decode_rotation_on_is_attention_in_unrotated_basis():
+    rng = np.random.default_rng(44)
+    d, Hkv, G, T, bits = 64, 1, 2, 9, 3
+    c = oracle.lloyd_max_gaussian(bits).astype(np.float32)
+    s = rand_signs(rng, d)
+    R = oracle.rotation_matrix(d, s)
+    cache, khat_r, vhat_r = _random_cb_cache(rng, 1, Hkv, T, d, bits, c)
+    q = rng.standard_normal((1, G, d)).astype(np.float32)
+    out = oracle.sdpa_cb_decode(q, cache, [T], s, bits, c, 0.3, Hkv)
+    for h in range(G):
+        want = _numpy_attention(q[0, h].astype(np.float64), khat_r[0, 0] @ R, vhat_r[0, 0] @ R, 0.3)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-11, atol=1e-12)
+
+
+def test_cb_append_rotates_then_quantizes_rows_at_pos():
+    rng = np.random.default_rng(45)
+    d, bits = 128, 2
+    c = oracle.lloyd_max_gaussian(bits).astype(np.float32)
+    s = rand_signs(rng, d)
+    k = rng.standard_normal((1, 2, 3, d)).astype(np.float32)
+    v = rng.standard_normal((1, 2, 3, d)).astype(np.float32)
+    cache = oracle.empty_cb_cache(1, 2, 8, d, bits)
+    oracle.quantize_append_cb(k, v, [4], s, bits, c, cache)
+    for h in range(2):
+        idx, sc = oracle.cb_quantize_vectors(oracle.rotate(k[0, h], s), bits, c)
+        np.testing.assert_array_equal(cache[0][0, h, 4:7], oracle.cb_pack(idx, bits))
+        np.testing.assert_array_equal(cache[1][0, h, 4:7], sc)
+        assert not cache[0][0, h, :4].any() and not cache[0][0, h, 7:].any()
