@@ -23,7 +23,9 @@ SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_t
            "tq_sdpa_int4_decode", "tq_sdpa_int4_decode_append", "tq_sdpa_int4_decode_lse",
            "tq_merge_lse", "tq_sdpa_int4_decode_static_scratch", "tq_dequantize",
            "tq_decode_srft_workspace_bytes", "tq_quantize_append_srft", "tq_sdpa_int4_decode_srft",
-           "tq_sdpa_int4_decode_append_srft", "tq_status_string")
+           "tq_sdpa_int4_decode_append_srft", "tq_lloyd_max_gaussian", "tq_decode_cb_workspace_bytes",
+           "tq_quantize_append_cb", "tq_sdpa_cb_decode", "tq_sdpa_cb_decode_append",
+           "tq_status_string")
 
 _lib = None
 
@@ -76,6 +78,19 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode_append_srft.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P, P,
                                                     P, P, i64, P, i32, P, P, P, f32, P, P, sz, P]
     lib.tq_sdpa_int4_decode_append_srft.restype = i32
+    lib.tq_lloyd_max_gaussian.argtypes = [i32, P]
+    lib.tq_lloyd_max_gaussian.restype = i32
+    lib.tq_decode_cb_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.tq_decode_cb_workspace_bytes.restype = sz
+    lib.tq_quantize_append_cb.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P,
+                                          P, i64, P]
+    lib.tq_quantize_append_cb.restype = i32
+    lib.tq_sdpa_cb_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P,
+                                      i32, P, f32, P, P, sz, P]
+    lib.tq_sdpa_cb_decode.restype = i32
+    lib.tq_sdpa_cb_decode_append.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, i32, P, P,
+                                             P, P, P, i64, P, i32, P, f32, P, P, sz, P]
+    lib.tq_sdpa_cb_decode_append.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -269,3 +284,65 @@ def sdpa_int4_decode_append_srft(q, k_new, v_new, k_packed, k_scales, v_packed, 
         _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode_append_srft")
+
+
+# ------------------------------------------------------------ codebook variant
+# AdapTQ's Max-Lloyd codebook indices at 2, 3 or 4 bits (see include/tq.h).
+
+def lloyd_max_gaussian(bits: int) -> torch.Tensor:
+    """The Gaussian Max-Lloyd codebook (float32 CPU tensor of 2**bits levels), from libtq."""
+    out = torch.empty(1 << bits, dtype=torch.float32)
+    rc = load().tq_lloyd_max_gaussian(bits, ctypes.c_void_p(out.data_ptr()))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_lloyd_max_gaussian")
+    return out
+
+
+def decode_cb_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx) -> int:
+    return int(load().tq_decode_cb_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx))
+
+
+def quantize_append_cb(k, v, pos, signs, bits, levels, k_packed, k_scales, v_packed, v_scales,
+                       stream=None):
+    """Quantize k, v [B][Hkv][n_new][d] into codebook-cache rows pos[b] .. pos[b]+n_new-1."""
+    _need_cuda(k, v, pos, signs, levels, k_packed, k_scales, v_packed, v_scales)
+    B, H, n, d = k.shape
+    rc = load().tq_quantize_append_cb(_ptr(k), _ptr(v), _dtype_code(k), B, H, n, d, 32, int(bits),
+                                      _ptr(levels), _ptr(pos), _ptr(signs), _ptr(k_packed),
+                                      _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+                                      k_packed.shape[2], _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_quantize_append_cb")
+
+
+def sdpa_cb_decode(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs, bits,
+                   levels, attn_scale, out, workspace, stream=None):
+    """out[B][Hq][d] (fp32) = attention of q over a codebook cache."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels, out, workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_cb_decode(
+        _ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, int(bits), _ptr(levels), _ptr(k_packed),
+        _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), k_packed.shape[2], _ptr(ctx_lens),
+        int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_cb_decode")
+
+
+def sdpa_cb_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                          max_ctx, signs, bits, levels, attn_scale, out, workspace, stream=None):
+    """One decode step over a codebook cache (append at row ctx_lens[b]-1, then attend)."""
+    _need_cuda(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels,
+               out, workspace)
+    if k_new.dtype != v_new.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_cb_decode_append(
+        _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq, Hkv, d, 32,
+        int(bits), _ptr(levels), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+        k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_cb_decode_append")

@@ -112,3 +112,72 @@ class Int4KVCache:
         _lib.dequantize(self.k_packed, self.k_scales, rows, k, stream)
         _lib.dequantize(self.v_packed, self.v_scales, rows, v, stream)
         return k, v
+
+
+class CodebookKVCache:
+    """The codebook variant of the cache (AdapTQ post: 2-, 3- or 4-bit indices
+    into a Max-Lloyd codebook; int2 is the 2-bit case): the same calls as
+    Int4KVCache.  levels: float32 [2**bits] increasing (default: the Gaussian
+    Max-Lloyd codebook from libtq); signs: the Hadamard rotation, or None."""
+
+    def __init__(self, batch: int, num_kv_heads: int, head_dim: int, capacity: int, bits: int = 2,
+                 device="cuda", signs: torch.Tensor | None = None,
+                 levels: torch.Tensor | None = None):
+        if head_dim not in (128, 256):
+            raise ValueError("head_dim must be 128 or 256")
+        if bits not in (2, 3, 4):
+            raise ValueError("bits must be 2, 3 or 4")
+        self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
+        self.bits = bits
+        dev = torch.device(device)
+        rb = head_dim * bits // 8
+        shape = (batch, num_kv_heads, capacity)
+        self.k_packed = torch.zeros(*shape, rb, dtype=torch.uint8, device=dev)
+        self.v_packed = torch.zeros(*shape, rb, dtype=torch.uint8, device=dev)
+        self.k_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
+        self.v_scales = torch.zeros(*shape, head_dim // 32, dtype=torch.float32, device=dev)
+        self.signs = None if signs is None else signs.to(device=dev, dtype=torch.int8).contiguous()
+        if levels is None:
+            levels = _lib.lloyd_max_gaussian(bits)
+        self.levels = levels.to(device=dev, dtype=torch.float32).contiguous()
+        self._ws = None
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.k_packed, self.v_packed, self.k_scales, self.v_scales))
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor, stream=None) -> None:
+        _lib.quantize_append_cb(k, v, pos, self.signs, self.bits, self.levels, self.k_packed,
+                                self.k_scales, self.v_packed, self.v_scales, stream)
+
+    def workspace(self, num_q_heads: int, max_ctx: int) -> torch.Tensor:
+        need = _lib.decode_cb_workspace_bytes(self.batch, num_q_heads, self.num_kv_heads,
+                                              self.head_dim, max_ctx)
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
+        return self._ws
+
+    def decode(self, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
+               attn_scale: float | None = None, out: torch.Tensor | None = None, stream=None):
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_cb_decode(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales, ctx_lens,
+                            max_ctx, self.signs, self.bits, self.levels, attn_scale, out, ws, stream)
+        return out
+
+    def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float | None = None,
+                      out: torch.Tensor | None = None, stream=None):
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_cb_decode_append(q, k_new, v_new, self.k_packed, self.k_scales, self.v_packed,
+                                   self.v_scales, ctx_lens, max_ctx, self.signs, self.bits,
+                                   self.levels, attn_scale, out, ws, stream)
+        return out

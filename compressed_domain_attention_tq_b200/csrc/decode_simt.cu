@@ -10,7 +10,12 @@
 //
 // CTA (chunk, kv head, sequence): loads the G = Hq/Hkv query rows, rotates
 // them with the cache's signs, then streams the chunk's K/V tiles through
-// shared memory.  Each chunk leaves (running max m in log2 units, sum l,
+// shared memory.  Template FMT selects the cache format: 0 = int4 codes in the
+// interleaved layout; 2, 3, 4 = the codebook variant's indices of that many
+// bits (codebook.cu), whose scores use lookup tables (AdapTQ post, section
+// "precomputed lookup tables"): with 2 bits one table of 16 partial dot
+// products per pair of coordinates and head, read with the pair's 4 index bits;
+// with 3 and 4 bits the codebook level times the query coordinate.  Each chunk leaves (running max m in log2 units, sum l,
 // unnormalized acc[d]) per query head in the workspace; merge.cu combines the
 // chunks and rotates the result back.
 #include <cuda_bf16.h>
@@ -44,10 +49,12 @@ __host__ __device__ constexpr int simt_token_parts(int G, int slices) {
   return best;
 }
 
-// Row pitch of a staged packed row in 32-bit words: odd, so lanes reading the
-// same offset of consecutive rows hit distinct banks.
-template <int D>
-__host__ __device__ constexpr int simt_pitch_words() { return D / 8 + 1; }
+// Packed row size in 32-bit words, and the staged row pitch: odd, so lanes
+// reading the same offset of consecutive rows hit distinct banks.
+template <int D, int FMT>
+__host__ __device__ constexpr int simt_row_words() { return FMT == 0 ? D / 8 : D * FMT / 32; }
+template <int D, int FMT>
+__host__ __device__ constexpr int simt_pitch_words() { return simt_row_words<D, FMT>() + 1; }
 
 // Code m of a 16-bit half-word (in-group coordinates 4r .. 4r+3 of one group)
 // as the exact float 16^m c.  t = hw ^ 0x8888 holds the biased nibbles c + 8;
@@ -58,6 +65,18 @@ __host__ __device__ constexpr int simt_pitch_words() { return D / 8 + 1; }
 __device__ __forceinline__ float code16m(uint32_t t, int m) {
   return __int_as_float((int)((t & (0xFu << (4 * m))) | 0x4B000000u)) -
          (8388608.0f + 8.0f * (float)(1 << (4 * m)));
+}
+
+// Index j (0..31) of a codebook group held in words gw[0 .. FMT-1]: bits
+// FMT*j .. FMT*j + FMT - 1 of the group's little-endian bit string.
+template <int FMT>
+__device__ __forceinline__ uint32_t cb_index(const uint32_t* gw, int j) {
+  const int bit = FMT * j;
+  if constexpr (FMT == 3) {  // may straddle two words
+    return __funnelshift_r(gw[bit >> 5], gw[(bit >> 5) + 1], bit & 31) & 7u;
+  } else {
+    return (gw[bit >> 5] >> (bit & 31)) & ((1u << FMT) - 1u);
+  }
 }
 
 // In-place Walsh-Hadamard transform of `n` rows of length D in shared memory
@@ -92,10 +111,12 @@ __device__ __forceinline__ int clamp_ctx(int T, int max_ctx) {
   return T < 1 ? 1 : (T > max_ctx ? max_ctx : T);
 }
 
-template <int D>
+template <int D, int FMT>
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   constexpr int NG = D / 32;
-  constexpr int PW = simt_pitch_words<D>();     // staged row pitch (words)
+  constexpr int RW = simt_row_words<D, FMT>();  // packed row (words)
+  constexpr int PW = simt_pitch_words<D, FMT>();  // staged row pitch (words)
+  constexpr int L = FMT == 0 ? 0 : 1 << FMT;   // codebook levels
   constexpr int SLICES = D / 8;                 // 8-coordinate slices per head
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -116,10 +137,13 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   float* mstate = scl + 4 * kTile * NG;                        // [G] running max (log2)
   float* lstate = mstate + 16;                                 // [G] running sum
   float* alpha = lstate + 16;                                  // [G] rescale of this tile
+  float* cbk = alpha + 16;                                     // [16] codebook levels
+  float* lut = cbk + 16;                                       // [G][D/2][16] (FMT 2)
   // [2 buffers][K, V][kTile][PW] staged packed rows; after the last tile the same
   // space holds the token parts' sums [TP][G][D] (TP > 1)
-  uint32_t* tiles = reinterpret_cast<uint32_t*>(alpha + 16);
+  uint32_t* tiles = reinterpret_cast<uint32_t*>(lut + (FMT == 2 ? G * D * 8 : 0));
   float* red = reinterpret_cast<float*>(tiles);
+  if (FMT != 0 && threadIdx.x < L) cbk[threadIdx.x] = a.levels[threadIdx.x];
 
   // q' = attn_scale * log2(e) * R q (the SRFT variant's R q comes rotated in q_rot)
   const int64_t qbase = ((int64_t)b * a.Hq + (int64_t)kvh * G) * D;
@@ -139,9 +163,17 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   }
   const float qmul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
   __syncthreads();
-  // 16^-(i mod 4): the codes of the score loop come scaled by 16^(i mod 4)
+  // int4: 16^-(i mod 4), as the codes of the score loop come scaled by 16^(i mod 4)
   for (int i = threadIdx.x; i < G * D; i += kThreads)
-    qs[i] *= qmul * __int_as_float((127 - 4 * (i & 3)) << 23);
+    qs[i] *= FMT == 0 ? qmul * __int_as_float((127 - 4 * (i & 3)) << 23) : qmul;
+  if constexpr (FMT == 2) {  // pair tables: lut[h][p][e] = C[e & 3] q'[2p] + C[e >> 2] q'[2p + 1]
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * D * 8; i += kThreads) {
+      const int e = i & 15, hp = i >> 4;  // hp = h * (D/2) + p
+      const int h = hp / (D / 2), pp = hp % (D / 2);
+      lut[i] = fmaf(cbk[e & 3], qs[h * D + 2 * pp], cbk[e >> 2] * qs[h * D + 2 * pp + 1]);
+    }
+  }
   if (threadIdx.x < 16) {
     mstate[threadIdx.x] = -INFINITY;
     lstate[threadIdx.x] = 0.0f;
@@ -164,10 +196,10 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     const int nt = min(kTile, t_end - t0);
     uint32_t* kt = tiles + buf * 2 * kTile * PW;
     uint32_t* vt = kt + kTile * PW;
-    const uint32_t* kg = reinterpret_cast<const uint32_t*>(a.k_packed + (rowbase + t0) * (D / 2));
-    const uint32_t* vg = reinterpret_cast<const uint32_t*>(a.v_packed + (rowbase + t0) * (D / 2));
-    for (int idx = threadIdx.x; idx < nt * (D / 8); idx += kThreads) {
-      const int r = idx / (D / 8), w = idx % (D / 8);
+    const uint32_t* kg = reinterpret_cast<const uint32_t*>(a.k_packed) + (rowbase + t0) * RW;
+    const uint32_t* vg = reinterpret_cast<const uint32_t*>(a.v_packed) + (rowbase + t0) * RW;
+    for (int idx = threadIdx.x; idx < nt * RW; idx += kThreads) {
+      const int r = idx / RW, w = idx % RW;
       cp_async4(kt + r * PW + w, kg + idx);
       cp_async4(vt + r * PW + w, vg + idx);
     }
@@ -200,7 +232,35 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
       const int tt = SP == 2 ? (idx >> 1) : idx % kTile;
       const int h = SP == 2 ? 0 : idx / kTile;
       float s = 0.0f;
-      if (tt < nt) {
+      if (tt < nt && FMT == 2) {  // pair tables: 16 pairs per group, two words
+        const uint32_t* row = ktile + tt * PW;
+        const float* lh = lut + h * D * 8;
+        for (int g = 0; g < NG; ++g) {
+          float d0 = 0.0f, d1 = 0.0f;
+          for (int w = (SP == 2 ? part : 0); w < (SP == 2 ? part + 1 : 2); ++w) {
+            const uint32_t word = row[2 * g + w];
+            const float* lp = lh + (16 * g + 8 * w) * 16;
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+              d0 += lp[16 * k + ((word >> (4 * k)) & 15u)];
+              d1 += lp[16 * (k + 1) + ((word >> (4 * k + 4)) & 15u)];
+            }
+          }
+          s = fmaf(kscale[tt * NG + g], d0 + d1, s);
+        }
+      } else if (tt < nt && FMT != 0) {  // codebook level x query coordinate
+        const uint32_t* row = ktile + tt * PW;
+        const int j_lo = SP == 2 ? 16 * part : 0, j_hi = SP == 2 ? j_lo + 16 : 32;
+        for (int g = 0; g < NG; ++g) {
+          const uint32_t* gw = row + FMT * g;
+          float d0 = 0.0f, d1 = 0.0f;
+          for (int j = j_lo; j < j_hi; j += 2) {
+            d0 = fmaf(qs[h * D + 32 * g + j], cbk[cb_index<FMT>(gw, j)], d0);
+            d1 = fmaf(qs[h * D + 32 * g + j + 1], cbk[cb_index<FMT>(gw, j + 1)], d1);
+          }
+          s = fmaf(kscale[tt * NG + g], d0 + d1, s);
+        }
+      } else if (tt < nt) {
         const uint16_t* row = reinterpret_cast<const uint16_t*>(ktile + tt * PW);
         const int r_lo = SP == 2 ? 4 * part : 0, r_hi = SP == 2 ? r_lo + 4 : 8;
         for (int g = 0; g < NG; ++g) {
@@ -258,12 +318,21 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
         }
         for (int tt = tp; tt < nt; tt += TP) {
           const float pw = sp[h * kTile + tt] * vscale[tt * NG + g];
-          const uint16_t* row = reinterpret_cast<const uint16_t*>(vtile + tt * PW);
-          const uint32_t t0 = row[r0 * NG + g] ^ 0x8888u, t1 = row[(r0 + 1) * NG + g] ^ 0x8888u;
+          if constexpr (FMT == 0) {
+            const uint16_t* row = reinterpret_cast<const uint16_t*>(vtile + tt * PW);
+            const uint32_t t0 = row[r0 * NG + g] ^ 0x8888u, t1 = row[(r0 + 1) * NG + g] ^ 0x8888u;
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            acc[it][m] = fmaf(pw, code16m(t0, m), acc[it][m]);
-            acc[it][4 + m] = fmaf(pw, code16m(t1, m), acc[it][4 + m]);
+            for (int m = 0; m < 4; ++m) {
+              acc[it][m] = fmaf(pw, code16m(t0, m), acc[it][m]);
+              acc[it][4 + m] = fmaf(pw, code16m(t1, m), acc[it][4 + m]);
+            }
+          } else {  // the slice's 8 indices: FMT * 8 bits at bit FMT * 8 * (sl % 4) of the group
+            const uint32_t* gw = vtile + tt * PW + FMT * g;
+            const int bit = FMT * 8 * (sl % 4);
+            const uint32_t v8 = __funnelshift_r(gw[bit >> 5], gw[(bit >> 5) + 1], bit & 31);
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+              acc[it][m] = fmaf(pw, cbk[(v8 >> (FMT * m)) & (L - 1)], acc[it][m]);
           }
         }
       }
@@ -271,11 +340,12 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     __syncthreads();  // the tile's buffers and scores are free for the next stage
   }
 
-  // slot e of a P.V item holds 16^(e mod 4) times its sum
+  if constexpr (FMT == 0) {  // slot e of a P.V item holds 16^(e mod 4) times its sum
 #pragma unroll
-  for (int it = 0; it < 4; ++it)
+    for (int it = 0; it < 4; ++it)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[it][e] *= __int_as_float((127 - 4 * (e & 3)) << 23);
+      for (int e = 0; e < 8; ++e) acc[it][e] *= __int_as_float((127 - 4 * (e & 3)) << 23);
+  }
 
   // partials: ws[b][hq][chunk][0..D) = acc, [D] = m, [D+1] = l
   float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) + a.plan.header_bytes);
@@ -321,39 +391,55 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   }
 }
 
-template <int D>
+template <int D, int FMT>
 size_t simt_smem_bytes(int G) {
   constexpr int NG = D / 32;
   const int TP = simt_token_parts(G, D / 8);
-  const size_t tile_words = 4 * (size_t)kTile * simt_pitch_words<D>();
+  const size_t tile_words = 4 * (size_t)kTile * simt_pitch_words<D, FMT>();
   const size_t red_words = TP > 1 ? (size_t)TP * G * D : 0;
-  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 48) +
+  const size_t lut_words = FMT == 2 ? (size_t)G * D * 8 : 0;
+  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 64 + lut_words) +
          sizeof(uint32_t) * (tile_words > red_words ? tile_words : red_words);
 }
 
-template <int D>
+template <int D, int FMT>
 size_t simt_smem_max() {  // over every group size the host accepts (up to 16 query heads)
   size_t m = 0;
-  for (int G = 1; G <= 16; ++G) m = simt_smem_bytes<D>(G) > m ? simt_smem_bytes<D>(G) : m;
+  for (int G = 1; G <= 16; ++G) {
+    const size_t b = simt_smem_bytes<D, FMT>(G);
+    m = b > m ? b : m;
+  }
   return m;
 }
 
-template <int D>
+template <int D, int FMT = 0>
 cudaError_t launch_simt_d(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   dim3 grid(a.plan.n_chunks, a.Hkv, a.B);
   static std::atomic<uint64_t> smem_set{0};
-  const cudaError_t e = ensure_smem_limit(decode_simt_kernel<D>, (int)simt_smem_max<D>(), smem_set);
+  const cudaError_t e =
+      ensure_smem_limit(decode_simt_kernel<D, FMT>, (int)simt_smem_max<D, FMT>(), smem_set);
   if (e != cudaSuccess) return e;
-  decode_simt_kernel<D><<<grid, kThreads, simt_smem_bytes<D>(G), stream>>>(a);
+  decode_simt_kernel<D, FMT><<<grid, kThreads, simt_smem_bytes<D, FMT>(G), stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_simt_cb(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.cb_bits) {
+    case 2: return launch_simt_d<D, 2>(a, stream);
+    case 3: return launch_simt_d<D, 3>(a, stream);
+    case 4: return launch_simt_d<D, 4>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
-// head_dim 128 or 256; with the SRFT variant (rotated queries given) any
-// multiple of 32 up to 256
+// int4: head_dim 128 or 256, and with the SRFT variant (rotated queries given)
+// any multiple of 32 up to 256; codebook variant: head_dim 128 or 256
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.cb_bits != 0) return a.d == 128 ? launch_simt_cb<128>(a, stream) : launch_simt_cb<256>(a, stream);
   switch (a.d) {
     case 32: return launch_simt_d<32>(a, stream);
     case 64: return launch_simt_d<64>(a, stream);

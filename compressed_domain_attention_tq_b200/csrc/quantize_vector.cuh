@@ -13,13 +13,11 @@
 
 namespace tq {
 
+// Lane l loads coordinates E*l .. E*l+E-1 (E = D/32) of one fp32 or bf16 vector.
 template <int D>
-__device__ __forceinline__ void quantize_vector_warp(const void* src, bool bf16, const int8_t* signs,
-                                                     uint8_t* packed_row, float* scale_row, int lane) {
-  constexpr int E = D / 32;   // coordinates per lane
-  constexpr int GL = 32 / E;  // lanes per quantization group
-  constexpr int NG = D / 32;
-  float x[E];
+__device__ __forceinline__ void load_vector_warp(const void* src, bool bf16, float (&x)[D / 32],
+                                                 int lane) {
+  constexpr int E = D / 32;
   if (bf16) {
     const uint16_t* s16 = static_cast<const uint16_t*>(src) + lane * E;
 #pragma unroll
@@ -29,6 +27,13 @@ __device__ __forceinline__ void quantize_vector_warp(const void* src, bool bf16,
 #pragma unroll
     for (int e = 0; e < E; ++e) x[e] = s32[e];
   }
+}
+
+// In place: x <- H_D (signs (.) x) / sqrt(D) for the lane layout above (D = 128
+// or 256), butterflies in the order bits 1, 2, 4, ...; nothing when signs is NULL.
+template <int D>
+__device__ __forceinline__ void rotate_vector_warp(float (&x)[D / 32], const int8_t* signs, int lane) {
+  constexpr int E = D / 32;
   if (signs) {
 #pragma unroll
     for (int e = 0; e < E; ++e)
@@ -53,6 +58,17 @@ __device__ __forceinline__ void quantize_vector_warp(const void* src, bool bf16,
 #pragma unroll
     for (int e = 0; e < E; ++e) x[e] *= norm;
   }
+}
+
+template <int D>
+__device__ __forceinline__ void quantize_vector_warp(const void* src, bool bf16, const int8_t* signs,
+                                                     uint8_t* packed_row, float* scale_row, int lane) {
+  constexpr int E = D / 32;   // coordinates per lane
+  constexpr int GL = 32 / E;  // lanes per quantization group
+  constexpr int NG = D / 32;
+  float x[E];
+  load_vector_warp<D>(src, bf16, x, lane);
+  rotate_vector_warp<D>(x, signs, lane);
   float amax = 0.0f;
 #pragma unroll
   for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));

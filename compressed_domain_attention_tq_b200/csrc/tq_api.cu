@@ -20,12 +20,13 @@ static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // an item is one (sequence, kv head, chunk).  The tensor-core decode runs
 // persistent CTAs, one per SM; the CUDA-core decode runs one 128-thread CTA
 // per item, several resident per SM.
-bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan, bool srft) {
+bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan, PlanKind kind) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
+  const bool srft = kind == PlanKind::kSrft;
   if (srft ? !srft_head_dim_supported(d) : (d != 128 && d != 256)) return false;
   const int64_t units = (int64_t)B * Hkv;
-  const bool mma = decode_mma_supported(d, Hq / Hkv);
-  const int64_t step = decode_stage_tokens(d, Hq / Hkv), per_item_cost = mma ? 384 : 256;
+  const bool mma = kind != PlanKind::kCodebook && decode_mma_supported(d, Hq / Hkv);
+  const int64_t step = mma ? decode_stage_tokens(d, Hq / Hkv) : 128, per_item_cost = mma ? 384 : 256;
   const int64_t slots = mma ? kSmCount : 4 * kSmCount;
   const int64_t max_n = ceil_div(max_ctx, step);
   int64_t best_chunk = ceil_div(max_ctx, step) * step, best_cost = -1;
@@ -63,16 +64,24 @@ static tq_status cuda_status(cudaError_t e, const char* where) {
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// The rotation of a call: the Hadamard rotation (signs) or none, or the SRFT
-// variant (srft: signs, optional per-coordinate scales of K and V).
+// The variant of a call: the int4 cache with the Hadamard rotation (signs) or
+// none; the SRFT variant (srft: signs, optional per-coordinate scales of K and
+// V); or the codebook variant (cb_bits 2..4 with its levels, Hadamard or none).
 struct Rotation {
   bool srft = false;
   const float* lambda_k = nullptr;
   const float* lambda_v = nullptr;
+  int cb_bits = 0;
+  const float* levels = nullptr;
 };
 
 static bool head_dim_ok(int d, const Rotation& rot) {
   return rot.srft ? srft_head_dim_supported(d) : (d == 128 || d == 256);
+}
+
+static bool codebook_ok(const Rotation& rot) {
+  return rot.cb_bits == 0 || ((rot.cb_bits >= 2 && rot.cb_bits <= 4) && rot.levels != nullptr &&
+                              (reinterpret_cast<uintptr_t>(rot.levels) & 3u) == 0);
 }
 
 }  // namespace tq
@@ -108,6 +117,8 @@ static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, 
   if ((int64_t)batch * num_kv_heads * n_new > INT32_MAX) return TQ_ERR_INVALID_ARG;
   if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (rot.cb_bits != 0 && (rot.cb_bits < 2 || rot.cb_bits > 4)) return TQ_ERR_UNSUPPORTED;
+  if (!codebook_ok(rot)) return TQ_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_packed) || !aligned16(v_packed) ||
       !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(rot.lambda_k) ||
       !aligned4(rot.lambda_v))
@@ -129,8 +140,13 @@ static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, 
   a.capacity = capacity;
   a.lambda_k = rot.lambda_k;
   a.lambda_v = rot.lambda_v;
+  a.cb_bits = rot.cb_bits;
+  a.levels = rot.levels;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  return cuda_status(rot.srft ? launch_quantize_srft(a, s) : launch_quantize(a, s), where);
+  const cudaError_t e = rot.srft ? launch_quantize_srft(a, s)
+                        : rot.cb_bits ? launch_quantize_cb(a, s)
+                                      : launch_quantize(a, s);
+  return cuda_status(e, where);
 }
 
 extern "C" {
@@ -154,6 +170,39 @@ tq_status tq_quantize_append_srft(const void* k, const void* v, tq_dtype in_dtyp
   return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs,
                        Rotation{true, lambda_k, lambda_v}, k_packed, k_scales, v_packed,
                        v_scales, capacity, cuda_stream, "tq_quantize_append_srft");
+}
+
+tq_status tq_quantize_append_cb(const void* k, const void* v, tq_dtype in_dtype, int32_t batch,
+                                int32_t num_kv_heads, int32_t n_new, int32_t head_dim,
+                                int32_t group, int32_t bits, const float* levels,
+                                const int32_t* pos, const int8_t* signs, uint8_t* k_packed,
+                                float* k_scales, uint8_t* v_packed, float* v_scales,
+                                int64_t capacity, void* cuda_stream) {
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs, r,
+                       k_packed, k_scales, v_packed, v_scales, capacity, cuda_stream,
+                       "tq_quantize_append_cb");
+}
+
+tq_status tq_lloyd_max_gaussian(int32_t bits, float* levels) {
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  if (!levels) return TQ_ERR_INVALID_ARG;
+  double c[16];
+  lloyd_max_gaussian(bits, c);
+  for (int i = 0; i < (1 << bits); ++i) levels[i] = (float)c[i];
+  return TQ_OK;
+}
+
+size_t tq_decode_cb_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t max_ctx) {
+  DecodePlan p;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p,
+                        PlanKind::kCodebook))
+    return 0;
+  return p.ws_bytes;
 }
 
 tq_status tq_dequantize(const uint8_t* packed, const float* scales, int32_t n_seq, int32_t rows,
@@ -187,7 +236,8 @@ size_t tq_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
 size_t tq_decode_srft_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                       int32_t head_dim, int32_t max_ctx) {
   DecodePlan p;
-  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p, true)) return 0;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p, PlanKind::kSrft))
+    return 0;
   return p.ws_bytes;
 }
 
@@ -226,12 +276,16 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
   if (group != kGroup) return TQ_ERR_UNSUPPORTED;
   if (num_q_heads / num_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
+  if (!codebook_ok(rot)) return TQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(v_packed) ||
       !aligned16(k_scales) || !aligned16(v_scales) || (lse && (reinterpret_cast<uintptr_t>(lse) & 7u)) ||
       !aligned4(rot.lambda_k) || !aligned4(rot.lambda_v))
     return TQ_ERR_INVALID_ARG;
   DecodeArgs a;
-  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan, rot.srft))
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &a.plan,
+                        rot.srft ? PlanKind::kSrft
+                        : rot.cb_bits ? PlanKind::kCodebook
+                                      : PlanKind::kInt4))
     return TQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < a.plan.ws_bytes) return TQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
@@ -258,11 +312,13 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   a.lse = lse;
   a.lambda_k = rot.lambda_k;
   a.lambda_v = rot.lambda_v;
+  a.cb_bits = rot.cb_bits;
+  a.levels = rot.levels;
   a.q_rot = rot.srft ? reinterpret_cast<const float*>(static_cast<unsigned char*>(workspace) +
                                                       a.plan.qrot_offset)
                      : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const bool mma = decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
+  const bool mma = rot.cb_bits == 0 && decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
   if (append && mma && !rot.srft) {  // the decode kernel quantizes the new tokens itself
     a.k_new = k_new;
     a.v_new = v_new;
@@ -286,7 +342,11 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     qa.capacity = capacity;
     qa.lambda_k = rot.lambda_k;
     qa.lambda_v = rot.lambda_v;
-    const cudaError_t e = rot.srft ? launch_quantize_srft(qa, s) : launch_quantize(qa, s);
+    qa.cb_bits = rot.cb_bits;
+    qa.levels = rot.levels;
+    const cudaError_t e = rot.srft ? launch_quantize_srft(qa, s)
+                          : rot.cb_bits ? launch_quantize_cb(qa, s)
+                                        : launch_quantize(qa, s);
     if (e != cudaSuccess) return cuda_status(e, where);
   }
   if (rot.srft) {  // rotated queries into the workspace, read by the decode kernel
@@ -365,6 +425,43 @@ tq_status tq_sdpa_int4_decode_append_srft(
                      head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
                      max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
                      "tq_sdpa_int4_decode_append_srft", nullptr, Rotation{true, lambda_k, lambda_v});
+}
+
+tq_status tq_sdpa_cb_decode(const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t group, int32_t bits,
+                           const float* levels, const uint8_t* k_packed, const float* k_scales,
+                           const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                           const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                           float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream) {
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_cb_decode", nullptr, r);
+}
+
+tq_status tq_sdpa_cb_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
+                                   const void* v_new, tq_dtype kv_dtype, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t group, int32_t bits, const float* levels,
+                                   uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                                   float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+                                   int32_t max_ctx, const int8_t* signs, float attn_scale,
+                                   float* out, void* workspace, size_t workspace_bytes,
+                                   void* cuda_stream) {
+  if (!k_new || !v_new) return TQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  return decode_impl(q, q_dtype, k_new, v_new, kv_dtype, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_cb_decode_append", nullptr, r);
 }
 
 tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,

@@ -22,10 +22,12 @@ struct DecodePlan {
   size_t ws_bytes;  // header + partials (+ rotated queries)
 };
 
-// srft: the SRFT variant's plan (any head_dim accepted by srft_head_dim_supported,
-// plus room for the rotated queries); otherwise head_dim 128 or 256.
+// kind: the int4 cache (head_dim 128 or 256), the SRFT variant (any head_dim
+// accepted by srft_head_dim_supported, plus room for the rotated queries), or
+// the codebook variant (head_dim 128 or 256, always the CUDA-core decode).
+enum class PlanKind { kInt4, kSrft, kCodebook };
 bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan,
-                      bool srft = false);
+                      PlanKind kind = PlanKind::kInt4);
 
 struct QuantizeArgs {
   const void* k;
@@ -43,6 +45,8 @@ struct QuantizeArgs {
   int max_ctx = 0;
   const float* lambda_k = nullptr;  // SRFT variant: per-coordinate scales (NULL = ones)
   const float* lambda_v = nullptr;
+  int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
+  const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
 };
 
 struct DequantizeArgs {
@@ -78,6 +82,8 @@ struct DecodeArgs {
                                     // the decode kernels read these instead of rotating q
   const float* lambda_k = nullptr;  // SRFT variant: per-coordinate scales (NULL = ones)
   const float* lambda_v = nullptr;
+  int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
+  const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
 };
 
 // Raise a kernel's dynamic shared memory limit once per device (the first
@@ -106,6 +112,8 @@ bool srft_head_dim_supported(int d);
 cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_quantize_cb(const QuantizeArgs& a, cudaStream_t stream);
+void lloyd_max_gaussian(int bits, double* levels);
 cudaError_t launch_merge_lse(const float* outs, const float* lses, int n_parts, int64_t n_heads,
                              int d, float* out, cudaStream_t stream);
 

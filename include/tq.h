@@ -337,6 +337,61 @@ TQ_API tq_status tq_sdpa_int4_decode_append_srft(
     const float* lambda_v, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
     void* cuda_stream);
 
+/*
+ * Codebook variant (the AdapTQ post, sections "unified SIMD pipeline",
+ * "precomputed lookup tables", "performance and quality": 2-, 3- and 4-bit
+ * indices into a Max-Lloyd codebook with +-3 sigma clipping; int2 is the
+ * future work of Open-TQ-Metal).  After the Hadamard rotation of the int4
+ * calls (signs, or none), each group of 32 coordinates y stores
+ *     sigma = fl32(sqrt(S / 32)), S = sum of y^2 accumulated in fp64,
+ *     index_j = #{ i : u_j > t_i },  u_j = clamp(fl32(y_j / sigma), -3, 3)
+ *               (u_j = 0 when sigma = 0),  t_i = fl32(fl32(C_i + C_{i+1}) * 0.5),
+ * and the value sigma * C[index].  Layout (row-major, dense):
+ *  - packed cache: uint8 [B][Hkv][capacity][d * bits / 8]; a row holds its
+ *    d/32 groups in order, 4 * bits bytes each; index j of a group occupies
+ *    bits bits*j .. bits*j + bits - 1 of the group's little-endian bit string.
+ *  - scales: float [B][Hkv][capacity][d/32] (sigma per group).
+ *  - levels: float [2^bits] on the device, strictly increasing (not checked
+ *    on the device; the host checks only the pointer, 4-byte aligned).
+ * head_dim 128 or 256; bits 2, 3 or 4 (else TQ_ERR_UNSUPPORTED); every other
+ * argument, alignment rule and error is that of the int4 calls.  The decode
+ * runs on CUDA cores; with 2 bits its scores read tables of 16 partial dot
+ * products per pair of query coordinates (the post's lookup tables).
+ */
+
+/* The Gaussian Max-Lloyd codebook of 2^bits levels (N(0,1) cell means at
+ * midpoint thresholds), written to a HOST array of 2^bits floats. */
+TQ_API tq_status tq_lloyd_max_gaussian(int32_t bits, float* levels);
+
+/* Workspace bytes for tq_sdpa_cb_decode(_append); 0 for invalid sizes. */
+TQ_API size_t tq_decode_cb_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                           int32_t num_kv_heads, int32_t head_dim,
+                                           int32_t max_ctx);
+
+/* tq_quantize_append for a codebook cache (one warp per vector). */
+TQ_API tq_status tq_quantize_append_cb(
+    const void* k, const void* v, tq_dtype in_dtype, int32_t batch, int32_t num_kv_heads,
+    int32_t n_new, int32_t head_dim, int32_t group, int32_t bits, const float* levels,
+    const int32_t* pos, const int8_t* signs, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, void* cuda_stream);
+
+/* tq_sdpa_int4_decode over a codebook cache (split-K decode + merge). */
+TQ_API tq_status tq_sdpa_cb_decode(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, int32_t bits, const float* levels, const uint8_t* k_packed,
+    const float* k_scales, const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+    const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, float attn_scale, float* out,
+    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* tq_sdpa_int4_decode_append over a codebook cache (append launch, then decode). */
+TQ_API tq_status tq_sdpa_cb_decode_append(
+    const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
+    int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+    float* v_scales, int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx,
+    const int8_t* signs, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+    void* cuda_stream);
+
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);
 

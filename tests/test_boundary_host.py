@@ -211,3 +211,40 @@ def test_product_path_has_no_oracle_import():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "oracle.c" not in txt and "liboracle" not in txt, f
+
+
+def test_codebook_generator_matches_oracle(lib):
+    """libtq's Gaussian Max-Lloyd codebook (host code) equals the oracle's in fp32."""
+    import numpy as np
+
+    import oracle
+    for bits in (2, 3, 4):
+        np.testing.assert_array_equal(_lib.lloyd_max_gaussian(bits).numpy(),
+                                      oracle.lloyd_max_gaussian(bits).astype(np.float32))
+
+
+def test_codebook_calls_reject_on_host(lib):
+    fb = FakeBuffers()
+    args = lambda **kw: dict(dict(k=fb.p(0), v=fb.p(4096), dtype=1, B=1, H=2, n=3, d=128, group=32,
+                                  bits=2, levels=fb.p(8192), pos=fb.p(512), signs=None,
+                                  kp=fb.p(1024), ks=fb.p(2048), vp=fb.p(3072), vs=fb.p(16384),
+                                  cap=16, stream=None), **kw)
+    def q(**kw):
+        a = args(**kw)
+        return lib.tq_quantize_append_cb(a["k"], a["v"], a["dtype"], a["B"], a["H"], a["n"], a["d"],
+                                         a["group"], a["bits"], a["levels"], a["pos"], a["signs"],
+                                         a["kp"], a["ks"], a["vp"], a["vs"], a["cap"], a["stream"])
+    assert q(bits=1) == _lib.TQ_ERR_UNSUPPORTED and q(bits=5) == _lib.TQ_ERR_UNSUPPORTED
+    assert q(levels=None) == _lib.TQ_ERR_INVALID_ARG and q(levels=fb.p(8194)) == _lib.TQ_ERR_INVALID_ARG
+    assert q(d=96) == _lib.TQ_ERR_UNSUPPORTED and q(k=None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_lloyd_max_gaussian(5, None) == _lib.TQ_ERR_UNSUPPORTED
+    assert lib.tq_lloyd_max_gaussian(2, None) == _lib.TQ_ERR_INVALID_ARG
+    assert _lib.decode_cb_workspace_bytes(1, 8, 2, 96, 64) == 0
+    assert _lib.decode_cb_workspace_bytes(1, 8, 2, 128, 64) > 0
+    def dec(bits=2, levels=fb.p(8192), ws_bytes=1 << 15):
+        return lib.tq_sdpa_cb_decode(fb.p(0), 1, 1, 8, 2, 128, 32, bits, levels, fb.p(1024),
+                                     fb.p(2048), fb.p(3072), fb.p(4096), 64, fb.p(512), 64, None,
+                                     0.125, fb.p(8192), fb.p(16384), ws_bytes, None)
+    assert dec(bits=7) == _lib.TQ_ERR_UNSUPPORTED
+    assert dec(levels=None) == _lib.TQ_ERR_INVALID_ARG
+    assert dec(ws_bytes=100) == _lib.TQ_ERR_WORKSPACE
