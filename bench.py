@@ -62,7 +62,8 @@ def measured_peaks():
 
 def kv_bytes(w, ctx_tokens):
     """Packed codes + fp32 scales of K and V read by one decode (all sequences)."""
-    per_vec = w.head_dim // 2 + 4 * (w.head_dim // 32)
+    code_bytes = w.head_dim * w.cb_bits // 8 if w.cb_bits else w.head_dim // 2
+    per_vec = code_bytes + 4 * (w.head_dim // 32)
     return 2 * per_vec * w.num_kv_heads * int(sum(ctx_tokens))
 
 
@@ -168,8 +169,11 @@ def run_tq(args):
     srft = w.rotation and w.rotation_kind == "srft"
     lk, lv = wl.make_lambdas(w, seed)
     ctx = wl.make_context_lengths(w, seed)                    # cached tokens per sequence
-    cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs,
-                           rotation="srft" if srft else "hadamard", lambda_k=lk, lambda_v=lv)
+    if w.cb_bits:
+        cache = tq.CodebookKVCache(B, Hkv, d, w.capacity, w.cb_bits, dev, signs)
+    else:
+        cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs,
+                               rotation="srft" if srft else "hadamard", lambda_k=lk, lambda_v=lv)
     k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
     pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -189,7 +193,8 @@ def run_tq(args):
                 times.append(e0.elapsed_time(e1) / 1e3)
         t = min(times)
         nvec = 2 * B * Hkv * k_all.shape[2]
-        moved = k_all.numel() * k_all.element_size() * 2 + nvec * (d // 2 + 4 * (d // 32))
+        code_bytes = d * w.cb_bits // 8 if w.cb_bits else d // 2
+        moved = k_all.numel() * k_all.element_size() * 2 + nvec * (code_bytes + 4 * (d // 32))
         prefill = {"tokens": int(k_all.shape[2]), "us": round(t * 1e6, 2),
                    "tokens_per_s": round(B * k_all.shape[2] / t, 1),
                    "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),
@@ -317,26 +322,32 @@ def run_tq(args):
         import numpy as np
         cache.decode(q, ctx_dev, max_ctx, scale, out)
         Qm, Om = basis_maps(d, signs, lk, lv, srft, dev)
-        bl = dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, Qm, Om,
-                                     min(args.steps, 50), 3, stream)
-        o_ours, o_bl = out.double().flatten(1), bl.pop("out").double().flatten(1)
-        bl["cosine_vs_int4_path_min"] = round(float(torch.nn.functional.cosine_similarity(
-            o_ours, o_bl, dim=1).min()), 5)
-        bl["int4_decode_speedup"] = round(bl["dequantize_then_attend_us"] / (dec_s * 1e6), 2)
-        baseline = bl
-        khat, _ = cache.dequantize(ctx0 + 1, torch.float32)
+        khat = None
+        if not w.cb_bits:  # tq_dequantize reads the int4 layout
+            bl = dequant_attend_baseline(cache, q, ctx_dev, max_ctx, scale, Qm, Om,
+                                         min(args.steps, 50), 3, stream)
+            o_ours, o_bl = out.double().flatten(1), bl.pop("out").double().flatten(1)
+            bl["cosine_vs_int4_path_min"] = round(float(torch.nn.functional.cosine_similarity(
+                o_ours, o_bl, dim=1).min()), 5)
+            bl["int4_decode_speedup"] = round(bl["dequantize_then_attend_us"] / (dec_s * 1e6), 2)
+            baseline = bl
+            khat, _ = cache.dequantize(ctx0 + 1, torch.float32)
+            khat = khat[0, :n_fid].cpu().numpy()
         G = Hq // Hkv
         fid_k = np.concatenate([fid_k.numpy(), k_new[0, :n_fid].float().cpu().numpy()], 1)
         fid_v = np.concatenate([fid_v.numpy(), v_new[0, :n_fid].float().cpu().numpy()], 1)
         fid = fidelity(fid_k, fid_v, q[0, :n_fid * G].float().cpu().numpy(),
-                       out[0, :n_fid * G].cpu().numpy(), khat[0, :n_fid].cpu().numpy(),
-                       Qm.cpu().numpy(), scale, G)
+                       out[0, :n_fid * G].cpu().numpy(), khat, Qm.cpu().numpy(), scale, G)
         fid["sample"] = f"sequence 0, kv heads 0..{n_fid - 1} ({n_fid * G} query heads), {ctx0 + 1} tokens"
         del khat
 
     kvb = kv_bytes(w, (ctx + 1).tolist())
-    mma = (d == 128 and Hq // Hkv <= 8) or (d == 256 and Hq // Hkv <= 4)
-    if srft:
+    mma = not w.cb_bits and ((d == 128 and Hq // Hkv <= 8) or (d == 256 and Hq // Hkv <= 4))
+    if w.cb_bits:
+        launches_per_step = 3
+        step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): quantize-append "
+                     "of the new token, split-K decode, merge (3 launches)")
+    elif srft:
         launches_per_step = 4
         step_desc = ("tq_sdpa_int4_decode_append_srft: SRFT quantize-append of the new token, query "
                      "rotation, split-K decode, merge with the inverse transform (4 launches)")
@@ -365,6 +376,7 @@ def run_tq(args):
         "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
                    "context": max_ctx,
                    "rotation": (w.rotation_kind if w.rotation else False),
+                   "codes": f"{w.cb_bits}-bit Max-Lloyd codebook" if w.cb_bits else "int4",
                    "attn_scale": scale,
                    "kv_bytes_per_step": kvb,
                    "l2": (f"flushed by a {flush.numel()} B write before each step inside the "
@@ -501,10 +513,12 @@ def fidelity(k_h, v_h, q_h, out_h, khat_h, Qm, scale, G):
         O = (P.T @ V) / P.sum(0)[:, None]
         Og = out_h[h * G:(h + 1) * G].astype(np.float64)
         cos += list((O * Og).sum(1) / (np.linalg.norm(O, axis=1) * np.linalg.norm(Og, axis=1)))
-        Sq = khat_h[h].astype(np.float64) @ (Q @ Qm.T).T
-        agree += list(S.argmax(0) == Sq.argmax(0))
+        if khat_h is not None:
+            Sq = khat_h[h].astype(np.float64) @ (Q @ Qm.T).T
+            agree += list(S.argmax(0) == Sq.argmax(0))
     return {"cosine_min": round(float(min(cos)), 7), "cosine_mean": round(float(np.mean(cos)), 7),
-            "top1_qk_argmax_agreement": round(float(np.mean(agree)), 4), "query_heads": len(cos)}
+            "top1_qk_argmax_agreement": round(float(np.mean(agree)), 4) if agree else None,
+            "query_heads": len(cos)}
 
 
 def oracle_sample(w, seed, kv_head=0):
@@ -528,10 +542,14 @@ def oracle_sample(w, seed, kv_head=0):
     signs = wl.make_signs(w.head_dim, seed).numpy() if w.rotation else None
     lk, lv = wl.make_lambdas(w, seed)
     lam = None if lk is None else (lk.numpy(), lv.numpy())
-    cache = oracle.empty_cache(1, 1, w.capacity, w.head_dim)
+    if w.cb_bits:
+        cache = oracle.empty_cb_cache(1, 1, w.capacity, w.head_dim, w.cb_bits)
+    else:
+        cache = oracle.empty_cache(1, 1, w.capacity, w.head_dim)
     thr = oracle.max_threads()
+    levels = oracle.lloyd_max_gaussian(w.cb_bits).astype(np.float32) if w.cb_bits else None
     s = dict(k_new=bits(k[:, :, -1:]), v_new=bits(v[:, :, -1:]), q=bits(q), signs=signs, lam=lam,
-             cache=cache, threads=thr, G=G, T=w.capacity - 1)
+             cache=cache, threads=thr, G=G, T=w.capacity - 1, cb_bits=w.cb_bits, levels=levels)
     t0 = time.perf_counter()
     oracle_append(s, bits(k[:, :, :-1]), bits(v[:, :, :-1]), 0)
     s["prefill_s"] = time.perf_counter() - t0
@@ -540,7 +558,10 @@ def oracle_sample(w, seed, kv_head=0):
 
 def oracle_append(s, k, v, pos):
     import oracle
-    if s["lam"] is None:
+    if s["cb_bits"]:
+        oracle.quantize_append_cb(k, v, [pos], s["signs"], s["cb_bits"], s["levels"], s["cache"],
+                                  threads=s["threads"])
+    elif s["lam"] is None:
         oracle.quantize_append(k, v, [pos], s["signs"], s["cache"], threads=s["threads"])
     else:
         oracle.quantize_append_srft(k, v, [pos], s["signs"], s["lam"][0], s["lam"][1], s["cache"],
@@ -550,6 +571,9 @@ def oracle_append(s, k, v, pos):
 def oracle_step(s, w):
     import oracle
     oracle_append(s, s["k_new"], s["v_new"], s["T"])
+    if s["cb_bits"]:
+        return oracle.sdpa_cb_decode(s["q"], s["cache"], [s["T"] + 1], s["signs"], s["cb_bits"],
+                                     s["levels"], w.attn_scales[0], 1, threads=s["threads"])
     if s["lam"] is None:
         return oracle.sdpa_int4_decode(s["q"], s["cache"], [s["T"] + 1], s["signs"],
                                        w.attn_scales[0], 1, threads=s["threads"])
@@ -565,7 +589,7 @@ def cpu_baseline(w, seed):
         oracle_step(s, w)
         ts.append(time.perf_counter() - t0)
     t = min(ts)
-    kvb = 2 * (s["T"] + 1) * (w.head_dim // 2 + 4 * (w.head_dim // 32))
+    kvb = kv_bytes(w, [s["T"] + 1]) // w.num_kv_heads
     return {"value": round(kvb / t / 1e9, 4), "unit": "GB/s", "cores": s["threads"], "kind": "oracle",
             "us_per_step_sample": round(t * 1e6, 1),
             "sample": (f"kv head 0 of {w.num_kv_heads} ({s['G']} query heads) at {s['T'] + 1}-token "
@@ -588,7 +612,7 @@ def run_reference(args):
         oracle_step(s, w)
         ts.append(time.perf_counter() - t0)
     t = sum(ts) / len(ts)
-    kvb = 2 * (s["T"] + 1) * (w.head_dim // 2 + 4 * (w.head_dim // 32))
+    kvb = kv_bytes(w, [s["T"] + 1]) // w.num_kv_heads
     val = kvb / t / 1e9
     sample = (f"kv head 0 of {w.num_kv_heads} ({s['G']} query heads) at {s['T'] + 1}-token context; "
               f"each step = oracle quantize-append of 1 token + fp64 decode")

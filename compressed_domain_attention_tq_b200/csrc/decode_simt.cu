@@ -49,6 +49,11 @@ __host__ __device__ constexpr int simt_token_parts(int G, int slices) {
   return best;
 }
 
+// Token parts of the shared-code P.V items of codebook caches: one item per
+// (8-dim slice, part) fills the block's 128 threads.
+template <int D>
+__host__ __device__ constexpr int simt_shared_token_parts() { return kThreads / (D / 8); }
+
 // Packed row size in 32-bit words, and the staged row pitch: odd, so lanes
 // reading the same offset of consecutive rows hit distinct banks.
 template <int D, int FMT>
@@ -112,11 +117,12 @@ __device__ __forceinline__ int clamp_ctx(int T, int max_ctx) {
 }
 
 template <int D, int FMT>
-__global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel(DecodeArgs a) {
   constexpr int NG = D / 32;
   constexpr int RW = simt_row_words<D, FMT>();  // packed row (words)
   constexpr int PW = simt_pitch_words<D, FMT>();  // staged row pitch (words)
   constexpr int L = FMT == 0 ? 0 : 1 << FMT;   // codebook levels
+  constexpr uint32_t LMASK = FMT == 0 ? 1u : (uint32_t)(L - 1);
   constexpr int SLICES = D / 8;                 // 8-coordinate slices per head
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -188,6 +194,16 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     for (int e = 0; e < 8; ++e) acc[it][e] = 0.0f;
   // score parts: two threads per token when there is a single head
   const int SP = G == 1 ? 2 : 1;
+  // Codebook caches with 2..8 heads per kv head: every code is decoded once per
+  // token and used by all heads (scores: thread = token half; P.V: item =
+  // (8-dim slice, token part) over all heads, TPS = 128 / slices token parts).
+  const bool shared = FMT != 0 && G >= 2 && G <= 8;
+  constexpr int TPS = simt_shared_token_parts<D>();
+  float acc2[FMT != 0 ? 8 : 1][8];
+#pragma unroll
+  for (int h = 0; h < (FMT != 0 ? 8 : 1); ++h)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc2[h][e] = 0.0f;
 
   const int64_t rowbase = ((int64_t)b * a.Hkv + kvh) * a.capacity;
   // Tiles are staged by 4-byte cp.async into two buffers: tile i + 1 is in
@@ -227,7 +243,39 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
     const float* vscale = kscale + kTile * NG;
 
     // scores S[h][t] = sum_g s_k[t][g] sum_{j in g} c[t][j] q'[h][32 g + j]
-    for (int idx = threadIdx.x; idx < kTile * G * SP; idx += kThreads) {
+    if (FMT != 0 && shared) {  // thread = (token, half of each group); all heads
+      const int tt = threadIdx.x >> 1, half = threadIdx.x & 1;
+      float s[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) s[h] = 0.0f;
+      if (tt < nt) {
+        const uint32_t* row = ktile + tt * PW;
+        for (int g = 0; g < NG; ++g) {
+          const uint32_t* gw = row + (FMT != 0 ? FMT : 1) * g;
+          float dg[8];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) dg[h] = 0.0f;
+#pragma unroll 4
+          for (int j = 16 * half; j < 16 * half + 16; ++j) {
+            const float c = cbk[cb_index<(FMT != 0 ? FMT : 2)>(gw, j)];
+            const float* qj = qs + 32 * g + j;
+#pragma unroll
+            for (int h = 0; h < 8; ++h)
+              if (h < G) dg[h] = fmaf(qj[h * D], c, dg[h]);
+          }
+          const float sk = kscale[tt * NG + g];
+#pragma unroll
+          for (int h = 0; h < 8; ++h) s[h] = fmaf(sk, dg[h], s[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < G) {
+          const float v = s[h] + __shfl_xor_sync(0xffffffffu, s[h], 1);
+          if (half == 0) sp[h * kTile + tt] = tt < nt ? v : -INFINITY;
+        }
+    }
+    for (int idx = threadIdx.x; idx < (shared ? 0 : kTile * G * SP); idx += kThreads) {
       const int part = SP == 2 ? (idx & 1) : 0;
       const int tt = SP == 2 ? (idx >> 1) : idx % kTile;
       const int h = SP == 2 ? 0 : idx / kTile;
@@ -303,11 +351,39 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
       }
     }
     __syncthreads();
+    if (FMT != 0 && shared && threadIdx.x < SLICES * TPS) {  // item (sl, tp) for all heads
+      const int sl = threadIdx.x % SLICES, tp = threadIdx.x / SLICES;
+      const int g = sl / 4, bit = (FMT != 0 ? FMT : 1) * 8 * (sl % 4);
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < G) {
+          const float al = alpha[h];
+          if (al != 1.0f) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc2[h][e] *= al;
+          }
+        }
+      for (int tt = tp; tt < nt; tt += TPS) {
+        const uint32_t* gw = vtile + tt * PW + (FMT != 0 ? FMT : 1) * g;
+        const uint32_t v8 = __funnelshift_r(gw[bit >> 5], gw[(bit >> 5) + 1], bit & 31);
+        float c[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) c[m] = cbk[(v8 >> ((FMT != 0 ? FMT : 1) * m)) & LMASK];
+        const float sv = vscale[tt * NG + g];
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+          if (h < G) {
+            const float pw = sp[h * kTile + tt] * sv;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc2[h][m] = fmaf(pw, c[m], acc2[h][m]);
+          }
+      }
+    }
     // P.V on the packed values: item (h, tp, sl) adds tokens tp, tp + TP, ... of the tile
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int item = threadIdx.x + it * kThreads;
-      if (item < items) {
+      if (!shared && item < items) {
         const int sl = item % SLICES, rest = item / SLICES;
         const int tp = rest % TP, h = rest / TP;
         const int g = sl / 4, r0 = (sl % 4) * 2;
@@ -332,7 +408,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
             const uint32_t v8 = __funnelshift_r(gw[bit >> 5], gw[(bit >> 5) + 1], bit & 31);
 #pragma unroll
             for (int m = 0; m < 8; ++m)
-              acc[it][m] = fmaf(pw, cbk[(v8 >> (FMT * m)) & (L - 1)], acc[it][m]);
+              acc[it][m] = fmaf(pw, cbk[(v8 >> (FMT * m)) & LMASK], acc[it][m]);
           }
         }
       }
@@ -350,7 +426,24 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
   // partials: ws[b][hq][chunk][0..D) = acc, [D] = m, [D+1] = l
   float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) + a.plan.header_bytes);
   const int stride = a.plan.part_stride;
-  if (TP == 1) {
+  if (shared) {  // sum the TPS token parts in shared memory (fixed order: deterministic)
+    if (threadIdx.x < SLICES * TPS) {
+      const int sl = threadIdx.x % SLICES, tp = threadIdx.x / SLICES;
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < G)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) red[(tp * G + h) * D + sl * 8 + e] = acc2[h][e];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+      float v = 0.0f;
+      for (int tp = 0; tp < TPS; ++tp) v += red[tp * G * D + i];
+      const int h = i / D, c = i % D;
+      const int64_t hq = (int64_t)kvh * G + h;
+      part[(((int64_t)b * a.Hq + hq) * a.plan.n_chunks + chunk) * stride + c] = v;
+    }
+  } else if (TP == 1) {
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int item = threadIdx.x + it * kThreads;
@@ -396,7 +489,8 @@ size_t simt_smem_bytes(int G) {
   constexpr int NG = D / 32;
   const int TP = simt_token_parts(G, D / 8);
   const size_t tile_words = 4 * (size_t)kTile * simt_pitch_words<D, FMT>();
-  const size_t red_words = TP > 1 ? (size_t)TP * G * D : 0;
+  size_t red_words = TP > 1 ? (size_t)TP * G * D : 0;
+  if (FMT != 0 && G >= 2 && G <= 8) red_words = (size_t)simt_shared_token_parts<D>() * G * D;
   const size_t lut_words = FMT == 2 ? (size_t)G * D * 8 : 0;
   return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 64 + lut_words) +
          sizeof(uint32_t) * (tile_words > red_words ? tile_words : red_words);
