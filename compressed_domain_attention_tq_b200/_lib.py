@@ -25,7 +25,7 @@ SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_t
            "tq_decode_srft_workspace_bytes", "tq_quantize_append_srft", "tq_sdpa_int4_decode_srft",
            "tq_sdpa_int4_decode_append_srft", "tq_lloyd_max_gaussian", "tq_decode_cb_workspace_bytes",
            "tq_quantize_append_cb", "tq_sdpa_cb_decode", "tq_sdpa_cb_decode_append",
-           "tq_status_string")
+           "tq_sdpa_int4_decode_srft_lse", "tq_sdpa_cb_decode_lse", "tq_status_string")
 
 _lib = None
 
@@ -91,6 +91,12 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_cb_decode_append.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, i32, P, P,
                                              P, P, P, i64, P, i32, P, f32, P, P, sz, P]
     lib.tq_sdpa_cb_decode_append.restype = i32
+    lib.tq_sdpa_int4_decode_srft_lse.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i64,
+                                                 P, i32, P, P, P, f32, P, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_srft_lse.restype = i32
+    lib.tq_sdpa_cb_decode_lse.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P,
+                                          i32, P, f32, P, P, P, sz, P]
+    lib.tq_sdpa_cb_decode_lse.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -346,3 +352,34 @@ def sdpa_cb_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scale
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_cb_decode_append")
+
+
+def sdpa_int4_decode_srft_lse(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs,
+                              lambda_k, lambda_v, attn_scale, out, lse, workspace, stream=None):
+    """sdpa_int4_decode_srft that also writes lse[B][Hq][2] per head."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, lambda_k, lambda_v, out,
+               lse, workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_int4_decode_srft_lse(
+        _ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+        _ptr(v_scales), k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs),
+        _ptr(lambda_k), _ptr(lambda_v), float(attn_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_int4_decode_srft_lse")
+
+
+def sdpa_cb_decode_lse(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs, bits,
+                       levels, attn_scale, out, lse, workspace, stream=None):
+    """sdpa_cb_decode that also writes lse[B][Hq][2] per head."""
+    _need_cuda(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels, out, lse, workspace)
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_cb_decode_lse(
+        _ptr(q), _dtype_code(q), B, Hq, Hkv, d, 32, int(bits), _ptr(levels), _ptr(k_packed),
+        _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), k_packed.shape[2], _ptr(ctx_lens),
+        int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_cb_decode_lse")

@@ -82,6 +82,21 @@ class Int4KVCache:
                               ctx_lens, max_ctx, self.signs, attn_scale, out, ws, stream)
         return out
 
+    def decode_lse(self, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float,
+                   out: torch.Tensor, lse: torch.Tensor, stream=None):
+        """decode that also writes each head's softmax state lse[B][Hq][2] (for merging
+        outputs over disjoint parts of a context)."""
+        ws = self.workspace(q.shape[1], max_ctx)
+        if self.srft:
+            _lib.sdpa_int4_decode_srft_lse(q, self.k_packed, self.k_scales, self.v_packed,
+                                           self.v_scales, ctx_lens, max_ctx, self.signs,
+                                           self.lambda_k, self.lambda_v, attn_scale, out, lse, ws,
+                                           stream)
+        else:
+            _lib.sdpa_int4_decode_lse(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
+                                      ctx_lens, max_ctx, self.signs, attn_scale, out, lse, ws, stream)
+        return out
+
     def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                       ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float | None = None,
                       out: torch.Tensor | None = None, stream=None):
@@ -180,4 +195,13 @@ class CodebookKVCache:
         _lib.sdpa_cb_decode_append(q, k_new, v_new, self.k_packed, self.k_scales, self.v_packed,
                                    self.v_scales, ctx_lens, max_ctx, self.signs, self.bits,
                                    self.levels, attn_scale, out, ws, stream)
+        return out
+
+    def decode_lse(self, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float,
+                   out: torch.Tensor, lse: torch.Tensor, stream=None):
+        """decode that also writes each head's softmax state lse[B][Hq][2]."""
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_cb_decode_lse(q, self.k_packed, self.k_scales, self.v_packed, self.v_scales,
+                                ctx_lens, max_ctx, self.signs, self.bits, self.levels, attn_scale,
+                                out, lse, ws, stream)
         return out

@@ -42,21 +42,18 @@ def decode(cache, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
            stream=None) -> torch.Tensor:
     """Attention of q [B][Hq][d] over the union of every rank's shard.
 
-    cache      this rank's Int4KVCache (its shard, rows 0 .. ctx_lens[b]-1).
+    cache      this rank's Int4KVCache or CodebookKVCache (its shard, rows 0 .. ctx_lens[b]-1);
+               every rotation and code format the caches support.
     ctx_lens   this rank's shard lengths (device int32 [B], each >= 1).
     max_ctx    host bound on this rank's ctx_lens.
     Every rank calls this with the same q, attn_scale and group; every rank
     returns the full output (fp32 [B][Hq][d], unrotated basis)."""
-    if cache.srft:
-        raise NotImplementedError("context-parallel decode runs on Hadamard-rotated caches")
     if attn_scale is None:
         attn_scale = 1.0 / math.sqrt(cache.head_dim)
     B, Hq, d = q.shape
     local = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
     lse = torch.empty(B, Hq, 2, dtype=torch.float32, device=q.device)
-    ws = cache.workspace(Hq, max_ctx)
-    _lib.sdpa_int4_decode_lse(q, cache.k_packed, cache.k_scales, cache.v_packed, cache.v_scales,
-                              ctx_lens, max_ctx, cache.signs, attn_scale, local, lse, ws, stream)
+    cache.decode_lse(q, ctx_lens, max_ctx, attn_scale, local, lse, stream)
     outs, lses = gather_parts(local, lse, group)
     if out is None:
         out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)

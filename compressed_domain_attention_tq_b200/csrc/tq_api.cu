@@ -444,6 +444,42 @@ tq_status tq_sdpa_cb_decode(const void* q, tq_dtype q_dtype, int32_t batch, int3
                      "tq_sdpa_cb_decode", nullptr, r);
 }
 
+tq_status tq_sdpa_int4_decode_srft_lse(const void* q, tq_dtype q_dtype, int32_t batch,
+                                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                       int32_t group, const uint8_t* k_packed,
+                                       const float* k_scales, const uint8_t* v_packed,
+                                       const float* v_scales, int64_t capacity,
+                                       const int32_t* ctx_lens, int32_t max_ctx,
+                                       const int8_t* signs, const float* lambda_k,
+                                       const float* lambda_v, float attn_scale, float* out,
+                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       void* cuda_stream) {
+  if (!lse) return TQ_ERR_INVALID_ARG;
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_int4_decode_srft_lse", lse, Rotation{true, lambda_k, lambda_v});
+}
+
+tq_status tq_sdpa_cb_decode_lse(const void* q, tq_dtype q_dtype, int32_t batch,
+                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t group, int32_t bits, const float* levels,
+                                const uint8_t* k_packed, const float* k_scales,
+                                const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+                                const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+                                float attn_scale, float* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* cuda_stream) {
+  if (!lse) return TQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  return decode_impl(q, q_dtype, nullptr, nullptr, TQ_F32, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_cb_decode_lse", lse, r);
+}
+
 tq_status tq_sdpa_cb_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
                                    const void* v_new, tq_dtype kv_dtype, int32_t batch,
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,

@@ -327,6 +327,16 @@ TQ_API tq_status tq_sdpa_int4_decode_srft(
     int32_t max_ctx, const int8_t* signs, const float* lambda_k, const float* lambda_v,
     float attn_scale, float* out, void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/* tq_sdpa_int4_decode_srft that also returns each head's softmax state (as
+ * tq_sdpa_int4_decode_lse), for tq_merge_lse across context parts. */
+TQ_API tq_status tq_sdpa_int4_decode_srft_lse(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, const uint8_t* k_packed, const float* k_scales,
+    const uint8_t* v_packed, const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, const float* lambda_k, const float* lambda_v,
+    float attn_scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
+    void* cuda_stream);
+
 /* tq_sdpa_int4_decode_append over an SRFT cache: the new tokens are quantized
  * by a tq_quantize_append_srft launch, then the query attends. */
 TQ_API tq_status tq_sdpa_int4_decode_append_srft(
@@ -382,6 +392,15 @@ TQ_API tq_status tq_sdpa_cb_decode(
     const float* k_scales, const uint8_t* v_packed, const float* v_scales, int64_t capacity,
     const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, float attn_scale, float* out,
     void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* tq_sdpa_cb_decode that also returns each head's softmax state (as
+ * tq_sdpa_int4_decode_lse), for tq_merge_lse across context parts. */
+TQ_API tq_status tq_sdpa_cb_decode_lse(
+    const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t group, int32_t bits, const float* levels, const uint8_t* k_packed,
+    const float* k_scales, const uint8_t* v_packed, const float* v_scales, int64_t capacity,
+    const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs, float attn_scale, float* out,
+    float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /* tq_sdpa_int4_decode_append over a codebook cache (append launch, then decode). */
 TQ_API tq_status tq_sdpa_cb_decode_append(

@@ -100,3 +100,50 @@ def test_lse_of_one_part_reproduces_plain_decode():
     assert torch.equal(o1, o2)
     assert torch.allclose(m, o2, rtol=1e-6, atol=1e-7)
     assert bool((l[..., 1] >= 1.0).all())  # the sum includes the maximum's own weight 1
+
+
+def _srft_and_cb_caches(B, Hkv, d, T, g):
+    """Host inputs plus an SRFT and a 3-bit codebook cache of them (oracle-quantized)."""
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16)
+    return k, v
+
+
+@pytest.mark.parametrize("kind", ["srft", "cb3"])
+def test_context_parallel_srft_and_codebook_caches(kind):
+    """context_parallel's per-shard decode (decode_lse of each cache kind) merged with
+    tq_merge_lse equals the whole-cache decode of the same kind."""
+    require_cuda()
+    from compressed_domain_attention_tq_b200 import CodebookKVCache, Int4KVCache
+    B, Hkv, G, d = 1, 2, 4, (96 if kind == "srft" else 128)
+    T = 2500
+    g = torch.Generator().manual_seed(77 if kind == "srft" else 78)
+    k, v = _srft_and_cb_caches(B, Hkv, d, T, g)
+    q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+    lam = torch.exp2(torch.empty(2, d).uniform_(-0.25, 0.25, generator=g))
+
+    def make(cap):
+        if kind == "srft":
+            return Int4KVCache(B, Hkv, d, cap, signs=signs, rotation="srft", lambda_k=lam[0],
+                               lambda_v=lam[1])
+        return CodebookKVCache(B, Hkv, d, cap, 3, signs=signs)
+
+    zero = torch.zeros(B, dtype=torch.int32, device="cuda")
+    whole = make(T)
+    whole.append(k.cuda(), v.cuda(), zero)
+    full = whole.decode(q, torch.tensor([T], dtype=torch.int32, device="cuda"), T, 0.1)
+    outs, lses = [], []
+    for s0, s1 in ((0, 1000), (1000, 1001), (1001, T)):
+        part = make(s1 - s0)
+        part.append(k[:, :, s0:s1].contiguous().cuda(), v[:, :, s0:s1].contiguous().cuda(), zero)
+        o = torch.empty(B, Hkv * G, d, device="cuda")
+        l = torch.empty(B, Hkv * G, 2, device="cuda")
+        part.decode_lse(q, torch.tensor([s1 - s0], dtype=torch.int32, device="cuda"), s1 - s0, 0.1, o, l)
+        outs.append(o)
+        lses.append(l)
+    merged = torch.empty_like(full)
+    _lib.merge_lse(torch.stack(outs).contiguous(), torch.stack(lses).contiguous(), merged)
+    torch.cuda.synchronize()
+    a, b = merged.cpu().numpy(), full.cpu().numpy()
+    assert np.linalg.norm(a - b) <= 2e-6 * np.linalg.norm(b), np.linalg.norm(a - b) / np.linalg.norm(b)
