@@ -189,22 +189,55 @@ def merge_lse(outs, lses, out, stream=None):
         raise TQError(rc, "tq_merge_lse")
 
 
-def sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
-                            max_ctx, signs, attn_scale, out, workspace, stream=None):
-    """One decode step: quantize k_new, v_new [B][Hkv][1][d] into row ctx_lens[b]-1
-    of the cache, then out[B][Hq][d] = attention of q over rows 0..ctx_lens[b]-1."""
+def _decode_append_args(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx,
+                        signs, attn_scale, out, workspace, stream):
     _need_cuda(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out, workspace)
     if k_new.dtype != v_new.dtype:
         raise TypeError("k_new and v_new must share dtype")
     B, Hq, d = q.shape
     Hkv = k_packed.shape[1]
-    rc = load().tq_sdpa_int4_decode_append(
-        _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq, Hkv, d, 32,
-        _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), k_packed.shape[2],
-        _ptr(ctx_lens), int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream))
+    i32, f32, sz = ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    return (_ptr(q), i32(_dtype_code(q)), _ptr(k_new), _ptr(v_new), i32(_dtype_code(k_new)), i32(B),
+            i32(Hq), i32(Hkv), i32(d), i32(32), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+            _ptr(v_scales), ctypes.c_int64(k_packed.shape[2]), _ptr(ctx_lens), i32(int(max_ctx)),
+            _ptr(signs), f32(float(attn_scale)), _ptr(out), _ptr(workspace),
+            sz(workspace.numel() * workspace.element_size()), _stream(stream))
+
+
+def sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                            max_ctx, signs, attn_scale, out, workspace, stream=None):
+    """One decode step: quantize k_new, v_new [B][Hkv][1][d] into row ctx_lens[b]-1
+    of the cache, then out[B][Hq][d] = attention of q over rows 0..ctx_lens[b]-1."""
+    rc = load().tq_sdpa_int4_decode_append(*_decode_append_args(
+        q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx, signs,
+        attn_scale, out, workspace, stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_int4_decode_append")
+
+
+class BoundCall:
+    """A libtq call whose arguments were checked and marshalled once: each call
+    enqueues the same work again on the same buffers and stream (a decode loop
+    that refills its input buffers and reuses its output).  Saves the per-call
+    Python work of building the C arguments."""
+
+    def __init__(self, fn, args, where, keep):
+        self._fn, self._args, self._where = fn, args, where
+        self._keep = keep  # the tensors behind the pointers stay alive with the call
+
+    def __call__(self):
+        rc = self._fn(*self._args)
+        if rc != TQ_OK:
+            raise TQError(rc, self._where)
+
+
+def bind_sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                                 max_ctx, signs, attn_scale, out, workspace, stream=None) -> BoundCall:
+    """sdpa_int4_decode_append prepared for repeated calls on the same buffers."""
+    args = _decode_append_args(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                               max_ctx, signs, attn_scale, out, workspace, stream)
+    keep = (q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, out, workspace)
+    return BoundCall(load().tq_sdpa_int4_decode_append, args, "tq_sdpa_int4_decode_append", keep)
 
 
 def sdpa_int4_decode_static_scratch(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_ctx,

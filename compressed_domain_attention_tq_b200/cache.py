@@ -118,6 +118,24 @@ class Int4KVCache:
                                      ws, stream)
         return out
 
+    def bind_decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                           ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float | None = None,
+                           out: torch.Tensor | None = None, stream=None):
+        """decode_append prepared once for a serving loop that refills q, k_new, v_new and
+        ctx_lens in place: returns (step, out), where step() enqueues one decode step on
+        these buffers (the Hadamard-rotated cache; one C call per step)."""
+        if self.srft:
+            raise NotImplementedError("bind_decode_append runs on Hadamard-rotated caches")
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        step = _lib.bind_sdpa_int4_decode_append(q, k_new, v_new, self.k_packed, self.k_scales,
+                                                 self.v_packed, self.v_scales, ctx_lens, max_ctx,
+                                                 self.signs, attn_scale, out, ws, stream)
+        return step, out
+
     def dequantize(self, rows: int, dtype=torch.bfloat16, stream=None):
         """Dequantized K and V of rows 0 .. rows-1 of every sequence, [B][Hkv][rows][d]
         in the rotated basis (scale * code; not used by decode)."""

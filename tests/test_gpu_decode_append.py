@@ -79,3 +79,36 @@ def test_fused_step_vs_oracle_fp32_inputs():
     cache = [t.cpu().numpy() for t in c]
     want = oracle.sdpa_int4_decode(to_oracle(q), cache, [2049], None, scale, Hkv, threads=THREADS)
     check_attention(out.cpu().numpy(), want, cache, [2049], G, "fused step")
+
+
+def test_bound_decode_append_matches_plain_call_on_refilled_buffers():
+    """Int4KVCache.bind_decode_append: the prepared step, called after the inputs are
+    refilled in place, gives bit-identical caches and outputs to the plain call."""
+    require_cuda()
+    import torch
+    from compressed_domain_attention_tq_b200 import Int4KVCache
+    B, Hkv, G, d, T = 1, 2, 8, 128, 1200
+    g = torch.Generator().manual_seed(91)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+    caches = [Int4KVCache(B, Hkv, d, T + 4, signs=signs) for _ in range(2)]
+    for c in caches:
+        c.append(k, v, torch.zeros(B, dtype=torch.int32, device="cuda"))
+    q = torch.empty(B, Hkv * G, d, dtype=torch.bfloat16, device="cuda")
+    kn = torch.empty(B, Hkv, 1, d, dtype=torch.bfloat16, device="cuda")
+    vn = torch.empty_like(kn)
+    ctx = torch.empty(B, dtype=torch.int32, device="cuda")
+    step, out_b = caches[0].bind_decode_append(q, kn, vn, ctx, T + 4, 0.09)
+    for i in range(3):
+        q.copy_(torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16))
+        kn.copy_(torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16))
+        vn.copy_(torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16))
+        ctx.fill_(T + 1 + i)
+        step()
+        out_p = caches[1].decode_append(q, kn, vn, ctx, T + 4, 0.09)
+        torch.cuda.synchronize()
+        assert torch.equal(out_b, out_p)
+    for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
+                    (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
+        assert torch.equal(a, b)
