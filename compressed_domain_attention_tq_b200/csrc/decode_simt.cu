@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel
   float* lstate = mstate + 16;                                 // [G] running sum
   float* alpha = lstate + 16;                                  // [G] rescale of this tile
   float* cbk = alpha + 16;                                     // [16] codebook levels
-  float* lut = cbk + 16;                                       // [G][D/2][16] (FMT 2)
+  float* qT = cbk + 16;                                        // [D][8] query, heads fastest (FMT != 0)
+  float* spT = qT + (FMT != 0 ? D * 8 : 0);                    // [kTile][8] weights, heads fastest
+  float* lut = spT + (FMT != 0 ? kTile * 8 : 0);               // [G][D/2][16] (FMT 2)
   // [2 buffers][K, V][kTile][PW] staged packed rows; after the last tile the same
   // space holds the token parts' sums [TP][G][D] (TP > 1)
   uint32_t* tiles = reinterpret_cast<uint32_t*>(lut + (FMT == 2 ? G * D * 8 : 0));
@@ -172,6 +174,14 @@ __global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel
   // int4: 16^-(i mod 4), as the codes of the score loop come scaled by 16^(i mod 4)
   for (int i = threadIdx.x; i < G * D; i += kThreads)
     qs[i] *= FMT == 0 ? qmul * __int_as_float((127 - 4 * (i & 3)) << 23) : qmul;
+  if constexpr (FMT != 0) {  // transposed copies for the shared-code path (absent heads: 0)
+    __syncthreads();
+    for (int i = threadIdx.x; i < D * 8; i += kThreads) {
+      const int j = i >> 3, h = i & 7;
+      qT[i] = h < G ? qs[h * D + j] : 0.0f;
+    }
+    for (int i = threadIdx.x; i < kTile * 8; i += kThreads) spT[i] = 0.0f;
+  }
   if constexpr (FMT == 2) {  // pair tables: lut[h][p][e] = C[e & 3] q'[2p] + C[e >> 2] q'[2p + 1]
     __syncthreads();
     for (int i = threadIdx.x; i < G * D * 8; i += kThreads) {
@@ -255,13 +265,24 @@ __global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel
           float dg[8];
 #pragma unroll
           for (int h = 0; h < 8; ++h) dg[h] = 0.0f;
-#pragma unroll 4
-          for (int j = 16 * half; j < 16 * half + 16; ++j) {
-            const float c = cbk[cb_index<(FMT != 0 ? FMT : 2)>(gw, j)];
-            const float* qj = qs + 32 * g + j;
+          // this half's 16 indices (FMT * 16 bits from bit FMT * 16 * half) in one register pair
+          constexpr int FB = FMT != 0 ? FMT : 2;
+          const int b0 = FB * 16 * half;
+          const uint64_t bits = ((uint64_t)gw[(b0 >> 5) + 1] << 32 | gw[b0 >> 5]) >> (b0 & 31);
 #pragma unroll
-            for (int h = 0; h < 8; ++h)
-              if (h < G) dg[h] = fmaf(qj[h * D], c, dg[h]);
+          for (int jl = 0; jl < 16; ++jl) {
+            const int j = 16 * half + jl;
+            const float c = cbk[(uint32_t)(bits >> (FB * jl)) & ((1u << FB) - 1u)];
+            const float4 qa = *reinterpret_cast<const float4*>(qT + (32 * g + j) * 8);
+            const float4 qb = *reinterpret_cast<const float4*>(qT + (32 * g + j) * 8 + 4);
+            dg[0] = fmaf(qa.x, c, dg[0]);
+            dg[1] = fmaf(qa.y, c, dg[1]);
+            dg[2] = fmaf(qa.z, c, dg[2]);
+            dg[3] = fmaf(qa.w, c, dg[3]);
+            dg[4] = fmaf(qb.x, c, dg[4]);
+            dg[5] = fmaf(qb.y, c, dg[5]);
+            dg[6] = fmaf(qb.z, c, dg[6]);
+            dg[7] = fmaf(qb.w, c, dg[7]);
           }
           const float sk = kscale[tt * NG + g];
 #pragma unroll
@@ -340,6 +361,10 @@ __global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel
         const float p0 = exp2f(s0 - m_new), p1 = exp2f(s1 - m_new);
         sp[h * kTile + lane] = p0;
         sp[h * kTile + lane + 32] = p1;
+        if (FMT != 0 && shared) {
+          spT[lane * 8 + h] = p0;
+          spT[(lane + 32) * 8 + h] = p1;
+        }
         float sum = p0 + p1;
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
@@ -370,12 +395,15 @@ __global__ void __launch_bounds__(kThreads, FMT == 0 ? 5 : 3) decode_simt_kernel
 #pragma unroll
         for (int m = 0; m < 8; ++m) c[m] = cbk[(v8 >> ((FMT != 0 ? FMT : 1) * m)) & LMASK];
         const float sv = vscale[tt * NG + g];
+        const float4 pa = *reinterpret_cast<const float4*>(spT + tt * 8);
+        const float4 pb = *reinterpret_cast<const float4*>(spT + tt * 8 + 4);
+        const float pw[8] = {pa.x * sv, pa.y * sv, pa.z * sv, pa.w * sv,
+                             pb.x * sv, pb.y * sv, pb.z * sv, pb.w * sv};
 #pragma unroll
         for (int h = 0; h < 8; ++h)
           if (h < G) {
-            const float pw = sp[h * kTile + tt] * sv;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) acc2[h][m] = fmaf(pw, c[m], acc2[h][m]);
+            for (int m = 0; m < 8; ++m) acc2[h][m] = fmaf(pw[h], c[m], acc2[h][m]);
           }
       }
     }
@@ -492,7 +520,9 @@ size_t simt_smem_bytes(int G) {
   size_t red_words = TP > 1 ? (size_t)TP * G * D : 0;
   if (FMT != 0 && G >= 2 && G <= 8) red_words = (size_t)simt_shared_token_parts<D>() * G * D;
   const size_t lut_words = FMT == 2 ? (size_t)G * D * 8 : 0;
-  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 64 + lut_words) +
+  const size_t tr_words = FMT != 0 ? (size_t)D * 8 + kTile * 8 : 0;  // qT, spT
+  return sizeof(float) * ((size_t)G * D + (size_t)G * kTile + 4 * kTile * NG + 64 + lut_words +
+                          tr_words) +
          sizeof(uint32_t) * (tile_words > red_words ? tile_words : red_words);
 }
 
