@@ -319,6 +319,9 @@ __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* s
     t = t0;
   }
   const int n = min(C::ST, t1 - t);
+  if (a.q_rot_overlap == 2 && t + n == t1 &&
+      t1 == clamp_ctx_mma(a.ctx_lens[b], a.max_ctx))  // holds the row the preceding grid appends
+    asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t cb = n * C::RB, sb = n * C::NG * 4;
   unsigned char* stg = smem + slot * C::STAGE;
   const int64_t row = ((int64_t)b * a.Hkv + kvh) * a.capacity + t;
@@ -1008,7 +1011,7 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   const int grid = n_items < sms ? n_items : sms;
-  if (a.q_rot != nullptr) {  // overlap the query-rotation grid (see prep_query)
+  if (a.q_rot != nullptr && a.q_rot_overlap) {  // overlap the query-rotation grid (see prep_query)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(C::THREADS);

@@ -17,6 +17,8 @@
 //   srft_query_kernel     one warp per pair of query heads -> q_r (fp32) in the
 //                         decode workspace; the decode kernels read it instead
 //                         of rotating q themselves.
+//   srft_prep_kernel      one decode step's new-token quantization and query
+//                         rotation in one launch (the fused step's first kernel).
 //   srft_merge_kernel     one CTA per pair of query heads: the split-K log-sum-
 //                         exp merge of each head, 1 / lambda_V, then one warp
 //                         maps both heads back.
@@ -47,6 +49,92 @@ __device__ __forceinline__ float int4_code(float x, float s, float r, bool big) 
   return fminf(fmaxf(c, -7.0f), 7.0f);
 }
 
+// Per-lane constants of the SRFT quantizer: signs at j = lane + 32 j2 and
+// lambda / (2 sqrt d) at k = k2 + M brev5(lane).
+template <int M>
+struct SrftLaneConsts {
+  float sg[M], mk[M], mv[M];
+  __device__ __forceinline__ void load(const QuantizeArgs& a, int lane) {
+    constexpr int D = 32 * M;
+    const float norm = 0.5f / sqrtf((float)D);
+#pragma unroll
+    for (int j2 = 0; j2 < M; ++j2) sg[j2] = a.signs ? (float)a.signs[lane + 32 * j2] : 1.0f;
+#pragma unroll
+    for (int k2 = 0; k2 < M; ++k2) {
+      const int k = k2 + M * brev5(lane);
+      mk[k2] = a.lambda_k ? norm * a.lambda_k[k] : norm;
+      mv[k2] = a.lambda_v ? norm * a.lambda_v[k] : norm;
+    }
+  }
+};
+
+// One warp quantizes the K and V rows of vector pair p ((sequence, kv head)
+// row-major, then token) into the cache; yk, yv: this warp's 2 x d floats of
+// shared memory for the transpose.
+template <int M>
+__device__ __forceinline__ void srft_quantize_pair(const QuantizeArgs& a, int p,
+                                                   const HartleyTwiddles<M>& tw,
+                                                   const SrftLaneConsts<M>& lc, float* yk, float* yv,
+                                                   int lane) {
+  constexpr int D = 32 * M;
+  const int bh = p / a.n_new, n = p % a.n_new;
+  const int b = bh / a.Hkv;
+  int64_t pos = (int64_t)a.pos[b] + n;
+  if (a.pos_is_ctx) pos = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
+  if (pos < 0 || pos >= a.capacity) return;  // the whole warp
+  const int64_t row = (int64_t)bh * a.capacity + pos;
+  float re[M], im[M];
+#pragma unroll
+  for (int j2 = 0; j2 < M; ++j2) {
+    const int64_t idx = (int64_t)p * D + lane + 32 * j2;
+    float xk, xv;
+    if (a.bf16) {
+      xk = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.k)[idx] << 16);
+      xv = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.v)[idx] << 16);
+    } else {
+      xk = static_cast<const float*>(a.k)[idx];
+      xv = static_cast<const float*>(a.v)[idx];
+    }
+    re[j2] = lc.sg[j2] * xk;
+    im[j2] = lc.sg[j2] * xv;
+  }
+  float hx[M], hy[M];
+  hartley_pair_warp<M>(re, im, tw, hx, hy);
+#pragma unroll
+  for (int k2 = 0; k2 < M; ++k2) {
+    const int k = k2 + M * brev5(lane);
+    yk[k] = hx[k2] * lc.mk[k2];
+    yv[k] = hy[k2] * lc.mv[k2];
+  }
+  __syncwarp();
+  // lane holds in-group coordinate j = lane of every group g (coordinate 32 g + lane)
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    const float* y = kv ? yv : yk;
+    uint8_t* prow = (kv ? a.v_packed : a.k_packed) + row * (D / 2);
+    float* srow = (kv ? a.v_scales : a.k_scales) + row * M;
+#pragma unroll
+    for (int g = 0; g < M; ++g) {
+      const float x = y[32 * g + lane];
+      float amax = fabsf(x);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = __fdiv_rn(amax, 7.0f);
+      const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+      const float c = s > 0.0f ? int4_code(x, s, r, !(r <= 3.0e38f)) : 0.0f;
+      // byte (j / 4) * 2M + 2 g + (j % 4) / 2, nibble j % 2: four lanes make one half-word
+      // c + 1.5 * 2^23 has the bits 0x4B400000 + c: its low nibble is c's two's complement
+      uint32_t nib = (__float_as_uint(c + kRneMagic) & 0xFu) << (4 * (lane & 3));
+      nib |= __shfl_xor_sync(0xffffffffu, nib, 1);
+      nib |= __shfl_xor_sync(0xffffffffu, nib, 2);
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint16_t*>(prow + (lane >> 2) * 2 * M + 2 * g) = (uint16_t)nib;
+      if (lane == g) srow[g] = s;
+    }
+  }
+  __syncwarp();
+}
+
 template <int M>
 __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArgs a) {
   constexpr int D = 32 * M;
@@ -54,93 +142,22 @@ __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArg
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   HartleyTwiddles<M> tw;
   hartley_twiddles<M>(tw, lane);
-  const float norm = 0.5f / sqrtf((float)D);
-  float sg[M], mk[M], mv[M];
-#pragma unroll
-  for (int j2 = 0; j2 < M; ++j2) sg[j2] = a.signs ? (float)a.signs[lane + 32 * j2] : 1.0f;
-#pragma unroll
-  for (int k2 = 0; k2 < M; ++k2) {
-    const int k = k2 + M * brev5(lane);
-    mk[k2] = a.lambda_k ? norm * a.lambda_k[k] : norm;
-    mv[k2] = a.lambda_v ? norm * a.lambda_v[k] : norm;
-  }
-  float* yk = ybuf[warp][0];
-  float* yv = ybuf[warp][1];
+  SrftLaneConsts<M> lc;
+  lc.load(a, lane);
   const int pairs = a.B * a.Hkv * a.n_new;  // < 2^31 (checked on the host)
-  for (int p = blockIdx.x * kQWarps + warp; p < pairs; p += gridDim.x * kQWarps) {
-    const int bh = p / a.n_new, n = p % a.n_new;
-    const int b = bh / a.Hkv;
-    int64_t pos = (int64_t)a.pos[b] + n;
-    if (a.pos_is_ctx) pos = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
-    if (pos < 0 || pos >= a.capacity) continue;  // the whole warp
-    const int64_t row = (int64_t)bh * a.capacity + pos;
-    float re[M], im[M];
-#pragma unroll
-    for (int j2 = 0; j2 < M; ++j2) {
-      const int64_t idx = (int64_t)p * D + lane + 32 * j2;
-      float xk, xv;
-      if (a.bf16) {
-        xk = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.k)[idx] << 16);
-        xv = __uint_as_float((uint32_t)static_cast<const uint16_t*>(a.v)[idx] << 16);
-      } else {
-        xk = static_cast<const float*>(a.k)[idx];
-        xv = static_cast<const float*>(a.v)[idx];
-      }
-      re[j2] = sg[j2] * xk;
-      im[j2] = sg[j2] * xv;
-    }
-    float hx[M], hy[M];
-    hartley_pair_warp<M>(re, im, tw, hx, hy);
-#pragma unroll
-    for (int k2 = 0; k2 < M; ++k2) {
-      const int k = k2 + M * brev5(lane);
-      yk[k] = hx[k2] * mk[k2];
-      yv[k] = hy[k2] * mv[k2];
-    }
-    __syncwarp();
-    // lane holds in-group coordinate j = lane of every group g (coordinate 32 g + lane)
-#pragma unroll
-    for (int kv = 0; kv < 2; ++kv) {
-      const float* y = kv ? yv : yk;
-      uint8_t* prow = (kv ? a.v_packed : a.k_packed) + row * (D / 2);
-      float* srow = (kv ? a.v_scales : a.k_scales) + row * M;
-#pragma unroll
-      for (int g = 0; g < M; ++g) {
-        const float x = y[32 * g + lane];
-        float amax = fabsf(x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float s = __fdiv_rn(amax, 7.0f);
-        const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
-        const float c = s > 0.0f ? int4_code(x, s, r, !(r <= 3.0e38f)) : 0.0f;
-        // byte (j / 4) * 2M + 2 g + (j % 4) / 2, nibble j % 2: four lanes make one half-word
-        // c + 1.5 * 2^23 has the bits 0x4B400000 + c: its low nibble is c's two's complement
-        uint32_t nib = (__float_as_uint(c + kRneMagic) & 0xFu) << (4 * (lane & 3));
-        nib |= __shfl_xor_sync(0xffffffffu, nib, 1);
-        nib |= __shfl_xor_sync(0xffffffffu, nib, 2);
-        if ((lane & 3) == 0)
-          *reinterpret_cast<uint16_t*>(prow + (lane >> 2) * 2 * M + 2 * g) = (uint16_t)nib;
-        if (lane == g) srow[g] = s;
-      }
-    }
-    __syncwarp();
-  }
+  for (int p = blockIdx.x * kQWarps + warp; p < pairs; p += gridDim.x * kQWarps)
+    srft_quantize_pair<M>(a, p, tw, lc, ybuf[warp][0], ybuf[warp][1], lane);
 }
 
+// One warp rotates query heads h0 = 2 (p mod ceil(Hq/2)) and h0 + 1 of sequence
+// p / ceil(Hq/2) into the workspace: q_rot = F (signs (.) q) / lambda_K.
 template <int M>
-__global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
+__device__ __forceinline__ void srft_query_pair(const DecodeArgs& a, int64_t p,
+                                                const HartleyTwiddles<M>& tw, int lane) {
   constexpr int D = 32 * M;
-  // the decode kernel may start streaming the cache now; it waits for this
-  // grid (griddepcontrol.wait) before it reads the rotated queries
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pairs_per_b = (a.Hq + 1) / 2;
-  const int64_t p = (int64_t)blockIdx.x * 4 + warp;
-  if (p >= (int64_t)a.B * pairs_per_b) return;  // the whole warp
   const int b = (int)(p / pairs_per_b), h0 = 2 * (int)(p % pairs_per_b);
   const bool two = h0 + 1 < a.Hq;
-  HartleyTwiddles<M> tw;
-  hartley_twiddles<M>(tw, lane);
   float re[M], im[M];
   const int64_t base0 = ((int64_t)b * a.Hq + h0) * D;
 #pragma unroll
@@ -170,6 +187,45 @@ __global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
     const float mul = a.lambda_k ? __fdiv_rn(norm, a.lambda_k[k]) : norm;
     q_rot[base0 + k] = hx[k2] * mul;
     if (two) q_rot[base0 + D + k] = hy[k2] * mul;
+  }
+}
+
+template <int M>
+__global__ void __launch_bounds__(128) srft_query_kernel(DecodeArgs a) {
+  // the decode kernel may start streaming the cache now; it waits for this
+  // grid (griddepcontrol.wait) before it reads the rotated queries
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t p = (int64_t)blockIdx.x * 4 + warp;
+  if (p >= (int64_t)a.B * ((a.Hq + 1) / 2)) return;  // the whole warp
+  HartleyTwiddles<M> tw;
+  hartley_twiddles<M>(tw, lane);
+  srft_query_pair<M>(a, p, tw, lane);
+}
+
+// One decode step's preparation in one launch: warps [0, npk) quantize the new
+// token's K/V pairs (one per sequence and kv head) into the cache, the next
+// warps rotate the query pairs.
+template <int M>
+__global__ void __launch_bounds__(128) srft_prep_kernel(QuantizeArgs qa, DecodeArgs a) {
+  constexpr int D = 32 * M;
+  // the decode may start streaming now: it waits for this grid before it reads the
+  // rotated queries and before it copies a sequence's last (appended) row
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float ybuf[4][2][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 4 + warp;
+  const int npk = qa.B * qa.Hkv * qa.n_new;
+  const int64_t npq = (int64_t)a.B * ((a.Hq + 1) / 2);
+  if (w >= npk + npq) return;  // the whole warp
+  HartleyTwiddles<M> tw;
+  hartley_twiddles<M>(tw, lane);
+  if (w < npk) {
+    SrftLaneConsts<M> lc;
+    lc.load(qa, lane);
+    srft_quantize_pair<M>(qa, (int)w, tw, lc, ybuf[warp][0], ybuf[warp][1], lane);
+  } else {
+    srft_query_pair<M>(a, w - npk, tw, lane);
   }
 }
 
@@ -263,6 +319,13 @@ cudaError_t launch_srft_query_m(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 template <int M>
+cudaError_t launch_srft_prep_m(const QuantizeArgs& qa, const DecodeArgs& a, cudaStream_t stream) {
+  const int64_t warps = (int64_t)qa.B * qa.Hkv * qa.n_new + (int64_t)a.B * ((a.Hq + 1) / 2);
+  srft_prep_kernel<M><<<(unsigned)((warps + 3) / 4), 128, 0, stream>>>(qa, a);
+  return cudaGetLastError();
+}
+
+template <int M>
 cudaError_t launch_srft_merge_m(const DecodeArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * ((a.Hq + 1) / 2));
@@ -307,6 +370,20 @@ cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream) {
 cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream) {
   const int d = a.d;
   TQ_SRFT_DISPATCH(launch_srft_merge_m, a)
+}
+
+cudaError_t launch_srft_prep(const QuantizeArgs& qa, const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.d / 32) {
+    case 1: return launch_srft_prep_m<1>(qa, a, stream);
+    case 2: return launch_srft_prep_m<2>(qa, a, stream);
+    case 3: return launch_srft_prep_m<3>(qa, a, stream);
+    case 4: return launch_srft_prep_m<4>(qa, a, stream);
+    case 5: return launch_srft_prep_m<5>(qa, a, stream);
+    case 6: return launch_srft_prep_m<6>(qa, a, stream);
+    case 7: return launch_srft_prep_m<7>(qa, a, stream);
+    case 8: return launch_srft_prep_m<8>(qa, a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tq

@@ -322,6 +322,29 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   if (append && mma && !rot.srft) {  // the decode kernel quantizes the new tokens itself
     a.k_new = k_new;
     a.v_new = v_new;
+  } else if (append && rot.srft) {  // new tokens and query rotation in one launch
+    QuantizeArgs qa;
+    qa.k = k_new;
+    qa.v = v_new;
+    qa.bf16 = kv_dtype == TQ_BF16;
+    qa.B = batch;
+    qa.Hkv = num_kv_heads;
+    qa.n_new = 1;
+    qa.d = head_dim;
+    qa.pos = ctx_lens;
+    qa.pos_is_ctx = 1;
+    qa.max_ctx = max_ctx;
+    qa.signs = signs;
+    qa.k_packed = const_cast<uint8_t*>(k_packed);
+    qa.k_scales = const_cast<float*>(k_scales);
+    qa.v_packed = const_cast<uint8_t*>(v_packed);
+    qa.v_scales = const_cast<float*>(v_scales);
+    qa.capacity = capacity;
+    qa.lambda_k = rot.lambda_k;
+    qa.lambda_v = rot.lambda_v;
+    const cudaError_t e = launch_srft_prep(qa, a, s);
+    if (e != cudaSuccess) return cuda_status(e, where);
+    a.q_rot_overlap = 2;
   } else if (append) {  // the CUDA-core decode: one small-append launch first
     QuantizeArgs qa;
     qa.k = k_new;
@@ -349,7 +372,8 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
                                         : launch_quantize(qa, s);
     if (e != cudaSuccess) return cuda_status(e, where);
   }
-  if (rot.srft) {  // rotated queries into the workspace, read by the decode kernel
+  if (rot.srft && !append) {  // rotated queries into the workspace, read by the decode kernel
+    a.q_rot_overlap = 1;         // the rotation writes no cache rows: the decode may overlap it
     const cudaError_t e = launch_srft_query(a, s);
     if (e != cudaSuccess) return cuda_status(e, where);
   }

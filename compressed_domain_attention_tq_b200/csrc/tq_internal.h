@@ -80,6 +80,10 @@ struct DecodeArgs {
   float* lse;  // NULL, or [B][Hq][2]: each head's (max in log2 units, sum) for merging contexts
   const float* q_rot = nullptr;     // SRFT variant: [B][Hq][d] rotated queries F(sigma q)/lambda_K;
                                     // the decode kernels read these instead of rotating q
+  int q_rot_overlap = 0;            // the tensor-core decode may start while the preceding grid
+                                    // runs (programmatic dependent launch): 1 = that grid only
+                                    // rotates the queries; 2 = it also appends each sequence's
+                                    // last row, so the copy of that row waits for it
   const float* lambda_k = nullptr;  // SRFT variant: per-coordinate scales (NULL = ones)
   const float* lambda_v = nullptr;
   int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
@@ -112,6 +116,7 @@ bool srft_head_dim_supported(int d);
 cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_srft_prep(const QuantizeArgs& qa, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_quantize_cb(const QuantizeArgs& a, cudaStream_t stream);
 void lloyd_max_gaussian(int bits, double* levels);
 cudaError_t launch_merge_lse(const float* outs, const float* lses, int n_parts, int64_t n_heads,

@@ -337,8 +337,9 @@ TQ_API tq_status tq_sdpa_int4_decode_srft_lse(
     float attn_scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
     void* cuda_stream);
 
-/* tq_sdpa_int4_decode_append over an SRFT cache: the new tokens are quantized
- * by a tq_quantize_append_srft launch, then the query attends. */
+/* tq_sdpa_int4_decode_append over an SRFT cache: one launch quantizes the new
+ * tokens (as tq_quantize_append_srft, bit-identically) and rotates the
+ * queries, then the query attends. */
 TQ_API tq_status tq_sdpa_int4_decode_append_srft(
     const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
     int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
