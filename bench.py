@@ -360,9 +360,10 @@ def run_tq(args):
         step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): quantize-append "
                      "of the new token, split-K decode, merge (3 launches)")
     elif srft:
-        launches_per_step = 4
-        step_desc = ("tq_sdpa_int4_decode_append_srft: SRFT quantize-append of the new token, query "
-                     "rotation, split-K decode, merge with the inverse transform (4 launches)")
+        launches_per_step = 3
+        step_desc = ("tq_sdpa_int4_decode_append_srft: one launch quantizes the new token (SRFT) and "
+                     "rotates the queries, then split-K decode and merge with the inverse transform "
+                     "(3 launches)")
     elif mma:
         launches_per_step = 2
         step_desc = ("tq_sdpa_int4_decode_append: the decode kernel quantizes the new token of each "
