@@ -290,33 +290,33 @@ def run_tq(args):
         step_s, dec_s, q_s, two_s = tt.tolist()
     del g_step, g_dec, g_flush, g_two
 
-    # end to end through the public API with pinned host buffers: each step's inputs
-    # (q, k_new, v_new) sit in one pinned staging buffer and go up in one copy; the
-    # step is one prepared library call (Int4KVCache.bind_decode_append) where the
-    # cache supports it, else the plain call; the output comes back in one copy
-    in_bytes = [t.numel() * t.element_size() for t in (q, k_new, v_new)]
-    offs = [0, in_bytes[0], in_bytes[0] + in_bytes[1]]
-    h_in = torch.empty(sum(in_bytes), dtype=torch.uint8).pin_memory()
-    d_in = torch.empty(sum(in_bytes), dtype=torch.uint8, device=dev)
-    views = []
-    for t, o, nb in zip((q, k_new, v_new), offs, in_bytes):
-        views.append((h_in[o:o + nb].view(t.dtype).view(t.shape), d_in[o:o + nb].view(t.dtype).view(t.shape)))
-    for (h, _), t in zip(views, (q, k_new, v_new)):
-        h.copy_(t.cpu())
-    d_q, d_k, d_v = (dv for _, dv in views)
+    # end to end through the C ABI with HOST buffers: the step's q, k_new, v_new and
+    # output are pinned host tensors; tq_sdpa_int4_decode_append_host enqueues their
+    # copies and the step in one call (a prepared call, Int4KVCache.bind_decode_append_host).
+    # Caches without that call: one pinned copy up, the public step call, one copy back.
+    h_q, h_k, h_v = (t.cpu().pin_memory() for t in (q, k_new, v_new))
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
     if not (w.cb_bits or srft):
-        bound, _ = cache.bind_decode_append(d_q, d_k, d_v, ctx_dev, max_ctx, scale, out)
+        host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale)
+
+        def e2e_step():
+            host_step()
     else:
-        bound = lambda: cache.decode_append(d_q, d_k, d_v, ctx_dev, max_ctx, scale, out)
+        d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+        def e2e_step():
+            d_q.copy_(h_q, non_blocking=True)
+            d_k.copy_(h_k, non_blocking=True)
+            d_v.copy_(h_v, non_blocking=True)
+            cache.decode_append(d_q, d_k, d_v, ctx_dev, max_ctx, scale, out)
+            h_out.copy_(out, non_blocking=True)
     e2e_t = []
     for i in range(args.warmup + args.steps):
         flush.fill_(i & 0xFF)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        d_in.copy_(h_in, non_blocking=True)
-        bound()
-        h_out.copy_(out, non_blocking=True)
+        e2e_step()
         b.record(stream)
         b.synchronize()
         if i >= args.warmup:
@@ -403,15 +403,15 @@ def run_tq(args):
                      "algorithmic_bytes": algo, "traffic": ncu_traffic("decode", w.name)},
         "e2e": {"value": round(world * kvb / e2e_s / 1e9, 1), "unit": "GB/s",
                 "us_per_step": round(e2e_s * 1e6, 2),
-                "h2d_bytes_per_step": int(h_in.numel()),
+                "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())},
         "gpu_launches": launches_per_step * args.steps,
         "step": step_desc,
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
                   "launching stream (decode split from a K-decode graph; the two-call step "
-                  "from a third graph); e2e: per step, one pinned host-to-device copy of the "
-                  "step's inputs, the public API step call, one device-to-host copy of the "
-                  "output, between CUDA events",
+                  "from a third graph); e2e: per step, tq_sdpa_int4_decode_append_host on "
+                  "pinned host buffers (copies of q, k_new, v_new up, the step, the output "
+                  "down) between CUDA events",
         "clocks": clocks,
         "bulk_prefill": prefill,
         "bf16_dequantize_then_attend": baseline,

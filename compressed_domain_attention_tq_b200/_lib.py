@@ -25,7 +25,9 @@ SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_t
            "tq_decode_srft_workspace_bytes", "tq_quantize_append_srft", "tq_sdpa_int4_decode_srft",
            "tq_sdpa_int4_decode_append_srft", "tq_lloyd_max_gaussian", "tq_decode_cb_workspace_bytes",
            "tq_quantize_append_cb", "tq_sdpa_cb_decode", "tq_sdpa_cb_decode_append",
-           "tq_sdpa_int4_decode_srft_lse", "tq_sdpa_cb_decode_lse", "tq_status_string")
+           "tq_sdpa_int4_decode_srft_lse", "tq_sdpa_cb_decode_lse",
+           "tq_decode_append_host_workspace_bytes", "tq_sdpa_int4_decode_append_host",
+           "tq_status_string")
 
 _lib = None
 
@@ -97,6 +99,11 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_cb_decode_lse.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P,
                                           i32, P, f32, P, P, P, sz, P]
     lib.tq_sdpa_cb_decode_lse.restype = i32
+    lib.tq_decode_append_host_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    lib.tq_decode_append_host_workspace_bytes.restype = sz
+    lib.tq_sdpa_int4_decode_append_host.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P,
+                                                    P, P, P, i64, P, i32, P, f32, P, P, sz, P]
+    lib.tq_sdpa_int4_decode_append_host.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -416,3 +423,41 @@ def sdpa_cb_decode_lse(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_
         workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != TQ_OK:
         raise TQError(rc, "tq_sdpa_cb_decode_lse")
+
+
+# -------------------------------------------------- host-buffer decode step
+
+def decode_append_host_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx,
+                                       q_dtype=torch.bfloat16, kv_dtype=torch.bfloat16) -> int:
+    code = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16}
+    return int(load().tq_decode_append_host_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
+                                                            max_ctx, code[q_dtype], code[kv_dtype]))
+
+
+def _host(*ts):
+    for t in ts:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("the step's inputs and output must be contiguous host tensors")
+
+
+def bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed,
+                                      v_scales, ctx_lens, max_ctx, signs, attn_scale, out_host,
+                                      workspace, stream=None) -> BoundCall:
+    """A prepared decode step whose q, k_new, v_new and output live in (pinned) host
+    memory: each call enqueues their copies, the step and the copy back on the stream."""
+    _host(q_host, k_new_host, v_new_host, out_host)
+    _need_cuda(k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, workspace)
+    if k_new_host.dtype != v_new_host.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q_host.shape
+    Hkv = k_packed.shape[1]
+    i32, f32, sz = ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    args = (_ptr(q_host), i32(_dtype_code(q_host)), _ptr(k_new_host), _ptr(v_new_host),
+            i32(_dtype_code(k_new_host)), i32(B), i32(Hq), i32(Hkv), i32(d), i32(32), _ptr(k_packed),
+            _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), ctypes.c_int64(k_packed.shape[2]),
+            _ptr(ctx_lens), i32(int(max_ctx)), _ptr(signs), f32(float(attn_scale)), _ptr(out_host),
+            _ptr(workspace), sz(workspace.numel() * workspace.element_size()), _stream(stream))
+    keep = (q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs,
+            out_host, workspace)
+    return BoundCall(load().tq_sdpa_int4_decode_append_host, args,
+                     "tq_sdpa_int4_decode_append_host", keep)

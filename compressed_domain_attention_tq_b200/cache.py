@@ -136,6 +136,28 @@ class Int4KVCache:
                                                  self.signs, attn_scale, out, ws, stream)
         return step, out
 
+    def bind_decode_append_host(self, q_host: torch.Tensor, k_new_host: torch.Tensor,
+                                v_new_host: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
+                                out_host: torch.Tensor, attn_scale: float | None = None,
+                                stream=None):
+        """A prepared decode step on HOST buffers (q, k_new, v_new, out; pin them): each
+        call of the returned step enqueues their copies and the step in one library call
+        (tq_sdpa_int4_decode_append_host); Hadamard-rotated caches."""
+        if self.srft:
+            raise NotImplementedError("bind_decode_append_host runs on Hadamard-rotated caches")
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        need = _lib.decode_append_host_workspace_bytes(self.batch, q_host.shape[1], self.num_kv_heads,
+                                                       self.head_dim, max_ctx, q_host.dtype,
+                                                       k_new_host.dtype)
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
+        return _lib.bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host, self.k_packed,
+                                                      self.k_scales, self.v_packed, self.v_scales,
+                                                      ctx_lens, max_ctx, self.signs, attn_scale,
+                                                      out_host, ws, stream)
+
     def dequantize(self, rows: int, dtype=torch.bfloat16, stream=None):
         """Dequantized K and V of rows 0 .. rows-1 of every sequence, [B][Hkv][rows][d]
         in the rotated basis (scale * code; not used by decode)."""

@@ -524,6 +524,81 @@ tq_status tq_sdpa_cb_decode_append(const void* q, tq_dtype q_dtype, const void* 
                      "tq_sdpa_cb_decode_append", nullptr, r);
 }
 
+// Device staging of the host-buffer step call, after the decode workspace:
+// q [B][Hq][d], k_new and v_new [B][Hkv][d], out [B][Hq][d] (each 256-byte aligned).
+struct HostStaging {
+  size_t q, k, v, out, total;
+};
+
+static bool host_staging(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t max_ctx, tq_dtype q_dtype, tq_dtype kv_dtype,
+                         HostStaging* hs) {
+  DecodePlan p;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p)) return false;
+  if ((q_dtype != TQ_F32 && q_dtype != TQ_BF16) || (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16))
+    return false;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t qb = (size_t)batch * num_q_heads * head_dim * (q_dtype == TQ_BF16 ? 2 : 4);
+  const size_t kb = (size_t)batch * num_kv_heads * head_dim * (kv_dtype == TQ_BF16 ? 2 : 4);
+  hs->q = up(p.ws_bytes);
+  hs->k = hs->q + up(qb);
+  hs->v = hs->k + up(kb);
+  hs->out = hs->v + up(kb);
+  hs->total = hs->out + (size_t)batch * num_q_heads * head_dim * 4;
+  return true;
+}
+
+size_t tq_decode_append_host_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t head_dim,
+                                             int32_t max_ctx, tq_dtype q_dtype,
+                                             tq_dtype kv_dtype) {
+  HostStaging hs;
+  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype, &hs))
+    return 0;
+  return hs.total;
+}
+
+tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
+                                          const void* k_new_host, const void* v_new_host,
+                                          tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim, int32_t group,
+                                          uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                                          float* v_scales, int64_t capacity,
+                                          const int32_t* ctx_lens, int32_t max_ctx,
+                                          const int8_t* signs, float attn_scale, float* out_host,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* cuda_stream) {
+  if (!q_host || !k_new_host || !v_new_host || !out_host) return TQ_ERR_INVALID_ARG;
+  HostStaging hs;
+  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype, &hs)) {
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+    if (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+    if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+    return TQ_ERR_INVALID_ARG;
+  }
+  if (!workspace || workspace_bytes < hs.total) return TQ_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t qb = hs.k - hs.q, kb = hs.v - hs.k;  // padded sizes; copy the exact bytes
+  const size_t q_bytes = (size_t)batch * num_q_heads * head_dim * (q_dtype == TQ_BF16 ? 2 : 4);
+  const size_t kv_bytes = (size_t)batch * num_kv_heads * head_dim * (kv_dtype == TQ_BF16 ? 2 : 4);
+  const size_t out_bytes = (size_t)batch * num_q_heads * head_dim * 4;
+  (void)qb;
+  (void)kb;
+  cudaError_t e = cudaMemcpyAsync(ws + hs.q, q_host, q_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + hs.k, k_new_host, kv_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + hs.v, v_new_host, kv_bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e, "tq_sdpa_int4_decode_append_host");
+  const tq_status st = decode_impl(
+      ws + hs.q, q_dtype, ws + hs.k, ws + hs.v, kv_dtype, batch, num_q_heads, num_kv_heads,
+      head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens, max_ctx, signs,
+      attn_scale, reinterpret_cast<float*>(ws + hs.out), workspace, hs.q, cuda_stream,
+      "tq_sdpa_int4_decode_append_host");
+  if (st != TQ_OK) return st;
+  return cuda_status(cudaMemcpyAsync(out_host, ws + hs.out, out_bytes, cudaMemcpyDeviceToHost, s),
+                     "tq_sdpa_int4_decode_append_host");
+}
+
 tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
                                      const void* v_new, tq_dtype kv_dtype, int32_t batch,
                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,

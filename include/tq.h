@@ -191,6 +191,35 @@ TQ_API tq_status tq_sdpa_int4_decode_append(
     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * tq_sdpa_int4_decode_append_host -- tq_sdpa_int4_decode_append with the step's
+ * inputs and output in HOST memory: it enqueues the host-to-device copies of
+ * q, k_new and v_new into staging space at the end of the workspace, the
+ * decode step, and the device-to-host copy of the output, all on cuda_stream,
+ * and returns without synchronizing (the output is in out_host once the stream
+ * reaches that point).  Host buffers should be pinned (cudaHostAlloc) for the
+ * copies to be asynchronous; pageable memory works but the copies then stage
+ * through the driver.
+ *
+ *  q_host          [B][Hq][d] of q_dtype; k_new_host, v_new_host [B][Hkv][1][d] of
+ *                  kv_dtype; out_host [B][Hq][d] fp32.
+ *  workspace       device, workspace_bytes >= tq_decode_append_host_workspace_bytes().
+ * The cache buffers, ctx_lens and signs are device pointers, as in
+ * tq_sdpa_int4_decode_append, whose errors it returns (TQ_ERR_INVALID_ARG also
+ * for a NULL host pointer).
+ */
+TQ_API size_t tq_decode_append_host_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                    int32_t num_kv_heads, int32_t head_dim,
+                                                    int32_t max_ctx, tq_dtype q_dtype,
+                                                    tq_dtype kv_dtype);
+
+TQ_API tq_status tq_sdpa_int4_decode_append_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales,
+    int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+    float attn_scale, float* out_host, void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * tq_sdpa_int4_decode_lse -- tq_sdpa_int4_decode that also returns each head's
  * softmax state, so that outputs over disjoint parts of a context (for
  * instance the token shards of several GPUs) can be combined exactly with

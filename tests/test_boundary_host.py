@@ -248,3 +248,19 @@ def test_codebook_calls_reject_on_host(lib):
     assert dec(bits=7) == _lib.TQ_ERR_UNSUPPORTED
     assert dec(levels=None) == _lib.TQ_ERR_INVALID_ARG
     assert dec(ws_bytes=100) == _lib.TQ_ERR_WORKSPACE
+
+
+def test_host_step_rejects_on_host(lib):
+    fb = FakeBuffers()
+    need = lib.tq_decode_append_host_workspace_bytes(1, 8, 2, 128, 64, 1, 1)
+    assert need > _lib.decode_workspace_bytes(1, 8, 2, 128, 64)
+    assert lib.tq_decode_append_host_workspace_bytes(1, 8, 2, 96, 64, 1, 1) == 0
+    def call(q=fb.p(0), out=fb.p(4096), ws_bytes=1 << 16, d=128, qd=1):
+        return lib.tq_sdpa_int4_decode_append_host(
+            q, qd, fb.p(8192), fb.p(12288), 1, 1, 8, 2, d, 32, fb.p(1024), fb.p(2048), fb.p(3072),
+            fb.p(4096), 64, fb.p(512), 64, None, 0.125, out, fb.p(16384), ws_bytes, None)
+    assert call(q=None) == _lib.TQ_ERR_INVALID_ARG
+    assert call(out=None) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d=96) == _lib.TQ_ERR_UNSUPPORTED
+    assert call(qd=7) == _lib.TQ_ERR_INVALID_ARG
+    assert call(ws_bytes=need - 1) == _lib.TQ_ERR_WORKSPACE

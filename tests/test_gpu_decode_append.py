@@ -112,3 +112,33 @@ def test_bound_decode_append_matches_plain_call_on_refilled_buffers():
     for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
                     (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
         assert torch.equal(a, b)
+
+
+def test_host_buffer_step_matches_device_step():
+    """tq_sdpa_int4_decode_append_host on pinned host buffers writes the same cache
+    rows and returns the same output (bit for bit) as the device-buffer step."""
+    require_cuda()
+    import torch
+    from compressed_domain_attention_tq_b200 import Int4KVCache
+    B, Hkv, G, d, T = 2, 2, 8, 128, 900
+    g = torch.Generator().manual_seed(93)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+    caches = [Int4KVCache(B, Hkv, d, T + 2, signs=signs) for _ in range(2)]
+    for c in caches:
+        c.append(k, v, torch.zeros(B, dtype=torch.int32, device="cuda"))
+    q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+    ctx = torch.tensor([T + 1, T - 40], dtype=torch.int32, device="cuda")
+    hq, hk, hv = q.pin_memory(), kn.pin_memory(), vn.pin_memory()
+    hout = torch.empty(B, Hkv * G, d, dtype=torch.float32).pin_memory()
+    step = caches[0].bind_decode_append_host(hq, hk, hv, ctx, T + 2, hout, 0.1)
+    step()
+    out_d = caches[1].decode_append(q.cuda(), kn.cuda(), vn.cuda(), ctx, T + 2, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, out_d.cpu())
+    for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
+                    (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
+        assert torch.equal(a, b)
