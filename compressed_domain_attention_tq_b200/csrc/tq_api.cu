@@ -289,6 +289,11 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     return TQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < a.plan.ws_bytes) return TQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
+  // Test hooks (environment): TQ_TEST_FAIL_LAUNCH fails the call as a failed launch would,
+  // before anything is enqueued; TQ_TEST_STARVE_PIPELINE makes the tensor-core decode's
+  // bounded waits for its first copies run out (its outputs are then NaN).
+  if (getenv("TQ_TEST_FAIL_LAUNCH")) return cuda_status(cudaErrorLaunchFailure, where);
+  a.test_starve = getenv("TQ_TEST_STARVE_PIPELINE") != nullptr;
   a.q = q;
   a.q_bf16 = q_dtype == TQ_BF16;
   a.B = batch;

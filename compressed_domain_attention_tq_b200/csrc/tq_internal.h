@@ -80,6 +80,8 @@ struct DecodeArgs {
   float* lse;  // NULL, or [B][Hq][2]: each head's (max in log2 units, sum) for merging contexts
   const float* q_rot = nullptr;     // SRFT variant: [B][Hq][d] rotated queries F(sigma q)/lambda_K;
                                     // the decode kernels read these instead of rotating q
+  int test_starve = 0;              // test hook: the tensor-core decode withholds each CTA's
+                                    // first copy, so its waits run out (the abort path)
   int q_rot_overlap = 0;            // the tensor-core decode may start while the preceding grid
                                     // runs (programmatic dependent launch): 1 = that grid only
                                     // rotates the queries; 2 = it also appends each sequence's
