@@ -67,10 +67,18 @@ def kv_bytes(w, ctx_tokens):
     return 2 * per_vec * w.num_kv_heads * int(sum(ctx_tokens))
 
 
-def lib_source_hash():
+# Sources that determine each profiled kernel's code and launch shape; a
+# committed DRAM-traffic figure counts only while their hash is unchanged.
+KERNEL_SOURCES = {
+    "decode": ["decode_mma.cu", "quantize_vector.cuh", "tq_internal.h", "tq_api.cu"],
+    "quantize_bulk": ["quantize.cu", "quantize_vector.cuh", "tq_internal.h", "tq_api.cu"],
+}
+
+
+def kernel_source_hash(kernel_key):
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "compressed_domain_attention_tq_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in sorted(KERNEL_SOURCES[kernel_key]):
         with open(os.path.join(cs, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -85,7 +93,8 @@ def ncu_traffic(kernel_key, workload):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_hash") != lib_source_hash() or e.get("workload_name") != workload:
+    if (not e or e.get("source_hash") != kernel_source_hash(kernel_key)
+            or e.get("workload_name") != workload):
         return None
     return e.get("dram_bytes_per_launch")
 

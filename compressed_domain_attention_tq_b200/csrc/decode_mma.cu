@@ -27,6 +27,8 @@
 //    the product.  Each head's rotated, scaled query is first multiplied by a
 //    power of two so its largest element lies in [2^13, 2^14) (f16 range).
 //    Per group of 32 dims the product is scaled by the token's fp32 K scale.
+//    The K codes enter as exact f16 subnormals (c + 8) 2^-24 (one LOP3 per two
+//    codes); the epilogue scales by 2^24 and removes the offset 8 sum_g q.
 //  - P.V: the operand is P' = 2^(S - m - F) * s_v[token, group], split into
 //    hi + lo.  F (per warp) keeps P' below 2^15: it is set from the first
 //    tile's V scales and raised, with an exact power-of-two rescale of the
@@ -163,6 +165,15 @@ __device__ __forceinline__ uint32_t codes_hi(uint32_t x) {
   return hfma2(and_xor(x, 0x00F000F0u, 0x64806480u), 0x2C002C00u, 0xD480D480u);  // /16 - 72
 }
 
+// Score operand: two int4 codes -> f16x2 in one LOP3, without the subtraction.
+// Flipping bit 3 gives u = c + 8 in 1..15, which OR-ed under a zero exponent is
+// the subnormal f16 u * 2^-24 (bits 4..7: 16 u * 2^-24), exact.  The query
+// entries that meet the bits 4..7 codes are divided by 16, so an MMA over a
+// group yields 2^-24 sum_j q_j (c_j + 8); the tile epilogue scales it by 2^24
+// and removes 8 sum_j q_j, a constant of (head, group).
+__device__ __forceinline__ uint32_t kcodes_lo(uint32_t x) { return and_xor(x, 0x000F000Fu, 0x00080008u); }
+__device__ __forceinline__ uint32_t kcodes_hi(uint32_t x) { return and_xor(x, 0x00F000F0u, 0x00800080u); }
+
 // fp32 pair -> f16x2 (low half = lo_elem)
 __device__ __forceinline__ uint32_t f16x2(float lo_elem, float hi_elem) {
   uint32_t d;
@@ -237,7 +248,8 @@ struct Cfg {
   static constexpr int QA = al(CUR + 32);                    // f16 [NG][2][16][16] score A
   static constexpr int QS = al(QA + NG * 2 * 16 * 16 * 2);   // float [NH][D] query
   static constexpr int QEXP = al(QS + 4 * NH * D);           // float [NH]
-  static constexpr int MACC = al(QEXP + 4 * 8);              // float [NW][NH][D]
+  static constexpr int QK8 = al(QEXP + 4 * 8);               // float [NH][NG] -8 sum_g q
+  static constexpr int MACC = al(QK8 + 4 * NH * NG);         // float [NW][NH][D]
   static constexpr int MM = al(MACC + 4 * NW * NH * D);      // float [NW][NH] max
   static constexpr int ML = al(MM + 4 * NW * NH);            // float [NW][NH] sum
   static constexpr int MW = al(ML + 4 * NW * NH);            // float [NW][NH] weight
@@ -348,6 +360,7 @@ template <int D, int PATH>
 struct WarpState {
   float acc[Cfg<D, PATH>::NACC][4];  // P.V accumulators (fragments), scaled by 2^-F
   uint32_t qa_addr;                  // this lane's ldmatrix row address of the score A tiles
+  uint32_t k8_addr;                  // shared address of -8 sum_g q of this thread's head
   float m;                           // running max of this thread's head (log2 units)
   float2 l;                          // this thread's share of the running sum (two partial
                                      // sums, added at the end), scaled by 2^-F
@@ -471,15 +484,23 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   // Score A tiles in shared memory, f16 [group][k-step][row][k]: row r < 8 is
   // the hi part of head h(r), row 8 + r its lo part; MMA index k of k-step ks
   // is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in which
-  // the K-code words are unpacked.  The two 16-byte halves of a row swap when
-  // row bit 2 is set, so ldmatrix phases hit distinct banks.
+  // the K-code words are unpacked; k >= 8 meets the codes of bits 4..7, whose
+  // operand carries a factor 16 (kcodes_hi), so those entries are q / 16.  The
+  // two 16-byte halves of a row swap when row bit 2 is set, so ldmatrix phases
+  // hit distinct banks.  Beside them, -8 sum_g q per head and group.
   __half* qa = reinterpret_cast<__half*>(smem + C::QA);
+  if (threadIdx.x < C::NH * C::NG) {
+    const int h = threadIdx.x / C::NG, g = threadIdx.x % C::NG;
+    float sum = 0.0f;
+    for (int j = 0; j < 32; ++j) sum += qs[h * D + 32 * g + j];
+    reinterpret_cast<float*>(smem + C::QK8)[threadIdx.x] = -8.0f * sum;
+  }
   for (int idx = threadIdx.x; idx < (D / 32) * 2 * 256; idx += C::THREADS) {
     const int k = idx & 15, row = (idx >> 4) & 15, gks = idx >> 8;
     const int g = gks >> 1, ks = gks & 1;
     const int hr = PATH == 0 ? (row & 7) : ((row & 7) >> 1);
     const int dim = 32 * g + 8 * ((k & 7) >> 1) + 2 * ks + (k >> 3) + 4 * (k & 1);
-    const float v = qs[hr * D + dim];
+    const float v = qs[hr * D + dim] * ((k >> 3) ? 0.0625f : 1.0f);  // exact
     const __half hi = __float2half_rn(v);
     const __half val = row < 8 ? hi : __float2half_rn(v - __half2float(hi));
     const int half16 = (k >> 3) ^ ((row >> 2) & 1);
@@ -492,6 +513,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     const int mi = lane >> 3, row = (lane & 7) + 8 * (mi & 1), kb = mi >> 1;
     st.qa_addr = smem_u32(smem + C::QA) + row * 32 + ((kb ^ ((row >> 2) & 1)) * 16);
   }
+  st.k8_addr = smem_u32(smem + C::QK8) + hrow * C::NG * 4;
   st.qexp = qexp[hrow];
 }
 
@@ -517,7 +539,9 @@ __device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
 // krow[nt]: tile row of score n-tile nt's column gid.
 
 // Scores before the qexp factor, S = sum_g s_k[t, g] (q_hi + q_lo) . c_k[t, g];
-// unless FULL, rows past nvalid get -inf.  Branch-free.
+// unless FULL, rows past nvalid get -inf.  Branch-free.  Per group the two
+// MMAs give x = 2^-24 sum_j q_j (c_j + 8) (kcodes_lo / kcodes_hi), and the
+// group's term is s_k (2^24 x - 8 sum_j q_j).
 template <int D, int PATH, int TPW, bool FULL>
 __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, int nvalid, int tig,
                                             const int (&rho)[4], const int (&krow)[2],
@@ -553,6 +577,12 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
         sk[u][i][4 * q + 3] = v.w;
       }
   }
+  float k8[NG];  // -8 sum_g q of this thread's head
+#pragma unroll
+  for (int q = 0; q < NG / 4; ++q)
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(k8[4 * q]), "=f"(k8[4 * q + 1]), "=f"(k8[4 * q + 2]), "=f"(k8[4 * q + 3])
+                 : "r"(st.k8_addr + 16 * q));
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
@@ -571,9 +601,10 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
             prmt(kw[u][nt][g / 2], kw[u][nt][NG / 2 + g / 2], (g & 1) ? 0x7632u : 0x5410u);
         const uint32_t Y = X >> 8;
         float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], codes_lo(X), codes_hi(X));
-        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], codes_lo(Y), codes_hi(Y));
-        const float2 x = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
+        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], kcodes_lo(X), kcodes_hi(X));
+        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], kcodes_lo(Y), kcodes_hi(Y));
+        const float2 x = __ffma2_rn(__fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3])),
+                                    make_float2(16777216.0f, 16777216.0f), make_float2(k8[g], k8[g]));
         S[u][2 * nt] = fmaf(sk[u][2 * nt][g], x.x, S[u][2 * nt]);
         S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], x.y, S[u][2 * nt + 1]);
       }
