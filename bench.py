@@ -394,7 +394,8 @@ def run_tq(args):
         "two_call_step_us": round(two_s * 1e6, 2),
         "pct_of_8TBps": round(100 * kvb / step_s / 1e9 / NOMINAL_HBM_GBS, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 codes, fp32 accumulation", "data": "synthetic (seeded N(0,1), bf16)",
+        "dtype": (f"{w.cb_bits}-bit codebook indices, fp32 accumulation" if w.cb_bits
+                  else "int4 codes, fp32 accumulation"), "data": "synthetic (seeded N(0,1), bf16)",
         "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
                    "context": max_ctx,
                    "rotation": (w.rotation_kind if w.rotation else False),
@@ -406,7 +407,9 @@ def run_tq(args):
                          (f"not flushed: each step reads {kvb} B of packed cache, more than the "
                           f"{l2_bytes} B L2"),
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "sdpa_int4 decode (split-K + merge)",
+        "roofline": {"bound": "hbm",
+                     "kernel": (f"{w.cb_bits}-bit codebook decode (split-K + merge)" if w.cb_bits
+                                else "sdpa_int4 decode (split-K + merge)"),
                      "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_bytes": algo, "traffic": ncu_traffic("decode", w.name)},

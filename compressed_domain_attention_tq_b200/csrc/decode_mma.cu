@@ -224,15 +224,14 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) 
 // live in shared memory); larger ones walk every (sequence, kv head, chunk).
 constexpr int kMaxListB = 1024;
 
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 struct Cfg {
   static constexpr int NW = 8;                  // warps per CTA (all consumers)
   static constexpr int TPW = D == 128 ? 2 : 1;  // 16-token tiles per warp per stage
   static constexpr int THREADS = 32 * NW;
   static constexpr int ST = 16 * TPW * NW;      // tokens per pipeline stage
   static constexpr int NG = D / 32;             // quantization groups per vector
-  static constexpr int RB = D / 2;              // packed bytes per row
-  static constexpr int SB = 2 * NG;             // bytes of one of a row's 8 sub-blocks
+  static constexpr int RB = FMT ? D * FMT / 8 : D / 2;  // packed bytes per row
   static constexpr int NH = PATH == 0 ? 8 : 4;  // query heads per kv head (max)
   static constexpr int NACC = PATH == 0 ? 4 * NG : 2 * NG;  // accumulator fragments
   static constexpr int NS = D == 128 ? 4 : 3;                // pipeline stages
@@ -256,8 +255,10 @@ struct Cfg {
   static constexpr int MTOT = al(MW + 4 * NW * NH);          // float [NH] max, [NH] sum
   static constexpr int ABORT = al(MTOT + 4 * 2 * NH);        // int
   static constexpr int PFX = al(ABORT + 16);                 // int [kMaxListB + 1] item prefix
-  static constexpr int BYTES = PFX + 4 * (kMaxListB + 1);
+  static constexpr int LUT = al(PFX + 4 * (kMaxListB + 1));  // codebook: uint2 [2^(2 FMT)]
+  static constexpr int BYTES = LUT + (FMT ? 8 << (2 * FMT) : 0);
   static_assert(BYTES <= 227 * 1024, "shared memory");
+  static_assert(FMT == 0 || (PATH == 0 && D == 128), "codebook decode: heads on rows, d = 128");
   static_assert(STAGE % 16 == 0 && VC % 16 == 0 && KS % 16 == 0 && VS % 16 == 0, "alignment");
 };
 
@@ -312,10 +313,10 @@ __device__ __forceinline__ bool item_range(const DecodeArgs& a, const int* pfx, 
 // in smem + PFX is used (both set once at kernel start and only read after).
 // Issues the next stage of this CTA's stage sequence
 // into `slot`; returns false when the sequence is exhausted.
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* smem, int* cur,
                                            uint64_t* full, int slot) {
-  using C = Cfg<D, PATH>;
+  using C = Cfg<D, PATH, FMT>;
   const int n_items = cur[6];
   const int* pfx = cur[7] ? reinterpret_cast<const int*>(smem + C::PFX) : nullptr;
   int it = cur[0], t = cur[1], t1 = cur[2];
@@ -356,15 +357,17 @@ __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* s
 }
 
 // Per-thread state of one warp for one item.
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 struct WarpState {
-  float acc[Cfg<D, PATH>::NACC][4];  // P.V accumulators (fragments), scaled by 2^-F
+  float acc[Cfg<D, PATH, FMT>::NACC][4];  // P.V accumulators (fragments), scaled by 2^-F
   uint32_t qa_addr;                  // this lane's ldmatrix row address of the score A tiles
   uint32_t k8_addr;                  // shared address of -8 sum_g q of this thread's head
   float m;                           // running max of this thread's head (log2 units)
   float2 l;                          // this thread's share of the running sum (two partial
                                      // sums, added at the end), scaled by 2^-F
   float qexp;                        // 2^E of this thread's head (query normalisation)
+  float cexp;                        // codebook: 2^e, the levels' normalisation (else 1)
+  uint32_t lut;                      // codebook: shared address of the level-pair table
   int F;                             // V-scale normalisation exponent
   bool fset;                         // F chosen for this item
 };
@@ -372,11 +375,11 @@ struct WarpState {
 // Rotated, scaled query of the item's G heads -> smem (normalised by a power
 // of two per head), then every thread builds its score A fragments.  Warp
 // w < NH prepares head w; the FWHT runs in registers and shuffles.
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, unsigned char* smem,
-                                           WarpState<D, PATH>& st, bool start_stream,
+                                           WarpState<D, PATH, FMT>& st, bool start_stream,
                                            int* cur, uint64_t* full) {
-  using C = Cfg<D, PATH>;
+  using C = Cfg<D, PATH, FMT>;
   constexpr int E = D / 32;  // elements per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv;
@@ -390,7 +393,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     if (a.k_new != nullptr) asm volatile("bar.sync 2, 96;" ::: "memory");
     if (threadIdx.x == C::THREADS - 32)
       for (int s = 0; s < C::NS; ++s)
-        if (!issue_next<D, PATH>(a, smem, cur, full, s)) break;
+        if (!issue_next<D, PATH, FMT>(a, smem, cur, full, s)) break;
   }
   for (int hh = 0; hh < HPW; ++hh) {
     const int h = warp * HPW + hh;
@@ -482,14 +485,16 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   }
   barrier_all<C::THREADS>();
   // Score A tiles in shared memory, f16 [group][k-step][row][k]: row r < 8 is
-  // the hi part of head h(r), row 8 + r its lo part; MMA index k of k-step ks
-  // is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in which
-  // the K-code words are unpacked; k >= 8 meets the codes of bits 4..7, whose
-  // operand carries a factor 16 (kcodes_hi), so those entries are q / 16.  The
-  // two 16-byte halves of a row swap when row bit 2 is set, so ldmatrix phases
-  // hit distinct banks.  Beside them, -8 sum_g q per head and group.
+  // the hi part of head h(r), row 8 + r its lo part.  int4: MMA index k of
+  // k-step ks is coordinate 32g + 8((k%8)/2) + 2ks + k/8 + 4(k%2), the order in
+  // which the K-code words are unpacked; k >= 8 meets the codes of bits 4..7,
+  // whose operand carries a factor 16 (kcodes_hi), so those entries are q / 16.
+  // Codebook: coordinate 32g + 8((k%8)/2) + 4ks + 2(k/8) + k%2, the index pairs
+  // of tile_scores_cb.  The two 16-byte halves of a row swap when row bit 2 is
+  // set, so ldmatrix phases hit distinct banks.  Beside them (int4), -8 sum_g q
+  // per head and group.
   __half* qa = reinterpret_cast<__half*>(smem + C::QA);
-  if (threadIdx.x < C::NH * C::NG) {
+  if (FMT == 0 && threadIdx.x < C::NH * C::NG) {
     const int h = threadIdx.x / C::NG, g = threadIdx.x % C::NG;
     float sum = 0.0f;
     for (int j = 0; j < 32; ++j) sum += qs[h * D + 32 * g + j];
@@ -499,8 +504,9 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     const int k = idx & 15, row = (idx >> 4) & 15, gks = idx >> 8;
     const int g = gks >> 1, ks = gks & 1;
     const int hr = PATH == 0 ? (row & 7) : ((row & 7) >> 1);
-    const int dim = 32 * g + 8 * ((k & 7) >> 1) + 2 * ks + (k >> 3) + 4 * (k & 1);
-    const float v = qs[hr * D + dim] * ((k >> 3) ? 0.0625f : 1.0f);  // exact
+    const int dim = FMT ? 32 * g + 8 * ((k & 7) >> 1) + 4 * ks + 2 * (k >> 3) + (k & 1)
+                        : 32 * g + 8 * ((k & 7) >> 1) + 2 * ks + (k >> 3) + 4 * (k & 1);
+    const float v = qs[hr * D + dim] * ((FMT == 0 && (k >> 3)) ? 0.0625f : 1.0f);  // exact
     const __half hi = __float2half_rn(v);
     const __half val = row < 8 ? hi : __float2half_rn(v - __half2float(hi));
     const int half16 = (k >> 3) ^ ((row >> 2) & 1);
@@ -514,14 +520,14 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     st.qa_addr = smem_u32(smem + C::QA) + row * 32 + ((kb ^ ((row >> 2) & 1)) * 16);
   }
   st.k8_addr = smem_u32(smem + C::QK8) + hrow * C::NG * 4;
-  st.qexp = qexp[hrow];
+  st.qexp = qexp[hrow] * st.cexp;
 }
 
-template <int D, int PATH>
-__device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
+template <int D, int PATH, int FMT>
+__device__ __forceinline__ void scale_acc(WarpState<D, PATH, FMT>& st, float f) {
   const float2 ff = make_float2(f, f);
 #pragma unroll
-  for (int j = 0; j < Cfg<D, PATH>::NACC; ++j)
+  for (int j = 0; j < Cfg<D, PATH, FMT>::NACC; ++j)
 #pragma unroll
     for (int r = 0; r < 4; r += 2) {
       const float2 v = __fmul2_rn(make_float2(st.acc[j][r], st.acc[j][r + 1]), ff);
@@ -542,12 +548,12 @@ __device__ __forceinline__ void scale_acc(WarpState<D, PATH>& st, float f) {
 // unless FULL, rows past nvalid get -inf.  Branch-free.  Per group the two
 // MMAs give x = 2^-24 sum_j q_j (c_j + 8) (kcodes_lo / kcodes_hi), and the
 // group's term is s_k (2^24 x - 8 sum_j q_j).
-template <int D, int PATH, int TPW, bool FULL>
+template <int D, int PATH, int FMT, int TPW, bool FULL>
 __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, int nvalid, int tig,
                                             const int (&rho)[4], const int (&krow)[2],
-                                            const WarpState<D, PATH>& st, float (&S)[TPW][4]) {
-  using C = Cfg<D, PATH>;
-  constexpr int NG = C::NG, RB = C::RB, SB = C::SB;
+                                            const WarpState<D, PATH, FMT>& st, float (&S)[TPW][4]) {
+  using C = Cfg<D, PATH, FMT>;
+  constexpr int NG = C::NG, RB = C::RB, SB = 2 * NG;  // SB: bytes of one of a row's 8 sub-blocks
   const unsigned char* kc = stg + C::KC + r0 * RB;
   const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
   uint32_t kw[TPW][2][NG];  // per tile and n-tile: sub-blocks 2tig, 2tig+1 of token krow[nt]
@@ -616,10 +622,88 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
       for (int i = 0; i < 4; ++i) S[u][i] = 16 * u + rho[i] < nvalid ? S[u][i] : -INFINITY;
 }
 
+// Codebook scores.  Per group the B operand is the levels C[index] of the
+// token's coordinates, as f16 hi + lo parts read from the level-pair table
+// (entry i0 | i1 << FMT holds C[i0], C[i1] as an f16x2 hi part and an f16x2 lo
+// part), so the group's product sum_j (q_hi + q_lo)_j (C_hi + C_lo)[index_j]
+// collects all four partial products in one accumulator; then
+// S = sum_g sigma_k[t, g] x_g.  Thread tig takes in-group coordinates 8tig ..
+// 8tig + 7 (bits 8 FMT tig .. of the group's bit string) as the index pairs
+// (8tig + 2m, 8tig + 2m + 1), m = 0..3.  Branch-free.
+template <int D, int PATH, int FMT, int TPW, bool FULL>
+__device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int r0, int nvalid, int tig,
+                                               const int (&rho)[4], const int (&krow)[2],
+                                               const WarpState<D, PATH, FMT>& st,
+                                               const unsigned char* lutp, float (&S)[TPW][4]) {
+  using C = Cfg<D, PATH, FMT>;
+  constexpr int NG = C::NG, RB = C::RB, GB = 4 * FMT;  // GB: bytes per group
+  constexpr uint32_t KM = (1u << (2 * FMT)) - 1;  // key mask
+  const unsigned char* kc = stg + C::KC + r0 * RB;
+  const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
+  // the thread's 8 FMT bits of a group start at byte FMT tig of the group
+  const int wo = (FMT * tig) >> 2, sh = 8 * ((FMT * tig) & 3);
+  uint32_t pc[TPW][2][NG];
+  float sk[TPW][4][NG];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const uint32_t* gw =
+            reinterpret_cast<const uint32_t*>(kc + (16 * u + krow[nt]) * RB + g * GB) + wo;
+        pc[u][nt][g] = FMT == 3 ? __funnelshift_r(gw[0], gw[1], sh) : gw[0] >> sh;
+      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < NG / 4; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(ks + (16 * u + rho[i]) * NG)[q];
+        sk[u][i][4 * q] = v.x;
+        sk[u][i][4 * q + 1] = v.y;
+        sk[u][i][4 * q + 2] = v.z;
+        sk[u][i][4 * q + 3] = v.w;
+      }
+  }
+#pragma unroll
+  for (int u = 0; u < TPW; ++u)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) S[u][i] = 0.0f;
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    uint32_t a[2][4];
+    ldsm_x4(st.qa_addr + (2 * g) * 512, a[0][0], a[0][1], a[0][2], a[0][3]);
+    ldsm_x4(st.qa_addr + (2 * g + 1) * 512, a[1][0], a[1][1], a[1][2], a[1][3]);
+#pragma unroll
+    for (int u = 0; u < TPW; ++u)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const uint32_t x = pc[u][nt][g];
+        uint2 e[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          e[m] = *reinterpret_cast<const uint2*>(lutp + (((x >> (2 * FMT * m)) & KM) << 3));
+        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], e[0].x, e[1].x);
+        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], e[0].y, e[1].y);
+        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], e[2].x, e[3].x);
+        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], e[2].y, e[3].y);
+        const float2 x2 = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
+        S[u][2 * nt] = fmaf(sk[u][2 * nt][g], x2.x, S[u][2 * nt]);
+        S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], x2.y, S[u][2 * nt + 1]);
+      }
+  }
+  if (!FULL)
+#pragma unroll
+    for (int u = 0; u < TPW; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S[u][i] = 16 * u + rho[i] < nvalid ? S[u][i] : -INFINITY;
+}
+
 // Running max of this thread's head (log2 units) over the tiles' scores; when
 // it grows, the accumulators and the running sum are rescaled.
-template <int D, int PATH, int TPW>
-__device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], WarpState<D, PATH>& st) {
+template <int D, int PATH, int FMT, int TPW>
+__device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], WarpState<D, PATH, FMT>& st) {
   float mx;
   if (TPW == 2)
     mx = fmax3(fmax3(S[0][0], S[0][1], S[0][2]), fmax3(S[0][3], S[TPW - 1][0], S[TPW - 1][1]),
@@ -639,10 +723,10 @@ __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], Warp
 }
 
 // V scales of the warp's rows (unless FULL, zero past nvalid).
-template <int D, int PATH, int TPW, bool FULL>
+template <int D, int PATH, int FMT, int TPW, bool FULL>
 __device__ __forceinline__ void load_vscales(const unsigned char* stg, int r0, int nvalid,
                                              const int (&rho)[4], float (&sv)[TPW][4][D / 32]) {
-  using C = Cfg<D, PATH>;
+  using C = Cfg<D, PATH, FMT>;
   constexpr int NG = C::NG;
   const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
 #pragma unroll
@@ -665,10 +749,10 @@ __device__ __forceinline__ void load_vscales(const unsigned char* stg, int r0, i
 // follows the largest V scale seen (raised with an exact power-of-two rescale
 // of acc, l and these weights, which is rare, so the weights are computed
 // first with the current F and the check runs beside them).
-template <int D, int PATH, int TPW>
+template <int D, int PATH, int FMT, int TPW>
 __device__ __forceinline__ void tile_weights(const float (&S)[TPW][4],
                                              const float (&sv)[TPW][4][D / 32],
-                                             WarpState<D, PATH>& st, float (&p)[TPW][4]) {
+                                             WarpState<D, PATH, FMT>& st, float (&p)[TPW][4]) {
   constexpr int NG = D / 32, NV = 4 * TPW * NG;
   // m = -inf only while every score so far is -inf (no real token yet)
   const float mF = st.m == -INFINITY ? 0.0f : st.m + (float)st.F;
@@ -722,13 +806,13 @@ __device__ __forceinline__ void tile_weights(const float (&S)[TPW][4],
 }
 
 // P.V on the packed values with P' = p' * s_v split into hi + lo.  Branch-free.
-template <int D, int PATH, int TPW>
+template <int D, int PATH, int FMT, int TPW>
 __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gid,
                                         const int (&rho)[4], const float (&p)[TPW][4],
                                         const float (&sv)[TPW][4][D / 32],
-                                        WarpState<D, PATH>& st) {
-  using C = Cfg<D, PATH>;
-  constexpr int NG = C::NG, RB = C::RB, SB = C::SB;
+                                        WarpState<D, PATH, FMT>& st) {
+  using C = Cfg<D, PATH, FMT>;
+  constexpr int NG = C::NG, RB = C::RB, SB = 2 * NG;  // SB: bytes of one of a row's 8 sub-blocks
   const unsigned char* vc = stg + C::VC + r0 * RB;
 #pragma unroll
   for (int u = 0; u < TPW; ++u) {
@@ -795,29 +879,108 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
   }
 }
 
+// Codebook P.V (heads on rows): as tile_pv with the B operand the levels of
+// coordinates 32g + 4 gid + e (n-tile e) of the token pairs (rho0, rho1) and
+// (rho2, rho3), hi and lo parts from the level-pair table, both products in
+// the same accumulator.  Branch-free.
+template <int D, int PATH, int FMT, int TPW>
+__device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int gid,
+                                           const int (&rho)[4], const float (&p)[TPW][4],
+                                           const float (&sv)[TPW][4][D / 32],
+                                           WarpState<D, PATH, FMT>& st, const unsigned char* lutp) {
+  using C = Cfg<D, PATH, FMT>;
+  constexpr int NG = C::NG, RB = C::RB, GB = 4 * FMT;  // GB: bytes per group
+  constexpr uint32_t M = (1u << FMT) - 1;
+  const unsigned char* vc = stg + C::VC + r0 * RB;
+  const int bo = 4 * FMT * gid;  // bit offset of this thread's 4 indices in a group
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+    uint32_t f[2][NG];  // per token pair: indices of row rho[2j] | those of rho[2j + 1] << 16
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        uint32_t v[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const unsigned char* rp = vc + (16 * u + rho[2 * j + r]) * RB + g * GB;
+          if (FMT == 2) {
+            v[r] = rp[gid];
+          } else if (FMT == 4) {
+            v[r] = reinterpret_cast<const uint16_t*>(rp)[gid];
+          } else {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(rp) + (bo >> 5);
+            v[r] = __funnelshift_r(w[0], w[1], bo & 31) & 0xFFFu;
+          }
+        }
+        f[j][g] = v[0] | (v[1] << 16);
+      }
+#pragma unroll
+    for (int gp = 0; gp < NG; gp += 2) {
+      float wh[4][2], wl[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __fmul2_rn(make_float2(p[u][i], p[u][i]),
+                                    make_float2(sv[u][i][gp], sv[u][i][gp + 1]));
+        const float2 h = make_float2(split_hi(x.x), split_hi(x.y));
+        const float2 l = __ffma2_rn(h, make_float2(-1.0f, -1.0f), x);  // exact
+        wh[i][0] = h.x;
+        wh[i][1] = h.y;
+        wl[i][0] = l.x;
+        wl[i][1] = l.y;
+      }
+#pragma unroll
+      for (int eg = 0; eg < 2; ++eg) {
+        const int g = gp + eg;
+        const uint32_t a0 = f16x2(wh[0][eg], wh[1][eg]), a1 = f16x2(wl[0][eg], wl[1][eg]);
+        const uint32_t a2 = f16x2(wh[2][eg], wh[3][eg]), a3 = f16x2(wl[2][eg], wl[3][eg]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint2 b[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t t = f[j][g];
+            const uint32_t key = ((t >> (FMT * e)) & M) | (((t >> (16 + FMT * e)) & M) << FMT);
+            b[j] = *reinterpret_cast<const uint2*>(lutp + (key << 3));
+          }
+          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, b[0].x, b[1].x);
+          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, b[0].y, b[1].y);
+        }
+      }
+    }
+  }
+}
+
 // One warp's share of a stage: scores, softmax update and P.V of its TPW tiles
 // (rows r0 .. r0 + 16 TPW - 1, of which the first nvalid are real tokens).
-template <int D, int PATH, int TPW, bool FULL>
+template <int D, int PATH, int FMT, int TPW, bool FULL>
 __device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, int nvalid, int gid,
                                             int tig, const int (&rho)[4], const int (&krow)[2],
-                                            WarpState<D, PATH>& st) {
+                                            WarpState<D, PATH, FMT>& st,
+                                            const unsigned char* lutp) {
   float S[TPW][4], p[TPW][4], sv[TPW][4][D / 32];
-  tile_scores<D, PATH, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
-  tile_max<D, PATH, TPW>(tig, S, st);
-  load_vscales<D, PATH, TPW, FULL>(stg, r0, nvalid, rho, sv);
-  tile_weights<D, PATH, TPW>(S, sv, st, p);
-  tile_pv<D, PATH, TPW>(stg, r0, gid, rho, p, sv, st);
+  if constexpr (FMT == 0)
+    tile_scores<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
+  else
+    tile_scores_cb<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, lutp, S);
+  tile_max<D, PATH, FMT, TPW>(tig, S, st);
+  load_vscales<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, rho, sv);
+  tile_weights<D, PATH, FMT, TPW>(S, sv, st, p);
+  if constexpr (FMT == 0)
+    tile_pv<D, PATH, FMT, TPW>(stg, r0, gid, rho, p, sv, st);
+  else
+    tile_pv_cb<D, PATH, FMT, TPW>(stg, r0, gid, rho, p, sv, st, lutp);
 }
 
 // End of an item: the warps' (max, sum, acc) per head are merged in shared
 // memory and written as the item's split-K partial (max reported as m + F,
 // with sum and acc scaled by 2^-F).  If the pipeline gave up, the partial's
 // max is NaN, so the decode's output for these heads is NaN.
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* smem,
-                                            const WarpState<D, PATH>& st, int b, int kvh, int c,
+                                            const WarpState<D, PATH, FMT>& st, int b, int kvh, int c,
                                             bool aborted) {
-  using C = Cfg<D, PATH>;
+  using C = Cfg<D, PATH, FMT>;
   constexpr int NH = C::NH, NG = C::NG, NW = C::NW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -838,12 +1001,13 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
       ml[warp * NH + gid] = l;
     }
     float* dst = macc + (warp * NH + gid) * D;
+    const float ce = FMT ? st.cexp : 1.0f;  // codebook: the levels' normalisation
 #pragma unroll
     for (int g = 0; g < NG; ++g)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        dst[32 * g + 8 * tig + cc] = st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2];
-        dst[32 * g + 8 * tig + 4 + cc] = st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3];
+        dst[32 * g + 8 * tig + cc] = (st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2]) * ce;
+        dst[32 * g + 8 * tig + 4 + cc] = (st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3]) * ce;
       }
   } else {
     if (tig == 0 && (gid & 1) == 0) {
@@ -894,9 +1058,9 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
   }
 }
 
-template <int D, int PATH>
-__global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(DecodeArgs a) {
-  using C = Cfg<D, PATH>;
+template <int D, int PATH, int FMT>
+__global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kernel(DecodeArgs a) {
+  using C = Cfg<D, PATH, FMT>;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR);
   int* cnt = reinterpret_cast<int*>(smem + C::CNT);
@@ -952,6 +1116,29 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
     cur[6] = pfx != nullptr ? pfx[a.B] : a.B * a.Hkv * a.plan.n_chunks;
     cur[7] = pfx != nullptr;
   }
+  // Codebook: the level-pair table, the levels normalised by 2^-e so that the
+  // largest magnitude lies in [0.5, 1) (exact; 2^e is put back on the scores
+  // and the output): entry i0 | i1 << FMT = (C[i0], C[i1]) as f16x2 hi parts
+  // (round to nearest) and f16x2 lo parts (the remainders, rounded).
+  float cexp = 1.0f;
+  if constexpr (FMT != 0) {
+    constexpr int L = 1 << FMT;
+    float lmax = 0.0f;
+    for (int i = 0; i < L; ++i) lmax = fmaxf(lmax, fabsf(a.levels[i]));
+    int e = 0;
+    if (lmax > 0.0f) frexpf(lmax, &e);
+    cexp = ldexpf(1.0f, e);
+    uint2* lut = reinterpret_cast<uint2*>(smem + C::LUT);
+    for (int key = threadIdx.x; key < L * L; key += C::THREADS) {
+      const float c0 = ldexpf(a.levels[key & (L - 1)], -e), c1 = ldexpf(a.levels[key >> FMT], -e);
+      const __half h0 = __float2half_rn(c0), h1 = __float2half_rn(c1);
+      const __half l0 = __float2half_rn(c0 - __half2float(h0));
+      const __half l1 = __float2half_rn(c1 - __half2float(h1));
+      lut[key] = make_uint2((uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16),
+                            (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16));
+    }
+  }
+  const unsigned char* lutp = smem + C::LUT;
   __syncthreads();
 
   // Fused append: for every (sequence, kv head) whose last chunk is one of this
@@ -961,7 +1148,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   // generic writes before the bulk copies, which the last warp issues only
   // after named barrier 2 (both warps arrive here exactly once).
   static_assert(C::NW == 8, "the fused append uses warps 4, 5 and 7");
-  if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
+  if (FMT == 0 && a.k_new != nullptr && (warp == 4 || warp == 5)) {
     const bool isv = warp == 5;
     const int eb = a.kv_bf16 ? 2 : 4;
     for (int it = blockIdx.x; it < cur[6]; it += gridDim.x) {
@@ -983,7 +1170,8 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   const int rho[4] = {slot_row(2 * tig), slot_row(2 * tig + 1), 8 + slot_row(2 * tig),
                       8 + slot_row(2 * tig + 1)};
   const int krow[2] = {slot_row(gid), 8 + slot_row(gid)};
-  WarpState<D, PATH> st;
+  WarpState<D, PATH, FMT> st;
+  st.cexp = cexp;
   uint32_t sc = 0;  // stages consumed so far
   for (int it = blockIdx.x; it < cur[6]; it += gridDim.x) {
     int b, kvh, c, t0, t1;
@@ -994,7 +1182,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
       const int raw = a.ctx_lens[b];
       static_cast<int32_t*>(a.workspace)[b] = (raw < 1 || raw > a.max_ctx) ? 1 : 0;
     }
-    prep_query<D, PATH>(a, b, kvh, smem, st, sc == 0, cur, full);
+    prep_query<D, PATH, FMT>(a, b, kvh, smem, st, sc == 0, cur, full);
 #pragma unroll
     for (int j = 0; j < C::NACC; ++j)
 #pragma unroll
@@ -1011,20 +1199,20 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
       mbar_wait(full + slot, (sc / C::NS) & 1, abort);
       const int nv = min(C::ST, t1 - t0 - k * C::ST) - r0;  // real rows from r0 on
       if (nv >= 16 * C::TPW)
-        stage_tiles<D, PATH, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st);
+        stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
       else if (nv > 0)
-        stage_tiles<D, PATH, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st);
+        stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
       __syncwarp();
       if (lane == 0) {  // the last warp out of the stage refills it
         __threadfence_block();
         if (atomicAdd(cnt + slot, 1) == C::NW - 1) {
           cnt[slot] = 0;
           __threadfence_block();
-          if (!*abort) issue_next<D, PATH>(a, smem, cur, full, slot);
+          if (!*abort) issue_next<D, PATH, FMT>(a, smem, cur, full, slot);
         }
       }
     }
-    finish_item<D, PATH>(a, smem, st, b, kvh, c, *abort != 0);
+    finish_item<D, PATH, FMT>(a, smem, st, b, kvh, c, *abort != 0);
   }
   if (threadIdx.x == 0 && *abort) {  // copies still in flight must land before exit
     const uint32_t issued = (uint32_t)cur[5];
@@ -1033,11 +1221,11 @@ __global__ void __launch_bounds__(Cfg<D, PATH>::THREADS, 1) decode_mma_kernel(De
   }
 }
 
-template <int D, int PATH>
+template <int D, int PATH, int FMT>
 cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
-  using C = Cfg<D, PATH>;
+  using C = Cfg<D, PATH, FMT>;
   static std::atomic<uint64_t> smem_set{0};
-  const cudaError_t e = ensure_smem_limit(decode_mma_kernel<D, PATH>, C::BYTES, smem_set);
+  const cudaError_t e = ensure_smem_limit(decode_mma_kernel<D, PATH, FMT>, C::BYTES, smem_set);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kSmCount;
   cudaGetDevice(&dev);
@@ -1055,9 +1243,9 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<D, PATH>, a);
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<D, PATH, FMT>, a);
   }
-  decode_mma_kernel<D, PATH><<<grid, C::THREADS, C::BYTES, stream>>>(a);
+  decode_mma_kernel<D, PATH, FMT><<<grid, C::THREADS, C::BYTES, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -1067,16 +1255,27 @@ bool decode_mma_supported(int d, int G) {
   return (d == 128 && G >= 1 && G <= 8) || (d == 256 && G >= 1 && G <= 4);
 }
 
+bool decode_mma_cb_supported(int d, int G) { return d == 128 && G >= 5 && G <= 8; }
+
 int decode_stage_tokens(int d, int G) {
   if (!decode_mma_supported(d, G)) return 128;
-  return d == 128 ? Cfg<128, 0>::ST : Cfg<256, 1>::ST;
+  return d == 128 ? Cfg<128, 0, 0>::ST : Cfg<256, 1, 0>::ST;
 }
 
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
-  if (a.d == 128 && G >= 5 && G <= 8) return launch_mma<128, 0>(a, stream);
-  if (a.d == 128 && G >= 1 && G <= 4) return launch_mma<128, 1>(a, stream);
-  if (a.d == 256 && G >= 1 && G <= 4) return launch_mma<256, 1>(a, stream);
+  if (a.cb_bits != 0) {
+    if (!decode_mma_cb_supported(a.d, G)) return cudaErrorNotSupported;
+    switch (a.cb_bits) {
+      case 2: return launch_mma<128, 0, 2>(a, stream);
+      case 3: return launch_mma<128, 0, 3>(a, stream);
+      case 4: return launch_mma<128, 0, 4>(a, stream);
+      default: return cudaErrorNotSupported;
+    }
+  }
+  if (a.d == 128 && G >= 5 && G <= 8) return launch_mma<128, 0, 0>(a, stream);
+  if (a.d == 128 && G >= 1 && G <= 4) return launch_mma<128, 1, 0>(a, stream);
+  if (a.d == 256 && G >= 1 && G <= 4) return launch_mma<256, 1, 0>(a, stream);
   return cudaErrorNotSupported;
 }
 

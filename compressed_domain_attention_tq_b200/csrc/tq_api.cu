@@ -25,7 +25,8 @@ bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* pl
   const bool srft = kind == PlanKind::kSrft;
   if (srft ? !srft_head_dim_supported(d) : (d != 128 && d != 256)) return false;
   const int64_t units = (int64_t)B * Hkv;
-  const bool mma = kind != PlanKind::kCodebook && decode_mma_supported(d, Hq / Hkv);
+  const bool mma = kind == PlanKind::kCodebook ? decode_mma_cb_supported(d, Hq / Hkv)
+                                              : decode_mma_supported(d, Hq / Hkv);
   const int64_t step = mma ? decode_stage_tokens(d, Hq / Hkv) : 128, per_item_cost = mma ? 384 : 256;
   const int64_t slots = mma ? kSmCount : 4 * kSmCount;
   const int64_t max_n = ceil_div(max_ctx, step);
@@ -323,8 +324,9 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
                                                       a.plan.qrot_offset)
                      : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const bool mma = rot.cb_bits == 0 && decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
-  if (append && mma && !rot.srft) {  // the decode kernel quantizes the new tokens itself
+  const bool mma = rot.cb_bits ? decode_mma_cb_supported(head_dim, num_q_heads / num_kv_heads)
+                               : decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
+  if (append && mma && !rot.srft && !rot.cb_bits) {  // the decode kernel quantizes the new tokens itself
     a.k_new = k_new;
     a.v_new = v_new;
   } else if (append && rot.srft) {  // new tokens and query rotation in one launch
@@ -350,7 +352,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     const cudaError_t e = launch_srft_prep(qa, a, s);
     if (e != cudaSuccess) return cuda_status(e, where);
     a.q_rot_overlap = 2;
-  } else if (append) {  // the CUDA-core decode: one small-append launch first
+  } else if (append) {  // the CUDA-core or codebook decode: one small-append launch first
     QuantizeArgs qa;
     qa.k = k_new;
     qa.v = v_new;

@@ -111,6 +111,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 bool decode_mma_supported(int d, int G);
+bool decode_mma_cb_supported(int d, int G);  // codebook caches on the tensor-core decode
 int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);

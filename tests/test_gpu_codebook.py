@@ -137,6 +137,47 @@ def test_cb_decode_matches_oracle(bits, B, Hkv, G, d, ctx):
     check_attention_cb(got, want, cache, ctx, G, bits, lv, f"cb{bits} B={B} Hkv={Hkv} G={G} d={d}")
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("G", [5, 6, 7, 8])
+def test_cb_tensor_core_decode_ragged_batch(bits, G):
+    """The tensor-core codebook decode (5..8 query heads per kv head, d = 128):
+    two sequences of different lengths, each over several 256-token stages and
+    split-K chunks, with ragged tails and (G < 8) padding heads."""
+    require_cuda()
+    B, Hkv, d, ctx = 2, 2, 128, [3001, 517]
+    seed = 300 + 10 * bits + G
+    T = max(ctx)
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, seed, heavy=True)
+    signs = signs_for(d, seed + 1)
+    lv = levels_for(bits)
+    cache = oracle_cb_cache(k, v, signs, bits, lv)
+    got = cb_decode(upload_cache(cache), q, ctx, T, signs, bits, lv, 1 / math.sqrt(d), Hkv)
+    want = oracle.sdpa_cb_decode(to_oracle(q), cache, ctx, signs.numpy(), bits, lv.numpy(),
+                                 1 / math.sqrt(d), Hkv, threads=THREADS)
+    check_attention_cb(got, want, cache, ctx, G, bits, lv, f"cb{bits} G={G} ragged")
+
+
+@pytest.mark.parametrize("bits,mul,off", [(2, 1e3, 0.3), (3, 1e-3, -0.2), (4, 37.0, 0.05)])
+def test_cb_tensor_core_decode_custom_levels(bits, mul, off):
+    """Levels other than the Gaussian codebook: asymmetric and far from 1 in
+    magnitude (the tensor-core decode normalises them by a power of two before
+    splitting them into f16 parts), at attn_scale 1.0 and 1/sqrt(d)."""
+    require_cuda()
+    B, Hkv, G, d, T = 1, 2, 8, 128, 1200
+    seed = 400 + bits
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, seed)
+    signs = signs_for(d, seed + 1)
+    lv = ((levels_for(bits).double() + off) * mul).float()
+    assert torch.all(lv[1:] > lv[:-1])
+    cache = oracle_cb_cache(k, v, signs, bits, lv)
+    for scale in (1 / math.sqrt(d), 1.0):
+        got = cb_decode(upload_cache(cache), q, [T], T, signs, bits, lv, scale, Hkv)
+        want = oracle.sdpa_cb_decode(to_oracle(q), cache, [T], signs.numpy(), bits, lv.numpy(),
+                                     scale, Hkv, threads=THREADS)
+        check_attention_cb(got, want, cache, [T], G, bits, lv,
+                           f"cb{bits} levels x{mul}+{off} scale={scale:.3g}")
+
+
 def test_cb_decode_rotation_off_fp32_query_attn_scale_one():
     require_cuda()
     B, Hkv, G, d, T, bits = 1, 2, 2, 128, 700, 3
