@@ -395,8 +395,12 @@ TQ_API tq_status tq_sdpa_int4_decode_append_srft(
  *    on the device; the host checks only the pointer, 4-byte aligned).
  * head_dim 128 or 256; bits 2, 3 or 4 (else TQ_ERR_UNSUPPORTED); every other
  * argument, alignment rule and error is that of the int4 calls.  The decode
- * runs on CUDA cores; with 2 bits its scores read tables of 16 partial dot
- * products per pair of query coordinates (the post's lookup tables).
+ * runs on the tensor cores for head_dim 128 with 5..8 query heads per kv head
+ * (levels as f16 hi + lo parts read from a table over index pairs), on CUDA
+ * cores otherwise (with 2 bits its scores there read tables of 16 partial dot
+ * products per pair of query coordinates: the post's lookup tables).  Levels
+ * of any finite magnitude are accepted: the tensor-core decode scales them by
+ * a power of two before splitting them.
  */
 
 /* The Gaussian Max-Lloyd codebook of 2^bits levels (N(0,1) cell means at
