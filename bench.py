@@ -70,7 +70,7 @@ def kv_bytes(w, ctx_tokens):
 # Sources that determine each profiled kernel's code and launch shape; a
 # committed DRAM-traffic figure counts only while their hash is unchanged.
 KERNEL_SOURCES = {
-    "decode": ["decode_mma.cu", "quantize_vector.cuh", "tq_internal.h", "tq_api.cu"],
+    "decode": ["decode_mma.cu", "quantize_vector.cuh", "cb_vector.cuh", "tq_internal.h", "tq_api.cu"],
     "quantize_bulk": ["quantize.cu", "quantize_vector.cuh", "tq_internal.h", "tq_api.cu"],
 }
 
@@ -364,7 +364,13 @@ def run_tq(args):
 
     kvb = kv_bytes(w, (ctx + 1).tolist())
     mma = not w.cb_bits and ((d == 128 and Hq // Hkv <= 8) or (d == 256 and Hq // Hkv <= 4))
-    if w.cb_bits:
+    mma_cb = bool(w.cb_bits) and d == 128 and 5 <= Hq // Hkv <= 8
+    if mma_cb:
+        launches_per_step = 2
+        step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): the tensor-core "
+                     "decode kernel quantizes the new token of each kv head into the cache, then "
+                     "attends (split-K kernel + merge, 2 launches)")
+    elif w.cb_bits:
         launches_per_step = 3
         step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): quantize-append "
                      "of the new token, split-K decode, merge (3 launches)")

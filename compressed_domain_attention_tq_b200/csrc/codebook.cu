@@ -9,13 +9,14 @@
 // 4 * bits bytes; index j of a group occupies bits bits*j .. bits*j + bits - 1
 // of the group's little-endian bit string.
 //
-// Here: the quantize-append kernel (one warp per vector, Hadamard rotation as
-// in the int4 path) and the host-side Gaussian Max-Lloyd generator.  The
-// decode is decode_simt.cu's kernel instantiated for the codebook formats.
+// Here: the quantize-append kernel (one warp per vector: cb_vector.cuh) and the
+// host-side Gaussian Max-Lloyd generator.  The decode is decode_mma.cu's
+// tensor-core kernel (5..8 query heads per kv head, d = 128) or decode_simt.cu's
+// kernel, both instantiated for the codebook formats.
 #include <math.h>
 #include <stdint.h>
 
-#include "quantize_vector.cuh"
+#include "cb_vector.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -23,9 +24,6 @@ namespace {
 
 template <int D, int BITS>
 __global__ void __launch_bounds__(128) cb_quantize_kernel(QuantizeArgs a) {
-  constexpr int E = D / 32;   // coordinates per lane (E consecutive ones)
-  constexpr int GL = 32 / E;  // lanes per group
-  constexpr int L = 1 << BITS;
   const int lane = threadIdx.x & 31;
   const int64_t per_kv = (int64_t)a.B * a.Hkv * a.n_new;
   const int64_t vec = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -38,50 +36,11 @@ __global__ void __launch_bounds__(128) cb_quantize_kernel(QuantizeArgs a) {
   if (a.pos_is_ctx) p = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
   if (p < 0 || p >= a.capacity) return;  // the whole warp
   const int64_t row = bh * a.capacity + p;
-
-  float t[L - 1];  // thresholds between adjacent levels
-#pragma unroll
-  for (int i = 0; i + 1 < L; ++i) t[i] = __fmul_rn(__fadd_rn(a.levels[i], a.levels[i + 1]), 0.5f);
-
-  float x[E];
   const int eb = a.bf16 ? 2 : 4;
-  load_vector_warp<D>(static_cast<const unsigned char*>(kv ? a.v : a.k) + rem * D * eb, a.bf16, x, lane);
-  rotate_vector_warp<D>(x, a.signs, lane);
-
-  // the group's sum of squares in fp64: this lane's E, then the group's GL lanes
-  double S = 0.0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) S += (double)x[e] * (double)x[e];
-#pragma unroll
-  for (int o = 1; o < GL; o <<= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-  const float sigma = (float)sqrt(S / 32.0);
-
-  // indices of this lane's E coordinates, packed at bit BITS * j0 of the group
-  uint32_t bits = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float u = sigma > 0.0f ? __fdiv_rn(x[e], sigma) : 0.0f;
-    u = fminf(fmaxf(u, -3.0f), 3.0f);
-    uint32_t k = 0;
-#pragma unroll
-    for (int i = 0; i + 1 < L; ++i) k += u > t[i] ? 1u : 0u;
-    bits |= k << (BITS * e);
-  }
-  const int g = lane / GL, j0 = E * (lane % GL);
-  const int off = BITS * j0;  // bit offset of this lane's indices in the group
-  uint32_t* prow = reinterpret_cast<uint32_t*>((kv ? a.v_packed : a.k_packed) + row * (D * BITS / 8));
-  const uint64_t wide = bits;
-#pragma unroll
-  for (int w = 0; w < BITS; ++w) {  // the group's BITS words
-    const int sh = off - 32 * w;
-    uint32_t c = 0;
-    if (sh >= 0 && sh < 32) c = (uint32_t)(wide << sh);
-    else if (sh < 0 && sh > -32) c = (uint32_t)(wide >> -sh);
-#pragma unroll
-    for (int o = 1; o < GL; o <<= 1) c |= __shfl_xor_sync(0xffffffffu, c, o);
-    if (lane % GL == w) prow[BITS * g + w] = c;
-  }
-  if (lane % GL == 0) ((kv ? a.v_scales : a.k_scales) + row * (D / 32))[g] = sigma;
+  cb_quantize_vector_warp<D, BITS>(static_cast<const unsigned char*>(kv ? a.v : a.k) + rem * D * eb,
+                                   a.bf16, a.signs, a.levels,
+                                   (kv ? a.v_packed : a.k_packed) + row * (D * BITS / 8),
+                                   (kv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
 }
 
 template <int D, int BITS>

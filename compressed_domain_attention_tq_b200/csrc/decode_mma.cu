@@ -49,6 +49,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "cb_vector.cuh"
 #include "quantize_vector.cuh"
 #include "tq_internal.h"
 
@@ -1148,7 +1149,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
   // generic writes before the bulk copies, which the last warp issues only
   // after named barrier 2 (both warps arrive here exactly once).
   static_assert(C::NW == 8, "the fused append uses warps 4, 5 and 7");
-  if (FMT == 0 && a.k_new != nullptr && (warp == 4 || warp == 5)) {
+  if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
     const bool isv = warp == 5;
     const int eb = a.kv_bf16 ? 2 : 4;
     for (int it = blockIdx.x; it < cur[6]; it += gridDim.x) {
@@ -1157,10 +1158,13 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       if (t1 != clamp_ctx_mma(a.ctx_lens[b], a.max_ctx)) continue;  // not the last chunk
       const int64_t bh = (int64_t)b * a.Hkv + kvh;
       const int64_t row = bh * a.capacity + (t1 - 1);
-      quantize_vector_warp<D>(static_cast<const unsigned char*>(isv ? a.v_new : a.k_new) + bh * D * eb,
-                              a.kv_bf16, a.signs,
-                              const_cast<uint8_t*>(isv ? a.v_packed : a.k_packed) + row * (D / 2),
-                              const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
+      const unsigned char* src = static_cast<const unsigned char*>(isv ? a.v_new : a.k_new) + bh * D * eb;
+      uint8_t* prow = const_cast<uint8_t*>(isv ? a.v_packed : a.k_packed) + row * C::RB;
+      float* srow = const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32);
+      if constexpr (FMT == 0)
+        quantize_vector_warp<D>(src, a.kv_bf16, a.signs, prow, srow, lane);
+      else
+        cb_quantize_vector_warp<D, FMT>(src, a.kv_bf16, a.signs, a.levels, prow, srow, lane);
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
     asm volatile("bar.arrive 2, 96;" ::: "memory");

@@ -326,7 +326,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const bool mma = rot.cb_bits ? decode_mma_cb_supported(head_dim, num_q_heads / num_kv_heads)
                                : decode_mma_supported(head_dim, num_q_heads / num_kv_heads);
-  if (append && mma && !rot.srft && !rot.cb_bits) {  // the decode kernel quantizes the new tokens itself
+  if (append && mma && !rot.srft) {  // the decode kernel quantizes the new tokens itself
     a.k_new = k_new;
     a.v_new = v_new;
   } else if (append && rot.srft) {  // new tokens and query rotation in one launch
@@ -352,7 +352,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     const cudaError_t e = launch_srft_prep(qa, a, s);
     if (e != cudaSuccess) return cuda_status(e, where);
     a.q_rot_overlap = 2;
-  } else if (append) {  // the CUDA-core or codebook decode: one small-append launch first
+  } else if (append) {  // the CUDA-core decode: one small-append launch first
     QuantizeArgs qa;
     qa.k = k_new;
     qa.v = v_new;

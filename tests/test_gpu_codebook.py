@@ -217,3 +217,42 @@ def test_cb_engine_step_and_determinism():
     want = oracle.sdpa_cb_decode(to_oracle(q), cache, [T], signs.numpy(), bits, c.levels.cpu().numpy(),
                                  1 / math.sqrt(d), Hkv, threads=THREADS)
     check_attention_cb(outs[0], want, cache, [T], G, bits, c.levels.cpu(), "cb engine")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_cb_fused_step_ragged_batch(bits):
+    """decode_append on the tensor-core codebook path (the decode kernel
+    quantizes each sequence's new token into row ctx - 1 itself): two
+    sequences of different lengths, 6 query heads per kv head.  Bit-identical
+    to append-then-decode, and the oracle agrees on the resulting cache."""
+    require_cuda()
+    B, Hkv, G, d, ctx = 2, 2, 6, 128, [1800, 333]
+    T = max(ctx)
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 500 + bits)
+    signs = signs_for(d, 501 + bits)
+    ct = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    kn = torch.stack([k[b, :, ctx[b] - 1] for b in range(B)])[:, :, None].contiguous().cuda()
+    vn = torch.stack([v[b, :, ctx[b] - 1] for b in range(B)])[:, :, None].contiguous().cuda()
+    outs, caches = [], []
+    for fused in (True, False):
+        c = CodebookKVCache(B, Hkv, d, T, bits, signs=signs)
+        c.append(k.cuda(), v.cuda(), torch.zeros(B, dtype=torch.int32, device="cuda"))
+        for b in range(B):  # rows ctx - 1 .. hold stale data the step must overwrite
+            c.k_packed[b, :, ctx[b] - 1:].fill_(0x5A)
+            c.v_packed[b, :, ctx[b] - 1:].fill_(0xA5)
+        if fused:
+            out = c.decode_append(q.cuda(), kn, vn, ct, T)
+        else:
+            c.append(kn, vn, ct - 1)
+            out = c.decode(q.cuda(), ct, T)
+        torch.cuda.synchronize()
+        outs.append(out.cpu().numpy())
+        caches.append([t.cpu().numpy() for t in (c.k_packed, c.k_scales, c.v_packed, c.v_scales)])
+    np.testing.assert_array_equal(outs[0], outs[1])
+    for b in range(B):
+        for a0, a1 in zip(caches[0], caches[1]):
+            np.testing.assert_array_equal(a0[b, :, :ctx[b]], a1[b, :, :ctx[b]])
+    lv = c.levels.cpu()
+    want = oracle.sdpa_cb_decode(to_oracle(q), caches[0], ctx, signs.numpy(), bits, lv.numpy(),
+                                 1 / math.sqrt(d), Hkv, threads=THREADS)
+    check_attention_cb(outs[0], want, caches[0], ctx, G, bits, lv, f"cb{bits} fused step")
