@@ -13,7 +13,8 @@
 //   srft_quantize_kernel  one warp per (sequence, kv head, token): K and V of
 //                         the token form one complex transform; then group
 //                         abs-max, int4 codes and the packed row layout of the
-//                         Hadamard path.
+//                         Hadamard path.  For d = 128 and 256 the team kernel
+//                         (srft_team.cuh: d / 16 lanes per token) does the same.
 //   srft_query_kernel     one warp per pair of query heads -> q_r (fp32) in the
 //                         decode workspace; the decode kernels read it instead
 //                         of rotating q themselves.
@@ -27,12 +28,14 @@
 #include <stdint.h>
 
 #include "srft.cuh"
+#include "srft_team.cuh"
 #include "tq_internal.h"
 
 namespace tq {
 namespace {
 
 constexpr int kQWarps = 8;  // warps per quantize CTA
+constexpr int kTeamMinTokens = 64;  // appends of at least this many tokens per row use the team kernel
 constexpr float kRneMagic = 12582912.0f;                   // 1.5 * 2^23: x + M rounds x to an integer
 constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21 (exact)
 constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21 (exact)
@@ -147,6 +150,193 @@ __global__ void __launch_bounds__(32 * kQWarps) srft_quantize_kernel(QuantizeArg
   const int pairs = a.B * a.Hkv * a.n_new;  // < 2^31 (checked on the host)
   for (int p = blockIdx.x * kQWarps + warp; p < pairs; p += gridDim.x * kQWarps)
     srft_quantize_pair<M>(a, p, tw, lc, ybuf[warp][0], ybuf[warp][1], lane);
+}
+
+// Per-CTA tables of the team quantizer: signs (+-1) and lambda / (2 sqrt d).
+template <int D>
+struct TeamTables {
+  float sgn[D], lk[D], lv[D];
+  __device__ __forceinline__ void build(const QuantizeArgs& a) {
+    const float norm = 0.5f / sqrtf((float)D);
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      sgn[i] = a.signs ? (float)a.signs[i] : 1.0f;
+      lk[i] = a.lambda_k ? norm * a.lambda_k[i] : norm;
+      lv[i] = a.lambda_v ? norm * a.lambda_v[i] : norm;
+    }
+  }
+};
+
+// Cache row of vector pair p ((sequence, kv head) row-major, then token), or
+// false when its position is outside the cache.
+__device__ __forceinline__ bool team_pair_row(const QuantizeArgs& a, int p, int64_t& row) {
+  const int bh = p / a.n_new, n = p - bh * a.n_new;
+  const int b = bh / a.Hkv;
+  int64_t pos = (int64_t)a.pos[b] + n;
+  if (a.pos_is_ctx) pos = (int64_t)min(max(a.pos[b], 1), a.max_ctx) - 1 + n;
+  row = (int64_t)bh * a.capacity + pos;
+  return pos >= 0 && pos < a.capacity;
+}
+
+// Team lane t (of P) quantizes one vector pair from re = sigma (.) k and
+// im = sigma (.) v at j = t + P j2 into cache row `row` (stores only if ok;
+// a team without a pair still takes part in the shuffles).  After the
+// transform the lane owns coordinates 16 k1 .. 16 k1 + 15 (k1 = brev(t)):
+// half of group k1 / 2, whose other half is in lane t ^ P/2; its codes are
+// four half-words of the packed row, at byte (j / 4) * 2 ng + 2 g for the
+// in-group coordinates j = 16 (k1 % 2) + 4 q .. 4 q + 3.
+template <int P>
+__device__ __forceinline__ void srft_quantize_team(const QuantizeArgs& a, int64_t row, bool ok,
+                                                   const float (&re)[16], const float (&im)[16],
+                                                   const TeamConsts<P>& c,
+                                                   const TeamTables<16 * P>& tb, int t,
+                                                   int team_base) {
+  constexpr int D = 16 * P, NG = D / 32, L = TeamConsts<P>::L;
+  float hx[16], hy[16];
+  hartley_pair_team<P>(re, im, c, team_base, hx, hy);
+  const int k1 = brev_bits<L>(t), g = k1 >> 1, half = k1 & 1;
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    const float* lam = (kv ? tb.lv : tb.lk) + 16 * k1;
+    const float* h = kv ? hy : hx;
+    float y[16];  // coordinate 16 k1 + k2 in y[k2]
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 l = reinterpret_cast<const float4*>(lam)[q];
+      y[4 * q] = h[brev4c(4 * q)] * l.x;
+      y[4 * q + 1] = h[brev4c(4 * q + 1)] * l.y;
+      y[4 * q + 2] = h[brev4c(4 * q + 2)] * l.z;
+      y[4 * q + 3] = h[brev4c(4 * q + 3)] * l.w;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int k2 = 0; k2 < 16; ++k2) amax = fmaxf(amax, fabsf(y[k2]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, P / 2));
+    const float s = __fdiv_rn(amax, 7.0f);
+    const float r = s > 0.0f ? __frcp_rn(s) : 0.0f;
+    // int4_code's bracketed reciprocals, unrolled: where both brackets give the
+    // same integer, x * r_lo + 1.5 * 2^23 has the bits 0x4B400000 + c, so its
+    // low nibble is the code's two's complement (|x / s| <= 7, so no clamp
+    // binds); if any of the lane's 16 disagree (or s is subnormal) the lane
+    // redoes them with the IEEE division, as int4_code does
+    const float rl = r * kBracketLo, rh = r * kBracketHi;
+    bool slow = !(r <= 3.0e38f);
+    uint32_t hw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      hw[q] = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = fmaf(y[4 * q + e], rl, kRneMagic), hi = fmaf(y[4 * q + e], rh, kRneMagic);
+        slow |= lo != hi;
+        hw[q] |= (__float_as_uint(lo) & 0xFu) << (4 * e);
+      }
+    }
+    if (slow) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        hw[q] = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float cc =
+              s > 0.0f ? fminf(fmaxf(rintf(__fdiv_rn(y[4 * q + e], s)), -7.0f), 7.0f) : 0.0f;
+          hw[q] |= (__float_as_uint(cc + kRneMagic) & 0xFu) << (4 * e);
+        }
+      }
+    }
+    uint8_t* prow = (kv ? a.v_packed : a.k_packed) + row * (D / 2);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (ok) *reinterpret_cast<uint16_t*>(prow + (4 * half + q) * 2 * NG + 2 * g) = (uint16_t)hw[q];
+    if (ok && half == 0) ((kv ? a.v_scales : a.k_scales) + row * NG)[g] = s;
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
+// Bulk quantize-append for d = 16 P: each warp takes 32 / P pairs per step,
+// grid-stride.  bf16 inputs are staged in shared memory by 16-byte async
+// copies one step ahead (two buffers per warp; a pair's K and V rows at a
+// pitch of 4 d + 16 bytes, so the teams' 2-byte reads fall in distinct
+// banks); fp32 inputs are loaded directly.
+template <int P>
+__global__ void __launch_bounds__(256) srft_quantize_team_kernel(QuantizeArgs a) {
+  constexpr int D = 16 * P, TPW = 32 / P;
+  constexpr int PITCH = 4 * D + 16;           // bytes per staged pair (bf16 K row, V row, pad)
+  constexpr int CHUNKS = TPW * (4 * D / 16);  // 16-byte copies per warp step (= 128)
+  static_assert(CHUNKS == 128, "four copies per lane");
+  __shared__ __align__(16) TeamTables<D> tb;
+  __shared__ __align__(16) unsigned char stage[8][2][TPW * PITCH];
+  tb.build(a);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = lane & (P - 1), team_base = lane & ~(P - 1), q = lane / P;
+  TeamConsts<P> c;
+  team_consts<P>(c, t);
+  const int pairs = a.B * a.Hkv * a.n_new;  // < 2^31 (checked on the host)
+  const int stride = gridDim.x * 8 * TPW;
+  const int base0 = (blockIdx.x * 8 + warp) * TPW;
+  if (!a.bf16) {
+    for (int base = base0; base < pairs; base += stride) {
+      const int p = base + q;
+      int64_t row = 0;
+      const bool ok = p < pairs && team_pair_row(a, p, row);
+      float re[16], im[16];
+#pragma unroll
+      for (int j2 = 0; j2 < 16; ++j2) {
+        const int j = t + P * j2;
+        const float sg = tb.sgn[j];
+        re[j2] = ok ? sg * static_cast<const float*>(a.k)[(int64_t)p * D + j] : 0.0f;
+        im[j2] = ok ? sg * static_cast<const float*>(a.v)[(int64_t)p * D + j] : 0.0f;
+      }
+      srft_quantize_team<P>(a, row, ok, re, im, c, tb, t, team_base);
+    }
+    return;
+  }
+  // copies of one warp step: chunk i covers bytes 16 w .. of pair base + qq's K (kv = 0) or V row
+  auto issue = [&](int base, unsigned char* buf) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int ch = lane + 32 * r;
+      const int qq = ch / (4 * D / 16), w = ch % (4 * D / 16);
+      const int kv = w / (2 * D / 16), off = 16 * (w % (2 * D / 16));
+      const int p = base + qq;
+      if (p < pairs)
+        cp_async16(buf + qq * PITCH + kv * 2 * D + off,
+                   static_cast<const unsigned char*>(kv ? a.v : a.k) + (int64_t)p * 2 * D + off);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (base0 < pairs) issue(base0, stage[warp][0]);
+  int it = 0;
+  for (int base = base0; base < pairs; base += stride, ++it) {
+    const int nb = base + stride;
+    if (nb < pairs) issue(nb, stage[warp][(it + 1) & 1]);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncwarp();
+    const unsigned char* buf = stage[warp][it & 1] + q * PITCH;
+    const int p = base + q;
+    int64_t row = 0;
+    const bool ok = p < pairs && team_pair_row(a, p, row);
+    float re[16], im[16];
+#pragma unroll
+    for (int j2 = 0; j2 < 16; ++j2) {
+      const int j = t + P * j2;
+      const float sg = tb.sgn[j];
+      const uint32_t uk = reinterpret_cast<const uint16_t*>(buf)[j];
+      const uint32_t uv = reinterpret_cast<const uint16_t*>(buf + 2 * D)[j];
+      re[j2] = ok ? sg * __uint_as_float(uk << 16) : 0.0f;
+      im[j2] = ok ? sg * __uint_as_float(uv << 16) : 0.0f;
+    }
+    srft_quantize_team<P>(a, row, ok, re, im, c, tb, t, team_base);
+    __syncwarp();  // every lane is done with this buffer before it is refilled
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // One warp rotates query heads h0 = 2 (p mod ceil(Hq/2)) and h0 + 1 of sequence
@@ -304,6 +494,20 @@ __global__ void __launch_bounds__(32 * M) srft_merge_kernel(DecodeArgs a) {
 template <int M>
 cudaError_t launch_quantize_srft_m(const QuantizeArgs& a, cudaStream_t stream) {
   const int64_t pairs = (int64_t)a.B * a.Hkv * a.n_new;
+  // d = 128, 256 with a prefill-sized n_new: d / 16 lanes per pair.  Appends of
+  // fewer tokens keep the one-warp kernel, the transform of the decode step's
+  // fused append, so both give the same rows; the team kernel's own rounding
+  // (another factorisation of the same DFT) can differ from it in the last bit.
+  if constexpr (M == 4 || M == 8) {
+    if (a.n_new >= kTeamMinTokens) {
+      constexpr int TPW = 16 / M;  // pairs per warp
+      int64_t blocks = (pairs + 8 * TPW - 1) / (8 * TPW);
+      const int64_t cap = (int64_t)kSmCount * 8;
+      if (blocks > cap) blocks = cap;
+      srft_quantize_team_kernel<2 * M><<<(unsigned)blocks, 256, 0, stream>>>(a);
+      return cudaGetLastError();
+    }
+  }
   int64_t blocks = (pairs + kQWarps - 1) / kQWarps;
   const int64_t cap = (int64_t)kSmCount * (M <= 4 ? 8 : 4);
   if (blocks > cap) blocks = cap;
