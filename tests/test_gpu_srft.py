@@ -144,11 +144,14 @@ def test_srft_decode_without_lambda_or_signs():
     srft_parity(1, 1, 2, 160, [500], signs=False, seed=13)
 
 
-def test_srft_decode_append_equals_two_calls_and_oracle():
+@pytest.mark.parametrize("d,G", [(96, 4), (128, 4), (128, 8), (256, 2)])
+def test_srft_decode_append_equals_two_calls_and_oracle(d, G):
     """The fused step writes the same cache row and gives the same output as
-    quantize-append then decode; both agree with the oracle."""
+    quantize-append then decode; both agree with the oracle.  d = 96 runs the
+    CUDA-core decode, d = 128 and 256 the tensor-core decode, each after the
+    preparation kernel (new token and query rotation in one launch)."""
     require_cuda()
-    B, Hkv, G, d, T = 2, 2, 4, 96, 900
+    B, Hkv, T = 2, 2, 900
     k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 21)
     sg, lk, lv = signs_for(d, 22), lam_for(d, 23), lam_for(d, 24)
     ctx = [T, T - 100]
