@@ -307,7 +307,8 @@ def run_tq(args):
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
     if not (w.cb_bits or srft):
-        host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale)
+        host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale,
+                                                  graph=True)
 
         def e2e_step():
             host_step()
@@ -428,8 +429,9 @@ def run_tq(args):
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
                   "launching stream (decode split from a K-decode graph; the two-call step "
                   "from a third graph); e2e: per step, tq_sdpa_int4_decode_append_host on "
-                  "pinned host buffers (copies of q, k_new, v_new up, the step, the output "
-                  "down) between CUDA events",
+                  "pinned host buffers (the kernels read q, k_new, v_new and write the output "
+                  "over the bus), replayed from a CUDA graph (Int4KVCache.bind_decode_append_host("
+                  "graph=True)), between CUDA events",
         "clocks": clocks,
         "bulk_prefill": prefill,
         "bf16_dequantize_then_attend": baseline,

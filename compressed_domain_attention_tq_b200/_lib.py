@@ -238,6 +238,31 @@ class BoundCall:
             raise TQError(rc, self._where)
 
 
+class GraphedCall:
+    """A prepared call captured once into a CUDA graph: each call replays the
+    graph on the current stream, so the work the library call enqueues is
+    launched at once instead of call by call from the host.  make_call(stream)
+    builds the call on a stream; it runs once uncaptured first (the library's
+    one-time per-kernel set-up), then is captured.  Host buffers must be
+    pinned; a replay uses what the buffers hold when it runs."""
+
+    def __init__(self, make_call):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            first = make_call(side)
+            first()
+        torch.cuda.current_stream().wait_stream(side)
+        self._graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self._graph):
+            captured = make_call(torch.cuda.current_stream())
+            captured()
+        self._keep = (first, captured)
+
+    def __call__(self):
+        self._graph.replay()
+
+
 def bind_sdpa_int4_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
                                  max_ctx, signs, attn_scale, out, workspace, stream=None) -> BoundCall:
     """sdpa_int4_decode_append prepared for repeated calls on the same buffers."""

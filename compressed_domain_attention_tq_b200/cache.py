@@ -139,10 +139,12 @@ class Int4KVCache:
     def bind_decode_append_host(self, q_host: torch.Tensor, k_new_host: torch.Tensor,
                                 v_new_host: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
                                 out_host: torch.Tensor, attn_scale: float | None = None,
-                                stream=None):
+                                stream=None, graph: bool = False):
         """A prepared decode step on HOST buffers (q, k_new, v_new, out; pin them): each
-        call of the returned step enqueues their copies and the step in one library call
-        (tq_sdpa_int4_decode_append_host); Hadamard-rotated caches."""
+        call of the returned step runs tq_sdpa_int4_decode_append_host (on pinned, mapped
+        buffers the kernels read and write them directly); Hadamard-rotated caches.
+        graph=True captures that call once into a CUDA graph (after running it once) and
+        each call of the step replays the graph on the current stream."""
         if self.srft:
             raise NotImplementedError("bind_decode_append_host runs on Hadamard-rotated caches")
         if attn_scale is None:
@@ -153,10 +155,14 @@ class Int4KVCache:
         if need == 0:
             raise ValueError("invalid decode sizes")
         ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
-        return _lib.bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host, self.k_packed,
-                                                      self.k_scales, self.v_packed, self.v_scales,
-                                                      ctx_lens, max_ctx, self.signs, attn_scale,
-                                                      out_host, ws, stream)
+
+        def make(s):
+            return _lib.bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host,
+                                                          self.k_packed, self.k_scales,
+                                                          self.v_packed, self.v_scales, ctx_lens,
+                                                          max_ctx, self.signs, attn_scale, out_host,
+                                                          ws, s)
+        return _lib.GraphedCall(make) if graph else make(stream)
 
     def dequantize(self, rows: int, dtype=torch.bfloat16, stream=None):
         """Dequantized K and V of rows 0 .. rows-1 of every sequence, [B][Hkv][rows][d]

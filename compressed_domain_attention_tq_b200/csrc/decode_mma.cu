@@ -413,6 +413,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
           x[e + 3] = v.w;
         }
       } else if (a.q_bf16) {  // E consecutive bf16 values: one 8- or 16-byte load
+        if (a.inputs_pending) asm volatile("griddepcontrol.wait;" ::: "memory");
         uint32_t u[E / 2];
         if (E == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + base);
@@ -429,6 +430,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
         for (int e = 0; e < E; ++e)
           x[e] = __uint_as_float(e & 1 ? (u[e / 2] & 0xFFFF0000u) : (u[e / 2] << 16));
       } else {
+        if (a.inputs_pending) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
         for (int e = 0; e < E; e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + base + e);
@@ -1158,6 +1160,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       if (t1 != clamp_ctx_mma(a.ctx_lens[b], a.max_ctx)) continue;  // not the last chunk
       const int64_t bh = (int64_t)b * a.Hkv + kvh;
       const int64_t row = bh * a.capacity + (t1 - 1);
+      if (a.inputs_pending) asm volatile("griddepcontrol.wait;" ::: "memory");  // k_new, v_new
       const unsigned char* src = static_cast<const unsigned char*>(isv ? a.v_new : a.k_new) + bh * D * eb;
       uint8_t* prow = const_cast<uint8_t*>(isv ? a.v_packed : a.k_packed) + row * C::RB;
       float* srow = const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32);
@@ -1236,7 +1239,9 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = a.B * a.Hkv * a.plan.n_chunks;
   const int grid = n_items < sms ? n_items : sms;
-  if (a.q_rot != nullptr && a.q_rot_overlap) {  // overlap the query-rotation grid (see prep_query)
+  // overlap the preceding grid that rotates the queries or gathers the step's
+  // inputs: programmatic dependent launch (the kernel waits where it reads them)
+  if ((a.q_rot != nullptr && a.q_rot_overlap) || a.inputs_pending) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(C::THREADS);

@@ -20,7 +20,36 @@ static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // an item is one (sequence, kv head, chunk).  The tensor-core decode runs
 // persistent CTAs, one per SM; the CUDA-core decode runs one 128-thread CTA
 // per item, several resident per SM.
+static bool make_decode_plan_uncached(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan,
+                                      PlanKind kind);
+
+// The plan depends only on its arguments; each thread keeps its last one, so
+// a decode loop with fixed sizes does the search once.
 bool make_decode_plan(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan, PlanKind kind) {
+  struct Last {
+    int B = 0, Hq = 0, Hkv = 0, d = 0, max_ctx = 0;
+    PlanKind kind = PlanKind::kInt4;
+    DecodePlan plan{};
+  };
+  thread_local Last last;
+  if (last.B == B && last.Hq == Hq && last.Hkv == Hkv && last.d == d && last.max_ctx == max_ctx &&
+      last.kind == kind && B > 0) {
+    *plan = last.plan;
+    return true;
+  }
+  if (!make_decode_plan_uncached(B, Hq, Hkv, d, max_ctx, plan, kind)) return false;
+  last.B = B;
+  last.Hq = Hq;
+  last.Hkv = Hkv;
+  last.d = d;
+  last.max_ctx = max_ctx;
+  last.kind = kind;
+  last.plan = *plan;
+  return true;
+}
+
+static bool make_decode_plan_uncached(int B, int Hq, int Hkv, int d, int max_ctx, DecodePlan* plan,
+                                      PlanKind kind) {
   if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || max_ctx < 1) return false;
   const bool srft = kind == PlanKind::kSrft;
   if (srft ? !srft_head_dim_supported(d) : (d != 128 && d != 256)) return false;
@@ -253,6 +282,36 @@ int32_t tq_decode_chunk_tokens(int32_t batch, int32_t num_q_heads, int32_t num_k
 
 // Shared by tq_sdpa_int4_decode and tq_sdpa_int4_decode_append (k_new, v_new
 // non-NULL: append the new token of every (sequence, kv head) first).
+// A host-buffer step's inputs, moved into the workspace's staging space by
+// decode_impl once the call is validated, before its first launch: by the
+// gather kernel when the host buffers are mapped, else by three copies.
+struct HostInputs {
+  bool gather;
+  const void *q, *k, *v;  // host buffers (their device addresses when gather)
+  unsigned char *dq, *dk, *dv;
+  size_t q_bytes, kv_bytes;
+};
+
+__global__ void host_gather_kernel(const uint4* q, uint4* dq, int64_t nq, const uint4* k, uint4* dk,
+                                   const uint4* v, uint4* dv, int64_t nkv);
+
+static cudaError_t move_host_inputs(const HostInputs& h, cudaStream_t s) {
+  if (h.gather) {
+    const int64_t nq = (int64_t)(h.q_bytes / 16), nkv = (int64_t)(h.kv_bytes / 16);
+    const int64_t n = nq > nkv ? nq : nkv;
+    const unsigned blocks = (unsigned)(n / 256 + 1 < 64 ? n / 256 + 1 : 64);
+    host_gather_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const uint4*>(h.q), reinterpret_cast<uint4*>(h.dq), nq,
+        static_cast<const uint4*>(h.k), reinterpret_cast<uint4*>(h.dk),
+        static_cast<const uint4*>(h.v), reinterpret_cast<uint4*>(h.dv), nkv);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaMemcpyAsync(h.dq, h.q, h.q_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h.dk, h.k, h.kv_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h.dv, h.v, h.kv_bytes, cudaMemcpyHostToDevice, s);
+  return e;
+}
+
 static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new,
                              tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
                              int32_t num_kv_heads, int32_t head_dim, int32_t group,
@@ -261,7 +320,8 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
                              const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
                              float attn_scale, float* out, void* workspace, size_t workspace_bytes,
                              void* cuda_stream, const char* where, float* lse = nullptr,
-                             const Rotation& rot = Rotation{}) {
+                             const Rotation& rot = Rotation{},
+                             const HostInputs* host_in = nullptr) {
   if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
     return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
@@ -295,6 +355,11 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   // bounded waits for its first copies run out (its outputs are then NaN).
   if (getenv("TQ_TEST_FAIL_LAUNCH")) return cuda_status(cudaErrorLaunchFailure, where);
   a.test_starve = getenv("TQ_TEST_STARVE_PIPELINE") != nullptr;
+  if (host_in != nullptr) {
+    const cudaError_t e = move_host_inputs(*host_in, static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return cuda_status(e, where);
+    a.inputs_pending = host_in->gather;  // the tensor-core decode overlaps the gather kernel
+  }
   a.q = q;
   a.q_bf16 = q_dtype == TQ_BF16;
   a.B = batch;
@@ -565,6 +630,41 @@ size_t tq_decode_append_host_workspace_bytes(int32_t batch, int32_t num_q_heads,
   return hs.total;
 }
 
+}  // extern "C"
+
+// Copies the step's inputs from mapped host memory into the workspace's
+// staging space: byte ranges that start 16-byte aligned and are multiples of
+// 16 bytes long, as 16-byte loads spread over the grid, so each input crosses
+// the bus once, in full coalesced requests (the decode then reads it from
+// device memory: every CTA of a kv head reads its queries).
+__global__ void host_gather_kernel(const uint4* q, uint4* dq, int64_t nq, const uint4* k, uint4* dk,
+                                   const uint4* v, uint4* dv, int64_t nkv) {
+  // the tensor-core decode may start streaming the cache now; it waits for
+  // this grid before it reads q, k_new and v_new
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nq; i += stride) dq[i] = q[i];
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nkv; i += stride) {
+    dk[i] = k[i];
+    dv[i] = v[i];
+  }
+}
+
+// The device address of a host buffer that kernels can access directly
+// (page-locked and mapped under unified addressing) when it is 16-byte
+// aligned there, else nullptr.
+static void* device_view(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the query's error
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+  return aligned16(at.devicePointer) ? at.devicePointer : nullptr;
+}
+
+extern "C" {
+
 tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
                                           const void* k_new_host, const void* v_new_host,
                                           tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
@@ -586,21 +686,32 @@ tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
   if (!workspace || workspace_bytes < hs.total) return TQ_ERR_WORKSPACE;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const size_t qb = hs.k - hs.q, kb = hs.v - hs.k;  // padded sizes; copy the exact bytes
   const size_t q_bytes = (size_t)batch * num_q_heads * head_dim * (q_dtype == TQ_BF16 ? 2 : 4);
   const size_t kv_bytes = (size_t)batch * num_kv_heads * head_dim * (kv_dtype == TQ_BF16 ? 2 : 4);
   const size_t out_bytes = (size_t)batch * num_q_heads * head_dim * 4;
-  (void)qb;
-  (void)kb;
-  cudaError_t e = cudaMemcpyAsync(ws + hs.q, q_host, q_bytes, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + hs.k, k_new_host, kv_bytes, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + hs.v, v_new_host, kv_bytes, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_status(e, "tq_sdpa_int4_decode_append_host");
+  // mapped host buffers: one small kernel gathers the inputs into the staging
+  // space and the merge writes the output into out_host, no copies
+  const void* dq = device_view(q_host);
+  const void* dk = device_view(k_new_host);
+  const void* dv = device_view(v_new_host);
+  void* dout = device_view(out_host);
+  const bool mapped = dq && dk && dv && dout && q_bytes % 16 == 0 && kv_bytes % 16 == 0;
+  HostInputs hin;
+  hin.gather = mapped;
+  hin.q = mapped ? dq : q_host;
+  hin.k = mapped ? dk : k_new_host;
+  hin.v = mapped ? dv : v_new_host;
+  hin.dq = ws + hs.q;
+  hin.dk = ws + hs.k;
+  hin.dv = ws + hs.v;
+  hin.q_bytes = q_bytes;
+  hin.kv_bytes = kv_bytes;
   const tq_status st = decode_impl(
       ws + hs.q, q_dtype, ws + hs.k, ws + hs.v, kv_dtype, batch, num_q_heads, num_kv_heads,
       head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens, max_ctx, signs,
-      attn_scale, reinterpret_cast<float*>(ws + hs.out), workspace, hs.q, cuda_stream,
-      "tq_sdpa_int4_decode_append_host");
+      attn_scale, mapped ? static_cast<float*>(dout) : reinterpret_cast<float*>(ws + hs.out),
+      workspace, hs.q, cuda_stream, "tq_sdpa_int4_decode_append_host", nullptr, Rotation{}, &hin);
+  if (st != TQ_OK || mapped) return st;
   if (st != TQ_OK) return st;
   return cuda_status(cudaMemcpyAsync(out_host, ws + hs.out, out_bytes, cudaMemcpyDeviceToHost, s),
                      "tq_sdpa_int4_decode_append_host");

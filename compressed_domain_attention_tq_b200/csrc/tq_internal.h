@@ -90,6 +90,9 @@ struct DecodeArgs {
   const float* lambda_v = nullptr;
   int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
   const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
+  int inputs_pending = 0;           // q, k_new and v_new are written by the preceding kernel:
+                                    // the tensor-core decode is launched as its programmatic
+                                    // dependent and waits for it before reading them
 };
 
 // Raise a kernel's dynamic shared memory limit once per device (the first

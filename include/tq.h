@@ -196,9 +196,15 @@ TQ_API tq_status tq_sdpa_int4_decode_append(
  * q, k_new and v_new into staging space at the end of the workspace, the
  * decode step, and the device-to-host copy of the output, all on cuda_stream,
  * and returns without synchronizing (the output is in out_host once the stream
- * reaches that point).  Host buffers should be pinned (cudaHostAlloc) for the
- * copies to be asynchronous; pageable memory works but the copies then stage
- * through the driver.
+ * reaches that point).  When all four host buffers are page-locked and mapped
+ * into the device's address space (cudaHostAlloc / cudaMallocHost memory under
+ * unified addressing, as cudaPointerGetAttributes reports) and 16-byte
+ * aligned, no copies are enqueued: a small kernel reads q, k_new and v_new
+ * over the bus into the staging space and the merge kernel writes the output
+ * into out_host directly (the same bytes cross the bus).  Otherwise
+ * the inputs and output are staged as above; pageable memory works, the
+ * copies then staging through the driver.  Either way the host buffers must
+ * not change (inputs) or be read (output) until the stream has passed the step.
  *
  *  q_host          [B][Hq][d] of q_dtype; k_new_host, v_new_host [B][Hkv][1][d] of
  *                  kv_dtype; out_host [B][Hq][d] fp32.

@@ -114,9 +114,12 @@ def test_bound_decode_append_matches_plain_call_on_refilled_buffers():
         assert torch.equal(a, b)
 
 
-def test_host_buffer_step_matches_device_step():
-    """tq_sdpa_int4_decode_append_host on pinned host buffers writes the same cache
-    rows and returns the same output (bit for bit) as the device-buffer step."""
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_buffer_step_matches_device_step(pinned):
+    """tq_sdpa_int4_decode_append_host on host buffers writes the same cache rows
+    and returns the same output (bit for bit) as the device-buffer step: pinned
+    (mapped) buffers are read and written by the kernels directly, pageable ones
+    are staged through the workspace by copies."""
     require_cuda()
     import torch
     from compressed_domain_attention_tq_b200 import Int4KVCache
@@ -132,13 +135,55 @@ def test_host_buffer_step_matches_device_step():
     kn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
     vn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
     ctx = torch.tensor([T + 1, T - 40], dtype=torch.int32, device="cuda")
-    hq, hk, hv = q.pin_memory(), kn.pin_memory(), vn.pin_memory()
-    hout = torch.empty(B, Hkv * G, d, dtype=torch.float32).pin_memory()
+    if pinned:
+        hq, hk, hv = q.pin_memory(), kn.pin_memory(), vn.pin_memory()
+        hout = torch.empty(B, Hkv * G, d, dtype=torch.float32).pin_memory()
+    else:
+        hq, hk, hv = q.clone(), kn.clone(), vn.clone()
+        hout = torch.empty(B, Hkv * G, d, dtype=torch.float32)
     step = caches[0].bind_decode_append_host(hq, hk, hv, ctx, T + 2, hout, 0.1)
     step()
     out_d = caches[1].decode_append(q.cuda(), kn.cuda(), vn.cuda(), ctx, T + 2, 0.1)
     torch.cuda.synchronize()
     assert torch.equal(hout, out_d.cpu())
+    for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
+                    (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
+        assert torch.equal(a, b)
+
+
+def test_graphed_host_buffer_step_matches_direct_calls():
+    """bind_decode_append_host(graph=True): the step captured once into a CUDA
+    graph and replayed gives, step after step with new host inputs, the same
+    output and cache rows (bit for bit) as the direct host-buffer call."""
+    require_cuda()
+    from compressed_domain_attention_tq_b200 import Int4KVCache
+    B, Hkv, G, d, T = 2, 2, 8, 128, 700
+    g = torch.Generator().manual_seed(94)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+    caches = [Int4KVCache(B, Hkv, d, T + 4, signs=signs) for _ in range(2)]
+    for c in caches:
+        c.append(k, v, torch.zeros(B, dtype=torch.int32, device="cuda"))
+    ctx = torch.tensor([T + 1, T - 60], dtype=torch.int32, device="cuda")
+    hosts = [(torch.zeros(B, Hkv * G, d, dtype=torch.bfloat16).pin_memory(),
+              torch.zeros(B, Hkv, 1, d, dtype=torch.bfloat16).pin_memory(),
+              torch.zeros(B, Hkv, 1, d, dtype=torch.bfloat16).pin_memory(),
+              torch.zeros(B, Hkv * G, d, dtype=torch.float32).pin_memory()) for _ in range(2)]
+    steps = [caches[0].bind_decode_append_host(*hosts[0][:3], ctx, T + 4, hosts[0][3], 0.1,
+                                               graph=True),
+             caches[1].bind_decode_append_host(*hosts[1][:3], ctx, T + 4, hosts[1][3], 0.1)]
+    for i in range(3):
+        q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16)
+        kn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+        vn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+        for (hq, hk, hv, _), step in zip(hosts, steps):
+            hq.copy_(q)
+            hk.copy_(kn)
+            hv.copy_(vn)
+            step()
+            torch.cuda.synchronize()
+        assert torch.equal(hosts[0][3], hosts[1][3]), f"step {i}"
     for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
                     (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
         assert torch.equal(a, b)
