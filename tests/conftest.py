@@ -17,7 +17,7 @@ def require_cuda():
     """GPU tests fail loudly (never skip) when no device is present."""
     import torch
     if not torch.cuda.is_available():
-        pytest.fail("this test needs a CUDA device; run it on the GPU box (-m gpu)")
+        pytest.fail("this test needs a CUDA device (run the -m gpu tests on a machine with one)")
 
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
