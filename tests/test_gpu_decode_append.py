@@ -187,3 +187,45 @@ def test_graphed_host_buffer_step_matches_direct_calls():
     for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
                     (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("case", ["unaligned", "fp32"])
+def test_host_buffer_step_fallbacks_and_dtypes(case):
+    """tq_sdpa_int4_decode_append_host with pinned buffers that are not 16-byte
+    aligned (the staged copies are used instead of the gather kernel) and with
+    fp32 inputs (the gather kernel moves 4-byte elements): bit-identical to the
+    device-buffer step."""
+    require_cuda()
+    from compressed_domain_attention_tq_b200 import Int4KVCache
+    B, Hkv, G, d, T = 1, 2, 8, 128, 600
+    dt = torch.float32 if case == "fp32" else torch.bfloat16
+    g = torch.Generator().manual_seed(95)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(dt).cuda()
+    v = torch.randn(B, Hkv, T, d, generator=g).to(dt).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+    caches = [Int4KVCache(B, Hkv, d, T + 2, signs=signs) for _ in range(2)]
+    for c in caches:
+        c.append(k, v, torch.zeros(B, dtype=torch.int32, device="cuda"))
+    q = torch.randn(B, Hkv * G, d, generator=g).to(dt)
+    kn = torch.randn(B, Hkv, 1, d, generator=g).to(dt)
+    vn = torch.randn(B, Hkv, 1, d, generator=g).to(dt)
+    ctx = torch.tensor([T + 1], dtype=torch.int32, device="cuda")
+
+    def pinned_like(t, shift):
+        # a pinned buffer whose data starts `shift` elements into its allocation
+        buf = torch.empty(t.numel() + shift, dtype=t.dtype).pin_memory()
+        view = buf[shift:].view(t.shape)
+        view.copy_(t)
+        return view
+
+    shift = 1 if case == "unaligned" else 0
+    hq, hk, hv = pinned_like(q, shift), pinned_like(kn, shift), pinned_like(vn, shift)
+    hout = pinned_like(torch.zeros(B, Hkv * G, d), shift)
+    step = caches[0].bind_decode_append_host(hq, hk, hv, ctx, T + 2, hout, 0.1)
+    step()
+    out_d = caches[1].decode_append(q.cuda(), kn.cuda(), vn.cuda(), ctx, T + 2, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, out_d.cpu())
+    for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
+                    (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
+        assert torch.equal(a, b)
