@@ -428,10 +428,15 @@ def run_tq(args):
         "step": step_desc,
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
                   "launching stream (decode split from a K-decode graph; the two-call step "
-                  "from a third graph); e2e: per step, tq_sdpa_int4_decode_append_host on "
-                  "pinned host buffers (the kernels read q, k_new, v_new and write the output "
-                  "over the bus), replayed from a CUDA graph (Int4KVCache.bind_decode_append_host("
-                  "graph=True)), between CUDA events",
+                  "from a third graph); e2e: " + (
+                      "per step, tq_sdpa_int4_decode_append_host on pinned host buffers (a "
+                      "gather kernel reads q, k_new, v_new over the bus, the merge writes the "
+                      "output into host memory), replayed from a CUDA graph "
+                      "(Int4KVCache.bind_decode_append_host(graph=True)), between CUDA events"
+                      if not (w.cb_bits or srft) else
+                      "per step, copies of q, k_new, v_new from pinned host memory, the "
+                      "public decode_append call, and the copy of the output back, between "
+                      "CUDA events"),
         "clocks": clocks,
         "bulk_prefill": prefill,
         "bf16_dequantize_then_attend": baseline,
