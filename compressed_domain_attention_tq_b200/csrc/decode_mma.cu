@@ -884,8 +884,8 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
 
 // Codebook P.V (heads on rows): as tile_pv with the B operand the levels of
 // coordinates 32g + 4 gid + e (n-tile e) of the token pairs (rho0, rho1) and
-// (rho2, rho3), hi and lo parts from the level-pair table, both products in
-// the same accumulator.  Branch-free.
+// (rho2, rho3), hi and lo parts from the level-pair table (one lookup per row
+// and pair of coordinates), both products in the same accumulator.  Branch-free.
 template <int D, int PATH, int FMT, int TPW>
 __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int gid,
                                            const int (&rho)[4], const float (&p)[TPW][4],
@@ -893,30 +893,25 @@ __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int
                                            WarpState<D, PATH, FMT>& st, const unsigned char* lutp) {
   using C = Cfg<D, PATH, FMT>;
   constexpr int NG = C::NG, RB = C::RB, GB = 4 * FMT;  // GB: bytes per group
-  constexpr uint32_t M = (1u << FMT) - 1;
+  constexpr uint32_t KM = (1u << (2 * FMT)) - 1;      // key mask (two indices)
   const unsigned char* vc = stg + C::VC + r0 * RB;
   const int bo = 4 * FMT * gid;  // bit offset of this thread's 4 indices in a group
 #pragma unroll
   for (int u = 0; u < TPW; ++u) {
-    uint32_t f[2][NG];  // per token pair: indices of row rho[2j] | those of rho[2j + 1] << 16
+    uint32_t f[4][NG];  // row rho[i]'s indices of dims 32g + 4 gid .. + 3 (4 FMT bits)
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
-        uint32_t v[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const unsigned char* rp = vc + (16 * u + rho[2 * j + r]) * RB + g * GB;
-          if (FMT == 2) {
-            v[r] = rp[gid];
-          } else if (FMT == 4) {
-            v[r] = reinterpret_cast<const uint16_t*>(rp)[gid];
-          } else {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(rp) + (bo >> 5);
-            v[r] = __funnelshift_r(w[0], w[1], bo & 31) & 0xFFFu;
-          }
+        const unsigned char* rp = vc + (16 * u + rho[i]) * RB + g * GB;
+        if (FMT == 2) {
+          f[i][g] = rp[gid];
+        } else if (FMT == 4) {
+          f[i][g] = reinterpret_cast<const uint16_t*>(rp)[gid];
+        } else {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(rp) + (bo >> 5);
+          f[i][g] = __funnelshift_r(w[0], w[1], bo & 31);
         }
-        f[j][g] = v[0] | (v[1] << 16);
       }
 #pragma unroll
     for (int gp = 0; gp < NG; gp += 2) {
@@ -937,17 +932,22 @@ __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int
         const int g = gp + eg;
         const uint32_t a0 = f16x2(wh[0][eg], wh[1][eg]), a1 = f16x2(wl[0][eg], wl[1][eg]);
         const uint32_t a2 = f16x2(wh[2][eg], wh[3][eg]), a3 = f16x2(wl[2][eg], wl[3][eg]);
+        // level pairs of dims (4 gid, 4 gid + 1) and (4 gid + 2, 4 gid + 3) of each row,
+        // then byte permutes pair the rows: n-tile e takes the half holding dim 4 gid + e
+        uint2 lv[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+            lv[i][m] = *reinterpret_cast<const uint2*>(lutp + (((f[i][g] >> (2 * FMT * m)) & KM) << 3));
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          uint2 b[2];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const uint32_t t = f[j][g];
-            const uint32_t key = ((t >> (FMT * e)) & M) | (((t >> (16 + FMT * e)) & M) << FMT);
-            b[j] = *reinterpret_cast<const uint2*>(lutp + (key << 3));
-          }
-          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, b[0].x, b[1].x);
-          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, b[0].y, b[1].y);
+          const int m = e >> 1;
+          const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
+          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, prmt(lv[0][m].x, lv[1][m].x, sel),
+                   prmt(lv[2][m].x, lv[3][m].x, sel));
+          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, prmt(lv[0][m].y, lv[1][m].y, sel),
+                   prmt(lv[2][m].y, lv[3][m].y, sel));
         }
       }
     }
