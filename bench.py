@@ -76,11 +76,17 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel_key):
+    """Hash of the code in a kernel's sources: comments and layout do not count."""
+    import re
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "compressed_domain_attention_tq_b200", "csrc")
     for f in sorted(KERNEL_SOURCES[kernel_key]):
-        with open(os.path.join(cs, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(cs, f), encoding="utf-8") as fh:
+            code = fh.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        code = " ".join(code.split())
+        h.update(f.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

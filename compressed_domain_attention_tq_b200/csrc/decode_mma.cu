@@ -42,6 +42,14 @@
 //    above with each head on two neighbouring rows; P.V C = V^T x [P' hi,
 //    P' lo per head] with dims on the rows, so the accumulator is d/16 x 4
 //    registers.
+// Cache formats (template FMT):
+//  - FMT 0: int4 codes (above).
+//  - FMT 2, 3, 4: codebook indices of that many bits (PATH 0 only).  Each CTA
+//    first builds a table over index pairs holding the two levels as f16 hi
+//    and lo parts (levels scaled by a power of two into [0.5, 1)).  Every MMA
+//    operand register is then one 8-byte table read, and each k-step runs
+//    twice (hi levels, lo levels) into the same accumulator; sigma is applied
+//    per group as the int4 scale is.
 // Token order: slot k of a 16-token tile holds tile row pi(k), chosen so that
 // the K-code and scale loads of a warp hit distinct shared-memory banks.
 #include <cuda_bf16.h>
