@@ -115,6 +115,19 @@ def test_decode_attn_scale_one_d128_peaked():
     parity(1, 2, 8, 128, [2000], scale=1.0, seed=51)
 
 
+@pytest.mark.parametrize("B,G", [(1100, 8), (1030, 2)])
+def test_decode_large_batch_without_item_list(B, G):
+    """More sequences than the tensor-core decode's in-shared-memory item list
+    holds (1024): the kernel walks every (sequence, kv head, chunk) of the plan,
+    and the items past a short sequence's end do no work.  Ragged lengths from 1
+    to 700 tokens against the oracle for every sequence."""
+    require_cuda()
+    rng = np.random.default_rng(B + G)
+    ctx = [int(x) for x in rng.integers(1, 701, size=B)]
+    ctx[0] = 700
+    parity(B, 1, G, 128, ctx, seed=B + G)
+
+
 def test_decode_flags_and_clamping():
     require_cuda()
     B, Hkv, G, d, T = 3, 1, 4, 128, 200
