@@ -256,3 +256,22 @@ def test_cb_fused_step_ragged_batch(bits):
     want = oracle.sdpa_cb_decode(to_oracle(q), caches[0], ctx, signs.numpy(), bits, lv.numpy(),
                                  1 / math.sqrt(d), Hkv, threads=THREADS)
     check_attention_cb(outs[0], want, caches[0], ctx, G, bits, lv, f"cb{bits} fused step")
+
+
+def test_cb_tensor_core_decode_large_batch():
+    """1030 ragged sequences (more than the decode's in-shared-memory item
+    list holds): the tensor-core codebook decode walks every item of the plan."""
+    require_cuda()
+    B, Hkv, G, d, bits = 1030, 1, 8, 128, 3
+    rng = np.random.default_rng(7)
+    ctx = [int(x) for x in rng.integers(1, 400, size=B)]
+    ctx[0] = 400
+    T = max(ctx)
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 77)
+    signs = signs_for(d, 78)
+    lv = levels_for(bits)
+    cache = oracle_cb_cache(k, v, signs, bits, lv)
+    got = cb_decode(upload_cache(cache), q, ctx, T, signs, bits, lv, 1 / math.sqrt(d), Hkv)
+    want = oracle.sdpa_cb_decode(to_oracle(q), cache, ctx, signs.numpy(), bits, lv.numpy(),
+                                 1 / math.sqrt(d), Hkv, threads=THREADS)
+    check_attention_cb(got, want, cache, ctx, G, bits, lv, "cb3 B=1030")

@@ -212,3 +212,21 @@ def test_srft_cache_engine_end_to_end():
     check_attention(out.cpu().numpy(), want, cache, [T], G, "srft engine")
     ref = oracle_srft_cache(k, v, sg, lk, lv)
     compare(cache, ref, d, True, "srft engine cache", SCALE_ULP)
+
+
+def test_srft_decode_large_ragged_batch():
+    """1030 ragged sequences with the SRFT rotation on the tensor-core decode
+    (query rotation kernel over every sequence, items past short sequences)."""
+    require_cuda()
+    B, Hkv, G, d = 1030, 1, 8, 128
+    rng = np.random.default_rng(9)
+    ctx = [int(x) for x in rng.integers(1, 300, size=B)]
+    ctx[0] = 300
+    T = max(ctx)
+    k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 91)
+    sg, lk, lv = signs_for(d, 92), lam_for(d, 93), lam_for(d, 94)
+    cache = oracle_srft_cache(k, v, sg, lk, lv)
+    got = srft_decode(upload_cache(cache), q, ctx, T, sg, lk, lv, 0.09, Hkv)
+    want = oracle.sdpa_int4_decode_srft(to_oracle(q), cache, ctx, sg.numpy(), lk.numpy(),
+                                        lv.numpy(), 0.09, Hkv, threads=THREADS)
+    check_attention(got, want, cache, ctx, G, "srft B=1030")
