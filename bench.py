@@ -312,21 +312,11 @@ def run_tq(args):
     h_q, h_k, h_v = (t.cpu().pin_memory() for t in (q, k_new, v_new))
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
-    if not (w.cb_bits or srft):
-        host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale,
-                                                  graph=True)
+    host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale,
+                                              graph=True)
 
-        def e2e_step():
-            host_step()
-    else:
-        d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
-
-        def e2e_step():
-            d_q.copy_(h_q, non_blocking=True)
-            d_k.copy_(h_k, non_blocking=True)
-            d_v.copy_(h_v, non_blocking=True)
-            cache.decode_append(d_q, d_k, d_v, ctx_dev, max_ctx, scale, out)
-            h_out.copy_(out, non_blocking=True)
+    def e2e_step():
+        host_step()
     e2e_t = []
     for i in range(args.warmup + args.steps):
         flush.fill_(i & 0xFF)
@@ -434,15 +424,11 @@ def run_tq(args):
         "step": step_desc,
         "timing": "device: one CUDA graph of K steps replayed between CUDA events on the "
                   "launching stream (decode split from a K-decode graph; the two-call step "
-                  "from a third graph); e2e: " + (
-                      "per step, tq_sdpa_int4_decode_append_host on pinned host buffers (a "
-                      "gather kernel reads q, k_new, v_new over the bus, the merge writes the "
-                      "output into host memory), replayed from a CUDA graph "
-                      "(Int4KVCache.bind_decode_append_host(graph=True)), between CUDA events"
-                      if not (w.cb_bits or srft) else
-                      "per step, copies of q, k_new, v_new from pinned host memory, the "
-                      "public decode_append call, and the copy of the output back, between "
-                      "CUDA events"),
+                  "from a third graph); e2e: per step, the host-buffer decode step "
+                  "(tq_sdpa_int4_decode_append_host, or its SRFT / codebook form) on pinned "
+                  "host buffers (a gather kernel reads q, k_new, v_new over the bus, the merge "
+                  "writes the output into host memory), replayed from a CUDA graph "
+                  "(cache.bind_decode_append_host(graph=True)), between CUDA events",
         "clocks": clocks,
         "bulk_prefill": prefill,
         "bf16_dequantize_then_attend": baseline,

@@ -27,6 +27,8 @@ SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_t
            "tq_quantize_append_cb", "tq_sdpa_cb_decode", "tq_sdpa_cb_decode_append",
            "tq_sdpa_int4_decode_srft_lse", "tq_sdpa_cb_decode_lse",
            "tq_decode_append_host_workspace_bytes", "tq_sdpa_int4_decode_append_host",
+           "tq_decode_append_host_srft_workspace_bytes", "tq_sdpa_int4_decode_append_srft_host",
+           "tq_decode_append_host_cb_workspace_bytes", "tq_sdpa_cb_decode_append_host",
            "tq_status_string")
 
 _lib = None
@@ -104,6 +106,16 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_int4_decode_append_host.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, P,
                                                     P, P, P, i64, P, i32, P, f32, P, P, sz, P]
     lib.tq_sdpa_int4_decode_append_host.restype = i32
+    for name in ("tq_decode_append_host_srft_workspace_bytes", "tq_decode_append_host_cb_workspace_bytes"):
+        getattr(lib, name).argtypes = [i32, i32, i32, i32, i32, i32, i32]
+        getattr(lib, name).restype = sz
+    lib.tq_sdpa_int4_decode_append_srft_host.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32,
+                                                         P, P, P, P, i64, P, i32, P, P, P, f32, P, P,
+                                                         sz, P]
+    lib.tq_sdpa_int4_decode_append_srft_host.restype = i32
+    lib.tq_sdpa_cb_decode_append_host.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, i32, P,
+                                                  P, P, P, P, i64, P, i32, P, f32, P, P, sz, P]
+    lib.tq_sdpa_cb_decode_append_host.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -453,10 +465,15 @@ def sdpa_cb_decode_lse(q, k_packed, k_scales, v_packed, v_scales, ctx_lens, max_
 # -------------------------------------------------- host-buffer decode step
 
 def decode_append_host_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx,
-                                       q_dtype=torch.bfloat16, kv_dtype=torch.bfloat16) -> int:
+                                       q_dtype=torch.bfloat16, kv_dtype=torch.bfloat16,
+                                       kind="int4") -> int:
+    """Workspace bytes of a host-buffer step; kind: "int4", "srft" or "cb"."""
     code = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16}
-    return int(load().tq_decode_append_host_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
-                                                            max_ctx, code[q_dtype], code[kv_dtype]))
+    fn = {"int4": "tq_decode_append_host_workspace_bytes",
+          "srft": "tq_decode_append_host_srft_workspace_bytes",
+          "cb": "tq_decode_append_host_cb_workspace_bytes"}[kind]
+    return int(getattr(load(), fn)(batch, num_q_heads, num_kv_heads, head_dim, max_ctx,
+                                   code[q_dtype], code[kv_dtype]))
 
 
 def _host(*ts):
@@ -486,3 +503,51 @@ def bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host, k_packed, 
             out_host, workspace)
     return BoundCall(load().tq_sdpa_int4_decode_append_host, args,
                      "tq_sdpa_int4_decode_append_host", keep)
+
+
+def bind_sdpa_int4_decode_append_srft_host(q_host, k_new_host, v_new_host, k_packed, k_scales,
+                                           v_packed, v_scales, ctx_lens, max_ctx, signs, lambda_k,
+                                           lambda_v, attn_scale, out_host, workspace,
+                                           stream=None) -> BoundCall:
+    """bind_sdpa_int4_decode_append_host for an SRFT-rotated cache."""
+    _host(q_host, k_new_host, v_new_host, out_host)
+    _need_cuda(k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, lambda_k, lambda_v,
+               workspace)
+    if k_new_host.dtype != v_new_host.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q_host.shape
+    Hkv = k_packed.shape[1]
+    i32, f32, sz = ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    args = (_ptr(q_host), i32(_dtype_code(q_host)), _ptr(k_new_host), _ptr(v_new_host),
+            i32(_dtype_code(k_new_host)), i32(B), i32(Hq), i32(Hkv), i32(d), i32(32), _ptr(k_packed),
+            _ptr(k_scales), _ptr(v_packed), _ptr(v_scales), ctypes.c_int64(k_packed.shape[2]),
+            _ptr(ctx_lens), i32(int(max_ctx)), _ptr(signs), _ptr(lambda_k), _ptr(lambda_v),
+            f32(float(attn_scale)), _ptr(out_host), _ptr(workspace),
+            sz(workspace.numel() * workspace.element_size()), _stream(stream))
+    keep = (q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs,
+            lambda_k, lambda_v, out_host, workspace)
+    return BoundCall(load().tq_sdpa_int4_decode_append_srft_host, args,
+                     "tq_sdpa_int4_decode_append_srft_host", keep)
+
+
+def bind_sdpa_cb_decode_append_host(q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed,
+                                    v_scales, ctx_lens, max_ctx, signs, bits, levels, attn_scale,
+                                    out_host, workspace, stream=None) -> BoundCall:
+    """bind_sdpa_int4_decode_append_host for a codebook cache."""
+    _host(q_host, k_new_host, v_new_host, out_host)
+    _need_cuda(k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels, workspace)
+    if k_new_host.dtype != v_new_host.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q_host.shape
+    Hkv = k_packed.shape[1]
+    i32, f32, sz = ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    args = (_ptr(q_host), i32(_dtype_code(q_host)), _ptr(k_new_host), _ptr(v_new_host),
+            i32(_dtype_code(k_new_host)), i32(B), i32(Hq), i32(Hkv), i32(d), i32(32), i32(int(bits)),
+            _ptr(levels), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+            ctypes.c_int64(k_packed.shape[2]), _ptr(ctx_lens), i32(int(max_ctx)), _ptr(signs),
+            f32(float(attn_scale)), _ptr(out_host), _ptr(workspace),
+            sz(workspace.numel() * workspace.element_size()), _stream(stream))
+    keep = (q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs,
+            levels, out_host, workspace)
+    return BoundCall(load().tq_sdpa_cb_decode_append_host, args, "tq_sdpa_cb_decode_append_host",
+                     keep)

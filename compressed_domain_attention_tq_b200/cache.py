@@ -141,22 +141,26 @@ class Int4KVCache:
                                 out_host: torch.Tensor, attn_scale: float | None = None,
                                 stream=None, graph: bool = False):
         """A prepared decode step on HOST buffers (q, k_new, v_new, out; pin them): each
-        call of the returned step runs tq_sdpa_int4_decode_append_host (on pinned, mapped
-        buffers the kernels read and write them directly); Hadamard-rotated caches.
-        graph=True captures that call once into a CUDA graph (after running it once) and
-        each call of the step replays the graph on the current stream."""
-        if self.srft:
-            raise NotImplementedError("bind_decode_append_host runs on Hadamard-rotated caches")
+        call of the returned step runs tq_sdpa_int4_decode_append_host (or its SRFT form;
+        on pinned, mapped buffers a gather kernel reads the inputs and the merge writes the
+        output directly).  graph=True captures that call once into a CUDA graph (after
+        running it once) and each call of the step replays the graph on the current stream."""
         if attn_scale is None:
             attn_scale = 1.0 / math.sqrt(self.head_dim)
         need = _lib.decode_append_host_workspace_bytes(self.batch, q_host.shape[1], self.num_kv_heads,
                                                        self.head_dim, max_ctx, q_host.dtype,
-                                                       k_new_host.dtype)
+                                                       k_new_host.dtype,
+                                                       "srft" if self.srft else "int4")
         if need == 0:
             raise ValueError("invalid decode sizes")
         ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
 
         def make(s):
+            if self.srft:
+                return _lib.bind_sdpa_int4_decode_append_srft_host(
+                    q_host, k_new_host, v_new_host, self.k_packed, self.k_scales, self.v_packed,
+                    self.v_scales, ctx_lens, max_ctx, self.signs, self.lambda_k, self.lambda_v,
+                    attn_scale, out_host, ws, s)
             return _lib.bind_sdpa_int4_decode_append_host(q_host, k_new_host, v_new_host,
                                                           self.k_packed, self.k_scales,
                                                           self.v_packed, self.v_scales, ctx_lens,
@@ -242,6 +246,29 @@ class CodebookKVCache:
                                    self.v_scales, ctx_lens, max_ctx, self.signs, self.bits,
                                    self.levels, attn_scale, out, ws, stream)
         return out
+
+    def bind_decode_append_host(self, q_host: torch.Tensor, k_new_host: torch.Tensor,
+                                v_new_host: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
+                                out_host: torch.Tensor, attn_scale: float | None = None,
+                                stream=None, graph: bool = False):
+        """Int4KVCache.bind_decode_append_host for the codebook cache
+        (tq_sdpa_cb_decode_append_host)."""
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        need = _lib.decode_append_host_workspace_bytes(self.batch, q_host.shape[1], self.num_kv_heads,
+                                                       self.head_dim, max_ctx, q_host.dtype,
+                                                       k_new_host.dtype, "cb")
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
+
+        def make(s):
+            return _lib.bind_sdpa_cb_decode_append_host(q_host, k_new_host, v_new_host,
+                                                        self.k_packed, self.k_scales, self.v_packed,
+                                                        self.v_scales, ctx_lens, max_ctx, self.signs,
+                                                        self.bits, self.levels, attn_scale,
+                                                        out_host, ws, s)
+        return _lib.GraphedCall(make) if graph else make(stream)
 
     def decode_lse(self, q: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float,
                    out: torch.Tensor, lse: torch.Tensor, stream=None):

@@ -604,9 +604,10 @@ struct HostStaging {
 
 static bool host_staging(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                          int32_t head_dim, int32_t max_ctx, tq_dtype q_dtype, tq_dtype kv_dtype,
-                         HostStaging* hs) {
+                         PlanKind kind, HostStaging* hs) {
   DecodePlan p;
-  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p)) return false;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &p, kind))
+    return false;
   if ((q_dtype != TQ_F32 && q_dtype != TQ_BF16) || (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16))
     return false;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -625,7 +626,31 @@ size_t tq_decode_append_host_workspace_bytes(int32_t batch, int32_t num_q_heads,
                                              int32_t max_ctx, tq_dtype q_dtype,
                                              tq_dtype kv_dtype) {
   HostStaging hs;
-  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype, &hs))
+  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype,
+                    PlanKind::kInt4, &hs))
+    return 0;
+  return hs.total;
+}
+
+size_t tq_decode_append_host_srft_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                  int32_t num_kv_heads, int32_t head_dim,
+                                                  int32_t max_ctx, tq_dtype q_dtype,
+                                                  tq_dtype kv_dtype) {
+  HostStaging hs;
+  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype,
+                    PlanKind::kSrft, &hs))
+    return 0;
+  return hs.total;
+}
+
+size_t tq_decode_append_host_cb_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                int32_t num_kv_heads, int32_t head_dim,
+                                                int32_t max_ctx, tq_dtype q_dtype,
+                                                tq_dtype kv_dtype) {
+  HostStaging hs;
+  if (head_dim != 128 && head_dim != 256) return 0;
+  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype,
+                    PlanKind::kCodebook, &hs))
     return 0;
   return hs.total;
 }
@@ -665,22 +690,30 @@ static void* device_view(const void* p) {
 
 extern "C" {
 
-tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
-                                          const void* k_new_host, const void* v_new_host,
-                                          tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
-                                          int32_t num_kv_heads, int32_t head_dim, int32_t group,
-                                          uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
-                                          float* v_scales, int64_t capacity,
-                                          const int32_t* ctx_lens, int32_t max_ctx,
-                                          const int8_t* signs, float attn_scale, float* out_host,
-                                          void* workspace, size_t workspace_bytes,
-                                          void* cuda_stream) {
+}  // extern "C"
+
+// The fused step with its inputs and output in host memory, for every cache
+// format (rot): mapped host buffers through the gather kernel and direct
+// output writes, else staging copies (see include/tq.h).
+static tq_status host_step(const void* q_host, tq_dtype q_dtype, const void* k_new_host,
+                           const void* v_new_host, tq_dtype kv_dtype, int32_t batch,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t group, uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                           float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+                           int32_t max_ctx, const int8_t* signs, float attn_scale,
+                           float* out_host, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream, const char* where, const Rotation& rot) {
   if (!q_host || !k_new_host || !v_new_host || !out_host) return TQ_ERR_INVALID_ARG;
+  const PlanKind kind = rot.srft ? PlanKind::kSrft
+                        : rot.cb_bits ? PlanKind::kCodebook
+                                      : PlanKind::kInt4;
   HostStaging hs;
-  if (!host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype, &hs)) {
+  if ((kind == PlanKind::kCodebook && head_dim != 128 && head_dim != 256) ||
+      !host_staging(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, q_dtype, kv_dtype, kind,
+                    &hs)) {
     if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
     if (kv_dtype != TQ_F32 && kv_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
-    if (head_dim != 128 && head_dim != 256) return TQ_ERR_UNSUPPORTED;
+    if (!head_dim_ok(head_dim, rot)) return TQ_ERR_UNSUPPORTED;
     return TQ_ERR_INVALID_ARG;
   }
   if (!workspace || workspace_bytes < hs.total) return TQ_ERR_WORKSPACE;
@@ -710,11 +743,62 @@ tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
       ws + hs.q, q_dtype, ws + hs.k, ws + hs.v, kv_dtype, batch, num_q_heads, num_kv_heads,
       head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens, max_ctx, signs,
       attn_scale, mapped ? static_cast<float*>(dout) : reinterpret_cast<float*>(ws + hs.out),
-      workspace, hs.q, cuda_stream, "tq_sdpa_int4_decode_append_host", nullptr, Rotation{}, &hin);
+      workspace, hs.q, cuda_stream, where, nullptr, rot, &hin);
   if (st != TQ_OK || mapped) return st;
-  if (st != TQ_OK) return st;
   return cuda_status(cudaMemcpyAsync(out_host, ws + hs.out, out_bytes, cudaMemcpyDeviceToHost, s),
-                     "tq_sdpa_int4_decode_append_host");
+                     where);
+}
+
+extern "C" {
+
+tq_status tq_sdpa_int4_decode_append_host(const void* q_host, tq_dtype q_dtype,
+                                          const void* k_new_host, const void* v_new_host,
+                                          tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim, int32_t group,
+                                          uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+                                          float* v_scales, int64_t capacity,
+                                          const int32_t* ctx_lens, int32_t max_ctx,
+                                          const int8_t* signs, float attn_scale, float* out_host,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* cuda_stream) {
+  return host_step(q_host, q_dtype, k_new_host, v_new_host, kv_dtype, batch, num_q_heads,
+                   num_kv_heads, head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity,
+                   ctx_lens, max_ctx, signs, attn_scale, out_host, workspace, workspace_bytes,
+                   cuda_stream, "tq_sdpa_int4_decode_append_host", Rotation{});
+}
+
+tq_status tq_sdpa_int4_decode_append_srft_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales,
+    int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+    const float* lambda_k, const float* lambda_v, float attn_scale, float* out_host,
+    void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  Rotation r;
+  r.srft = true;
+  r.lambda_k = lambda_k;
+  r.lambda_v = lambda_v;
+  return host_step(q_host, q_dtype, k_new_host, v_new_host, kv_dtype, batch, num_q_heads,
+                   num_kv_heads, head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity,
+                   ctx_lens, max_ctx, signs, attn_scale, out_host, workspace, workspace_bytes,
+                   cuda_stream, "tq_sdpa_int4_decode_append_srft_host", r);
+}
+
+tq_status tq_sdpa_cb_decode_append_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out_host, void* workspace,
+    size_t workspace_bytes, void* cuda_stream) {
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  return host_step(q_host, q_dtype, k_new_host, v_new_host, kv_dtype, batch, num_q_heads,
+                   num_kv_heads, head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity,
+                   ctx_lens, max_ctx, signs, attn_scale, out_host, workspace, workspace_bytes,
+                   cuda_stream, "tq_sdpa_cb_decode_append_host", r);
 }
 
 tq_status tq_sdpa_int4_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,

@@ -383,6 +383,21 @@ TQ_API tq_status tq_sdpa_int4_decode_append_srft(
     const float* lambda_v, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
     void* cuda_stream);
 
+/* tq_sdpa_int4_decode_append_srft with q, k_new, v_new and out in HOST memory,
+ * as tq_sdpa_int4_decode_append_host (the same mapped-buffer and staging
+ * forms); workspace_bytes >= tq_decode_append_host_srft_workspace_bytes(). */
+TQ_API size_t tq_decode_append_host_srft_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                         int32_t num_kv_heads, int32_t head_dim,
+                                                         int32_t max_ctx, tq_dtype q_dtype,
+                                                         tq_dtype kv_dtype);
+TQ_API tq_status tq_sdpa_int4_decode_append_srft_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales,
+    int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx, const int8_t* signs,
+    const float* lambda_k, const float* lambda_v, float attn_scale, float* out_host,
+    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 /*
  * Codebook variant (the AdapTQ post, sections "unified SIMD pipeline",
  * "precomputed lookup tables", "performance and quality": 2-, 3- and 4-bit
@@ -450,6 +465,21 @@ TQ_API tq_status tq_sdpa_cb_decode_append(
     float* v_scales, int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx,
     const int8_t* signs, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
     void* cuda_stream);
+
+/* tq_sdpa_cb_decode_append with q, k_new, v_new and out in HOST memory, as
+ * tq_sdpa_int4_decode_append_host (the same mapped-buffer and staging forms);
+ * workspace_bytes >= tq_decode_append_host_cb_workspace_bytes(). */
+TQ_API size_t tq_decode_append_host_cb_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                       int32_t num_kv_heads, int32_t head_dim,
+                                                       int32_t max_ctx, tq_dtype q_dtype,
+                                                       tq_dtype kv_dtype);
+TQ_API tq_status tq_sdpa_cb_decode_append_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out_host, void* workspace,
+    size_t workspace_bytes, void* cuda_stream);
 
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);

@@ -229,3 +229,54 @@ def test_host_buffer_step_fallbacks_and_dtypes(case):
     for a, b in zip((caches[0].k_packed, caches[0].k_scales, caches[0].v_packed, caches[0].v_scales),
                     (caches[1].k_packed, caches[1].k_scales, caches[1].v_packed, caches[1].v_scales)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("kind", ["srft", "cb2", "cb3"])
+def test_host_buffer_step_srft_and_codebook(kind):
+    """The host-buffer step of the SRFT and codebook caches (pinned buffers:
+    gather kernel and direct output writes; then graph replay) equals their
+    device-buffer step bit for bit, cache rows included."""
+    require_cuda()
+    from compressed_domain_attention_tq_b200 import CodebookKVCache, Int4KVCache
+    B, Hkv, G, d, T = 2, 2, 8, 128, 500
+    g = torch.Generator().manual_seed(96)
+    k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
+    signs = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
+
+    def make():
+        if kind == "srft":
+            lk = torch.rand(d, generator=g) * 0.5 + 0.75
+            lv = torch.rand(d, generator=g) * 0.5 + 0.75
+            return Int4KVCache(B, Hkv, d, T + 2, signs=signs, rotation="srft",
+                               lambda_k=lk, lambda_v=lv)
+        return CodebookKVCache(B, Hkv, d, T + 2, int(kind[2]), signs=signs)
+
+    gstate = g.get_state()
+    caches = []
+    for _ in range(3):
+        g.set_state(gstate)
+        c = make()
+        c.append(k, v, torch.zeros(B, dtype=torch.int32, device="cuda"))
+        caches.append(c)
+    q = torch.randn(B, Hkv * G, d, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, Hkv, 1, d, generator=g).to(torch.bfloat16)
+    ctx = torch.tensor([T + 1, T - 30], dtype=torch.int32, device="cuda")
+    outs = []
+    for i, graph in enumerate((False, True)):
+        hq, hk, hv = q.pin_memory(), kn.pin_memory(), vn.pin_memory()
+        hout = torch.zeros(B, Hkv * G, d, dtype=torch.float32).pin_memory()
+        step = caches[i].bind_decode_append_host(hq, hk, hv, ctx, T + 2, hout, 0.1, graph=graph)
+        step()
+        torch.cuda.synchronize()
+        outs.append(hout.clone())
+    out_d = caches[2].decode_append(q.cuda(), kn.cuda(), vn.cuda(), ctx, T + 2, 0.1)
+    torch.cuda.synchronize()
+    for o in outs:
+        assert torch.equal(o, out_d.cpu())
+    for c in caches[:2]:
+        for a, b in zip((c.k_packed, c.k_scales, c.v_packed, c.v_scales),
+                        (caches[2].k_packed, caches[2].k_scales, caches[2].v_packed,
+                         caches[2].v_scales)):
+            assert torch.equal(a, b)
