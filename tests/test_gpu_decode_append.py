@@ -231,14 +231,16 @@ def test_host_buffer_step_fallbacks_and_dtypes(case):
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("kind", ["srft", "cb2", "cb3"])
-def test_host_buffer_step_srft_and_codebook(kind):
+@pytest.mark.parametrize("kind,G,d", [("srft", 8, 128), ("cb2", 8, 128), ("cb3", 8, 128),
+                                       ("srft", 4, 96), ("cb2", 2, 128)])
+def test_host_buffer_step_srft_and_codebook(kind, G, d):
     """The host-buffer step of the SRFT and codebook caches (pinned buffers:
     gather kernel and direct output writes; then graph replay) equals their
-    device-buffer step bit for bit, cache rows included."""
+    device-buffer step bit for bit, cache rows included, on the tensor-core
+    decode and (d = 96, two heads per kv head) on the CUDA-core decode."""
     require_cuda()
     from compressed_domain_attention_tq_b200 import CodebookKVCache, Int4KVCache
-    B, Hkv, G, d, T = 2, 2, 8, 128, 500
+    B, Hkv, T = 2, 2, 500
     g = torch.Generator().manual_seed(96)
     k = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
     v = torch.randn(B, Hkv, T, d, generator=g).to(torch.bfloat16).cuda()
