@@ -264,3 +264,37 @@ def test_host_step_rejects_on_host(lib):
     assert call(d=96) == _lib.TQ_ERR_UNSUPPORTED
     assert call(qd=7) == _lib.TQ_ERR_INVALID_ARG
     assert call(ws_bytes=need - 1) == _lib.TQ_ERR_WORKSPACE
+
+
+def test_variant_host_steps_reject_on_host(lib):
+    """The SRFT and codebook host-buffer steps validate like the int4 one
+    before anything is enqueued."""
+    fb = FakeBuffers()
+    need_s = lib.tq_decode_append_host_srft_workspace_bytes(1, 8, 2, 96, 64, 1, 1)
+    need_c = lib.tq_decode_append_host_cb_workspace_bytes(1, 8, 2, 128, 64, 1, 1)
+    assert need_s > 0 and need_c > 0
+    assert lib.tq_decode_append_host_srft_workspace_bytes(1, 8, 2, 80, 64, 1, 1) == 0
+    assert lib.tq_decode_append_host_cb_workspace_bytes(1, 8, 2, 96, 64, 1, 1) == 0
+
+    def srft(q=fb.p(0), out=fb.p(4096), ws_bytes=1 << 16, d=96):
+        return lib.tq_sdpa_int4_decode_append_srft_host(
+            q, 1, fb.p(8192), fb.p(12288), 1, 1, 8, 2, d, 32, fb.p(1024), fb.p(2048), fb.p(3072),
+            fb.p(4096), 64, fb.p(512), 64, None, None, None, 0.125, out, fb.p(16384), ws_bytes,
+            None)
+
+    assert srft(q=None) == _lib.TQ_ERR_INVALID_ARG
+    assert srft(out=None) == _lib.TQ_ERR_INVALID_ARG
+    assert srft(d=80) == _lib.TQ_ERR_UNSUPPORTED
+    assert srft(ws_bytes=need_s - 1) == _lib.TQ_ERR_WORKSPACE
+
+    def cb(bits=2, levels=fb.p(256), ws_bytes=1 << 16, d=128, q=fb.p(0)):
+        return lib.tq_sdpa_cb_decode_append_host(
+            q, 1, fb.p(8192), fb.p(12288), 1, 1, 8, 2, d, 32, bits, levels, fb.p(1024), fb.p(2048),
+            fb.p(3072), fb.p(4096), 64, fb.p(512), 64, None, 0.125, fb.p(4096), fb.p(16384),
+            ws_bytes, None)
+
+    assert cb(bits=5) == _lib.TQ_ERR_UNSUPPORTED
+    assert cb(d=96) == _lib.TQ_ERR_UNSUPPORTED
+    assert cb(q=None) == _lib.TQ_ERR_INVALID_ARG
+    assert cb(ws_bytes=need_c - 1) == _lib.TQ_ERR_WORKSPACE
+    assert cb(levels=None) == _lib.TQ_ERR_INVALID_ARG
