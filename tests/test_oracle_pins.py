@@ -646,6 +646,23 @@ def test_cb_decode_brute_force_rotation_off(bits):
             np.testing.assert_allclose(out[b, h], want, rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("bits,mul,off", [(2, 1e3, 0.3), (3, 1e-3, -0.2), (4, 37.0, 0.05)])
+def test_cb_decode_custom_levels_brute_force(bits, mul, off):
+    """Levels other than the Gaussian codebook (shifted, far from 1 in
+    magnitude): the decode is still attention over sigma * C[index]."""
+    rng = np.random.default_rng(bits + 60)
+    B, Hkv, G, T, d = 1, 2, 2, 13, 64
+    c = ((oracle.lloyd_max_gaussian(bits) + off) * mul).astype(np.float32)
+    assert np.all(np.diff(c) > 0)
+    cache, khat, vhat = _random_cb_cache(rng, B, Hkv, T, d, bits, c)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    scale = 0.05 / mul
+    out = oracle.sdpa_cb_decode(q, cache, [T], None, bits, c, scale, Hkv)
+    for h in range(Hkv * G):
+        want = _numpy_attention(q[0, h].astype(np.float64), khat[0, h // G], vhat[0, h // G], scale)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-11, atol=1e-12 * max(1.0, mul))
+
+
 def test_cb_decode_rotation_on_is_attention_in_unrotated_basis():
     rng = np.random.default_rng(44)
     d, Hkv, G, T, bits = 64, 1, 2, 9, 3
