@@ -573,6 +573,24 @@ def test_cb_quantizer_is_nearest_level_with_rms_scale(bits):
             np.testing.assert_array_equal(idx[r, 32 * g:32 * g + 32], want)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_cb_quantizer_custom_levels_is_nearest_level(bits):
+    """With any increasing levels (here uneven and asymmetric) the index is the
+    nearest level to the clipped, rms-scaled coordinate."""
+    rng = np.random.default_rng(bits + 70)
+    c = np.sort(rng.uniform(-2.6, 2.2, 1 << bits)).astype(np.float32)
+    y = (rng.standard_normal((100, 64)) * np.exp(rng.uniform(-3, 3, (100, 1)))).astype(np.float32)
+    idx, sc = oracle.cb_quantize_vectors(y, bits, c)
+    for r in range(100):
+        for g in range(2):
+            yg = y[r, 32 * g:32 * g + 32]
+            s = _rms_sigma(yg)
+            assert sc[r, g] == s
+            u = np.clip((yg / s).astype(np.float32), -3, 3).astype(np.float64)
+            want = np.argmin(np.abs(u[:, None] - c[None, :].astype(np.float64)), axis=1)
+            np.testing.assert_array_equal(idx[r, 32 * g:32 * g + 32], want)
+
+
 def test_cb_quantizer_tie_and_zero_group_take_the_lower_level():
     c = oracle.lloyd_max_gaussian(2).astype(np.float32)        # middle threshold is exactly 0
     y = np.zeros((2, 32), np.float32)
