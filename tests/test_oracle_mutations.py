@@ -49,6 +49,11 @@ MUTATIONS = {
     "lloyd_cell_mean_sign": ("double m = (pa - pb) / (cb - ca);", "double m = (pb - pa) / (cb - ca);"),
     "cb_value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP] * (double)C[ci[i]]",
                                    "(double)sv[0] * (double)C[ci[i]]"),
+    # mistakes that only show with levels that are not symmetric about zero
+    "cb_threshold_assumes_symmetric": ("volatile float sum = C[i] + C[i + 1];",
+                                       "volatile float sum = C[i] - C[L - 2 - i];"),
+    "cb_score_level_mirrored": ("(double)sk[i / ORACLE_GROUP] * (double)C[ci[i]]",
+                                "(double)sk[i / ORACLE_GROUP] * -(double)C[(1 << bits) - 1 - ci[i]]"),
 }
 
 
