@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--decode-kernel", choices=["mma_sync", "tcgen05"], default="mma_sync",
+                    help="int4 decode kernel at head_dim 128 (mma_sync: the default; tcgen05: "
+                         "the tensor-memory kernel, for comparison)")
     return ap.parse_args()
 
 
@@ -175,6 +178,8 @@ def run_tq(args):
 
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", torch.cuda.current_device())
+    from compressed_domain_attention_tq_b200 import _lib
+    _lib.set_test_hooks(_lib.TEST_HOOK_TCGEN05_DECODE if args.decode_kernel == "tcgen05" else 0)
     w = wl.WORKLOADS[args.workload]
     seed = args.seed + 1000 * rank
     B, Hq, Hkv, d, T = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.context
@@ -400,7 +405,7 @@ def run_tq(args):
         "dtype": (f"{w.cb_bits}-bit codebook indices, fp32 accumulation" if w.cb_bits
                   else "int4 codes, fp32 accumulation"), "data": "synthetic (seeded N(0,1), bf16)",
         "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
-                   "context": max_ctx,
+                   "context": max_ctx, "decode_kernel": args.decode_kernel,
                    "rotation": (w.rotation_kind if w.rotation else False),
                    "codes": f"{w.cb_bits}-bit Max-Lloyd codebook" if w.cb_bits else "int4",
                    "attn_scale": scale,

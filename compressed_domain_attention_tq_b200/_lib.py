@@ -118,12 +118,25 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_cb_decode_append_host.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
+    lib.tq_set_test_hooks.argtypes = [ctypes.c_uint32]
+    lib.tq_set_test_hooks.restype = None
     _lib = lib
     return lib
 
 
 def status_string(status: int) -> str:
     return load().tq_status_string(status).decode()
+
+
+# tq_set_test_hooks bits (include/tq.h); testing and kernel comparisons only
+TEST_HOOK_FAIL_LAUNCH = 1
+TEST_HOOK_STARVE_PIPELINE = 2
+TEST_HOOK_TCGEN05_DECODE = 4
+
+
+def set_test_hooks(hooks: int) -> None:
+    """Process-wide test switches of libtq (0 = normal operation)."""
+    load().tq_set_test_hooks(int(hooks))
 
 
 def _ptr(t):

@@ -1239,7 +1239,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
 template <int D, int PATH, int FMT>
 cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
   using C = Cfg<D, PATH, FMT>;
-  static std::atomic<uint64_t> smem_set{0};
+  static SmemLimitSet smem_set;
   const cudaError_t e = ensure_smem_limit(decode_mma_kernel<D, PATH, FMT>, C::BYTES, smem_set);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = kSmCount;

@@ -540,7 +540,7 @@ template <int D, int FMT = 0>
 cudaError_t launch_simt_d(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   dim3 grid(a.plan.n_chunks, a.Hkv, a.B);
-  static std::atomic<uint64_t> smem_set{0};
+  static SmemLimitSet smem_set;
   const cudaError_t e =
       ensure_smem_limit(decode_simt_kernel<D, FMT>, (int)simt_smem_max<D, FMT>(), smem_set);
   if (e != cudaSuccess) return e;

@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(QHalf::THREADS, 1) quantize_half_kernel(Quanti
 
 template <bool ROT>
 cudaError_t launch_half(const QuantizeArgs& a, cudaStream_t stream) {
-  static std::atomic<uint64_t> smem_set{0};
+  static SmemLimitSet smem_set;
   const cudaError_t e = ensure_smem_limit(quantize_half_kernel<ROT>, QHalf::BYTES, smem_set);
   if (e != cudaSuccess) return e;
   const int64_t nbatch = (2LL * a.B * a.Hkv * a.n_new + 15) / 16;
@@ -608,7 +608,7 @@ cudaError_t launch_half(const QuantizeArgs& a, cudaStream_t stream) {
 template <int D, bool BF16, bool ROT>
 cudaError_t launch_q(const QuantizeArgs& a, cudaStream_t stream) {
   using Q = QCfg<BF16>;
-  static std::atomic<uint64_t> smem_set{0};
+  static SmemLimitSet smem_set;
   const cudaError_t e = ensure_smem_limit(quantize_staged_kernel<D, BF16, ROT>, Q::BYTES, smem_set);
   if (e != cudaSuccess) return e;
   const int64_t nbatch = (2LL * a.B * a.Hkv * a.n_new + 32 / (D / 128) - 1) / (32 / (D / 128));

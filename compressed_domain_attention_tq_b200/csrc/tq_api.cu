@@ -7,12 +7,52 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/tq.h"
 #include "tq_internal.h"
 
 namespace tq {
 
 static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Driver entry points for the context identity, looked up once through the
+// runtime (libtq links no driver library).
+namespace {
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxFns& ctx_fns() {
+  static const CtxFns fns = [] {
+    CtxFns f;
+    cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p1, 4000, cudaEnableDefault, &q1) ==
+            cudaSuccess &&
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &p2, 12000, cudaEnableDefault, &q2) ==
+            cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess && q2 == cudaDriverEntryPointSuccess) {
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p1);
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p2);
+    }
+    return f;
+  }();
+  return fns;
+}
+}  // namespace
+
+bool current_context_id(unsigned long long* id) {
+  const CtxFns& f = ctx_fns();
+  if (f.get_current == nullptr || f.get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return f.get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Test hooks (bits of tq_set_test_hooks), off unless a test turns them on.
+std::atomic<unsigned> g_test_hooks{0};
 
 // Split the context into chunks (multiples of the decode's pipeline stage,
 // 192 or 128 tokens): pick the chunk count per sequence that minimises
@@ -119,6 +159,8 @@ static bool codebook_ok(const Rotation& rot) {
 using namespace tq;
 
 extern "C" {
+
+void tq_set_test_hooks(uint32_t hooks) { g_test_hooks.store(hooks, std::memory_order_relaxed); }
 
 const char* tq_status_string(tq_status status) {
   switch (status) {
@@ -350,11 +392,12 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     return TQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < a.plan.ws_bytes) return TQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return TQ_ERR_INVALID_ARG;
-  // Test hooks (environment): TQ_TEST_FAIL_LAUNCH fails the call as a failed launch would,
-  // before anything is enqueued; TQ_TEST_STARVE_PIPELINE makes the tensor-core decode's
-  // bounded waits for its first copies run out (its outputs are then NaN).
-  if (getenv("TQ_TEST_FAIL_LAUNCH")) return cuda_status(cudaErrorLaunchFailure, where);
-  a.test_starve = getenv("TQ_TEST_STARVE_PIPELINE") != nullptr;
+  // Test hooks (tq_set_test_hooks; off in normal use): fail the call as a failed launch
+  // would, before anything is enqueued; or make the tensor-core decode's bounded waits for
+  // its first copies run out (its outputs are then NaN).
+  const unsigned hooks = g_test_hooks.load(std::memory_order_relaxed);
+  if (hooks & TQ_TEST_HOOK_FAIL_LAUNCH) return cuda_status(cudaErrorLaunchFailure, where);
+  a.test_starve = (hooks & TQ_TEST_HOOK_STARVE_PIPELINE) != 0;
   if (host_in != nullptr) {
     const cudaError_t e = move_host_inputs(*host_in, static_cast<cudaStream_t>(cuda_stream));
     if (e != cudaSuccess) return cuda_status(e, where);
@@ -449,7 +492,9 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     const cudaError_t e = launch_srft_query(a, s);
     if (e != cudaSuccess) return cuda_status(e, where);
   }
-  const cudaError_t e = mma ? launch_decode_mma(a, s) : launch_decode_simt(a, s);
+  const bool tc = rot.cb_bits == 0 && decode_tc_supported(head_dim, num_q_heads / num_kv_heads) &&
+                  (hooks & TQ_TEST_HOOK_TCGEN05_DECODE);
+  const cudaError_t e = tc ? launch_decode_tc(a, s) : mma ? launch_decode_mma(a, s) : launch_decode_simt(a, s);
   if (e != cudaSuccess) return cuda_status(e, where);
   return cuda_status(rot.srft ? launch_merge_srft(a, s) : launch_merge(a, s), where);
 }

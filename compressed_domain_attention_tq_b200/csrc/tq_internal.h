@@ -95,18 +95,36 @@ struct DecodeArgs {
                                     // dependent and waits for it before reading them
 };
 
-// Raise a kernel's dynamic shared memory limit once per device (the first
-// launch on each device), so later launches, including those made while a
-// stream is being captured into a CUDA graph, only enqueue work.
+// Identity of the CUDA context current on the calling thread: unique for the
+// life of the process (a device reset, or a context the caller creates with the
+// driver API, gives a new one).  Returns false when no context is current yet
+// (the runtime binds one on this thread's first runtime call) or the driver
+// cannot be queried.
+bool current_context_id(unsigned long long* id);
+
+// Test hooks set by tq_set_test_hooks (bits TQ_TEST_HOOK_*), read once per call.
+extern std::atomic<unsigned> g_test_hooks;
+
+// Contexts in which a kernel's dynamic shared memory limit has been raised.
+// Function attributes live in the context that loaded the kernel, so the
+// limit is raised once per context (the first launch there); later launches,
+// including those made while a stream is being captured into a CUDA graph,
+// only enqueue work.
+struct SmemLimitSet {
+  static constexpr int kSlots = 8;
+  std::atomic<unsigned long long> ctx[kSlots] = {};
+  std::atomic<unsigned> next{0};
+};
+
 template <typename Kernel>
-cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+cudaError_t ensure_smem_limit(Kernel kernel, int bytes, SmemLimitSet& done) {
+  unsigned long long id = 0;
+  if (current_context_id(&id))
+    for (int i = 0; i < SmemLimitSet::kSlots; ++i)
+      if (done.ctx[i].load(std::memory_order_acquire) == id) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && (id != 0 || current_context_id(&id)))
+    done.ctx[done.next.fetch_add(1) % SmemLimitSet::kSlots].store(id, std::memory_order_release);
   return e;
 }
 
@@ -117,6 +135,9 @@ bool decode_mma_supported(int d, int G);
 bool decode_mma_cb_supported(int d, int G);  // codebook caches on the tensor-core decode
 int decode_stage_tokens(int d, int G);  // tokens per pipeline stage of the decode path
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
+bool decode_tc_supported(int d, int G);  // the tcgen05 decode (int4 cache, d = 128, G <= 8)
+int decode_tc_tile_tokens();
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 bool srft_head_dim_supported(int d);
 cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream);

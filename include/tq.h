@@ -481,6 +481,25 @@ TQ_API tq_status tq_sdpa_cb_decode_append_host(
     int32_t max_ctx, const int8_t* signs, float attn_scale, float* out_host, void* workspace,
     size_t workspace_bytes, void* cuda_stream);
 
+/*
+ * tq_set_test_hooks -- testing only; leave at 0 (the default) in normal use.
+ * Sets process-wide switches read once by every later decode call:
+ *  - TQ_TEST_HOOK_FAIL_LAUNCH: decode calls return TQ_ERR_CUDA after
+ *    validation, before enqueueing anything (as a failed launch would).
+ *  - TQ_TEST_HOOK_STARVE_PIPELINE: the tensor-core decode kernels withhold
+ *    each CTA's first copy, so their bounded waits run out (about 2 s); the
+ *    call's outputs are then NaN and the context stays usable.
+ *  - TQ_TEST_HOOK_TCGEN05_DECODE: the int4 decode at head_dim 128 with up to
+ *    8 query heads per kv head runs on the tcgen05 / tensor-memory kernel
+ *    instead of the default warp-level mma.sync kernel (for comparing the
+ *    two; the default is the faster one on B200 for this decode).
+ * No counterpart on the method's pages.
+ */
+#define TQ_TEST_HOOK_FAIL_LAUNCH 1u
+#define TQ_TEST_HOOK_STARVE_PIPELINE 2u
+#define TQ_TEST_HOOK_TCGEN05_DECODE 4u
+TQ_API void tq_set_test_hooks(uint32_t hooks);
+
 /* tq_status_string -- static English text for a status code. */
 TQ_API const char* tq_status_string(tq_status status);
 

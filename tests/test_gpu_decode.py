@@ -176,7 +176,7 @@ def test_decode_zero_v_prefix(d, G):
         check_attention(got, want, cache, [T], G, f"zero V prefix d={d} G={G}")
 
 
-def test_injected_launch_failure_enqueues_nothing(monkeypatch):
+def test_injected_launch_failure_enqueues_nothing():
     """Host-side fault injection: the call reports TQ_ERR_CUDA and leaves the output alone."""
     require_cuda()
     B, Hkv, G, d, T = 1, 2, 8, 128, 300
@@ -184,16 +184,20 @@ def test_injected_launch_failure_enqueues_nothing(monkeypatch):
     cache = upload_cache(oracle_cache(k, v, None))
     ws = torch.empty(_lib.decode_workspace_bytes(B, Hkv * G, Hkv, d, T), dtype=torch.uint8, device="cuda")
     out = torch.full((B, Hkv * G, d), 7.0, device="cuda")
-    monkeypatch.setenv("TQ_TEST_FAIL_LAUNCH", "1")
-    with pytest.raises(_lib.TQError) as err:
-        _lib.sdpa_int4_decode(q.cuda(), *cache, torch.tensor([T], dtype=torch.int32, device="cuda"), T,
-                              None, 0.1, out, ws)
+    _lib.set_test_hooks(_lib.TEST_HOOK_FAIL_LAUNCH)
+    try:
+        with pytest.raises(_lib.TQError) as err:
+            _lib.sdpa_int4_decode(q.cuda(), *cache, torch.tensor([T], dtype=torch.int32, device="cuda"), T,
+                                  None, 0.1, out, ws)
+    finally:
+        _lib.set_test_hooks(0)
     assert err.value.status == _lib.TQ_ERR_CUDA
     torch.cuda.synchronize()
     assert torch.all(out == 7.0)
 
 
-def test_starved_pipeline_gives_up_and_context_stays_usable(monkeypatch):
+@pytest.mark.parametrize("hooks", [0, 4], ids=["mma_sync", "tcgen05"])
+def test_starved_pipeline_gives_up_and_context_stays_usable(hooks):
     """The tensor-core decode's waits for its copies are bounded: with each CTA's
     first copy withheld (test hook), the waits run out after about two seconds, the
     kernel ends, the heads' outputs are NaN, and the next call on the same context
@@ -203,10 +207,15 @@ def test_starved_pipeline_gives_up_and_context_stays_usable(monkeypatch):
     k, v, q = make_case(B, Hkv, G, d, T, torch.bfloat16, 62)
     cache = oracle_cache(k, v, None)
     dev = upload_cache(cache)
-    monkeypatch.setenv("TQ_TEST_STARVE_PIPELINE", "1")
-    got, _ = run_decode(dev, q, [T], T, None, 0.1, Hkv)
+    _lib.set_test_hooks(hooks | _lib.TEST_HOOK_STARVE_PIPELINE)
+    try:
+        got, _ = run_decode(dev, q, [T], T, None, 0.1, Hkv)
+    finally:
+        _lib.set_test_hooks(hooks)
     assert np.all(np.isnan(got))
-    monkeypatch.delenv("TQ_TEST_STARVE_PIPELINE")
-    got, flags = run_decode(dev, q, [T], T, None, 0.1, Hkv)
+    try:
+        got, flags = run_decode(dev, q, [T], T, None, 0.1, Hkv)
+    finally:
+        _lib.set_test_hooks(0)
     want = oracle.sdpa_int4_decode(to_oracle(q), cache, [T], None, 0.1, Hkv, threads=THREADS)
     check_attention(got, want, cache, [T], G, "after a starved call")
