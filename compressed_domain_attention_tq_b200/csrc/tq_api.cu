@@ -354,6 +354,37 @@ static cudaError_t move_host_inputs(const HostInputs& h, cudaStream_t s) {
   return e;
 }
 
+namespace tq {
+
+// The checks tq_sdpa_int4_decode makes before it looks at the workspace, in
+// the same order and with the same results (used by the static-scratch call,
+// which must report invalid arguments before its own size limit).
+tq_status validate_decode_args(const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t group,
+                               const uint8_t* k_packed, const float* k_scales, const uint8_t* v_packed,
+                               const float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+                               int32_t max_ctx, float attn_scale, const float* out) {
+  if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !ctx_lens || !out)
+    return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (batch < 1 || num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads != 0)
+    return TQ_ERR_INVALID_ARG;
+  if (max_ctx < 1 || capacity < max_ctx) return TQ_ERR_INVALID_ARG;
+  if (!(attn_scale > 0.0f) || !isfinite(attn_scale)) return TQ_ERR_INVALID_ARG;
+  if (!head_dim_ok(head_dim, Rotation{})) return TQ_ERR_UNSUPPORTED;
+  if (group != kGroup) return TQ_ERR_UNSUPPORTED;
+  if (num_q_heads / num_kv_heads > 16) return TQ_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_packed) || !aligned16(v_packed) ||
+      !aligned16(k_scales) || !aligned16(v_scales))
+    return TQ_ERR_INVALID_ARG;
+  DecodePlan plan;
+  if (!make_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, max_ctx, &plan))
+    return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
+}  // namespace tq
+
 static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new,
                              tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads,
                              int32_t num_kv_heads, int32_t head_dim, int32_t group,

@@ -7,6 +7,8 @@
 
 #include <atomic>
 
+#include "../../include/tq.h"
+
 namespace tq {
 
 constexpr int kGroup = 32;  // quantization group (rotated coordinates)
@@ -101,6 +103,14 @@ struct DecodeArgs {
 // (the runtime binds one on this thread's first runtime call) or the driver
 // cannot be queried.
 bool current_context_id(unsigned long long* id);
+
+// The argument checks of tq_sdpa_int4_decode that precede the workspace check
+// (returns TQ_OK or that call's error status).
+tq_status validate_decode_args(const void* q, tq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t group, const uint8_t* k_packed,
+                         const float* k_scales, const uint8_t* v_packed, const float* v_scales,
+                         int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx, float attn_scale,
+                         const float* out);
 
 // Test hooks set by tq_set_test_hooks (bits TQ_TEST_HOOK_*), read once per call.
 extern std::atomic<unsigned> g_test_hooks;

@@ -20,6 +20,7 @@ MUTATIONS = {
     "output_not_inverse_rotated": ("acc += O[(int64_t)j * d + i] * orot[i];",
                                    "acc += O[(int64_t)i * d + j] * orot[i];"),
     "signs_applied_after_hadamard": ("* (double)signs[j];", "* (double)signs[i];"),
+    "append_leaves_rotation_off": ("n_new, d, pos, R, R, k_packed", "n_new, d, pos, NULL, NULL, k_packed"),
     "value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP] * (double)codes[i]",
                                 "(double)sv[0] * (double)codes[i]"),
     "gqa_map_modulo": ("hk = hq / G;\n    int64_t T = ctx_lens[b];\n    double qv[512], qr[512], orot[512];\n    int8_t codes",

@@ -373,6 +373,35 @@ def test_end_to_end_on_grid_rotation_off_is_exact_attention():
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
 
 
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_end_to_end_on_grid_hadamard_rotation_is_exact_attention(d):
+    """K and V are built so that their rotated images R x (R = H diag(signs) /
+    sqrt(d), H from the Sylvester recursion above, not the oracle's) lie on the
+    int4 grid: quantize-append with rotation on must store exactly those codes,
+    and decode must give the unquantized attention over the original vectors.
+    Catches signs applied after H instead of before, a transposed rotation, a
+    missing 1/sqrt(d) in either direction and a query left unrotated."""
+    rng = np.random.default_rng(d + 1)
+    B, Hkv, G, T = 1, 2, 3, 11
+    s = rand_signs(rng, d)
+    R = sylvester(d) * s.astype(np.float64)[None, :] / np.sqrt(d)
+    c = rng.integers(-7, 8, (2, B, Hkv, T, d))
+    c[..., ::32] = 7                      # a full-scale code in every group
+    yk, yv = c[0] * 0.25, c[1] * 0.125
+    k = (yk @ R).astype(np.float32)       # x = R^T y, so R x = y
+    v = (yv @ R).astype(np.float32)
+    cache = oracle.empty_cache(B, Hkv, T, d)
+    oracle.quantize_append(k, v, [0], s, cache)
+    codes_k = oracle.unpack(cache[0].reshape(-1, d // 2), d).reshape(c[0].shape)
+    codes_v = oracle.unpack(cache[2].reshape(-1, d // 2), d).reshape(c[1].shape)
+    np.testing.assert_array_equal(codes_k, c[0])
+    np.testing.assert_array_equal(codes_v, c[1])
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    got = oracle.sdpa_int4_decode(q, cache, [T], s, 0.3, Hkv)
+    want = oracle.exact_attention(q, k, v, [T], 0.3)
+    np.testing.assert_allclose(got, want, rtol=2e-6, atol=2e-6 * np.abs(want).max())
+
+
 def test_exact_attention_brute_force():
     rng = np.random.default_rng(13)
     B, Hkv, G, T, d = 1, 2, 2, 9, 32
