@@ -13,10 +13,13 @@ line (rank 0).
 
 Timing: one CUDA graph of exactly K steps replayed between CUDA events on the
 launching stream (a second graph of K decodes splits the step into quantize-append
-and decode); no L2 flush when a step reads more bytes than the L2 holds, else a
-256 MiB write before each step whose separately timed cost is subtracted;
-barrier + synchronize around the timed region, max over ranks.  e2e: the same
-step through the public API with pinned host copies, timed per step.
+and decode).  The steps rotate over copies of the packed cache, as many as it
+takes for their bytes to exceed twice the L2, so no step reads bytes its
+predecessor left in the L2.  Barrier + synchronize around the timed region, max
+over ranks.  The per-step distribution (median, P95) comes from graphs of 10
+steps replayed at least 20 times between events.  e2e: the same step through the
+public API with host buffers, timed per step.  A "configs" block repeats the
+step measurement for the other synthetic configurations (1-GPU runs).
 """
 from __future__ import annotations
 
@@ -47,6 +50,7 @@ def parse():
     ap.add_argument("--workload", default="llama70b_gqa_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' block")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--decode-kernel", choices=["mma_sync", "tcgen05"], default="mma_sync",
                     help="int4 decode kernel at head_dim 128 (mma_sync: the default; tcgen05: "
@@ -61,6 +65,51 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def replica(cache):
+    """A second cache object holding copies of `cache`'s packed tensors (same
+    contents at other addresses), with its own workspace."""
+    import copy
+    c = copy.copy(cache)
+    for name in ("k_packed", "v_packed", "k_scales", "v_scales"):
+        setattr(c, name, getattr(cache, name).clone())
+    c._ws = None
+    return c
+
+
+def rotation_count(step_bytes, l2_bytes, cap_bytes=4 << 30, cache_bytes=None):
+    """Cache copies the timed steps rotate over: enough that the bytes read by
+    consecutive steps exceed twice the L2 (at least 2), within cap_bytes."""
+    n = max(2, -(-2 * l2_bytes // max(step_bytes, 1)))
+    if cache_bytes:
+        n = max(2, min(n, cap_bytes // cache_bytes))
+    return int(n)
+
+
+def window_times(torch, stream, fn, n_rot, windows, per_window):
+    """Per-step times (s) of `windows` replays of a graph of `per_window` calls
+    fn(i) (i rotating over n_rot caches), each replay between CUDA events."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(per_window):
+            fn(i % n_rot)
+    g.replay()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(windows + 1)]
+    evs[0].record(stream)
+    for r in range(windows):
+        g.replay()
+        evs[r + 1].record(stream)
+    torch.cuda.synchronize()
+    t = [evs[r].elapsed_time(evs[r + 1]) / 1e3 / per_window for r in range(windows)]
+    del g
+    return t
+
+
+def percentile(xs, p):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, max(0, int(math.ceil(p / 100.0 * len(xs))) - 1))]
 
 
 def kv_bytes(w, ctx_tokens):
@@ -238,41 +287,36 @@ def run_tq(args):
     scale = w.attn_scales[0]
     ws = cache.workspace(Hq, max_ctx)
 
-    def step():  # one decode step in one call: append the new token, then attend
-        cache.decode_append(q, k_new, v_new, ctx_dev, max_ctx, scale, out)
+    # The timed steps rotate over copies of the packed cache (same contents, other
+    # addresses), enough that consecutive steps' bytes exceed twice the L2: no step
+    # re-reads bytes its predecessor left in the L2.
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    kvb_step = kv_bytes(w, (ctx + 1).tolist())
+    n_rot = rotation_count(kvb_step, l2_bytes, cache_bytes=cache.nbytes())
+    caches = [cache] + [replica(cache) for _ in range(n_rot - 1)]
+    del flush
 
-    for i in range(args.warmup):
-        flush.fill_(i & 0xFF)
-        step()
+    def step(i):  # one decode step in one call: append the new token, then attend
+        caches[i].decode_append(q, k_new, v_new, ctx_dev, max_ctx, scale, out)
+
+    def dec(i):
+        caches[i].decode(q, ctx_dev, max_ctx, scale, out)
+
+    def two(i):  # the same step as two calls (append, then decode)
+        caches[i].append(k_new, v_new, pos)
+        caches[i].decode(q, ctx_dev, max_ctx, scale, out)
+
+    for i in range(max(args.warmup, n_rot)):
+        step(i % n_rot)
     torch.cuda.synchronize()
     # Device timing: one CUDA graph holds exactly K steps (quantize-append + decode),
     # replayed once between CUDA events, so per-launch host and graph-launch latency
-    # is amortised; a second graph of K decodes splits the step.  No L2 flush: the
-    # packed cache read by every step is larger than the L2 (stated in config).
-    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
-    kvb_step = kv_bytes(w, (ctx + 1).tolist())
-    use_flush = kvb_step <= l2_bytes  # else every step's reads already exceed the L2
-    g_step, g_dec, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    g_two = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        for i in range(args.steps):
-            if use_flush:
-                flush.fill_(i & 0xFF)
-            step()
-    with torch.cuda.graph(g_two):  # the same step as two calls (append, then decode)
-        for i in range(args.steps):
-            if use_flush:
-                flush.fill_(i & 0xFF)
-            cache.append(k_new, v_new, pos)
-            cache.decode(q, ctx_dev, max_ctx, scale, out)
-    with torch.cuda.graph(g_dec):
-        for i in range(args.steps):
-            if use_flush:
-                flush.fill_(i & 0xFF)
-            cache.decode(q, ctx_dev, max_ctx, scale, out)
-    with torch.cuda.graph(g_flush):
-        for i in range(args.steps if use_flush else 0):
-            flush.fill_(i & 0xFF)
+    # is amortised; a second graph of K decodes splits the step.
+    g_step, g_dec, g_two = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    for g, fn in ((g_step, step), (g_dec, dec), (g_two, two)):
+        with torch.cuda.graph(g):
+            for i in range(args.steps):
+                fn(i % n_rot)
     for i in range(max(1, args.warmup // args.steps + 1)):
         g_step.replay()
         g_dec.replay()
@@ -284,31 +328,31 @@ def run_tq(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     ev[0].record(stream)
     g_step.replay()
     ev[1].record(stream)
     g_dec.replay()
     ev[2].record(stream)
-    if use_flush:
-        g_flush.replay()
-    ev[3].record(stream)
     g_two.replay()
-    ev[4].record(stream)
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    # the per-step distribution: graphs of 10 steps, replayed >= 20 times
+    win = window_times(torch, stream, step, n_rot, max(20, args.steps // 10), 10)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
-    flush_s = ev[2].elapsed_time(ev[3]) / 1e3 / args.steps if use_flush else 0.0
-    step_s = ev[0].elapsed_time(ev[1]) / 1e3 / args.steps - flush_s
-    dec_s = ev[1].elapsed_time(ev[2]) / 1e3 / args.steps - flush_s
-    two_s = ev[3].elapsed_time(ev[4]) / 1e3 / args.steps - flush_s
+    step_s = ev[0].elapsed_time(ev[1]) / 1e3 / args.steps
+    dec_s = ev[1].elapsed_time(ev[2]) / 1e3 / args.steps
+    two_s = ev[2].elapsed_time(ev[3]) / 1e3 / args.steps
     q_s = max(step_s - dec_s, 0.0)
+    p50_s, p95_s = percentile(win, 50), percentile(win, 95)
     if world > 1:
-        tt = torch.tensor([step_s, dec_s, q_s, two_s], dtype=torch.float64, device=dev)
+        tt = torch.tensor([step_s, dec_s, q_s, two_s, p50_s, p95_s], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        step_s, dec_s, q_s, two_s = tt.tolist()
-    del g_step, g_dec, g_flush, g_two
+        step_s, dec_s, q_s, two_s, p50_s, p95_s = tt.tolist()
+    del g_step, g_dec, g_two
 
     # end to end through the C ABI with HOST buffers: the step's q, k_new, v_new and
     # output are pinned host tensors; tq_sdpa_int4_decode_append_host enqueues their
@@ -317,17 +361,14 @@ def run_tq(args):
     h_q, h_k, h_v = (t.cpu().pin_memory() for t in (q, k_new, v_new))
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v))
-    host_step = cache.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale,
-                                              graph=True)
+    host_steps = [c.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale, graph=True)
+                  for c in caches]
 
-    def e2e_step():
-        host_step()
     e2e_t = []
     for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xFF)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        e2e_step()
+        host_steps[i % n_rot]()
         b.record(stream)
         b.synchronize()
         if i >= args.warmup:
@@ -398,6 +439,8 @@ def run_tq(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
         "us_per_step": round(step_s * 1e6, 2), "decode_us": round(dec_s * 1e6, 2),
+        "p50_us": round(p50_s * 1e6, 2), "p95_us": round(p95_s * 1e6, 2),
+        "distribution": f"{len(win)} replays of a 10-step graph (per-step mean of each replay)",
         "append_in_step_us": round(q_s * 1e6, 2),
         "two_call_step_us": round(two_s * 1e6, 2),
         "pct_of_8TBps": round(100 * kvb / step_s / 1e9 / NOMINAL_HBM_GBS, 1),
@@ -410,10 +453,8 @@ def run_tq(args):
                    "codes": f"{w.cb_bits}-bit Max-Lloyd codebook" if w.cb_bits else "int4",
                    "attn_scale": scale,
                    "kv_bytes_per_step": kvb,
-                   "l2": (f"flushed by a {flush.numel()} B write before each step inside the "
-                          f"graph; its separately timed cost is subtracted") if use_flush else
-                         (f"not flushed: each step reads {kvb} B of packed cache, more than the "
-                          f"{l2_bytes} B L2"),
+                   "l2": (f"rotated over {n_rot} caches: consecutive steps read {n_rot * kvb} B "
+                          f"of packed cache, more than twice the {l2_bytes} B L2"),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm",
                      "kernel": (f"{w.cb_bits}-bit codebook decode (split-K + merge)" if w.cb_bits
@@ -439,6 +480,8 @@ def run_tq(args):
         "bf16_dequantize_then_attend": baseline,
         "fidelity_vs_unquantized_fp64": fid,
     }
+    if rank == 0 and world == 1 and not args.no_configs:
+        res["configs"] = measure_configs(args, dev, stream, seed, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, seed)
     if rank == 0:
@@ -446,6 +489,137 @@ def run_tq(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# The other synthetic configurations, each measured like the main workload's
+# step (rotation over cache copies, graph timing, windows for median / P95,
+# e2e through the host-buffer call): (workload, rotation on?, attn_scale index).
+CONFIGS = (("tiny_mha_4k", False, 0), ("tiny_mha_4k", True, 0), ("llama70b_gqa_32k", True, 0),
+           ("ragged_b16", True, 0), ("wide_d256", True, 0), ("wide_d256", True, 1))
+
+
+def measure_config(name, rot, scale_idx, args, dev, stream, seed, peak, want_fidelity=False):
+    """One configuration's decode step on this GPU: the fused append + decode
+    (tq_sdpa_int4_decode_append), the decode alone, their median and P95 over
+    graph replays, the host-buffer e2e step, and the decode's roofline fraction."""
+    import dataclasses
+
+    import torch
+
+    import compressed_domain_attention_tq_b200 as tq
+    from compressed_domain_attention_tq_b200 import workloads as wl
+    w = dataclasses.replace(wl.WORKLOADS[name], rotation=rot)
+    B, Hq, Hkv, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
+    scale = w.attn_scales[scale_idx]
+    signs = wl.make_signs(d, seed) if rot else None
+    ctx = wl.make_context_lengths(w, seed)
+    cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
+    k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
+    cache.append(k_all, v_all, torch.zeros(B, dtype=torch.int32, device=dev))
+    fid_in = None
+    k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
+    if want_fidelity:  # sequence 0's first two kv heads, unquantized, with the appended token
+        c0 = int(ctx[0])
+        fid_in = (torch.cat([k_all[0, :2, :c0], k_new[0, :2]], 1).float().cpu().numpy(),
+                  torch.cat([v_all[0, :2, :c0], v_new[0, :2]], 1).float().cpu().numpy())
+    del k_all, v_all
+    q = wl.make_query(w, seed, device=dev)
+    ctx_dev = (ctx + 1).to(dev)
+    max_ctx = int((ctx + 1).max())
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    kvb = kv_bytes(w, (ctx + 1).tolist())
+    n_rot = rotation_count(kvb, l2_bytes, cache_bytes=cache.nbytes())
+    caches = [cache] + [replica(cache) for _ in range(n_rot - 1)]
+
+    def step(i):
+        caches[i].decode_append(q, k_new, v_new, ctx_dev, max_ctx, scale, out)
+
+    def dec(i):
+        caches[i].decode(q, ctx_dev, max_ctx, scale, out)
+
+    steps = max(n_rot, 40 // n_rot * n_rot)
+    for i in range(max(args.warmup, n_rot)):
+        step(i % n_rot)
+    torch.cuda.synchronize()
+    res = {}
+    for key, fn in (("step", step), ("decode", dec)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(i % n_rot)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[key] = e0.elapsed_time(e1) / 1e3 / steps
+        del g
+    win = window_times(torch, stream, step, n_rot, 20, 10)
+    # e2e: the host-buffer step (pinned q, k_new, v_new in, output out), per step
+    h_q, h_k, h_v = (t.cpu().pin_memory() for t in (q, k_new, v_new))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hs = [c.bind_decode_append_host(h_q, h_k, h_v, ctx_dev, max_ctx, h_out, scale, graph=True)
+          for c in caches]
+    e2e = []
+    for i in range(args.warmup + 20):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        hs[i % n_rot]()
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e.append(a.elapsed_time(b) / 1e3)
+    algo = kvb + q.numel() * q.element_size() + out.numel() * out.element_size()
+    entry = {
+        "workload": w.name, "rotation": "hadamard" if rot else False, "attn_scale": scale,
+        "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "context_max": max_ctx,
+        "kv_bytes_per_step": kvb,
+        "us_per_step": round(res["step"] * 1e6, 2), "decode_us": round(res["decode"] * 1e6, 2),
+        "p50_us": round(percentile(win, 50) * 1e6, 2), "p95_us": round(percentile(win, 95) * 1e6, 2),
+        "kv_GB_per_s": round(kvb / res["step"] / 1e9, 1),
+        "roofline_frac": round(algo / res["decode"] / 1e9 / peak, 4),
+        "e2e_us": round(sum(e2e) / len(e2e) * 1e6, 2),
+        "l2": f"rotated over {n_rot} caches",
+    }
+    if want_fidelity:
+        caches[0].decode(q, ctx_dev, max_ctx, scale, out)
+        G = Hq // Hkv
+        entry["_fidelity_out"] = out[0, :2 * G].cpu().numpy()
+        entry["_fidelity_in"] = (fid_in, q[0, :2 * G].float().cpu().numpy(), signs, G)
+    del caches, hs
+    torch.cuda.synchronize()
+    return entry
+
+
+def measure_configs(args, dev, stream, seed, peak):
+    """The CONFIGS block, and the wide-head configuration's fidelity at
+    attn_scale 1.0 against 1/16 (directional error 1 - cosine to unquantized
+    attention, and their ratio)."""
+    import torch
+    entries, fid = [], {}
+    for name, rot, si in CONFIGS:
+        e = measure_config(name, rot, si, args, dev, stream, seed, peak, want_fidelity=name == "wide_d256")
+        if "_fidelity_out" in e:
+            (k_h, v_h), q_h, signs, G = e.pop("_fidelity_in")
+            o = e.pop("_fidelity_out")
+            Qm, _ = basis_maps(e["head_dim"], signs, None, None, False, torch.device("cpu"))
+            f = fidelity(k_h, v_h, q_h, o, None, Qm.numpy(), e["attn_scale"], G)
+            fid[e["attn_scale"]] = f
+            e["fidelity_vs_unquantized_fp64"] = f
+        entries.append(e)
+        torch.cuda.empty_cache()
+    block = {"entries": entries}
+    if len(fid) == 2:
+        lo, hi = min(fid), max(fid)
+        err = {s_: 1.0 - fid[s_]["cosine_mean"] for s_ in fid}
+        block["wide_d256_attn_scale_directional_error"] = {
+            "one_minus_cosine_mean_at_1.0": round(err[hi], 7),
+            "one_minus_cosine_mean_at_1/16": round(err[lo], 7),
+            "ratio": round(err[hi] / err[lo], 2) if err[lo] > 0 else None,
+            "sample": "sequence 0, kv heads 0..1, unquantized fp64 softmax attention vs the int4 path"}
+    return block
 
 
 def rotation_matrix(d, signs, device):
@@ -627,8 +801,15 @@ def cpu_baseline(w, seed):
         ts.append(time.perf_counter() - t0)
     t = min(ts)
     kvb = kv_bytes(w, [s["T"] + 1]) // w.num_kv_heads
-    return {"value": round(kvb / t / 1e9, 4), "unit": "GB/s", "cores": s["threads"], "kind": "oracle",
+    cores = s["threads"]
+    s["threads"] = 1  # the same step on one core, once
+    t0 = time.perf_counter()
+    oracle_step(s, w)
+    t1 = time.perf_counter() - t0
+    return {"value": round(kvb / t / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "us_per_step_sample": round(t * 1e6, 1),
+            "single_thread": {"value": round(kvb / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "us_per_step_sample": round(t1 * 1e6, 1)},
             "sample": (f"kv head 0 of {w.num_kv_heads} ({s['G']} query heads) at {s['T'] + 1}-token "
                        f"context: quantize-append 1 token + decode, best of 3; oracle prefill of the "
                        f"sample took {s['prefill_s']:.1f} s")}
