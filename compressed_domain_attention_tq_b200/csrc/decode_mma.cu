@@ -252,8 +252,8 @@ struct Cfg {
   static constexpr int al(int x) { return (x + 127) / 128 * 128; }  // 128-byte regions
   static constexpr int BAR = NS * STAGE;                     // uint64 full[NS]
   static constexpr int CNT = al(BAR + 8 * NS);               // int finished-warp count[NS]
-  static constexpr int CUR = al(CNT + 4 * NS);               // int refill cursor[8]
-  static constexpr int QA = al(CUR + 32);                    // f16 [NG][2][16][16] score A
+  static constexpr int CUR = al(CNT + 4 * NS);               // int refill cursor[8], queue[3]
+  static constexpr int QA = al(CUR + 44);                    // f16 [NG][2][16][16] score A
   static constexpr int QS = al(QA + NG * 2 * 16 * 16 * 2);   // float [NH][D] query
   static constexpr int QEXP = al(QS + 4 * NH * D);           // float [NH]
   static constexpr int QK8 = al(QEXP + 4 * 8);               // float [NH][NG] -8 sum_g q
@@ -365,6 +365,29 @@ __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* s
   return true;
 }
 
+// Refill queue (cur[8] stages freed by every warp, cur[9] refills issued,
+// cur[10] lock; lane 0 of a warp only).  A stage freed by the last warp to
+// finish it is only queued; the refill is issued by the next warp to finish a
+// stage, which is one of the fastest, instead of by the last one, whose
+// refills would otherwise keep it last (and alone doing every refill) for the
+// rest of the item.  Refills are issued in order under the lock.
+template <int D, int PATH, int FMT>
+__device__ __forceinline__ void service_refills(const DecodeArgs& a, unsigned char* smem, int* cur,
+                                                uint64_t* full, volatile int* abort) {
+  using C = Cfg<D, PATH, FMT>;
+  volatile int* q = cur + 8;
+  if (q[1] >= q[0] || *abort) return;
+  if (atomicCAS(cur + 10, 0, 1) != 0) return;  // another warp is issuing
+  __threadfence_block();
+  while (q[1] < q[0] && !*abort) {
+    const int r = q[1];
+    issue_next<D, PATH, FMT>(a, smem, cur, full, r % C::NS);
+    q[1] = r + 1;
+  }
+  __threadfence_block();
+  atomicExch(cur + 10, 0);
+}
+
 // Per-thread state of one warp for one item.
 template <int D, int PATH, int FMT>
 struct WarpState {
@@ -404,14 +427,29 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
       for (int s = 0; s < C::NS; ++s)
         if (!issue_next<D, PATH, FMT>(a, smem, cur, full, s)) break;
   }
-  for (int hh = 0; hh < HPW; ++hh) {
-    const int h = warp * HPW + hh;
-    if (warp >= C::NW / 2 || h >= C::NH) break;
-    float x[E];
-    if (h < G) {
+  // every head of this warp is loaded first, so all their loads (and the signs)
+  // are in flight together: one memory latency for the warp, not one per head
+  float xs[HPW][E];
+  int8_t sg[E];
+  const bool wht = a.signs != nullptr && a.q_rot == nullptr;
+  if (warp < C::NW / 2) {
+    if (a.q_rot != nullptr || a.inputs_pending)
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // written by the preceding grid
+    if (wht) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) sg[e] = a.signs[lane * E + e];  // bytes: no alignment needed
+    }
+#pragma unroll
+    for (int hh = 0; hh < HPW; ++hh) {
+      const int h = warp * HPW + hh;
+      float* x = xs[hh];
+      if (h >= C::NH || h >= G) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = 0.0f;
+        continue;
+      }
       const int64_t base = ((int64_t)b * a.Hq + (int64_t)kvh * G + h) * D + lane * E;
       if (a.q_rot != nullptr) {  // SRFT variant: the query is already rotated (fp32)
-        asm volatile("griddepcontrol.wait;" ::: "memory");  // by the preceding grid
 #pragma unroll
         for (int e = 0; e < E; e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(a.q_rot + base + e);
@@ -421,7 +459,6 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
           x[e + 3] = v.w;
         }
       } else if (a.q_bf16) {  // E consecutive bf16 values: one 8- or 16-byte load
-        if (a.inputs_pending) asm volatile("griddepcontrol.wait;" ::: "memory");
         uint32_t u[E / 2];
         if (E == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + base);
@@ -438,7 +475,6 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
         for (int e = 0; e < E; ++e)
           x[e] = __uint_as_float(e & 1 ? (u[e / 2] & 0xFFFF0000u) : (u[e / 2] << 16));
       } else {
-        if (a.inputs_pending) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
         for (int e = 0; e < E; e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + base + e);
@@ -448,11 +484,14 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
           x[e + 3] = v.w;
         }
       }
-      const bool wht = a.signs != nullptr && a.q_rot == nullptr;
+    }
+  }
+  for (int hh = 0; hh < HPW; ++hh) {
+    const int h = warp * HPW + hh;
+    if (warp >= C::NW / 2 || h >= C::NH) break;
+    float* x = xs[hh];
+    if (h < G) {
       if (wht) {
-        int8_t sg[E];  // byte loads: the signs pointer has no alignment requirement
-#pragma unroll
-        for (int e = 0; e < E; ++e) sg[e] = a.signs[lane * E + e];
 #pragma unroll
         for (int e = 0; e < E; ++e) x[e] *= (float)sg[e];
 #pragma unroll
@@ -1086,6 +1125,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
     *abort = 0;
     cur[0] = (int)blockIdx.x - (int)gridDim.x;  // before this CTA's first item
     cur[1] = cur[2] = cur[3] = cur[4] = cur[5] = 0;
+    cur[8] = cur[9] = cur[10] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the merge kernel may be scheduled now; it waits for this grid's writes
@@ -1218,12 +1258,15 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       else if (nv > 0)
         stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
       __syncwarp();
-      if (lane == 0) {  // the last warp out of the stage refills it
+      if (lane == 0) {
+        // first the refills queued by earlier stages, then this warp leaves the
+        // stage; the last warp out only queues the stage's refill
+        service_refills<D, PATH, FMT>(a, smem, cur, full, abort);
         __threadfence_block();
         if (atomicAdd(cnt + slot, 1) == C::NW - 1) {
           cnt[slot] = 0;
           __threadfence_block();
-          if (!*abort) issue_next<D, PATH, FMT>(a, smem, cur, full, slot);
+          atomicAdd(cur + 8, 1);
         }
       }
     }
