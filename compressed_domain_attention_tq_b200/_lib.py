@@ -132,6 +132,7 @@ def status_string(status: int) -> str:
 TEST_HOOK_FAIL_LAUNCH = 1
 TEST_HOOK_STARVE_PIPELINE = 2
 TEST_HOOK_TCGEN05_DECODE = 4
+TEST_HOOK_BUTTERFLY_QUANTIZE = 8
 
 
 def set_test_hooks(hooks: int) -> None:

@@ -633,6 +633,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   }
   const bool rot = a.signs != nullptr;
   if (a.d == 128) {
+    if (a.bf16 && rot && !a.butterfly_rotation && quantize_tc_supported(a)) return launch_quantize_tc(a, stream);
     if (a.bf16) return rot ? launch_half<true>(a, stream) : launch_half<false>(a, stream);
     return rot ? launch_q<128, false, true>(a, stream) : launch_q<128, false, false>(a, stream);
   }

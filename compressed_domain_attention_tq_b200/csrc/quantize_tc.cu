@@ -1,0 +1,372 @@
+// quantize_tc.cu -- bulk quantize-append of bf16 K/V at head_dim 128 with the
+// rotation on the fifth-generation tensor cores.
+//
+// The rotated vector is y = R x with R = H diag(signs) / sqrt(128) (AdapTQ
+// post, "Fast Hadamard Rotation (HAR)"; the sign-randomized Hadamard of the
+// SRFT post).  For bf16 inputs every product x_k * (+-1) is exact, so the
+// unnormalised rotation of a tile of 128 vectors is one 128 x 128 x 128 bf16
+// product with fp32 accumulation: D = X B, B[k][n] = signs[k] * H[k][n]
+// (H[k][n] = (-1)^popcount(k & n), the Sylvester Hadamard matrix).  The
+// butterfly form of the other quantize kernels spends about six of its ~16
+// instructions per coordinate on this; here it costs eight tcgen05.mma per
+// tile, and the CUDA cores only do the group abs-max, the codes and the
+// packing (SRFT post, core method: scale, group abs-max and int4 packing
+// fused into one pass).
+//
+// One persistent CTA per SM, warp-specialised:
+//  - warp 8 (one thread) streams 128-vector input tiles into a ring of five
+//    32 KB shared-memory stages with TMA (two 64-element boxes per tile, the
+//    128-byte swizzle the MMA reads);
+//  - warp 9 (one thread) issues the eight K = 16 MMAs of a tile into one of
+//    two 128-column fp32 accumulators in tensor memory;
+//  - warps 0-3 and 4-7 (one thread per vector, warp w reads tensor-memory
+//    lanes 32 (w % 4) ..) take the accumulators of even and odd tiles in turn:
+//    group-32 abs-max, scale, codes, nibble packing, 16-byte stores.
+// Every wait is bounded (tc::mbar_wait); a CTA whose wait gives up writes NaN
+// scales into every row it did not finish, so the failure shows in the cache.
+//
+// Codes.  With y = fl(D c), c = fl(1 / sqrt(128)), the stored values are
+// s = fl(max|y| / 7) and q = rne(fl(y / s)), the definition the oracle and
+// the other kernels follow.  max|y| = fl(max|D| c) (rounding is monotone).
+// q is found without forming y: D is rounded twice to an integer, with
+// fl(fl(c / s) (1 -+ 2^-21)) as factors; the two bracket fl(y / s) (their
+// relative distance, 2^-21, exceeds the four roundings of 2^-24 between
+// them), so when both give the same integer it is q; otherwise (a value
+// within ~1e-6 of a half-integer, or s below 2^-100, where y could be
+// subnormal) the group is recomputed as fl(y / s) with the IEEE division.
+// The accumulation order inside the tensor core is not the butterflies' one,
+// so this kernel's rotated values can differ from theirs in the last bits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "tc_ptx.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+using namespace tc;
+
+constexpr int kRows = 128;          // vectors per tile (MMA M)
+constexpr int kNS = 5;              // input stages
+constexpr int kStage = kRows * 256; // one tile of bf16 input (two 16 KB swizzled halves)
+constexpr int kThreads = 320;       // 8 epilogue warps, producer, MMA issuer
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kTmemCols = 256;      // two 128-column accumulators
+
+constexpr float kInvSqrt128 = 0.08838834764831844f;
+constexpr float kRneMagic = 12582912.0f;                    // 1.5 * 2^23
+constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21
+constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21
+constexpr float kFastScaleMin = 7.888609052210118e-31f;     // 2^-100
+
+// shared-memory layout (offsets from a 1024-byte aligned base)
+constexpr int kOffB = 0;                         // B, 32 KB
+constexpr int kOffStage = 32768;                 // kNS stages
+constexpr int kOffBar = kOffStage + kNS * kStage;
+constexpr int kFull = 0, kEmpty = kNS, kDFull = 2 * kNS, kDEmpty = 2 * kNS + 2, kMmaDone = 2 * kNS + 4;
+constexpr int kNBar = 2 * kNS + 5;
+constexpr int kOffMisc = kOffBar + 8 * kNBar;    // tensor-memory base, abort flag
+constexpr int kSmemBytes = kOffMisc + 16 + 1024; // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+// idesc: bf16 A and B (type 1), f32 accumulation, both K-major, M = N = 128
+constexpr uint32_t kIdesc = idesc_f16(128, 128, 0, 0) | (1u << 7) | (1u << 10);
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+struct Tiles {
+  int64_t rows;      // vectors per tensor (B * Hkv * n_new)
+  int64_t per;       // tiles per tensor
+  __device__ int64_t total() const { return 2 * per; }
+};
+
+// Destination row of input vector `row` of the K (kv = 0) or V tensor, or -1
+// when its position falls outside the cache.
+__device__ __forceinline__ int64_t dest_row(const QuantizeArgs& a, int64_t row) {
+  const uint32_t r32 = (uint32_t)row, bh = r32 / (uint32_t)a.n_new;
+  const uint32_t n = r32 - bh * (uint32_t)a.n_new;
+  const int b = (int)(bh / (uint32_t)a.Hkv);
+  const int64_t p = (int64_t)a.pos[b] + n;
+  if (p < 0 || p >= a.capacity) return -1;
+  return (int64_t)bh * a.capacity + p;
+}
+
+// One group of 32 coordinates of this thread's vector: d[] = unnormalised
+// rotated values D (fp32 bits) -> scale, and the codes as the floats
+// kRneMagic + q (bits 0x4B400000 + q).
+__device__ __forceinline__ float quantize_group(const uint32_t (&d)[32], uint32_t (&code)[32]) {
+  float m[11];
+#pragma unroll
+  for (int j = 0; j < 10; ++j)
+    m[j] = fmax3(fabsf(__uint_as_float(d[3 * j])), fabsf(__uint_as_float(d[3 * j + 1])),
+                 fabsf(__uint_as_float(d[3 * j + 2])));
+  m[10] = fmaxf(fabsf(__uint_as_float(d[30])), fabsf(__uint_as_float(d[31])));
+  const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]),
+                           fmax3(fmax3(m[6], m[7], m[8]), m[9], m[10]));
+  const float s = __fdiv_rn(amax * kInvSqrt128, 7.0f);
+  const float r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+  const float cr = r * kInvSqrt128;
+  const float2 rlo = make_float2(cr * kBracketLo, cr * kBracketLo);
+  const float2 rhi = make_float2(cr * kBracketHi, cr * kBracketHi);
+  const float2 magic = make_float2(kRneMagic, kRneMagic);
+  uint32_t diff = (s > 0.0f && s < kFastScaleMin) || !(r <= 3.0e38f) ? 1u : 0u;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float2 v = make_float2(__uint_as_float(d[j]), __uint_as_float(d[j + 1]));
+    const float2 flo = __ffma2_rn(v, rlo, magic), fhi = __ffma2_rn(v, rhi, magic);
+    diff |= (__float_as_uint(flo.x) ^ __float_as_uint(fhi.x)) | (__float_as_uint(flo.y) ^ __float_as_uint(fhi.y));
+    code[j] = __float_as_uint(flo.x);
+    code[j + 1] = __float_as_uint(flo.y);
+  }
+  if (diff) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float y = __uint_as_float(d[j]) * kInvSqrt128;
+      float q = rintf(__fdiv_rn(y, s));
+      q = fminf(fmaxf(q, -7.0f), 7.0f);
+      code[j] = __float_as_uint(kRneMagic + q);  // exact: |q| <= 7
+    }
+  }
+  return s;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    quantize_tc_kernel(const QuantizeArgs a, const __grid_constant__ CUtensorMap map_k,
+                       const __grid_constant__ CUtensorMap map_v) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the 128-byte swizzle is a function of absolute shared-memory address bits
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  int* misc = reinterpret_cast<int*>(smem + kOffMisc);
+  volatile int* abort = misc + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Tiles tl;
+  tl.rows = (int64_t)a.B * a.Hkv * a.n_new;
+  tl.per = (tl.rows + kRows - 1) / kRows;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(bar + kFull + s, 1);
+      mbar_init(bar + kEmpty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar + kDFull + b, 1);
+      mbar_init(bar + kDEmpty + b, 4);
+    }
+    mbar_init(bar + kMmaDone, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(misc), kTmemCols);
+    tmem_relinquish();
+  }
+  // B^T[n][k] = signs[k] (-1)^popcount(n & k) as bf16 +-1, K-major: row n of
+  // K-half h at h * 16 KB + 128 n, its 16-byte chunk c at (c ^ (n % 8)) * 16
+  {
+    unsigned char* bsm = smem + kOffB;
+    for (int i = threadIdx.x; i < 128 * 16; i += kThreads) {
+      const int n = i >> 4, kc = i & 15;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t pair = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int k = 8 * kc + 2 * e + h;
+          const bool neg = ((a.signs[k] < 0) ? 1 : 0) ^ (__popc(n & k) & 1);
+          pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
+        }
+        w[e] = pair;
+      }
+      *reinterpret_cast<uint4*>(bsm + (kc >> 3) * 16384 + n * 128 + (((kc & 7) ^ (n & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // operand for the tensor cores
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tbase = static_cast<uint32_t>(misc[0]);
+  const int64_t t_first = blockIdx.x, t_step = gridDim.x;
+
+  if (warp < 8) {
+    // ============================================================ epilogue
+    const int set = warp >> 2, quarter = warp & 3;
+    const uint32_t taddr = tbase + ((uint32_t)(32 * quarter) << 16) + 128u * set;
+    uint32_t u = 0;
+    bool failed = false;
+    for (int64_t t = t_first + set * t_step; t < tl.total(); t += 2 * t_step, ++u) {
+      const int kv = t >= tl.per;
+      const int64_t row = (t - kv * tl.per) * kRows + 32 * quarter + lane;
+      const int64_t dst = row < tl.rows ? dest_row(a, row) : -1;
+      if (!failed) {
+        const bool ok = mbar_wait(bar + kDFull + set, u & 1, abort);
+        failed = !__all_sync(0xffffffffu, ok);
+      }
+      if (failed) {
+        if (dst >= 0)
+          *reinterpret_cast<float4*>((kv ? a.v_scales : a.k_scales) + dst * 4) =
+              make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                          __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+        continue;
+      }
+      fence_after();
+      // groups in the order 1, 0, 3, 2: the nibbles of row word 2 jb + p are,
+      // from the top, in-group 4 jb + 3 .. 4 jb of group 2p + 1, then of 2p
+      uint32_t words[16];
+      float sc[4];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        uint32_t wv[8];
+#pragma unroll
+        for (int jb = 0; jb < 8; ++jb) wv[jb] = 0u;
+#pragma unroll
+        for (int h = 1; h >= 0; --h) {
+          const int g = 2 * p + h;
+          uint32_t d[32];
+          tld_x32(taddr + 32u * g, d);
+          wait_ld();
+          if (g == 2) {  // the last group read: the accumulator is free
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar + kDEmpty + set);
+          }
+          uint32_t code[32];
+          sc[g] = quantize_group(d, code);
+#pragma unroll
+          for (int jb = 0; jb < 8; ++jb)
+#pragma unroll
+            for (int kk = 3; kk >= 0; --kk) wv[jb] = (wv[jb] << 4) + code[4 * jb + kk];
+        }
+        // each nibble holds bits 0x4B400000 + q: remove the constant (leaving
+        // q + 8 per nibble, no borrows), then flip bit 3 of every nibble
+        constexpr uint32_t kBias = (0x4B400000u - 8u) * 0x11111111u;
+#pragma unroll
+        for (int jb = 0; jb < 8; ++jb) words[2 * jb + p] = (wv[jb] - kBias) ^ 0x88888888u;
+      }
+      if (dst >= 0) {
+        uint4* out = reinterpret_cast<uint4*>((kv ? a.v_packed : a.k_packed) + dst * 64);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) out[c] = make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+        *reinterpret_cast<float4*>((kv ? a.v_scales : a.k_scales) + dst * 4) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+      }
+    }
+  } else if (warp == kProducerWarp) {
+    // ============================================================ producer
+    if (lane == 0) {
+      uint32_t i = 0;
+      for (int64_t t = t_first; t < tl.total(); t += t_step, ++i) {
+        const int s = i % kNS;
+        if (i >= kNS && !mbar_wait(bar + kEmpty + s, ((i / kNS) - 1) & 1, abort)) break;
+        if (a.test_starve && i == 0) continue;  // test hook: the first stage never arrives
+        const int kv = t >= tl.per;
+        const int y = (int)((t - kv * tl.per) * kRows);
+        unsigned char* stg = smem + kOffStage + s * kStage;
+        mbar_arrive_expect_tx(bar + kFull + s, (uint32_t)kStage);
+        const CUtensorMap* m = kv ? &map_v : &map_k;
+        tma_load_2d(stg, m, 0, y, bar + kFull + s);
+        tma_load_2d(stg + kStage / 2, m, 64, y, bar + kFull + s);
+      }
+      // copies still in flight land before the CTA exits
+      const uint32_t first = i > (uint32_t)kNS ? i - kNS : 0;
+      for (uint32_t v = first; v < i; ++v) {
+        if (a.test_starve && v == 0) continue;
+        mbar_drain(bar + kFull + v % kNS, (v / kNS) & 1);
+      }
+    }
+  } else {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint64_t db = smem_desc_sw128(smem_u32(smem + kOffB));
+      const uint64_t da = smem_desc_sw128(smem_u32(smem + kOffStage));
+      uint32_t i = 0;
+      for (int64_t t = t_first; t < tl.total(); t += t_step, ++i) {
+        const int s = i % kNS, b = i & 1;
+        if (!mbar_wait(bar + kFull + s, (i / kNS) & 1, abort)) break;
+        if (i >= 2 && !mbar_wait(bar + kDEmpty + b, ((i >> 1) - 1) & 1, abort)) break;
+        fence_after();
+        const uint64_t das = da + (uint64_t)((s * kStage) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          // K step ks: K-half ks / 4 (16 KB apart), 32 bytes per step inside a row
+          const uint64_t off = (uint64_t)((((ks >> 2) * 16384) + (ks & 3) * 32) >> 4);
+          mma_ss(tbase + 128u * b, das + off, db + off, kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar + kEmpty + s);
+        mma_commit(bar + kDFull + b);
+      }
+      mma_commit(bar + kMmaDone);
+      mbar_drain(bar + kMmaDone, 0);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tbase, kTmemCols);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// rows x 128 bf16, 64 x 128-element boxes with the 128-byte swizzle (rows
+// past the end read as zeros)
+bool input_map(CUtensorMap* m, const void* base, int64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kRows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool quantize_tc_supported(const QuantizeArgs& a) {
+  const int64_t rows = (int64_t)a.B * a.Hkv * a.n_new;
+  return a.d == 128 && a.bf16 && a.signs != nullptr && !a.pos_is_ctx && a.cb_bits == 0 &&
+         a.lambda_k == nullptr && a.lambda_v == nullptr && rows <= (int64_t)INT32_MAX - kRows &&
+         encode_fn() != nullptr;
+}
+
+cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream) {
+  if (!quantize_tc_supported(a)) return cudaErrorNotSupported;
+  static SmemLimitSet smem_set;
+  const cudaError_t e = ensure_smem_limit(quantize_tc_kernel, kSmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = (int64_t)a.B * a.Hkv * a.n_new;
+  CUtensorMap mk, mv;
+  if (!input_map(&mk, a.k, rows) || !input_map(&mv, a.v, rows)) return cudaErrorInvalidValue;
+  int dev = 0, sms = kSmCount;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = 2 * ((rows + kRows - 1) / kRows);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  quantize_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a, mk, mv);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,11 +1,11 @@
 // tc_ptx.cuh -- thin wrappers over the sm_100a instructions of the tensor-core
-// decode (decode_tc.cu): mbarriers, bulk and tensor (TMA) async copies,
+// kernels (decode_tc.cu, quantize_tc.cu): mbarriers, bulk and tensor (TMA) async copies,
 // tensor-memory allocation, loads and stores, and the fifth-generation MMA
 // (tcgen05.mma, kind::f16) with its shared-memory and instruction descriptors.
 //
-// Descriptor encodings (checked against a CPU product on B200 before use):
+// Descriptor encodings (each checked against a CPU product on B200):
 //  - instruction descriptor, kind::f16 with f32 accumulation: bit 4 = 1 (f32
-//    accumulator), bits 7..9 / 10..12 = 0 (f16 A / B), bit 15 / 16 = A / B
+//    accumulator), bits 7..9 / 10..12 = A / B type (0 f16, 1 bf16), bit 15 / 16 = A / B
 //    major-ness (0 K-major, 1 MN-major), N >> 3 at bit 17, M >> 4 at bit 24;
 //  - shared-memory descriptor without swizzle: address >> 4 at bit 0, the
 //    byte stride between core matrices along K (>> 4) at bit 16, the stride
@@ -90,6 +90,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// 2-D tiled tensor copy global -> shared (no multicast); x is the innermost
+// coordinate in elements (x * element size a multiple of 16 bytes).
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 3-D tiled tensor copy global -> shared (no multicast); x is the innermost
 // coordinate (bytes of a uint8 tensor: a multiple of 16).
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z,
@@ -152,11 +162,34 @@ __device__ __forceinline__ void tst_16x256b_x4(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
+// 32 lanes x 32 bits, 32 consecutive columns
+__device__ __forceinline__ void tld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
 // --------------------------------------------------------------------- MMA
 
 __host__ __device__ constexpr uint64_t smem_desc(uint32_t addr, uint32_t k_stride, uint32_t mn_stride) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((k_stride >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((mn_stride >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// Shared-memory descriptor of a K-major operand in the 128-byte swizzled
+// layout (what a TMA copy with CU_TENSOR_MAP_SWIZZLE_128B writes for rows of
+// 128 bytes): 8-row atoms of 1024 bytes, atoms 1024 bytes apart along M or N,
+// layout type 2 at bit 61.  The atom must start on a 1024-byte boundary; a
+// K step inside the 128-byte row adds its byte offset to the address.
+__host__ __device__ constexpr uint64_t smem_desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major) {
@@ -171,6 +204,16 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t bde
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D (tensor memory) (+)= A (shared memory) x B (shared memory), one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

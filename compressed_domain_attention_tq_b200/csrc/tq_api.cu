@@ -214,6 +214,9 @@ static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, 
   a.lambda_v = rot.lambda_v;
   a.cb_bits = rot.cb_bits;
   a.levels = rot.levels;
+  const unsigned hooks = g_test_hooks.load(std::memory_order_relaxed);
+  a.test_starve = (hooks & TQ_TEST_HOOK_STARVE_PIPELINE) != 0;
+  a.butterfly_rotation = (hooks & TQ_TEST_HOOK_BUTTERFLY_QUANTIZE) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const cudaError_t e = rot.srft ? launch_quantize_srft(a, s)
                         : rot.cb_bits ? launch_quantize_cb(a, s)

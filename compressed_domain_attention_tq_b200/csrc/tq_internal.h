@@ -49,6 +49,8 @@ struct QuantizeArgs {
   const float* lambda_v = nullptr;
   int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
   const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
+  int test_starve = 0;              // test hook: the tensor-core kernel withholds its first copy
+  int butterfly_rotation = 0;       // test hook: CUDA-core butterflies instead of the tensor cores
 };
 
 struct DequantizeArgs {
@@ -139,6 +141,8 @@ cudaError_t ensure_smem_limit(Kernel kernel, int bytes, SmemLimitSet& done) {
 }
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+bool quantize_tc_supported(const QuantizeArgs& a);  // bulk bf16, d = 128, rotation on
+cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 bool decode_mma_supported(int d, int G);

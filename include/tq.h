@@ -483,21 +483,28 @@ TQ_API tq_status tq_sdpa_cb_decode_append_host(
 
 /*
  * tq_set_test_hooks -- testing only; leave at 0 (the default) in normal use.
- * Sets process-wide switches read once by every later decode call:
+ * Sets process-wide switches read once by every later decode or quantize
+ * call:
  *  - TQ_TEST_HOOK_FAIL_LAUNCH: decode calls return TQ_ERR_CUDA after
  *    validation, before enqueueing anything (as a failed launch would).
- *  - TQ_TEST_HOOK_STARVE_PIPELINE: the tensor-core decode kernels withhold
- *    each CTA's first copy, so their bounded waits run out (about 2 s); the
- *    call's outputs are then NaN and the context stays usable.
+ *  - TQ_TEST_HOOK_STARVE_PIPELINE: the tensor-core decode kernels and the
+ *    tensor-core bulk quantize withhold each CTA's first copy, so their
+ *    bounded waits run out (about 2 s); a decode's outputs are then NaN, a
+ *    bulk quantize writes NaN scales into the rows it did not finish, and the
+ *    context stays usable.
  *  - TQ_TEST_HOOK_TCGEN05_DECODE: the int4 decode at head_dim 128 with up to
  *    8 query heads per kv head runs on the tcgen05 / tensor-memory kernel
  *    instead of the default warp-level mma.sync kernel (for comparing the
  *    two; the default is the faster one on B200 for this decode).
+ *  - TQ_TEST_HOOK_BUTTERFLY_QUANTIZE: bulk quantize-appends of bf16 vectors
+ *    at head_dim 128 with rotation rotate with fp32 butterflies on the CUDA
+ *    cores instead of the tensor-core product (for comparing the two).
  * No counterpart on the method's pages.
  */
 #define TQ_TEST_HOOK_FAIL_LAUNCH 1u
 #define TQ_TEST_HOOK_STARVE_PIPELINE 2u
 #define TQ_TEST_HOOK_TCGEN05_DECODE 4u
+#define TQ_TEST_HOOK_BUTTERFLY_QUANTIZE 8u
 TQ_API void tq_set_test_hooks(uint32_t hooks);
 
 /* tq_status_string -- static English text for a status code. */
