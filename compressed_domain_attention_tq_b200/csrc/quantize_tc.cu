@@ -21,21 +21,34 @@
 //    two 128-column fp32 accumulators in tensor memory;
 //  - warps 0-3 and 4-7 (one thread per vector, warp w reads tensor-memory
 //    lanes 32 (w % 4) ..) take the accumulators of even and odd tiles in turn:
-//    group-32 abs-max, scale, codes, nibble packing, 16-byte stores.
+//    group-32 abs-max, scale, codes, nibble packing, 16-byte stores.  A tile's
+//    groups are handled in two pairs; the second pair's tensor-memory loads
+//    are in flight while the first is quantized.
+// The epilogue warps build B in shared memory while the first input copies
+// are in flight; the MMA issuer waits for it on a named barrier.
 // Every wait is bounded (tc::mbar_wait); a CTA whose wait gives up writes NaN
 // scales into every row it did not finish, so the failure shows in the cache.
 //
 // Codes.  With y = fl(D c), c = fl(1 / sqrt(128)), the stored values are
 // s = fl(max|y| / 7) and q = rne(fl(y / s)), the definition the oracle and
 // the other kernels follow.  max|y| = fl(max|D| c) (rounding is monotone).
+// fl(a / 7) is computed as fl(a zh + fl(a zl)), zh = fl(1/7), zl = fl(1/7 -
+// zh): division by a divisor known in advance (Brisebarre, Muller and Raina,
+// IEEE Trans. Computers 2004).  It is exact here because a / 7 lies at least
+// 1/14 of an ulp from every rounding midpoint while the two-term error is
+// below 2^-24 ulp (checked over every significand on the CPU); below a =
+// 2^-90, where a zl would lose bits, the IEEE division runs instead.
 // q is found without forming y: D is rounded twice to an integer, with
-// fl(fl(c / s) (1 -+ 2^-21)) as factors; the two bracket fl(y / s) (their
-// relative distance, 2^-21, exceeds the four roundings of 2^-24 between
+// fl(fl(c r) (1 -+ 2^-21)) as factors, r the hardware reciprocal of s
+// (relative error below 2^-23); the two bracket fl(y / s) (their relative
+// distance, 2^-21, exceeds 2^-23 plus the four roundings of 2^-24 between
 // them), so when both give the same integer it is q; otherwise (a value
 // within ~1e-6 of a half-integer, or s below 2^-100, where y could be
 // subnormal) the group is recomputed as fl(y / s) with the IEEE division.
 // The accumulation order inside the tensor core is not the butterflies' one,
-// so this kernel's rotated values can differ from theirs in the last bits.
+// so this kernel's rotated values can differ from theirs in the last bits;
+// when every partial sum is exact (small-integer inputs) the two kernels
+// give identical bits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -61,7 +74,10 @@ constexpr float kInvSqrt128 = 0.08838834764831844f;
 constexpr float kRneMagic = 12582912.0f;                    // 1.5 * 2^23
 constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21
 constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21
-constexpr float kFastScaleMin = 7.888609052210118e-31f;     // 2^-100
+constexpr float kFastScaleMin = 0x1p-100f;
+constexpr float kDiv7Min = 0x1p-90f;          // fl(a / 7) by the two-constant form from here up
+constexpr float kSeventhHi = 0x1.24924ap-3f;  // fl(1/7)
+constexpr float kSeventhLo = -0x1.b6db6ep-28f;  // fl(1/7 - fl(1/7))
 
 // shared-memory layout (offsets from a 1024-byte aligned base)
 constexpr int kOffB = 0;                         // B, 32 KB
@@ -99,10 +115,33 @@ __device__ __forceinline__ int64_t dest_row(const QuantizeArgs& a, int64_t row) 
   return (int64_t)bh * a.capacity + p;
 }
 
+// fl(a / 7) for a >= 0 (NaN and infinity through the IEEE division)
+__device__ __forceinline__ float div7(float a) {
+  return (a >= kDiv7Min && a <= 3.4028234663852886e38f) ? __fmaf_rn(a, kSeventhHi, __fmul_rn(a, kSeventhLo))
+                                                         : __fdiv_rn(a, 7.0f);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The 32 registers written by a tensor-memory load are used only after this
+// point (the load completes at tcgen05.wait::ld, which the compiler does not
+// know about).
+__device__ __forceinline__ void tie32(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]),
+                 "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
 // One group of 32 coordinates of this thread's vector: d[] = unnormalised
-// rotated values D (fp32 bits) -> scale, and the codes as the floats
-// kRneMagic + q (bits 0x4B400000 + q).
-__device__ __forceinline__ float quantize_group(const uint32_t (&d)[32], uint32_t (&code)[32]) {
+// rotated values D (fp32 bits) -> the scale, and in hw[jb] the codes of
+// in-group coordinates 4 jb .. 4 jb + 3 as sum_kk 16^kk (0x4B400000 + q)
+// (mod 2^32; each code is the float kRneMagic + q).
+__device__ __forceinline__ float quantize_group(const uint32_t (&d)[32], uint32_t (&hw)[8]) {
   float m[11];
 #pragma unroll
   for (int j = 0; j < 10; ++j)
@@ -111,31 +150,54 @@ __device__ __forceinline__ float quantize_group(const uint32_t (&d)[32], uint32_
   m[10] = fmaxf(fabsf(__uint_as_float(d[30])), fabsf(__uint_as_float(d[31])));
   const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]),
                            fmax3(fmax3(m[6], m[7], m[8]), m[9], m[10]));
-  const float s = __fdiv_rn(amax * kInvSqrt128, 7.0f);
-  const float r = (s > 0.0f) ? __frcp_rn(s) : 0.0f;
+  const float s = div7(amax * kInvSqrt128);
+  const float r = (s > 0.0f) ? rcp_approx(s) : 0.0f;
   const float cr = r * kInvSqrt128;
   const float2 rlo = make_float2(cr * kBracketLo, cr * kBracketLo);
   const float2 rhi = make_float2(cr * kBracketHi, cr * kBracketHi);
   const float2 magic = make_float2(kRneMagic, kRneMagic);
-  uint32_t diff = (s > 0.0f && s < kFastScaleMin) || !(r <= 3.0e38f) ? 1u : 0u;
+  uint32_t diff[4] = {(s > 0.0f && s < kFastScaleMin) || !(r <= 3.0e38f) ? 1u : 0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    const float2 v = make_float2(__uint_as_float(d[j]), __uint_as_float(d[j + 1]));
-    const float2 flo = __ffma2_rn(v, rlo, magic), fhi = __ffma2_rn(v, rhi, magic);
-    diff |= (__float_as_uint(flo.x) ^ __float_as_uint(fhi.x)) | (__float_as_uint(flo.y) ^ __float_as_uint(fhi.y));
-    code[j] = __float_as_uint(flo.x);
-    code[j + 1] = __float_as_uint(flo.y);
+  for (int jb = 0; jb < 8; ++jb) {
+    uint32_t c[4];
+#pragma unroll
+    for (int h = 0; h < 4; h += 2) {
+      const int j = 4 * jb + h;
+      const float2 v = make_float2(__uint_as_float(d[j]), __uint_as_float(d[j + 1]));
+      const float2 flo = __ffma2_rn(v, rlo, magic), fhi = __ffma2_rn(v, rhi, magic);
+      diff[jb & 3] |= (__float_as_uint(flo.x) ^ __float_as_uint(fhi.x)) |
+                      (__float_as_uint(flo.y) ^ __float_as_uint(fhi.y));
+      c[h] = __float_as_uint(flo.x);
+      c[h + 1] = __float_as_uint(flo.y);
+    }
+    hw[jb] = ((((c[3] << 4) + c[2]) << 4) + c[1]) * 16u + c[0];
   }
-  if (diff) {
+  if (diff[0] | diff[1] | diff[2] | diff[3]) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float y = __uint_as_float(d[j]) * kInvSqrt128;
-      float q = rintf(__fdiv_rn(y, s));
-      q = fminf(fmaxf(q, -7.0f), 7.0f);
-      code[j] = __float_as_uint(kRneMagic + q);  // exact: |q| <= 7
+    for (int jb = 0; jb < 8; ++jb) {
+      uint32_t c[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float y = __uint_as_float(d[4 * jb + h]) * kInvSqrt128;
+        float q = rintf(__fdiv_rn(y, s));
+        q = fminf(fmaxf(q, -7.0f), 7.0f);
+        c[h] = __float_as_uint(kRneMagic + q);  // exact: |q| <= 7
+      }
+      hw[jb] = ((((c[3] << 4) + c[2]) << 4) + c[1]) * 16u + c[0];
     }
   }
   return s;
+}
+
+// Row words 2 jb + p of the pair of groups (2p + 1, 2p): nibbles from the
+// top are in-group 4 jb + 3 .. 4 jb of group 2p + 1, then of group 2p.  The
+// constant 0x4B400000 of each code is removed (leaving q + 8 per nibble, no
+// borrows), then bit 3 of every nibble is flipped (two's complement nibbles).
+__device__ __forceinline__ void pack_pair(const uint32_t (&hw_hi)[8], const uint32_t (&hw_lo)[8], int p,
+                                          uint32_t (&words)[16]) {
+  constexpr uint32_t kBias = (0x4B400000u - 8u) * 0x11111111u;
+#pragma unroll
+  for (int jb = 0; jb < 8; ++jb) words[2 * jb + p] = ((hw_hi[jb] << 16) + hw_lo[jb] - kBias) ^ 0x88888888u;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -169,29 +231,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(reinterpret_cast<uint32_t*>(misc), kTmemCols);
     tmem_relinquish();
   }
-  // B^T[n][k] = signs[k] (-1)^popcount(n & k) as bf16 +-1, K-major: row n of
-  // K-half h at h * 16 KB + 128 n, its 16-byte chunk c at (c ^ (n % 8)) * 16
-  {
-    unsigned char* bsm = smem + kOffB;
-    for (int i = threadIdx.x; i < 128 * 16; i += kThreads) {
-      const int n = i >> 4, kc = i & 15;
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        uint32_t pair = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int k = 8 * kc + 2 * e + h;
-          const bool neg = ((a.signs[k] < 0) ? 1 : 0) ^ (__popc(n & k) & 1);
-          pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
-        }
-        w[e] = pair;
-      }
-      *reinterpret_cast<uint4*>(bsm + (kc >> 3) * 16384 + n * 128 + (((kc & 7) ^ (n & 7)) << 4)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // operand for the tensor cores
-  }
   fence_before();
   __syncthreads();
   fence_after();
@@ -199,6 +238,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t t_first = blockIdx.x, t_step = gridDim.x;
 
   if (warp < 8) {
+    // B^T[n][k] = signs[k] (-1)^popcount(n & k) as bf16 +-1, K-major: row n
+    // of K-half h at h * 16 KB + 128 n, its 16-byte chunk c at (c ^ (n % 8)) * 16.
+    // Thread t builds chunk t % 16 (k = 8 (t % 16) .. + 7) of rows t / 16 + 16 it.
+    {
+      const int kc = threadIdx.x & 15;
+      uint32_t neg8 = 0;  // bit e: signs[8 kc + e] < 0
+#pragma unroll
+      for (int e = 0; e < 8; ++e) neg8 |= (a.signs[8 * kc + e] < 0 ? 1u : 0u) << e;
+      // bit e of kWalsh[m] = parity(m & e), m < 8
+      constexpr uint64_t kWalsh = 0x963C5AF066CCAA00ull;
+      unsigned char* bsm = smem + kOffB;
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int n = (threadIdx.x >> 4) + 16 * it;
+        const uint32_t par = (uint32_t)(__popc(n & (8 * kc)) & 1) * 0xFFu;
+        const uint32_t neg = neg8 ^ par ^ (uint32_t)((kWalsh >> (8 * (n & 7))) & 0xFFu);
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] = 0x3F803F80u | (((neg >> (2 * e)) & 1u) << 15) | (((neg >> (2 * e + 1)) & 1u) << 31);
+        *reinterpret_cast<uint4*>(bsm + (kc >> 3) * 16384 + n * 128 + (((kc & 7) ^ (n & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // operand for the tensor cores
+      asm volatile("bar.arrive 1, 288;" ::: "memory");                // B is ready
+    }
     // ============================================================ epilogue
     const int set = warp >> 2, quarter = warp & 3;
     const uint32_t taddr = tbase + ((uint32_t)(32 * quarter) << 16) + 128u * set;
@@ -220,39 +285,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       fence_after();
-      // groups in the order 1, 0, 3, 2: the nibbles of row word 2 jb + p are,
-      // from the top, in-group 4 jb + 3 .. 4 jb of group 2p + 1, then of 2p
-      uint32_t words[16];
+      uint32_t d1[32], d0[32], d3[32], d2[32], hw_a[8], hw_b[8], words[16];
       float sc[4];
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        uint32_t wv[8];
-#pragma unroll
-        for (int jb = 0; jb < 8; ++jb) wv[jb] = 0u;
-#pragma unroll
-        for (int h = 1; h >= 0; --h) {
-          const int g = 2 * p + h;
-          uint32_t d[32];
-          tld_x32(taddr + 32u * g, d);
-          wait_ld();
-          if (g == 2) {  // the last group read: the accumulator is free
-            fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar + kDEmpty + set);
-          }
-          uint32_t code[32];
-          sc[g] = quantize_group(d, code);
-#pragma unroll
-          for (int jb = 0; jb < 8; ++jb)
-#pragma unroll
-            for (int kk = 3; kk >= 0; --kk) wv[jb] = (wv[jb] << 4) + code[4 * jb + kk];
-        }
-        // each nibble holds bits 0x4B400000 + q: remove the constant (leaving
-        // q + 8 per nibble, no borrows), then flip bit 3 of every nibble
-        constexpr uint32_t kBias = (0x4B400000u - 8u) * 0x11111111u;
-#pragma unroll
-        for (int jb = 0; jb < 8; ++jb) words[2 * jb + p] = (wv[jb] - kBias) ^ 0x88888888u;
-      }
+      tld_x32(taddr + 32u, d1);
+      tld_x32(taddr, d0);
+      wait_ld();
+      tie32(d1);
+      tie32(d0);
+      tld_x32(taddr + 96u, d3);  // in flight while groups 1 and 0 are quantized
+      tld_x32(taddr + 64u, d2);
+      sc[1] = quantize_group(d1, hw_a);
+      sc[0] = quantize_group(d0, hw_b);
+      pack_pair(hw_a, hw_b, 0, words);
+      wait_ld();
+      tie32(d3);
+      tie32(d2);
+      fence_before();  // every load of the accumulator is done: hand it back
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kDEmpty + set);
+      sc[3] = quantize_group(d3, hw_a);
+      sc[2] = quantize_group(d2, hw_b);
+      pack_pair(hw_a, hw_b, 1, words);
       if (dst >= 0) {
         uint4* out = reinterpret_cast<uint4*>((kv ? a.v_packed : a.k_packed) + dst * 64);
 #pragma unroll
@@ -285,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ============================================================ MMA issuer
+    asm volatile("bar.sync 1, 288;" ::: "memory");  // B built by the epilogue warps
     if (lane == 0) {
       const uint64_t db = smem_desc_sw128(smem_u32(smem + kOffB));
       const uint64_t da = smem_desc_sw128(smem_u32(smem + kOffStage));

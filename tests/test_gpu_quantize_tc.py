@@ -82,6 +82,32 @@ def test_tc_quantize_agrees_with_butterfly_kernel():
     assert n_diff <= 1e-5 * n_tot
 
 
+def test_tc_quantize_bit_identical_to_butterfly_kernel_on_exact_inputs():
+    """Small-integer inputs times a power of two per vector: every partial sum
+    of both rotations is exact, so both kernels round the same rotated values
+    and must give identical bits (scale division by 7, reciprocal bracket,
+    fallbacks and packing all included).  Zero vectors included.  (Against the
+    oracle such inputs are a poor case: many y / s fall exactly on a
+    half-integer in exact arithmetic, where fl(D c) and the oracle's correctly
+    rounded rotation may round apart; oracle parity is the other tests'.)"""
+    require_cuda()
+    B, H, n, d = 1, 6, 1500, 128
+    g = torch.Generator().manual_seed(21)
+    ints = torch.randint(-8, 9, (B, H, n, d), generator=g).float()
+    ints[:, :, 5] = 0
+    ints[:, :, 6] = 0
+    ints[:, :, 6, 40] = 3
+    e = torch.randint(-40, 41, (B, H, n, 1), generator=g).float()
+    x = (ints * torch.exp2(e)).to(torch.bfloat16)
+    assert torch.equal(x.float(), ints * torch.exp2(e))
+    y = (-x.float() * 0.5).to(torch.bfloat16)
+    signs = _signs(d, 22)
+    tc = _quantize(x, y, [0], signs, n)
+    bf = _quantize(x, y, [0], signs, n, _lib.TEST_HOOK_BUTTERFLY_QUANTIZE)
+    for a, b in zip(tc, bf):
+        np.testing.assert_array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
 def test_tc_quantize_extreme_values():
     """bf16 subnormals, values near the bf16 maximum over 128 (no fp32
     overflow in the rotation), one huge and many tiny values in one vector,
