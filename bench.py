@@ -52,6 +52,11 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' block")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--mode", choices=["replicas", "context-parallel"], default="replicas",
+                    help="replicas: each rank decodes its own copy of the workload (no collective); "
+                         "context-parallel: one context split into contiguous token shards over the "
+                         "ranks, per step a shard decode, an NCCL all-gather of the (o, max, sum) "
+                         "parts and tq_merge_lse")
     ap.add_argument("--decode-kernel", choices=["mma_sync", "tcgen05"], default="mma_sync",
                     help="int4 decode kernel at head_dim 128 (mma_sync: the default; tcgen05: "
                          "the tensor-memory kernel, for comparison)")
@@ -854,10 +859,203 @@ def run_reference(args):
     }), flush=True)
 
 
+def cp_measure(name, args, world, rank, dev, stream, l2_bytes):
+    """Context-parallel decode of one workload: this rank's shard timings (s),
+    max over ranks, and the byte counts."""
+    import torch
+    import torch.distributed as dist
+
+    import compressed_domain_attention_tq_b200 as tq
+    from compressed_domain_attention_tq_b200 import _lib
+    from compressed_domain_attention_tq_b200 import context_parallel as cp
+    from compressed_domain_attention_tq_b200 import workloads as wl
+    w = wl.WORKLOADS[name]
+    if w.ragged is not None or w.cb_bits or (w.rotation and w.rotation_kind == "srft"):
+        raise ValueError(f"context-parallel bench: {name} is not an equal-length int4 workload")
+    B, Hq, Hkv, d, T = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.context
+    seed = args.seed  # one global context: every rank draws from the same seed
+    t0, t1 = cp.shard_range(T, world, rank)
+    n = t1 - t0
+    signs = wl.make_signs(d, seed) if w.rotation else None
+    cache = tq.Int4KVCache(B, Hkv, d, n, dev, signs)
+    chunk = 1 << 18  # draw and quantize the shard in pieces (bounded bf16 staging)
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        k, v = wl.make_kv_shard(w, seed, t0 + c0, t0 + c1, device=dev)
+        cache.append(k, v, torch.full((B,), c0, dtype=torch.int32, device=dev))
+        del k, v
+    q = wl.make_query(w, seed, device=dev)
+    scale = w.attn_scales[0]
+    ctx_dev = torch.full((B,), n, dtype=torch.int32, device=dev)
+    shard_bytes = kv_bytes(w, [n] * B)
+    total_bytes = kv_bytes(w, [T] * B)
+    n_rot = rotation_count(shard_bytes, l2_bytes, cache_bytes=cache.nbytes())
+    caches = [cache] + [replica(cache) for _ in range(n_rot - 1)]
+    local = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, Hq, 2, dtype=torch.float32, device=dev)
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    K = args.steps
+
+    def shard(i):
+        caches[i % n_rot].decode_lse(q, ctx_dev, n, scale, local, lse)
+
+    parts = cp.gather_parts(local, lse)
+
+    def merge():
+        _lib.merge_lse(parts[0], parts[1], out)
+
+    def step(i):
+        nonlocal parts
+        shard(i)
+        parts = cp.gather_parts(local, lse)
+        merge()
+
+    for i in range(max(args.warmup, n_rot)):
+        step(i)
+    torch.cuda.synchronize()
+
+    def graph_time(fn):  # K calls in one CUDA graph, replayed between events
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(K):
+                fn(i)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / 1e3 / K
+
+    def eager_time(fn):  # K calls enqueued back to back, between events
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / K
+
+    # end to end: q from pinned host memory, the step, the output back to pinned host memory
+    h_q = q.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def host_step(i):
+        q.copy_(h_q, non_blocking=True)
+        step(i)
+        h_out.copy_(out, non_blocking=True)
+
+    shard_s = graph_time(shard)
+    merge_s = graph_time(lambda i: merge())
+    gather_s = eager_time(lambda i: cp.gather_parts(local, lse))
+    step_s = eager_time(step)
+    e2e_s = eager_time(host_step)
+    t = torch.tensor([shard_s, gather_s, merge_s, step_s, e2e_s], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    shard_s, gather_s, merge_s, step_s, e2e_s = t.tolist()
+    # the merged output against this rank's own whole-context decode is not
+    # available (no rank holds the whole context); report the output's norm
+    # agreement across ranks instead: every rank must hold the same result
+    chk = out.double().norm().reshape(1)
+    if world > 1:
+        lo, hi = chk.clone(), chk.clone()
+        dist.all_reduce(lo, op=dist.ReduceOp.MIN)
+        dist.all_reduce(hi, op=dist.ReduceOp.MAX)
+        same = bool(lo.item() == hi.item())
+    else:
+        same = True
+    del caches, cache
+    torch.cuda.empty_cache()
+    return {"workload": name, "context": T, "shard_tokens": [cp.shard_range(T, world, r)[1] -
+                                                               cp.shard_range(T, world, r)[0]
+                                                               for r in range(world)],
+            "shard_bytes_max": kv_bytes(w, [cp.shard_range(T, world, 0)[1]] * B),
+            "kv_bytes": total_bytes, "step_s": step_s, "shard_s": shard_s, "gather_s": gather_s,
+            "merge_s": merge_s, "n_rot": n_rot, "outputs_equal_across_ranks": same,
+            "gather_bytes_per_rank": int((local.numel() + lse.numel()) * 4), "e2e_s": e2e_s,
+            "h2d_bytes": int(h_q.numel() * h_q.element_size()),
+            "d2h_bytes": int(h_out.numel() * h_out.element_size())}
+
+
+def run_context_parallel(args):
+    """bench.py --mode context-parallel: one context split over the ranks."""
+    import torch
+    import torch.distributed as dist
+    from compressed_domain_attention_tq_b200 import _lib
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _lib.set_test_hooks(_lib.TEST_HOOK_TCGEN05_DECODE if args.decode_kernel == "tcgen05" else 0)
+    stream = torch.cuda.current_stream()
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    peak, peak_kind = measured_peaks()
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+    main_r = cp_measure(args.workload, args, world, rank, dev, stream, l2_bytes)
+    long_r = cp_measure("llama70b_gqa_1m", args, world, rank, dev, stream, l2_bytes)
+    clocks = sampler.stop() if sampler else None
+
+    def entry(r):
+        return {"workload": r["workload"], "context": r["context"], "shard_tokens": r["shard_tokens"],
+                "us_per_step": round(r["step_s"] * 1e6, 2),
+                "kv_GB_per_s": round(r["kv_bytes"] / r["step_s"] / 1e9, 1),
+                "shard_decode_us": round(r["shard_s"] * 1e6, 2),
+                "gather_us": round(r["gather_s"] * 1e6, 2),
+                "merge_lse_us": round(r["merge_s"] * 1e6, 2),
+                "shard_roofline_frac": round(r["shard_bytes_max"] / r["shard_s"] / 1e9 / peak, 4),
+                "outputs_equal_across_ranks": r["outputs_equal_across_ranks"],
+                "l2": f"shard decodes rotated over {r['n_rot']} cache copies"}
+
+    m = main_r
+    res = {
+        "metric": METRIC, "value": round(m["kv_bytes"] / m["step_s"] / 1e9, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(m["step_s"] * 1e3, 5), "us_per_step": round(m["step_s"] * 1e6, 2),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "int4 codes, fp32 accumulation", "data": "synthetic (seeded N(0,1), bf16)",
+        "config": {"workload": m["workload"], "mode": "context-parallel", "context": m["context"],
+                   "parallelism": f"context shards x{world}",
+                   "partitioning": ("contiguous token shards of the one sequence, rank r holding "
+                                    "tokens [r T / N, (r + 1) T / N); per step every rank decodes its "
+                                    "shard (tq_sdpa_int4_decode_lse), the ranks all-gather the "
+                                    "(o, max, sum) parts over NCCL, every rank merges them "
+                                    "(tq_merge_lse)"),
+                   "gather_bytes_per_rank": m["gather_bytes_per_rank"], "decode_kernel": args.decode_kernel},
+        "context_parallel": entry(m),
+        "long_context": entry(long_r),
+        "roofline": {"bound": "hbm", "kernel": "sdpa_int4 decode of one shard (split-K + merge)",
+                     "achieved": round(m["shard_bytes_max"] / m["shard_s"] / 1e9, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(m["shard_bytes_max"] / m["shard_s"] / 1e9 / peak, 4),
+                     "peak_kind": peak_kind, "traffic": None},
+        "e2e": {"value": round(m["kv_bytes"] / m["e2e_s"] / 1e9, 1), "unit": "GB/s",
+                "us_per_step": round(m["e2e_s"] * 1e6, 2), "h2d_bytes_per_step": m["h2d_bytes"],
+                "d2h_bytes_per_step": m["d2h_bytes"]},
+        "gpu_launches": 3 * args.steps,
+        "step": ("per rank: tq_sdpa_int4_decode_lse on its shard (split-K kernel + merge, 2 launches), "
+                 "NCCL all_gather of the (o, max, sum) parts, tq_merge_lse (1 launch)"),
+        "timing": ("shard decode and tq_merge_lse: K calls in one CUDA graph each, between CUDA "
+                   "events; gather and the whole step: K eager calls back to back between events "
+                   "(includes host enqueue time where it exceeds the device time); e2e: the eager "
+                   "step with q copied in from pinned host memory and the output copied back; "
+                   "every figure the max over ranks"),
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "context-parallel":
+        run_context_parallel(args)
     else:
         run_tq(args)
 

@@ -23,15 +23,30 @@ import torch.distributed as dist
 from . import _lib
 
 
+def shard_range(total: int, world: int, rank: int) -> tuple[int, int]:
+    """Tokens [start, stop) of a `total`-token context held by `rank` of `world`:
+    contiguous shards in rank order, the first total % world ranks one token
+    longer.  Every rank holds at least one token (total >= world)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    if total < world:
+        raise ValueError(f"{total} tokens cannot give each of {world} ranks a shard")
+    base, extra = divmod(total, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
 def gather_parts(out: torch.Tensor, lse: torch.Tensor, group=None):
     """All-gather every rank's out [B][Hq][d] and lse [B][Hq][2] (float32):
-    returns (outs [R][B][Hq][d], lses [R][B][Hq][2]) in rank order."""
-    world = dist.get_world_size(group)
+    returns (outs [R][B][Hq][d], lses [R][B][Hq][2]) in rank order.  With one
+    rank (or no initialized process group) the parts are views of out and lse."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world == 1:
+        return out.unsqueeze(0), lse.unsqueeze(0)
     n_out = out.numel()
     packed = torch.cat([out.reshape(-1), lse.reshape(-1)])
-    parts = [torch.empty_like(packed) for _ in range(world)]
-    dist.all_gather(parts, packed, group=group)
-    g = torch.stack(parts)
+    g = torch.empty(world, packed.numel(), dtype=packed.dtype, device=packed.device)
+    dist.all_gather(list(g.unbind(0)), packed, group=group)  # rows of g, in rank order
     outs = g[:, :n_out].reshape(world, *out.shape).contiguous()
     lses = g[:, n_out:].reshape(world, *lse.shape).contiguous()
     return outs, lses

@@ -78,6 +78,11 @@ WORKLOADS = {
         capacity=65537, in_dtype=torch.bfloat16, rotation=True,
         attn_scales=(1.0, 1 / 16.0),
         notes="32/16 GQA, d=256; attn_scale 1.0 and 1/sqrt(256)"),
+    "llama70b_gqa_1m": Workload(
+        "llama70b_gqa_1m", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=1048576, capacity=1048577, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0,
+        notes="the 64/8 GQA layer at 1M tokens: the context-parallel decode's long case"),
     "llama70b_gqa_128k_srft": Workload(
         "llama70b_gqa_128k_srft", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
         context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
@@ -166,6 +171,14 @@ def make_kv(w: Workload, seed: int, device="cpu", tokens: int | None = None,
         k = torch.where(m, k * w.heavy_scale, k)
         v = torch.where(m, v * w.heavy_scale, v)
     return k.to(w.in_dtype), v.to(w.in_dtype)
+
+
+def make_kv_shard(w: Workload, seed: int, start: int, stop: int, device="cpu"):
+    """K, V of context tokens [start, stop) of every sequence, as held by one
+    rank of a context-parallel decode ([B][Hkv][stop - start][d]).  The whole
+    context is defined as the concatenation of its shards, each drawn from
+    its own start offset, so a rank draws only its own tokens."""
+    return make_kv(w, seed, device=device, tokens=stop - start, token_offset=20_000_033 + start)
 
 
 def make_query(w: Workload, seed: int, device="cpu", step: int = 0) -> torch.Tensor:
