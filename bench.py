@@ -128,7 +128,7 @@ def kv_bytes(w, ctx_tokens):
 # committed DRAM-traffic figure counts only while their hash is unchanged.
 KERNEL_SOURCES = {
     "decode": ["decode_mma.cu", "quantize_vector.cuh", "cb_vector.cuh", "tq_internal.h", "tq_api.cu"],
-    "quantize_bulk": ["quantize.cu", "quantize_vector.cuh", "tq_internal.h", "tq_api.cu"],
+    "quantize_bulk": ["quantize_tc.cu", "tc_ptx.cuh", "quantize.cu", "tq_internal.h", "tq_api.cu"],
 }
 
 

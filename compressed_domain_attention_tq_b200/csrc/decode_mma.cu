@@ -13,9 +13,10 @@
 // head, context chunk).  Each item's rows (packed K, packed V, K scales, V
 // scales) stream through a ring of shared-memory stages filled by 1-D bulk
 // async copies that complete on mbarriers.  There is no producer warp: every
-// warp takes TPW 16-token tiles of each stage, and the last warp to finish a
-// stage (counted with a shared-memory atomic) refills it with the next stage,
-// so all warps of the CTA compute.  Each warp keeps its own running (max, sum,
+// warp takes TPW 16-token tiles of each stage; the last warp to finish a stage
+// (counted with a shared-memory atomic) queues its refill, and the next warp to
+// leave any stage issues the queued refills in stage order, so all warps of the
+// CTA compute and the slowest warp does not also carry the refills.  Each warp keeps its own running (max, sum,
 // acc); the warps are merged per item in shared memory into one split-K
 // partial (max in log2 units, sum, unnormalized acc[d]) per query head, and
 // merge.cu combines the chunks and rotates the output back.
