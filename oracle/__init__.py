@@ -100,6 +100,13 @@ def _load():
     lib.oracle_sdpa_cb_decode.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, i64, P, P,
                                           f64, P, i32]
     lib.oracle_sdpa_cb_decode.restype = i32
+    lib.oracle_uniform_levels.argtypes = [i32, P]
+    lib.oracle_uniform_levels.restype = i32
+    lib.oracle_uniform_quantize_vector.argtypes = [i32, P, i32, P, P]
+    lib.oracle_uniform_quantize_vector.restype = None
+    lib.oracle_quantize_append_uniform.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, P, P,
+                                                   P, P, i64, i32]
+    lib.oracle_quantize_append_uniform.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     _lib = lib
@@ -419,6 +426,44 @@ def quantize_append_cb(k, v, pos, signs, bits: int, levels, cache, threads: int 
                                            threads)
     if rc != 0:
         raise ValueError(f"oracle_quantize_append_cb failed ({rc})")
+
+
+def uniform_levels(bits: int) -> np.ndarray:
+    """The decode-side table of a uniform low-bit cache: levels[u] = u - m, m = 2^(bits-1) - 1."""
+    out = np.empty(1 << bits, dtype=np.float32)
+    if _load().oracle_uniform_levels(bits, _ptr(out)) != 0:
+        raise ValueError(f"uniform levels: bits must be 2..4, got {bits}")
+    return out
+
+
+def uniform_quantize_vectors(y: np.ndarray, bits: int):
+    """Uniform abs-max indices c + m (uint8 (n, d)) and scales (float32 (n, d/32)) of rotated rows y."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    n, d = y.shape
+    idx = np.empty((n, d), dtype=np.uint8)
+    scales = np.empty((n, d // _GROUP), dtype=np.float32)
+    lib = _load()
+    for r in range(n):
+        lib.oracle_uniform_quantize_vector(d, _ptr(y[r]), bits, _ptr(idx[r]), _ptr(scales[r]))
+    return idx, scales
+
+
+def quantize_append_uniform(k, v, pos, signs, bits: int, cache, threads: int = 1) -> None:
+    """Uniform low-bit variant of quantize_append into a codebook-layout cache."""
+    k, dt = _input_array(k)
+    v, dt2 = _input_array(v)
+    if dt != dt2 or k.shape != v.shape:
+        raise ValueError("k and v must share dtype and shape")
+    B, Hkv, n_new, d = k.shape
+    kp, ks, vp, vs = cache
+    cap = kp.shape[2]
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    s = _signs_array(signs)
+    rc = _load().oracle_quantize_append_uniform(_ptr(k), _ptr(v), dt, B, Hkv, n_new, d, _ptr(pos),
+                                                _ptr(s), bits, _ptr(kp), _ptr(ks), _ptr(vp), _ptr(vs),
+                                                cap, threads)
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_append_uniform failed ({rc})")
 
 
 def sdpa_cb_decode(q, cache, ctx_lens, signs, bits: int, levels, attn_scale: float,

@@ -48,6 +48,13 @@
  *    of the group's 4*bits bytes, groups in order.  The Gaussian Max-Lloyd
  *    codebook is the fixed point of "thresholds at midpoints, levels at the
  *    cell means of N(0,1)".
+ *  - uniform low-bit variant ([OTM-F], future work: int2; read as the int4
+ *    quantizer at fewer bits): with m = 2^(bits-1) - 1, per group of 32
+ *    rotated coordinates s = fl32(amax / m) (fp32 IEEE division; s = amax at
+ *    two bits), c = clamp(rne(fl32(y / s)), -m, m), stored as the index c + m
+ *    in the codebook layout; the value is s * c.  The cache is a codebook
+ *    cache whose levels are the integers C[u] = u - m (u < 2^bits; the top
+ *    index is never written).
  *  - SRFT variant ([SRFT], core method: a sign-randomized Fourier transform
  *    instead of the Hadamard one, usable at widths that are not powers of
  *    two, followed by a per-coordinate scale lambda): the transform is the
@@ -560,6 +567,86 @@ int oracle_quantize_append_cb(const void* k, const void* v, int in_dtype, int B,
       if (R) oracle_rotate_vector(d, R, x, y);
       else memcpy(y, x, sizeof(float) * (size_t)d);
       oracle_cb_quantize_vector(d, y, bits, C, ci, (kv ? v_scales : k_scales) + row * ng);
+      oracle_cb_pack_vector(d, bits, ci, (kv ? v_packed : k_packed) + row * rowb);
+    }
+  }
+  free(R);
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* uniform low-bit variant ([OTM-F] future work: int2)                  */
+/* ------------------------------------------------------------------ */
+
+/* levels[u] = u - m, m = 2^(bits-1) - 1, u < 2^bits: the decode-side table */
+int oracle_uniform_levels(int bits, float* levels) {
+  if (bits < 2 || bits > 4) return -1;
+  int m = (1 << (bits - 1)) - 1;
+  for (int u = 0; u < (1 << bits); ++u) levels[u] = (float)(u - m);
+  return 0;
+}
+
+/* indices[d] (c + m), scales[d/32] of an already-rotated vector y */
+void oracle_uniform_quantize_vector(int d, const float* y, int bits, uint8_t* idx, float* scales) {
+  int ng = d / ORACLE_GROUP, m = (1 << (bits - 1)) - 1;
+  for (int g = 0; g < ng; ++g) {
+    const float* yg = y + g * ORACLE_GROUP;
+    float amax = 0.0f;
+    for (int j = 0; j < ORACLE_GROUP; ++j) {
+      float a = fabsf(yg[j]);
+      if (a > amax) amax = a;
+    }
+    volatile float top = (float)m;        /* keep the division in fp32 IEEE */
+    float s = amax / top;
+    scales[g] = s;
+    for (int j = 0; j < ORACLE_GROUP; ++j) {
+      int c = 0;
+      if (amax > 0.0f) {
+        volatile float uq = yg[j] / s;    /* fp32 quotient, rounded once */
+        float rq = nearbyintf(uq);        /* round half to even (default mode) */
+        if (rq > (float)m) rq = (float)m;
+        if (rq < (float)-m) rq = (float)-m;
+        c = (int)rq;
+      }
+      idx[g * ORACLE_GROUP + j] = (uint8_t)(c + m);
+    }
+  }
+}
+
+/* Hadamard rotation (signs) or none, then the uniform quantizer; cache rows of
+   d * bits / 8 bytes (codebook layout) and d / 32 scales. */
+int oracle_quantize_append_uniform(const void* k, const void* v, int in_dtype, int B, int Hkv,
+                                   int n_new, int d, const int32_t* pos, const int8_t* signs,
+                                   int bits, uint8_t* k_packed, float* k_scales,
+                                   uint8_t* v_packed, float* v_scales, int64_t capacity,
+                                   int nthreads) {
+  if ((d & (d - 1)) != 0 || check_append(B, n_new, d, pos, capacity) != 0) return -1;
+  if (bits < 2 || bits > 4) return -1;
+  double* R = NULL;
+  if (signs) {
+    R = (double*)malloc(sizeof(double) * (size_t)d * d);
+    if (!R) return -2;
+    oracle_rotation_matrix(d, signs, R);
+  }
+  int ng = d / ORACLE_GROUP, rowb = d * bits / 8;
+  int64_t nvec = (int64_t)B * Hkv * n_new;
+#ifdef _OPENMP
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#endif
+  for (int64_t idx = 0; idx < nvec; ++idx) {
+    float x[512], y[512];
+    uint8_t ci[512];
+    int64_t b = idx / ((int64_t)Hkv * n_new);
+    int64_t h = (idx / n_new) % Hkv;
+    int64_t n = idx % n_new;
+    int64_t row = ((int64_t)b * Hkv + h) * capacity + pos[b] + n;
+    for (int kv = 0; kv < 2; ++kv) {
+      const void* src = kv ? v : k;
+      for (int i = 0; i < d; ++i) x[i] = load_input(src, in_dtype, idx * d + i);
+      if (R) oracle_rotate_vector(d, R, x, y);
+      else memcpy(y, x, sizeof(float) * (size_t)d);
+      oracle_uniform_quantize_vector(d, y, bits, ci, (kv ? v_scales : k_scales) + row * ng);
       oracle_cb_pack_vector(d, bits, ci, (kv ? v_packed : k_packed) + row * rowb);
     }
   }

@@ -50,6 +50,12 @@ MUTATIONS = {
     "lloyd_cell_mean_sign": ("double m = (pa - pb) / (cb - ca);", "double m = (pb - pa) / (cb - ca);"),
     "cb_value_scale_wrong_group": ("(double)sv[i / ORACLE_GROUP] * (double)C[ci[i]]",
                                    "(double)sv[0] * (double)C[ci[i]]"),
+    "uniform_divisor_m_plus_1": ("float s = amax / top;", "float s = amax / (top + 1.0f);"),
+    "uniform_round_half_away": ("float rq = nearbyintf(uq);", "float rq = roundf(uq);"),
+    "uniform_clamp_below_m": ("if (rq > (float)m) rq = (float)m;", "if (rq > (float)(m - 1)) rq = (float)(m - 1);"),
+    "uniform_twos_complement_index": ("idx[g * ORACLE_GROUP + j] = (uint8_t)(c + m);",
+                                      "idx[g * ORACLE_GROUP + j] = (uint8_t)(c & ((1 << bits) - 1));"),
+    "uniform_levels_shifted": ("levels[u] = (float)(u - m);", "levels[u] = (float)(u - m - 1);"),
     # mistakes that only show with levels that are not symmetric about zero
     "cb_threshold_assumes_symmetric": ("volatile float sum = C[i] + C[i + 1];",
                                        "volatile float sum = C[i] - C[L - 2 - i];"),

@@ -738,3 +738,115 @@ def test_cb_append_rotates_then_quantizes_rows_at_pos():
         np.testing.assert_array_equal(cache[0][0, h, 4:7], oracle.cb_pack(idx, bits))
         np.testing.assert_array_equal(cache[1][0, h, 4:7], sc)
         assert not cache[0][0, h, :4].any() and not cache[0][0, h, 7:].any()
+
+
+# ---------------------------------------------------------------------------
+# Uniform low-bit variant (Open-TQ-Metal forum summary, future work: int2; read
+# as the int4 quantizer at fewer bits): m = 2^(bits-1) - 1, s = fl32(amax / m),
+# c = clamp(rne(fl32(y / s)), -m, m), stored as index c + m in the codebook
+# layout; the decode-side levels are C[u] = u - m.
+
+def test_uniform_levels_are_the_integer_codes():
+    np.testing.assert_array_equal(oracle.uniform_levels(2), [-1, 0, 1, 2])
+    np.testing.assert_array_equal(oracle.uniform_levels(3), [-3, -2, -1, 0, 1, 2, 3, 4])
+    np.testing.assert_array_equal(oracle.uniform_levels(4), np.arange(16) - 7)
+
+
+def test_uniform_2bit_hand_values():
+    """amax 1 gives s = 1: codes are rne(y), ties to even on both sides of 0."""
+    y = np.zeros((1, 32), np.float32)
+    y[0, :8] = [1.0, 0.5, -0.5, 0.49999997, -0.50000006, 0.0, 0.75, -1.0]
+    idx, sc = oracle.uniform_quantize_vectors(y, 2)
+    assert sc[0, 0] == 1.0
+    np.testing.assert_array_equal(idx[0, :8], np.array([1, 0, 0, 0, -1, 0, 1, -1]) + 1)
+    assert np.all(idx[0, 8:] == 1)
+
+
+def test_uniform_3bit_hand_values():
+    """amax 3 gives s = 3/3 = 1; amax 1.5 gives s = 0.5 exactly."""
+    y = np.zeros((2, 32), np.float32)
+    y[0, :8] = [3.0, 2.5, 1.5, -2.5, -0.5, 0.4, -3.0, 2.6]
+    y[1, :6] = [1.5, 0.25, 0.75, -1.25, 1.0, -0.3]
+    idx, sc = oracle.uniform_quantize_vectors(y, 3)
+    assert sc[0, 0] == 1.0 and sc[1, 0] == 0.5
+    np.testing.assert_array_equal(idx[0, :8], np.array([3, 2, 2, -2, 0, 0, -3, 3]) + 3)
+    np.testing.assert_array_equal(idx[1, :6], np.array([3, 0, 2, -2, 2, -1]) + 3)
+
+
+def test_uniform_4bit_is_the_int4_quantizer():
+    """At four bits m = 7: the same scales and codes as the int4 path."""
+    rng = np.random.default_rng(70)
+    y = (rng.standard_normal((40, 128)) * np.exp(rng.uniform(-6, 6, (40, 1)))).astype(np.float32)
+    y[3] = 0.0
+    idx, sc = oracle.uniform_quantize_vectors(y, 4)
+    codes, sc4 = oracle.quantize_vectors(y)
+    np.testing.assert_array_equal(sc.view(np.uint32), sc4.view(np.uint32))
+    np.testing.assert_array_equal(idx.astype(np.int64) - 7, codes.astype(np.int64))
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_uniform_quantizer_invariants(bits):
+    """Half-step bound, the abs-max element at +-m, sign symmetry, exact
+    power-of-two scale equivariance, zero groups."""
+    m = (1 << (bits - 1)) - 1
+    rng = np.random.default_rng(71 + bits)
+    y = (rng.standard_normal((60, 128)) * np.exp(rng.uniform(-8, 8, (60, 1)))).astype(np.float32)
+    y[5, 32:64] = 0.0
+    idx, sc = oracle.uniform_quantize_vectors(y, bits)
+    c = idx.astype(np.int64) - m
+    assert c.min() >= -m and c.max() <= m
+    s = np.repeat(sc.astype(np.float64), 32, axis=1)
+    err = np.abs(y.astype(np.float64) - s * c)
+    assert np.all(err <= s * (0.5 + 1e-6))
+    g = y.reshape(60, 4, 32)
+    top = np.abs(g).argmax(axis=2)
+    for r in range(60):
+        for k in range(4):
+            if sc[r, k] > 0:
+                assert abs(c[r, 32 * k + top[r, k]]) == m
+    assert sc[5, 1] == 0.0 and np.all(idx[5, 32:64] == m)
+    idx_neg, sc_neg = oracle.uniform_quantize_vectors(-y, bits)
+    np.testing.assert_array_equal(idx_neg.astype(np.int64) - m, -c)
+    np.testing.assert_array_equal(sc_neg, sc)
+    idx2, sc2 = oracle.uniform_quantize_vectors(y * np.float32(2.0 ** -5), bits)
+    np.testing.assert_array_equal(idx2, idx)
+    np.testing.assert_array_equal(sc2, sc * np.float32(2.0 ** -5))
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_uniform_append_rotates_then_quantizes_rows_at_pos(bits):
+    rng = np.random.default_rng(72 + bits)
+    d = 128
+    s = rand_signs(rng, d)
+    k = rng.standard_normal((1, 2, 3, d)).astype(np.float32)
+    v = rng.standard_normal((1, 2, 3, d)).astype(np.float32)
+    cache = oracle.empty_cb_cache(1, 2, 8, d, bits)
+    oracle.quantize_append_uniform(k, v, [4], s, bits, cache)
+    for h in range(2):
+        for src, kp, ks in ((k, cache[0], cache[1]), (v, cache[2], cache[3])):
+            idx, sc = oracle.uniform_quantize_vectors(oracle.rotate(src[0, h], s), bits)
+            np.testing.assert_array_equal(kp[0, h, 4:7], oracle.cb_pack(idx, bits))
+            np.testing.assert_array_equal(ks[0, h, 4:7], sc)
+            assert not kp[0, h, :4].any() and not kp[0, h, 7:].any()
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_uniform_decode_is_attention_over_s_times_c(bits):
+    """A uniform cache decoded with its integer levels is softmax attention
+    over s * c (numpy brute force, rotation off)."""
+    m = (1 << (bits - 1)) - 1
+    rng = np.random.default_rng(74 + bits)
+    B, Hkv, G, T, d = 1, 2, 2, 21, 64
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    cache = oracle.empty_cb_cache(B, Hkv, T, d, bits)
+    oracle.quantize_append_uniform(k, v, [0], None, bits, cache)
+    ik = oracle.cb_unpack(cache[0].reshape(-1, cache[0].shape[-1]), d, bits).reshape(B, Hkv, T, d)
+    iv = oracle.cb_unpack(cache[2].reshape(-1, cache[2].shape[-1]), d, bits).reshape(B, Hkv, T, d)
+    khat = np.repeat(cache[1].astype(np.float64), 32, axis=-1) * (ik.astype(np.float64) - m)
+    vhat = np.repeat(cache[3].astype(np.float64), 32, axis=-1) * (iv.astype(np.float64) - m)
+    q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
+    out = oracle.sdpa_cb_decode(q, cache, [T], None, bits, oracle.uniform_levels(bits), 0.3, Hkv)
+    for h in range(Hkv * G):
+        want = _numpy_attention(q[0, h].astype(np.float64), khat[0, h // G], vhat[0, h // G], 0.3)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-12, atol=1e-13)
