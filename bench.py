@@ -243,7 +243,9 @@ def run_tq(args):
     srft = w.rotation and w.rotation_kind == "srft"
     lk, lv = wl.make_lambdas(w, seed)
     ctx = wl.make_context_lengths(w, seed)                    # cached tokens per sequence
-    if w.cb_bits:
+    if w.cb_bits and w.cb_uniform:
+        cache = tq.UniformKVCache(B, Hkv, d, w.capacity, w.cb_bits, dev, signs)
+    elif w.cb_bits:
         cache = tq.CodebookKVCache(B, Hkv, d, w.capacity, w.cb_bits, dev, signs)
     else:
         cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs,
@@ -420,14 +422,16 @@ def run_tq(args):
     kvb = kv_bytes(w, (ctx + 1).tolist())
     mma = not w.cb_bits and ((d == 128 and Hq // Hkv <= 8) or (d == 256 and Hq // Hkv <= 4))
     mma_cb = bool(w.cb_bits) and d == 128 and 5 <= Hq // Hkv <= 8
+    cb_name = (f"uniform int{w.cb_bits} codes" if w.cb_uniform else f"{w.cb_bits}-bit Max-Lloyd codebook")
+    cb_call = "tq_sdpa_uniform_decode_append" if w.cb_uniform else "tq_sdpa_cb_decode_append"
     if mma_cb:
         launches_per_step = 2
-        step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): the tensor-core "
+        step_desc = (f"{cb_call} ({cb_name}): the tensor-core "
                      "decode kernel quantizes the new token of each kv head into the cache, then "
                      "attends (split-K kernel + merge, 2 launches)")
     elif w.cb_bits:
         launches_per_step = 3
-        step_desc = (f"tq_sdpa_cb_decode_append ({w.cb_bits}-bit Max-Lloyd codebook): quantize-append "
+        step_desc = (f"{cb_call} ({cb_name}): quantize-append "
                      "of the new token, split-K decode, merge (3 launches)")
     elif srft:
         launches_per_step = 3
@@ -457,19 +461,19 @@ def run_tq(args):
         "two_call_step_us": round(two_s * 1e6, 2),
         "pct_of_8TBps": round(100 * kvb / step_s / 1e9 / NOMINAL_HBM_GBS, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": (f"{w.cb_bits}-bit codebook indices, fp32 accumulation" if w.cb_bits
+        "dtype": (f"{cb_name} (codebook layout), fp32 accumulation" if w.cb_bits
                   else "int4 codes, fp32 accumulation"), "data": "synthetic (seeded N(0,1), bf16)",
         "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": d,
                    "context": max_ctx, "decode_kernel": args.decode_kernel,
                    "rotation": (w.rotation_kind if w.rotation else False),
-                   "codes": f"{w.cb_bits}-bit Max-Lloyd codebook" if w.cb_bits else "int4",
+                   "codes": cb_name if w.cb_bits else "int4",
                    "attn_scale": scale,
                    "kv_bytes_per_step": kvb,
                    "l2": (f"rotated over {n_rot} caches: consecutive steps read {n_rot * kvb} B "
                           f"of packed cache, more than twice the {l2_bytes} B L2"),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm",
-                     "kernel": (f"{w.cb_bits}-bit codebook decode (split-K + merge)" if w.cb_bits
+                     "kernel": (f"{cb_name} decode on the codebook path (split-K + merge)" if w.cb_bits
                                 else "sdpa_int4 decode (split-K + merge)"),
                      "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4), "peak_kind": peak_kind,
@@ -770,9 +774,13 @@ def oracle_sample(w, seed, kv_head=0):
     else:
         cache = oracle.empty_cache(1, 1, w.capacity, w.head_dim)
     thr = oracle.max_threads()
-    levels = oracle.lloyd_max_gaussian(w.cb_bits).astype(np.float32) if w.cb_bits else None
+    levels = None
+    if w.cb_bits:
+        levels = (oracle.uniform_levels(w.cb_bits) if w.cb_uniform
+                  else oracle.lloyd_max_gaussian(w.cb_bits).astype(np.float32))
     s = dict(k_new=bits(k[:, :, -1:]), v_new=bits(v[:, :, -1:]), q=bits(q), signs=signs, lam=lam,
-             cache=cache, threads=thr, G=G, T=w.capacity - 1, cb_bits=w.cb_bits, levels=levels)
+             cache=cache, threads=thr, G=G, T=w.capacity - 1, cb_bits=w.cb_bits, levels=levels,
+             cb_uniform=w.cb_uniform)
     t0 = time.perf_counter()
     oracle_append(s, bits(k[:, :, :-1]), bits(v[:, :, :-1]), 0)
     s["prefill_s"] = time.perf_counter() - t0
@@ -781,7 +789,10 @@ def oracle_sample(w, seed, kv_head=0):
 
 def oracle_append(s, k, v, pos):
     import oracle
-    if s["cb_bits"]:
+    if s["cb_bits"] and s["cb_uniform"]:
+        oracle.quantize_append_uniform(k, v, [pos], s["signs"], s["cb_bits"], s["cache"],
+                                       threads=s["threads"])
+    elif s["cb_bits"]:
         oracle.quantize_append_cb(k, v, [pos], s["signs"], s["cb_bits"], s["levels"], s["cache"],
                                   threads=s["threads"])
     elif s["lam"] is None:

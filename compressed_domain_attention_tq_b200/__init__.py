@@ -4,7 +4,7 @@ sm_100a) behind the C ABI of include/tq.h; this package is its binding.
 """
 from ._lib import (TQError, decode_chunk_tokens, decode_workspace_bytes, load,
                    quantize_append, sdpa_int4_decode, status_string)
-from .cache import CodebookKVCache, Int4KVCache
+from .cache import CodebookKVCache, Int4KVCache, UniformKVCache
 
-__all__ = ["CodebookKVCache", "Int4KVCache", "TQError", "decode_chunk_tokens", "decode_workspace_bytes", "load",
+__all__ = ["CodebookKVCache", "Int4KVCache", "UniformKVCache", "TQError", "decode_chunk_tokens", "decode_workspace_bytes", "load",
            "quantize_append", "sdpa_int4_decode", "status_string"]

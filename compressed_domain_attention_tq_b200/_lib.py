@@ -29,7 +29,8 @@ SYMBOLS = ("tq_quantize_append", "tq_decode_workspace_bytes", "tq_decode_chunk_t
            "tq_decode_append_host_workspace_bytes", "tq_sdpa_int4_decode_append_host",
            "tq_decode_append_host_srft_workspace_bytes", "tq_sdpa_int4_decode_append_srft_host",
            "tq_decode_append_host_cb_workspace_bytes", "tq_sdpa_cb_decode_append_host",
-           "tq_status_string")
+           "tq_uniform_levels", "tq_quantize_append_uniform", "tq_sdpa_uniform_decode_append",
+           "tq_sdpa_uniform_decode_append_host", "tq_status_string")
 
 _lib = None
 
@@ -116,6 +117,15 @@ def load() -> ctypes.CDLL:
     lib.tq_sdpa_cb_decode_append_host.argtypes = [P, i32, P, P, i32, i32, i32, i32, i32, i32, i32, P,
                                                   P, P, P, P, i64, P, i32, P, f32, P, P, sz, P]
     lib.tq_sdpa_cb_decode_append_host.restype = i32
+    lib.tq_uniform_levels.argtypes = [i32, P]
+    lib.tq_uniform_levels.restype = i32
+    lib.tq_quantize_append_uniform.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P,
+                                               P, P, i64, P]
+    lib.tq_quantize_append_uniform.restype = i32
+    lib.tq_sdpa_uniform_decode_append.argtypes = lib.tq_sdpa_cb_decode_append.argtypes
+    lib.tq_sdpa_uniform_decode_append.restype = i32
+    lib.tq_sdpa_uniform_decode_append_host.argtypes = lib.tq_sdpa_cb_decode_append_host.argtypes
+    lib.tq_sdpa_uniform_decode_append_host.restype = i32
     lib.tq_status_string.argtypes = [i32]
     lib.tq_status_string.restype = ctypes.c_char_p
     lib.tq_set_test_hooks.argtypes = [ctypes.c_uint32]
@@ -395,6 +405,46 @@ def lloyd_max_gaussian(bits: int) -> torch.Tensor:
     return out
 
 
+def uniform_levels(bits: int) -> torch.Tensor:
+    """The levels of a uniform low-bit cache, u - (2^(bits-1) - 1) (float32 CPU tensor), from libtq."""
+    out = torch.empty(1 << bits, dtype=torch.float32)
+    rc = load().tq_uniform_levels(bits, ctypes.c_void_p(out.data_ptr()))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_uniform_levels")
+    return out
+
+
+def quantize_append_uniform(k, v, pos, signs, bits, k_packed, k_scales, v_packed, v_scales,
+                            stream=None):
+    """Quantize k, v [B][Hkv][n_new][d] into uniform low-bit cache rows pos[b] .. pos[b]+n_new-1."""
+    _need_cuda(k, v, pos, signs, k_packed, k_scales, v_packed, v_scales)
+    B, H, n, d = k.shape
+    rc = load().tq_quantize_append_uniform(_ptr(k), _ptr(v), _dtype_code(k), B, H, n, d, 32, int(bits),
+                                           _ptr(pos), _ptr(signs), _ptr(k_packed), _ptr(k_scales),
+                                           _ptr(v_packed), _ptr(v_scales), k_packed.shape[2],
+                                           _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_quantize_append_uniform")
+
+
+def sdpa_uniform_decode_append(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens,
+                               max_ctx, signs, bits, levels, attn_scale, out, workspace, stream=None):
+    """One decode step over a uniform low-bit cache (levels = uniform_levels(bits) on the device)."""
+    _need_cuda(q, k_new, v_new, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels,
+               out, workspace)
+    if k_new.dtype != v_new.dtype:
+        raise TypeError("k_new and v_new must share dtype")
+    B, Hq, d = q.shape
+    Hkv = k_packed.shape[1]
+    rc = load().tq_sdpa_uniform_decode_append(
+        _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq, Hkv, d, 32,
+        int(bits), _ptr(levels), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+        k_packed.shape[2], _ptr(ctx_lens), int(max_ctx), _ptr(signs), float(attn_scale), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != TQ_OK:
+        raise TQError(rc, "tq_sdpa_uniform_decode_append")
+
+
 def decode_cb_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx) -> int:
     return int(load().tq_decode_cb_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_ctx))
 
@@ -546,8 +596,9 @@ def bind_sdpa_int4_decode_append_srft_host(q_host, k_new_host, v_new_host, k_pac
 
 def bind_sdpa_cb_decode_append_host(q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed,
                                     v_scales, ctx_lens, max_ctx, signs, bits, levels, attn_scale,
-                                    out_host, workspace, stream=None) -> BoundCall:
-    """bind_sdpa_int4_decode_append_host for a codebook cache."""
+                                    out_host, workspace, stream=None, uniform=False) -> BoundCall:
+    """bind_sdpa_int4_decode_append_host for a codebook cache (uniform: a uniform
+    low-bit cache, tq_sdpa_uniform_decode_append_host)."""
     _host(q_host, k_new_host, v_new_host, out_host)
     _need_cuda(k_packed, k_scales, v_packed, v_scales, ctx_lens, signs, levels, workspace)
     if k_new_host.dtype != v_new_host.dtype:
@@ -563,5 +614,5 @@ def bind_sdpa_cb_decode_append_host(q_host, k_new_host, v_new_host, k_packed, k_
             sz(workspace.numel() * workspace.element_size()), _stream(stream))
     keep = (q_host, k_new_host, v_new_host, k_packed, k_scales, v_packed, v_scales, ctx_lens, signs,
             levels, out_host, workspace)
-    return BoundCall(load().tq_sdpa_cb_decode_append_host, args, "tq_sdpa_cb_decode_append_host",
-                     keep)
+    name = "tq_sdpa_uniform_decode_append_host" if uniform else "tq_sdpa_cb_decode_append_host"
+    return BoundCall(getattr(load(), name), args, name, keep)

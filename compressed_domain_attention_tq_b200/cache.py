@@ -278,3 +278,57 @@ class CodebookKVCache:
                                 ctx_lens, max_ctx, self.signs, self.bits, self.levels, attn_scale,
                                 out, lse, ws, stream)
         return out
+
+
+class UniformKVCache(CodebookKVCache):
+    """The uniform low-bit variant (Open-TQ-Metal forum summary, future work:
+    int2; the int4 quantizer at bits = 2 or 3): per group of 32 rotated
+    coordinates s = fl32(amax / m), m = 2^(bits-1) - 1, codes
+    clamp(rne(y / s), -m, m) stored as indices c + m in the codebook layout.
+    Decoded as a codebook cache whose levels are the integers u - m (the
+    levels attribute); the same calls as Int4KVCache."""
+
+    def __init__(self, batch: int, num_kv_heads: int, head_dim: int, capacity: int, bits: int = 2,
+                 device="cuda", signs: torch.Tensor | None = None):
+        super().__init__(batch, num_kv_heads, head_dim, capacity, bits, device, signs,
+                         levels=_lib.uniform_levels(bits))
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor, stream=None) -> None:
+        _lib.quantize_append_uniform(k, v, pos, self.signs, self.bits, self.k_packed, self.k_scales,
+                                     self.v_packed, self.v_scales, stream)
+
+    def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      ctx_lens: torch.Tensor, max_ctx: int, attn_scale: float | None = None,
+                      out: torch.Tensor | None = None, stream=None):
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        ws = self.workspace(q.shape[1], max_ctx)
+        _lib.sdpa_uniform_decode_append(q, k_new, v_new, self.k_packed, self.k_scales, self.v_packed,
+                                        self.v_scales, ctx_lens, max_ctx, self.signs, self.bits,
+                                        self.levels, attn_scale, out, ws, stream)
+        return out
+
+    def bind_decode_append_host(self, q_host: torch.Tensor, k_new_host: torch.Tensor,
+                                v_new_host: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int,
+                                out_host: torch.Tensor, attn_scale: float | None = None,
+                                stream=None, graph: bool = False):
+        """Int4KVCache.bind_decode_append_host for the uniform cache
+        (tq_sdpa_uniform_decode_append_host)."""
+        if attn_scale is None:
+            attn_scale = 1.0 / math.sqrt(self.head_dim)
+        need = _lib.decode_append_host_workspace_bytes(self.batch, q_host.shape[1], self.num_kv_heads,
+                                                       self.head_dim, max_ctx, q_host.dtype,
+                                                       k_new_host.dtype, "cb")
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        ws = torch.empty(need, dtype=torch.uint8, device=self.k_packed.device)
+
+        def make(s):
+            return _lib.bind_sdpa_cb_decode_append_host(q_host, k_new_host, v_new_host,
+                                                        self.k_packed, self.k_scales, self.v_packed,
+                                                        self.v_scales, ctx_lens, max_ctx, self.signs,
+                                                        self.bits, self.levels, attn_scale,
+                                                        out_host, ws, s, uniform=True)
+        return _lib.GraphedCall(make) if graph else make(stream)

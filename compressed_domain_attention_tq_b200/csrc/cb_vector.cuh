@@ -9,6 +9,11 @@
 // string.  Lane l holds coordinates E*l .. E*l+E-1 (E = D/32); the rotation is
 // the int4 warp quantizer's.  Used by the codebook quantize kernel and by the
 // decode kernel's fused append.
+//
+// With `uniform` the same row format holds the uniform low-bit variant (the
+// int4 quantizer at BITS bits: Open-TQ-Metal forum summary, future work int2):
+// m = 2^(BITS-1) - 1, s = fl32(amax / m), index = clamp(rne(fl32(y / s)), -m, m)
+// + m, read back through the levels C[u] = u - m; `levels` is not read.
 #pragma once
 #include <math.h>
 #include <stdint.h>
@@ -21,36 +26,52 @@ template <int D, int BITS>
 __device__ __forceinline__ void cb_quantize_vector_warp(const void* src, bool bf16,
                                                         const int8_t* signs, const float* levels,
                                                         uint8_t* prow_bytes, float* srow,
-                                                        int lane) {
+                                                        int lane, bool uniform = false) {
   constexpr int E = D / 32;   // coordinates per lane (E consecutive ones)
   constexpr int GL = 32 / E;  // lanes per group
   constexpr int L = 1 << BITS;
-  float t[L - 1];  // thresholds between adjacent levels
-#pragma unroll
-  for (int i = 0; i + 1 < L; ++i) t[i] = __fmul_rn(__fadd_rn(levels[i], levels[i + 1]), 0.5f);
+  constexpr int M = (1 << (BITS - 1)) - 1;  // uniform: largest code
 
   float x[E];
   load_vector_warp<D>(src, bf16, x, lane);
   rotate_vector_warp<D>(x, signs, lane);
 
-  // the group's sum of squares in fp64: this lane's E, then the group's GL lanes
-  double S = 0.0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) S += (double)x[e] * (double)x[e];
-#pragma unroll
-  for (int o = 1; o < GL; o <<= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-  const float sigma = (float)sqrt(S / 32.0);
-
   // indices of this lane's E coordinates, packed at bit BITS * j0 of the group
   uint32_t bits = 0;
+  float sigma;
+  if (uniform) {
+    float amax = 0.0f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float u = sigma > 0.0f ? __fdiv_rn(x[e], sigma) : 0.0f;
-    u = fminf(fmaxf(u, -3.0f), 3.0f);
-    uint32_t k = 0;
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
 #pragma unroll
-    for (int i = 0; i + 1 < L; ++i) k += u > t[i] ? 1u : 0u;
-    bits |= k << (BITS * e);
+    for (int o = 1; o < GL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    sigma = __fdiv_rn(amax, (float)M);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float c = amax > 0.0f ? rintf(__fdiv_rn(x[e], sigma)) : 0.0f;
+      c = fminf(fmaxf(c, (float)-M), (float)M);
+      bits |= (uint32_t)((int)c + M) << (BITS * e);
+    }
+  } else {
+    float t[L - 1];  // thresholds between adjacent levels
+#pragma unroll
+    for (int i = 0; i + 1 < L; ++i) t[i] = __fmul_rn(__fadd_rn(levels[i], levels[i + 1]), 0.5f);
+    // the group's sum of squares in fp64: this lane's E, then the group's GL lanes
+    double S = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) S += (double)x[e] * (double)x[e];
+#pragma unroll
+    for (int o = 1; o < GL; o <<= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    sigma = (float)sqrt(S / 32.0);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float u = sigma > 0.0f ? __fdiv_rn(x[e], sigma) : 0.0f;
+      u = fminf(fmaxf(u, -3.0f), 3.0f);
+      uint32_t k = 0;
+#pragma unroll
+      for (int i = 0; i + 1 < L; ++i) k += u > t[i] ? 1u : 0u;
+      bits |= k << (BITS * e);
+    }
   }
   const int g = lane / GL, j0 = E * (lane % GL);
   const int off = BITS * j0;  // bit offset of this lane's indices in the group

@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(128) cb_quantize_kernel(QuantizeArgs a) {
   cb_quantize_vector_warp<D, BITS>(static_cast<const unsigned char*>(kv ? a.v : a.k) + rem * D * eb,
                                    a.bf16, a.signs, a.levels,
                                    (kv ? a.v_packed : a.k_packed) + row * (D * BITS / 8),
-                                   (kv ? a.v_scales : a.k_scales) + row * (D / 32), lane);
+                                   (kv ? a.v_scales : a.k_scales) + row * (D / 32), lane,
+                                   a.cb_uniform != 0);
 }
 
 template <int D, int BITS>

@@ -680,8 +680,9 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
 // collects all four partial products in one accumulator; then
 // S = sum_g sigma_k[t, g] x_g.  Thread tig takes in-group coordinates 8tig ..
 // 8tig + 7 (bits 8 FMT tig .. of the group's bit string) as the index pairs
-// (8tig + 2m, 8tig + 2m + 1), m = 0..3.  Branch-free.
-template <int D, int PATH, int FMT, int TPW, bool FULL>
+// (8tig + 2m, 8tig + 2m + 1), m = 0..3.  Branch-free.  EXACT: every level is
+// an f16 (the lo parts are zero), so only the hi parts are read and multiplied.
+template <int D, int PATH, int FMT, int TPW, bool FULL, bool EXACT>
 __device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int r0, int nvalid, int tig,
                                                const int (&rho)[4], const int (&krow)[2],
                                                const WarpState<D, PATH, FMT>& st,
@@ -732,13 +733,16 @@ __device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int r0,
         const uint32_t x = pc[u][nt][g];
         uint2 e[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          e[m] = *reinterpret_cast<const uint2*>(lutp + (((x >> (2 * FMT * m)) & KM) << 3));
+        for (int m = 0; m < 4; ++m) {
+          const unsigned char* ep = lutp + (((x >> (2 * FMT * m)) & KM) << 3);
+          if (EXACT) e[m] = make_uint2(*reinterpret_cast<const uint32_t*>(ep), 0u);
+          else e[m] = *reinterpret_cast<const uint2*>(ep);
+        }
         float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], e[0].x, e[1].x);
-        mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], e[0].y, e[1].y);
+        if (!EXACT) mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], e[0].y, e[1].y);
         mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], e[2].x, e[3].x);
-        mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], e[2].y, e[3].y);
+        if (!EXACT) mma16816(c, a[1][0], a[1][1], a[1][2], a[1][3], e[2].y, e[3].y);
         const float2 x2 = __fadd2_rn(make_float2(c[0], c[1]), make_float2(c[2], c[3]));
         S[u][2 * nt] = fmaf(sk[u][2 * nt][g], x2.x, S[u][2 * nt]);
         S[u][2 * nt + 1] = fmaf(sk[u][2 * nt + 1][g], x2.y, S[u][2 * nt + 1]);
@@ -934,7 +938,7 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
 // coordinates 32g + 4 gid + e (n-tile e) of the token pairs (rho0, rho1) and
 // (rho2, rho3), hi and lo parts from the level-pair table (one lookup per row
 // and pair of coordinates), both products in the same accumulator.  Branch-free.
-template <int D, int PATH, int FMT, int TPW>
+template <int D, int PATH, int FMT, int TPW, bool EXACT>
 __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int gid,
                                            const int (&rho)[4], const float (&p)[TPW][4],
                                            const float (&sv)[TPW][4][D / 32],
@@ -986,16 +990,20 @@ __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int m = 0; m < 2; ++m)
-            lv[i][m] = *reinterpret_cast<const uint2*>(lutp + (((f[i][g] >> (2 * FMT * m)) & KM) << 3));
+          for (int m = 0; m < 2; ++m) {
+            const unsigned char* ep = lutp + (((f[i][g] >> (2 * FMT * m)) & KM) << 3);
+            if (EXACT) lv[i][m] = make_uint2(*reinterpret_cast<const uint32_t*>(ep), 0u);
+            else lv[i][m] = *reinterpret_cast<const uint2*>(ep);
+          }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int m = e >> 1;
           const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
           mma16816(st.acc[4 * g + e], a0, a1, a2, a3, prmt(lv[0][m].x, lv[1][m].x, sel),
                    prmt(lv[2][m].x, lv[3][m].x, sel));
-          mma16816(st.acc[4 * g + e], a0, a1, a2, a3, prmt(lv[0][m].y, lv[1][m].y, sel),
-                   prmt(lv[2][m].y, lv[3][m].y, sel));
+          if (!EXACT)
+            mma16816(st.acc[4 * g + e], a0, a1, a2, a3, prmt(lv[0][m].y, lv[1][m].y, sel),
+                     prmt(lv[2][m].y, lv[3][m].y, sel));
         }
       }
     }
@@ -1004,7 +1012,7 @@ __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int
 
 // One warp's share of a stage: scores, softmax update and P.V of its TPW tiles
 // (rows r0 .. r0 + 16 TPW - 1, of which the first nvalid are real tokens).
-template <int D, int PATH, int FMT, int TPW, bool FULL>
+template <int D, int PATH, int FMT, int TPW, bool FULL, bool EXACT = false>
 __device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, int nvalid, int gid,
                                             int tig, const int (&rho)[4], const int (&krow)[2],
                                             WarpState<D, PATH, FMT>& st,
@@ -1013,14 +1021,14 @@ __device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, in
   if constexpr (FMT == 0)
     tile_scores<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
   else
-    tile_scores_cb<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, lutp, S);
+    tile_scores_cb<D, PATH, FMT, TPW, FULL, EXACT>(stg, r0, nvalid, tig, rho, krow, st, lutp, S);
   tile_max<D, PATH, FMT, TPW>(tig, S, st);
   load_vscales<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, rho, sv);
   tile_weights<D, PATH, FMT, TPW>(S, sv, st, p);
   if constexpr (FMT == 0)
     tile_pv<D, PATH, FMT, TPW>(stg, r0, gid, rho, p, sv, st);
   else
-    tile_pv_cb<D, PATH, FMT, TPW>(stg, r0, gid, rho, p, sv, st, lutp);
+    tile_pv_cb<D, PATH, FMT, TPW, EXACT>(stg, r0, gid, rho, p, sv, st, lutp);
 }
 
 // End of an item: the warps' (max, sum, acc) per head are merged in shared
@@ -1173,6 +1181,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
   // and the output): entry i0 | i1 << FMT = (C[i0], C[i1]) as f16x2 hi parts
   // (round to nearest) and f16x2 lo parts (the remainders, rounded).
   float cexp = 1.0f;
+  bool exact = false;  // every normalised level is an f16: the lo parts are zero
   if constexpr (FMT != 0) {
     constexpr int L = 1 << FMT;
     float lmax = 0.0f;
@@ -1180,6 +1189,11 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
     int e = 0;
     if (lmax > 0.0f) frexpf(lmax, &e);
     cexp = ldexpf(1.0f, e);
+    exact = true;
+    for (int i = 0; i < L; ++i) {
+      const float c = ldexpf(a.levels[i], -e);
+      exact = exact && __half2float(__float2half_rn(c)) == c;
+    }
     uint2* lut = reinterpret_cast<uint2*>(smem + C::LUT);
     for (int key = threadIdx.x; key < L * L; key += C::THREADS) {
       const float c0 = ldexpf(a.levels[key & (L - 1)], -e), c1 = ldexpf(a.levels[key >> FMT], -e);
@@ -1216,7 +1230,8 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       if constexpr (FMT == 0)
         quantize_vector_warp<D>(src, a.kv_bf16, a.signs, prow, srow, lane);
       else
-        cb_quantize_vector_warp<D, FMT>(src, a.kv_bf16, a.signs, a.levels, prow, srow, lane);
+        cb_quantize_vector_warp<D, FMT>(src, a.kv_bf16, a.signs, a.levels, prow, srow, lane,
+                                        a.cb_uniform != 0);
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
     asm volatile("bar.arrive 2, 96;" ::: "memory");
@@ -1254,10 +1269,24 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       const unsigned char* stg = smem + slot * C::STAGE;
       mbar_wait(full + slot, (sc / C::NS) & 1, abort);
       const int nv = min(C::ST, t1 - t0 - k * C::ST) - r0;  // real rows from r0 on
-      if (nv >= 16 * C::TPW)
-        stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
-      else if (nv > 0)
-        stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+      if constexpr (FMT != 0) {
+        if (exact) {
+          if (nv >= 16 * C::TPW)
+            stage_tiles<D, PATH, FMT, C::TPW, true, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+          else if (nv > 0)
+            stage_tiles<D, PATH, FMT, C::TPW, false, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+        } else {
+          if (nv >= 16 * C::TPW)
+            stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+          else if (nv > 0)
+            stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+        }
+      } else {
+        if (nv >= 16 * C::TPW)
+          stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+        else if (nv > 0)
+          stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+      }
       __syncwarp();
       if (lane == 0) {
         // first the refills queued by earlier stages, then this warp leaves the

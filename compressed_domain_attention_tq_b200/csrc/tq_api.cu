@@ -143,6 +143,7 @@ struct Rotation {
   const float* lambda_v = nullptr;
   int cb_bits = 0;
   const float* levels = nullptr;
+  bool cb_uniform = false;  // uniform low-bit indices in the codebook layout (levels u - m)
 };
 
 static bool head_dim_ok(int d, const Rotation& rot) {
@@ -150,8 +151,10 @@ static bool head_dim_ok(int d, const Rotation& rot) {
 }
 
 static bool codebook_ok(const Rotation& rot) {
-  return rot.cb_bits == 0 || ((rot.cb_bits >= 2 && rot.cb_bits <= 4) && rot.levels != nullptr &&
-                              (reinterpret_cast<uintptr_t>(rot.levels) & 3u) == 0);
+  if (rot.cb_bits == 0) return true;
+  if (rot.cb_bits < 2 || rot.cb_bits > 4) return false;
+  if (rot.cb_uniform && rot.levels == nullptr) return true;  // a uniform quantize reads no levels
+  return rot.levels != nullptr && (reinterpret_cast<uintptr_t>(rot.levels) & 3u) == 0;
 }
 
 }  // namespace tq
@@ -214,6 +217,7 @@ static tq_status quantize_impl(const void* k, const void* v, tq_dtype in_dtype, 
   a.lambda_v = rot.lambda_v;
   a.cb_bits = rot.cb_bits;
   a.levels = rot.levels;
+  a.cb_uniform = rot.cb_uniform ? 1 : 0;
   const unsigned hooks = g_test_hooks.load(std::memory_order_relaxed);
   a.test_starve = (hooks & TQ_TEST_HOOK_STARVE_PIPELINE) != 0;
   a.butterfly_rotation = (hooks & TQ_TEST_HOOK_BUTTERFLY_QUANTIZE) != 0;
@@ -260,6 +264,29 @@ tq_status tq_quantize_append_cb(const void* k, const void* v, tq_dtype in_dtype,
   return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs, r,
                        k_packed, k_scales, v_packed, v_scales, capacity, cuda_stream,
                        "tq_quantize_append_cb");
+}
+
+tq_status tq_quantize_append_uniform(const void* k, const void* v, tq_dtype in_dtype,
+                                     int32_t batch, int32_t num_kv_heads, int32_t n_new,
+                                     int32_t head_dim, int32_t group, int32_t bits,
+                                     const int32_t* pos, const int8_t* signs, uint8_t* k_packed,
+                                     float* k_scales, uint8_t* v_packed, float* v_scales,
+                                     int64_t capacity, void* cuda_stream) {
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.cb_uniform = true;
+  return quantize_impl(k, v, in_dtype, batch, num_kv_heads, n_new, head_dim, group, pos, signs, r,
+                       k_packed, k_scales, v_packed, v_scales, capacity, cuda_stream,
+                       "tq_quantize_append_uniform");
+}
+
+tq_status tq_uniform_levels(int32_t bits, float* levels) {
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  if (!levels) return TQ_ERR_INVALID_ARG;
+  const int m = (1 << (bits - 1)) - 1;
+  for (int u = 0; u < (1 << bits); ++u) levels[u] = (float)(u - m);
+  return TQ_OK;
 }
 
 tq_status tq_lloyd_max_gaussian(int32_t bits, float* levels) {
@@ -462,6 +489,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
   a.lambda_v = rot.lambda_v;
   a.cb_bits = rot.cb_bits;
   a.levels = rot.levels;
+  a.cb_uniform = rot.cb_uniform ? 1 : 0;
   a.q_rot = rot.srft ? reinterpret_cast<const float*>(static_cast<unsigned char*>(workspace) +
                                                       a.plan.qrot_offset)
                      : nullptr;
@@ -516,6 +544,7 @@ static tq_status decode_impl(const void* q, tq_dtype q_dtype, const void* k_new,
     qa.lambda_v = rot.lambda_v;
     qa.cb_bits = rot.cb_bits;
     qa.levels = rot.levels;
+    qa.cb_uniform = rot.cb_uniform ? 1 : 0;
     const cudaError_t e = rot.srft ? launch_quantize_srft(qa, s)
                           : rot.cb_bits ? launch_quantize_cb(qa, s)
                                         : launch_quantize(qa, s);
@@ -653,6 +682,28 @@ tq_status tq_sdpa_cb_decode_lse(const void* q, tq_dtype q_dtype, int32_t batch,
                      head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
                      max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
                      "tq_sdpa_cb_decode_lse", lse, r);
+}
+
+tq_status tq_sdpa_uniform_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
+                                        const void* v_new, tq_dtype kv_dtype, int32_t batch,
+                                        int32_t num_q_heads, int32_t num_kv_heads,
+                                        int32_t head_dim, int32_t group, int32_t bits,
+                                        const float* levels, uint8_t* k_packed, float* k_scales,
+                                        uint8_t* v_packed, float* v_scales, int64_t capacity,
+                                        const int32_t* ctx_lens, int32_t max_ctx,
+                                        const int8_t* signs, float attn_scale, float* out,
+                                        void* workspace, size_t workspace_bytes,
+                                        void* cuda_stream) {
+  if (!k_new || !v_new || !levels) return TQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  r.cb_uniform = true;
+  return decode_impl(q, q_dtype, k_new, v_new, kv_dtype, batch, num_q_heads, num_kv_heads,
+                     head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity, ctx_lens,
+                     max_ctx, signs, attn_scale, out, workspace, workspace_bytes, cuda_stream,
+                     "tq_sdpa_uniform_decode_append", nullptr, r);
 }
 
 tq_status tq_sdpa_cb_decode_append(const void* q, tq_dtype q_dtype, const void* k_new,
@@ -861,6 +912,25 @@ tq_status tq_sdpa_int4_decode_append_srft_host(
                    num_kv_heads, head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity,
                    ctx_lens, max_ctx, signs, attn_scale, out_host, workspace, workspace_bytes,
                    cuda_stream, "tq_sdpa_int4_decode_append_srft_host", r);
+}
+
+tq_status tq_sdpa_uniform_decode_append_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out_host, void* workspace,
+    size_t workspace_bytes, void* cuda_stream) {
+  if (!levels) return TQ_ERR_INVALID_ARG;
+  if (bits < 2 || bits > 4) return TQ_ERR_UNSUPPORTED;
+  Rotation r;
+  r.cb_bits = bits;
+  r.levels = levels;
+  r.cb_uniform = true;
+  return host_step(q_host, q_dtype, k_new_host, v_new_host, kv_dtype, batch, num_q_heads,
+                   num_kv_heads, head_dim, group, k_packed, k_scales, v_packed, v_scales, capacity,
+                   ctx_lens, max_ctx, signs, attn_scale, out_host, workspace, workspace_bytes,
+                   cuda_stream, "tq_sdpa_uniform_decode_append_host", r);
 }
 
 tq_status tq_sdpa_cb_decode_append_host(

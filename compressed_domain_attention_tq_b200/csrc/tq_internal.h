@@ -49,6 +49,7 @@ struct QuantizeArgs {
   const float* lambda_v = nullptr;
   int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
   const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
+  int cb_uniform = 0;               // uniform low-bit variant (abs-max scale, index c + m) of cb_bits
   int test_starve = 0;              // test hook: the tensor-core kernel withholds its first copy
   int butterfly_rotation = 0;       // test hook: CUDA-core butterflies instead of the tensor cores
 };
@@ -94,6 +95,7 @@ struct DecodeArgs {
   const float* lambda_v = nullptr;
   int cb_bits = 0;                  // codebook variant: bits per index (2, 3, 4), else 0
   const float* levels = nullptr;    // codebook variant: 2^cb_bits increasing levels (device)
+  int cb_uniform = 0;               // the fused append writes uniform low-bit indices
   int inputs_pending = 0;           // q, k_new and v_new are written by the preceding kernel:
                                     // the tensor-core decode is launched as its programmatic
                                     // dependent and waits for it before reading them

@@ -43,6 +43,7 @@ class Workload:
     append_per_step: int = 1      # tokens quantize-appended per decode step
     rotation_kind: str = "hadamard"   # "hadamard" or "srft" (when rotation is on)
     cb_bits: int = 0                  # codebook variant: bits per index (2, 3, 4); 0 = int4
+    cb_uniform: bool = False          # with cb_bits: the uniform low-bit variant (abs-max, index c + m)
     lambda_spread: float = 0.25       # srft: lambda = 2^U(-spread, spread) per coordinate
     notes: str = field(default="", compare=False)
 
@@ -99,6 +100,18 @@ WORKLOADS = {
         context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
         attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0, cb_bits=3,
         notes="the 128K GQA layer with 3-bit Max-Lloyd codebook indices (AdapTQ)"),
+    "llama70b_gqa_128k_int2": Workload(
+        "llama70b_gqa_128k_int2", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0, cb_bits=2,
+        cb_uniform=True,
+        notes="the 128K GQA layer with uniform int2 codes (abs-max, codes -1..1; Open-TQ-Metal int2)"),
+    "llama70b_gqa_128k_int3": Workload(
+        "llama70b_gqa_128k_int3", batch=1, num_q_heads=64, num_kv_heads=8, head_dim=128,
+        context=131072, capacity=131073, in_dtype=torch.bfloat16, rotation=True,
+        attn_scales=(1 / math.sqrt(128),), outlier_channels=4, outlier_scale=10.0, cb_bits=3,
+        cb_uniform=True,
+        notes="the 128K GQA layer with uniform int3 codes (abs-max, codes -3..3)"),
     "mha32_d96_32k": Workload(
         "mha32_d96_32k", batch=1, num_q_heads=32, num_kv_heads=32, head_dim=96, context=32768,
         capacity=32769, in_dtype=torch.bfloat16, rotation=True,
@@ -204,4 +217,4 @@ def shrink(w: Workload, context: int, batch: int | None = None,
                     outlier_channels=w.outlier_channels, outlier_scale=w.outlier_scale,
                     heavy_row_frac=w.heavy_row_frac, heavy_scale=w.heavy_scale, ragged=rag,
                     append_per_step=w.append_per_step, rotation_kind=w.rotation_kind,
-                    lambda_spread=w.lambda_spread, cb_bits=w.cb_bits)
+                    lambda_spread=w.lambda_spread, cb_bits=w.cb_bits, cb_uniform=w.cb_uniform)

@@ -482,6 +482,53 @@ TQ_API tq_status tq_sdpa_cb_decode_append_host(
     size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * Uniform low-bit variant (Open-TQ-Metal forum summary, future work: int2;
+ * read as the int4 quantizer at fewer bits).  With m = 2^(bits-1) - 1 each
+ * group of 32 rotated coordinates y stores
+ *     s = fl32(amax / m) (IEEE fp32 division; s = amax at two bits),
+ *     index_j = clamp(rne(fl32(y_j / s)), -m, m) + m   (0 codes when s = 0),
+ * in the codebook layout above, scales = s.  The value is s * (index - m): a
+ * uniform cache is a codebook cache whose levels are the integers u - m
+ * (tq_uniform_levels), so tq_sdpa_cb_decode, tq_sdpa_cb_decode_lse and
+ * tq_decode_cb_workspace_bytes serve it with those levels.  Only the calls
+ * that quantize differ: tq_quantize_append_uniform, and the decode steps that
+ * append the new token, whose levels argument must hold tq_uniform_levels(bits)
+ * on the device.  bits 2, 3 or 4 (4 gives the int4 codes in this layout);
+ * arguments, alignment and errors as the codebook calls.
+ */
+
+/* levels[u] = u - m for u < 2^bits, written to a HOST array of 2^bits floats. */
+TQ_API tq_status tq_uniform_levels(int32_t bits, float* levels);
+
+/* tq_quantize_append into a uniform low-bit cache (one warp per vector). */
+TQ_API tq_status tq_quantize_append_uniform(
+    const void* k, const void* v, tq_dtype in_dtype, int32_t batch, int32_t num_kv_heads,
+    int32_t n_new, int32_t head_dim, int32_t group, int32_t bits, const int32_t* pos,
+    const int8_t* signs, uint8_t* k_packed, float* k_scales, uint8_t* v_packed, float* v_scales,
+    int64_t capacity, void* cuda_stream);
+
+/* tq_sdpa_cb_decode_append for a uniform cache: the new token is quantized
+ * with the uniform rule (inside the decode launch where the codebook decode
+ * does that), then the decode runs with `levels` (= tq_uniform_levels). */
+TQ_API tq_status tq_sdpa_uniform_decode_append(
+    const void* q, tq_dtype q_dtype, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+    int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t group,
+    int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales, uint8_t* v_packed,
+    float* v_scales, int64_t capacity, const int32_t* ctx_lens, int32_t max_ctx,
+    const int8_t* signs, float attn_scale, float* out, void* workspace, size_t workspace_bytes,
+    void* cuda_stream);
+
+/* tq_sdpa_uniform_decode_append with q, k_new, v_new and out in HOST memory
+ * (as tq_sdpa_cb_decode_append_host; its workspace size call serves). */
+TQ_API tq_status tq_sdpa_uniform_decode_append_host(
+    const void* q_host, tq_dtype q_dtype, const void* k_new_host, const void* v_new_host,
+    tq_dtype kv_dtype, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t group, int32_t bits, const float* levels, uint8_t* k_packed, float* k_scales,
+    uint8_t* v_packed, float* v_scales, int64_t capacity, const int32_t* ctx_lens,
+    int32_t max_ctx, const int8_t* signs, float attn_scale, float* out_host, void* workspace,
+    size_t workspace_bytes, void* cuda_stream);
+
+/*
  * tq_set_test_hooks -- testing only; leave at 0 (the default) in normal use.
  * Sets process-wide switches read once by every later decode or quantize
  * call:

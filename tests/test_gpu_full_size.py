@@ -19,7 +19,7 @@ import pytest
 import torch
 
 import oracle
-from compressed_domain_attention_tq_b200 import CodebookKVCache, Int4KVCache
+from compressed_domain_attention_tq_b200 import CodebookKVCache, Int4KVCache, UniformKVCache
 from compressed_domain_attention_tq_b200 import workloads as wl
 from conftest import require_cuda
 from helpers import THREADS, check_attention, to_oracle
@@ -128,7 +128,7 @@ def test_full_size_mha32_d96_32k():
 
 
 def _run_workload_cb(name, seed=0, sample_rows=32, sample_heads=2):
-    """Codebook workloads: bulk append by the CUDA path, one appended token,
+    """Codebook and uniform low-bit workloads: bulk append by the CUDA path, one appended token,
     decode over the whole context; sampled rows' indices and scales and
     sampled kv heads' outputs against the oracle (same gates as the codebook
     tests: at most 0.01% of indices differ, each by one level, scales within 4
@@ -141,7 +141,8 @@ def _run_workload_cb(name, seed=0, sample_rows=32, sample_heads=2):
     G = Hq // Hkv
     signs = wl.make_signs(d, seed) if w.rotation else None
     ctx = wl.make_context_lengths(w, seed)
-    cache = CodebookKVCache(B, Hkv, d, w.capacity, bits, dev, signs)
+    cache = (UniformKVCache(B, Hkv, d, w.capacity, bits, dev, signs) if w.cb_uniform
+             else CodebookKVCache(B, Hkv, d, w.capacity, bits, dev, signs))
     k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
     cache.append(k_all, v_all, torch.zeros(B, dtype=torch.int32, device=dev))
     k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
@@ -162,8 +163,12 @@ def _run_workload_cb(name, seed=0, sample_rows=32, sample_heads=2):
         xk = k_all[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
         xv = v_all[b:b + 1, h:h + 1, t:t + 1].contiguous().cpu()
         ref = oracle.empty_cb_cache(1, 1, 1, d, bits)
-        oracle.quantize_append_cb(to_oracle(xk), to_oracle(xv), np.zeros(1, np.int32), sg, bits,
-                                  lv.numpy(), ref)
+        if w.cb_uniform:
+            oracle.quantize_append_uniform(to_oracle(xk), to_oracle(xv), np.zeros(1, np.int32), sg,
+                                           bits, ref)
+        else:
+            oracle.quantize_append_cb(to_oracle(xk), to_oracle(xv), np.zeros(1, np.int32), sg, bits,
+                                      lv.numpy(), ref)
         for packed, scales, rp, rs in ((cache.k_packed, cache.k_scales, ref[0], ref[1]),
                                        (cache.v_packed, cache.v_scales, ref[2], ref[3])):
             got_i = oracle.cb_unpack(packed[b, h, t:t + 1].cpu().numpy(), d, bits).astype(np.int64)
@@ -190,6 +195,7 @@ def _run_workload_cb(name, seed=0, sample_rows=32, sample_heads=2):
                            f"{name} b={b} kv head {h}")
 
 
-@pytest.mark.parametrize("name", ["llama70b_gqa_128k_cb2", "llama70b_gqa_128k_cb3"])
+@pytest.mark.parametrize("name", ["llama70b_gqa_128k_cb2", "llama70b_gqa_128k_cb3",
+                                  "llama70b_gqa_128k_int2", "llama70b_gqa_128k_int3"])
 def test_full_size_codebook_128k(name):
     _run_workload_cb(name)
