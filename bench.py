@@ -272,14 +272,16 @@ def run_tq(args):
         code_bytes = d * w.cb_bits // 8 if w.cb_bits else d // 2
         moved = k_all.numel() * k_all.element_size() * 2 + nvec * (code_bytes + 4 * (d // 32))
         hbm_peak, peak_kind = measured_peaks()
-        tc_rotation = (w.rotation and not srft and not w.cb_bits and d == 128 and
-                       k_all.dtype == torch.bfloat16 and nvec > 8192)
+        tc_rotation = (w.rotation and not w.cb_bits and k_all.dtype == torch.bfloat16 and nvec > 8192
+                       and (d == 128 or (srft and d <= 128)))
         prefill = {"tokens": int(k_all.shape[2]), "us": round(t * 1e6, 2),
                    "tokens_per_s": round(B * k_all.shape[2] / t, 1),
                    "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),
                    "bytes_moved": int(moved),
                    "roofline_frac": round(moved / t / 1e9 / hbm_peak, 3), "peak_kind": peak_kind,
-                   "kernel": ("quantize_tc_kernel (rotation as a tcgen05 bf16 product)" if tc_rotation
+                   "kernel": (("quantize_srft_tc_kernel (Hartley transform as a tcgen05 product, "
+                               "three bf16 parts)" if srft else
+                               "quantize_tc_kernel (rotation as a tcgen05 bf16 product)") if tc_rotation
                               else "CUDA-core quantize kernel"),
                    "timing": "min of 3 calls, each after a 256 MiB L2 flush"}
     else:

@@ -36,6 +36,7 @@ namespace {
 
 constexpr int kQWarps = 8;  // warps per quantize CTA
 constexpr int kTeamMinTokens = 64;  // appends of at least this many tokens per row use the team kernel
+constexpr int64_t kSrftTcMinVectors = 8192;  // bulk appends of more vectors use the tensor-core kernel
 constexpr float kRneMagic = 12582912.0f;                   // 1.5 * 2^23: x + M rounds x to an integer
 constexpr float kBracketLo = 1.0f - 4.76837158203125e-07f;  // 1 - 2^-21 (exact)
 constexpr float kBracketHi = 1.0f + 4.76837158203125e-07f;  // 1 + 2^-21 (exact)
@@ -494,6 +495,8 @@ __global__ void __launch_bounds__(32 * M) srft_merge_kernel(DecodeArgs a) {
 template <int M>
 cudaError_t launch_quantize_srft_m(const QuantizeArgs& a, cudaStream_t stream) {
   const int64_t pairs = (int64_t)a.B * a.Hkv * a.n_new;
+  // bulk bf16 appends at d <= 128: the transform as a tensor-core product
+  if (2 * pairs > kSrftTcMinVectors && quantize_srft_tc_supported(a)) return launch_quantize_srft_tc(a, stream);
   // d = 128, 256 with a prefill-sized n_new: d / 16 lanes per pair.  Appends of
   // fewer tokens keep the one-warp kernel, the transform of the decode step's
   // fused append, so both give the same rows; the team kernel's own rounding

@@ -157,6 +157,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 bool srft_head_dim_supported(int d);
 cudaError_t launch_quantize_srft(const QuantizeArgs& a, cudaStream_t stream);
+bool quantize_srft_tc_supported(const QuantizeArgs& a);  // bf16, d = 32 .. 128 (multiple of 32)
+cudaError_t launch_quantize_srft_tc(const QuantizeArgs& a, cudaStream_t stream);
 cudaError_t launch_srft_query(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_srft(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_srft_prep(const QuantizeArgs& qa, const DecodeArgs& a, cudaStream_t stream);
