@@ -228,6 +228,39 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^e as a float for |e| <= 126
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
+// The NG fp32 scales of one row (rows are NG * 4 bytes: 16-byte units when NG
+// is a multiple of 4, else 4-byte aligned).
+template <int NG>
+__device__ __forceinline__ void load_row_scales(const float* p, float (&out)[NG]) {
+  if constexpr (NG % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < NG / 4; ++q) {
+      const float4 v = reinterpret_cast<const float4*>(p)[q];
+      out[4 * q] = v.x;
+      out[4 * q + 1] = v.y;
+      out[4 * q + 2] = v.z;
+      out[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < NG; ++g) out[g] = p[g];
+  }
+}
+
+// K codes of group g for one token: the half-words of sub-blocks 2tig and
+// 2tig + 1 (in-group coordinates 8tig .. 8tig + 7) in one word.  kw holds the
+// two sub-blocks' bytes as words: NG = 4, 8: sub-block 0 in words 0 .. NG/2 - 1,
+// sub-block 1 after it; NG = 3: 12 bytes, g0 g1 | g2 g0' | g1' g2'.
+template <int NG>
+__device__ __forceinline__ uint32_t kcode_word(const uint32_t (&kw)[NG], int g) {
+  if constexpr (NG == 3) {
+    return g == 0 ? prmt(kw[0], kw[1], 0x7610u) : g == 1 ? prmt(kw[0], kw[2], 0x5432u)
+                                                          : prmt(kw[1], kw[2], 0x7610u);
+  } else {
+    return prmt(kw[g / 2], kw[NG / 2 + g / 2], (g & 1) ? 0x7632u : 0x5410u);
+  }
+}
+
 // ------------------------------------------------------------ configuration
 
 // Batches up to this size use the list of non-empty items (its prefix sums
@@ -237,24 +270,28 @@ constexpr int kMaxListB = 1024;
 template <int D, int PATH, int FMT>
 struct Cfg {
   static constexpr int NW = 8;                  // warps per CTA (all consumers)
-  static constexpr int TPW = D == 128 ? 2 : 1;  // 16-token tiles per warp per stage
+  static constexpr int TPW = D == 256 ? 1 : 2;  // 16-token tiles per warp per stage
   static constexpr int THREADS = 32 * NW;
   static constexpr int ST = 16 * TPW * NW;      // tokens per pipeline stage
   static constexpr int NG = D / 32;             // quantization groups per vector
   static constexpr int RB = FMT ? D * FMT / 8 : D / 2;  // packed bytes per row
   static constexpr int NH = PATH == 0 ? 8 : 4;  // query heads per kv head (max)
   static constexpr int NACC = PATH == 0 ? 4 * NG : 2 * NG;  // accumulator fragments
-  static constexpr int NS = D == 128 ? 4 : 3;                // pipeline stages
+  static constexpr int NS = D == 256 ? 3 : 4;                // pipeline stages
+  // scale rows of 12 bytes (d = 96) are not 16-byte copy units: a stage's
+  // scales arrive as the 16-byte aligned superset, SPAD bytes more per region
+  static constexpr int SPAD = (NG % 4) ? 32 : 0;
   static constexpr int KC = 0;                               // stage: packed K rows
   static constexpr int VC = ST * RB;                         //        packed V rows
   static constexpr int KS = 2 * ST * RB;                     //        K scales
-  static constexpr int VS = KS + ST * NG * 4;                //        V scales
-  static constexpr int STAGE = VS + ST * NG * 4;
+  static constexpr int VS = KS + ST * NG * 4 + SPAD;         //        V scales
+  static constexpr int STAGE = VS + ST * NG * 4 + SPAD;
   static constexpr int al(int x) { return (x + 127) / 128 * 128; }  // 128-byte regions
   static constexpr int BAR = NS * STAGE;                     // uint64 full[NS]
   static constexpr int CNT = al(BAR + 8 * NS);               // int finished-warp count[NS]
   static constexpr int CUR = al(CNT + 4 * NS);               // int refill cursor[8], queue[3]
-  static constexpr int QA = al(CUR + 44);                    // f16 [NG][2][16][16] score A
+  static constexpr int SKEW = al(CUR + 44);                  // int [NS] first scale row's byte offset
+  static constexpr int QA = al(SKEW + 4 * NS);               // f16 [NG][2][16][16] score A
   static constexpr int QS = al(QA + NG * 2 * 16 * 16 * 2);   // float [NH][D] query
   static constexpr int QEXP = al(QS + 4 * NH * D);           // float [NH]
   static constexpr int QK8 = al(QEXP + 4 * 8);               // float [NH][NG] -8 sum_g q
@@ -345,17 +382,42 @@ __device__ __forceinline__ bool issue_next(const DecodeArgs& a, unsigned char* s
   if (a.q_rot_overlap == 2 && t + n == t1 &&
       t1 == clamp_ctx_mma(a.ctx_lens[b], a.max_ctx))  // holds the row the preceding grid appends
     asm volatile("griddepcontrol.wait;" ::: "memory");
-  const uint32_t cb = n * C::RB, sb = n * C::NG * 4;
+  const uint32_t cb = n * C::RB;
   unsigned char* stg = smem + slot * C::STAGE;
   const int64_t row = ((int64_t)b * a.Hkv + kvh) * a.capacity + t;
   uint64_t* bar = full + slot;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // earlier reads of the slot
+  // scales: bytes [s0, s1) of each scales tensor; with rows of 16-byte multiples
+  // one copy, else the 16-byte aligned superset from a0 (the first row lands
+  // s0 - a0 bytes into the region), its last few bytes by plain loads where the
+  // superset would run past the end of the tensor
+  const int64_t s0 = row * C::NG * 4, s1 = (row + n) * C::NG * 4;
+  int64_t a0 = s0, bulk_end = s1;
+  if constexpr (C::SPAD != 0) {
+    const int64_t tot = (int64_t)a.B * a.Hkv * a.capacity * C::NG * 4;
+    a0 = s0 & ~(int64_t)15;
+    const int64_t a1 = (s1 + 15) & ~(int64_t)15;
+    bulk_end = a1 <= tot ? a1 : (tot & ~(int64_t)15);
+  }
+  const uint32_t sb = (uint32_t)(bulk_end - a0);
+  reinterpret_cast<int*>(smem + C::SKEW)[slot] = (int)(s0 - a0);
   if (!(a.test_starve && cur[5] == 0)) {  // test hook: the first stage never arrives
+    if constexpr (C::SPAD != 0) {
+      for (int64_t o = bulk_end; o < s1; o += 4) {  // < 16 bytes at the end of the tensor
+        const uint32_t d = (uint32_t)(o - a0);
+        *reinterpret_cast<float*>(stg + C::KS + d) = *reinterpret_cast<const float*>(
+            reinterpret_cast<const unsigned char*>(a.k_scales) + o);
+        *reinterpret_cast<float*>(stg + C::VS + d) = *reinterpret_cast<const float*>(
+            reinterpret_cast<const unsigned char*>(a.v_scales) + o);
+      }
+    }
     mbar_arrive_expect_tx(bar, 2 * cb + 2 * sb);
     bulk_g2s(stg + C::KC, a.k_packed + row * C::RB, cb, bar);
     bulk_g2s(stg + C::VC, a.v_packed + row * C::RB, cb, bar);
-    bulk_g2s(stg + C::KS, a.k_scales + row * C::NG, sb, bar);
-    bulk_g2s(stg + C::VS, a.v_scales + row * C::NG, sb, bar);
+    if (sb > 0) {
+      bulk_g2s(stg + C::KS, reinterpret_cast<const unsigned char*>(a.k_scales) + a0, sb, bar);
+      bulk_g2s(stg + C::VS, reinterpret_cast<const unsigned char*>(a.v_scales) + a0, sb, bar);
+    }
   }
   cur[0] = it;
   cur[1] = t + C::ST;
@@ -450,9 +512,16 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
         continue;
       }
       const int64_t base = ((int64_t)b * a.Hq + (int64_t)kvh * G + h) * D + lane * E;
-      if (a.q_rot != nullptr) {  // SRFT variant: the query is already rotated (fp32)
+      if (E % 4 != 0) {  // d = 96: E = 3 consecutive values, 4-byte loads
+        const float* src = a.q_rot != nullptr ? a.q_rot + base : nullptr;
 #pragma unroll
-        for (int e = 0; e < E; e += 4) {
+        for (int e = 0; e < E; ++e)
+          x[e] = src ? src[e]
+                     : a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[base + e])
+                                : static_cast<const float*>(a.q)[base + e];
+      } else if (a.q_rot != nullptr) {  // SRFT variant: the query is already rotated (fp32)
+#pragma unroll
+        for (int e = 0; e < (E % 4 == 0 ? E : 0); e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(a.q_rot + base + e);
           x[e] = v.x;
           x[e + 1] = v.y;
@@ -477,7 +546,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
           x[e] = __uint_as_float(e & 1 ? (u[e / 2] & 0xFFFF0000u) : (u[e / 2] << 16));
       } else {
 #pragma unroll
-        for (int e = 0; e < E; e += 4) {
+        for (int e = 0; e < (E % 4 == 0 ? E : 0); e += 4) {
           const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + base + e);
           x[e] = v.x;
           x[e + 1] = v.y;
@@ -492,6 +561,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
     if (warp >= C::NW / 2 || h >= C::NH) break;
     float* x = xs[hh];
     if (h < G) {
+      if constexpr ((E & (E - 1)) == 0) {  // the Hadamard rotation needs a power-of-two width
       if (wht) {
 #pragma unroll
         for (int e = 0; e < E; ++e) x[e] *= (float)sg[e];
@@ -511,6 +581,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
             const float v = __shfl_xor_sync(kFull, x[e], bit);
             x[e] = (lane & bit) ? v - x[e] : x[e] + v;
           }
+      }
       }
       const float mul = a.attn_scale * kLog2e * (wht ? rsqrtf((float)D) : 1.0f);
       float amax = 0.0f;
@@ -600,46 +671,50 @@ __device__ __forceinline__ void scale_acc(WarpState<D, PATH, FMT>& st, float f) 
 // MMAs give x = 2^-24 sum_j q_j (c_j + 8) (kcodes_lo / kcodes_hi), and the
 // group's term is s_k (2^24 x - 8 sum_j q_j).
 template <int D, int PATH, int FMT, int TPW, bool FULL>
-__device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, int nvalid, int tig,
+__device__ __forceinline__ void tile_scores(const unsigned char* stg, int skew, int r0, int nvalid, int tig,
                                             const int (&rho)[4], const int (&krow)[2],
                                             const WarpState<D, PATH, FMT>& st, float (&S)[TPW][4]) {
   using C = Cfg<D, PATH, FMT>;
   constexpr int NG = C::NG, RB = C::RB, SB = 2 * NG;  // SB: bytes of one of a row's 8 sub-blocks
   const unsigned char* kc = stg + C::KC + r0 * RB;
-  const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
+  const float* ks = reinterpret_cast<const float*>(stg + C::KS + skew) + r0 * NG;
   uint32_t kw[TPW][2][NG];  // per tile and n-tile: sub-blocks 2tig, 2tig+1 of token krow[nt]
   float sk[TPW][4][NG];
 #pragma unroll
   for (int u = 0; u < TPW; ++u) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const uint4* kp = reinterpret_cast<const uint4*>(kc + (16 * u + krow[nt]) * RB + 2 * SB * tig);
+      const unsigned char* kb = kc + (16 * u + krow[nt]) * RB + 2 * SB * tig;
+      if constexpr (NG % 4 == 0) {
+        const uint4* kp = reinterpret_cast<const uint4*>(kb);
 #pragma unroll
-      for (int q = 0; q < NG / 4; ++q) {
-        const uint4 v = kp[q];
-        kw[u][nt][4 * q] = v.x;
-        kw[u][nt][4 * q + 1] = v.y;
-        kw[u][nt][4 * q + 2] = v.z;
-        kw[u][nt][4 * q + 3] = v.w;
+        for (int q = 0; q < NG / 4; ++q) {
+          const uint4 v = kp[q];
+          kw[u][nt][4 * q] = v.x;
+          kw[u][nt][4 * q + 1] = v.y;
+          kw[u][nt][4 * q + 2] = v.z;
+          kw[u][nt][4 * q + 3] = v.w;
+        }
+      } else {  // 12 bytes at a 4-byte aligned offset
+#pragma unroll
+        for (int q = 0; q < NG; ++q) kw[u][nt][q] = reinterpret_cast<const uint32_t*>(kb)[q];
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int q = 0; q < NG / 4; ++q) {
-        const float4 v = reinterpret_cast<const float4*>(ks + (16 * u + rho[i]) * NG)[q];
-        sk[u][i][4 * q] = v.x;
-        sk[u][i][4 * q + 1] = v.y;
-        sk[u][i][4 * q + 2] = v.z;
-        sk[u][i][4 * q + 3] = v.w;
-      }
+    for (int i = 0; i < 4; ++i) load_row_scales<NG>(ks + (16 * u + rho[i]) * NG, sk[u][i]);
   }
   float k8[NG];  // -8 sum_g q of this thread's head
+  if constexpr (NG % 4 == 0) {
 #pragma unroll
-  for (int q = 0; q < NG / 4; ++q)
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(k8[4 * q]), "=f"(k8[4 * q + 1]), "=f"(k8[4 * q + 2]), "=f"(k8[4 * q + 3])
-                 : "r"(st.k8_addr + 16 * q));
+    for (int q = 0; q < NG / 4; ++q)
+      asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                   : "=f"(k8[4 * q]), "=f"(k8[4 * q + 1]), "=f"(k8[4 * q + 2]), "=f"(k8[4 * q + 3])
+                   : "r"(st.k8_addr + 16 * q));
+  } else {
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(k8[q]) : "r"(st.k8_addr + 4 * q));
+  }
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
@@ -654,8 +729,7 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         // in-group coordinates 8tig .. 8tig+7 of group g, nibble j <-> 8tig + j
-        const uint32_t X =
-            prmt(kw[u][nt][g / 2], kw[u][nt][NG / 2 + g / 2], (g & 1) ? 0x7632u : 0x5410u);
+        const uint32_t X = kcode_word<NG>(kw[u][nt], g);
         const uint32_t Y = X >> 8;
         float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         mma16816(c, a[0][0], a[0][1], a[0][2], a[0][3], kcodes_lo(X), kcodes_hi(X));
@@ -683,7 +757,7 @@ __device__ __forceinline__ void tile_scores(const unsigned char* stg, int r0, in
 // (8tig + 2m, 8tig + 2m + 1), m = 0..3.  Branch-free.  EXACT: every level is
 // an f16 (the lo parts are zero), so only the hi parts are read and multiplied.
 template <int D, int PATH, int FMT, int TPW, bool FULL, bool EXACT>
-__device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int r0, int nvalid, int tig,
+__device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int skew, int r0, int nvalid, int tig,
                                                const int (&rho)[4], const int (&krow)[2],
                                                const WarpState<D, PATH, FMT>& st,
                                                const unsigned char* lutp, float (&S)[TPW][4]) {
@@ -691,7 +765,7 @@ __device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int r0,
   constexpr int NG = C::NG, RB = C::RB, GB = 4 * FMT;  // GB: bytes per group
   constexpr uint32_t KM = (1u << (2 * FMT)) - 1;  // key mask
   const unsigned char* kc = stg + C::KC + r0 * RB;
-  const float* ks = reinterpret_cast<const float*>(stg + C::KS) + r0 * NG;
+  const float* ks = reinterpret_cast<const float*>(stg + C::KS + skew) + r0 * NG;
   // the thread's 8 FMT bits of a group start at byte FMT tig of the group
   const int wo = (FMT * tig) >> 2, sh = 8 * ((FMT * tig) & 3);
   uint32_t pc[TPW][2][NG];
@@ -779,24 +853,20 @@ __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], Warp
 
 // V scales of the warp's rows (unless FULL, zero past nvalid).
 template <int D, int PATH, int FMT, int TPW, bool FULL>
-__device__ __forceinline__ void load_vscales(const unsigned char* stg, int r0, int nvalid,
+__device__ __forceinline__ void load_vscales(const unsigned char* stg, int skew, int r0, int nvalid,
                                              const int (&rho)[4], float (&sv)[TPW][4][D / 32]) {
   using C = Cfg<D, PATH, FMT>;
   constexpr int NG = C::NG;
-  const float* vs = reinterpret_cast<const float*>(stg + C::VS) + r0 * NG;
+  const float* vs = reinterpret_cast<const float*>(stg + C::VS + skew) + r0 * NG;
 #pragma unroll
   for (int u = 0; u < TPW; ++u)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const bool ok = FULL || 16 * u + rho[i] < nvalid;
+      float v[NG];
+      load_row_scales<NG>(vs + (16 * u + rho[i]) * NG, v);
 #pragma unroll
-      for (int q = 0; q < NG / 4; ++q) {
-        const float4 v = reinterpret_cast<const float4*>(vs + (16 * u + rho[i]) * NG)[q];
-        sv[u][i][4 * q] = ok ? v.x : 0.0f;
-        sv[u][i][4 * q + 1] = ok ? v.y : 0.0f;
-        sv[u][i][4 * q + 2] = ok ? v.z : 0.0f;
-        sv[u][i][4 * q + 3] = ok ? v.w : 0.0f;
-      }
+      for (int g = 0; g < NG; ++g) sv[u][i][g] = ok ? v[g] : 0.0f;
     }
 }
 
@@ -871,11 +941,15 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
   const unsigned char* vc = stg + C::VC + r0 * RB;
 #pragma unroll
   for (int u = 0; u < TPW; ++u) {
-    uint32_t vw[4][NG / 2];  // sub-block gid of rows rho[0..3] of tile u
+    uint32_t vw[4][(NG + 1) / 2];  // sub-block gid of rows rho[0..3] of tile u (group pairs)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const unsigned char* vp = vc + (16 * u + rho[i]) * RB + SB * gid;
-      if (NG == 4) {
+      if constexpr (NG == 3) {  // 6 bytes at a 2-byte aligned offset: g0 g1 | g2
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(vp);
+        vw[i][0] = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+        vw[i][1] = h[2];
+      } else if (NG == 4) {
         const uint2 v = *reinterpret_cast<const uint2*>(vp);
         vw[i][0] = v.x;
         vw[i][1] = v.y;
@@ -893,12 +967,14 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
 #pragma unroll
     for (int gp = 0; gp < NG; gp += 2) {
       // P' = p' * s_v of rows rho[0..3] for groups gp, gp + 1, split exactly
-      // into f16-representable hi + lo (two groups per packed multiply)
+      // into f16-representable hi + lo (two groups per packed multiply; an odd
+      // last group repeats its own scale in the unused half)
+      const int g1 = gp + 1 < NG ? gp + 1 : gp;
       float wh[4][2], wl[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 x = __fmul2_rn(make_float2(p[u][i], p[u][i]),
-                                    make_float2(sv[u][i][gp], sv[u][i][gp + 1]));
+                                    make_float2(sv[u][i][gp], sv[u][i][g1]));
         const float2 h = make_float2(split_hi(x.x), split_hi(x.y));
         const float2 l = __ffma2_rn(h, make_float2(-1.0f, -1.0f), x);  // exact
         wh[i][0] = h.x;
@@ -909,6 +985,7 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int g = gp + e;
+        if (g >= NG) break;  // odd NG: the last pair has one group
         const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
         // codes c = 0..3 of dims 32g + 4gid + c: low halves rows rho0 / rho2,
         // high halves rows rho1 / rho3
@@ -1013,17 +1090,17 @@ __device__ __forceinline__ void tile_pv_cb(const unsigned char* stg, int r0, int
 // One warp's share of a stage: scores, softmax update and P.V of its TPW tiles
 // (rows r0 .. r0 + 16 TPW - 1, of which the first nvalid are real tokens).
 template <int D, int PATH, int FMT, int TPW, bool FULL, bool EXACT = false>
-__device__ __forceinline__ void stage_tiles(const unsigned char* stg, int r0, int nvalid, int gid,
+__device__ __forceinline__ void stage_tiles(const unsigned char* stg, int skew, int r0, int nvalid, int gid,
                                             int tig, const int (&rho)[4], const int (&krow)[2],
                                             WarpState<D, PATH, FMT>& st,
                                             const unsigned char* lutp) {
   float S[TPW][4], p[TPW][4], sv[TPW][4][D / 32];
   if constexpr (FMT == 0)
-    tile_scores<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, tig, rho, krow, st, S);
+    tile_scores<D, PATH, FMT, TPW, FULL>(stg, skew, r0, nvalid, tig, rho, krow, st, S);
   else
-    tile_scores_cb<D, PATH, FMT, TPW, FULL, EXACT>(stg, r0, nvalid, tig, rho, krow, st, lutp, S);
+    tile_scores_cb<D, PATH, FMT, TPW, FULL, EXACT>(stg, skew, r0, nvalid, tig, rho, krow, st, lutp, S);
   tile_max<D, PATH, FMT, TPW>(tig, S, st);
-  load_vscales<D, PATH, FMT, TPW, FULL>(stg, r0, nvalid, rho, sv);
+  load_vscales<D, PATH, FMT, TPW, FULL>(stg, skew, r0, nvalid, rho, sv);
   tile_weights<D, PATH, FMT, TPW>(S, sv, st, p);
   if constexpr (FMT == 0)
     tile_pv<D, PATH, FMT, TPW>(stg, r0, gid, rho, p, sv, st);
@@ -1227,11 +1304,13 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       const unsigned char* src = static_cast<const unsigned char*>(isv ? a.v_new : a.k_new) + bh * D * eb;
       uint8_t* prow = const_cast<uint8_t*>(isv ? a.v_packed : a.k_packed) + row * C::RB;
       float* srow = const_cast<float*>(isv ? a.v_scales : a.k_scales) + row * (D / 32);
-      if constexpr (FMT == 0)
-        quantize_vector_warp<D>(src, a.kv_bf16, a.signs, prow, srow, lane);
-      else
+      if constexpr (FMT == 0) {
+        if constexpr (D == 128 || D == 256)  // other widths are SRFT caches, never fused here
+          quantize_vector_warp<D>(src, a.kv_bf16, a.signs, prow, srow, lane);
+      } else {
         cb_quantize_vector_warp<D, FMT>(src, a.kv_bf16, a.signs, a.levels, prow, srow, lane,
                                         a.cb_uniform != 0);
+      }
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
     asm volatile("bar.arrive 2, 96;" ::: "memory");
@@ -1268,24 +1347,25 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
       const int slot = sc % C::NS;
       const unsigned char* stg = smem + slot * C::STAGE;
       mbar_wait(full + slot, (sc / C::NS) & 1, abort);
+      const int skew = C::SPAD ? reinterpret_cast<const int*>(smem + C::SKEW)[slot] : 0;
       const int nv = min(C::ST, t1 - t0 - k * C::ST) - r0;  // real rows from r0 on
       if constexpr (FMT != 0) {
         if (exact) {
           if (nv >= 16 * C::TPW)
-            stage_tiles<D, PATH, FMT, C::TPW, true, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+            stage_tiles<D, PATH, FMT, C::TPW, true, true>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
           else if (nv > 0)
-            stage_tiles<D, PATH, FMT, C::TPW, false, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+            stage_tiles<D, PATH, FMT, C::TPW, false, true>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
         } else {
           if (nv >= 16 * C::TPW)
-            stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+            stage_tiles<D, PATH, FMT, C::TPW, true>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
           else if (nv > 0)
-            stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+            stage_tiles<D, PATH, FMT, C::TPW, false>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
         }
       } else {
         if (nv >= 16 * C::TPW)
-          stage_tiles<D, PATH, FMT, C::TPW, true>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+          stage_tiles<D, PATH, FMT, C::TPW, true>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
         else if (nv > 0)
-          stage_tiles<D, PATH, FMT, C::TPW, false>(stg, r0, nv, gid, tig, rho, krow, st, lutp);
+          stage_tiles<D, PATH, FMT, C::TPW, false>(stg, skew, r0, nv, gid, tig, rho, krow, st, lutp);
       }
       __syncwarp();
       if (lane == 0) {
@@ -1342,14 +1422,14 @@ cudaError_t launch_mma(const DecodeArgs& a, cudaStream_t stream) {
 }  // namespace
 
 bool decode_mma_supported(int d, int G) {
-  return (d == 128 && G >= 1 && G <= 8) || (d == 256 && G >= 1 && G <= 4);
+  return (d == 128 && G >= 1 && G <= 8) || ((d == 96 || d == 256) && G >= 1 && G <= 4);
 }
 
 bool decode_mma_cb_supported(int d, int G) { return d == 128 && G >= 5 && G <= 8; }
 
 int decode_stage_tokens(int d, int G) {
   if (!decode_mma_supported(d, G)) return 128;
-  return d == 128 ? Cfg<128, 0, 0>::ST : Cfg<256, 1, 0>::ST;
+  return d == 128 ? Cfg<128, 0, 0>::ST : d == 96 ? Cfg<96, 1, 0>::ST : Cfg<256, 1, 0>::ST;
 }
 
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
@@ -1366,6 +1446,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
   if (a.d == 128 && G >= 5 && G <= 8) return launch_mma<128, 0, 0>(a, stream);
   if (a.d == 128 && G >= 1 && G <= 4) return launch_mma<128, 1, 0>(a, stream);
   if (a.d == 256 && G >= 1 && G <= 4) return launch_mma<256, 1, 0>(a, stream);
+  if (a.d == 96 && G >= 1 && G <= 4) return launch_mma<96, 1, 0>(a, stream);
   return cudaErrorNotSupported;
 }
 
