@@ -273,7 +273,7 @@ def run_tq(args):
         moved = k_all.numel() * k_all.element_size() * 2 + nvec * (code_bytes + 4 * (d // 32))
         hbm_peak, peak_kind = measured_peaks()
         tc_rotation = (w.rotation and not w.cb_bits and k_all.dtype == torch.bfloat16 and nvec > 8192
-                       and (d == 128 or (srft and d <= 128)))
+                       and ((not srft and d in (128, 256)) or (srft and d <= 128)))
         prefill = {"tokens": int(k_all.shape[2]), "us": round(t * 1e6, 2),
                    "tokens_per_s": round(B * k_all.shape[2] / t, 1),
                    "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),

@@ -637,6 +637,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
     if (a.bf16) return rot ? launch_half<true>(a, stream) : launch_half<false>(a, stream);
     return rot ? launch_q<128, false, true>(a, stream) : launch_q<128, false, false>(a, stream);
   }
+  if (a.bf16 && rot && !a.butterfly_rotation && quantize_tc_supported(a)) return launch_quantize_tc(a, stream);
   if (a.bf16) return rot ? launch_q<256, true, true>(a, stream) : launch_q<256, true, false>(a, stream);
   return rot ? launch_q<256, false, true>(a, stream) : launch_q<256, false, false>(a, stream);
 }

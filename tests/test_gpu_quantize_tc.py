@@ -1,7 +1,8 @@
 """The tensor-core bulk quantizer (quantize_tc.cu) against the oracle.
 
 Bulk quantize-appends (more than 8192 vectors) of bf16 vectors at head_dim 128
-with rotation run the rotation as a bf16 tcgen05 product on 128-vector tiles;
+and 256 with rotation run the rotation as a bf16 tcgen05 product on 128-vector
+tiles (at 256: two 128-wide products P, Q and y = (P +- Q) / 16);
 TQ_TEST_HOOK_BUTTERFLY_QUANTIZE selects the fp32 butterfly kernel instead.
 Bars as in test_gpu_quantize: at most 0.01% of codes differ from the oracle's,
 each by 1, scales within 4 ulp.  Cases: ragged last tiles, several sequences
@@ -44,15 +45,15 @@ def _signs(d, seed):
     return (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.int8)
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("B,H,n,pos,extra", [
     (1, 8, 1100, [0], 3),          # 8800 vectors per tensor: 68.75 tiles
     (3, 2, 1501, [0, 7, 100], 0),  # rows of the last two sequences run past the capacity
     (2, 5, 1000, [3, 0], 9),
 ])
-def test_tc_quantize_matches_oracle(B, H, n, pos, extra):
+def test_tc_quantize_matches_oracle(d, B, H, n, pos, extra):
     require_cuda()
-    d = 128
-    k, v = inputs(B, H, n, d, torch.bfloat16, 31 * n + B)
+    k, v = inputs(B, H, n, d, torch.bfloat16, 31 * n + B + d)
     signs = _signs(d, n)
     cap = n + extra
     assert 2 * B * H * n > 8192   # the bulk path
@@ -69,11 +70,12 @@ def test_tc_quantize_matches_oracle(B, H, n, pos, extra):
     compare(got, ref, d, True, f"B={B} H={H} n={n} pos={pos}")
 
 
-def test_tc_quantize_agrees_with_butterfly_kernel():
+@pytest.mark.parametrize("d", [128, 256])
+def test_tc_quantize_agrees_with_butterfly_kernel(d):
     """Same inputs through both bulk kernels: the rotations differ only in the
     order of fp32 roundings, so codes match except at near-ties."""
     require_cuda()
-    B, H, n, d = 2, 4, 1300, 128
+    B, H, n = 2, 4, 1300
     k, v = inputs(B, H, n, d, torch.bfloat16, 77)
     signs = _signs(d, 78)
     tc = _quantize(k, v, [0, 5], signs, n + 5)
@@ -82,7 +84,8 @@ def test_tc_quantize_agrees_with_butterfly_kernel():
     assert n_diff <= 1e-5 * n_tot
 
 
-def test_tc_quantize_bit_identical_to_butterfly_kernel_on_exact_inputs():
+@pytest.mark.parametrize("d", [128, 256])
+def test_tc_quantize_bit_identical_to_butterfly_kernel_on_exact_inputs(d):
     """Small-integer inputs times a power of two per vector: every partial sum
     of both rotations is exact, so both kernels round the same rotated values
     and must give identical bits (scale division by 7, reciprocal bracket,
@@ -91,7 +94,7 @@ def test_tc_quantize_bit_identical_to_butterfly_kernel_on_exact_inputs():
     half-integer in exact arithmetic, where fl(D c) and the oracle's correctly
     rounded rotation may round apart; oracle parity is the other tests'.)"""
     require_cuda()
-    B, H, n, d = 1, 6, 1500, 128
+    B, H, n = 1, 6, 1500
     g = torch.Generator().manual_seed(21)
     ints = torch.randint(-8, 9, (B, H, n, d), generator=g).float()
     ints[:, :, 5] = 0
@@ -108,12 +111,13 @@ def test_tc_quantize_bit_identical_to_butterfly_kernel_on_exact_inputs():
         np.testing.assert_array_equal(a.view(np.uint8), b.view(np.uint8))
 
 
-def test_tc_quantize_extreme_values():
-    """bf16 subnormals, values near the bf16 maximum over 128 (no fp32
+@pytest.mark.parametrize("d", [128, 256])
+def test_tc_quantize_extreme_values(d):
+    """bf16 subnormals, values near the bf16 maximum over d (no fp32
     overflow in the rotation), one huge and many tiny values in one vector,
     single spikes and zero vectors, inside a bulk call."""
     require_cuda()
-    d, n = 128, 4500
+    n = 4500
     g = torch.Generator().manual_seed(11)
     x = torch.randn(1, 2, n, d, generator=g)
     sub = torch.finfo(torch.float32).tiny  # 2^-126
@@ -121,7 +125,7 @@ def test_tc_quantize_extreme_values():
         torch.full((d,), 3.0) * sub * 0.25,                        # all subnormal
         torch.where(torch.arange(d) % 2 == 0, 1.0, 0.5) * sub * 0.03,
         torch.cat([torch.ones(1), torch.full((d - 1,), sub * 0.5)]),  # one normal, rest subnormal
-        torch.linspace(-1.0, 1.0, d) * 2.0 ** 120,                 # near the bf16 maximum / 2^7
+        torch.linspace(-1.0, 1.0, d) * 2.0 ** 119,                 # near the bf16 maximum / 2^8
         torch.cat([torch.full((1,), 1e30), torch.full((d - 1,), 1e-30)]),
         torch.cat([torch.full((3,), -2.0 ** 100), torch.randn(d - 3, generator=g)]),
         torch.eye(d)[17] * 5.0,
@@ -139,12 +143,13 @@ def test_tc_quantize_extreme_values():
     compare(got, ref, d, True, "extremes")
 
 
-def test_tc_quantize_starved_pipeline_writes_nan_scales_then_recovers():
+@pytest.mark.parametrize("d", [128, 256])
+def test_tc_quantize_starved_pipeline_writes_nan_scales_then_recovers(d):
     """With every CTA's first copy withheld the kernel's bounded waits run out:
     every written row gets NaN scales.  The next call on the context is
     correct."""
     require_cuda()
-    B, H, n, d = 1, 8, 1100, 128
+    B, H, n = 1, 8, 1100
     k, v = inputs(B, H, n, d, torch.bfloat16, 5)
     signs = _signs(d, 6)
     bad = _quantize(k, v, [0], signs, n, _lib.TEST_HOOK_STARVE_PIPELINE)
