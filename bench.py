@@ -223,6 +223,42 @@ def dist_setup(args):
     return world, rank, local
 
 
+def prefill_timing(torch, cache, k_all, v_all, pos0, stream, flush, w, srft=False):
+    """The bulk prefill of k_all, v_all [B][Hkv][n][d] into rows 0 .. n-1 of
+    `cache` (one quantize-append call): the minimum of 3 calls timed with CUDA
+    events, each after an L2 flush (a write of `flush`), and its HBM roofline
+    fraction over the bytes the call must move (bf16 inputs read once, codes
+    and fp32 scales written once)."""
+    times = []
+    for i in range(4):
+        flush.fill_(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.append(k_all, v_all, pos0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = min(times)
+    B, _, n, d = k_all.shape
+    nvec = 2 * B * k_all.shape[1] * n
+    code_bytes = d * w.cb_bits // 8 if w.cb_bits else d // 2
+    moved = k_all.numel() * k_all.element_size() * 2 + nvec * (code_bytes + 4 * (d // 32))
+    hbm_peak, peak_kind = measured_peaks()
+    tc_rotation = (w.rotation and not w.cb_bits and k_all.dtype == torch.bfloat16 and nvec > 8192
+                   and ((not srft and d in (128, 256)) or (srft and d <= 128)))
+    return {"tokens": int(n), "us": round(t * 1e6, 2),
+            "tokens_per_s": round(B * n / t, 1),
+            "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),
+            "bytes_moved": int(moved),
+            "roofline_frac": round(moved / t / 1e9 / hbm_peak, 3), "peak_kind": peak_kind,
+            "kernel": (("quantize_srft_tc_kernel (Hartley transform as a tcgen05 product, "
+                        "three bf16 parts)" if srft else
+                        "quantize_tc_kernel (rotation as a tcgen05 bf16 product)") if tc_rotation
+                       else "CUDA-core quantize kernel"),
+            "timing": "min of 3 calls, each after a 256 MiB L2 flush"}
+
+
 def run_tq(args):
     import torch
     import torch.distributed as dist
@@ -257,33 +293,7 @@ def run_tq(args):
     # bulk prefill: all cached tokens quantized in one call
     prefill = None
     if not args.no_prefill:
-        times = []
-        for i in range(4):
-            flush.fill_(i)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            cache.append(k_all, v_all, pos0)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if i:
-                times.append(e0.elapsed_time(e1) / 1e3)
-        t = min(times)
-        nvec = 2 * B * Hkv * k_all.shape[2]
-        code_bytes = d * w.cb_bits // 8 if w.cb_bits else d // 2
-        moved = k_all.numel() * k_all.element_size() * 2 + nvec * (code_bytes + 4 * (d // 32))
-        hbm_peak, peak_kind = measured_peaks()
-        tc_rotation = (w.rotation and not w.cb_bits and k_all.dtype == torch.bfloat16 and nvec > 8192
-                       and ((not srft and d in (128, 256)) or (srft and d <= 128)))
-        prefill = {"tokens": int(k_all.shape[2]), "us": round(t * 1e6, 2),
-                   "tokens_per_s": round(B * k_all.shape[2] / t, 1),
-                   "GB_per_s": round(moved / t / 1e9, 1), "ns_per_vec": round(t / nvec * 1e9, 4),
-                   "bytes_moved": int(moved),
-                   "roofline_frac": round(moved / t / 1e9 / hbm_peak, 3), "peak_kind": peak_kind,
-                   "kernel": (("quantize_srft_tc_kernel (Hartley transform as a tcgen05 product, "
-                               "three bf16 parts)" if srft else
-                               "quantize_tc_kernel (rotation as a tcgen05 bf16 product)") if tc_rotation
-                              else "CUDA-core quantize kernel"),
-                   "timing": "min of 3 calls, each after a 256 MiB L2 flush"}
+        prefill = prefill_timing(torch, cache, k_all, v_all, pos0, stream, flush, w, srft)
     else:
         cache.append(k_all, v_all, pos0)
     # host copy of sequence 0's first kv heads for the fidelity report
@@ -517,7 +527,8 @@ CONFIGS = (("tiny_mha_4k", False, 0), ("tiny_mha_4k", True, 0), ("llama70b_gqa_3
 
 
 def measure_config(name, rot, scale_idx, args, dev, stream, seed, peak, want_fidelity=False):
-    """One configuration's decode step on this GPU: the fused append + decode
+    """One configuration on this GPU: the bulk prefill of its cached context
+    (one quantize-append call), the decode step as the fused append + decode
     (tq_sdpa_int4_decode_append), the decode alone, their median and P95 over
     graph replays, the host-buffer e2e step, and the decode's roofline fraction."""
     import dataclasses
@@ -533,7 +544,10 @@ def measure_config(name, rot, scale_idx, args, dev, stream, seed, peak, want_fid
     ctx = wl.make_context_lengths(w, seed)
     cache = tq.Int4KVCache(B, Hkv, d, w.capacity, dev, signs)
     k_all, v_all = wl.make_kv(w, seed, device=dev, tokens=w.capacity - 1)
-    cache.append(k_all, v_all, torch.zeros(B, dtype=torch.int32, device=dev))
+    pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    prefill = prefill_timing(torch, cache, k_all, v_all, pos0, stream, flush, w)
+    del flush
     fid_in = None
     k_new, v_new = wl.make_kv(w, seed, device=dev, tokens=1, token_offset=10_000_019)
     if want_fidelity:  # sequence 0's first two kv heads, unquantized, with the appended token
@@ -600,6 +614,7 @@ def measure_config(name, rot, scale_idx, args, dev, stream, seed, peak, want_fid
         "roofline_frac": round(algo / res["decode"] / 1e9 / peak, 4),
         "e2e_us": round(sum(e2e) / len(e2e) * 1e6, 2),
         "l2": f"rotated over {n_rot} caches",
+        "prefill": {k_: prefill[k_] for k_ in ("tokens", "us", "GB_per_s", "roofline_frac", "kernel")},
     }
     if want_fidelity:
         caches[0].decode(q, ctx_dev, max_ctx, scale, out)
