@@ -35,11 +35,21 @@
 //    tile's V scales and raised, with an exact power-of-two rescale of the
 //    accumulators and the running sum, whenever a later tile would overflow.
 //    The partial then reports max m + F.
-// Two arrangements (template PATH):
-//  - PATH 0 (heads on rows, 5..8 query heads per kv head, d = 128): scores
-//    C = [q hi; q lo] x K^T; P.V C = [P' hi; P' lo] x V, where the score
-//    accumulator fragment is reused as the P.V A operand without shuffles.
-//  - PATH 1 (dims on rows, 1..4 query heads, d = 128 or 256): scores as
+// Three arrangements (template PATH):
+//  - PATH 0 (heads on rows, 5..8 query heads per kv head, d = 128; the
+//    codebook caches): scores C = [q hi; q lo] x K^T; P.V C = [P' hi; P' lo]
+//    x V, where the score accumulator fragment is reused as the P.V A operand
+//    without shuffles.  The accumulator holds the hi and lo rows apart:
+//    d/8 x 4 registers.
+//  - PATH 2 (5..8 query heads, d = 128, int4): scores as PATH 0; P.V with
+//    dims on the rows, C = V^T x P' hi + V^T x P' lo (two MMAs into one
+//    accumulator), where the score fragment of head gid is already the B
+//    operand of column gid.  The same MMA count as PATH 0 with half the
+//    accumulator registers (d/16 x 4), which buys a third 16-token tile per
+//    warp: the kernel is bound by the latency of each tile's dependent chain
+//    (scores, max, weights, P.V), so the number of tiles in flight per
+//    scheduler sets the speed.
+//  - PATH 1 (dims on rows, 1..4 query heads, d = 96, 128 or 256): scores as
 //    above with each head on two neighbouring rows; P.V C = V^T x [P' hi,
 //    P' lo per head] with dims on the rows, so the accumulator is d/16 x 4
 //    registers.
@@ -270,14 +280,14 @@ constexpr int kMaxListB = 1024;
 template <int D, int PATH, int FMT>
 struct Cfg {
   static constexpr int NW = 8;                  // warps per CTA (all consumers)
-  static constexpr int TPW = D == 256 ? 1 : 2;  // 16-token tiles per warp per stage
+  static constexpr int TPW = D == 256 ? 1 : PATH == 2 ? 3 : 2;  // 16-token tiles per warp per stage
   static constexpr int THREADS = 32 * NW;
   static constexpr int ST = 16 * TPW * NW;      // tokens per pipeline stage
   static constexpr int NG = D / 32;             // quantization groups per vector
   static constexpr int RB = FMT ? D * FMT / 8 : D / 2;  // packed bytes per row
-  static constexpr int NH = PATH == 0 ? 8 : 4;  // query heads per kv head (max)
+  static constexpr int NH = PATH == 1 ? 4 : 8;  // query heads per kv head (max)
   static constexpr int NACC = PATH == 0 ? 4 * NG : 2 * NG;  // accumulator fragments
-  static constexpr int NS = D == 256 ? 3 : 4;                // pipeline stages
+  static constexpr int NS = D == 256 || PATH == 2 ? 3 : 4;   // pipeline stages
   // scale rows of 12 bytes (d = 96) are not 16-byte copy units: a stage's
   // scales arrive as the 16-byte aligned superset, SPAD bytes more per region
   static constexpr int SPAD = (NG % 4) ? 32 : 0;
@@ -625,7 +635,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   for (int idx = threadIdx.x; idx < (D / 32) * 2 * 256; idx += C::THREADS) {
     const int k = idx & 15, row = (idx >> 4) & 15, gks = idx >> 8;
     const int g = gks >> 1, ks = gks & 1;
-    const int hr = PATH == 0 ? (row & 7) : ((row & 7) >> 1);
+    const int hr = PATH == 1 ? ((row & 7) >> 1) : (row & 7);
     const int dim = FMT ? 32 * g + 8 * ((k & 7) >> 1) + 4 * ks + 2 * (k >> 3) + (k & 1)
                         : 32 * g + 8 * ((k & 7) >> 1) + 2 * ks + (k >> 3) + 4 * (k & 1);
     const float v = qs[hr * D + dim] * ((FMT == 0 && (k >> 3)) ? 0.0625f : 1.0f);  // exact
@@ -636,13 +646,26 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   }
   barrier_all<C::THREADS>();
   const int gid = lane >> 2;
-  const int hrow = PATH == 0 ? gid : gid >> 1;
+  const int hrow = PATH == 1 ? gid >> 1 : gid;
   {
     const int mi = lane >> 3, row = (lane & 7) + 8 * (mi & 1), kb = mi >> 1;
     st.qa_addr = smem_u32(smem + C::QA) + row * 32 + ((kb ^ ((row >> 2) & 1)) * 16);
   }
   st.k8_addr = smem_u32(smem + C::QK8) + hrow * C::NG * 4;
   st.qexp = qexp[hrow] * st.cexp;
+}
+
+template <int D, int PATH, int FMT>
+__device__ __forceinline__ void scale_acc2(WarpState<D, PATH, FMT>& st, float f0, float f1) {
+  const float2 ff = make_float2(f0, f1);
+#pragma unroll
+  for (int j = 0; j < Cfg<D, PATH, FMT>::NACC; ++j)
+#pragma unroll
+    for (int r = 0; r < 4; r += 2) {
+      const float2 v = __fmul2_rn(make_float2(st.acc[j][r], st.acc[j][r + 1]), ff);
+      st.acc[j][r] = v.x;
+      st.acc[j][r + 1] = v.y;
+    }
 }
 
 template <int D, int PATH, int FMT>
@@ -833,19 +856,23 @@ __device__ __forceinline__ void tile_scores_cb(const unsigned char* stg, int ske
 // it grows, the accumulators and the running sum are rescaled.
 template <int D, int PATH, int FMT, int TPW>
 __device__ __forceinline__ void tile_max(int tig, const float (&S)[TPW][4], WarpState<D, PATH, FMT>& st) {
-  float mx;
-  if (TPW == 2)
-    mx = fmax3(fmax3(S[0][0], S[0][1], S[0][2]), fmax3(S[0][3], S[TPW - 1][0], S[TPW - 1][1]),
-               fmaxf(S[TPW - 1][2], S[TPW - 1][3]));
-  else
-    mx = fmaxf(fmax3(S[0][0], S[0][1], S[0][2]), S[0][3]);
+  float mx = fmaxf(fmax3(S[0][0], S[0][1], S[0][2]), S[0][3]);
+#pragma unroll
+  for (int u = 1; u < TPW; ++u)
+    mx = fmax3(mx, fmax3(S[u][0], S[u][1], S[u][2]), S[u][3]);
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
   const float m_new = fmaxf(st.m, mx * st.qexp);
   if (__any_sync(kFull, m_new > st.m)) {
     const float alpha = ex2(st.m - m_new);  // 0 on the first tile, 1 if unchanged
-    // PATH 1 accumulates head tig; its softmax state lives on lane 8 * tig
-    scale_acc(st, PATH == 0 ? alpha : __shfl_sync(kFull, alpha, 8 * tig));
+    if (PATH == 0) {
+      scale_acc(st, alpha);
+    } else if (PATH == 1) {  // accumulates head tig; its softmax state lives on lane 8 * tig
+      scale_acc(st, __shfl_sync(kFull, alpha, 8 * tig));
+    } else {  // accumulator columns: heads 2tig (lane 8 tig) and 2tig + 1 (lane 8 tig + 4)
+      const float a0 = __shfl_sync(kFull, alpha, 8 * tig), a1 = __shfl_sync(kFull, alpha, 8 * tig + 4);
+      scale_acc2(st, a0, a1);
+    }
     st.l = __fmul2_rn(st.l, make_float2(alpha, alpha));
     st.m = m_new;
   }
@@ -998,6 +1025,16 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
           mma16816(st.acc[4 * g + 1], a0, a1, a2, a3, codes_hi(X), codes_hi(Y));
           mma16816(st.acc[4 * g + 2], a0, a1, a2, a3, codes_lo(X >> 8), codes_lo(Y >> 8));
           mma16816(st.acc[4 * g + 3], a0, a1, a2, a3, codes_hi(X >> 8), codes_hi(Y >> 8));
+        } else if (PATH == 2) {  // B: the weights of head gid, hi part, then lo part
+          const uint32_t bh0 = f16x2(wh[0][e], wh[1][e]), bh1 = f16x2(wh[2][e], wh[3][e]);
+          const uint32_t bl0 = f16x2(wl[0][e], wl[1][e]), bl1 = f16x2(wl[2][e], wl[3][e]);
+          const uint32_t x0 = codes_lo(X), x1 = codes_hi(X), y0 = codes_lo(Y), y1 = codes_hi(Y);
+          mma16816(st.acc[2 * g + 0], x0, x1, y0, y1, bh0, bh1);
+          mma16816(st.acc[2 * g + 0], x0, x1, y0, y1, bl0, bl1);
+          const uint32_t x2 = codes_lo(X >> 8), x3 = codes_hi(X >> 8);
+          const uint32_t y2 = codes_lo(Y >> 8), y3 = codes_hi(Y >> 8);
+          mma16816(st.acc[2 * g + 1], x2, x3, y2, y3, bh0, bh1);
+          mma16816(st.acc[2 * g + 1], x2, x3, y2, y3, bl0, bl1);
         } else {
           const bool lo = gid & 1;  // column gid = (head gid / 2, part gid % 2)
           const uint32_t b0 = f16x2(lo ? wl[0][e] : wh[0][e], lo ? wl[1][e] : wh[1][e]);
@@ -1144,6 +1181,23 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
       for (int cc = 0; cc < 4; ++cc) {
         dst[32 * g + 8 * tig + cc] = (st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2]) * ce;
         dst[32 * g + 8 * tig + 4 + cc] = (st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3]) * ce;
+      }
+  } else if (PATH == 2) {
+    if (tig == 0) {
+      mm[warp * NH + gid] = m;
+      ml[warp * NH + gid] = l;
+    }
+    // fragment 2g + pp: rows gid, gid + 8 are dims 32g + 4gid + 2pp (+1),
+    // columns 2tig, 2tig + 1 are heads
+    float* d0 = macc + (warp * NH + 2 * tig) * D;
+    float* d1 = d0 + D;
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        const int dim = 32 * g + 4 * gid + 2 * pp;
+        *reinterpret_cast<float2*>(d0 + dim) = make_float2(st.acc[2 * g + pp][0], st.acc[2 * g + pp][2]);
+        *reinterpret_cast<float2*>(d1 + dim) = make_float2(st.acc[2 * g + pp][1], st.acc[2 * g + pp][3]);
       }
   } else {
     if (tig == 0 && (gid & 1) == 0) {
@@ -1429,7 +1483,8 @@ bool decode_mma_cb_supported(int d, int G) { return d == 128 && G >= 5 && G <= 8
 
 int decode_stage_tokens(int d, int G) {
   if (!decode_mma_supported(d, G)) return 128;
-  return d == 128 ? Cfg<128, 0, 0>::ST : d == 96 ? Cfg<96, 1, 0>::ST : Cfg<256, 1, 0>::ST;
+  return d == 128 ? (G >= 5 ? Cfg<128, 2, 0>::ST : Cfg<128, 1, 0>::ST)
+                   : d == 96 ? Cfg<96, 1, 0>::ST : Cfg<256, 1, 0>::ST;
 }
 
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
@@ -1443,7 +1498,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
       default: return cudaErrorNotSupported;
     }
   }
-  if (a.d == 128 && G >= 5 && G <= 8) return launch_mma<128, 0, 0>(a, stream);
+  if (a.d == 128 && G >= 5 && G <= 8) return launch_mma<128, 2, 0>(a, stream);
   if (a.d == 128 && G >= 1 && G <= 4) return launch_mma<128, 1, 0>(a, stream);
   if (a.d == 256 && G >= 1 && G <= 4) return launch_mma<256, 1, 0>(a, stream);
   if (a.d == 96 && G >= 1 && G <= 4) return launch_mma<96, 1, 0>(a, stream);
