@@ -305,8 +305,10 @@ struct Cfg {
   static constexpr int QS = al(QA + NG * 2 * 16 * 16 * 2);   // float [NH][D] query
   static constexpr int QEXP = al(QS + 4 * NH * D);           // float [NH]
   static constexpr int QK8 = al(QEXP + 4 * 8);               // float [NH][NG] -8 sum_g q
-  static constexpr int MACC = al(QK8 + 4 * NH * NG);         // float [NW][NH][D]
-  static constexpr int MM = al(MACC + 4 * NW * NH * D);      // float [NW][NH] max
+  // the warps' accumulators merge through MB buffers (more than 8 warps: in rounds)
+  static constexpr int MB = NW < 8 ? NW : 8;
+  static constexpr int MACC = al(QK8 + 4 * NH * NG);         // float [MB][NH][D]
+  static constexpr int MM = al(MACC + 4 * MB * NH * D);      // float [NW][NH] max
   static constexpr int ML = al(MM + 4 * NW * NH);            // float [NW][NH] sum
   static constexpr int MW = al(ML + 4 * NW * NH);            // float [NW][NH] weight
   static constexpr int MTOT = al(MW + 4 * NW * NH);          // float [NH] max, [NH] sum
@@ -493,7 +495,7 @@ __device__ __forceinline__ void prep_query(const DecodeArgs& a, int b, int kvh, 
   // Heads are prepared by warps 0 .. NW/2 - 1 (two heads each when NH == 8)
   // while the last warp issues the first copies; with a fused append it first
   // waits (named barrier 2, warps 4, 5 and NW - 1) for the new tokens' rows.
-  constexpr int HPW = C::NH / (C::NW / 2) > 0 ? C::NH / (C::NW / 2) : 1;  // heads per warp
+  constexpr int HPW = (C::NH + C::NW / 2 - 1) / (C::NW / 2);  // heads per warp
   if (start_stream && threadIdx.x >= C::THREADS - 32) {
     if (a.k_new != nullptr) asm volatile("bar.sync 2, 96;" ::: "memory");
     if (threadIdx.x == C::THREADS - 32)
@@ -1168,7 +1170,74 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
   l += __shfl_xor_sync(kFull, l, 1);
   l += __shfl_xor_sync(kFull, l, 2);
   const float m = aborted ? __int_as_float(0x7fc00000) : st.m + (float)st.F;
-  if (PATH == 0) {
+  const int tid = threadIdx.x;
+  if constexpr (PATH == 2) {
+    // softmax states first; then each warp adds its accumulator, weighted, into
+    // buffer warp % MB, one round of MB warps at a time
+    constexpr int MB = C::MB;
+    if (tig == 0) {
+      mm[warp * NH + gid] = m;
+      ml[warp * NH + gid] = l;
+    }
+    barrier_all<C::THREADS>();
+    if (tid < NH) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, mm[w * NH + tid]);
+      float L = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float wt = exp2f(mm[w * NH + tid] - M);  // NaN if that warp gave up
+        mw[w * NH + tid] = wt;
+        L = fmaf(wt, ml[w * NH + tid], L);
+      }
+      mtot[tid] = M;
+      mtot[NH + tid] = L;
+    }
+    barrier_all<C::THREADS>();
+    // fragment 2g + pp: rows gid, gid + 8 are dims 32g + 4gid + 2pp (+1),
+    // columns 2tig, 2tig + 1 are heads
+    const float w0 = mw[warp * NH + 2 * tig], w1 = mw[warp * NH + 2 * tig + 1];
+    float* d0 = macc + ((warp % MB) * NH + 2 * tig) * D;
+    float* d1 = d0 + D;
+    for (int r = 0; r * MB < NW; ++r) {
+      if (warp / MB == r) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            const int dim = 32 * g + 4 * gid + 2 * pp;
+            float2 v0 = make_float2(w0 * st.acc[2 * g + pp][0], w0 * st.acc[2 * g + pp][2]);
+            float2 v1 = make_float2(w1 * st.acc[2 * g + pp][1], w1 * st.acc[2 * g + pp][3]);
+            if (r > 0) {
+              const float2 o0 = *reinterpret_cast<const float2*>(d0 + dim);
+              const float2 o1 = *reinterpret_cast<const float2*>(d1 + dim);
+              v0 = make_float2(v0.x + o0.x, v0.y + o0.y);
+              v1 = make_float2(v1.x + o1.x, v1.y + o1.y);
+            }
+            *reinterpret_cast<float2*>(d0 + dim) = v0;
+            *reinterpret_cast<float2*>(d1 + dim) = v1;
+          }
+      }
+      barrier_all<C::THREADS>();
+    }
+    const int stride = a.plan.part_stride;
+    float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(a.workspace) +
+                                           a.plan.header_bytes);
+    for (int idx = tid; idx < G * D; idx += C::THREADS) {
+      const int h = idx / D, i = idx % D;
+      float s = 0.0f;
+#pragma unroll
+      for (int w = 0; w < MB; ++w) s += macc[(w * NH + h) * D + i];
+      float* dst = part + (((int64_t)b * a.Hq + (int64_t)kvh * G + h) * a.plan.n_chunks + c) * stride;
+      dst[i] = s;
+      if (i == 0) {
+        dst[D] = mtot[h];
+        dst[D + 1] = mtot[NH + h];
+      }
+    }
+    return;
+  } else if (PATH == 0) {
     if (tig == 0) {
       mm[warp * NH + gid] = m;
       ml[warp * NH + gid] = l;
@@ -1181,23 +1250,6 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
       for (int cc = 0; cc < 4; ++cc) {
         dst[32 * g + 8 * tig + cc] = (st.acc[4 * g + cc][0] + st.acc[4 * g + cc][2]) * ce;
         dst[32 * g + 8 * tig + 4 + cc] = (st.acc[4 * g + cc][1] + st.acc[4 * g + cc][3]) * ce;
-      }
-  } else if (PATH == 2) {
-    if (tig == 0) {
-      mm[warp * NH + gid] = m;
-      ml[warp * NH + gid] = l;
-    }
-    // fragment 2g + pp: rows gid, gid + 8 are dims 32g + 4gid + 2pp (+1),
-    // columns 2tig, 2tig + 1 are heads
-    float* d0 = macc + (warp * NH + 2 * tig) * D;
-    float* d1 = d0 + D;
-#pragma unroll
-    for (int g = 0; g < NG; ++g)
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        const int dim = 32 * g + 4 * gid + 2 * pp;
-        *reinterpret_cast<float2*>(d0 + dim) = make_float2(st.acc[2 * g + pp][0], st.acc[2 * g + pp][2]);
-        *reinterpret_cast<float2*>(d1 + dim) = make_float2(st.acc[2 * g + pp][1], st.acc[2 * g + pp][3]);
       }
   } else {
     if (tig == 0 && (gid & 1) == 0) {
@@ -1215,7 +1267,6 @@ __device__ __forceinline__ void finish_item(const DecodeArgs& a, unsigned char* 
       }
   }
   barrier_all<C::THREADS>();
-  const int tid = threadIdx.x;
   if (tid < G) {
     float M = -INFINITY;
 #pragma unroll
@@ -1344,7 +1395,7 @@ __global__ void __launch_bounds__(Cfg<D, PATH, FMT>::THREADS, 1) decode_mma_kern
   // first query.  Only that chunk reads the row; the proxy fence orders these
   // generic writes before the bulk copies, which the last warp issues only
   // after named barrier 2 (both warps arrive here exactly once).
-  static_assert(C::NW == 8, "the fused append uses warps 4, 5 and 7");
+  static_assert(C::NW >= 8, "the fused append uses warps 4, 5 and the last");
   if (a.k_new != nullptr && (warp == 4 || warp == 5)) {
     const bool isv = warp == 5;
     const int eb = a.kv_bf16 ? 2 : 4;
