@@ -37,10 +37,10 @@
 //    The partial then reports max m + F.
 // Three arrangements (template PATH):
 //  - PATH 0 (heads on rows, 5..8 query heads per kv head, d = 128; the
-//    codebook caches): scores C = [q hi; q lo] x K^T; P.V C = [P' hi; P' lo]
-//    x V, where the score accumulator fragment is reused as the P.V A operand
-//    without shuffles.  The accumulator holds the hi and lo rows apart:
-//    d/8 x 4 registers.
+//    codebook caches only): scores C = [q hi; q lo] x K^T; P.V C = [P' hi;
+//    P' lo] x levels, where the score accumulator fragment is reused as the
+//    P.V A operand without shuffles.  The accumulator holds the hi and lo rows
+//    apart: d/8 x 4 registers.
 //  - PATH 2 (5..8 query heads, d = 128, int4): scores as PATH 0; P.V with
 //    dims on the rows, C = V^T x P' hi + V^T x P' lo (two MMAs into one
 //    accumulator), where the score fragment of head gid is already the B
@@ -1020,7 +1020,7 @@ __device__ __forceinline__ void tile_pv(const unsigned char* stg, int r0, int gi
         // high halves rows rho1 / rho3
         const uint32_t X = prmt(vw[0][g / 2], vw[1][g / 2], sel);
         const uint32_t Y = prmt(vw[2][g / 2], vw[3][g / 2], sel);
-        if (PATH == 0) {
+        if (PATH == 0) {  // (no int4 launch takes PATH 0; the codebook caches use tile_pv_cb)
           const uint32_t a0 = f16x2(wh[0][e], wh[1][e]), a1 = f16x2(wl[0][e], wl[1][e]);
           const uint32_t a2 = f16x2(wh[2][e], wh[3][e]), a3 = f16x2(wl[2][e], wl[3][e]);
           mma16816(st.acc[4 * g + 0], a0, a1, a2, a3, codes_lo(X), codes_lo(Y));
