@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other configurations' block")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--context", type=int, default=0,
+                    help="the workload at this many cached tokens per sequence (same batch and "
+                         "heads): small cases for profiling captures; 0 = the workload's own")
     ap.add_argument("--mode", choices=["replicas", "context-parallel"], default="replicas",
                     help="replicas: each rank decodes its own copy of the workload (no collective); "
                          "context-parallel: one context split into contiguous token shards over the "
@@ -254,6 +257,7 @@ def prefill_timing(torch, cache, k_all, v_all, pos0, stream, flush, w, srft=Fals
             "roofline_frac": round(moved / t / 1e9 / hbm_peak, 3), "peak_kind": peak_kind,
             "kernel": (("quantize_srft_tc_kernel (Hartley transform as a tcgen05 product, "
                         "three bf16 parts)" if srft else
+                        "quantize_tc256_kernel (H_2 x H_128: two tcgen05 bf16 products)" if d == 256 else
                         "quantize_tc_kernel (rotation as a tcgen05 bf16 product)") if tc_rotation
                        else "CUDA-core quantize kernel"),
             "timing": "min of 3 calls, each after a 256 MiB L2 flush"}
@@ -271,6 +275,8 @@ def run_tq(args):
     from compressed_domain_attention_tq_b200 import _lib
     _lib.set_test_hooks(_lib.TEST_HOOK_TCGEN05_DECODE if args.decode_kernel == "tcgen05" else 0)
     w = wl.WORKLOADS[args.workload]
+    if args.context:
+        w = wl.shrink(w, context=args.context)
     seed = args.seed + 1000 * rank
     B, Hq, Hkv, d, T = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.context
     stream = torch.cuda.current_stream()
