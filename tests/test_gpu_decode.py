@@ -84,6 +84,16 @@ def test_decode_chunk_boundaries(d):
                 parity(B, Hkv, G, d, [t], seed=t, max_ctx=T)
 
 
+@pytest.mark.parametrize("G", [3, 5, 6, 7])
+@pytest.mark.parametrize("scale", [None, 1.0])
+def test_decode_group_sizes_with_unused_head_columns(G, scale):
+    """3..7 query heads per kv head: the tensor-core decode's MMA tiles are
+    sized for 4 or 8 heads, so some head columns carry no query; contexts of
+    several 384-token stages with ragged last stages."""
+    require_cuda()
+    parity(2, 2, G, 128, [1000, 2893], scale=scale, seed=60 + G)
+
+
 @pytest.mark.parametrize("rot", [False, True])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_decode_tiny_mha_full_size(rot, dtype):
