@@ -120,10 +120,13 @@ __global__ void __launch_bounds__(256) merge_lse_kernel(const float* __restrict_
 
 template <int D>
 cudaError_t launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
+  static SmemLimitSet smem_set;
+  const cudaError_t e = ensure_smem_limit(merge_kernel<D>, kMergeSmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * a.Hq);
   cfg.blockDim = dim3(D);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = merge_smem_bytes((long long)a.B * a.Hq);  // residency cap, not used
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -534,10 +534,13 @@ cudaError_t launch_srft_prep_m(const QuantizeArgs& qa, const DecodeArgs& a, cuda
 
 template <int M>
 cudaError_t launch_srft_merge_m(const DecodeArgs& a, cudaStream_t stream) {
+  static SmemLimitSet smem_set;
+  const cudaError_t e = ensure_smem_limit(srft_merge_kernel<M>, kMergeSmemBytes, smem_set);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.B * ((a.Hq + 1) / 2));
   cfg.blockDim = dim3(32 * M);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = merge_smem_bytes((long long)a.B * ((a.Hq + 1) / 2));  // residency cap, not used
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

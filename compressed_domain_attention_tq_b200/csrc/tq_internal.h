@@ -142,6 +142,18 @@ cudaError_t ensure_smem_limit(Kernel kernel, int bytes, SmemLimitSet& done) {
   return e;
 }
 
+// The merge kernels follow the split-K decode as its programmatic dependents,
+// so their CTAs may start while the decode's CTAs still hold their SMs.  Small
+// as they are, every one of them would then start on the few SMs the decode
+// leaves free and run the whole merge there.  Each merge CTA therefore asks
+// for this much dynamic shared memory, which it does not use: at most two fit
+// on an SM, and the rest start on the SMs the decode releases.  Grids of more
+// than two CTAs per SM skip the cap, which would split them into waves.
+constexpr int kMergeSmemBytes = 100 * 1024;
+inline int merge_smem_bytes(long long merge_ctas) {
+  return merge_ctas <= 2LL * kSmCount ? kMergeSmemBytes : 0;
+}
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 bool quantize_tc_supported(const QuantizeArgs& a);  // bulk bf16, d = 128, rotation on
 cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream);
