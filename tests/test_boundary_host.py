@@ -54,7 +54,11 @@ def test_status_strings(lib):
 def test_decode_plan_properties(lib, B, Hq, Hkv, d, T):
     chunk = _lib.decode_chunk_tokens(B, Hq, Hkv, d, T)
     ws = _lib.decode_workspace_bytes(B, Hq, Hkv, d, T)
-    assert chunk % 64 == 0 and chunk >= 128       # whole pipeline stages (128 or 192 tokens)
+    # whole pipeline stages of the decode that serves the shape: 384 tokens at d = 128 with
+    # 5..8 query heads per kv head, 256 at d = 128 with 1..4, 128 otherwise
+    G = Hq // Hkv
+    stage = 384 if (d == 128 and 5 <= G <= 8) else 256 if (d == 128 and G <= 4) else 128
+    assert chunk % stage == 0 and chunk >= 128
     n_chunks = -(-T // chunk)
     # (sequence, kv head, chunk) items fill their waves over the 148 SMs well
     if T >= 128 * 148:
